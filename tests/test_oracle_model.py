@@ -1,0 +1,183 @@
+"""Whole-decoder pins for the CPU oracle on the 2-layer config: an fp64 brute
+force, the transformers Llama model, special cases and invariants."""
+import copy
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.brute import Brute, bf16_bits_to_f64
+from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
+
+
+def _np_cache(t):
+    return oracle.bits(t).copy()
+
+
+@pytest.fixture(scope="module")
+def setup(tiny_cfg, tiny_weights):
+    cfg = tiny_cfg
+    om = oracle.Model(cfg, tiny_weights)
+    k, v = make_kv_cache(cfg, batch=2, max_seq=160, past=[128, 40], seed=1)
+    toks = make_tokens(cfg, 2, seed=2).numpy()
+    return cfg, om, k, v, toks
+
+
+def _brute_caches(cfg, k, v, b):
+    K = [bf16_bits_to_f64(k[l, b]).copy() for l in range(cfg.n_layers)]
+    V = [bf16_bits_to_f64(v[l, b]).copy() for l in range(cfg.n_layers)]
+    return K, V
+
+
+def test_oracle_vs_fp64_brute_same_rounding_points(setup, tiny_weights, tiny_cfg):
+    cfg, om, k, v, toks = setup
+    kc, vc = _np_cache(k), _np_cache(v)
+    pos = np.array([128, 40], np.int32)
+    logits = om.decode_step(toks, pos, kc, vc)
+    br = Brute(cfg, tiny_weights)
+    for b in range(2):
+        K, V = _brute_caches(cfg, k, v, b)
+        ref = br.decode_step(int(toks[b]), int(pos[b]), K, V, rounding=True)
+        assert int(np.argmax(logits[b])) == int(np.argmax(ref))
+        # the new KV slot agrees with the brute force's to one bf16 ulp
+        for l in range(cfg.n_layers):
+            got_k = bf16_bits_to_f64(kc[l, b, :, pos[b]])
+            assert np.all(np.abs(got_k - K[l][:, pos[b]]) <= 2.0 ** -7 * np.abs(K[l][:, pos[b]]) + 1e-6)
+    # Same rounding points, fp32 vs fp64 arithmetic in between. When no bf16 rounding
+    # decision flips, the two agree to fp32 accuracy (~1e-6 relative); a flip moves one
+    # value by one bf16 ulp, and a flip in a final-norm output (|y| ~ 3, ulp 2^-6) moves
+    # logits by up to ulp * max|E| ~ 1e-3 each. So: steps without a flip agree to 1e-5
+    # (a systematic slip would spoil every step), and every step stays < 8e-3.
+    single_k, single_v = make_kv_cache(cfg, 1, 160, past=128)
+    rel = []
+    for tok in make_tokens(cfg, 16, seed=9).numpy():
+        kc1, vc1 = _np_cache(single_k), _np_cache(single_v)
+        lo = om.decode_step(np.array([tok]), np.array([128]), kc1, vc1)[0]
+        K, V = _brute_caches(cfg, single_k, single_v, 0)
+        ref = br.decode_step(int(tok), 128, K, V, rounding=True)
+        rel.append(np.max(np.abs(lo - ref)) / np.max(np.abs(ref)))
+    assert sum(r <= 1e-5 for r in rel) >= 3, rel
+    assert max(rel) <= 8e-3
+
+
+def test_oracle_vs_exact_fp64_decoder(setup, tiny_weights):
+    cfg, om, k, v, toks = setup
+    kc, vc = _np_cache(k), _np_cache(v)
+    pos = np.array([128, 40], np.int32)
+    logits = om.decode_step(toks, pos, kc, vc)
+    br = Brute(cfg, tiny_weights)
+    for b in range(2):
+        K, V = _brute_caches(cfg, k, v, b)
+        ref = br.decode_step(int(toks[b]), int(pos[b]), K, V, rounding=False)
+        # bf16 rounding at R1..R6 only: stays within the GPU bar's 1e-2 * max|logit|
+        assert np.max(np.abs(logits[b] - ref)) <= 1e-2 * np.max(np.abs(ref))
+
+
+def test_oracle_vs_transformers_llama(setup, tiny_weights):
+    """Library reduction: HF LlamaForCausalLM (fp32, eager, no rope scaling) fed the same
+    weights and the same past K/V returns the same logits up to bf16 rounding."""
+    from transformers import LlamaConfig, LlamaForCausalLM
+    from transformers.cache_utils import DynamicCache
+    cfg, om, k, v, toks = setup
+    w = tiny_weights
+    hc = LlamaConfig(vocab_size=cfg.vocab, hidden_size=cfg.hidden, intermediate_size=cfg.ffn,
+                     num_hidden_layers=cfg.n_layers, num_attention_heads=cfg.n_heads,
+                     num_key_value_heads=cfg.n_kv_heads, head_dim=cfg.head_dim,
+                     rms_norm_eps=cfg.rms_eps, rope_theta=cfg.rope_theta,
+                     tie_word_embeddings=True, max_position_embeddings=4096,
+                     attention_bias=False, mlp_bias=False)
+    hc._attn_implementation = "eager"
+    model = LlamaForCausalLM(hc).to(torch.float64).eval()
+    sd = {"model.embed_tokens.weight": w.embed, "model.norm.weight": w.final_norm,
+          "lm_head.weight": w.embed}
+    for l in range(cfg.n_layers):
+        p = f"model.layers.{l}."
+        sd.update({p + "self_attn.q_proj.weight": w.wq[l], p + "self_attn.k_proj.weight": w.wk[l],
+                   p + "self_attn.v_proj.weight": w.wv[l], p + "self_attn.o_proj.weight": w.wo[l],
+                   p + "mlp.gate_proj.weight": w.wgate[l], p + "mlp.up_proj.weight": w.wup[l],
+                   p + "mlp.down_proj.weight": w.wdown[l], p + "input_layernorm.weight": w.attn_norm[l],
+                   p + "post_attention_layernorm.weight": w.mlp_norm[l]})
+    model.load_state_dict({n: t.to(torch.float64) for n, t in sd.items()}, strict=False)
+    kc, vc = _np_cache(k), _np_cache(v)
+    b, pos = 0, 128
+    ours = om.decode_step(toks[:1], np.array([pos], np.int32), kc[:, :1].copy(), vc[:, :1].copy())
+    cache = DynamicCache()
+    for l in range(cfg.n_layers):
+        cache.update(k[l, b, :, :pos].to(torch.float64)[None], v[l, b, :, :pos].to(torch.float64)[None], l)
+    with torch.no_grad():
+        out = model(input_ids=torch.tensor([[int(toks[0])]]), position_ids=torch.tensor([[pos]]),
+                    past_key_values=cache, use_cache=True)
+    ref = out.logits[0, -1].numpy()
+    assert np.max(np.abs(ours[0] - ref)) <= 1e-2 * np.max(np.abs(ref))
+    assert int(np.argmax(ours[0])) == int(np.argmax(ref))
+
+
+def test_zero_residual_branches_give_embedding_logits(tiny_cfg):
+    """W_o = W_down = 0: every layer is the identity on x, so logits = E . rms(E[t]) and the
+    largest logit is the token itself (its row aligns with itself)."""
+    w = make_weights(tiny_cfg, seed=3)
+    w.wo = [torch.zeros_like(t) for t in w.wo]
+    w.wdown = [torch.zeros_like(t) for t in w.wdown]
+    om = oracle.Model(tiny_cfg, w)
+    k, v = make_kv_cache(tiny_cfg, 1, 64, past=20)
+    kc, vc = _np_cache(k), _np_cache(v)
+    E = oracle.bits(w.embed)
+    for t in (0, 17, 4095):
+        logits = om.decode_step(np.array([t]), np.array([20]), kc, vc)[0]
+        y = oracle.rmsnorm(E[t], oracle.bits(w.final_norm), tiny_cfg.rms_eps)
+        ref = bf16_bits_to_f64(E) @ bf16_bits_to_f64(y)
+        assert np.max(np.abs(logits - ref)) <= 1e-5 * np.max(np.abs(ref))
+        assert oracle.argmax(logits) == t
+
+
+def test_incremental_decode_equals_causal_forward(tiny_cfg, tiny_weights):
+    """Feeding a prefix one token at a time through the cache reproduces the exact
+    cache-free causal forward at every position (up to bf16 rounding)."""
+    cfg = tiny_cfg
+    om = oracle.Model(cfg, tiny_weights)
+    T = 12
+    toks = make_tokens(cfg, T, seed=5).numpy()
+    k, v = make_kv_cache(cfg, 1, 32, past=0)
+    kc, vc = _np_cache(k), _np_cache(v)
+    inc = np.stack([om.decode_step(toks[t:t + 1], np.array([t]), kc, vc)[0] for t in range(T)])
+    full = Brute(cfg, tiny_weights).causal_forward(toks)
+    for t in range(T):
+        assert np.max(np.abs(inc[t] - full[t])) <= 1e-2 * np.max(np.abs(full[t]))
+
+
+def test_kv_write_touches_only_slot_pos(setup):
+    cfg, om, k, v, toks = setup
+    kc, vc = _np_cache(k), _np_cache(v)
+    k0, v0 = kc.copy(), vc.copy()
+    pos = np.array([128, 40], np.int32)
+    om.decode_step(toks, pos, kc, vc)
+    for b in range(2):
+        mask = np.ones(kc.shape[3], bool)
+        mask[pos[b]] = False
+        assert np.array_equal(kc[:, b][:, :, mask], k0[:, b][:, :, mask])
+        assert np.array_equal(vc[:, b][:, :, mask], v0[:, b][:, :, mask])
+        assert not np.array_equal(kc[:, b, :, pos[b]], k0[:, b, :, pos[b]])
+
+
+def test_batch_rows_are_independent(setup):
+    cfg, om, k, v, toks = setup
+    pos = np.array([128, 40], np.int32)
+    kc, vc = _np_cache(k), _np_cache(v)
+    both = om.decode_step(toks, pos, kc, vc)
+    for b in range(2):
+        kb, vb = _np_cache(k)[:, b:b + 1].copy(), _np_cache(v)[:, b:b + 1].copy()
+        one = om.decode_step(toks[b:b + 1], pos[b:b + 1], kb, vb)
+        assert np.array_equal(one[0], both[b])
+        assert np.array_equal(kb[:, 0], kc[:, b])
+
+
+def test_bad_inputs_rejected_without_writes(setup):
+    cfg, om, k, v, toks = setup
+    kc, vc = _np_cache(k), _np_cache(v)
+    k0 = kc.copy()
+    with pytest.raises(ValueError):
+        om.decode_step(np.array([cfg.vocab]), np.array([3]), kc[:, :1].copy(), vc[:, :1].copy())
+    with pytest.raises(ValueError):
+        om.decode_step(np.array([1]), np.array([160]), kc[:, :1].copy(), vc[:, :1].copy())
+    assert np.array_equal(kc, k0)
