@@ -1,0 +1,393 @@
+"""Benchmark: one decode step of the Llama-3.2-1B-shaped decoder at batch 1 with
+128 cached positions, run as one persistent megakernel launch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mk|reference]
+
+Prints ONE JSON line (rank 0). For N > 1 (torchrun, one process per GPU) every
+rank runs an independent replica of the step (the path has no exchange step):
+``value`` is the sum of all replicas' tokens/s, timed as the max over ranks.
+
+Timing: CUDA events on the launching stream, W untimed warm-up steps, K timed
+steps, a device synchronisation and a barrier on both sides. The weights
+(2.47 GB) are far larger than the 126 MB L2, so every step streams them from
+HBM; no separate L2 flush is needed.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs/decode step & tokens/s, Llama-1B-style bf16 bs1; HBM GB/s vs peak"
+PAST = 128            # cached positions before the step
+BATCH = 1
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+PROFILE_FILE = os.path.join(ROOT, "profiles", "megakernel_llama1b_bs1_ctx128.md")
+KERNEL_SOURCES = ["mk_device.cuh", "megakernel.cu", "mk_internal.h"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "persistent_megakernel_interpreter_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    try:
+        text = open(PROFILE_FILE).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (m_hash and m_bytes) or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        mhz, max_mhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                max_mhz = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup(n_gpus: int):
+    """(rank, world, local_rank, group-or-None). torchrun sets the env."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return 0, 1, 0, None
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    import datetime
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local, dist
+
+
+def aggregate(elapsed_ms: float, units: float, dist, device=None):
+    """Max of the elapsed time and sum of the units over ranks (all ranks call it)."""
+    if dist is None:
+        return elapsed_ms, units
+    import torch
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def workload_config(n_gpus: int):
+    return {"workload": "Llama-3.2-1B-shaped decoder, one decode step, batch 1, 128 cached "
+                        "positions (129 keys), random bf16 weights N(0,0.02), KV N(0,1)",
+            "layers": 16, "hidden": 2048, "heads": "32q/8kv x 64", "ffn": 8192, "vocab": 128256,
+            "global_batch": BATCH * n_gpus, "seq_len": PAST + 1,
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": "no flush: the 2.47 GB of weights streamed per step exceed the 126 MB L2"}
+
+
+def time_oracle(cfg, w, k, v, budget_s: float):
+    """The CPU oracle on this host's cores: full decode steps of the same workload until
+    ``budget_s`` has passed (at least one). Returns (tokens/s, steps, threads, s/step)."""
+    import numpy as np
+    import oracle
+    from persistent_megakernel_interpreter_b200.inputs import make_tokens
+    om = oracle.Model(cfg, w)
+    kc, vc = oracle.bits(k).copy(), oracle.bits(v).copy()
+    toks = make_tokens(cfg, 1, seed=2).numpy()
+    threads = oracle.max_threads()
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        om.decode_step(toks, np.array([PAST]), kc, vc, threads=threads)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return BATCH * n / el, n, threads, el / n
+
+
+def run_reference(args):
+    rank, world, local, dist = dist_setup(args.gpus)
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    from persistent_megakernel_interpreter_b200.config import LLAMA_1B
+    from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_weights
+    cfg = LLAMA_1B
+    w = make_weights(cfg, seed=0)
+    k, v = make_kv_cache(cfg, BATCH, PAST + 1, PAST, seed=1)
+    # each timed step is one full oracle decode step; warm-up steps are untimed
+    import numpy as np
+    import oracle
+    from persistent_megakernel_interpreter_b200.inputs import make_tokens
+    om = oracle.Model(cfg, w)
+    kc, vc = oracle.bits(k).copy(), oracle.bits(v).copy()
+    toks = make_tokens(cfg, 1, seed=2).numpy()
+    threads = oracle.max_threads()
+    steps = max(1, min(args.steps, 20))
+    for _ in range(min(args.warmup, 2)):
+        om.decode_step(toks, np.array([PAST]), kc, vc, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        om.decode_step(toks, np.array([PAST]), kc, vc, threads=threads)
+    el = time.perf_counter() - t0
+    value = BATCH * steps / el
+    sample = f"{steps} full decode steps of the workload (oracle, fp32 C, {threads} threads)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 2),
+            "ms_per_step": 1e3 * el / steps, "us_per_step": 1e6 * el / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_mk(args):
+    import numpy as np
+    import torch
+    rank, world, local, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from persistent_megakernel_interpreter_b200.config import LLAMA_1B
+    from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
+    from persistent_megakernel_interpreter_b200.model import Megakernel
+    cfg = LLAMA_1B
+    w = make_weights(cfg, seed=0)
+    k, v = make_kv_cache(cfg, BATCH, PAST + 1, PAST, seed=1)
+    mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=PAST + 1)
+    torch.cuda.empty_cache()
+    info = mk.build_schedule(BATCH, PAST + 1)
+    kd, vd = k.to(dev), v.to(dev)
+    tokens = make_tokens(cfg, BATCH, seed=2).to(dev)
+    positions = torch.full((BATCH,), PAST, dtype=torch.int32, device=dev)
+    logits = torch.empty(BATCH, cfg.vocab, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    bytes_step = cfg.step_bytes(BATCH, PAST)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+
+    # ---------------- device-timed megakernel steps
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            mk.decode_step(tokens, positions, kd, vd, logits, stream)
+    code, msg = mk.status()
+    if code != 0:
+        raise RuntimeError(f"warm-up step failed: {msg}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local) as clocks:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            mk.decode_step(tokens, positions, kd, vd, logits, stream)
+            ev[i][1].record(stream)
+        end.record(stream)
+        barrier()
+    elapsed = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    code, msg = mk.status()
+    if code != 0:
+        raise RuntimeError(f"timed step failed: {msg}")
+    t_max, units = aggregate(elapsed, BATCH * args.steps, dist, dev if dist is not None and
+                             torch.distributed.get_backend() == "nccl" else None)
+
+    # ---------------- end to end through the host-buffer entry point
+    th = torch.zeros(BATCH, dtype=torch.int32).pin_memory()
+    th.copy_(tokens.cpu())
+    ph = torch.full((BATCH,), PAST, dtype=torch.int32).pin_memory()
+    lh = torch.empty(BATCH, cfg.vocab, dtype=torch.float32).pin_memory()
+    for _ in range(min(args.warmup, 10)):
+        mk.decode_step_host(th, ph, kd, vd, lh, stream)
+    e2e_steps = max(1, args.steps // 4)
+    barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        mk.decode_step_host(th, ph, kd, vd, lh, stream)
+    s1.record(stream)
+    barrier()
+    e2e_max, e2e_units = aggregate(s0.elapsed_time(s1), BATCH * e2e_steps, dist,
+                                   dev if dist is not None and torch.distributed.get_backend() == "nccl" else None)
+
+    # ---------------- the multi-kernel bubble baseline, replayed from a CUDA graph
+    base = None
+    if not args.skip_baseline:
+        with torch.cuda.stream(stream):
+            mk.baseline_decode_step(tokens, positions, kd, vd, logits, stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                mk.baseline_decode_step(tokens, positions, kd, vd, logits, stream)
+            for _ in range(args.warmup):
+                g.replay()
+        nb = max(1, args.steps // 4)
+        barrier()
+        b0 = torch.cuda.Event(enable_timing=True)
+        b1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            b0.record(stream)
+            for _ in range(nb):
+                g.replay()
+            b1.record(stream)
+        barrier()
+        bt, _ = aggregate(b0.elapsed_time(b1), nb, dist,
+                          dev if dist is not None and torch.distributed.get_backend() == "nccl" else None)
+        base = {"us_per_step": 1e3 * bt / nb, "launches_per_step": 2 + 6 * cfg.n_layers,
+                "replay": "CUDA graph"}
+        del g
+        code, msg = mk.status()
+        if code != 0:
+            raise RuntimeError(f"baseline step failed: {msg}")
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        val, n, threads, sps = time_oracle(cfg, w, k, v, args.cpu_budget)
+        cpu = {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} full decode step(s) of this workload, {sps:.2f} s each"}
+
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        per_launch_ms = statistics.mean(launch_ms)
+        achieved = bytes_step / (per_launch_ms * 1e-3) / 1e9
+        traffic = profiled_traffic()
+        ms_per_step = t_max / args.steps
+        line = {
+            "metric": METRIC, "value": units / (t_max * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "us_per_step": 1e3 * ms_per_step,
+            "us_per_launch_median": 1e3 * statistics.median(launch_ms),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                         "traffic": traffic, "algorithmic_bytes": bytes_step,
+                         "kernel": "megakernel"},
+            "e2e": {"value": e2e_units / (e2e_max * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * 4 * BATCH,
+                    "d2h_bytes_per_step": 4 * BATCH * cfg.vocab,
+                    "us_per_step": 1e3 * e2e_max / e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "multikernel_baseline": base,
+            "schedule": {"n_sm": info.n_sm, "instructions": info.n_instr,
+                         "ring_stages": info.n_stages, "stage_bytes": info.stage_bytes,
+                         "attn_partitions": info.n_parts},
+        }
+        print(json.dumps(line), flush=True)
+    mk.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mk(args)
+
+
+if __name__ == "__main__":
+    main()

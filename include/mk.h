@@ -1,0 +1,228 @@
+/*
+ * mk.h -- C ABI of the persistent decode megakernel library (libmk.so).
+ *
+ * One decode step of a Llama-style decoder (batch 1 or a few sequences) runs as
+ * ONE persistent sm_100a kernel: one CTA per SM, each working through a
+ * host-built list of instructions, with dependencies between instructions
+ * expressed as counters in global memory rather than kernel boundaries. This is
+ * the design of the "Look Ma, No Bubbles" Llama-3.2-1B megakernel (summaries:
+ * sections "Fusing Operations with an On-GPU Interpreter" and "Custom
+ * Synchronization Mechanism") and of the Cohere decode megakernel (section
+ * "Megakernel 是什么": a resident block per SM reading a host-written task list of
+ * tile-sized work items, with atomic-increment / spin-wait counters).
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented as "device" must be CUDA device memory of the handle's
+ *     device; "host" pointers are ordinary host memory.
+ *   - bf16 tensors are arrays of uint16 bit patterns (IEEE bfloat16), row-major.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - No entry point throws; each returns an mk_status. Host-checkable errors are
+ *     returned before anything is enqueued. Errors found by the GPU during a step
+ *     are recorded on the device and reported by mk_get_status().
+ *   - A handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mk_status {
+    MK_OK = 0,
+    MK_ERR_INVALID_ARG = 1,   /* null pointer, bad size, batch > schedule batch ... */
+    MK_ERR_CUDA = 2,          /* a CUDA runtime call failed (message via mk_get_status) */
+    MK_ERR_UNSUPPORTED = 3,   /* shape this build has no kernel for, or the device cannot
+                                 keep one CTA resident on every SM */
+    MK_ERR_NO_SCHEDULE = 4,   /* mk_decode_step before mk_build_schedule */
+    MK_ERR_TIMEOUT = 5,       /* device: a counter or barrier wait ran past its budget */
+    MK_ERR_BAD_TOKEN = 6,     /* device: token outside [0, vocab) */
+    MK_ERR_BAD_POSITION = 7,  /* device: position outside [0, min(max_seq, max_ctx)) */
+    MK_ERR_OUT_OF_MEMORY = 8
+} mk_status;
+
+/* Model shape. The decoder is Llama-style: RMSNorm (eps inside the root),
+ * rotate-half RoPE with inv_freq_i = rope_theta^(-2i/head_dim), grouped-query
+ * attention (query head h reads KV head h / (n_heads / n_kv_heads)), SiLU-gated
+ * MLP, tied embeddings (the embedding table is also the LM head). */
+typedef struct mk_config {
+    int32_t n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
+    float rms_eps;
+    double rope_theta;
+    int32_t max_batch;   /* batch dimension of the KV cache and largest schedulable batch */
+    int32_t max_seq;     /* slot dimension of the KV cache */
+} mk_config;
+
+/* Weight pointers for mk_create. Matrices are bf16 row-major [out][in]:
+ *   wq [n_heads*head_dim][hidden], wk/wv [n_kv_heads*head_dim][hidden],
+ *   wo [hidden][n_heads*head_dim], wgate/wup [ffn][hidden], wdown [hidden][ffn],
+ *   embed [vocab][hidden]; norm vectors bf16 [hidden].
+ * Per-layer fields are HOST arrays of n_layers pointers. With mk_create the
+ * pointed-to tensors are device memory; with mk_pack_weights_host they are host
+ * memory. The library copies what it needs: the caller may free them after the
+ * call returns. */
+typedef struct mk_weights {
+    const void* embed;
+    const void* const* attn_norm;
+    const void* const* wq;
+    const void* const* wk;
+    const void* const* wv;
+    const void* const* wo;
+    const void* const* mlp_norm;
+    const void* const* wgate;
+    const void* const* wup;
+    const void* const* wdown;
+    const void* final_norm;
+} mk_weights;
+
+typedef struct mk_handle mk_handle;
+
+/* Create a handle on `device`: validates the shape, packs the weights into one
+ * library-owned device buffer (layout: see mk_pack_weights_host), builds the RoPE
+ * table (angles in double, cos/sin stored as float) and allocates the scratch
+ * (activations, attention partials, counters). Synchronous. On error *out is NULL. */
+mk_status mk_create(const mk_config* cfg, const mk_weights* w, int device, mk_handle** out);
+
+/* Options for mk_build_schedule; pass NULL for defaults. Zero fields mean "auto". */
+typedef struct mk_schedule_opts {
+    int32_t n_sm;            /* SMs to use (<= device SMs); 0 = all */
+    int32_t part_keys;       /* keys per attention partition (multiple of the ring's
+                                keys-per-stage); 0 = sized so partitions cover the SMs */
+    int32_t tiles_qkv;       /* 4-row tiles per instruction, per op; 0 = defaults */
+    int32_t tiles_o;
+    int32_t tiles_gateup;
+    int32_t rowblocks_down;
+    int32_t tiles_lm;
+    uint32_t seed;           /* 0 = plain greedy placement; else ties are broken by a
+                                seeded shuffle (for robustness tests) */
+    int32_t wait_timeout_ms; /* budget of every device wait; 0 = 2000 ms */
+    int32_t test_drop_item;  /* failure-detection test hook: 1-based index, in the global
+                                order, of one work item to leave out (its counter then never
+                                completes and the step ends with MK_ERR_TIMEOUT); 0 = none */
+} mk_schedule_opts;
+
+/* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)
+ * whose steps use at most `max_ctx` keys (position + 1 <= max_ctx <= max_seq), and
+ * upload them. Replaces any earlier schedule. Synchronous. */
+mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts);
+
+/* One decode step of the persistent megakernel, asynchronous on `stream`.
+ *   tokens, positions : device int32 [batch]
+ *   k_cache, v_cache  : device bf16 [n_layers][max_batch][n_kv_heads][max_seq][head_dim],
+ *                       caller-owned; sequence b reads slots 0..positions[b] and writes
+ *                       slot positions[b] (its RoPE'd key and its value)
+ *   logits            : device fp32 [batch][vocab]
+ * Enqueues exactly one cooperative kernel launch; no host synchronisation, no
+ * allocation. A step with a bad token or position writes no KV slot and leaves the
+ * logits unspecified; the error is reported by mk_get_status. */
+mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions,
+                         void* k_cache, void* v_cache, float* logits, void* stream);
+
+/* The same step as a sequence of ordinary kernels (one per op and layer), the
+ * multi-kernel "bubble" baseline; identical arguments, identical arithmetic, so
+ * its results equal mk_decode_step's bit for bit. Capturable in a CUDA graph. */
+mk_status mk_baseline_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions,
+                                  void* k_cache, void* v_cache, float* logits, void* stream);
+
+/* End-to-end step from HOST buffers: copies tokens and positions (host int32
+ * [batch], preferably pinned) to the device, runs mk_decode_step, copies the
+ * logits back to `logits_host` (fp32 [batch][vocab]) and synchronises `stream`.
+ * Uses handle-owned device staging (no allocation per call). Returns the
+ * host-side status; device-detected errors are reported by mk_get_status. */
+mk_status mk_decode_step_host(mk_handle* h, const int32_t* tokens_host,
+                              const int32_t* positions_host, void* k_cache, void* v_cache,
+                              float* logits_host, void* stream);
+
+/* Synchronises the device, then reports and clears the device-side error state.
+ * *device_status receives the first error recorded since the last call (MK_OK if
+ * none); msg (may be NULL) receives a one-line description. After an error every
+ * step is skipped until this call clears it. Returns MK_ERR_CUDA if the sync fails. */
+mk_status mk_get_status(mk_handle* h, mk_status* device_status, char* msg, size_t msg_len);
+
+/* Frees everything the handle owns. NULL is allowed. */
+void mk_destroy(mk_handle* h);
+
+const char* mk_status_str(mk_status s);
+
+/* ------------------------------------------------------------------ inspection */
+
+/* One instruction of the per-SM lists (48 bytes). The kinds: */
+enum {
+    MK_OP_QKV = 1,     /* RMSNorm + QKV matvec + RoPE; writes q and the KV slot */
+    MK_OP_ATTN = 2,    /* split-K GQA attention partial; the last partition merges */
+    MK_OP_OPROJ = 3,   /* O-projection + residual */
+    MK_OP_GATEUP = 4,  /* RMSNorm + gate/up matvec + SiLU-gated product */
+    MK_OP_DOWN = 5,    /* down-projection over 4 chunks + residual */
+    MK_OP_LMHEAD = 6   /* final RMSNorm + LM head */
+};
+#define MK_NO_COUNTER 0xffffffffu
+
+typedef struct mk_instr {
+    uint16_t op, layer;
+    uint16_t batch;      /* sequence (MK_OP_ATTN), else 0 */
+    uint16_t group;      /* KV group (QKV, ATTN) or MLP chunk (GATEUP), else 0 */
+    uint32_t first;      /* first 4-row tile / row block (DOWN) / first key (ATTN) */
+    uint32_t count;      /* tiles / row blocks / keys */
+    uint32_t seq;        /* index of its first ring stage fill in this SM's stream */
+    uint32_t nfill;      /* ring stage fills it consumes */
+    uint32_t wait_ctr;   /* counter waited on (MK_NO_COUNTER: none); DOWN waits on the
+                            4 consecutive chunk counters wait_ctr .. wait_ctr+3 */
+    uint32_t wait_n;     /* increments that counter receives per step */
+    uint32_t signal_ctr; /* counter incremented by one when done */
+    uint32_t aux_ctr;    /* ATTN: counter incremented by the merging (last) partition */
+    uint32_t aux_n;      /* ATTN: partitions per (sequence, group) */
+    uint32_t reserved;
+} mk_instr;
+
+typedef struct mk_schedule_info {
+    int32_t n_sm, batch, max_ctx, part_keys, n_parts, keys_per_stage;
+    int32_t stage_bytes, n_stages, n_counters, n_instr;
+    uint64_t bytes_per_step;    /* weight + KV bytes one step streams */
+    uint64_t max_sm_bytes;      /* largest per-SM share of those bytes */
+    uint64_t min_sm_bytes;
+} mk_schedule_info;
+
+/* Plans a schedule on the host only (no device, no handle): writes up to
+ * `cap` instructions to instr_out (may be NULL to query), n_sm+1 list offsets to
+ * sm_offsets (may be NULL) and the summary to info. `stage_bytes` is the ring
+ * stage size the kernel would use (0 = the library's choice for this shape).
+ * Returns MK_ERR_INVALID_ARG if cap is too small (info->n_instr says how many). */
+mk_status mk_plan_schedule_host(const mk_config* cfg, int batch, int max_ctx, int n_sm,
+                                const mk_schedule_opts* opts, mk_instr* instr_out, size_t cap,
+                                int32_t* sm_offsets, mk_schedule_info* info);
+
+/* Summary of the handle's current schedule. */
+mk_status mk_get_schedule_info(mk_handle* h, mk_schedule_info* info);
+
+/* Copies the handle's step counters (uint32 each) to host memory: the
+ * dependency counters, then epoch, then the end-of-step arrival count.
+ * *n_total receives how many exist; at most n are copied. Synchronous. */
+mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_total);
+
+/* Bytes of the packed weight buffer for `cfg`. */
+size_t mk_packed_bytes(const mk_config* cfg);
+
+/* Packs host weights into `dst` (host, mk_packed_bytes(cfg) bytes) with the same
+ * layout mk_create builds on the device, 256-byte aligned regions in this order:
+ *   embed      [vocab][hidden] unchanged (it is also the LM head);
+ *   per layer:
+ *     QKV      4-row tiles of [4][hidden]; KV group g holds, in order, its
+ *              n_heads/n_kv_heads query heads, key head g, value head g; a query or
+ *              key head's tile j holds rows {2j, 2j+d/2, 2j+1, 2j+1+d/2} (the two
+ *              RoPE pairs), a value head's tile j rows {4j..4j+3};
+ *     O        wo unchanged [hidden][n_heads*head_dim];
+ *     gate/up  tile j = rows {gate 2j, up 2j, gate 2j+1, up 2j+1} of [4][hidden];
+ *     down     for row block r (rows 4r..4r+3), chunk c (columns c*ffn/4 ..): a
+ *              [4][ffn/4] tile, ordered [r][c];
+ *   norms      attn_norm[l], mlp_norm[l] for each layer, then final_norm.
+ * Bit copy only. */
+mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights* w, void* dst,
+                               size_t dst_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

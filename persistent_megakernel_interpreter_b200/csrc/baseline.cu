@@ -1,0 +1,170 @@
+// The multi-kernel "bubble" baseline: the same decode step as one ordinary
+// kernel per op and layer (about six launches per layer), the structure the
+// megakernel write-ups measure against (the "Look Ma, No Bubbles" summaries,
+// section "Memory Pipeline Bubbles Explained": every kernel boundary waits for
+// stragglers, pays launch and teardown, and cannot prefetch the next op's
+// weights). It uses the very same tile, epilogue and attention routines as the
+// megakernel, with weights read straight from global memory, so the two give
+// bit-identical results. Capturable in a CUDA graph.
+#include <cuda_runtime.h>
+
+#include "mk_device.cuh"
+
+namespace mk {
+
+constexpr int kBaseWarps = 8;
+constexpr int kBaseThreads = 32 * kBaseWarps;
+
+__device__ __forceinline__ bool step_failed(const Params& p) {
+    return ld_volatile_u32(&p.ctl->status) != 0u;
+}
+
+// Token and position checks, once per step, before any other kernel.
+__global__ void k_validate(const __grid_constant__ Params p) {
+    if (threadIdx.x != 0 || step_failed(p)) return;
+    for (int b = 0; b < p.B; ++b) {
+        const int tok = p.tokens[b], pos = p.positions[b];
+        uint32_t code = 0;
+        if (tok < 0 || tok >= p.V) code = MK_ERR_BAD_TOKEN;
+        else if (pos < 0 || pos >= p.max_seq || pos + 1 > p.max_ctx) code = MK_ERR_BAD_POSITION;
+        if (code) {
+            if (atomicCAS(&p.ctl->status, 0u, code) == 0u) {
+                p.ctl->info[0] = 0xffffffffu;
+                p.ctl->info[1] = b;
+                p.ctl->info[2] = (uint32_t)tok;
+                p.ctl->info[3] = (uint32_t)pos;
+            }
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ const uint8_t* op_tiles(const Params& p, int op, int l) {
+    const size_t lb = p.off_layer0 + (size_t)l * p.layer_stride;
+    switch (op) {
+        case MK_OP_QKV: return p.packed + lb + p.rel_qkv;
+        case MK_OP_OPROJ: return p.packed + lb + p.rel_o;
+        case MK_OP_GATEUP: return p.packed + lb + p.rel_gu;
+        default: return p.packed;  // LM head: the embedding table
+    }
+}
+
+template <int OP, int KC, int HD>
+__global__ void __launch_bounds__(kBaseThreads) k_tiles(const __grid_constant__ Params p, int l,
+                                                        uint32_t ntiles, uint32_t tile_bytes) {
+    if (step_failed(p)) return;
+    const int lane = threadIdx.x & 31;
+    const uint32_t gw = blockIdx.x * kBaseWarps + (threadIdx.x >> 5);
+    const uint32_t nw = gridDim.x * kBaseWarps;
+    if (gw >= ntiles) return;
+    const uint64_t pol = l2_evict_first_policy();
+    const uint8_t* base = op_tiles(p, OP, l);
+    uint32_t x[KC][4];
+    if (p.B == 1) prep_input<OP, KC>(p, l, 0, x, lane);
+    for (uint32_t t = gw; t < ntiles; t += nw) {
+        for (int b = 0; b < p.B; ++b) {
+            if (p.B > 1) prep_input<OP, KC>(p, l, b, x, lane);
+            float acc[4];
+            dot4<KC, false>(base + (size_t)t * tile_bytes, x, acc, lane, pol);
+            tile_epilogue<OP, HD>(p, l, b, t, acc, lane);
+        }
+    }
+}
+
+template <int KF>
+__global__ void __launch_bounds__(kBaseThreads) k_down(const __grid_constant__ Params p, int l) {
+    if (step_failed(p)) return;
+    const int lane = threadIdx.x & 31;
+    const uint32_t gw = blockIdx.x * kBaseWarps + (threadIdx.x >> 5);
+    const uint32_t nw = gridDim.x * kBaseWarps;
+    const uint64_t pol = l2_evict_first_policy();
+    const uint8_t* base = p.packed + p.off_layer0 + (size_t)l * p.layer_stride + p.rel_down;
+    const uint32_t nrb = p.H / 4;
+    for (uint32_t rb = gw; rb < nrb; rb += nw) {
+        for (int b = 0; b < p.B; ++b) {
+            float tot[4];
+            uint32_t x[KF][4];
+            for (int c = 0; c < 4; ++c) {
+                load_vec<KF>(p.hbuf + (size_t)b * p.F + (size_t)c * (p.F / 4), x, lane);
+                float acc[4];
+                dot4<KF, false>(base + ((size_t)rb * 4 + c) * p.tile_f, x, acc, lane, pol);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) tot[k] = (c == 0) ? acc[k] : tot[k] + acc[k];
+            }
+            residual_epilogue(p, p.x + (size_t)b * p.H, b, rb, tot, lane);
+        }
+    }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kBaseThreads) k_attn_partial(const __grid_constant__ Params p, int l) {
+    if (step_failed(p)) return;
+    extern __shared__ float sbuf_all[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gw = blockIdx.x * kBaseWarps + warp;
+    const int j = gw % p.n_parts, g = (gw / p.n_parts) % p.nkv, b = gw / (p.n_parts * p.nkv);
+    if (b >= p.B) return;
+    float* sbuf = sbuf_all + (size_t)warp * kMaxGroup * p.keys_per_stage;
+    const int pos = p.positions[b];
+    const int k0 = j * p.part_keys, k1 = min(k0 + p.part_keys, p.max_ctx);
+    AttnState<HD> st;
+    attn_init<HD>(p, b, g, st, lane);
+    const uint16_t* Kpos = p.kc + kv_off(p, l, b, g, pos);
+    const uint16_t* Vpos = p.vc + kv_off(p, l, b, g, pos);
+    for (int ka = k0; ka < k1; ka += p.keys_per_stage) {
+        const int kend = min(min(ka + p.keys_per_stage, k1), pos + 1);
+        if (ka >= kend) break;
+        attn_chunk<HD, false>(p, st, p.kc + kv_off(p, l, b, g, ka), p.vc + kv_off(p, l, b, g, ka),
+                              Kpos, Vpos, ka, kend, pos, sbuf, p.keys_per_stage, lane);
+    }
+    attn_store_partial<HD>(p, st, b, g, j, lane);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kBaseThreads) k_attn_merge(const __grid_constant__ Params p) {
+    if (step_failed(p)) return;
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kBaseWarps + (threadIdx.x >> 5);
+    if (gw >= p.B * p.nkv) return;
+    attn_merge<HD>(p, gw / p.nkv, gw % p.nkv, lane);
+}
+
+// ------------------------------------------------------------------ host-side launch
+
+template <int KH, int KO, int KF, int HD>
+static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
+    const uint32_t warps_cap = (uint32_t)n_sm * 16;
+    auto blocks_for = [&](uint32_t units) {
+        const uint32_t w = units < warps_cap ? units : warps_cap;
+        return (w + kBaseWarps - 1) / kBaseWarps;
+    };
+    const size_t attn_smem = (size_t)kBaseWarps * kMaxGroup * p.keys_per_stage * sizeof(float);
+    k_validate<<<1, 32, 0, st>>>(p);
+    const uint32_t tpg = (uint32_t)(p.group + 2) * (HD / 4);
+    for (int l = 0; l < p.L; ++l) {
+        const uint32_t nq = (uint32_t)p.nkv * tpg;
+        k_tiles<MK_OP_QKV, KH, HD><<<blocks_for(nq), kBaseThreads, 0, st>>>(p, l, nq, p.tile_h);
+        const uint32_t na = (uint32_t)(p.B * p.nkv * p.n_parts);
+        k_attn_partial<HD><<<(na + kBaseWarps - 1) / kBaseWarps, kBaseThreads, attn_smem, st>>>(p, l);
+        const uint32_t nm = (uint32_t)(p.B * p.nkv);
+        k_attn_merge<HD><<<(nm + kBaseWarps - 1) / kBaseWarps, kBaseThreads, 0, st>>>(p);
+        const uint32_t no = (uint32_t)p.H / 4;
+        k_tiles<MK_OP_OPROJ, KO, HD><<<blocks_for(no), kBaseThreads, 0, st>>>(p, l, no, p.tile_o);
+        const uint32_t ng = (uint32_t)p.F / 2;
+        k_tiles<MK_OP_GATEUP, KH, HD><<<blocks_for(ng), kBaseThreads, 0, st>>>(p, l, ng, p.tile_h);
+        k_down<KF><<<blocks_for((uint32_t)p.H / 4), kBaseThreads, 0, st>>>(p, l);
+    }
+    const uint32_t nl = (uint32_t)p.V / 4;
+    k_tiles<MK_OP_LMHEAD, KH, HD><<<blocks_for(nl), kBaseThreads, 0, st>>>(p, 0, nl, p.tile_h);
+    return cudaGetLastError();
+}
+
+cudaError_t baseline_launch(const Params& p, cudaStream_t stream, int n_sm) {
+    const int KH = p.H / 256, KO = p.Q / 256, KF = p.F / 1024;
+    if (KH == 2 && KO == 2 && KF == 2 && p.d == 64) return launch_all<2, 2, 2, 64>(p, stream, n_sm);
+    if (KH == 8 && KO == 8 && KF == 8 && p.d == 64) return launch_all<8, 8, 8, 64>(p, stream, n_sm);
+    if (KH == 12 && KO == 12 && KF == 8 && p.d == 128) return launch_all<12, 12, 8, 128>(p, stream, n_sm);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mk

@@ -1,0 +1,576 @@
+// Device building blocks shared by the persistent megakernel and the
+// multi-kernel baseline: PTX wrappers, the 4-row matvec tile, the fused
+// epilogues (RoPE + KV append, residual add, SiLU-gated product, logits) and
+// split-K decode attention with its merge.
+//
+// Work split inside a warp (batch-1 matvec, the memory-bound case the
+// megakernel write-ups target): lane `ln` owns input elements
+// (kc*32 + ln)*8 .. +7 for kc = 0..KC-1 (KC = in_dim / 256), holds them as fp32
+// in registers and reads the matching 16-byte pieces of each weight row, so
+// one warp-wide load covers 512 contiguous bytes of a row. Partial sums are
+// combined with an xor butterfly, which leaves the identical total in every
+// lane (each step adds the same two values in either order).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// One-dimensional bulk copy global -> this CTA's shared memory, completion
+// counted on `bar` (transaction bytes). No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Activations written earlier in the same kernel by other SMs: read at L2 (.cg).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint2 ld_cg_v2(const void* p) {
+    uint2 r;
+    asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_cg_u32(const void* p) {
+    uint32_t r;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ float ld_cg_f32(const float* p) {
+    float r;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(r) : "l"(p));
+    return r;
+}
+
+// Weights streamed once per step: read-only path, no L1 allocation, evict-first in L2.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p, uint64_t pol) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(pol));
+    return r;
+}
+
+__device__ __forceinline__ uint4 lds_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(smem_addr(p)));
+    return r;
+}
+
+// ------------------------------------------------------------------ bf16 helpers
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ float bf2f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+__device__ __forceinline__ float round_bf(float f) { return bf2f(f2bf(f)); }
+
+__device__ __forceinline__ void unpack8(uint4 u, float* v) {
+    v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+    v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
+}
+
+// Element `lane` (0..3) of a 4-vector without a dynamically indexed array.
+__device__ __forceinline__ float pick4(const float (&a)[4], int i) {
+    return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+    return v;
+}
+
+// ------------------------------------------------------------------ vectors in registers
+
+// Load a bf16 vector of KC*256 elements into the lane layout described above,
+// kept as packed bf16 pairs (the vectors a matvec consumes are bf16 values).
+template <int KC>
+__device__ __forceinline__ void load_vec(const uint16_t* src, uint32_t (&x)[KC][4], int lane) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        const uint4 u = ld_cg_v4(s + kc * 32 + lane);
+        x[kc][0] = u.x; x[kc][1] = u.y; x[kc][2] = u.z; x[kc][3] = u.w;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+}
+
+// RMSNorm in place on the register vector: x <- bf16((x * r) * w) with
+// r = 1 / sqrt(mean(x^2) + eps), mean over the KC*256 elements.
+template <int KC>
+__device__ __forceinline__ void rmsnorm_regs(uint32_t (&x)[KC][4], const uint16_t* w, float eps,
+                                             int lane) {
+    float ss = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = bf_lo(x[kc][e]), b = bf_hi(x[kc][e]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    ss = warp_sum(ss);
+    const float r = 1.0f / sqrtf(ss / (float)(KC * 256) + eps);
+    const uint4* wp = reinterpret_cast<const uint4*>(w);
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        const uint4 wv = ld_cg_v4(wp + kc * 32 + lane);
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __fmul_rn(__fmul_rn(bf_lo(x[kc][e]), r), bf_lo(ww[e]));
+            const float hi = __fmul_rn(__fmul_rn(bf_hi(x[kc][e]), r), bf_hi(ww[e]));
+            x[kc][e] = pack_bf2(lo, hi);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ the 4-row tile
+
+// acc += w.lo * x.lo; acc += w.hi * x.hi -- fp32 accumulation of exact bf16
+// products (the mixed-precision fma of sm_100), no unpacking.
+__device__ __forceinline__ void fma_bf2(float& acc, uint32_t w, uint32_t x) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w), "r"(x));
+}
+
+// acc[r] = W_tile[r] . x for the 4 rows of a [4][KC*256] bf16 tile. The tile is
+// in shared memory (SMEM) or read straight from global memory. Every lane
+// returns the same four totals.
+template <int KC, bool SMEM>
+__device__ __forceinline__ void dot4(const uint8_t* tile, const uint32_t (&x)[KC][4],
+                                     float (&acc)[4], int lane, uint64_t pol) {
+    const uint4* t = reinterpret_cast<const uint4*>(tile);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r] = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        uint4 w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint4* a = t + r * KC * 32 + kc * 32 + lane;
+            w[r] = SMEM ? lds_v4(a) : ld_stream_v4(a, pol);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            fma_bf2(acc[r], w[r].x, x[kc][0]);
+            fma_bf2(acc[r], w[r].y, x[kc][1]);
+            fma_bf2(acc[r], w[r].z, x[kc][2]);
+            fma_bf2(acc[r], w[r].w, x[kc][3]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r] = warp_sum(acc[r]);
+}
+
+// ------------------------------------------------------------------ per-op helpers
+
+__device__ __forceinline__ const uint16_t* norm_ptr(const Params& p, size_t off) {
+    return reinterpret_cast<const uint16_t*>(p.packed + off);
+}
+
+// Residual-stream input of layer l for sequence b: the embedding row at layer 0.
+__device__ __forceinline__ const uint16_t* x_in(const Params& p, int l, int b) {
+    if (l == 0) {
+        const int tok = p.tokens[b];
+        return reinterpret_cast<const uint16_t*>(p.packed) + (size_t)tok * p.H;
+    }
+    return p.x + (size_t)b * p.H;
+}
+
+__device__ __forceinline__ size_t kv_off(const Params& p, int l, int b, int g, int slot) {
+    return ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.max_seq + slot) * p.d;
+}
+
+// QKV tile epilogue: RoPE on query/key pairs, round to bf16 [R2], store q or the
+// KV slot. `tile` is the tile index inside the layer's QKV block.
+template <int HD>
+__device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint32_t tile,
+                                             const float (&acc)[4], int lane) {
+    if (lane >= 4) return;
+    constexpr int TPH = HD / 4;  // tiles per head
+    const int g = tile / (uint32_t)((p.group + 2) * TPH);
+    const int u = tile % (uint32_t)((p.group + 2) * TPH);
+    const int hs = u / TPH, j = u % TPH;
+    const int pos = p.positions[b];
+    if (hs <= p.group) {
+        // query head (hs < group) or key head (hs == group): rows {2j, 2j+d/2, 2j+1, 2j+1+d/2}
+        const int pair = lane >> 1;          // 0: freq 2j, 1: freq 2j+1
+        const int i = 2 * j + pair;
+        const float a = pair ? acc[2] : acc[0], bb = pair ? acc[3] : acc[1];
+        const float c = p.rope_cos[(size_t)pos * (HD / 2) + i];
+        const float s = p.rope_sin[(size_t)pos * (HD / 2) + i];
+        float out;
+        int dim;
+        if ((lane & 1) == 0) {
+            out = __fsub_rn(__fmul_rn(a, c), __fmul_rn(bb, s));
+            dim = i;
+        } else {
+            out = __fadd_rn(__fmul_rn(bb, c), __fmul_rn(a, s));
+            dim = i + HD / 2;
+        }
+        if (hs < p.group) {
+            const int head = g * p.group + hs;
+            p.q[(size_t)b * p.Q + (size_t)head * HD + dim] = f2bf(out);
+        } else {
+            p.kc[kv_off(p, l, b, g, pos) + dim] = f2bf(out);
+        }
+    } else {
+        p.vc[kv_off(p, l, b, g, pos) + 4 * j + lane] = f2bf(pick4(acc, lane));
+    }
+}
+
+__device__ __forceinline__ uint16_t ld_cg_u16(const uint16_t* p) {
+    uint16_t r;
+    asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+// x[b][row] = bf16(xin[row] + y) [R4, R6]. `xin` is the residual input (the
+// embedding row at layer 0, else x itself).
+__device__ __forceinline__ void residual_one(const Params& p, const uint16_t* xin, int b,
+                                             uint32_t row, float y) {
+    const float xv = bf2f(ld_cg_u16(xin + row));
+    p.x[(size_t)b * p.H + row] = f2bf(__fadd_rn(xv, y));
+}
+
+// The tile's 4 consecutive rows; lanes 0..3 write one each.
+__device__ __forceinline__ void residual_epilogue(const Params& p, const uint16_t* xin, int b,
+                                                  uint32_t tile, const float (&acc)[4], int lane) {
+    if (lane >= 4) return;
+    residual_one(p, xin, b, tile * 4 + lane, pick4(acc, lane));
+}
+
+// gate/up tile rows {g 2j, u 2j, g 2j+1, u 2j+1}: h = bf16((g / (1 + e^-g)) * u) [R5].
+__device__ __forceinline__ void gateup_epilogue(const Params& p, int b, uint32_t tile,
+                                                const float (&acc)[4], int lane) {
+    if (lane >= 2) return;
+    const float g = lane ? acc[2] : acc[0], u = lane ? acc[3] : acc[1];
+    const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+    p.hbuf[(size_t)b * p.F + 2 * tile + lane] = f2bf(__fmul_rn(silu, u));
+}
+
+__device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t tile,
+                                                const float (&acc)[4], int lane) {
+    if (lane >= 4) return;
+    p.logits[(size_t)b * p.V + tile * 4 + lane] = pick4(acc, lane);
+}
+
+// ------------------------------------------------------------------ matvec op inputs/outputs
+
+// Input vector of a matvec op for sequence b, in registers.
+template <int OP, int KC>
+__device__ __forceinline__ void prep_input(const Params& p, int l, int b, uint32_t (&x)[KC][4], int lane) {
+    if constexpr (OP == MK_OP_QKV) {
+        load_vec<KC>(x_in(p, l, b), x, lane);
+        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2), p.eps, lane);
+    } else if constexpr (OP == MK_OP_GATEUP) {
+        load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
+        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, lane);
+    } else if constexpr (OP == MK_OP_OPROJ) {
+        load_vec<KC>(p.attn + (size_t)b * p.Q, x, lane);
+    } else {  // LM head
+        load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
+        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, lane);
+    }
+}
+
+template <int OP, int HD>
+__device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uint32_t tile,
+                                              const float (&acc)[4], int lane) {
+    if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD>(p, l, b, tile, acc, lane);
+    else if constexpr (OP == MK_OP_GATEUP) gateup_epilogue(p, b, tile, acc, lane);
+    else if constexpr (OP == MK_OP_OPROJ) residual_epilogue(p, x_in(p, l, b), b, tile, acc, lane);
+    else logits_epilogue(p, b, tile, acc, lane);
+}
+
+// ------------------------------------------------------------------ decode attention
+
+// Lane layout for the scores: LPK lanes share one key (8 dims each); KPI keys per
+// warp-wide step. For the value sum each lane owns DPL consecutive dims.
+template <int HD>
+struct AttnShape {
+    static constexpr int LPK = HD / 8;
+    static constexpr int KPI = 32 / LPK;
+    static constexpr int DPL = HD / 32;
+};
+
+constexpr int kMaxGroup = 4;  // query heads per KV head handled by one instruction
+
+template <int HD>
+struct AttnState {
+    float q[kMaxGroup][8];                        // this lane's 8 query dims, per head
+    float m[kMaxGroup], l[kMaxGroup];             // running max and sum
+    float o[kMaxGroup][AttnShape<HD>::DPL];       // running unnormalised output
+};
+
+template <int HD>
+__device__ __forceinline__ void attn_init(const Params& p, int b, int g, AttnState<HD>& st,
+                                          int lane) {
+    using S = AttnShape<HD>;
+    const int dc = lane % S::LPK;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h < p.group) {
+            const uint16_t* qh = p.q + (size_t)b * p.Q + (size_t)(g * p.group + h) * HD;
+            unpack8(ld_cg_v4(qh + dc * 8), st.q[h]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st.q[h][e] = 0.f;
+        }
+        st.m[h] = -INFINITY;
+        st.l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < S::DPL; ++e) st.o[h][e] = 0.f;
+    }
+}
+
+// One chunk of keys [ka, kend) (kend <= pos + 1, ka < kend). Rows of keys < pos
+// come from Kc/Vc (row 0 = key ka; shared memory when SMEM, else global); the
+// key at `pos`, written earlier in this step, is read from the global cache.
+// `s` is this warp's score scratch in shared memory, [kMaxGroup][ks] floats.
+template <int HD, bool SMEM>
+__device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, const uint16_t* Kc,
+                                           const uint16_t* Vc, const uint16_t* Kpos,
+                                           const uint16_t* Vpos, int ka, int kend, int pos,
+                                           float* s, int ks, int lane) {
+    using S = AttnShape<HD>;
+    const int n = kend - ka;
+    const int dc = lane % S::LPK, kk = lane / S::LPK;
+    const float scale = 1.0f / sqrtf((float)HD);
+    // scores
+    for (int base = 0; base < n; base += S::KPI) {
+        const int j = base + kk;
+        float part[kMaxGroup];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) part[h] = 0.f;
+        if (j < n) {
+            const int key = ka + j;
+            uint4 raw;
+            if (key < pos)
+                raw = SMEM ? lds_v4(Kc + (size_t)j * HD + dc * 8) : ld_cg_v4(Kc + (size_t)j * HD + dc * 8);
+            else
+                raw = ld_cg_v4(Kpos + dc * 8);
+            float kv[8];
+            unpack8(raw, kv);
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) part[h] = fmaf(st.q[h][e], kv[e], part[h]);
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+            for (int m = S::LPK / 2; m > 0; m >>= 1)
+                part[h] += __shfl_xor_sync(0xffffffffu, part[h], m);
+        if (j < n && dc < p.group) {
+            float mine = 0.f;
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h)
+                if (dc == h) mine = part[h];
+            s[dc * ks + j] = mine * scale;
+        }
+    }
+    __syncwarp();
+    // online softmax update per head
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h >= p.group) continue;
+        float cm = -INFINITY;
+        for (int j = lane; j < n; j += 32) cm = fmaxf(cm, s[h * ks + j]);
+        cm = warp_max(cm);
+        const float m_new = fmaxf(st.m[h], cm);
+        const float alpha = expf(st.m[h] - m_new);   // 0 on the first chunk (m = -inf)
+        float cs = 0.f;
+        for (int j = lane; j < n; j += 32) {
+            const float e = expf(s[h * ks + j] - m_new);
+            s[h * ks + j] = e;
+            cs += e;
+        }
+        cs = warp_sum(cs);
+        st.l[h] = fmaf(st.l[h], alpha, cs);
+#pragma unroll
+        for (int e = 0; e < S::DPL; ++e) st.o[h][e] *= alpha;
+        st.m[h] = m_new;
+    }
+    __syncwarp();
+    // values
+    for (int j = 0; j < n; ++j) {
+        const int key = ka + j;
+        float v[S::DPL];
+        const uint16_t* vr = (key < pos) ? Vc + (size_t)j * HD : Vpos;
+        const bool from_smem = SMEM && key < pos;
+        if constexpr (S::DPL == 2) {
+            const uint32_t w = from_smem ? *reinterpret_cast<const uint32_t*>(vr + lane * 2)
+                                         : ld_cg_u32(vr + lane * 2);
+            v[0] = bf_lo(w);
+            v[1] = bf_hi(w);
+        } else {
+            static_assert(S::DPL == 4, "head_dim 64 or 128");
+            const uint2 w = from_smem ? *reinterpret_cast<const uint2*>(vr + lane * 4)
+                                      : ld_cg_v2(vr + lane * 4);
+            v[0] = bf_lo(w.x);
+            v[1] = bf_hi(w.x);
+            v[2] = bf_lo(w.y);
+            v[3] = bf_hi(w.y);
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            if (h >= p.group) continue;
+            const float e = s[h * ks + j];
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d) st.o[h][d] = fmaf(e, v[d], st.o[h][d]);
+        }
+    }
+    __syncwarp();
+}
+
+// Write the partition's (m, l, o) for the group's heads.
+template <int HD>
+__device__ __forceinline__ void attn_store_partial(const Params& p, const AttnState<HD>& st, int b,
+                                                   int g, int part, int lane) {
+    using S = AttnShape<HD>;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h >= p.group) continue;
+        const size_t hp = ((size_t)b * p.nq + (size_t)(g * p.group + h)) * p.n_parts + part;
+        if (lane == 0) {
+            p.part_ml[hp * 2] = st.m[h];
+            p.part_ml[hp * 2 + 1] = st.l[h];
+        }
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = st.o[h][d];
+    }
+}
+
+// Merge the n_parts partials of (b, g) in partition order; attn = bf16(O / L) [R3].
+template <int HD>
+__device__ __forceinline__ void attn_merge(const Params& p, int b, int g, int lane) {
+    using S = AttnShape<HD>;
+    for (int h = 0; h < p.group; ++h) {
+        const int head = g * p.group + h;
+        const size_t h0 = ((size_t)b * p.nq + head) * p.n_parts;
+        float M = -INFINITY;
+        for (int j = 0; j < p.n_parts; ++j) M = fmaxf(M, ld_cg_f32(p.part_ml + (h0 + j) * 2));
+        float L = 0.f, O[S::DPL];
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d) O[d] = 0.f;
+        for (int j = 0; j < p.n_parts; ++j) {
+            const float mj = ld_cg_f32(p.part_ml + (h0 + j) * 2);
+            const float lj = ld_cg_f32(p.part_ml + (h0 + j) * 2 + 1);
+            const float w = expf(mj - M);   // empty partitions: m = -inf -> 0
+            L = fmaf(w, lj, L);
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d)
+                O[d] = fmaf(w, ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d), O[d]);
+        }
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d)
+            p.attn[(size_t)b * p.Q + (size_t)head * HD + lane * S::DPL + d] = f2bf(__fdiv_rn(O[d], L));
+    }
+}
+
+}  // namespace mk

@@ -1,0 +1,96 @@
+// Internal definitions shared by the host code and the kernels of libmk.so:
+// the packed-weight layout, the kernel parameter block, the control block.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mk.h"
+
+namespace mk {
+
+constexpr int kConsumerWarps = 8;                    // warps that execute instructions
+constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one producer (loader) warp
+constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
+constexpr int kMaxLayers = 64;
+constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
+constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Byte offsets of every packed region (see mk_pack_weights_host in mk.h).
+struct Layout {
+    int L, H, nq, nkv, d, F, V;
+    int group;            // query heads per KV head
+    int Q, KVD;           // n_heads*head_dim, n_kv_heads*head_dim
+    int qkv_rows;         // Q + 2*KVD
+    int tiles_per_group;  // 4-row QKV tiles per KV group
+    // tile sizes in bytes
+    uint32_t tile_h;      // 4 x hidden (QKV, gate/up, LM head)
+    uint32_t tile_o;      // 4 x Q (O-projection)
+    uint32_t tile_f;      // 4 x ffn/4 (down, one chunk)
+    size_t off_embed, off_layer0, layer_stride;
+    size_t rel_qkv, rel_o, rel_gu, rel_down;  // within a layer
+    size_t off_norms, total;
+
+    size_t qkv(int l) const { return off_layer0 + (size_t)l * layer_stride + rel_qkv; }
+    size_t o(int l) const { return off_layer0 + (size_t)l * layer_stride + rel_o; }
+    size_t gu(int l) const { return off_layer0 + (size_t)l * layer_stride + rel_gu; }
+    size_t down(int l) const { return off_layer0 + (size_t)l * layer_stride + rel_down; }
+    size_t attn_norm(int l) const { return off_norms + (size_t)(2 * l) * H * 2; }
+    size_t mlp_norm(int l) const { return off_norms + (size_t)(2 * l + 1) * H * 2; }
+    size_t final_norm() const { return off_norms + (size_t)(2 * L) * H * 2; }
+};
+
+// Returns false if the shape is not one the kernels handle.
+bool make_layout(const mk_config& c, Layout* out, const char** why);
+
+// Control words, one 128-byte line each (see the megakernel for their protocol).
+struct Ctl {
+    uint32_t epoch;     uint32_t pad0[31];
+    uint32_t done;      uint32_t pad1[31];
+    uint32_t status;    uint32_t abort;  uint32_t info[6]; uint32_t pad2[24];
+};
+
+// Kernel parameter block (passed by value, __grid_constant__).
+struct Params {
+    // shape
+    int L, H, nq, nkv, d, F, V, group, Q, KVD;
+    int B, max_batch, max_seq, max_ctx;
+    float eps;
+    // packed weights
+    const uint8_t* packed;
+    size_t off_layer0, layer_stride, rel_qkv, rel_o, rel_gu, rel_down, off_norms;
+    uint32_t tile_h, tile_o, tile_f;
+    const float* rope_cos;   // [max_seq][d/2]
+    const float* rope_sin;
+    // per step
+    const int32_t* tokens;
+    const int32_t* positions;
+    uint16_t* kc;
+    uint16_t* vc;
+    float* logits;
+    // scratch
+    uint16_t* x;       // [B][H]   residual stream
+    uint16_t* q;       // [B][Q]
+    uint16_t* attn;    // [B][Q]
+    uint16_t* hbuf;    // [B][F]
+    float* part_ml;    // [B][nq][P][2]  (m, l)
+    float* part_o;     // [B][nq][P][d]
+    uint32_t* counters;
+    Ctl* ctl;
+    // schedule
+    const mk_instr* instrs;
+    const int32_t* sm_off;
+    int n_sm;
+    int part_keys, n_parts, keys_per_stage;
+    uint32_t stage_bytes;
+    int n_stages;
+    int n_counters;
+    uint64_t timeout_ns;
+};
+
+// Device status codes live in Ctl::status (values of mk_status).
+
+}  // namespace mk

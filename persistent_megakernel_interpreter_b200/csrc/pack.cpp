@@ -1,0 +1,173 @@
+// Weight packer: the row order and tiling of every matrix as the kernels read
+// it (documented with mk_pack_weights_host in mk.h). The packer is a list of
+// (destination offset, source pointer, bytes) copies -- a pure bit copy -- run
+// by a gather kernel on the device (mk_create) or by memcpy on the host.
+#include <string.h>
+
+#include <vector>
+
+#include "pack.h"
+
+namespace mk {
+
+bool make_layout(const mk_config& c, Layout* out, const char** why) {
+    auto fail = [&](const char* m) {
+        if (why) *why = m;
+        return false;
+    };
+    if (c.n_layers <= 0 || c.n_layers > kMaxLayers) return fail("n_layers out of range");
+    if (c.hidden <= 0 || c.n_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 || c.ffn <= 0 ||
+        c.vocab <= 0)
+        return fail("non-positive dimension");
+    if (c.n_heads % c.n_kv_heads) return fail("n_heads must be a multiple of n_kv_heads");
+    if (c.head_dim != 64 && c.head_dim != 128) return fail("head_dim must be 64 or 128");
+    const int group = c.n_heads / c.n_kv_heads;
+    if (group > 4) return fail("more than 4 query heads per KV head");
+    if (c.hidden % 256) return fail("hidden must be a multiple of 256");
+    if ((c.n_heads * c.head_dim) % 256) return fail("n_heads*head_dim must be a multiple of 256");
+    if (c.ffn % 1024) return fail("ffn must be a multiple of 1024");
+    if (c.vocab % 4) return fail("vocab must be a multiple of 4");
+    if (c.max_batch < 1 || c.max_batch > 8) return fail("max_batch must be in [1, 8]");
+    if (c.max_seq < 1) return fail("max_seq must be positive");
+    if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 0.0)) return fail("bad eps or rope_theta");
+    Layout L{};
+    L.L = c.n_layers; L.H = c.hidden; L.nq = c.n_heads; L.nkv = c.n_kv_heads; L.d = c.head_dim;
+    L.F = c.ffn; L.V = c.vocab; L.group = group;
+    L.Q = c.n_heads * c.head_dim;
+    L.KVD = c.n_kv_heads * c.head_dim;
+    L.qkv_rows = L.Q + 2 * L.KVD;
+    L.tiles_per_group = (group + 2) * (c.head_dim / 4);
+    L.tile_h = (uint32_t)(4 * L.H * 2);
+    L.tile_o = (uint32_t)(4 * L.Q * 2);
+    L.tile_f = (uint32_t)(4 * (L.F / 4) * 2);
+    size_t off = 0;
+    L.off_embed = off;
+    off = align_up(off + (size_t)L.V * L.H * 2, 256);
+    L.off_layer0 = off;
+    size_t rel = 0;
+    L.rel_qkv = rel;
+    rel = align_up(rel + (size_t)L.qkv_rows * L.H * 2, 256);
+    L.rel_o = rel;
+    rel = align_up(rel + (size_t)L.H * L.Q * 2, 256);
+    L.rel_gu = rel;
+    rel = align_up(rel + (size_t)2 * L.F * L.H * 2, 256);
+    L.rel_down = rel;
+    rel = align_up(rel + (size_t)L.H * L.F * 2, 256);
+    L.layer_stride = rel;
+    off += (size_t)L.L * L.layer_stride;
+    L.off_norms = off;
+    off = align_up(off + (size_t)(2 * L.L + 1) * L.H * 2, 256);
+    L.total = off;
+    *out = L;
+    return true;
+}
+
+namespace {
+constexpr size_t kMaxSeg = 1 << 20;  // split long copies so the gather kernel spreads them
+
+void add(std::vector<Segment>& v, size_t dst, const void* src, size_t bytes) {
+    const uint8_t* s = static_cast<const uint8_t*>(src);
+    while (bytes > 0) {
+        const size_t n = bytes < kMaxSeg ? bytes : kMaxSeg;
+        v.push_back(Segment{dst, s, (uint32_t)n, 0});
+        dst += n;
+        s += n;
+        bytes -= n;
+    }
+}
+}  // namespace
+
+std::vector<Segment> pack_segments(const Layout& L, const mk_weights& w) {
+    std::vector<Segment> v;
+    const size_t row_h = (size_t)L.H * 2;
+    add(v, L.off_embed, w.embed, (size_t)L.V * row_h);
+    for (int l = 0; l < L.L; ++l) {
+        const size_t lb = L.off_layer0 + (size_t)l * L.layer_stride;
+        // QKV, grouped by KV head; RoPE pairs kept inside one tile
+        size_t dst = lb + L.rel_qkv;
+        const uint8_t* wq = static_cast<const uint8_t*>(w.wq[l]);
+        const uint8_t* wk = static_cast<const uint8_t*>(w.wk[l]);
+        const uint8_t* wv = static_cast<const uint8_t*>(w.wv[l]);
+        for (int g = 0; g < L.nkv; ++g) {
+            for (int hs = 0; hs < L.group + 2; ++hs) {
+                const uint8_t* head;
+                if (hs < L.group) head = wq + (size_t)(g * L.group + hs) * L.d * row_h;
+                else if (hs == L.group) head = wk + (size_t)g * L.d * row_h;
+                else head = wv + (size_t)g * L.d * row_h;
+                for (int j = 0; j < L.d / 4; ++j) {
+                    for (int r = 0; r < 4; ++r) {
+                        int row;
+                        if (hs <= L.group) {
+                            const int pair = r >> 1, second = r & 1;
+                            row = 2 * j + pair + (second ? L.d / 2 : 0);
+                        } else {
+                            row = 4 * j + r;
+                        }
+                        add(v, dst, head + (size_t)row * row_h, row_h);
+                        dst += row_h;
+                    }
+                }
+            }
+        }
+        add(v, lb + L.rel_o, w.wo[l], (size_t)L.H * L.Q * 2);
+        // gate/up interleaved in pairs of rows
+        dst = lb + L.rel_gu;
+        const uint8_t* wg = static_cast<const uint8_t*>(w.wgate[l]);
+        const uint8_t* wu = static_cast<const uint8_t*>(w.wup[l]);
+        for (int j = 0; j < L.F / 2; ++j) {
+            const uint8_t* rows[4] = {wg + (size_t)(2 * j) * row_h, wu + (size_t)(2 * j) * row_h,
+                                      wg + (size_t)(2 * j + 1) * row_h, wu + (size_t)(2 * j + 1) * row_h};
+            for (int r = 0; r < 4; ++r) {
+                add(v, dst, rows[r], row_h);
+                dst += row_h;
+            }
+        }
+        // down: [row block][chunk][4][ffn/4]
+        dst = lb + L.rel_down;
+        const uint8_t* wd = static_cast<const uint8_t*>(w.wdown[l]);
+        const size_t fc = (size_t)(L.F / 4) * 2;
+        for (int rb = 0; rb < L.H / 4; ++rb)
+            for (int c = 0; c < 4; ++c)
+                for (int r = 0; r < 4; ++r) {
+                    add(v, dst, wd + (size_t)(4 * rb + r) * L.F * 2 + c * fc, fc);
+                    dst += fc;
+                }
+    }
+    for (int l = 0; l < L.L; ++l) {
+        add(v, L.off_norms + (size_t)(2 * l) * row_h, w.attn_norm[l], row_h);
+        add(v, L.off_norms + (size_t)(2 * l + 1) * row_h, w.mlp_norm[l], row_h);
+    }
+    add(v, L.off_norms + (size_t)(2 * L.L) * row_h, w.final_norm, row_h);
+    return v;
+}
+
+bool weights_complete(const Layout& L, const mk_weights& w) {
+    if (!w.embed || !w.final_norm || !w.attn_norm || !w.wq || !w.wk || !w.wv || !w.wo ||
+        !w.mlp_norm || !w.wgate || !w.wup || !w.wdown)
+        return false;
+    for (int l = 0; l < L.L; ++l)
+        if (!w.attn_norm[l] || !w.wq[l] || !w.wk[l] || !w.wv[l] || !w.wo[l] || !w.mlp_norm[l] ||
+            !w.wgate[l] || !w.wup[l] || !w.wdown[l])
+            return false;
+    return true;
+}
+
+}  // namespace mk
+
+extern "C" size_t mk_packed_bytes(const mk_config* cfg) {
+    mk::Layout L;
+    if (!cfg || !mk::make_layout(*cfg, &L, nullptr)) return 0;
+    return L.total;
+}
+
+extern "C" mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights* w, void* dst,
+                                          size_t dst_bytes) {
+    mk::Layout L;
+    if (!cfg || !w || !dst) return MK_ERR_INVALID_ARG;
+    if (!mk::make_layout(*cfg, &L, nullptr)) return MK_ERR_UNSUPPORTED;
+    if (dst_bytes < L.total || !mk::weights_complete(L, *w)) return MK_ERR_INVALID_ARG;
+    memset(dst, 0, L.total);
+    for (const mk::Segment& s : mk::pack_segments(L, *w))
+        memcpy(static_cast<uint8_t*>(dst) + s.dst, s.src, s.bytes);
+    return MK_OK;
+}

@@ -1,0 +1,33 @@
+// Host-side packer and schedule builder interfaces (internal to libmk.so).
+#pragma once
+
+#include <vector>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+struct Segment {
+    size_t dst;          // byte offset in the packed buffer
+    const void* src;     // source bytes (device pointer for mk_create, host for the host packer)
+    uint32_t bytes;
+    uint32_t pad;
+};
+
+std::vector<Segment> pack_segments(const Layout& L, const mk_weights& w);
+bool weights_complete(const Layout& L, const mk_weights& w);
+
+struct Plan {
+    std::vector<mk_instr> instrs;   // SM lists, concatenated
+    std::vector<int32_t> sm_off;    // n_sm + 1 offsets into instrs
+    mk_schedule_info info;
+};
+
+// Ring stage size and keys-per-stage the kernel uses for this shape.
+uint32_t default_stage_bytes(const Layout& L);
+int stages_for(const Layout& L, uint32_t stage_bytes);
+
+mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
+                        const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);
+
+}  // namespace mk

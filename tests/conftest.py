@@ -23,3 +23,12 @@ def tiny_cfg():
 def tiny_weights(tiny_cfg):
     from persistent_megakernel_interpreter_b200.inputs import make_weights
     return make_weights(tiny_cfg, seed=0)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Compile libmk.so (nvcc, sm_100a) and the oracle if their sources changed."""
+    from persistent_megakernel_interpreter_b200.build import build_library
+    import oracle
+    build_library()
+    oracle.build()

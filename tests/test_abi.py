@@ -1,0 +1,55 @@
+"""The C ABI: the library builds, loads on a machine without a GPU, and exports
+every entry point that include/mk.h declares."""
+import ctypes
+import os
+import re
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mk.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mk_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("mk_create", "mk_build_schedule", "mk_decode_step", "mk_baseline_decode_step",
+                     "mk_decode_step_host", "mk_get_status", "mk_destroy", "mk_status_str"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    from persistent_megakernel_interpreter_b200 import _lib
+    lib = _lib.lib()
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_struct_sizes():
+    from persistent_megakernel_interpreter_b200 import _lib
+    lib = _lib.lib()
+    assert lib.mk_status_str(0) == b"ok"
+    assert lib.mk_status_str(5) == b"device wait timed out"
+    assert ctypes.sizeof(_lib.MkInstr) == 48
+    # null handles are rejected, not dereferenced
+    assert lib.mk_decode_step(None, None, None, None, None, None, None) == 1
+    assert lib.mk_build_schedule(None, 1, 1, None) == 1
+    lib.mk_destroy(None)
+
+
+def test_create_rejects_unsupported_shapes():
+    from persistent_megakernel_interpreter_b200 import _lib
+    from persistent_megakernel_interpreter_b200.config import TINY
+    import dataclasses
+    lib = _lib.lib()
+    bad = dataclasses.replace(TINY, head_dim=96)
+    c = _lib.make_config(bad, 1, 16)
+    assert lib.mk_packed_bytes(ctypes.byref(c)) == 0
+    w = _lib.MkWeights()
+    h = ctypes.c_void_p()
+    assert lib.mk_create(ctypes.byref(c), ctypes.byref(w), 0, ctypes.byref(h)) == 3
+    assert not h.value

@@ -1,0 +1,260 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle, plus
+the integer/protocol properties that must hold bit for bit.
+
+Tolerance (stated in the decode-step target): max |logit_gpu - logit_oracle|
+<= 1e-2 * max |logit_oracle| per step, and greedy argmax agreement. Integer work
+is exact: untouched KV slots, counters, token ids."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B, TINY
+from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+def _bits(t):
+    return oracle.bits(t.cpu()).copy()
+
+
+class Case:
+    """One model on the GPU and on the oracle, with a KV cache on each side."""
+
+    def __init__(self, cfg, batch, max_seq, past, seed=0, norm_jitter=0.0, weights=None):
+        from persistent_megakernel_interpreter_b200.model import Megakernel
+        self.cfg, self.batch, self.max_seq = cfg, batch, max_seq
+        w = weights or make_weights(cfg, seed=seed, norm_jitter=norm_jitter)
+        self.orc = oracle.Model(cfg, w)
+        self.k, self.v = make_kv_cache(cfg, batch, max_seq, past, seed=seed + 1)
+        dev = w.to("cuda")
+        self.mk = Megakernel(cfg, dev, max_batch=batch, max_seq=max_seq)
+        del dev
+        self.kd, self.vd = self.k.cuda(), self.v.cuda()
+        self.logits = torch.empty(batch, cfg.vocab, dtype=torch.float32, device="cuda")
+
+    def gpu_step(self, tokens, positions, baseline=False):
+        t = torch.as_tensor(np.asarray(tokens), dtype=torch.int32).cuda()
+        p = torch.as_tensor(np.asarray(positions), dtype=torch.int32).cuda()
+        fn = self.mk.baseline_decode_step if baseline else self.mk.decode_step
+        fn(t, p, self.kd, self.vd, self.logits)
+        torch.cuda.synchronize()
+        return self.logits.cpu().numpy().copy()
+
+    def oracle_step(self, tokens, positions, kc=None, vc=None):
+        kc = _bits(self.k) if kc is None else kc
+        vc = _bits(self.v) if vc is None else vc
+        return self.orc.decode_step(np.asarray(tokens), np.asarray(positions), kc, vc), kc, vc
+
+
+def assert_logits_close(gpu, ref):
+    for b in range(ref.shape[0]):
+        err = np.max(np.abs(gpu[b] - ref[b]))
+        assert err <= TOL * np.max(np.abs(ref[b])), (b, err, np.max(np.abs(ref[b])))
+        assert int(np.argmax(gpu[b])) == int(np.argmax(ref[b]))
+
+
+def assert_kv_ok(case, kc_ref, vc_ref, positions):
+    """New slots close to the oracle's; every other slot bit-identical to before."""
+    kg, vg = _bits(case.kd), _bits(case.vd)
+    k0, v0 = _bits(case.k), _bits(case.v)
+    for b, p in enumerate(positions):
+        mask = np.ones(case.max_seq, bool)
+        mask[p] = False
+        assert np.array_equal(kg[:, b][:, :, mask], k0[:, b][:, :, mask])
+        assert np.array_equal(vg[:, b][:, :, mask], v0[:, b][:, :, mask])
+        for got, ref in ((kg, kc_ref), (vg, vc_ref)):
+            g = oracle.bf16_to_f32(got[:, b, :, p]).astype(np.float64)
+            r = oracle.bf16_to_f32(ref[:, b, :, p]).astype(np.float64)
+            assert np.max(np.abs(g - r)) <= TOL * np.max(np.abs(r))
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    c = Case(TINY, batch=2, max_seq=160, past=[128, 57])
+    c.mk.build_schedule(batch=2, max_ctx=160)
+    yield c
+    c.mk.close()
+
+
+def test_tiny_step_matches_oracle(tiny):
+    toks = make_tokens(TINY, 2, seed=2).numpy()
+    pos = [128, 57]
+    gpu = tiny.gpu_step(toks, pos)
+    code, msg = tiny.mk.status()
+    assert code == 0, msg
+    ref, kc, vc = tiny.oracle_step(toks, pos)
+    assert_logits_close(gpu, ref)
+    assert_kv_ok(tiny, kc, vc, pos)
+
+
+def test_megakernel_equals_baseline_bit_for_bit(tiny):
+    toks = make_tokens(TINY, 2, seed=3).numpy()
+    pos = [100, 3]
+    a = tiny.gpu_step(toks, pos)
+    ka, va = _bits(tiny.kd), _bits(tiny.vd)
+    b = tiny.gpu_step(toks, pos, baseline=True)
+    assert tiny.mk.status()[0] == 0
+    assert np.array_equal(a, b)
+    assert np.array_equal(ka, _bits(tiny.kd)) and np.array_equal(va, _bits(tiny.vd))
+
+
+def test_repeated_steps_are_identical_and_counters_exact(tiny):
+    toks = make_tokens(TINY, 2, seed=4).numpy()
+    pos = [128, 57]
+    tiny.gpu_step(toks, pos)
+    base = tiny.mk.counters()
+    outs = [tiny.gpu_step(toks, pos) for _ in range(3)]
+    assert all(np.array_equal(outs[0], o) for o in outs[1:])
+    after = tiny.mk.counters()
+    n = len(after) - 2
+    epoch0, epoch1 = base[n], after[n]
+    assert epoch1 == epoch0 + 3 and after[n + 1] == 0
+    for c in range(n):  # every counter advanced by exactly 3 steps' worth of signals
+        per_step = base[c] // epoch0 if epoch0 else None
+        assert after[c] == per_step * epoch1
+
+
+def test_schedule_placement_does_not_change_results(tiny):
+    toks = make_tokens(TINY, 2, seed=5).numpy()
+    pos = [128, 57]
+    info = tiny.mk.schedule_info()
+    ref = tiny.gpu_step(toks, pos)
+    for opts in (dict(n_sm=37), dict(seed=99), dict(n_sm=5, tiles_lm=3, tiles_qkv=1),
+                 dict(rowblocks_down=3, tiles_gateup=8, tiles_o=1)):
+        tiny.mk.build_schedule(2, 160, part_keys=info.part_keys, **opts)
+        assert np.array_equal(tiny.gpu_step(toks, pos), ref), opts
+    tiny.mk.build_schedule(2, 160)
+
+
+def test_split_k_partitions_agree_with_oracle(tiny):
+    """Any partition size gives the oracle's logits (the merge is exact up to rounding)."""
+    toks = make_tokens(TINY, 2, seed=6).numpy()
+    pos = [150, 20]
+    ref, _, _ = tiny.oracle_step(toks, pos)
+    kps = tiny.mk.schedule_info().keys_per_stage
+    for pk in (kps, 2 * kps, 160 // kps * kps + kps):
+        tiny.mk.build_schedule(2, 160, part_keys=pk)
+        assert_logits_close(tiny.gpu_step(toks, pos), ref)
+    tiny.mk.build_schedule(2, 160)
+
+
+def test_host_buffer_entry_point(tiny):
+    toks = make_tokens(TINY, 2, seed=7).numpy()
+    pos = [128, 57]
+    dev = tiny.gpu_step(toks, pos)
+    th = torch.as_tensor(toks, dtype=torch.int32).pin_memory()
+    ph = torch.as_tensor(pos, dtype=torch.int32).pin_memory()
+    out = torch.empty(2, TINY.vocab, dtype=torch.float32).pin_memory()
+    tiny.mk.decode_step_host(th, ph, tiny.kd, tiny.vd, out)
+    assert np.array_equal(out.numpy(), dev)
+
+
+def test_bad_token_and_position_are_reported_and_write_nothing(tiny):
+    kb, vb = _bits(tiny.kd), _bits(tiny.vd)
+    for baseline in (False, True):
+        tiny.gpu_step([TINY.vocab, 1], [10, 10], baseline=baseline)
+        code, msg = tiny.mk.status()
+        assert code == 6, msg
+        tiny.gpu_step([1, 2], [10, 160], baseline=baseline)
+        code, msg = tiny.mk.status()
+        assert code == 7, msg
+    assert np.array_equal(kb, _bits(tiny.kd)) and np.array_equal(vb, _bits(tiny.vd))
+    # the handle keeps working
+    toks, pos = make_tokens(TINY, 2, seed=8).numpy(), [128, 57]
+    ref, _, _ = tiny.oracle_step(toks, pos)
+    assert_logits_close(tiny.gpu_step(toks, pos), ref)
+    assert tiny.mk.status()[0] == 0
+
+
+def test_wait_timeout_is_reported_without_hanging(tiny):
+    """A schedule missing one producer (host-side injection): the waits give up
+    after their budget, the step reports MK_ERR_TIMEOUT, and the next step runs."""
+    tiny.mk.build_schedule(2, 160, test_drop_item=3, wait_timeout_ms=200)
+    tiny.gpu_step([1, 2], [5, 6])
+    code, msg = tiny.mk.status()
+    assert code == 5, msg
+    counters = tiny.mk.counters()
+    assert all(c == 0 for c in counters)  # reset by the last CTA of the failed step
+    tiny.mk.build_schedule(2, 160)
+    toks, pos = make_tokens(TINY, 2, seed=9).numpy(), [128, 57]
+    ref, _, _ = tiny.oracle_step(toks, pos)
+    assert_logits_close(tiny.gpu_step(toks, pos), ref)
+    assert tiny.mk.status()[0] == 0
+
+
+def test_tiny_greedy_decode_teacher_forced():
+    """32-token prompt from an empty cache, then greedy decoding; the oracle is fed
+    the GPU's tokens (teacher forcing) and must agree on every step's argmax."""
+    c = Case(TINY, batch=1, max_seq=64, past=0, seed=11)
+    c.mk.build_schedule(1, 64)
+    kc, vc = _bits(c.k), _bits(c.v)
+    prompt = make_tokens(TINY, 32, seed=12).numpy()
+    tok = int(prompt[0])
+    agree = 0
+    for p in range(56):
+        gpu = c.gpu_step([tok], [p])
+        ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
+        assert np.max(np.abs(gpu[0] - ref[0])) <= TOL * np.max(np.abs(ref[0]))
+        agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
+        tok = int(prompt[p + 1]) if p + 1 < 32 else int(np.argmax(gpu[0]))
+    assert agree >= 0.99 * 56
+    assert c.mk.status()[0] == 0
+    c.mk.close()
+
+
+def test_tiny_with_non_unit_norm_weights():
+    c = Case(TINY, batch=1, max_seq=140, past=130, seed=21, norm_jitter=0.1)
+    c.mk.build_schedule(1, 140)
+    toks, pos = make_tokens(TINY, 1, seed=22).numpy(), [130]
+    ref, kc, vc = c.oracle_step(toks, pos)
+    assert_logits_close(c.gpu_step(toks, pos), ref)
+    assert_kv_ok(c, kc, vc, pos)
+    c.mk.close()
+
+
+def test_3b_shape_batch8_two_layers():
+    """The 3B-style shape (hidden 3072, head_dim 128, 3 query heads per KV head) at
+    batch 8 with ragged positions, cut to two layers so the oracle stays quick."""
+    cfg = dataclasses.replace(LLAMA_3B, n_layers=2, name="3b-shape-2l")
+    past = [2048, 1, 700, 2047, 0, 64, 1500, 333]
+    c = Case(cfg, batch=8, max_seq=2049, past=past, seed=31)
+    c.mk.build_schedule(8, 2049)
+    toks = make_tokens(cfg, 8, seed=32).numpy()
+    ref, kc, vc = c.oracle_step(toks, past)
+    gpu = c.gpu_step(toks, past)
+    assert c.mk.status()[0] == 0
+    assert_logits_close(gpu, ref)
+    assert_kv_ok(c, kc, vc, past)
+    assert np.array_equal(c.gpu_step(toks, past, baseline=True), gpu)
+    c.mk.close()
+
+
+@pytest.fixture(scope="module")
+def llama1b():
+    c = Case(LLAMA_1B, batch=1, max_seq=129, past=128, seed=0)
+    c.mk.build_schedule(1, 129)
+    yield c
+    c.mk.close()
+
+
+def test_llama1b_step_matches_oracle(llama1b):
+    """The benchmark's workload and launch configuration (148 SMs, ctx 128)."""
+    toks, pos = make_tokens(LLAMA_1B, 1, seed=2).numpy(), [128]
+    gpu = llama1b.gpu_step(toks, pos)
+    assert llama1b.mk.status()[0] == 0
+    ref, kc, vc = llama1b.oracle_step(toks, pos)
+    assert_logits_close(gpu, ref)
+    assert_kv_ok(llama1b, kc, vc, pos)
+
+
+def test_llama1b_megakernel_equals_baseline(llama1b):
+    toks, pos = make_tokens(LLAMA_1B, 1, seed=3).numpy(), [128]
+    a = llama1b.gpu_step(toks, pos)
+    b = llama1b.gpu_step(toks, pos, baseline=True)
+    assert np.array_equal(a, b)

@@ -1,0 +1,96 @@
+"""Weight packer: host packing equals the layout documented in include/mk.h,
+re-derived here independently by unpacking (bit-exact round trip)."""
+import numpy as np
+import torch
+
+from persistent_megakernel_interpreter_b200.config import TINY, ModelConfig
+from persistent_megakernel_interpreter_b200.inputs import make_weights
+from persistent_megakernel_interpreter_b200.model import pack_weights_host
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _align(x, a=256):
+    return (x + a - 1) // a * a
+
+
+def unpack(cfg: ModelConfig, buf: np.ndarray):
+    """Inverse of the documented layout, written from the header's description."""
+    H, d, nq, nkv, F, V, L = cfg.hidden, cfg.head_dim, cfg.n_heads, cfg.n_kv_heads, cfg.ffn, cfg.vocab, cfg.n_layers
+    grp = nq // nkv
+    Q = nq * d
+    b16 = buf.view(np.uint16)
+    off = 0
+    E = b16[off // 2: off // 2 + V * H].reshape(V, H)
+    off = _align(V * H * 2)
+    layers = []
+    for l in range(L):
+        out = {}
+        # QKV
+        qkv_rows = Q + 2 * nkv * d
+        blk = b16[off // 2: off // 2 + qkv_rows * H].reshape(qkv_rows, H)
+        wq = np.zeros((Q, H), np.uint16)
+        wk = np.zeros((nkv * d, H), np.uint16)
+        wv = np.zeros((nkv * d, H), np.uint16)
+        r = 0
+        for g in range(nkv):
+            for hs in range(grp + 2):
+                for j in range(d // 4):
+                    for k in range(4):
+                        if hs <= grp:
+                            row = 2 * j + (k >> 1) + (d // 2 if k & 1 else 0)
+                        else:
+                            row = 4 * j + k
+                        if hs < grp:
+                            wq[(g * grp + hs) * d + row] = blk[r]
+                        elif hs == grp:
+                            wk[g * d + row] = blk[r]
+                        else:
+                            wv[g * d + row] = blk[r]
+                        r += 1
+        out.update(wq=wq, wk=wk, wv=wv)
+        off = _align(off + qkv_rows * H * 2)
+        out["wo"] = b16[off // 2: off // 2 + H * Q].reshape(H, Q)
+        off = _align(off + H * Q * 2)
+        gu = b16[off // 2: off // 2 + 2 * F * H].reshape(F // 2, 4, H)
+        out["wgate"] = np.stack([gu[:, 0], gu[:, 2]], axis=1).reshape(F, H)
+        out["wup"] = np.stack([gu[:, 1], gu[:, 3]], axis=1).reshape(F, H)
+        off = _align(off + 2 * F * H * 2)
+        dn = b16[off // 2: off // 2 + H * F].reshape(H // 4, 4, 4, F // 4)  # [rb][c][r][k]
+        out["wdown"] = dn.transpose(0, 2, 1, 3).reshape(H, F)
+        off = _align(off + H * F * 2)
+        layers.append(out)
+    norms = b16[off // 2: off // 2 + (2 * L + 1) * H].reshape(2 * L + 1, H)
+    return E, layers, norms
+
+
+def test_pack_roundtrip_bit_exact():
+    cfg = TINY
+    w = make_weights(cfg, seed=7, norm_jitter=0.1)
+    buf = pack_weights_host(cfg, w).numpy()
+    E, layers, norms = unpack(cfg, buf)
+    assert np.array_equal(E, _u16(w.embed))
+    for l in range(cfg.n_layers):
+        for name in ("wq", "wk", "wv", "wo", "wgate", "wup", "wdown"):
+            assert np.array_equal(layers[l][name], _u16(getattr(w, name)[l])), (l, name)
+        assert np.array_equal(norms[2 * l], _u16(w.attn_norm[l]))
+        assert np.array_equal(norms[2 * l + 1], _u16(w.mlp_norm[l]))
+    assert np.array_equal(norms[2 * cfg.n_layers], _u16(w.final_norm))
+
+
+def test_pack_is_a_permutation_of_the_input_bytes():
+    """Every input element appears exactly once; the rest of the buffer is zero padding."""
+    cfg = TINY
+    w = make_weights(cfg, seed=8, norm_jitter=0.1)
+    buf = pack_weights_host(cfg, w).numpy().view(np.uint16)
+    parts = [_u16(w.embed).ravel(), _u16(w.final_norm)]
+    for l in range(cfg.n_layers):
+        for name in ("wq", "wk", "wv", "wo", "wgate", "wup", "wdown", "attn_norm", "mlp_norm"):
+            parts.append(_u16(getattr(w, name)[l]).ravel())
+    src = np.concatenate(parts)
+    assert buf.size >= src.size
+    counts = np.bincount(buf, minlength=65536)
+    counts[0] -= buf.size - src.size
+    assert np.array_equal(counts, np.bincount(src, minlength=65536))
