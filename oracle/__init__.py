@@ -4,8 +4,9 @@ TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
 baseline may import this package; the product path never does. Nothing here
 imports the CUDA library, and the CUDA library shares no code with it.
 
-``decode_step`` is the oracle proper (fp32 over bf16 weights, rounding at the
-fixed points R1..R6 documented in ``oracle.c``). ``brute`` holds an
+``decode_step`` is the oracle proper (fp32 over bf16 weights and the bf16 KV
+cache; activations fp32; the key and value written to the cache rounded to bf16,
+as documented in ``oracle.c``). ``brute`` holds an
 independent fp64 NumPy restatement used to pin the oracle.
 """
 from __future__ import annotations
@@ -81,42 +82,47 @@ def bf16_to_f32(b: np.ndarray) -> np.ndarray:
     return out
 
 
-def rmsnorm(x_bits: np.ndarray, w_bits: np.ndarray, eps: float) -> np.ndarray:
-    x_bits, w_bits = bits(x_bits), bits(w_bits)
-    out = np.empty_like(x_bits)
-    lib().orc_rmsnorm(_p(x_bits), _p(w_bits), x_bits.size, eps, _p(out))
+def _f32(x) -> np.ndarray:
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def rmsnorm(x: np.ndarray, w_bits: np.ndarray, eps: float) -> np.ndarray:
+    """x fp32 [n], w bf16 bits [n] -> fp32 [n]."""
+    x, w_bits = _f32(x), bits(w_bits)
+    out = np.empty_like(x)
+    lib().orc_rmsnorm(_p(x), _p(w_bits), x.size, eps, _p(out))
     return out
 
 
 def rope(v: np.ndarray, pos: int, theta: float) -> np.ndarray:
-    """Rotate one head vector (fp32, length d) in place semantics; returns a copy."""
+    """Rotate one head vector (fp32, length d); returns the rotated copy."""
     v = np.array(v, dtype=np.float32, copy=True)
     lib().orc_rope(_p(v), v.size, pos, theta)
     return v
 
 
-def matvec(W_bits: np.ndarray, x_bits: np.ndarray, threads: int = 1) -> np.ndarray:
-    W_bits, x_bits = bits(W_bits), bits(x_bits)
+def matvec(W_bits: np.ndarray, x: np.ndarray, threads: int = 1) -> np.ndarray:
+    """W bf16 bits [rows][cols], x fp32 [cols] -> fp32 [rows]."""
+    W_bits, x = bits(W_bits), _f32(x)
     rows, cols = W_bits.shape
     y = np.empty(rows, dtype=np.float32)
-    lib().orc_matvec(_p(W_bits), _p(x_bits), rows, cols, _p(y), threads)
+    lib().orc_matvec(_p(W_bits), _p(x), rows, cols, _p(y), threads)
     return y
 
 
-def attention(q_bits, K_bits, V_bits, n_keys: int) -> np.ndarray:
-    """q: [nq][d]; K, V: [nkv][seq][d] (bf16 bits). Returns bf16 bits [nq][d]."""
-    q_bits, K_bits, V_bits = bits(q_bits), bits(K_bits), bits(V_bits)
-    nq, d = q_bits.shape
+def attention(q: np.ndarray, K_bits, V_bits, n_keys: int) -> np.ndarray:
+    """q fp32 [nq][d]; K, V bf16 bits [nkv][seq][d]. Returns fp32 [nq][d]."""
+    q, K_bits, V_bits = _f32(q), bits(K_bits), bits(V_bits)
+    nq, d = q.shape
     nkv, seq, _ = K_bits.shape
-    out = np.empty((nq, d), dtype=np.uint16)
-    lib().orc_attention(_p(q_bits), _p(K_bits), _p(V_bits), nq, nkv, d, n_keys, seq, _p(out))
+    out = np.empty((nq, d), dtype=np.float32)
+    lib().orc_attention(_p(q), _p(K_bits), _p(V_bits), nq, nkv, d, n_keys, seq, _p(out))
     return out
 
 
 def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
-    g = np.ascontiguousarray(g, dtype=np.float32)
-    u = np.ascontiguousarray(u, dtype=np.float32)
-    out = np.empty(g.shape, dtype=np.uint16)
+    g, u = _f32(g), _f32(u)
+    out = np.empty(g.shape, dtype=np.float32)
     lib().orc_silu_mul(_p(g), _p(u), g.size, _p(out))
     return out
 

@@ -4,9 +4,10 @@ TEST INFRASTRUCTURE ONLY. Written separately from the C oracle (different
 language, different loop structure: whole-matrix products, per-head slices), so
 an indexing or sign slip in one is unlikely to be repeated in the other.
 
-``decode_step(..., rounding=True)`` rounds to bf16 at the same points R1..R6
-as the oracle, but from fp64 values and with torch's bf16 conversion; with
-``rounding=False`` it is the exact fp64 decoder. ``causal_forward`` runs a
+``decode_step(..., rounding=True)`` rounds the key and value written to the
+cache to bf16, like the oracle, but from fp64 values and with torch's bf16
+conversion; with ``rounding=False`` it is the exact fp64 decoder (the cache
+then holds unrounded values). ``causal_forward`` runs a
 whole prefix with no cache at all (every position attends to its own
 prefix), which is what an incremental decode must reproduce.
 """
@@ -74,11 +75,11 @@ class Brute:
         grp = nq // nkv
         x = self.E[token].copy()
         for l, P in enumerate(self.layers):
-            xn = _rb(_rms(x, P["an"], c.rms_eps), r)
+            xn = _rms(x, P["an"], c.rms_eps)
             q = (P["wq"] @ xn).reshape(nq, d)
             k = (P["wk"] @ xn).reshape(nkv, d)
             v = (P["wv"] @ xn).reshape(nkv, d)
-            q = _rb(_rope_heads(q, pos, c.rope_theta), r)
+            q = _rope_heads(q, pos, c.rope_theta)
             K[l][:, pos, :] = _rb(_rope_heads(k, pos, c.rope_theta), r)
             V[l][:, pos, :] = _rb(v, r)
             o = np.empty((nq, d))
@@ -87,11 +88,11 @@ class Brute:
                 s = Kg @ q[h] / np.sqrt(d)
                 p = np.exp(s - s.max())
                 o[h] = (p / p.sum()) @ Vg
-            x = _rb(x + P["wo"] @ _rb(o.reshape(-1), r), r)
-            xn = _rb(_rms(x, P["mn"], c.rms_eps), r)
-            h = _rb(_silu(P["wg"] @ xn) * (P["wu"] @ xn), r)
-            x = _rb(x + P["wd"] @ h, r)
-        y = _rb(_rms(x, self.fn, c.rms_eps), r)
+            x = x + P["wo"] @ o.reshape(-1)
+            xn = _rms(x, P["mn"], c.rms_eps)
+            h = _silu(P["wg"] @ xn) * (P["wu"] @ xn)
+            x = x + P["wd"] @ h
+        y = _rms(x, self.fn, c.rms_eps)
         return self.E @ y
 
     def causal_forward(self, tokens) -> np.ndarray:

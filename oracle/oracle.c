@@ -14,24 +14,26 @@
  * head. Fusion reorders work but does not approximate, so the oracle is the
  * plain definition of that forward, written out step by step:
  *
- *   x   = E[token]                                   (bf16 row)
+ *   x   = E[token]                                   (bf16 row, as fp32)
  *   per layer:
- *     xn  = bf16((x_i * r) * w_i),  r = 1/sqrt(mean(x^2) + eps)        [R1]
+ *     xn  = (x_i * r) * w_i,  r = 1/sqrt(mean(x^2) + eps)
  *     q,k,v = W_q xn, W_k xn, W_v xn                 (fp32 dot products)
- *     RoPE on q and k (rotate-half pairs (i, i+d/2)); round q,k,v      [R2]
- *     k, v stored in cache slot `pos`
- *     attn_h = bf16(softmax(q_h . K_g / sqrt(d)) V_g), g = h / group   [R3]
- *     x   = bf16(x + W_o attn)                                          [R4]
- *     xn  = rmsnorm(x) with the MLP norm                                [R1]
- *     h   = bf16(silu(W_g xn) * (W_u xn))                               [R5]
- *     x   = bf16(x + W_d h)                                             [R6]
- *   logits = E' . bf16(rmsnorm(x) with the final norm)   (fp32, unrounded) [R7]
+ *     RoPE on q and k (rotate-half pairs (i, i+d/2))
+ *     k, v rounded to bf16 and stored in cache slot `pos`            [KV]
+ *     attn_h = softmax(q_h . K_g / sqrt(d)) V_g,  g = h / group
+ *     x   = x + W_o attn
+ *     xn  = rmsnorm(x) with the MLP norm
+ *     h   = silu(W_g xn) * (W_u xn)
+ *     x   = x + W_d h
+ *   logits = E . (rmsnorm(x) with the final norm)
  *
- * Precision: fp32 arithmetic over the same bf16 weights, with rounding to bf16
- * (round to nearest, ties to even) only at R1..R6. Every sum runs in plain
- * index order. The points where the write-ups are silent (pairing of RoPE,
- * frequency form, rounding points, position of the new token) follow the
- * readings listed with the design notes of this repository.
+ * Precision: fp32 arithmetic over the bf16 weights and the bf16 KV cache.
+ * Activations stay fp32 between steps; the one rounding to bf16 (round to
+ * nearest, ties to even) is where the data format forces it: the key and value
+ * written to the bf16 cache [KV]. Every sum runs in plain index order. The
+ * points where the write-ups are silent (activation precision, RoPE pairing and
+ * frequency form, position of the new token) follow the readings listed with
+ * the design notes of this repository.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math, so
  * no reassociation and no fused multiply-add).
@@ -71,16 +73,13 @@ void orc_bf16_to_f32(const uint16_t* in, float* out, int64_t n) {
     for (int64_t i = 0; i < n; ++i) out[i] = bf2f(in[i]);
 }
 
-/* ---- RMSNorm [R1]: eps inside the root, weight applied after scaling ---- */
+/* ---- RMSNorm: eps inside the root, weight applied after scaling ---- */
 
-void orc_rmsnorm(const uint16_t* x, const uint16_t* w, int n, float eps, uint16_t* out) {
+void orc_rmsnorm(const float* x, const uint16_t* w, int n, float eps, float* out) {
     float ss = 0.0f;
-    for (int i = 0; i < n; ++i) {
-        float v = bf2f(x[i]);
-        ss += v * v;
-    }
+    for (int i = 0; i < n; ++i) ss += x[i] * x[i];
     float r = 1.0f / sqrtf(ss / (float)n + eps);
-    for (int i = 0; i < n; ++i) out[i] = f2bf((bf2f(x[i]) * r) * bf2f(w[i]));
+    for (int i = 0; i < n; ++i) out[i] = (x[i] * r) * bf2f(w[i]);
 }
 
 /* ---- RoPE, rotate-half pairing (i, i + d/2), plain theta^(-2i/d) ----
@@ -99,40 +98,38 @@ void orc_rope(float* v, int d, int pos, double theta) {
     }
 }
 
-/* ---- y = W x, W bf16 [rows][cols] row-major, x bf16, y fp32 ---- */
+/* ---- y = W x, W bf16 [rows][cols] row-major, x and y fp32 ---- */
 
-void orc_matvec(const uint16_t* W, const uint16_t* x, int rows, int cols, float* y, int threads) {
-    float* xf = (float*)malloc(sizeof(float) * (size_t)cols);
-    for (int k = 0; k < cols; ++k) xf[k] = bf2f(x[k]);
+void orc_matvec(const uint16_t* W, const float* x, int rows, int cols, float* y, int threads) {
 #pragma omp parallel for schedule(static) num_threads(threads > 0 ? threads : 1)
     for (int r = 0; r < rows; ++r) {
         const uint16_t* wr = W + (size_t)r * (size_t)cols;
         float acc = 0.0f;
-        for (int k = 0; k < cols; ++k) acc += bf2f(wr[k]) * xf[k];
+        for (int k = 0; k < cols; ++k) acc += bf2f(wr[k]) * x[k];
         y[r] = acc;
     }
-    free(xf);
 }
 
-/* ---- decode attention for one sequence and one layer [R3] ----
- * q: bf16 [nq][d]; K, V: bf16 [nkv][seq_stride][d], keys 0..n_keys-1 valid.
- * Query head h reads KV head h / (nq / nkv). Scale 1/sqrt(d) in fp32. */
+/* ---- decode attention for one sequence and one layer ----
+ * q: fp32 [nq][d]; K, V: bf16 [nkv][seq_stride][d], keys 0..n_keys-1 valid.
+ * Query head h reads KV head h / (nq / nkv). Scale 1/sqrt(d) in fp32.
+ * out: fp32 [nq][d]. */
 
-void orc_attention(const uint16_t* q, const uint16_t* K, const uint16_t* V, int nq, int nkv,
-                   int d, int n_keys, int seq_stride, uint16_t* out) {
+void orc_attention(const float* q, const uint16_t* K, const uint16_t* V, int nq, int nkv,
+                   int d, int n_keys, int seq_stride, float* out) {
     int group = nq / nkv;
     float scale = 1.0f / sqrtf((float)d);
     float* s = (float*)malloc(sizeof(float) * (size_t)(n_keys > 0 ? n_keys : 1));
-    float* o = (float*)malloc(sizeof(float) * (size_t)d);
     for (int h = 0; h < nq; ++h) {
         int g = h / group;
-        const uint16_t* qh = q + (size_t)h * d;
+        const float* qh = q + (size_t)h * d;
         const uint16_t* Kg = K + (size_t)g * seq_stride * d;
         const uint16_t* Vg = V + (size_t)g * seq_stride * d;
+        float* o = out + (size_t)h * d;
         float m = -INFINITY;
         for (int j = 0; j < n_keys; ++j) {
             float dot = 0.0f;
-            for (int i = 0; i < d; ++i) dot += bf2f(qh[i]) * bf2f(Kg[(size_t)j * d + i]);
+            for (int i = 0; i < d; ++i) dot += qh[i] * bf2f(Kg[(size_t)j * d + i]);
             s[j] = dot * scale;
             if (s[j] > m) m = s[j];
         }
@@ -144,25 +141,15 @@ void orc_attention(const uint16_t* q, const uint16_t* K, const uint16_t* V, int 
         for (int i = 0; i < d; ++i) o[i] = 0.0f;
         for (int j = 0; j < n_keys; ++j)
             for (int i = 0; i < d; ++i) o[i] += s[j] * bf2f(Vg[(size_t)j * d + i]);
-        for (int i = 0; i < d; ++i) out[(size_t)h * d + i] = f2bf(o[i] / l);
+        for (int i = 0; i < d; ++i) o[i] = o[i] / l;
     }
     free(s);
-    free(o);
 }
 
-/* ---- SiLU-gated product [R5]: h = bf16((g / (1 + exp(-g))) * u) ---- */
+/* ---- SiLU-gated product: h = (g / (1 + exp(-g))) * u ---- */
 
-void orc_silu_mul(const float* g, const float* u, int n, uint16_t* out) {
-    for (int i = 0; i < n; ++i) {
-        float silu = g[i] / (1.0f + expf(-g[i]));
-        out[i] = f2bf(silu * u[i]);
-    }
-}
-
-/* ---- residual add: x = bf16(x + y) [R4, R6] ---- */
-
-static void residual(uint16_t* x, const float* y, int n) {
-    for (int i = 0; i < n; ++i) x[i] = f2bf(bf2f(x[i]) + y[i]);
+void orc_silu_mul(const float* g, const float* u, int n, float* out) {
+    for (int i = 0; i < n; ++i) out[i] = (g[i] / (1.0f + expf(-g[i]))) * u[i];
 }
 
 /* ---- greedy choice: largest logit, lowest index on ties ---- */
@@ -209,54 +196,52 @@ int orc_decode_step(const orc_model* m, int batch, const int32_t* tokens,
         if (tokens[b] < 0 || tokens[b] >= V || positions[b] < 0 || positions[b] >= max_seq)
             return -1;
 
-    uint16_t* x = (uint16_t*)malloc(2 * (size_t)H);
-    uint16_t* xn = (uint16_t*)malloc(2 * (size_t)H);
-    float* qf = (float*)malloc(4 * (size_t)Q);
+    float* x = (float*)malloc(4 * (size_t)H);
+    float* xn = (float*)malloc(4 * (size_t)H);
+    float* q = (float*)malloc(4 * (size_t)Q);
     float* kf = (float*)malloc(4 * (size_t)KV);
     float* vf = (float*)malloc(4 * (size_t)KV);
-    uint16_t* qb = (uint16_t*)malloc(2 * (size_t)Q);
-    uint16_t* attn = (uint16_t*)malloc(2 * (size_t)Q);
+    float* attn = (float*)malloc(4 * (size_t)Q);
     float* y = (float*)malloc(4 * (size_t)(H > F ? H : F));
     float* g = (float*)malloc(4 * (size_t)F);
     float* u = (float*)malloc(4 * (size_t)F);
-    uint16_t* hb = (uint16_t*)malloc(2 * (size_t)F);
+    float* hb = (float*)malloc(4 * (size_t)F);
     const size_t slot_stride = (size_t)max_seq * d;             /* one kv head */
     const size_t seq_stride = (size_t)nkv * slot_stride;        /* one sequence */
     const size_t layer_stride = (size_t)batch * seq_stride;     /* one layer */
 
     for (int b = 0; b < batch; ++b) {
         const int pos = positions[b];
-        memcpy(x, m->embed + (size_t)tokens[b] * H, 2 * (size_t)H);
+        orc_bf16_to_f32(m->embed + (size_t)tokens[b] * H, x, H);
         for (int l = 0; l < m->n_layers; ++l) {
             uint16_t* Kl = k_cache + (size_t)l * layer_stride + (size_t)b * seq_stride;
             uint16_t* Vl = v_cache + (size_t)l * layer_stride + (size_t)b * seq_stride;
             /* attention block */
             orc_rmsnorm(x, m->attn_norm[l], H, m->rms_eps, xn);
-            orc_matvec(m->wq[l], xn, Q, H, qf, threads);
+            orc_matvec(m->wq[l], xn, Q, H, q, threads);
             orc_matvec(m->wk[l], xn, KV, H, kf, threads);
             orc_matvec(m->wv[l], xn, KV, H, vf, threads);
-            for (int h = 0; h < nq; ++h) orc_rope(qf + (size_t)h * d, d, pos, m->rope_theta);
+            for (int h = 0; h < nq; ++h) orc_rope(q + (size_t)h * d, d, pos, m->rope_theta);
             for (int h = 0; h < nkv; ++h) orc_rope(kf + (size_t)h * d, d, pos, m->rope_theta);
-            orc_round_bf16(qf, qb, Q);
-            for (int h = 0; h < nkv; ++h) {
+            for (int h = 0; h < nkv; ++h) {   /* [KV]: the only rounding to bf16 */
                 orc_round_bf16(kf + (size_t)h * d, Kl + (size_t)h * slot_stride + (size_t)pos * d, d);
                 orc_round_bf16(vf + (size_t)h * d, Vl + (size_t)h * slot_stride + (size_t)pos * d, d);
             }
-            orc_attention(qb, Kl, Vl, nq, nkv, d, pos + 1, max_seq, attn);
+            orc_attention(q, Kl, Vl, nq, nkv, d, pos + 1, max_seq, attn);
             orc_matvec(m->wo[l], attn, H, Q, y, threads);
-            residual(x, y, H);
+            for (int i = 0; i < H; ++i) x[i] += y[i];
             /* MLP block */
             orc_rmsnorm(x, m->mlp_norm[l], H, m->rms_eps, xn);
             orc_matvec(m->wgate[l], xn, F, H, g, threads);
             orc_matvec(m->wup[l], xn, F, H, u, threads);
             orc_silu_mul(g, u, F, hb);
             orc_matvec(m->wdown[l], hb, H, F, y, threads);
-            residual(x, y, H);
+            for (int i = 0; i < H; ++i) x[i] += y[i];
         }
         orc_rmsnorm(x, m->final_norm, H, m->rms_eps, xn);
         orc_matvec(m->lm_head ? m->lm_head : m->embed, xn, V, H, logits + (size_t)b * V, threads);
     }
-    free(x); free(xn); free(qf); free(kf); free(vf); free(qb); free(attn);
+    free(x); free(xn); free(q); free(kf); free(vf); free(attn);
     free(y); free(g); free(u); free(hb);
     return 0;
 }
