@@ -191,10 +191,10 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         off = mk::align_up(off + bytes, 256);
         return o;
     };
-    const size_t o_x = take((size_t)batch * L.H * 2);
-    const size_t o_q = take((size_t)batch * L.Q * 2);
-    const size_t o_attn = take((size_t)batch * L.Q * 2);
-    const size_t o_h = take((size_t)batch * L.F * 2);
+    const size_t o_x = take((size_t)batch * L.H * 4);
+    const size_t o_q = take((size_t)batch * L.Q * 4);
+    const size_t o_attn = take((size_t)batch * L.Q * 4);
+    const size_t o_h = take((size_t)batch * L.F * 4);
     const size_t o_ml = take((size_t)batch * L.nq * I.n_parts * 2 * sizeof(float));
     const size_t o_po = take((size_t)batch * L.nq * I.n_parts * L.d * sizeof(float));
     const size_t o_ctr = take((size_t)I.n_counters * mk::kCounterStride * sizeof(uint32_t));
@@ -228,10 +228,10 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     p.tile_h = L.tile_h; p.tile_o = L.tile_o; p.tile_f = L.tile_f;
     p.rope_cos = h->rope;
     p.rope_sin = h->rope + (size_t)c.max_seq * (L.d / 2);
-    p.x = reinterpret_cast<uint16_t*>(sb + o_x);
-    p.q = reinterpret_cast<uint16_t*>(sb + o_q);
-    p.attn = reinterpret_cast<uint16_t*>(sb + o_attn);
-    p.hbuf = reinterpret_cast<uint16_t*>(sb + o_h);
+    p.x = reinterpret_cast<float*>(sb + o_x);
+    p.q = reinterpret_cast<float*>(sb + o_q);
+    p.attn = reinterpret_cast<float*>(sb + o_attn);
+    p.hbuf = reinterpret_cast<float*>(sb + o_h);
     p.part_ml = reinterpret_cast<float*>(sb + o_ml);
     p.part_o = reinterpret_cast<float*>(sb + o_po);
     p.counters = h->counters;
@@ -244,6 +244,7 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     p.keys_per_stage = I.keys_per_stage;
     p.stage_bytes = (uint32_t)I.stage_bytes;
     p.n_stages = I.n_stages;
+    p.warp_scratch_floats = mk::warp_scratch_floats(L, (uint32_t)I.stage_bytes);
     p.n_counters = I.n_counters;
     p.timeout_ns = mk::kDefaultTimeoutNs;
     if (opts && opts->wait_timeout_ms > 0) p.timeout_ns = (uint64_t)opts->wait_timeout_ms * 1000000ull;

@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kBaseThreads) k_tiles(const __grid_constant__ 
     if (gw >= ntiles) return;
     const uint64_t pol = l2_evict_first_policy();
     const uint8_t* base = op_tiles(p, OP, l);
-    uint32_t x[KC][4];
+    XRegs<KC> x;
     if (p.B == 1) prep_input<OP, KC>(p, l, 0, x, lane);
     for (uint32_t t = gw; t < ntiles; t += nw) {
         for (int b = 0; b < p.B; ++b) {
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kBaseThreads) k_down(const __grid_constant__ P
     for (uint32_t rb = gw; rb < nrb; rb += nw) {
         for (int b = 0; b < p.B; ++b) {
             float tot[4];
-            uint32_t x[KF][4];
+            XRegs<KF> x;
             for (int c = 0; c < 4; ++c) {
                 load_vec<KF>(p.hbuf + (size_t)b * p.F + (size_t)c * (p.F / 4), x, lane);
                 float acc[4];
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kBaseThreads) k_down(const __grid_constant__ P
 #pragma unroll
                 for (int k = 0; k < 4; ++k) tot[k] = (c == 0) ? acc[k] : tot[k] + acc[k];
             }
-            residual_epilogue(p, p.x + (size_t)b * p.H, b, rb, tot, lane);
+            residual_epilogue(p, false, b, rb, tot, lane);
         }
     }
 }

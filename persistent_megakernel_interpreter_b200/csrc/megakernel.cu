@@ -33,6 +33,11 @@ struct Ring {
     uint8_t* base;
     uint64_t* full;
     uint64_t* empty;
+    // Fill number the loader last armed on each stage. Consumer warps take
+    // instructions out of order and may look for a fill up to several laps ahead;
+    // an mbarrier parity alone only tells phases one lap apart, so a consumer
+    // first waits until its stage holds its fill, then waits on the parity.
+    volatile uint32_t* armed;
     uint32_t stage_bytes;
     uint32_t S;
     __device__ __forceinline__ uint8_t* stage(uint32_t seq) const {
@@ -91,11 +96,12 @@ __device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uin
 
 // All lanes wait for ring fill `seq` to land; warp-uniform exit.
 __device__ bool wait_full(const Params& p, const Ring& r, uint32_t seq, int lane) {
-    uint64_t* bar = r.full + seq % r.S;
+    const uint32_t s = seq % r.S;
+    uint64_t* bar = r.full + s;
     const uint32_t par = (seq / r.S) & 1u;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
-        const bool done = mbar_try_wait(bar, par);
+        const bool done = r.armed[s] == seq && mbar_try_wait(bar, par);
         if (__all_sync(0xffffffffu, done)) return true;
         if ((it & 15u) == 15u) {
             int bad = 0;
@@ -103,7 +109,7 @@ __device__ bool wait_full(const Params& p, const Ring& r, uint32_t seq, int lane
                 if (t0 == 0) t0 = global_timer_ns();
                 if (aborted(p)) bad = 1;
                 else if (global_timer_ns() - t0 > p.timeout_ns) {
-                    record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffeu, 0, par, 2);
+                    record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffeu, r.armed[s], par, 2);
                     bad = 1;
                 }
             }
@@ -128,12 +134,12 @@ __device__ __forceinline__ uint32_t target_of(uint32_t epoch, uint32_t n) { retu
 
 template <int OP, int KC, int HD>
 __device__ bool exec_tiles(const Params& p, const Ring& ring, const mk_instr& in, int lane,
-                           uint64_t pol, uint32_t epoch) {
+                           uint64_t pol, uint32_t epoch, float* slot) {
     if (in.wait_ctr != MK_NO_COUNTER &&
         !wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane))
         return false;
     const int l = in.layer;
-    uint32_t x[KC][4];
+    XSmem<KC> x{reinterpret_cast<float4*>(slot), reinterpret_cast<float4*>(slot) + KC * 32};
     if (p.B == 1) prep_input<OP, KC>(p, l, 0, x, lane);
     for (uint32_t t = 0; t < in.count; ++t) {
         const uint32_t seq = in.seq + t;
@@ -158,9 +164,10 @@ __device__ bool exec_tiles(const Params& p, const Ring& ring, const mk_instr& in
 // more sequences it holds one. Running sums live in the warp's scratch.
 template <int KF>
 __device__ bool exec_down(const Params& p, const Ring& ring, const mk_instr& in, int lane,
-                          uint64_t pol, uint32_t epoch, float* tot) {
+                          uint64_t pol, uint32_t epoch, float* slot) {
     const int nslot = (p.B > 1) ? p.B : (int)in.count;
-    uint32_t x[KF][4];
+    XSmem<KF> x{reinterpret_cast<float4*>(slot), reinterpret_cast<float4*>(slot) + KF * 32};
+    float* tot = slot + KF * 256;  // running sums, [nslot][4]
     for (int c = 0; c < 4; ++c) {
         if (!wait_counter(p, in.wait_ctr + c, target_of(epoch, in.wait_n), in.seq, lane)) return false;
         if (p.B == 1) load_vec<KF>(p.hbuf + (size_t)c * (p.F / 4), x, lane);
@@ -181,7 +188,7 @@ __device__ bool exec_down(const Params& p, const Ring& ring, const mk_instr& in,
     __syncwarp();
     for (int i = 0; i < nslot; ++i) {
         const int b = (p.B > 1) ? i : 0, r = (p.B > 1) ? 0 : i;
-        if (lane < 4) residual_one(p, p.x + (size_t)b * p.H, b, (in.first + r) * 4 + lane, tot[i * 4 + lane]);
+        if (lane < 4) residual_one(p, false, b, (in.first + r) * 4 + lane, tot[i * 4 + lane]);
     }
     __syncwarp();
     signal(p, in.signal_ctr, lane);
@@ -259,6 +266,7 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
             {
                 uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
                 uint64_t* bar = ring.full + s;
+                ring.armed[s] = seq;  // published by the release of the arrive below
                 if (in.op == MK_OP_ATTN) {
                     const int pos = p.positions[in.batch];
                     const int ka = (int)in.first + (int)t * p.keys_per_stage;
@@ -336,12 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     ring.S = (uint32_t)p.n_stages;
     ring.full = reinterpret_cast<uint64_t*>(smem + (size_t)p.n_stages * p.stage_bytes);
     ring.empty = ring.full + p.n_stages;
-    float* attn_scratch = reinterpret_cast<float*>(ring.empty + p.n_stages);
+    ring.armed = reinterpret_cast<volatile uint32_t*>(ring.empty + p.n_stages);
+    // each consumer warp's scratch slot: its matvec input vector, its attention
+    // scores, or its down-projection running sums (one instruction at a time)
+    float* warp_scratch = reinterpret_cast<float*>(
+        reinterpret_cast<uintptr_t>(ring.armed + p.n_stages + 3) & ~uintptr_t(15));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
             mbar_init(ring.full + s, 1);
             mbar_init(ring.empty + s, 1);
+            ring.armed[s] = 0xffffffffu;
         }
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
@@ -370,17 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else {
             const uint64_t pol = l2_evict_first_policy();
             const uint32_t epoch = s_epoch;
-            float* sbuf = attn_scratch + (size_t)warp * kMaxGroup * p.keys_per_stage;
+            float* slot = warp_scratch + (size_t)warp * p.warp_scratch_floats;
             for (int i = i0 + warp; i < i1; i += kConsumerWarps) {
                 const mk_instr in = p.instrs[i];
                 bool ok;
                 switch (in.op) {
-                    case MK_OP_QKV: ok = exec_tiles<MK_OP_QKV, KH, HD>(p, ring, in, lane, pol, epoch); break;
-                    case MK_OP_ATTN: ok = exec_attn<HD>(p, ring, in, lane, epoch, sbuf); break;
-                    case MK_OP_OPROJ: ok = exec_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, lane, pol, epoch); break;
-                    case MK_OP_GATEUP: ok = exec_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, lane, pol, epoch); break;
-                    case MK_OP_DOWN: ok = exec_down<KF>(p, ring, in, lane, pol, epoch, sbuf); break;
-                    default: ok = exec_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, lane, pol, epoch); break;
+                    case MK_OP_QKV: ok = exec_tiles<MK_OP_QKV, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
+                    case MK_OP_ATTN: ok = exec_attn<HD>(p, ring, in, lane, epoch, slot); break;
+                    case MK_OP_OPROJ: ok = exec_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, lane, pol, epoch, slot); break;
+                    case MK_OP_GATEUP: ok = exec_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
+                    case MK_OP_DOWN: ok = exec_down<KF>(p, ring, in, lane, pol, epoch, slot); break;
+                    default: ok = exec_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
                 }
                 if (!ok) break;
             }
@@ -408,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ------------------------------------------------------------------ host-side launch
 
 size_t megakernel_smem_bytes(const Params& p) {
-    return (size_t)p.n_stages * p.stage_bytes + (size_t)p.n_stages * 16 +
-           (size_t)kConsumerWarps * kMaxGroup * p.keys_per_stage * sizeof(float);
+    return (size_t)p.n_stages * p.stage_bytes + (size_t)p.n_stages * 20 + 16 +
+           (size_t)kConsumerWarps * p.warp_scratch_floats * sizeof(float);
 }
 
 using KernelFn = void (*)(Params);

@@ -3,6 +3,9 @@
 // epilogues (RoPE + KV append, residual add, SiLU-gated product, logits) and
 // split-K decode attention with its merge.
 //
+// Precision: bf16 weights and KV cache, fp32 arithmetic and fp32 activations;
+// the only rounding to bf16 is the key/value written to the cache.
+//
 // Work split inside a warp (batch-1 matvec, the memory-bound case the
 // megakernel write-ups target): lane `ln` owns input elements
 // (kc*32 + ln)*8 .. +7 for kc = 0..KC-1 (KC = in_dim / 256), holds them as fp32
@@ -178,71 +181,112 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ------------------------------------------------------------------ vectors in registers
 
-// Load a bf16 vector of KC*256 elements into the lane layout described above,
-// kept as packed bf16 pairs (the vectors a matvec consumes are bf16 values).
+// Input vectors of a matvec live either in registers (XRegs, the baseline
+// kernels) or in the warp's slot of shared memory (XSmem, the megakernel, whose
+// register file is shared with a deep instruction loop). Both hold lane `ln`'s
+// elements (kc*32 + ln)*8 .. +7 and feed the same FMA sequence, so the two give
+// identical sums. In XSmem the 8 elements sit as two float4 halves in separate
+// arrays, so a warp-wide 16-byte load is conflict-free.
 template <int KC>
-__device__ __forceinline__ void load_vec(const uint16_t* src, uint32_t (&x)[KC][4], int lane) {
+struct XRegs {
+    float v[KC][8];
+    __device__ __forceinline__ void put(int kc, int lane, const float* e) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[kc][i] = e[i];
+    }
+    __device__ __forceinline__ void get(int kc, int lane, float* e) const {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = v[kc][i];
+    }
+};
+
+template <int KC>
+struct XSmem {
+    float4* a;  // [KC*32] elements 0..3 of each 8-element piece
+    float4* b;  // [KC*32] elements 4..7
+    __device__ __forceinline__ void put(int kc, int lane, const float* e) {
+        a[kc * 32 + lane] = make_float4(e[0], e[1], e[2], e[3]);
+        b[kc * 32 + lane] = make_float4(e[4], e[5], e[6], e[7]);
+    }
+    __device__ __forceinline__ void get(int kc, int lane, float* e) const {
+        const float4 u = a[kc * 32 + lane], w = b[kc * 32 + lane];
+        e[0] = u.x; e[1] = u.y; e[2] = u.z; e[3] = u.w;
+        e[4] = w.x; e[5] = w.y; e[6] = w.z; e[7] = w.w;
+    }
+};
+
+// Load an fp32 vector of KC*256 elements.
+template <int KC, class X>
+__device__ __forceinline__ void load_vec(const float* src, X& x, int lane) {
     const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-        const uint4 u = ld_cg_v4(s + kc * 32 + lane);
-        x[kc][0] = u.x; x[kc][1] = u.y; x[kc][2] = u.z; x[kc][3] = u.w;
+        const uint4 a = ld_cg_v4(s + (kc * 32 + lane) * 2);
+        const uint4 b = ld_cg_v4(s + (kc * 32 + lane) * 2 + 1);
+        const float e[8] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
+                            __uint_as_float(a.w), __uint_as_float(b.x), __uint_as_float(b.y),
+                            __uint_as_float(b.z), __uint_as_float(b.w)};
+        x.put(kc, lane, e);
     }
 }
 
-__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
-    return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+// The same from a bf16 vector (the embedding row).
+template <int KC, class X>
+__device__ __forceinline__ void load_vec_bf16(const uint16_t* src, X& x, int lane) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        float e[8];
+        unpack8(ld_cg_v4(s + kc * 32 + lane), e);
+        x.put(kc, lane, e);
+    }
 }
 
-// RMSNorm in place on the register vector: x <- bf16((x * r) * w) with
-// r = 1 / sqrt(mean(x^2) + eps), mean over the KC*256 elements.
-template <int KC>
-__device__ __forceinline__ void rmsnorm_regs(uint32_t (&x)[KC][4], const uint16_t* w, float eps,
-                                             int lane) {
+// RMSNorm in place: x <- (x * r) * w with r = 1 / sqrt(mean(x^2) + eps), mean
+// over the KC*256 elements.
+template <int KC, class X>
+__device__ __forceinline__ void rmsnorm_vec(X& x, const uint16_t* w, float eps, int lane) {
     float ss = 0.f;
 #pragma unroll
-    for (int kc = 0; kc < KC; ++kc)
+    for (int kc = 0; kc < KC; ++kc) {
+        float e[8];
+        x.get(kc, lane, e);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float a = bf_lo(x[kc][e]), b = bf_hi(x[kc][e]);
-            ss = fmaf(a, a, ss);
-            ss = fmaf(b, b, ss);
-        }
+        for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
+    }
     ss = warp_sum(ss);
     const float r = 1.0f / sqrtf(ss / (float)(KC * 256) + eps);
     const uint4* wp = reinterpret_cast<const uint4*>(w);
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-        const uint4 wv = ld_cg_v4(wp + kc * 32 + lane);
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+        float e[8], wv[8];
+        x.get(kc, lane, e);
+        unpack8(ld_cg_v4(wp + kc * 32 + lane), wv);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float lo = __fmul_rn(__fmul_rn(bf_lo(x[kc][e]), r), bf_lo(ww[e]));
-            const float hi = __fmul_rn(__fmul_rn(bf_hi(x[kc][e]), r), bf_hi(ww[e]));
-            x[kc][e] = pack_bf2(lo, hi);
-        }
+        for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(__fmul_rn(e[i], r), wv[i]);
+        x.put(kc, lane, e);
     }
 }
 
 // ------------------------------------------------------------------ the 4-row tile
 
-// acc += w.lo * x.lo; acc += w.hi * x.hi -- fp32 accumulation of exact bf16
-// products (the mixed-precision fma of sm_100), no unpacking.
-__device__ __forceinline__ void fma_bf2(float& acc, uint32_t w, uint32_t x) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-        "mov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
-        "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
-        : "+f"(acc)
-        : "r"(w), "r"(x));
+__device__ __forceinline__ void fma8(float& acc, uint4 w, const float* x) {
+    acc = fmaf(bf_lo(w.x), x[0], acc);
+    acc = fmaf(bf_hi(w.x), x[1], acc);
+    acc = fmaf(bf_lo(w.y), x[2], acc);
+    acc = fmaf(bf_hi(w.y), x[3], acc);
+    acc = fmaf(bf_lo(w.z), x[4], acc);
+    acc = fmaf(bf_hi(w.z), x[5], acc);
+    acc = fmaf(bf_lo(w.w), x[6], acc);
+    acc = fmaf(bf_hi(w.w), x[7], acc);
 }
 
 // acc[r] = W_tile[r] . x for the 4 rows of a [4][KC*256] bf16 tile. The tile is
 // in shared memory (SMEM) or read straight from global memory. Every lane
 // returns the same four totals.
-template <int KC, bool SMEM>
-__device__ __forceinline__ void dot4(const uint8_t* tile, const uint32_t (&x)[KC][4],
-                                     float (&acc)[4], int lane, uint64_t pol) {
+template <int KC, bool SMEM, class X>
+__device__ __forceinline__ void dot4(const uint8_t* tile, const X& x, float (&acc)[4], int lane,
+                                     uint64_t pol) {
     const uint4* t = reinterpret_cast<const uint4*>(tile);
 #pragma unroll
     for (int r = 0; r < 4; ++r) acc[r] = 0.f;
@@ -254,13 +298,10 @@ __device__ __forceinline__ void dot4(const uint8_t* tile, const uint32_t (&x)[KC
             const uint4* a = t + r * KC * 32 + kc * 32 + lane;
             w[r] = SMEM ? lds_v4(a) : ld_stream_v4(a, pol);
         }
+        float e[8];
+        x.get(kc, lane, e);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            fma_bf2(acc[r], w[r].x, x[kc][0]);
-            fma_bf2(acc[r], w[r].y, x[kc][1]);
-            fma_bf2(acc[r], w[r].z, x[kc][2]);
-            fma_bf2(acc[r], w[r].w, x[kc][3]);
-        }
+        for (int r = 0; r < 4; ++r) fma8(acc[r], w[r], e);
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) acc[r] = warp_sum(acc[r]);
@@ -272,21 +313,18 @@ __device__ __forceinline__ const uint16_t* norm_ptr(const Params& p, size_t off)
     return reinterpret_cast<const uint16_t*>(p.packed + off);
 }
 
-// Residual-stream input of layer l for sequence b: the embedding row at layer 0.
-__device__ __forceinline__ const uint16_t* x_in(const Params& p, int l, int b) {
-    if (l == 0) {
-        const int tok = p.tokens[b];
-        return reinterpret_cast<const uint16_t*>(p.packed) + (size_t)tok * p.H;
-    }
-    return p.x + (size_t)b * p.H;
+// The embedding row of sequence b's token (the residual stream before layer 0).
+__device__ __forceinline__ const uint16_t* embed_row(const Params& p, int b) {
+    return reinterpret_cast<const uint16_t*>(p.packed) + (size_t)p.tokens[b] * p.H;
 }
 
 __device__ __forceinline__ size_t kv_off(const Params& p, int l, int b, int g, int slot) {
     return ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.max_seq + slot) * p.d;
 }
 
-// QKV tile epilogue: RoPE on query/key pairs, round to bf16 [R2], store q or the
-// KV slot. `tile` is the tile index inside the layer's QKV block.
+// QKV tile epilogue: RoPE on query/key pairs; q stays fp32, the key and value are
+// rounded to bf16 into the cache slot. `tile` is the tile index inside the
+// layer's QKV block.
 template <int HD>
 __device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint32_t tile,
                                              const float (&acc)[4], int lane) {
@@ -314,43 +352,37 @@ __device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint
         }
         if (hs < p.group) {
             const int head = g * p.group + hs;
-            p.q[(size_t)b * p.Q + (size_t)head * HD + dim] = f2bf(out);
+            p.q[(size_t)b * p.Q + (size_t)head * HD + dim] = out;
         } else {
-            p.kc[kv_off(p, l, b, g, pos) + dim] = f2bf(out);
+            p.kc[kv_off(p, l, b, g, pos) + dim] = f2bf(out);   // the cache is bf16
         }
     } else {
         p.vc[kv_off(p, l, b, g, pos) + 4 * j + lane] = f2bf(pick4(acc, lane));
     }
 }
 
-__device__ __forceinline__ uint16_t ld_cg_u16(const uint16_t* p) {
-    uint16_t r;
-    asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(r) : "l"(p));
-    return r;
-}
-
-// x[b][row] = bf16(xin[row] + y) [R4, R6]. `xin` is the residual input (the
-// embedding row at layer 0, else x itself).
-__device__ __forceinline__ void residual_one(const Params& p, const uint16_t* xin, int b,
-                                             uint32_t row, float y) {
-    const float xv = bf2f(ld_cg_u16(xin + row));
-    p.x[(size_t)b * p.H + row] = f2bf(__fadd_rn(xv, y));
+// x[b][row] = xin[row] + y. The residual input is x itself, except for the
+// first O-projection, whose input is the embedding row (`from_embed`).
+__device__ __forceinline__ void residual_one(const Params& p, bool from_embed, int b, uint32_t row,
+                                             float y) {
+    const float xv = from_embed ? bf2f(embed_row(p, b)[row]) : ld_cg_f32(p.x + (size_t)b * p.H + row);
+    p.x[(size_t)b * p.H + row] = __fadd_rn(xv, y);
 }
 
 // The tile's 4 consecutive rows; lanes 0..3 write one each.
-__device__ __forceinline__ void residual_epilogue(const Params& p, const uint16_t* xin, int b,
+__device__ __forceinline__ void residual_epilogue(const Params& p, bool from_embed, int b,
                                                   uint32_t tile, const float (&acc)[4], int lane) {
     if (lane >= 4) return;
-    residual_one(p, xin, b, tile * 4 + lane, pick4(acc, lane));
+    residual_one(p, from_embed, b, tile * 4 + lane, pick4(acc, lane));
 }
 
-// gate/up tile rows {g 2j, u 2j, g 2j+1, u 2j+1}: h = bf16((g / (1 + e^-g)) * u) [R5].
+// gate/up tile rows {g 2j, u 2j, g 2j+1, u 2j+1}: h = (g / (1 + e^-g)) * u.
 __device__ __forceinline__ void gateup_epilogue(const Params& p, int b, uint32_t tile,
                                                 const float (&acc)[4], int lane) {
     if (lane >= 2) return;
     const float g = lane ? acc[2] : acc[0], u = lane ? acc[3] : acc[1];
     const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
-    p.hbuf[(size_t)b * p.F + 2 * tile + lane] = f2bf(__fmul_rn(silu, u));
+    p.hbuf[(size_t)b * p.F + 2 * tile + lane] = __fmul_rn(silu, u);
 }
 
 __device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t tile,
@@ -361,20 +393,21 @@ __device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t
 
 // ------------------------------------------------------------------ matvec op inputs/outputs
 
-// Input vector of a matvec op for sequence b, in registers.
-template <int OP, int KC>
-__device__ __forceinline__ void prep_input(const Params& p, int l, int b, uint32_t (&x)[KC][4], int lane) {
+// Input vector of a matvec op for sequence b.
+template <int OP, int KC, class X>
+__device__ __forceinline__ void prep_input(const Params& p, int l, int b, X& x, int lane) {
     if constexpr (OP == MK_OP_QKV) {
-        load_vec<KC>(x_in(p, l, b), x, lane);
-        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2), p.eps, lane);
+        if (l == 0) load_vec_bf16<KC>(embed_row(p, b), x, lane);
+        else load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
+        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2), p.eps, lane);
     } else if constexpr (OP == MK_OP_GATEUP) {
         load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
-        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, lane);
+        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, lane);
     } else if constexpr (OP == MK_OP_OPROJ) {
         load_vec<KC>(p.attn + (size_t)b * p.Q, x, lane);
     } else {  // LM head
         load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
-        rmsnorm_regs<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, lane);
+        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, lane);
     }
 }
 
@@ -383,7 +416,7 @@ __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uin
                                               const float (&acc)[4], int lane) {
     if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD>(p, l, b, tile, acc, lane);
     else if constexpr (OP == MK_OP_GATEUP) gateup_epilogue(p, b, tile, acc, lane);
-    else if constexpr (OP == MK_OP_OPROJ) residual_epilogue(p, x_in(p, l, b), b, tile, acc, lane);
+    else if constexpr (OP == MK_OP_OPROJ) residual_epilogue(p, l == 0, b, tile, acc, lane);
     else logits_epilogue(p, b, tile, acc, lane);
 }
 
@@ -415,8 +448,12 @@ __device__ __forceinline__ void attn_init(const Params& p, int b, int g, AttnSta
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) {
         if (h < p.group) {
-            const uint16_t* qh = p.q + (size_t)b * p.Q + (size_t)(g * p.group + h) * HD;
-            unpack8(ld_cg_v4(qh + dc * 8), st.q[h]);
+            const float* qh = p.q + (size_t)b * p.Q + (size_t)(g * p.group + h) * HD + dc * 8;
+            const uint4 a = ld_cg_v4(qh), c = ld_cg_v4(qh + 4);
+            st.q[h][0] = __uint_as_float(a.x); st.q[h][1] = __uint_as_float(a.y);
+            st.q[h][2] = __uint_as_float(a.z); st.q[h][3] = __uint_as_float(a.w);
+            st.q[h][4] = __uint_as_float(c.x); st.q[h][5] = __uint_as_float(c.y);
+            st.q[h][6] = __uint_as_float(c.z); st.q[h][7] = __uint_as_float(c.w);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) st.q[h][e] = 0.f;
@@ -546,7 +583,7 @@ __device__ __forceinline__ void attn_store_partial(const Params& p, const AttnSt
     }
 }
 
-// Merge the n_parts partials of (b, g) in partition order; attn = bf16(O / L) [R3].
+// Merge the n_parts partials of (b, g) in partition order; attn = O / L.
 template <int HD>
 __device__ __forceinline__ void attn_merge(const Params& p, int b, int g, int lane) {
     using S = AttnShape<HD>;
@@ -569,7 +606,7 @@ __device__ __forceinline__ void attn_merge(const Params& p, int b, int g, int la
         }
 #pragma unroll
         for (int d = 0; d < S::DPL; ++d)
-            p.attn[(size_t)b * p.Q + (size_t)head * HD + lane * S::DPL + d] = f2bf(__fdiv_rn(O[d], L));
+            p.attn[(size_t)b * p.Q + (size_t)head * HD + lane * S::DPL + d] = __fdiv_rn(O[d], L);
     }
 }
 

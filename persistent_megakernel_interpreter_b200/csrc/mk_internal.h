@@ -72,10 +72,10 @@ struct Params {
     uint16_t* vc;
     float* logits;
     // scratch
-    uint16_t* x;       // [B][H]   residual stream
-    uint16_t* q;       // [B][Q]
-    uint16_t* attn;    // [B][Q]
-    uint16_t* hbuf;    // [B][F]
+    float* x;          // [B][H]   residual stream (fp32)
+    float* q;          // [B][Q]
+    float* attn;       // [B][Q]
+    float* hbuf;       // [B][F]
     float* part_ml;    // [B][nq][P][2]  (m, l)
     float* part_o;     // [B][nq][P][d]
     uint32_t* counters;
@@ -87,6 +87,7 @@ struct Params {
     int part_keys, n_parts, keys_per_stage;
     uint32_t stage_bytes;
     int n_stages;
+    int warp_scratch_floats;   // per consumer warp (multiple of 4)
     int n_counters;
     uint64_t timeout_ns;
 };

@@ -26,6 +26,8 @@ struct Plan {
 // Ring stage size and keys-per-stage the kernel uses for this shape.
 uint32_t default_stage_bytes(const Layout& L);
 int stages_for(const Layout& L, uint32_t stage_bytes);
+// Floats of shared-memory scratch per consumer warp of the megakernel.
+int warp_scratch_floats(const Layout& L, uint32_t stage_bytes);
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);

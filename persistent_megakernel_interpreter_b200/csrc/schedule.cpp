@@ -31,14 +31,18 @@ uint32_t default_stage_bytes(const Layout& L) {
     return (uint32_t)align_up(s, 128);
 }
 
-static size_t attn_scratch_bytes(const Layout& L, uint32_t stage_bytes) {
+int warp_scratch_floats(const Layout& L, uint32_t stage_bytes) {
     const int kps = (int)(stage_bytes / (4u * (uint32_t)L.d));
-    return (size_t)kConsumerWarps * 4 * kps * sizeof(float);
+    int n = std::max(L.H, L.Q);                 // a matvec input vector
+    n = std::max(n, L.F / 4 + 32);              // a down chunk + the running sums
+    n = std::max(n, 4 * kps);                   // attention scores
+    return (n + 3) / 4 * 4;
 }
 
 int stages_for(const Layout& L, uint32_t stage_bytes) {
-    const size_t budget = kSmemBudget - 1024 - attn_scratch_bytes(L, stage_bytes);
-    return (int)(budget / (stage_bytes + 16));
+    const size_t scratch = (size_t)kConsumerWarps * warp_scratch_floats(L, stage_bytes) * sizeof(float);
+    const size_t budget = kSmemBudget - 1024 - 16 - scratch;
+    return (int)(budget / (stage_bytes + 20));
 }
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,

@@ -38,6 +38,12 @@ class Case:
         self.kd, self.vd = self.k.cuda(), self.v.cuda()
         self.logits = torch.empty(batch, cfg.vocab, dtype=torch.float32, device="cuda")
 
+    def reset_kv(self):
+        """Restore the GPU caches to the generated contents (earlier steps wrote slots)."""
+        self.kd.copy_(self.k)
+        self.vd.copy_(self.v)
+        torch.cuda.synchronize()
+
     def gpu_step(self, tokens, positions, baseline=False):
         t = torch.as_tensor(np.asarray(tokens), dtype=torch.int32).cuda()
         p = torch.as_tensor(np.asarray(positions), dtype=torch.int32).cuda()
@@ -75,11 +81,17 @@ def assert_kv_ok(case, kc_ref, vc_ref, positions):
 
 
 @pytest.fixture(scope="module")
-def tiny():
+def tiny_case():
     c = Case(TINY, batch=2, max_seq=160, past=[128, 57])
     c.mk.build_schedule(batch=2, max_ctx=160)
     yield c
     c.mk.close()
+
+
+@pytest.fixture
+def tiny(tiny_case):
+    tiny_case.reset_kv()
+    return tiny_case
 
 
 def test_tiny_step_matches_oracle(tiny):
@@ -140,6 +152,7 @@ def test_split_k_partitions_agree_with_oracle(tiny):
     kps = tiny.mk.schedule_info().keys_per_stage
     for pk in (kps, 2 * kps, 160 // kps * kps + kps):
         tiny.mk.build_schedule(2, 160, part_keys=pk)
+        tiny.reset_kv()
         assert_logits_close(tiny.gpu_step(toks, pos), ref)
     tiny.mk.build_schedule(2, 160)
 
@@ -166,6 +179,7 @@ def test_bad_token_and_position_are_reported_and_write_nothing(tiny):
         assert code == 7, msg
     assert np.array_equal(kb, _bits(tiny.kd)) and np.array_equal(vb, _bits(tiny.vd))
     # the handle keeps working
+    tiny.reset_kv()
     toks, pos = make_tokens(TINY, 2, seed=8).numpy(), [128, 57]
     ref, _, _ = tiny.oracle_step(toks, pos)
     assert_logits_close(tiny.gpu_step(toks, pos), ref)
@@ -182,6 +196,7 @@ def test_wait_timeout_is_reported_without_hanging(tiny):
     counters = tiny.mk.counters()
     assert all(c == 0 for c in counters)  # reset by the last CTA of the failed step
     tiny.mk.build_schedule(2, 160)
+    tiny.reset_kv()
     toks, pos = make_tokens(TINY, 2, seed=9).numpy(), [128, 57]
     ref, _, _ = tiny.oracle_step(toks, pos)
     assert_logits_close(tiny.gpu_step(toks, pos), ref)
@@ -236,11 +251,17 @@ def test_3b_shape_batch8_two_layers():
 
 
 @pytest.fixture(scope="module")
-def llama1b():
+def llama1b_case():
     c = Case(LLAMA_1B, batch=1, max_seq=129, past=128, seed=0)
     c.mk.build_schedule(1, 129)
     yield c
     c.mk.close()
+
+
+@pytest.fixture
+def llama1b(llama1b_case):
+    llama1b_case.reset_kv()
+    return llama1b_case
 
 
 def test_llama1b_step_matches_oracle(llama1b):

@@ -137,7 +137,7 @@ def test_balance_1b():
     mean = info.bytes_per_step / 148
     assert info.max_sm_bytes <= mean * 1.02
     assert info.min_sm_bytes >= mean * 0.98
-    assert info.stage_bytes == 16384 and info.n_stages >= 12
+    assert info.stage_bytes == 16384 and info.n_stages >= 9
 
 
 def test_seeded_placement_is_also_valid():
