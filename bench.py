@@ -151,16 +151,17 @@ def aggregate(elapsed_ms: float, units: float, dist, device=None):
     return float(t.item()), float(u.item())
 
 
-def workload_config(n_gpus: int):
-    return {"workload": "Llama-3.2-1B-shaped decoder, one decode step, batch 1, 128 cached "
-                        "positions (129 keys), random bf16 weights N(0,0.02), KV N(0,1)",
-            "layers": 16, "hidden": 2048, "heads": "32q/8kv x 64", "ffn": 8192, "vocab": 128256,
-            "global_batch": BATCH * n_gpus, "seq_len": PAST + 1,
+def workload_config(n_gpus: int, layers: int = 16, past: int = PAST):
+    name = "Llama-3.2-1B" if layers == 16 else f"Llama-3.2-1B-shaped ({layers} of 16 layers)"
+    return {"workload": f"{name} decoder, one decode step, batch 1, {past} cached positions "
+                        f"({past + 1} keys), random bf16 weights N(0,0.02), KV N(0,1)",
+            "layers": layers, "hidden": 2048, "heads": "32q/8kv x 64", "ffn": 8192, "vocab": 128256,
+            "global_batch": BATCH * n_gpus, "seq_len": past + 1,
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
             "l2": "no flush: the 2.47 GB of weights streamed per step exceed the 126 MB L2"}
 
 
-def time_oracle(cfg, w, k, v, budget_s: float):
+def time_oracle(cfg, w, k, v, budget_s: float, past: int):
     """The CPU oracle on this host's cores: full decode steps of the same workload until
     ``budget_s`` has passed (at least one). Returns (tokens/s, steps, threads, s/step)."""
     import numpy as np
@@ -173,7 +174,7 @@ def time_oracle(cfg, w, k, v, budget_s: float):
     n = 0
     t0 = time.perf_counter()
     while True:
-        om.decode_step(toks, np.array([PAST]), kc, vc, threads=threads)
+        om.decode_step(toks, np.array([past]), kc, vc, threads=threads)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
@@ -232,18 +233,20 @@ def run_mk(args):
     from persistent_megakernel_interpreter_b200.config import LLAMA_1B
     from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
     from persistent_megakernel_interpreter_b200.model import Megakernel
-    cfg = LLAMA_1B
+    import dataclasses
+    cfg = dataclasses.replace(LLAMA_1B, n_layers=args.layers) if args.layers != 16 else LLAMA_1B
+    past = args.past
     w = make_weights(cfg, seed=0)
-    k, v = make_kv_cache(cfg, BATCH, PAST + 1, PAST, seed=1)
-    mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=PAST + 1)
+    k, v = make_kv_cache(cfg, BATCH, past + 1, past, seed=1)
+    mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=past + 1)
     torch.cuda.empty_cache()
-    info = mk.build_schedule(BATCH, PAST + 1)
+    info = mk.build_schedule(BATCH, past + 1)
     kd, vd = k.to(dev), v.to(dev)
     tokens = make_tokens(cfg, BATCH, seed=2).to(dev)
-    positions = torch.full((BATCH,), PAST, dtype=torch.int32, device=dev)
+    positions = torch.full((BATCH,), past, dtype=torch.int32, device=dev)
     logits = torch.empty(BATCH, cfg.vocab, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
-    bytes_step = cfg.step_bytes(BATCH, PAST)
+    bytes_step = cfg.step_bytes(BATCH, past)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -281,7 +284,7 @@ def run_mk(args):
     # ---------------- end to end through the host-buffer entry point
     th = torch.zeros(BATCH, dtype=torch.int32).pin_memory()
     th.copy_(tokens.cpu())
-    ph = torch.full((BATCH,), PAST, dtype=torch.int32).pin_memory()
+    ph = torch.full((BATCH,), past, dtype=torch.int32).pin_memory()
     lh = torch.empty(BATCH, cfg.vocab, dtype=torch.float32).pin_memory()
     for _ in range(min(args.warmup, 10)):
         mk.decode_step_host(th, ph, kd, vd, lh, stream)
@@ -330,7 +333,7 @@ def run_mk(args):
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
-        val, n, threads, sps = time_oracle(cfg, w, k, v, args.cpu_budget)
+        val, n, threads, sps = time_oracle(cfg, w, k, v, args.cpu_budget, past)
         cpu = {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} full decode step(s) of this workload, {sps:.2f} s each"}
 
@@ -346,7 +349,7 @@ def run_mk(args):
             "ms_per_step": ms_per_step, "us_per_step": 1e3 * ms_per_step,
             "us_per_launch_median": 1e3 * statistics.median(launch_ms),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(world),
+            "data": "synthetic", "config": workload_config(world, cfg.n_layers, past),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
                          "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
@@ -380,6 +383,10 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=16,
+                    help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
+                         "small profiling captures of the same kernels)")
+    ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -149,13 +149,16 @@ const char* mk_status_str(mk_status s);
 
 /* ------------------------------------------------------------------ inspection */
 
-/* One instruction of the per-SM lists (48 bytes). The kinds: */
+/* One instruction of the per-SM lists (48 bytes). An SM's CTA runs its list in
+ * order; each instruction is one "job" for all of the CTA's compute warps (a
+ * down-projection is four jobs, one per MLP chunk; up to eight consecutive
+ * attention items form one job, one item per warp). The kinds: */
 enum {
     MK_OP_QKV = 1,     /* RMSNorm + QKV matvec + RoPE; writes q and the KV slot */
-    MK_OP_ATTN = 2,    /* split-K GQA attention partial; the last partition merges */
-    MK_OP_OPROJ = 3,   /* O-projection + residual */
+    MK_OP_ATTN = 2,    /* one split-K GQA attention partial (sequence, KV group, key range) */
+    MK_OP_OPROJ = 3,   /* merge of the attention partials + O-projection + residual */
     MK_OP_GATEUP = 4,  /* RMSNorm + gate/up matvec + SiLU-gated product */
-    MK_OP_DOWN = 5,    /* down-projection over 4 chunks + residual */
+    MK_OP_DOWN = 5,    /* down-projection over the 4 MLP chunks + residual */
     MK_OP_LMHEAD = 6   /* final RMSNorm + LM head */
 };
 #define MK_NO_COUNTER 0xffffffffu
@@ -170,11 +173,13 @@ typedef struct mk_instr {
     uint32_t nfill;      /* ring stage fills it consumes */
     uint32_t wait_ctr;   /* counter waited on (MK_NO_COUNTER: none); DOWN waits on the
                             4 consecutive chunk counters wait_ctr .. wait_ctr+3 */
-    uint32_t wait_n;     /* increments that counter receives per step */
-    uint32_t signal_ctr; /* counter incremented by one when done */
-    uint32_t aux_ctr;    /* ATTN: counter incremented by the merging (last) partition */
-    uint32_t aux_n;      /* ATTN: partitions per (sequence, group) */
-    uint32_t reserved;
+    uint32_t wait_n;     /* increments that counter receives per step (DOWN: chunk 0) */
+    uint32_t signal_ctr; /* counter incremented by one when the instruction (for ATTN:
+                            its job) is done */
+    uint32_t job_items;  /* ATTN: items in the job this entry opens (1..8), 0 for the
+                            job's later items; others: 1 */
+    uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
+                            high 16 bits of aux0) and 3 (aux1); else 0 */
 } mk_instr;
 
 typedef struct mk_schedule_info {

@@ -37,7 +37,7 @@ class MkInstr(ctypes.Structure):
     _fields_ = [("op", ctypes.c_uint16), ("layer", ctypes.c_uint16), ("batch", ctypes.c_uint16),
                 ("group", ctypes.c_uint16)] + [(n, ctypes.c_uint32) for n in (
                     "first", "count", "seq", "nfill", "wait_ctr", "wait_n", "signal_ctr",
-                    "aux_ctr", "aux_n", "reserved")]
+                    "job_items", "aux0", "aux1")]
 
 
 class MkScheduleInfo(ctypes.Structure):

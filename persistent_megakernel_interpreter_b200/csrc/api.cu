@@ -244,7 +244,13 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     p.keys_per_stage = I.keys_per_stage;
     p.stage_bytes = (uint32_t)I.stage_bytes;
     p.n_stages = I.n_stages;
-    p.warp_scratch_floats = mk::warp_scratch_floats(L, (uint32_t)I.stage_bytes);
+    {
+        const mk::SlotPlan sp = mk::slot_plan(L, batch, (uint32_t)I.stage_bytes);
+        p.xs_slots = sp.xs_slots;
+        p.xs_slot_bytes = sp.slot_bytes;
+        p.xs_vec_floats = sp.vec_floats;
+        p.attn_item_bytes = sp.item_bytes;
+    }
     p.n_counters = I.n_counters;
     p.timeout_ns = mk::kDefaultTimeoutNs;
     if (opts && opts->wait_timeout_ms > 0) p.timeout_ns = (uint64_t)opts->wait_timeout_ms * 1000000ull;

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kBaseThreads) k_attn_partial(const __grid_cons
     const int pos = p.positions[b];
     const int k0 = j * p.part_keys, k1 = min(k0 + p.part_keys, p.max_ctx);
     AttnState<HD> st;
-    attn_init<HD>(p, b, g, st, lane);
+    attn_init<HD, false>(p, p.q + (size_t)b * p.Q + (size_t)g * p.group * HD, st, lane);
     const uint16_t* Kpos = p.kc + kv_off(p, l, b, g, pos);
     const uint16_t* Vpos = p.vc + kv_off(p, l, b, g, pos);
     for (int ka = k0; ka < k1; ka += p.keys_per_stage) {
@@ -125,8 +125,10 @@ __global__ void __launch_bounds__(kBaseThreads) k_attn_merge(const __grid_consta
     if (step_failed(p)) return;
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kBaseWarps + (threadIdx.x >> 5);
-    if (gw >= p.B * p.nkv) return;
-    attn_merge<HD>(p, gw / p.nkv, gw % p.nkv, lane);
+    if (gw >= p.B * p.nq) return;
+    const int b = gw / p.nq, head = gw % p.nq;
+    float* out = p.attn + (size_t)b * p.Q;
+    attn_merge_head<HD>(p, b, head, lane, [&](int e, float x) { out[e] = x; });
 }
 
 // ------------------------------------------------------------------ host-side launch
@@ -146,7 +148,7 @@ static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
         k_tiles<MK_OP_QKV, KH, HD><<<blocks_for(nq), kBaseThreads, 0, st>>>(p, l, nq, p.tile_h);
         const uint32_t na = (uint32_t)(p.B * p.nkv * p.n_parts);
         k_attn_partial<HD><<<(na + kBaseWarps - 1) / kBaseWarps, kBaseThreads, attn_smem, st>>>(p, l);
-        const uint32_t nm = (uint32_t)(p.B * p.nkv);
+        const uint32_t nm = (uint32_t)(p.B * p.nq);
         k_attn_merge<HD><<<(nm + kBaseWarps - 1) / kBaseWarps, kBaseThreads, 0, st>>>(p);
         const uint32_t no = (uint32_t)p.H / 4;
         k_tiles<MK_OP_OPROJ, KO, HD><<<blocks_for(no), kBaseThreads, 0, st>>>(p, l, no, p.tile_o);

@@ -4,19 +4,25 @@
 // sections "Fusing Operations with an On-GPU Interpreter", "Efficient Shared
 // Memory Management", "Custom Synchronization Mechanism"; and the Cohere decode
 // megakernel, sections on the host task list, weight prefetch ahead of
-// activation waits, and static per-opcode pipelines instead of paging):
+// activation waits, and static warp-specialised pipelines instead of paging):
 //
-//  * The host writes one instruction list per SM. Every CTA walks its list.
+//  * The host writes one instruction list per SM; the CTA runs it in order, one
+//    job at a time for all compute warps.
 //  * Warp 8 (the loader) streams, in list order, every byte the instructions
-//    will read from HBM that is already final at launch -- weight tiles and the
-//    cached KV slots -- into a ring of shared-memory stages with bulk async
-//    copies (cp.async.bulk, completion counted on an mbarrier, L2 evict-first).
-//    It never waits on a dependency counter, so weights for the next
-//    instructions arrive while the consumers still wait for activations.
-//  * Warps 0..7 (consumers) take instructions round-robin. Each waits for its
-//    input counter (acquire load, bounded spin), reads its small activation
-//    vector from L2, consumes its ring stages, writes its outputs and
-//    increments its output counter (release).
+//    read from HBM that is final at launch -- weight tiles and the cached KV
+//    slots -- into a ring of shared-memory stages with bulk async copies
+//    (cp.async.bulk, completion counted on an mbarrier, L2 evict-first). It
+//    never waits on a dependency counter, so the next instructions' weights
+//    arrive while the step still waits for their activations.
+//  * Warp 9 (the activation warp) runs ahead of the compute warps: for each job
+//    it waits for the job's input counter (acquire load, bounded spin), loads
+//    the small activation input from L2 and prepares it in one of a few
+//    shared-memory slots -- RMSNorm for QKV, gate/up and the LM head, the merge
+//    of the split-K attention partials for the O-projection, an MLP chunk for
+//    the down-projection, q and the new key/value for attention.
+//  * Warps 0..7 (compute) split each job's tiles (tile t goes to warp t mod 8),
+//    write the outputs, and the last warp to finish increments the job's
+//    output counter (release).
 //  * Counters only grow: a step waits for (epoch + 1) * n increments, and the
 //    last CTA to finish advances the epoch, so no reset kernel is needed.
 //  * Every wait is bounded by a time budget; on expiry the step records
@@ -28,20 +34,31 @@
 
 namespace mk {
 
-
 struct Ring {
     uint8_t* base;
     uint64_t* full;
     uint64_t* empty;
-    // Fill number the loader last armed on each stage. Consumer warps take
-    // instructions out of order and may look for a fill up to several laps ahead;
-    // an mbarrier parity alone only tells phases one lap apart, so a consumer
-    // first waits until its stage holds its fill, then waits on the parity.
+    // Fill number the loader last armed on each stage. Compute warps take a
+    // job's tiles in any order and may look for a fill up to several laps
+    // ahead; an mbarrier parity alone only tells phases one lap apart, so a
+    // warp first waits until its stage holds its fill, then waits on the parity.
     volatile uint32_t* armed;
     uint32_t stage_bytes;
     uint32_t S;
     __device__ __forceinline__ uint8_t* stage(uint32_t seq) const {
         return base + (size_t)(seq % S) * stage_bytes;
+    }
+};
+
+struct Slots {
+    uint8_t* base;
+    uint64_t* full;    // the activation warp arrives when a job's input is ready
+    uint64_t* empty;   // each compute warp arrives when it is done with the job
+    uint32_t* done;    // compute warps finished with the job (the last one signals)
+    uint32_t bytes;
+    uint32_t NS;
+    __device__ __forceinline__ uint8_t* slot(uint32_t job) const {
+        return base + (size_t)(job % NS) * bytes;
     }
 };
 
@@ -64,6 +81,8 @@ __device__ void record_error(const Params& p, uint32_t code, uint32_t a, uint32_
 __device__ __forceinline__ bool aborted(const Params& p) {
     return ld_volatile_u32(&p.ctl->abort) != 0u;
 }
+
+__device__ __forceinline__ uint32_t target_of(uint32_t epoch, uint32_t n) { return (epoch + 1u) * n; }
 
 // Lane 0 spins until counter `ctr` reaches `target` (wrap-safe); the result is
 // broadcast to the warp. False on abort or timeout.
@@ -94,14 +113,13 @@ __device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uin
     return ok != 0;
 }
 
-// All lanes wait for ring fill `seq` to land; warp-uniform exit.
-__device__ bool wait_full(const Params& p, const Ring& r, uint32_t seq, int lane) {
-    const uint32_t s = seq % r.S;
-    uint64_t* bar = r.full + s;
-    const uint32_t par = (seq / r.S) & 1u;
+// All lanes wait for phase `parity` of an mbarrier; warp-uniform exit. With
+// `armed`, first wait until the ring stage holds fill `seq`.
+__device__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const volatile uint32_t* armed,
+                         uint32_t seq, uint32_t site, int lane) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
-        const bool done = r.armed[s] == seq && mbar_try_wait(bar, par);
+        const bool done = (armed == nullptr || *armed == seq) && mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, done)) return true;
         if ((it & 15u) == 15u) {
             int bad = 0;
@@ -109,7 +127,7 @@ __device__ bool wait_full(const Params& p, const Ring& r, uint32_t seq, int lane
                 if (t0 == 0) t0 = global_timer_ns();
                 if (aborted(p)) bad = 1;
                 else if (global_timer_ns() - t0 > p.timeout_ns) {
-                    record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffeu, r.armed[s], par, 2);
+                    record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffff0u + site, 0, parity, site);
                     bad = 1;
                 }
             }
@@ -118,121 +136,235 @@ __device__ bool wait_full(const Params& p, const Ring& r, uint32_t seq, int lane
     }
 }
 
-__device__ __forceinline__ void release_stage(const Ring& r, uint32_t seq, int lane) {
+__device__ __forceinline__ bool wait_fill(const Params& p, const Ring& r, uint32_t seq, int lane) {
+    const uint32_t s = seq % r.S;
+    return wait_bar(p, r.full + s, (seq / r.S) & 1u, r.armed + s, seq, 2, lane);
+}
+
+__device__ __forceinline__ void release_fill(const Ring& r, uint32_t seq, int lane) {
     __syncwarp();
     if (lane == 0) mbar_arrive(r.empty + seq % r.S);
 }
 
-__device__ __forceinline__ void signal(const Params& p, uint32_t ctr, int lane) {
-    __syncwarp();
-    if (lane == 0 && ctr != MK_NO_COUNTER) red_release_add(p.counters + (size_t)ctr * kCounterStride, 1u);
+// ------------------------------------------------------------------ activation warp
+
+// The down-projection's chunk-c target (chunks may have different job counts).
+__device__ __forceinline__ uint32_t down_chunk_target(const mk_instr& in, int c) {
+    return c == 0 ? in.wait_n : c == 1 ? (in.aux0 & 0xffffu) : c == 2 ? (in.aux0 >> 16) : in.aux1;
 }
 
-__device__ __forceinline__ uint32_t target_of(uint32_t epoch, uint32_t n) { return (epoch + 1u) * n; }
+// Element e of an XSmem<KC> vector stored at `v`.
+__device__ __forceinline__ void xs_store(float* v, int KC, int e, float x) {
+    const int g8 = e >> 3, i = e & 7;
+    float* arr = (i < 4) ? v : v + KC * 128;
+    arr[g8 * 4 + (i & 3)] = x;
+}
 
-// ------------------------------------------------------------------ instruction bodies
+template <int KH, int KO, int KF, int HD>
+__device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane,
+                         uint32_t epoch) {
+    const mk_instr& in = ins[0];
+    const int l = in.layer;
+    float* sv = reinterpret_cast<float*>(slot);
+    switch (in.op) {
+        case MK_OP_QKV:
+        case MK_OP_GATEUP:
+        case MK_OP_LMHEAD: {
+            if (in.wait_ctr != MK_NO_COUNTER &&
+                !wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane))
+                return false;
+            for (int b = 0; b < p.B; ++b) {
+                XSmem<KH> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
+                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KH * 32};
+                if (in.op == MK_OP_QKV) prep_input<MK_OP_QKV, KH>(p, l, b, x, lane);
+                else if (in.op == MK_OP_GATEUP) prep_input<MK_OP_GATEUP, KH>(p, l, b, x, lane);
+                else prep_input<MK_OP_LMHEAD, KH>(p, l, b, x, lane);
+            }
+            return true;
+        }
+        case MK_OP_OPROJ: {
+            if (!wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane)) return false;
+            for (int b = 0; b < p.B; ++b) {
+                float* v = sv + (size_t)b * p.xs_vec_floats;
+                for (int head = 0; head < p.nq; ++head)
+                    attn_merge_head<HD>(p, b, head, lane, [&](int e, float x) { xs_store(v, KO, e, x); });
+            }
+            return true;
+        }
+        case MK_OP_DOWN: {
+            if (!wait_counter(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq, lane))
+                return false;
+            for (int b = 0; b < p.B; ++b) {
+                XSmem<KF> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
+                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KF * 32};
+                load_vec<KF>(p.hbuf + (size_t)b * p.F + (size_t)c * (p.F / 4), x, lane);
+            }
+            return true;
+        }
+        default: {  // attention items: q of the group's heads and the new key/value
+            const int items = (int)in.job_items;
+            for (int it = 0; it < items; ++it) {
+                const mk_instr& a = ins[it];
+                if (!wait_counter(p, a.wait_ctr, target_of(epoch, a.wait_n), a.seq, lane)) return false;
+                uint8_t* region = slot + (size_t)it * p.attn_item_bytes;
+                const float* qsrc = p.q + (size_t)a.batch * p.Q + (size_t)a.group * p.group * HD;
+                float* qdst = reinterpret_cast<float*>(region);
+                for (int e = lane * 4; e < p.group * HD; e += 128)
+                    *reinterpret_cast<uint4*>(qdst + e) = ld_cg_v4(qsrc + e);
+                const int pos = p.positions[a.batch];
+                const size_t off = kv_off(p, l, a.batch, a.group, pos);
+                uint16_t* kv = reinterpret_cast<uint16_t*>(region + (size_t)p.group * HD * 4);
+                constexpr int kPieces = HD / 8;  // 16-byte pieces per row
+                if (lane < kPieces) {
+                    *reinterpret_cast<uint4*>(kv + lane * 8) = ld_cg_v4(p.kc + off + lane * 8);
+                } else if (lane < 2 * kPieces) {
+                    const int q = lane - kPieces;
+                    *reinterpret_cast<uint4*>(kv + HD + q * 8) = ld_cg_v4(p.vc + off + q * 8);
+                }
+            }
+            return true;
+        }
+    }
+}
+
+template <int KH, int KO, int KF, int HD>
+__device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1, int lane,
+                                uint32_t epoch) {
+    uint32_t j = 0;
+    for (int i = i0; i < i1;) {
+        const mk_instr* ins = p.instrs + i;
+        const uint32_t op = ins[0].op;
+        const int items = (op == MK_OP_ATTN) ? (int)ins[0].job_items : 1;
+        const int njobs = (op == MK_OP_DOWN) ? 4 : 1;
+        for (int c = 0; c < njobs; ++c, ++j) {
+            const uint32_t s = j % sl.NS, use = j / sl.NS;
+            if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
+            if (!prep_job<KH, KO, KF, HD>(p, ins, c, sl.slot(j), lane, epoch)) return;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sl.full + s);  // release: the slot's contents
+        }
+        i += items;
+    }
+}
+
+// ------------------------------------------------------------------ compute warps
 
 template <int OP, int KC, int HD>
-__device__ bool exec_tiles(const Params& p, const Ring& ring, const mk_instr& in, int lane,
-                           uint64_t pol, uint32_t epoch, float* slot) {
-    if (in.wait_ctr != MK_NO_COUNTER &&
-        !wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane))
-        return false;
-    const int l = in.layer;
-    XSmem<KC> x{reinterpret_cast<float4*>(slot), reinterpret_cast<float4*>(slot) + KC * 32};
-    if (p.B == 1) prep_input<OP, KC>(p, l, 0, x, lane);
-    for (uint32_t t = 0; t < in.count; ++t) {
+__device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
+                              const float* sv, int warp, int lane, uint64_t pol) {
+    for (uint32_t t = warp; t < in.count; t += kConsumerWarps) {
         const uint32_t seq = in.seq + t;
-        if (!wait_full(p, ring, seq, lane)) return false;
+        if (!wait_fill(p, ring, seq, lane)) return false;
         const uint8_t* tile = ring.stage(seq);
         for (int b = 0; b < p.B; ++b) {
-            if (p.B > 1) prep_input<OP, KC>(p, l, b, x, lane);
+            float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
+            XSmem<KC> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KC * 32};
             float acc[4];
             dot4<KC, true>(tile, x, acc, lane, pol);
-            tile_epilogue<OP, HD>(p, l, b, in.first + t, acc, lane);
+            tile_epilogue<OP, HD>(p, in.layer, b, in.first + t, acc, lane);
         }
-        release_stage(ring, seq, lane);
+        release_fill(ring, seq, lane);
     }
-    signal(p, in.signal_ctr, lane);
     return true;
 }
 
-// Down-projection: row block(s) over the 4 chunks of h, each chunk waited for
-// separately (the per-chunk MLP counters of the 1B megakernel); partial sums
-// added in chunk order, then the residual [R6]. With one sequence an
-// instruction may hold several row blocks (fills ordered chunk-major); with
-// more sequences it holds one. Running sums live in the warp's scratch.
+// Down-projection, chunk c: row block r (warp r mod 8) adds W_d[:, chunk c] . h_c to
+// its running sums, chunks in order 0..3; after chunk 3 the residual.
 template <int KF>
-__device__ bool exec_down(const Params& p, const Ring& ring, const mk_instr& in, int lane,
-                          uint64_t pol, uint32_t epoch, float* slot) {
-    const int nslot = (p.B > 1) ? p.B : (int)in.count;
-    XSmem<KF> x{reinterpret_cast<float4*>(slot), reinterpret_cast<float4*>(slot) + KF * 32};
-    float* tot = slot + KF * 256;  // running sums, [nslot][4]
-    for (int c = 0; c < 4; ++c) {
-        if (!wait_counter(p, in.wait_ctr + c, target_of(epoch, in.wait_n), in.seq, lane)) return false;
-        if (p.B == 1) load_vec<KF>(p.hbuf + (size_t)c * (p.F / 4), x, lane);
-        for (int i = 0; i < nslot; ++i) {
-            const int b = (p.B > 1) ? i : 0, r = (p.B > 1) ? 0 : i;
-            const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
-            if (!wait_full(p, ring, seq, lane)) return false;
-            if (p.B > 1) load_vec<KF>(p.hbuf + (size_t)b * p.F + (size_t)c * (p.F / 4), x, lane);
+__device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
+                             const float* sv, float* tot, int warp, int lane, uint64_t pol) {
+    for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
+        const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
+        if (!wait_fill(p, ring, seq, lane)) return false;
+        for (int b = 0; b < p.B; ++b) {
+            float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
+            XSmem<KF> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KF * 32};
             float acc[4];
             dot4<KF, true>(ring.stage(seq), x, acc, lane, pol);
             if (lane < 4) {
-                const float v = pick4(acc, lane);
-                tot[i * 4 + lane] = (c == 0) ? v : tot[i * 4 + lane] + v;
+                float* t = tot + ((size_t)r * p.B + b) * 4 + lane;
+                const float y = pick4(acc, lane);
+                *t = (c == 0) ? y : *t + y;
+                if (c == 3) residual_one(p, false, b, (in.first + r) * 4 + lane, *t);
             }
-            if (p.B == 1 || i == nslot - 1) release_stage(ring, seq, lane);
         }
+        release_fill(ring, seq, lane);
     }
-    __syncwarp();
-    for (int i = 0; i < nslot; ++i) {
-        const int b = (p.B > 1) ? i : 0, r = (p.B > 1) ? 0 : i;
-        if (lane < 4) residual_one(p, false, b, (in.first + r) * 4 + lane, tot[i * 4 + lane]);
-    }
-    __syncwarp();
-    signal(p, in.signal_ctr, lane);
     return true;
 }
 
 template <int HD>
-__device__ bool exec_attn(const Params& p, const Ring& ring, const mk_instr& in, int lane,
-                          uint32_t epoch, float* sbuf) {
-    if (!wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane)) return false;
-    const int l = in.layer, b = in.batch, g = in.group;
+__device__ bool compute_attn(const Params& p, const Ring& ring, const mk_instr& a,
+                             const uint8_t* region, float* scores, int lane) {
+    const int b = a.batch, g = a.group;
     const int pos = p.positions[b];
     const int kps = p.keys_per_stage;
+    const float* q = reinterpret_cast<const float*>(region);
+    const uint16_t* knew = reinterpret_cast<const uint16_t*>(region + (size_t)p.group * HD * 4);
+    const uint16_t* vnew = knew + HD;
     AttnState<HD> st;
-    attn_init<HD>(p, b, g, st, lane);
-    const uint16_t* Kpos = p.kc + kv_off(p, l, b, g, pos);
-    const uint16_t* Vpos = p.vc + kv_off(p, l, b, g, pos);
-    for (uint32_t ci = 0; ci < in.nfill; ++ci) {
-        const uint32_t seq = in.seq + ci;
-        if (!wait_full(p, ring, seq, lane)) return false;
-        const int ka = (int)in.first + (int)ci * kps;
-        int kend = min(ka + kps, (int)(in.first + in.count));
-        kend = min(kend, pos + 1);
+    attn_init<HD, true>(p, q, st, lane);
+    for (uint32_t ci = 0; ci < a.nfill; ++ci) {
+        const uint32_t seq = a.seq + ci;
+        if (!wait_fill(p, ring, seq, lane)) return false;
+        const int ka = (int)a.first + (int)ci * kps;
+        const int kend = min(min(ka + kps, (int)(a.first + a.count)), pos + 1);
         if (ka < kend) {
             const uint16_t* Ks = reinterpret_cast<const uint16_t*>(ring.stage(seq));
             const uint16_t* Vs = Ks + (size_t)kps * HD;
-            attn_chunk<HD, true>(p, st, Ks, Vs, Kpos, Vpos, ka, kend, pos, sbuf, kps, lane);
+            attn_chunk<HD, true>(p, st, Ks, Vs, knew, vnew, ka, kend, pos, scores, kps, lane);
         }
-        release_stage(ring, seq, lane);
+        release_fill(ring, seq, lane);
     }
-    attn_store_partial<HD>(p, st, b, g, (int)(in.first / (uint32_t)p.part_keys), lane);
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-        const uint32_t old = atom_acq_rel_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
-        last = (old == epoch * in.aux_n + in.aux_n - 1u);
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    __syncwarp();
-    if (last) {
-        attn_merge<HD>(p, b, g, lane);
-        signal(p, in.aux_ctr, lane);
-    }
+    attn_store_partial<HD>(p, st, b, g, (int)(a.first / (uint32_t)p.part_keys), lane);
     return true;
+}
+
+template <int KH, int KO, int KF, int HD>
+__device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
+                             float* tot, int i0, int i1, int warp, int lane) {
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t j = 0;
+    for (int i = i0; i < i1;) {
+        const mk_instr in = p.instrs[i];
+        const int items = (in.op == MK_OP_ATTN) ? (int)in.job_items : 1;
+        const int njobs = (in.op == MK_OP_DOWN) ? 4 : 1;
+        for (int c = 0; c < njobs; ++c, ++j) {
+            const uint32_t s = j % sl.NS;
+            if (!wait_bar(p, sl.full + s, (j / sl.NS) & 1u, nullptr, j, 4, lane)) return;
+            const float* sv = reinterpret_cast<const float*>(sl.slot(j));
+            bool ok;
+            switch (in.op) {
+                case MK_OP_QKV: ok = compute_tiles<MK_OP_QKV, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_OPROJ: ok = compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_GATEUP: ok = compute_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_LMHEAD: ok = compute_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, pol); break;
+                default:
+                    ok = warp >= items ||
+                         compute_attn<HD>(p, ring, p.instrs[i + warp],
+                                          sl.slot(j) + (size_t)warp * p.attn_item_bytes, scores, lane);
+                    break;
+            }
+            if (!ok) return;
+            // job done for this warp; the last of the 8 publishes the job's counter
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                const uint32_t old = atomicAdd(sl.done + s, 1u);
+                if (old == kConsumerWarps - 1) {
+                    sl.done[s] = 0;
+                    const bool last_chunk = in.op != MK_OP_DOWN || c == 3;
+                    if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
+                        __threadfence();
+                        red_release_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
+                    }
+                }
+                mbar_arrive(sl.empty + s);
+            }
+        }
+        i += items;
+    }
 }
 
 // ------------------------------------------------------------------ the loader warp
@@ -247,7 +379,7 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
             const uint32_t seq = in.seq + t;
             const uint32_t s = seq % ring.S, use = seq / ring.S;
             if (use > 0) {
-                // wait for the consumers to release the previous fill of this stage
+                // wait for the compute warps to release the previous fill of this stage
                 uint64_t t0 = 0;
                 bool ok = true;
                 for (uint32_t it = 0; !mbar_try_wait(ring.empty + s, (use - 1) & 1u); ++it) {
@@ -338,23 +470,33 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes,
+                                     p.keys_per_stage);
     Ring ring;
-    ring.base = smem;
+    ring.base = smem + m.ring;
+    ring.full = reinterpret_cast<uint64_t*>(smem + m.full);
+    ring.empty = reinterpret_cast<uint64_t*>(smem + m.empty);
+    ring.armed = reinterpret_cast<volatile uint32_t*>(smem + m.armed);
     ring.stage_bytes = p.stage_bytes;
     ring.S = (uint32_t)p.n_stages;
-    ring.full = reinterpret_cast<uint64_t*>(smem + (size_t)p.n_stages * p.stage_bytes);
-    ring.empty = ring.full + p.n_stages;
-    ring.armed = reinterpret_cast<volatile uint32_t*>(ring.empty + p.n_stages);
-    // each consumer warp's scratch slot: its matvec input vector, its attention
-    // scores, or its down-projection running sums (one instruction at a time)
-    float* warp_scratch = reinterpret_cast<float*>(
-        reinterpret_cast<uintptr_t>(ring.armed + p.n_stages + 3) & ~uintptr_t(15));
+    Slots sl;
+    sl.base = smem + m.xs;
+    sl.full = reinterpret_cast<uint64_t*>(smem + m.xs_full);
+    sl.empty = reinterpret_cast<uint64_t*>(smem + m.xs_empty);
+    sl.done = reinterpret_cast<uint32_t*>(smem + m.xs_done);
+    sl.bytes = p.xs_slot_bytes;
+    sl.NS = (uint32_t)p.xs_slots;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
             mbar_init(ring.full + s, 1);
             mbar_init(ring.empty + s, 1);
             ring.armed[s] = 0xffffffffu;
+        }
+        for (int s = 0; s < p.xs_slots; ++s) {
+            mbar_init(sl.full + s, 1);
+            mbar_init(sl.empty + s, kConsumerWarps);
+            sl.done[s] = 0;
         }
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
@@ -378,25 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 
     if (!s_skip) {
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
-        if (warp == kConsumerWarps) {
+        if (warp == kLoaderWarp) {
             if (lane == 0) loader(p, ring, i0, i1);
+        } else if (warp == kPrepWarp) {
+            activation_warp<KH, KO, KF, HD>(p, sl, i0, i1, lane, s_epoch);
         } else {
-            const uint64_t pol = l2_evict_first_policy();
-            const uint32_t epoch = s_epoch;
-            float* slot = warp_scratch + (size_t)warp * p.warp_scratch_floats;
-            for (int i = i0 + warp; i < i1; i += kConsumerWarps) {
-                const mk_instr in = p.instrs[i];
-                bool ok;
-                switch (in.op) {
-                    case MK_OP_QKV: ok = exec_tiles<MK_OP_QKV, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
-                    case MK_OP_ATTN: ok = exec_attn<HD>(p, ring, in, lane, epoch, slot); break;
-                    case MK_OP_OPROJ: ok = exec_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, lane, pol, epoch, slot); break;
-                    case MK_OP_GATEUP: ok = exec_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
-                    case MK_OP_DOWN: ok = exec_down<KF>(p, ring, in, lane, pol, epoch, slot); break;
-                    default: ok = exec_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, lane, pol, epoch, slot); break;
-                }
-                if (!ok) break;
-            }
+            float* scores = reinterpret_cast<float*>(smem + m.scores) +
+                            (size_t)warp * kMaxGroupHeads * p.keys_per_stage;
+            compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
+                                         i0, i1, warp, lane);
         }
     }
     __syncthreads();
@@ -421,8 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ------------------------------------------------------------------ host-side launch
 
 size_t megakernel_smem_bytes(const Params& p) {
-    return (size_t)p.n_stages * p.stage_bytes + (size_t)p.n_stages * 20 + 16 +
-           (size_t)kConsumerWarps * p.warp_scratch_floats * sizeof(float);
+    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, p.keys_per_stage).total;
 }
 
 using KernelFn = void (*)(Params);

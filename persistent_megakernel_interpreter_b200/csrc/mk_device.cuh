@@ -440,16 +440,25 @@ struct AttnState {
     float o[kMaxGroup][AttnShape<HD>::DPL];       // running unnormalised output
 };
 
-template <int HD>
-__device__ __forceinline__ void attn_init(const Params& p, int b, int g, AttnState<HD>& st,
+// q for the group's heads: 8 dims per lane from qh (fp32 [group][HD]), read from
+// shared memory (SMEM) or global memory.
+template <int HD, bool SMEM>
+__device__ __forceinline__ void attn_init(const Params& p, const float* qg, AttnState<HD>& st,
                                           int lane) {
     using S = AttnShape<HD>;
     const int dc = lane % S::LPK;
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) {
         if (h < p.group) {
-            const float* qh = p.q + (size_t)b * p.Q + (size_t)(g * p.group + h) * HD + dc * 8;
-            const uint4 a = ld_cg_v4(qh), c = ld_cg_v4(qh + 4);
+            const float* qh = qg + (size_t)h * HD + dc * 8;
+            uint4 a, c;
+            if (SMEM) {
+                a = lds_v4(qh);
+                c = lds_v4(qh + 4);
+            } else {
+                a = ld_cg_v4(qh);
+                c = ld_cg_v4(qh + 4);
+            }
             st.q[h][0] = __uint_as_float(a.x); st.q[h][1] = __uint_as_float(a.y);
             st.q[h][2] = __uint_as_float(a.z); st.q[h][3] = __uint_as_float(a.w);
             st.q[h][4] = __uint_as_float(c.x); st.q[h][5] = __uint_as_float(c.y);
@@ -466,9 +475,10 @@ __device__ __forceinline__ void attn_init(const Params& p, int b, int g, AttnSta
 }
 
 // One chunk of keys [ka, kend) (kend <= pos + 1, ka < kend). Rows of keys < pos
-// come from Kc/Vc (row 0 = key ka; shared memory when SMEM, else global); the
-// key at `pos`, written earlier in this step, is read from the global cache.
-// `s` is this warp's score scratch in shared memory, [kMaxGroup][ks] floats.
+// come from Kc/Vc (row 0 = key ka); the key at `pos`, written earlier in this
+// step, from Kpos/Vpos. All four are bf16 rows in shared memory when SMEM, else
+// in global memory. `s` is this warp's score scratch in shared memory,
+// [kMaxGroup][ks] floats.
 template <int HD, bool SMEM>
 __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, const uint16_t* Kc,
                                            const uint16_t* Vc, const uint16_t* Kpos,
@@ -486,11 +496,8 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
         for (int h = 0; h < kMaxGroup; ++h) part[h] = 0.f;
         if (j < n) {
             const int key = ka + j;
-            uint4 raw;
-            if (key < pos)
-                raw = SMEM ? lds_v4(Kc + (size_t)j * HD + dc * 8) : ld_cg_v4(Kc + (size_t)j * HD + dc * 8);
-            else
-                raw = ld_cg_v4(Kpos + dc * 8);
+            const uint16_t* kr = (key < pos ? Kc + (size_t)j * HD : Kpos) + dc * 8;
+            const uint4 raw = SMEM ? lds_v4(kr) : ld_cg_v4(kr);
             float kv[8];
             unpack8(raw, kv);
 #pragma unroll
@@ -538,17 +545,14 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
     for (int j = 0; j < n; ++j) {
         const int key = ka + j;
         float v[S::DPL];
-        const uint16_t* vr = (key < pos) ? Vc + (size_t)j * HD : Vpos;
-        const bool from_smem = SMEM && key < pos;
+        const uint16_t* vr = (key < pos ? Vc + (size_t)j * HD : Vpos) + lane * S::DPL;
         if constexpr (S::DPL == 2) {
-            const uint32_t w = from_smem ? *reinterpret_cast<const uint32_t*>(vr + lane * 2)
-                                         : ld_cg_u32(vr + lane * 2);
+            const uint32_t w = SMEM ? *reinterpret_cast<const uint32_t*>(vr) : ld_cg_u32(vr);
             v[0] = bf_lo(w);
             v[1] = bf_hi(w);
         } else {
             static_assert(S::DPL == 4, "head_dim 64 or 128");
-            const uint2 w = from_smem ? *reinterpret_cast<const uint2*>(vr + lane * 4)
-                                      : ld_cg_v2(vr + lane * 4);
+            const uint2 w = SMEM ? *reinterpret_cast<const uint2*>(vr) : ld_cg_v2(vr);
             v[0] = bf_lo(w.x);
             v[1] = bf_hi(w.x);
             v[2] = bf_lo(w.y);
@@ -583,31 +587,30 @@ __device__ __forceinline__ void attn_store_partial(const Params& p, const AttnSt
     }
 }
 
-// Merge the n_parts partials of (b, g) in partition order; attn = O / L.
-template <int HD>
-__device__ __forceinline__ void attn_merge(const Params& p, int b, int g, int lane) {
+// Merge the n_parts partials of one head of sequence b in partition order:
+// attn = (sum_j e^(m_j - M) o_j) / (sum_j e^(m_j - M) l_j), M = max_j m_j. The
+// lane's DPL dims go to out[lane*DPL + d] through `put`.
+template <int HD, class Put>
+__device__ __forceinline__ void attn_merge_head(const Params& p, int b, int head, int lane,
+                                                Put&& put) {
     using S = AttnShape<HD>;
-    for (int h = 0; h < p.group; ++h) {
-        const int head = g * p.group + h;
-        const size_t h0 = ((size_t)b * p.nq + head) * p.n_parts;
-        float M = -INFINITY;
-        for (int j = 0; j < p.n_parts; ++j) M = fmaxf(M, ld_cg_f32(p.part_ml + (h0 + j) * 2));
-        float L = 0.f, O[S::DPL];
+    const size_t h0 = ((size_t)b * p.nq + head) * p.n_parts;
+    float M = -INFINITY;
+    for (int j = 0; j < p.n_parts; ++j) M = fmaxf(M, ld_cg_f32(p.part_ml + (h0 + j) * 2));
+    float L = 0.f, O[S::DPL];
 #pragma unroll
-        for (int d = 0; d < S::DPL; ++d) O[d] = 0.f;
-        for (int j = 0; j < p.n_parts; ++j) {
-            const float mj = ld_cg_f32(p.part_ml + (h0 + j) * 2);
-            const float lj = ld_cg_f32(p.part_ml + (h0 + j) * 2 + 1);
-            const float w = expf(mj - M);   // empty partitions: m = -inf -> 0
-            L = fmaf(w, lj, L);
-#pragma unroll
-            for (int d = 0; d < S::DPL; ++d)
-                O[d] = fmaf(w, ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d), O[d]);
-        }
+    for (int d = 0; d < S::DPL; ++d) O[d] = 0.f;
+    for (int j = 0; j < p.n_parts; ++j) {
+        const float mj = ld_cg_f32(p.part_ml + (h0 + j) * 2);
+        const float lj = ld_cg_f32(p.part_ml + (h0 + j) * 2 + 1);
+        const float w = expf(mj - M);   // empty partitions: m = -inf -> 0
+        L = fmaf(w, lj, L);
 #pragma unroll
         for (int d = 0; d < S::DPL; ++d)
-            p.attn[(size_t)b * p.Q + (size_t)head * HD + lane * S::DPL + d] = __fdiv_rn(O[d], L);
+            O[d] = fmaf(w, ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d), O[d]);
     }
+#pragma unroll
+    for (int d = 0; d < S::DPL; ++d) put(head * HD + lane * S::DPL + d, __fdiv_rn(O[d], L));
 }
 
 }  // namespace mk

@@ -7,11 +7,23 @@
 
 #include "mk.h"
 
+#ifdef __CUDACC__
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+
 namespace mk {
 
-constexpr int kConsumerWarps = 8;                    // warps that execute instructions
-constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one producer (loader) warp
+constexpr int kConsumerWarps = 8;                    // compute warps
+constexpr int kLoaderWarp = kConsumerWarps;          // streams weights and cached KV
+constexpr int kPrepWarp = kConsumerWarps + 1;        // waits on counters, prepares inputs
+constexpr int kThreads = 32 * (kConsumerWarps + 2);
 constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
+constexpr int kMaxAttnItems = kConsumerWarps;        // attention items per job, one per warp
+constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
+constexpr int kMaxBatch = 8;
+constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
@@ -42,6 +54,35 @@ struct Layout {
     size_t mlp_norm(int l) const { return off_norms + (size_t)(2 * l + 1) * H * 2; }
     size_t final_norm() const { return off_norms + (size_t)(2 * L) * H * 2; }
 };
+
+// Shared-memory map of the megakernel (byte offsets from the dynamic base).
+struct SmemLayout {
+    uint32_t ring, full, empty, armed;        // weight / cached-KV ring of S stages
+    uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
+    uint32_t scores;                          // per compute warp: attention scores
+    uint32_t tot;                             // down-projection running sums
+    uint32_t total;
+};
+
+MK_HD inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
+
+MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes,
+                                    int keys_per_stage) {
+    SmemLayout m;
+    uint32_t o = 0;
+    m.ring = o;      o += (uint32_t)S * stage_bytes;
+    m.full = o;      o += 8u * S;
+    m.empty = o;     o += 8u * S;
+    m.armed = o;     o = align16(o + 4u * S);
+    m.xs = o;        o += (uint32_t)NS * slot_bytes;
+    m.xs_full = o;   o += 8u * NS;
+    m.xs_empty = o;  o += 8u * NS;
+    m.xs_done = o;   o = align16(o + 4u * NS);
+    m.scores = o;    o += 4u * kConsumerWarps * kMaxGroupHeads * (uint32_t)keys_per_stage;
+    m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
+    m.total = align16(o);
+    return m;
+}
 
 // Returns false if the shape is not one the kernels handle.
 bool make_layout(const mk_config& c, Layout* out, const char** why);
@@ -87,7 +128,10 @@ struct Params {
     int part_keys, n_parts, keys_per_stage;
     uint32_t stage_bytes;
     int n_stages;
-    int warp_scratch_floats;   // per consumer warp (multiple of 4)
+    int xs_slots;              // activation slots (1..3)
+    uint32_t xs_slot_bytes;
+    uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
+    uint32_t attn_item_bytes;  // one attention item's q and new key/value inside a slot
     int n_counters;
     uint64_t timeout_ns;
 };

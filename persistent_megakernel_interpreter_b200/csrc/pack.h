@@ -23,11 +23,20 @@ struct Plan {
     mk_schedule_info info;
 };
 
-// Ring stage size and keys-per-stage the kernel uses for this shape.
+// Ring stage size the kernel uses for this shape.
 uint32_t default_stage_bytes(const Layout& L);
-int stages_for(const Layout& L, uint32_t stage_bytes);
-// Floats of shared-memory scratch per consumer warp of the megakernel.
-int warp_scratch_floats(const Layout& L, uint32_t stage_bytes);
+
+// Shared-memory budget split: activation slots and ring stages.
+struct SlotPlan {
+    int keys_per_stage;
+    uint32_t vec_floats;   // one sequence's input vector inside a slot
+    uint32_t item_bytes;   // one attention item (q and the new key/value) inside a slot
+    uint32_t slot_bytes;
+    int xs_slots;
+    int stages;
+    uint32_t smem_bytes;
+};
+SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes);
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);

@@ -6,16 +6,18 @@
 // "one tile of one operator" as the scheduling unit, each task waiting only for
 // the producers it reads). Here:
 //
-//  * Work items are emitted in one global order that is a topological order of
-//    the step: per layer QKV (per KV group) -> attention partitions -> O-proj ->
-//    gate/up (per MLP chunk) -> down (per row block), then the LM head.
-//  * Each item goes to the SM whose running byte total is smallest, so every
-//    prefix of the step is balanced across SMs to within one item (the
-//    wave-quantisation holes of a kernel-per-op engine are filled by the next
-//    op's items).
-//  * Each SM's list keeps the global order, so every wait refers to work that
-//    comes earlier everywhere: with all CTAs resident the step cannot deadlock.
-//  * Counter targets are the number of items that signal each counter.
+//  * Each op is cut into units (4-row tiles, down-projection row blocks,
+//    attention items); every unit goes to the SM whose running byte total is
+//    smallest, so every prefix of the step is balanced across SMs to within one
+//    unit (the wave-quantisation holes of a kernel-per-op engine are filled by
+//    the next op's units). An SM's units of one op form one contiguous range,
+//    split only where a counter boundary (KV group, MLP chunk) falls.
+//  * Ops are appended in one global topological order: per layer QKV (per KV
+//    group) -> attention items -> O-proj -> gate/up (per MLP chunk) -> down,
+//    then the LM head. Each SM's list keeps that order, so every wait refers to
+//    work that comes earlier everywhere: with all CTAs resident the step cannot
+//    deadlock.
+//  * Counter targets are the number of jobs that signal each counter.
 #include <algorithm>
 #include <numeric>
 #include <queue>
@@ -31,30 +33,39 @@ uint32_t default_stage_bytes(const Layout& L) {
     return (uint32_t)align_up(s, 128);
 }
 
-int warp_scratch_floats(const Layout& L, uint32_t stage_bytes) {
-    const int kps = (int)(stage_bytes / (4u * (uint32_t)L.d));
-    int n = std::max(L.H, L.Q);                 // a matvec input vector
-    n = std::max(n, L.F / 4 + 32);              // a down chunk + the running sums
-    n = std::max(n, 4 * kps);                   // attention scores
-    return (n + 3) / 4 * 4;
-}
-
-int stages_for(const Layout& L, uint32_t stage_bytes) {
-    const size_t scratch = (size_t)kConsumerWarps * warp_scratch_floats(L, stage_bytes) * sizeof(float);
-    const size_t budget = kSmemBudget - 1024 - 16 - scratch;
-    return (int)(budget / (stage_bytes + 20));
+SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
+    SlotPlan sp{};
+    sp.keys_per_stage = (int)(stage_bytes / (4u * (uint32_t)L.d));
+    sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
+    sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
+    sp.slot_bytes = align16(std::max((uint32_t)batch * sp.vec_floats * 4u,
+                                     (uint32_t)kMaxAttnItems * sp.item_bytes));
+    for (int ns = 3; ns >= 1; --ns) {
+        int S = 0;
+        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, sp.keys_per_stage).total + 1024 <=
+               kSmemBudget)
+            ++S;
+        if (S >= (ns > 1 ? 6 : 2) || ns == 1) {
+            sp.xs_slots = ns;
+            sp.stages = S;
+            break;
+        }
+    }
+    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes,
+                                sp.keys_per_stage).total;
+    return sp;
 }
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out) {
     mk_schedule_opts o{};
     if (opts) o = *opts;
-    if (batch < 1 || batch > 8 || max_ctx < 1 || n_sm < 1) return MK_ERR_INVALID_ARG;
+    if (batch < 1 || batch > kMaxBatch || max_ctx < 1 || n_sm < 1) return MK_ERR_INVALID_ARG;
     if (stage_bytes == 0) stage_bytes = default_stage_bytes(L);
     if (stage_bytes % 128 || stage_bytes < default_stage_bytes(L)) return MK_ERR_INVALID_ARG;
-    const int kps = (int)(stage_bytes / (4u * (uint32_t)L.d));
-    const int S = stages_for(L, stage_bytes);
-    if (kps < 1 || S < 2) return MK_ERR_UNSUPPORTED;
+    const SlotPlan sp = slot_plan(L, batch, stage_bytes);
+    const int kps = sp.keys_per_stage;
+    if (kps < 1 || sp.stages < 2) return MK_ERR_UNSUPPORTED;
 
     // attention partitions
     const int fills_per_seq = (max_ctx + kps - 1) / kps;
@@ -63,64 +74,104 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         if (o.part_keys % kps) return MK_ERR_INVALID_ARG;
         part_keys = o.part_keys;
     } else {
-        const int want = std::max(1, (2 * n_sm + batch * L.nkv - 1) / (batch * L.nkv));
+        const int want = std::max(1, (n_sm + batch * L.nkv - 1) / (batch * L.nkv));
         part_keys = kps * ((fills_per_seq + want - 1) / want);
     }
     const int n_parts = (max_ctx + part_keys - 1) / part_keys;
-
-    const int tq = o.tiles_qkv > 0 ? o.tiles_qkv : 2;
-    const int to = o.tiles_o > 0 ? o.tiles_o : 2;
-    const int tg = o.tiles_gateup > 0 ? o.tiles_gateup : 4;
-    int rd = o.rowblocks_down > 0 ? o.rowblocks_down : 1;
-    const int tl = o.tiles_lm > 0 ? o.tiles_lm : 8;
-    if (batch > 1) rd = 1;
-    if (rd > 8) return MK_ERR_INVALID_ARG;
-    const int gu_tiles_chunk = L.F / 8;  // gate/up tiles (2 outputs each) per MLP chunk
-    if (gu_tiles_chunk % tg) return MK_ERR_INVALID_ARG;
+    const int down_cap = std::max(1, std::min(o.rowblocks_down > 0 ? o.rowblocks_down : kMaxDownRows,
+                                              kMaxDownRows));
 
     // counters
     int nc = 0;
-    std::vector<int> c_qkv(L.L), c_part(L.L), c_attn(L.L), c_o(L.L), c_h(L.L), c_down(L.L);
+    std::vector<int> c_qkv(L.L), c_part(L.L), c_o(L.L), c_h(L.L), c_down(L.L);
     for (int l = 0; l < L.L; ++l) {
         c_qkv[l] = nc; nc += L.nkv;
-        c_part[l] = nc; nc += batch * L.nkv;
-        c_attn[l] = nc++;
+        c_part[l] = nc++;
         c_o[l] = nc++;
         c_h[l] = nc; nc += 4;
         c_down[l] = nc++;
     }
     const int c_lm = nc++;
 
-    struct Unit {
-        mk_instr in;
-        uint64_t bytes;
+    // placement state
+    std::vector<std::vector<mk_instr>> lists(n_sm);
+    std::vector<uint64_t> load(n_sm, 0);
+    std::vector<uint32_t> rank(n_sm);
+    std::iota(rank.begin(), rank.end(), 0u);
+    if (o.seed) {
+        std::mt19937 rng(o.seed);
+        std::shuffle(rank.begin(), rank.end(), rng);
+    }
+    constexpr uint64_t kJobOverhead = 4096;  // byte-equivalent cost of one job's sync and prep
+    using Key = std::pair<uint64_t, uint32_t>;  // (load, rank)
+    std::vector<int> sm_of_rank(n_sm);
+    for (int s = 0; s < n_sm; ++s) sm_of_rank[rank[s]] = s;
+    // Units of one op, each costing `unit_cost`: how many each SM takes (the SM
+    // with the smallest running total takes the next unit).
+    auto share = [&](int units, uint64_t unit_cost) {
+        std::priority_queue<Key, std::vector<Key>, std::greater<Key>> pq;
+        for (int s = 0; s < n_sm; ++s) pq.push({load[s], rank[s]});
+        std::vector<int> cnt(n_sm, 0);
+        for (int u = 0; u < units; ++u) {
+            Key k = pq.top();
+            pq.pop();
+            const int s = sm_of_rank[k.second];
+            cnt[s]++;
+            const uint64_t add = unit_cost + (cnt[s] == 1 ? kJobOverhead : 0);
+            load[s] += add;
+            pq.push({k.first + add, k.second});
+        }
+        return cnt;
     };
-    std::vector<Unit> units;
     auto mk_in = [](uint16_t op, int l) {
         mk_instr in{};
         in.op = op;
         in.layer = (uint16_t)l;
         in.wait_ctr = MK_NO_COUNTER;
         in.signal_ctr = MK_NO_COUNTER;
-        in.aux_ctr = MK_NO_COUNTER;
+        in.job_items = 1;
         return in;
     };
-    const uint32_t kv_key_bytes = 2u * (uint32_t)L.d * 2u;  // K and V of one key
-    for (int l = 0; l < L.L; ++l) {
-        for (int g = 0; g < L.nkv; ++g)
-            for (int t = 0; t < L.tiles_per_group; t += tq) {
-                mk_instr in = mk_in(MK_OP_QKV, l);
-                in.group = (uint16_t)g;
-                in.first = (uint32_t)(g * L.tiles_per_group + t);
-                in.count = (uint32_t)std::min(tq, L.tiles_per_group - t);
-                in.nfill = in.count;
-                if (l > 0) in.wait_ctr = (uint32_t)c_down[l - 1];
-                in.signal_ctr = (uint32_t)(c_qkv[l] + g);
-                units.push_back({in, (uint64_t)in.count * L.tile_h});
+    // Contiguous ranges [start, start+cnt) in SM order, cut at multiples of `cut`
+    // (counter boundaries) and at `cap` units per instruction.
+    auto emit_ranges = [&](const std::vector<int>& cnt, int cut, int cap, auto&& make) {
+        int start = 0;
+        for (int s = 0; s < n_sm; ++s) {
+            int a = start, e = start + cnt[s];
+            while (a < e) {
+                int b = std::min(e, (a / cut + 1) * cut);
+                b = std::min(b, a + cap);
+                lists[s].push_back(make(a, b - a));
+                a = b;
             }
+            start = e;
+        }
+    };
+    std::vector<uint32_t> signals(nc, 0);
+    const uint32_t kv_key_bytes = 2u * (uint32_t)L.d * 2u;
+    const int gu_tiles = L.F / 2, gu_chunk = L.F / 8;
+    for (int l = 0; l < L.L; ++l) {
+        // QKV: tiles grouped by KV group
+        emit_ranges(share(L.nkv * L.tiles_per_group, L.tile_h), L.tiles_per_group, 1 << 30,
+                    [&](int a, int n) {
+                        mk_instr in = mk_in(MK_OP_QKV, l);
+                        in.group = (uint16_t)(a / L.tiles_per_group);
+                        in.first = (uint32_t)a;
+                        in.count = in.nfill = (uint32_t)n;
+                        if (l > 0) in.wait_ctr = (uint32_t)c_down[l - 1];
+                        in.signal_ctr = (uint32_t)(c_qkv[l] + in.group);
+                        signals[in.signal_ctr]++;
+                        return in;
+                    });
+        // attention items, each to the least-loaded SM
+        std::vector<int> items_on(n_sm, 0);
         for (int b = 0; b < batch; ++b)
             for (int g = 0; g < L.nkv; ++g)
                 for (int j = 0; j < n_parts; ++j) {
+                    int best = 0;
+                    for (int s = 1; s < n_sm; ++s)
+                        if (load[s] < load[best] || (load[s] == load[best] && rank[s] < rank[best]))
+                            best = s;
                     mk_instr in = mk_in(MK_OP_ATTN, l);
                     in.batch = (uint16_t)b;
                     in.group = (uint16_t)g;
@@ -128,108 +179,90 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     in.count = (uint32_t)std::min(part_keys, max_ctx - j * part_keys);
                     in.nfill = (in.count + kps - 1) / kps;
                     in.wait_ctr = (uint32_t)(c_qkv[l] + g);
-                    in.signal_ctr = (uint32_t)(c_part[l] + b * L.nkv + g);
-                    in.aux_ctr = (uint32_t)c_attn[l];
-                    in.aux_n = (uint32_t)n_parts;
-                    units.push_back({in, (uint64_t)in.count * kv_key_bytes});
+                    in.signal_ctr = (uint32_t)c_part[l];
+                    lists[best].push_back(in);
+                    load[best] += (uint64_t)in.count * kv_key_bytes + kJobOverhead;
+                    items_on[best]++;
                 }
-        for (int t = 0; t < L.H / 4; t += to) {
-            mk_instr in = mk_in(MK_OP_OPROJ, l);
-            in.first = (uint32_t)t;
-            in.count = (uint32_t)std::min(to, L.H / 4 - t);
-            in.nfill = in.count;
-            in.wait_ctr = (uint32_t)c_attn[l];
-            in.signal_ctr = (uint32_t)c_o[l];
-            units.push_back({in, (uint64_t)in.count * L.tile_o});
-        }
-        for (int c = 0; c < 4; ++c)
-            for (int t = 0; t < gu_tiles_chunk; t += tg) {
-                mk_instr in = mk_in(MK_OP_GATEUP, l);
-                in.group = (uint16_t)c;
-                in.first = (uint32_t)(c * gu_tiles_chunk + t);
-                in.count = (uint32_t)tg;
-                in.nfill = in.count;
-                in.wait_ctr = (uint32_t)c_o[l];
-                in.signal_ctr = (uint32_t)(c_h[l] + c);
-                units.push_back({in, (uint64_t)in.count * L.tile_h});
+        // group each SM's items of this layer into jobs of up to kMaxAttnItems
+        for (int s = 0; s < n_sm; ++s) {
+            const int n = items_on[s];
+            mk_instr* first = lists[s].data() + lists[s].size() - n;
+            for (int k = 0; k < n; k += kMaxAttnItems) {
+                const int run = std::min(kMaxAttnItems, n - k);
+                for (int r = 0; r < run; ++r) first[k + r].job_items = r == 0 ? (uint32_t)run : 0u;
+                signals[c_part[l]]++;
             }
-        for (int r = 0; r < L.H / 4; r += rd) {
-            mk_instr in = mk_in(MK_OP_DOWN, l);
-            in.first = (uint32_t)r;
-            in.count = (uint32_t)std::min(rd, L.H / 4 - r);
-            in.nfill = 4 * in.count;
-            in.wait_ctr = (uint32_t)c_h[l];
-            in.signal_ctr = (uint32_t)c_down[l];
-            units.push_back({in, (uint64_t)in.nfill * L.tile_f});
         }
+        emit_ranges(share(L.H / 4, L.tile_o), 1 << 30, 1 << 30, [&](int a, int n) {
+            mk_instr in = mk_in(MK_OP_OPROJ, l);
+            in.first = (uint32_t)a;
+            in.count = in.nfill = (uint32_t)n;
+            in.wait_ctr = (uint32_t)c_part[l];
+            in.signal_ctr = (uint32_t)c_o[l];
+            signals[in.signal_ctr]++;
+            return in;
+        });
+        emit_ranges(share(gu_tiles, L.tile_h), gu_chunk, 1 << 30, [&](int a, int n) {
+            mk_instr in = mk_in(MK_OP_GATEUP, l);
+            in.group = (uint16_t)(a / gu_chunk);
+            in.first = (uint32_t)a;
+            in.count = in.nfill = (uint32_t)n;
+            in.wait_ctr = (uint32_t)c_o[l];
+            in.signal_ctr = (uint32_t)(c_h[l] + in.group);
+            signals[in.signal_ctr]++;
+            return in;
+        });
+        emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, batch > 1 ? 1 : down_cap,
+                    [&](int a, int n) {
+                        mk_instr in = mk_in(MK_OP_DOWN, l);
+                        in.first = (uint32_t)a;
+                        in.count = (uint32_t)n;
+                        in.nfill = 4u * (uint32_t)n;
+                        in.wait_ctr = (uint32_t)c_h[l];
+                        in.signal_ctr = (uint32_t)c_down[l];
+                        signals[in.signal_ctr]++;
+                        return in;
+                    });
     }
-    for (int t = 0; t < L.V / 4; t += tl) {
+    emit_ranges(share(L.V / 4, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
         mk_instr in = mk_in(MK_OP_LMHEAD, L.L - 1);
-        in.first = (uint32_t)t;
-        in.count = (uint32_t)std::min(tl, L.V / 4 - t);
-        in.nfill = in.count;
+        in.first = (uint32_t)a;
+        in.count = in.nfill = (uint32_t)n;
         in.wait_ctr = (uint32_t)c_down[L.L - 1];
         in.signal_ctr = (uint32_t)c_lm;
-        units.push_back({in, (uint64_t)in.count * L.tile_h});
-    }
+        signals[in.signal_ctr]++;
+        return in;
+    });
 
-    // targets: how many items signal each counter per step
-    std::vector<uint32_t> signals(nc, 0);
-    for (const Unit& u : units)
-        if (u.in.signal_ctr != MK_NO_COUNTER) signals[u.in.signal_ctr]++;
-    for (int l = 0; l < L.L; ++l) signals[c_attn[l]] = (uint32_t)(batch * L.nkv);  // merges
-    for (Unit& u : units) {
-        if (u.in.wait_ctr == MK_NO_COUNTER) continue;
-        u.in.wait_n = signals[u.in.wait_ctr];
-        if (u.in.op == MK_OP_DOWN)
-            for (int c = 1; c < 4; ++c)
-                if (signals[u.in.wait_ctr + c] != u.in.wait_n) return MK_ERR_UNSUPPORTED;
-    }
-
-    if (o.test_drop_item > 0) {
-        if ((size_t)o.test_drop_item > units.size()) return MK_ERR_INVALID_ARG;
-        units.erase(units.begin() + (o.test_drop_item - 1));
-    }
-
-    // placement: smallest running total first
-    constexpr uint64_t kItemOverhead = 2048;  // byte-equivalent cost of one item's sync
-    std::vector<std::vector<mk_instr>> lists(n_sm);
-    std::vector<uint64_t> load(n_sm, 0);
-    std::vector<uint32_t> tiebreak(n_sm);
-    std::iota(tiebreak.begin(), tiebreak.end(), 0u);
-    if (o.seed) {
-        std::mt19937 rng(o.seed);
-        std::shuffle(tiebreak.begin(), tiebreak.end(), rng);
-    }
-    using Key = std::pair<uint64_t, uint32_t>;  // (load, tiebreak rank)
-    std::priority_queue<Key, std::vector<Key>, std::greater<Key>> pq;
-    std::vector<int> sm_of_rank(n_sm);
-    for (int s = 0; s < n_sm; ++s) {
-        sm_of_rank[tiebreak[s]] = s;
-        pq.push({0, tiebreak[s]});
-    }
-    uint64_t total = 0;
-    for (const Unit& u : units) {
-        Key k = pq.top();
-        pq.pop();
-        const int s = sm_of_rank[k.second];
-        lists[s].push_back(u.in);
-        load[s] += u.bytes;
-        total += u.bytes;
-        pq.push({k.first + u.bytes + kItemOverhead, k.second});
-    }
-
+    // wait targets; fill numbering; the failure-injection hook
     Plan P;
     P.sm_off.push_back(0);
+    uint64_t total = 0;
     for (int s = 0; s < n_sm; ++s) {
         uint32_t seq = 0;
         for (mk_instr in : lists[s]) {
+            if (in.wait_ctr != MK_NO_COUNTER) in.wait_n = signals[in.wait_ctr];
             in.seq = seq;
             seq += in.nfill;
             P.instrs.push_back(in);
         }
         P.sm_off.push_back((int32_t)P.instrs.size());
     }
+    for (mk_instr& in : P.instrs)
+        if (in.op == MK_OP_DOWN) {
+            // each MLP chunk may have a different number of gate/up jobs
+            in.wait_n = signals[in.wait_ctr];
+            in.aux0 = signals[in.wait_ctr + 1] | (signals[in.wait_ctr + 2] << 16);
+            in.aux1 = signals[in.wait_ctr + 3];
+        }
+    if (o.test_drop_item > 0) {
+        if ((size_t)o.test_drop_item > P.instrs.size()) return MK_ERR_INVALID_ARG;
+        // the job's work still runs, but its completion is never signalled
+        mk_instr& in = P.instrs[o.test_drop_item - 1];
+        in.signal_ctr = MK_NO_COUNTER;
+    }
+    for (int s = 0; s < n_sm; ++s) total += load[s];
     mk_schedule_info& I = P.info;
     I = mk_schedule_info{};
     I.n_sm = n_sm;
@@ -239,12 +272,20 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     I.n_parts = n_parts;
     I.keys_per_stage = kps;
     I.stage_bytes = (int32_t)stage_bytes;
-    I.n_stages = S;
+    I.n_stages = sp.stages;
     I.n_counters = nc;
     I.n_instr = (int32_t)P.instrs.size();
-    I.bytes_per_step = total;
+    uint64_t bytes = 0;
+    for (const mk_instr& in : P.instrs) {
+        if (in.op == MK_OP_ATTN) bytes += (uint64_t)in.count * kv_key_bytes;
+        else if (in.op == MK_OP_DOWN) bytes += (uint64_t)in.nfill * L.tile_f;
+        else if (in.op == MK_OP_OPROJ) bytes += (uint64_t)in.count * L.tile_o;
+        else bytes += (uint64_t)in.count * L.tile_h;
+    }
+    I.bytes_per_step = bytes;
     I.max_sm_bytes = *std::max_element(load.begin(), load.end());
     I.min_sm_bytes = *std::min_element(load.begin(), load.end());
+    (void)total;
     *out = std::move(P);
     return MK_OK;
 }

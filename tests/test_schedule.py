@@ -1,8 +1,10 @@
 """Schedule builder (host only): coverage of every tile exactly once, counter
 targets, per-SM byte balance, and a CPU simulation of the megakernel's
-synchronisation protocol (loader ring of S stages, 8 consumer warps taking
-instructions round-robin, counters with targets) that must run to completion --
-i.e. the schedule cannot deadlock -- and end with every counter at its target."""
+synchronisation protocol -- a loader streaming fills through a ring of S
+stages, an activation warp preparing each job's input in one of NS slots once
+its counters are met, and 8 compute warps splitting each job's fills -- that
+must run to completion (the schedule cannot deadlock) and leave every counter
+at its target."""
 import collections
 
 import pytest
@@ -11,66 +13,104 @@ from persistent_megakernel_interpreter_b200 import _lib
 from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B, TINY
 from persistent_megakernel_interpreter_b200.model import plan_schedule
 
-W = 8  # consumer warps per CTA
+W = 8  # compute warps per CTA
 NO = _lib.NO_COUNTER
 
 
-def simulate(instrs, offs, n_counters, S):
+def jobs_of(lst):
+    """The kernel's job sequence for one SM list: (first instr index, chunk, n items)."""
+    jobs, i = [], 0
+    while i < len(lst):
+        ins = lst[i]
+        items = ins.job_items if ins.op == _lib.OP_ATTN else 1
+        assert items >= 1
+        for c in range(4 if ins.op == _lib.OP_DOWN else 1):
+            jobs.append((i, c, items))
+        i += items
+    return jobs
+
+
+def job_waits(lst, job):
+    i, c, items = job
+    ins = lst[i]
+    if ins.op == _lib.OP_ATTN:
+        return [(lst[i + k].wait_ctr, lst[i + k].wait_n) for k in range(items)]
+    if ins.op == _lib.OP_DOWN:
+        t = [ins.wait_n, ins.aux0 & 0xFFFF, ins.aux0 >> 16, ins.aux1][c]
+        return [(ins.wait_ctr + c, t)]
+    return [] if ins.wait_ctr == NO else [(ins.wait_ctr, ins.wait_n)]
+
+
+def job_fills(lst, job, w):
+    """Fills compute warp w consumes for the job."""
+    i, c, items = job
+    ins = lst[i]
+    if ins.op == _lib.OP_ATTN:
+        if w >= items:
+            return []
+        a = lst[i + w]
+        return list(range(a.seq, a.seq + a.nfill))
+    if ins.op == _lib.OP_DOWN:
+        return [ins.seq + c * ins.count + r for r in range(w, ins.count, W)]
+    return [ins.seq + t for t in range(w, ins.count, W)]
+
+
+def simulate(instrs, offs, n_counters, S, NS=2):
     n_sm = len(offs) - 1
     ctr = [0] * n_counters
     lists = [instrs[offs[s]:offs[s + 1]] for s in range(n_sm)]
+    jobs = [jobs_of(L) for L in lists]
     total_fills = [sum(i.nfill for i in L) for L in lists]
     issued = [0] * n_sm
     released = [bytearray(t) for t in total_fills]
-    pos = [[w for w in range(W)] for _ in range(n_sm)]       # next instruction index per warp
-    fill = [[0] * W for _ in range(n_sm)]
-    done = 0
-    n_total = len(instrs)
+    prepared = [0] * n_sm                       # jobs whose input is ready
+    done = [[0] * len(j) for j in jobs]         # warps finished per job
+    wjob = [[0] * W for _ in range(n_sm)]       # job each warp is on
+    wpos = [[0] * W for _ in range(n_sm)]       # fills consumed in that job
     changed = True
-    rounds = 0
     while changed:
         changed = False
-        rounds += 1
         for s in range(n_sm):
-            L = lists[s]
+            L, J = lists[s], jobs[s]
             while issued[s] < total_fills[s] and (issued[s] < S or released[s][issued[s] - S]):
                 issued[s] += 1
                 changed = True
+            while prepared[s] < len(J):
+                j = prepared[s]
+                if j >= NS and done[s][j - NS] < W:
+                    break
+                if any(ctr[c] < t for c, t in job_waits(L, J[j])):
+                    break
+                prepared[s] += 1
+                changed = True
             for w in range(W):
-                while pos[s][w] < len(L):
-                    ins = L[pos[s][w]]
-                    f = fill[s][w]
-                    if ins.op == _lib.OP_DOWN:
-                        c = min(f, ins.nfill - 1) // ins.count
-                        need = (ins.wait_ctr + c, ins.wait_n)
-                    elif ins.wait_ctr != NO:
-                        need = (ins.wait_ctr, ins.wait_n)
-                    else:
-                        need = None
-                    if need and f < ins.nfill and ctr[need[0]] < need[1]:
-                        break
-                    if f < ins.nfill:
-                        seq = ins.seq + f
-                        if seq >= issued[s]:
+                while wjob[s][w] < len(J) and wjob[s][w] < prepared[s]:
+                    j = wjob[s][w]
+                    fills = job_fills(L, J[j], w)
+                    k = wpos[s][w]
+                    if k < len(fills):
+                        if fills[k] >= issued[s]:
                             break
-                        released[s][seq] = 1
-                        fill[s][w] += 1
+                        released[s][fills[k]] = 1
+                        wpos[s][w] += 1
                         changed = True
                         continue
-                    # complete
-                    if ins.signal_ctr != NO:
-                        ctr[ins.signal_ctr] += 1
-                    if ins.op == _lib.OP_ATTN and ctr[ins.signal_ctr] == ins.aux_n:
-                        ctr[ins.aux_ctr] += 1
-                    done += 1
-                    pos[s][w] += W
-                    fill[s][w] = 0
+                    done[s][j] += 1
+                    if done[s][j] == W:
+                        i, c, _ = J[j]
+                        ins = L[i]
+                        if ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
+                            ctr[ins.signal_ctr] += 1
+                    wjob[s][w] += 1
+                    wpos[s][w] = 0
                     changed = True
-    return done == n_total, ctr, rounds
+    ok = all(all(d == W for d in dj) for dj in done)
+    return ok, ctr
 
 
 def check_plan(cfg, batch, max_ctx, n_sm, **opts):
     instrs, offs, info = plan_schedule(cfg, batch, max_ctx, n_sm, max_batch=8, max_seq=max_ctx, **opts)
+    n_sm = len(offs) - 1
     assert info.n_instr == len(instrs) and offs[-1] == len(instrs)
     # per-SM fill numbering is the prefix sum of fills
     for s in range(n_sm):
@@ -101,18 +141,19 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
     assert all(cov[(_lib.OP_LMHEAD, cfg.n_layers - 1, t)] for t in range(cfg.vocab // 4))
     assert len(cov) == (cfg.n_layers * (cfg.n_kv_heads * tpg + cfg.hidden // 2 + cfg.ffn // 2
                                         + batch * cfg.n_kv_heads * max_ctx) + cfg.vocab // 4)
-    # every signalled counter is waited for with the right count
-    signals = collections.Counter(i.signal_ctr for i in instrs)
-    for ins in instrs:
-        if ins.wait_ctr == NO:
-            continue
-        if ins.op == _lib.OP_OPROJ:
-            assert ins.wait_n == batch * cfg.n_kv_heads
-        elif ins.op == _lib.OP_DOWN:
-            for c in range(4):
-                assert signals[ins.wait_ctr + c] == ins.wait_n
-        else:
-            assert signals[ins.wait_ctr] == ins.wait_n
+    # every waited counter's target is the number of jobs that signal it
+    signals = collections.Counter()
+    for s_ in range(n_sm):
+        L = instrs[offs[s_]:offs[s_ + 1]]
+        for (i, c, items) in jobs_of(L):
+            ins = L[i]
+            if ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
+                signals[ins.signal_ctr] += 1
+    for s_ in range(n_sm):
+        L = instrs[offs[s_]:offs[s_ + 1]]
+        for job in jobs_of(L):
+            for c, t in job_waits(L, job):
+                assert signals[c] == t, (c, t, signals[c])
     return instrs, offs, info
 
 
@@ -122,14 +163,18 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
 ])
 def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm):
     instrs, offs, info = check_plan(cfg, batch, ctx, n_sm)
-    ok, ctr, rounds = simulate(instrs, offs, info.n_counters, info.n_stages)
-    assert ok, "simulated step did not complete"
-    signals = collections.Counter(i.signal_ctr for i in instrs if i.signal_ctr != NO)
+    for ns in (1, 2, 3):
+        ok, ctr = simulate(instrs, offs, info.n_counters, info.n_stages, ns)
+        assert ok, "simulated step did not complete"
+    n_sm_ = len(offs) - 1
+    signals = collections.Counter()
+    for s_ in range(n_sm_):
+        L = instrs[offs[s_]:offs[s_ + 1]]
+        for (i, c, items) in jobs_of(L):
+            if L[i].signal_ctr != NO and (L[i].op != _lib.OP_DOWN or c == 3):
+                signals[L[i].signal_ctr] += 1
     for c in range(info.n_counters):
-        expect = signals.get(c, 0)
-        if any(i.op == _lib.OP_ATTN and i.aux_ctr == c for i in instrs):
-            expect = batch * cfg.n_kv_heads
-        assert ctr[c] == expect, c
+        assert ctr[c] == signals.get(c, 0), c
 
 
 def test_balance_1b():
@@ -137,12 +182,12 @@ def test_balance_1b():
     mean = info.bytes_per_step / 148
     assert info.max_sm_bytes <= mean * 1.02
     assert info.min_sm_bytes >= mean * 0.98
-    assert info.stage_bytes == 16384 and info.n_stages >= 9
+    assert info.stage_bytes == 16384 and info.n_stages >= 10
 
 
 def test_seeded_placement_is_also_valid():
     instrs, offs, info = check_plan(TINY, 2, 100, 20, seed=1234)
-    ok, _, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
+    ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
     assert ok
 
 
@@ -150,5 +195,5 @@ def test_dropped_item_cannot_complete():
     """The failure-injection hook removes one producer: the protocol must stall
     (on the GPU the bounded waits then end the step with MK_ERR_TIMEOUT)."""
     instrs, offs, info = plan_schedule(TINY, 1, 64, 16, max_seq=64, test_drop_item=5)
-    ok, _, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
+    ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
     assert not ok
