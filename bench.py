@@ -330,6 +330,20 @@ def run_mk(args):
         if code != 0:
             raise RuntimeError(f"baseline step failed: {msg}")
 
+    # ---------------- optional per-job trace of one step (outside the timed region)
+    if args.trace and rank == 0:
+        import numpy as np
+        from persistent_megakernel_interpreter_b200.trace import format_summary, summarize
+        mk.build_schedule(BATCH, past + 1, trace=1)
+        for _ in range(3):
+            mk.decode_step(tokens, positions, kd, vd, logits, stream)
+        stream.synchronize()
+        tr = mk.trace()
+        np.save(args.trace, tr)
+        with open(os.path.splitext(args.trace)[0] + ".txt", "w") as f:
+            f.write(format_summary(summarize(tr)) + "\n")
+        mk.build_schedule(BATCH, past + 1)
+
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -387,6 +401,9 @@ def main(argv=None):
                     help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
                          "small profiling captures of the same kernels)")
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
+    ap.add_argument("--trace", default=None, metavar="FILE",
+                    help="after the timed run, trace one step's per-job timestamps and save "
+                         "them (.npy) with a text summary beside them")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -99,9 +99,11 @@ typedef struct mk_schedule_opts {
     uint32_t seed;           /* 0 = plain greedy placement; else ties are broken by a
                                 seeded shuffle (for robustness tests) */
     int32_t wait_timeout_ms; /* budget of every device wait; 0 = 2000 ms */
-    int32_t test_drop_item;  /* failure-detection test hook: 1-based index, in the global
-                                order, of one work item to leave out (its counter then never
-                                completes and the step ends with MK_ERR_TIMEOUT); 0 = none */
+    int32_t test_drop_item;  /* failure-detection test hook: 1-based index, in the list
+                                order, of one instruction whose completion is never signalled
+                                (its waiters then end the step with MK_ERR_TIMEOUT); 0 = none */
+    int32_t trace;           /* nonzero: every step records per-job timestamps (see
+                                mk_read_trace) */
 } mk_schedule_opts;
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)
@@ -206,6 +208,15 @@ mk_status mk_get_schedule_info(mk_handle* h, mk_schedule_info* info);
  * dependency counters, then epoch, then the end-of-step arrival count.
  * *n_total receives how many exist; at most n are copied. Synchronous. */
 mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_total);
+
+/* Per-job timestamps of the last traced step (schedule built with opts.trace):
+ * uint64 [n_sm][jobs][8] globaltimer nanoseconds -- 0 activation warp starts
+ * waiting for a free input slot, 1 slot free (input counter wait starts),
+ * 2 input counter reached, 3 input prepared, 4 compute warp 0 starts, 5 the
+ * job's last compute warp finished, 6 op | layer << 8 | chunk << 24; 7 unused.
+ * *jobs receives the per-SM job capacity; at most `bytes` are copied.
+ * Synchronous. */
+mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs);
 
 /* Bytes of the packed weight buffer for `cfg`. */
 size_t mk_packed_bytes(const mk_config* cfg);

@@ -30,7 +30,8 @@ class MkWeights(ctypes.Structure):
 class MkScheduleOpts(ctypes.Structure):
     _fields_ = [("n_sm", I32), ("part_keys", I32), ("tiles_qkv", I32), ("tiles_o", I32),
                 ("tiles_gateup", I32), ("rowblocks_down", I32), ("tiles_lm", I32),
-                ("seed", ctypes.c_uint32), ("wait_timeout_ms", I32), ("test_drop_item", I32)]
+                ("seed", ctypes.c_uint32), ("wait_timeout_ms", I32), ("test_drop_item", I32),
+                ("trace", I32)]
 
 
 class MkInstr(ctypes.Structure):
@@ -94,13 +95,14 @@ def lib() -> ctypes.CDLL:
     L.mk_get_schedule_info.argtypes = [P, ctypes.POINTER(MkScheduleInfo)]
     L.mk_read_counters.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_size_t,
                                    ctypes.POINTER(ctypes.c_size_t)]
+    L.mk_read_trace.argtypes = [P, P, ctypes.c_size_t, ctypes.POINTER(I32)]
     L.mk_packed_bytes.argtypes = [ctypes.POINTER(MkConfig)]
     L.mk_packed_bytes.restype = ctypes.c_size_t
     L.mk_pack_weights_host.argtypes = [ctypes.POINTER(MkConfig), ctypes.POINTER(MkWeights), P,
                                        ctypes.c_size_t]
     for f in ("mk_create", "mk_build_schedule", "mk_decode_step", "mk_baseline_decode_step",
               "mk_decode_step_host", "mk_get_status", "mk_plan_schedule_host",
-              "mk_get_schedule_info", "mk_read_counters", "mk_pack_weights_host"):
+              "mk_get_schedule_info", "mk_read_counters", "mk_pack_weights_host", "mk_read_trace"):
         getattr(L, f).restype = st
     _lib = L
     return L

@@ -52,6 +52,8 @@ struct mk_handle {
     mk_schedule_info info{};
     mk::Params params{};
     // staging for the host-buffer entry point
+    uint64_t* d_trace = nullptr;    // per-job timestamps (traced schedules only)
+    int trace_jobs = 0;
     int32_t* d_io = nullptr;        // tokens [max_batch], positions [max_batch]
     float* d_logits = nullptr;
     std::string msg;
@@ -76,6 +78,9 @@ void free_schedule(mk_handle* h) {
     cudaFree(h->d_sm_off);
     cudaFree(h->d_io);
     cudaFree(h->d_logits);
+    cudaFree(h->d_trace);
+    h->d_trace = nullptr;
+    h->trace_jobs = 0;
     h->scratch = nullptr;
     h->d_instrs = nullptr;
     h->d_sm_off = nullptr;
@@ -252,6 +257,24 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         p.attn_item_bytes = sp.item_bytes;
     }
     p.n_counters = I.n_counters;
+    if (opts && opts->trace) {
+        int most = 0;
+        for (int s = 0; s < n_sm; ++s) {
+            int jobs = 0;
+            for (int i = P.sm_off[s]; i < P.sm_off[s + 1];) {
+                const mk_instr& in = P.instrs[i];
+                jobs += in.op == MK_OP_DOWN ? 4 : 1;
+                i += in.op == MK_OP_ATTN ? (int)in.job_items : 1;
+            }
+            most = jobs > most ? jobs : most;
+        }
+        h->trace_jobs = most;
+        const size_t tb = (size_t)n_sm * most * mk::kTraceWords * sizeof(uint64_t);
+        MK_CUDA(h, cudaMalloc(&h->d_trace, tb));
+        MK_CUDA(h, cudaMemset(h->d_trace, 0, tb));
+    }
+    p.trace = h->d_trace;
+    p.trace_jobs = h->trace_jobs;
     p.timeout_ns = mk::kDefaultTimeoutNs;
     if (opts && opts->wait_timeout_ms > 0) p.timeout_ns = (uint64_t)opts->wait_timeout_ms * 1000000ull;
 
@@ -378,6 +401,18 @@ extern "C" mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, si
     MK_CUDA(h, cudaMemcpy(&c, h->ctl, sizeof(c), cudaMemcpyDeviceToHost));
     for (size_t i = 0; i < nc + 2 && i < n; ++i)
         host[i] = i < nc ? raw[i * mk::kCounterStride] : (i == nc ? c.epoch : c.done);
+    return MK_OK;
+}
+
+extern "C" mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h->has_schedule) return MK_ERR_NO_SCHEDULE;
+    if (jobs) *jobs = h->trace_jobs;
+    if (!h->d_trace || !host || bytes == 0) return MK_OK;
+    const size_t tb = (size_t)h->params.n_sm * h->trace_jobs * mk::kTraceWords * sizeof(uint64_t);
+    MK_CUDA(h, cudaSetDevice(h->device));
+    MK_CUDA(h, cudaDeviceSynchronize());
+    MK_CUDA(h, cudaMemcpy(host, h->d_trace, bytes < tb ? bytes : tb, cudaMemcpyDeviceToHost));
     return MK_OK;
 }
 

@@ -160,9 +160,23 @@ __device__ __forceinline__ void xs_store(float* v, int KC, int e, float x) {
     arr[g8 * 4 + (i & 3)] = x;
 }
 
+// Optional per-job timestamps (see TraceWord).
+__device__ __forceinline__ void trace(const Params& p, uint32_t job, int word, uint64_t v) {
+    if (p.trace != nullptr && job < (uint32_t)p.trace_jobs)
+        p.trace[((size_t)blockIdx.x * p.trace_jobs + job) * kTraceWords + word] = v;
+}
+
+// Wait for the job's input counter, then stamp the trace.
+__device__ __forceinline__ bool wait_input(const Params& p, uint32_t ctr, uint32_t target,
+                                           uint32_t where, int lane, uint32_t job) {
+    const bool ok = wait_counter(p, ctr, target, where, lane);
+    if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
+    return ok;
+}
+
 template <int KH, int KO, int KF, int HD>
 __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane,
-                         uint32_t epoch) {
+                         uint32_t epoch, uint32_t job) {
     const mk_instr& in = ins[0];
     const int l = in.layer;
     float* sv = reinterpret_cast<float*>(slot);
@@ -171,7 +185,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
         case MK_OP_GATEUP:
         case MK_OP_LMHEAD: {
             if (in.wait_ctr != MK_NO_COUNTER &&
-                !wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane))
+                !wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job))
                 return false;
             for (int b = 0; b < p.B; ++b) {
                 XSmem<KH> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
@@ -183,7 +197,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             return true;
         }
         case MK_OP_OPROJ: {
-            if (!wait_counter(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane)) return false;
+            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
             for (int b = 0; b < p.B; ++b) {
                 float* v = sv + (size_t)b * p.xs_vec_floats;
                 for (int head = 0; head < p.nq; ++head)
@@ -192,7 +206,8 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             return true;
         }
         case MK_OP_DOWN: {
-            if (!wait_counter(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq, lane))
+            if (!wait_input(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq,
+                            lane, job))
                 return false;
             for (int b = 0; b < p.B; ++b) {
                 XSmem<KF> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
@@ -205,7 +220,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             const int items = (int)in.job_items;
             for (int it = 0; it < items; ++it) {
                 const mk_instr& a = ins[it];
-                if (!wait_counter(p, a.wait_ctr, target_of(epoch, a.wait_n), a.seq, lane)) return false;
+                if (!wait_input(p, a.wait_ctr, target_of(epoch, a.wait_n), a.seq, lane, job)) return false;
                 uint8_t* region = slot + (size_t)it * p.attn_item_bytes;
                 const float* qsrc = p.q + (size_t)a.batch * p.Q + (size_t)a.group * p.group * HD;
                 float* qdst = reinterpret_cast<float*>(region);
@@ -238,10 +253,18 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
         const int njobs = (op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS, use = j / sl.NS;
+            if (lane == 0) {
+                trace(p, j, kTrSlotWait, global_timer_ns());
+                trace(p, j, kTrMeta, op | ((uint32_t)ins[0].layer << 8) | ((uint32_t)c << 24));
+            }
             if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
-            if (!prep_job<KH, KO, KF, HD>(p, ins, c, sl.slot(j), lane, epoch)) return;
+            if (lane == 0) trace(p, j, kTrCtrWait, global_timer_ns());
+            if (!prep_job<KH, KO, KF, HD>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
-            if (lane == 0) mbar_arrive(sl.full + s);  // release: the slot's contents
+            if (lane == 0) {
+                trace(p, j, kTrReady, global_timer_ns());
+                mbar_arrive(sl.full + s);  // release: the slot's contents
+            }
         }
         i += items;
     }
@@ -332,6 +355,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, sl.full + s, (j / sl.NS) & 1u, nullptr, j, 4, lane)) return;
+            if (warp == 0 && lane == 0) trace(p, j, kTrStart, global_timer_ns());
             const float* sv = reinterpret_cast<const float*>(sl.slot(j));
             bool ok;
             switch (in.op) {
@@ -354,6 +378,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 const uint32_t old = atomicAdd(sl.done + s, 1u);
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
+                    trace(p, j, kTrDone, global_timer_ns());
                     const bool last_chunk = in.op != MK_OP_DOWN || c == 3;
                     if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
                         __threadfence();

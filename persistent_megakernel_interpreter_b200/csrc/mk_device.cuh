@@ -108,28 +108,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Activations written earlier in the same kernel by other SMs: read at L2 (.cg).
+// Plain intrinsics (not volatile asm), so independent loads issue together; the
+// acquire loads that guard them clobber memory, so none is hoisted above its wait.
 __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
+    return __ldcg(reinterpret_cast<const uint4*>(p));
 }
 __device__ __forceinline__ uint2 ld_cg_v2(const void* p) {
-    uint2 r;
-    asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-    return r;
+    return __ldcg(reinterpret_cast<const uint2*>(p));
 }
 __device__ __forceinline__ uint32_t ld_cg_u32(const void* p) {
-    uint32_t r;
-    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(r) : "l"(p));
-    return r;
+    return __ldcg(reinterpret_cast<const unsigned int*>(p));
 }
-__device__ __forceinline__ float ld_cg_f32(const float* p) {
-    float r;
-    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(r) : "l"(p));
-    return r;
-}
+__device__ __forceinline__ float ld_cg_f32(const float* p) { return __ldcg(p); }
 
 // Weights streamed once per step: read-only path, no L1 allocation, evict-first in L2.
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p, uint64_t pol) {

@@ -134,6 +134,21 @@ struct Params {
     uint32_t attn_item_bytes;  // one attention item's q and new key/value inside a slot
     int n_counters;
     uint64_t timeout_ns;
+    // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)
+    uint64_t* trace;
+    int trace_jobs;
+};
+
+// Trace record of one job (globaltimer nanoseconds).
+enum TraceWord {
+    kTrSlotWait = 0,   // activation warp starts waiting for a free slot
+    kTrCtrWait = 1,    // slot free; starts waiting for the input counter
+    kTrCtrDone = 2,    // input counter reached
+    kTrReady = 3,      // input prepared, slot handed to the compute warps
+    kTrStart = 4,      // compute warp 0 starts the job
+    kTrDone = 5,       // last compute warp finished (job counter signalled)
+    kTrMeta = 6,       // op | layer << 8 | chunk << 24
+    kTraceWords = 8
 };
 
 // Device status codes live in Ctl::status (values of mk_status).
