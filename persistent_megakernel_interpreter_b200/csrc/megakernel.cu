@@ -184,9 +184,12 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
         case MK_OP_QKV:
         case MK_OP_GATEUP:
         case MK_OP_LMHEAD: {
-            if (in.wait_ctr != MK_NO_COUNTER &&
-                !wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job))
-                return false;
+            if (in.wait_ctr != MK_NO_COUNTER) {
+                if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job))
+                    return false;
+            } else if (lane == 0) {
+                trace(p, job, kTrCtrDone, global_timer_ns());
+            }
             for (int b = 0; b < p.B; ++b) {
                 XSmem<KH> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
                             reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KH * 32};
@@ -196,15 +199,9 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             }
             return true;
         }
-        case MK_OP_OPROJ: {
-            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
-            for (int b = 0; b < p.B; ++b) {
-                float* v = sv + (size_t)b * p.xs_vec_floats;
-                for (int head = 0; head < p.nq; ++head)
-                    attn_merge_head<HD>(p, b, head, lane, [&](int e, float x) { xs_store(v, KO, e, x); });
-            }
-            return true;
-        }
+        case MK_OP_OPROJ:
+            // the compute warps merge the attention partials themselves (in parallel)
+            return wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job);
         case MK_OP_DOWN: {
             if (!wait_input(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq,
                             lane, job))
@@ -271,6 +268,61 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 }
 
 // ------------------------------------------------------------------ compute warps
+
+// The O-projection's input: the merge of the split-K attention partials, heads
+// split over the compute warps (warp w: heads w, w+8, ...), written into the
+// job's slot; then a barrier among the compute warps. Per element the
+// arithmetic is the merge's (max, then fmaf sums in partition order), only the
+// loads are issued together: each lane holds one partition's (m, l).
+template <int HD>
+__device__ void merge_partials(const Params& p, float* sv, int KO, int warp, int lane) {
+    using S = AttnShape<HD>;
+    constexpr int kHW = 4;  // heads per warp (n_heads <= 32)
+    const int P = p.n_parts;
+    for (int b = 0; b < p.B; ++b) {
+        float* v = sv + (size_t)b * p.xs_vec_floats;
+        float mreg[kHW], lreg[kHW], M[kHW], L[kHW], O[kHW][S::DPL];
+#pragma unroll
+        for (int hi = 0; hi < kHW; ++hi) {
+            const int h = warp + hi * kConsumerWarps;
+            mreg[hi] = -INFINITY;
+            lreg[hi] = 0.f;
+            if (h < p.nq && lane < P) {
+                const size_t hp = ((size_t)b * p.nq + h) * P + lane;
+                mreg[hi] = ld_cg_f32(p.part_ml + hp * 2);
+                lreg[hi] = ld_cg_f32(p.part_ml + hp * 2 + 1);
+            }
+            M[hi] = warp_max(mreg[hi]);
+            L[hi] = 0.f;
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d) O[hi][d] = 0.f;
+        }
+#pragma unroll 4
+        for (int j = 0; j < P; ++j) {
+#pragma unroll
+            for (int hi = 0; hi < kHW; ++hi) {
+                const int h = warp + hi * kConsumerWarps;
+                const float mj = __shfl_sync(0xffffffffu, mreg[hi], j);
+                const float lj = __shfl_sync(0xffffffffu, lreg[hi], j);
+                if (h >= p.nq) continue;
+                const float w = expf(mj - M[hi]);   // empty partitions: m = -inf -> 0
+                L[hi] = fmaf(w, lj, L[hi]);
+                const float* o = p.part_o + (((size_t)b * p.nq + h) * P + j) * HD + lane * S::DPL;
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d) O[hi][d] = fmaf(w, ld_cg_f32(o + d), O[hi][d]);
+            }
+        }
+#pragma unroll
+        for (int hi = 0; hi < kHW; ++hi) {
+            const int h = warp + hi * kConsumerWarps;
+            if (h >= p.nq) continue;
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d)
+                xs_store(v, KO, h * HD + lane * S::DPL + d, __fdiv_rn(O[hi][d], L[hi]));
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
 
 template <int OP, int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
@@ -360,7 +412,10 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             bool ok;
             switch (in.op) {
                 case MK_OP_QKV: ok = compute_tiles<MK_OP_QKV, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
-                case MK_OP_OPROJ: ok = compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_OPROJ:
+                    merge_partials<HD>(p, const_cast<float*>(sv), KO, warp, lane);
+                    ok = compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol);
+                    break;
                 case MK_OP_GATEUP: ok = compute_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
                 case MK_OP_LMHEAD: ok = compute_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
                 case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, pol); break;

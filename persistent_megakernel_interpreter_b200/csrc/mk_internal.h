@@ -24,6 +24,7 @@ constexpr int kMaxAttnItems = kConsumerWarps;        // attention items per job,
 constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
+constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA

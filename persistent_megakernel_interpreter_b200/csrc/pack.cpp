@@ -23,6 +23,7 @@ bool make_layout(const mk_config& c, Layout* out, const char** why) {
     if (c.head_dim != 64 && c.head_dim != 128) return fail("head_dim must be 64 or 128");
     const int group = c.n_heads / c.n_kv_heads;
     if (group > 4) return fail("more than 4 query heads per KV head");
+    if (c.n_heads > 32) return fail("more than 32 query heads");
     if (c.hidden % 256) return fail("hidden must be a multiple of 256");
     if ((c.n_heads * c.head_dim) % 256) return fail("n_heads*head_dim must be a multiple of 256");
     if (c.ffn % 1024) return fail("ffn must be a multiple of 1024");

@@ -67,17 +67,21 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const int kps = sp.keys_per_stage;
     if (kps < 1 || sp.stages < 2) return MK_ERR_UNSUPPORTED;
 
-    // attention partitions
-    const int fills_per_seq = (max_ctx + kps - 1) / kps;
+    // attention partitions: about kTargetParts per (sequence, group), each item on
+    // its own SM; a partition is a multiple of 8 keys up to one ring stage, then a
+    // multiple of whole stages (the O-projection merges at most kMaxParts).
+    constexpr int kTargetParts = 8;
     int part_keys;
     if (o.part_keys > 0) {
-        if (o.part_keys % kps) return MK_ERR_INVALID_ARG;
+        if (o.part_keys > kps && o.part_keys % kps) return MK_ERR_INVALID_ARG;
         part_keys = o.part_keys;
     } else {
-        const int want = std::max(1, (n_sm + batch * L.nkv - 1) / (batch * L.nkv));
-        part_keys = kps * ((fills_per_seq + want - 1) / want);
+        const int want = std::max((max_ctx + kTargetParts - 1) / kTargetParts,
+                                  (max_ctx + kMaxParts - 1) / kMaxParts);
+        part_keys = want <= kps ? (want + 7) / 8 * 8 : (want + kps - 1) / kps * kps;
     }
     const int n_parts = (max_ctx + part_keys - 1) / part_keys;
+    if (n_parts > kMaxParts) return MK_ERR_INVALID_ARG;
     const int down_cap = std::max(1, std::min(o.rowblocks_down > 0 ? o.rowblocks_down : kMaxDownRows,
                                               kMaxDownRows));
 
