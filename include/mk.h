@@ -104,6 +104,8 @@ typedef struct mk_schedule_opts {
                                 (its waiters then end the step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
+    int32_t l2_prefetch_fills; /* how many ring fills ahead the loader pulls weights into
+                                L2; 0 = ring stages + 24, negative = off */
 } mk_schedule_opts;
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)

@@ -273,6 +273,9 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         MK_CUDA(h, cudaMalloc(&h->d_trace, tb));
         MK_CUDA(h, cudaMemset(h->d_trace, 0, tb));
     }
+    p.l2_prefetch_fills = (opts && opts->l2_prefetch_fills != 0)
+                              ? (opts->l2_prefetch_fills < 0 ? 0 : opts->l2_prefetch_fills)
+                              : I.n_stages + 24;
     p.trace = h->d_trace;
     p.trace_jobs = h->trace_jobs;
     p.timeout_ns = mk::kDefaultTimeoutNs;

@@ -66,7 +66,9 @@ __global__ void __launch_bounds__(kBaseThreads) k_tiles(const __grid_constant__ 
             if (p.B > 1) prep_input<OP, KC>(p, l, b, x, lane);
             float acc[4];
             dot4<KC, false>(base + (size_t)t * tile_bytes, x, acc, lane, pol);
-            tile_epilogue<OP, HD>(p, l, b, t, acc, lane);
+            RopeRow rr{nullptr, nullptr, 0};
+            if constexpr (OP == MK_OP_QKV) rr = rope_row_global(p, b);
+            tile_epilogue<OP, HD>(p, l, b, t, acc, lane, rr);
         }
     }
 }

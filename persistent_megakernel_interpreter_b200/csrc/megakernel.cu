@@ -197,6 +197,19 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
                 else if (in.op == MK_OP_GATEUP) prep_input<MK_OP_GATEUP, KH>(p, l, b, x, lane);
                 else prep_input<MK_OP_LMHEAD, KH>(p, l, b, x, lane);
             }
+            if (in.op == MK_OP_QKV) {
+                // the RoPE row of each sequence's position, for the epilogues
+                float* aux = sv + (size_t)p.B * p.xs_vec_floats;
+                for (int b = 0; b < p.B; ++b) {
+                    const int pos = p.positions[b];
+                    float* row = aux + (size_t)b * (HD + 4);
+                    for (int i = lane; i < HD / 2; i += 32) {
+                        row[i] = p.rope_cos[(size_t)pos * (HD / 2) + i];
+                        row[HD / 2 + i] = p.rope_sin[(size_t)pos * (HD / 2) + i];
+                    }
+                    if (lane == 0) reinterpret_cast<int*>(row)[HD] = pos;
+                }
+            }
             return true;
         }
         case MK_OP_OPROJ:
@@ -277,39 +290,67 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 template <int HD>
 __device__ void merge_partials(const Params& p, float* sv, int KO, int warp, int lane) {
     using S = AttnShape<HD>;
-    constexpr int kHW = 4;  // heads per warp (n_heads <= 32)
+    constexpr int kHW = 4;     // heads per warp (n_heads <= 32)
+    constexpr int kFast = 8;   // partitions whose outputs are loaded in one batch
     const int P = p.n_parts;
     for (int b = 0; b < p.B; ++b) {
         float* v = sv + (size_t)b * p.xs_vec_floats;
         float mreg[kHW], lreg[kHW], M[kHW], L[kHW], O[kHW][S::DPL];
+        float ov[kHW][kFast][S::DPL];
 #pragma unroll
         for (int hi = 0; hi < kHW; ++hi) {
             const int h = warp + hi * kConsumerWarps;
+            const size_t h0 = ((size_t)b * p.nq + h) * P;
             mreg[hi] = -INFINITY;
             lreg[hi] = 0.f;
             if (h < p.nq && lane < P) {
-                const size_t hp = ((size_t)b * p.nq + h) * P + lane;
-                mreg[hi] = ld_cg_f32(p.part_ml + hp * 2);
-                lreg[hi] = ld_cg_f32(p.part_ml + hp * 2 + 1);
+                mreg[hi] = ld_cg_f32(p.part_ml + (h0 + lane) * 2);
+                lreg[hi] = ld_cg_f32(p.part_ml + (h0 + lane) * 2 + 1);
             }
+#pragma unroll
+            for (int j = 0; j < kFast; ++j)
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d)
+                    ov[hi][j][d] = (h < p.nq && j < P)
+                                       ? ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d)
+                                       : 0.f;
+        }
+#pragma unroll
+        for (int hi = 0; hi < kHW; ++hi) {
             M[hi] = warp_max(mreg[hi]);
             L[hi] = 0.f;
 #pragma unroll
             for (int d = 0; d < S::DPL; ++d) O[hi][d] = 0.f;
         }
-#pragma unroll 4
-        for (int j = 0; j < P; ++j) {
+        for (int j0 = 0; j0 < P; j0 += kFast) {
+            if (j0 > 0) {  // more than kFast partitions: the next batch of outputs
 #pragma unroll
-            for (int hi = 0; hi < kHW; ++hi) {
-                const int h = warp + hi * kConsumerWarps;
-                const float mj = __shfl_sync(0xffffffffu, mreg[hi], j);
-                const float lj = __shfl_sync(0xffffffffu, lreg[hi], j);
-                if (h >= p.nq) continue;
-                const float w = expf(mj - M[hi]);   // empty partitions: m = -inf -> 0
-                L[hi] = fmaf(w, lj, L[hi]);
-                const float* o = p.part_o + (((size_t)b * p.nq + h) * P + j) * HD + lane * S::DPL;
+                for (int hi = 0; hi < kHW; ++hi) {
+                    const int h = warp + hi * kConsumerWarps;
+                    const size_t h0 = ((size_t)b * p.nq + h) * P;
 #pragma unroll
-                for (int d = 0; d < S::DPL; ++d) O[hi][d] = fmaf(w, ld_cg_f32(o + d), O[hi][d]);
+                    for (int j = 0; j < kFast; ++j)
+#pragma unroll
+                        for (int d = 0; d < S::DPL; ++d)
+                            ov[hi][j][d] = (h < p.nq && j0 + j < P)
+                                               ? ld_cg_f32(p.part_o + (h0 + j0 + j) * HD + lane * S::DPL + d)
+                                               : 0.f;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kFast; ++j) {
+                if (j0 + j >= P) break;
+#pragma unroll
+                for (int hi = 0; hi < kHW; ++hi) {
+                    const int h = warp + hi * kConsumerWarps;
+                    const float mj = __shfl_sync(0xffffffffu, mreg[hi], j0 + j);
+                    const float lj = __shfl_sync(0xffffffffu, lreg[hi], j0 + j);
+                    if (h >= p.nq) continue;
+                    const float w = expf(mj - M[hi]);   // empty partitions: m = -inf -> 0
+                    L[hi] = fmaf(w, lj, L[hi]);
+#pragma unroll
+                    for (int d = 0; d < S::DPL; ++d) O[hi][d] = fmaf(w, ov[hi][j][d], O[hi][d]);
+                }
             }
         }
 #pragma unroll
@@ -336,7 +377,12 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
             XSmem<KC> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KC * 32};
             float acc[4];
             dot4<KC, true>(tile, x, acc, lane, pol);
-            tile_epilogue<OP, HD>(p, in.layer, b, in.first + t, acc, lane);
+            RopeRow rr{nullptr, nullptr, 0};
+            if constexpr (OP == MK_OP_QKV) {
+                const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
+                rr = RopeRow{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
+            }
+            tile_epilogue<OP, HD>(p, in.layer, b, in.first + t, acc, lane, rr);
         }
         release_fill(ring, seq, lane);
     }
@@ -427,18 +473,17 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             }
             if (!ok) return;
             // job done for this warp; the last of the 8 publishes the job's counter
+            // (acquire-release at CTA scope on the shared count, then a GPU-scope
+            // release: the other warps' stores are ordered before the signal)
             __syncwarp();
             if (lane == 0) {
-                __threadfence();
-                const uint32_t old = atomicAdd(sl.done + s, 1u);
+                const uint32_t old = atom_shared_acq_rel_add(sl.done + s, 1u);
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
                     trace(p, j, kTrDone, global_timer_ns());
                     const bool last_chunk = in.op != MK_OP_DOWN || c == 3;
-                    if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
-                        __threadfence();
+                    if (last_chunk && in.signal_ctr != MK_NO_COUNTER)
                         red_release_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
-                    }
                 }
                 mbar_arrive(sl.empty + s);
             }
@@ -449,15 +494,74 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
 
 // ------------------------------------------------------------------ the loader warp
 
+// Global source of ring fill t of instruction `in`: one range (weights), or two
+// ranges of `bytes` each for attention (the cached keys and values < pos).
+struct FillSrc {
+    const uint8_t* a;
+    const uint8_t* b;
+    uint32_t bytes;
+};
+
+__device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& in, uint32_t t) {
+    const size_t lbase = p.off_layer0 + (size_t)in.layer * p.layer_stride;
+    switch (in.op) {
+        case MK_OP_ATTN: {
+            const int pos = p.positions[in.batch];
+            const int ka = (int)in.first + (int)t * p.keys_per_stage;
+            const int kend = min(ka + p.keys_per_stage, (int)(in.first + in.count));
+            const int np = max(0, min(kend, pos) - ka);  // cached keys (< pos)
+            const size_t off = kv_off(p, in.layer, in.batch, in.group, ka);
+            return {reinterpret_cast<const uint8_t*>(p.kc + off),
+                    reinterpret_cast<const uint8_t*>(p.vc + off), (uint32_t)np * p.d * 2};
+        }
+        case MK_OP_QKV:
+            return {p.packed + lbase + p.rel_qkv + (size_t)(in.first + t) * p.tile_h, nullptr, p.tile_h};
+        case MK_OP_OPROJ:
+            return {p.packed + lbase + p.rel_o + (size_t)(in.first + t) * p.tile_o, nullptr, p.tile_o};
+        case MK_OP_GATEUP:
+            return {p.packed + lbase + p.rel_gu + (size_t)(in.first + t) * p.tile_h, nullptr, p.tile_h};
+        case MK_OP_DOWN: {
+            const uint32_t c = t / in.count, r = t % in.count;
+            return {p.packed + lbase + p.rel_down + ((size_t)(in.first + r) * 4 + c) * p.tile_f, nullptr,
+                    p.tile_f};
+        }
+        default:  // LM head: rows of the (tied) embedding table
+            return {p.packed + (size_t)(in.first + t) * p.tile_h, nullptr, p.tile_h};
+    }
+}
+
+// One thread streams the SM's fills into the ring. A second cursor runs
+// `l2_prefetch_fills` fills ahead of it and pulls those bytes into L2, so HBM
+// keeps streaming while the ring is full and the compute warps wait for
+// activations; the ring copies then hit L2.
 __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
+    int pf_i = i0;
+    uint32_t pf_t = 0, pf_seq = 0;
     for (int i = i0; i < i1; ++i) {
         const mk_instr in = p.instrs[i];
-        const size_t lbase = p.off_layer0 + (size_t)in.layer * p.layer_stride;
         for (uint32_t t = 0; t < in.nfill; ++t) {
             const uint32_t seq = in.seq + t;
             const uint32_t s = seq % ring.S, use = seq / ring.S;
+            // keep the L2 prefetch cursor ahead
+            while (pf_seq < seq + (uint32_t)p.l2_prefetch_fills && pf_i < i1) {
+                const mk_instr pin = p.instrs[pf_i];
+                if (pf_t >= pin.nfill) {
+                    ++pf_i;
+                    pf_t = 0;
+                    continue;
+                }
+                if (pf_seq >= seq + (uint32_t)ring.S) {  // fills closer than the ring are copied soon
+                    const FillSrc f = fill_source(p, pin, pf_t);
+                    if (f.bytes) {
+                        prefetch_l2(f.a, f.bytes);
+                        if (f.b) prefetch_l2(f.b, f.bytes);
+                    }
+                }
+                ++pf_t;
+                ++pf_seq;
+            }
             if (use > 0) {
                 // wait for the compute warps to release the previous fill of this stage
                 uint64_t t0 = 0;
@@ -479,48 +583,16 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
                 uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
                 uint64_t* bar = ring.full + s;
                 ring.armed[s] = seq;  // published by the release of the arrive below
-                if (in.op == MK_OP_ATTN) {
-                    const int pos = p.positions[in.batch];
-                    const int ka = (int)in.first + (int)t * p.keys_per_stage;
-                    const int kend = min(ka + p.keys_per_stage, (int)(in.first + in.count));
-                    const int np = max(0, min(kend, pos) - ka);  // cached keys (< pos)
-                    const uint32_t bytes = (uint32_t)np * p.d * 2;
-                    mbar_arrive_expect_tx(bar, 2 * bytes);
-                    if (np > 0) {
-                        const size_t off = kv_off(p, in.layer, in.batch, in.group, ka);
-                        bulk_g2s(dst, p.kc + off, bytes, bar, pol);
-                        bulk_g2s(dst + (size_t)p.keys_per_stage * p.d * 2, p.vc + off, bytes, bar, pol);
+                const FillSrc f = fill_source(p, in, t);
+                if (f.b != nullptr) {  // attention: keys, then values half a stage later
+                    mbar_arrive_expect_tx(bar, 2 * f.bytes);
+                    if (f.bytes) {
+                        bulk_g2s(dst, f.a, f.bytes, bar, pol);
+                        bulk_g2s(dst + (size_t)p.keys_per_stage * p.d * 2, f.b, f.bytes, bar, pol);
                     }
                 } else {
-                    const uint8_t* src;
-                    uint32_t bytes;
-                    switch (in.op) {
-                        case MK_OP_QKV:
-                            src = p.packed + lbase + p.rel_qkv + (size_t)(in.first + t) * p.tile_h;
-                            bytes = p.tile_h;
-                            break;
-                        case MK_OP_OPROJ:
-                            src = p.packed + lbase + p.rel_o + (size_t)(in.first + t) * p.tile_o;
-                            bytes = p.tile_o;
-                            break;
-                        case MK_OP_GATEUP:
-                            src = p.packed + lbase + p.rel_gu + (size_t)(in.first + t) * p.tile_h;
-                            bytes = p.tile_h;
-                            break;
-                        case MK_OP_DOWN: {
-                            const uint32_t c = t / in.count, r = t % in.count;
-                            src = p.packed + lbase + p.rel_down +
-                                  ((size_t)(in.first + r) * 4 + c) * p.tile_f;
-                            bytes = p.tile_f;
-                            break;
-                        }
-                        default:  // LM head: rows of the (tied) embedding table
-                            src = p.packed + (size_t)(in.first + t) * p.tile_h;
-                            bytes = p.tile_h;
-                            break;
-                    }
-                    mbar_arrive_expect_tx(bar, bytes);
-                    bulk_g2s(dst, src, bytes, bar, pol);
+                    mbar_arrive_expect_tx(bar, f.bytes);
+                    bulk_g2s(dst, f.a, f.bytes, bar, pol);
                 }
             }
             issued = seq + 1;

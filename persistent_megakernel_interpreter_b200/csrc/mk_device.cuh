@@ -92,6 +92,21 @@ __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Shared-memory counter of a CTA: acquire-release at CTA scope.
+__device__ __forceinline__ uint32_t atom_shared_acq_rel_add(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "r"(smem_addr(p)), "r"(v)
+                 : "memory");
+    return old;
+}
+
+// Pull a byte range into L2 ahead of its use (no completion tracking).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
     uint32_t old;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
@@ -312,25 +327,39 @@ __device__ __forceinline__ size_t kv_off(const Params& p, int l, int b, int g, i
     return ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.max_seq + slot) * p.d;
 }
 
+// Per-sequence context of a tile epilogue: the position and its RoPE row
+// (cos[HD/2], sin[HD/2]), in global memory (baseline) or staged in shared
+// memory by the megakernel's activation warp -- the same values either way.
+struct RopeRow {
+    const float* cos;
+    const float* sin;
+    int pos;
+};
+
+__device__ __forceinline__ RopeRow rope_row_global(const Params& p, int b) {
+    const int pos = p.positions[b];
+    return {p.rope_cos + (size_t)pos * (p.d / 2), p.rope_sin + (size_t)pos * (p.d / 2), pos};
+}
+
 // QKV tile epilogue: RoPE on query/key pairs; q stays fp32, the key and value are
 // rounded to bf16 into the cache slot. `tile` is the tile index inside the
 // layer's QKV block.
 template <int HD>
 __device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint32_t tile,
-                                             const float (&acc)[4], int lane) {
+                                             const float (&acc)[4], int lane, const RopeRow& rr) {
     if (lane >= 4) return;
     constexpr int TPH = HD / 4;  // tiles per head
     const int g = tile / (uint32_t)((p.group + 2) * TPH);
     const int u = tile % (uint32_t)((p.group + 2) * TPH);
     const int hs = u / TPH, j = u % TPH;
-    const int pos = p.positions[b];
+    const int pos = rr.pos;
     if (hs <= p.group) {
         // query head (hs < group) or key head (hs == group): rows {2j, 2j+d/2, 2j+1, 2j+1+d/2}
         const int pair = lane >> 1;          // 0: freq 2j, 1: freq 2j+1
         const int i = 2 * j + pair;
         const float a = pair ? acc[2] : acc[0], bb = pair ? acc[3] : acc[1];
-        const float c = p.rope_cos[(size_t)pos * (HD / 2) + i];
-        const float s = p.rope_sin[(size_t)pos * (HD / 2) + i];
+        const float c = rr.cos[i];
+        const float s = rr.sin[i];
         float out;
         int dim;
         if ((lane & 1) == 0) {
@@ -403,8 +432,8 @@ __device__ __forceinline__ void prep_input(const Params& p, int l, int b, X& x, 
 
 template <int OP, int HD>
 __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uint32_t tile,
-                                              const float (&acc)[4], int lane) {
-    if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD>(p, l, b, tile, acc, lane);
+                                              const float (&acc)[4], int lane, const RopeRow& rr) {
+    if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD>(p, l, b, tile, acc, lane, rr);
     else if constexpr (OP == MK_OP_GATEUP) gateup_epilogue(p, b, tile, acc, lane);
     else if constexpr (OP == MK_OP_OPROJ) residual_epilogue(p, l == 0, b, tile, acc, lane);
     else logits_epilogue(p, b, tile, acc, lane);

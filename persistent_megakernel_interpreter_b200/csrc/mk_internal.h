@@ -134,6 +134,7 @@ struct Params {
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
     uint32_t attn_item_bytes;  // one attention item's q and new key/value inside a slot
     int n_counters;
+    int l2_prefetch_fills;     // how far (in fills) the L2 prefetch runs ahead of the ring
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)
     uint64_t* trace;

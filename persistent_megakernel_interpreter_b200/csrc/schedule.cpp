@@ -38,7 +38,9 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     sp.keys_per_stage = (int)(stage_bytes / (4u * (uint32_t)L.d));
     sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
     sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
-    sp.slot_bytes = align16(std::max((uint32_t)batch * sp.vec_floats * 4u,
+    // per sequence: the input vector, then (QKV jobs) the RoPE row cos[d/2], sin[d/2]
+    // and the position
+    sp.slot_bytes = align16(std::max((uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u,
                                      (uint32_t)kMaxAttnItems * sp.item_bytes));
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
