@@ -240,7 +240,12 @@ def run_mk(args):
     k, v = make_kv_cache(cfg, BATCH, past + 1, past, seed=1)
     mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=past + 1)
     torch.cuda.empty_cache()
-    info = mk.build_schedule(BATCH, past + 1)
+    sched_opts = {}
+    if args.l2_prefetch:
+        sched_opts["l2_prefetch_fills"] = args.l2_prefetch
+    if args.l2_evict_last:
+        sched_opts["l2_prefetch_evict_last"] = 1
+    info = mk.build_schedule(BATCH, past + 1, **sched_opts)
     kd, vd = k.to(dev), v.to(dev)
     tokens = make_tokens(cfg, BATCH, seed=2).to(dev)
     positions = torch.full((BATCH,), past, dtype=torch.int32, device=dev)
@@ -334,7 +339,7 @@ def run_mk(args):
     if args.trace and rank == 0:
         import numpy as np
         from persistent_megakernel_interpreter_b200.trace import format_summary, summarize
-        mk.build_schedule(BATCH, past + 1, trace=1)
+        mk.build_schedule(BATCH, past + 1, trace=1, **sched_opts)
         for _ in range(3):
             mk.decode_step(tokens, positions, kd, vd, logits, stream)
         stream.synchronize()
@@ -342,7 +347,7 @@ def run_mk(args):
         np.save(args.trace, tr)
         with open(os.path.splitext(args.trace)[0] + ".txt", "w") as f:
             f.write(format_summary(summarize(tr)) + "\n")
-        mk.build_schedule(BATCH, past + 1)
+        mk.build_schedule(BATCH, past + 1, **sched_opts)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -401,6 +406,9 @@ def main(argv=None):
                     help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
                          "small profiling captures of the same kernels)")
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
+    ap.add_argument("--l2-prefetch", type=int, default=0,
+                    help="L2 prefetch distance in fills (0 = library default, -1 = off)")
+    ap.add_argument("--l2-evict-last", action="store_true")
     ap.add_argument("--trace", default=None, metavar="FILE",
                     help="after the timed run, trace one step's per-job timestamps and save "
                          "them (.npy) with a text summary beside them")

@@ -104,8 +104,10 @@ typedef struct mk_schedule_opts {
                                 (its waiters then end the step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
-    int32_t l2_prefetch_fills; /* how many ring fills ahead the loader pulls weights into
-                                L2; 0 = ring stages + 24, negative = off */
+    int32_t l2_prefetch_fills; /* while the compute warps wait on activations, the loader
+                                pulls up to this many fills (counted from the next ring
+                                fill) into L2; 0 = ring stages + 24, negative = off */
+    int32_t l2_prefetch_evict_last; /* nonzero: those L2 prefetches carry an evict-last hint */
 } mk_schedule_opts;
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)

@@ -34,6 +34,10 @@
 
 namespace mk {
 
+// Each sequence's position, read once per step by thread 0 (constant during
+// the step) so the warps do not reload it from global memory.
+__shared__ int g_pos[kMaxBatch];
+
 struct Ring {
     uint8_t* base;
     uint64_t* full;
@@ -201,7 +205,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
                 // the RoPE row of each sequence's position, for the epilogues
                 float* aux = sv + (size_t)p.B * p.xs_vec_floats;
                 for (int b = 0; b < p.B; ++b) {
-                    const int pos = p.positions[b];
+                    const int pos = g_pos[b];
                     float* row = aux + (size_t)b * (HD + 4);
                     for (int i = lane; i < HD / 2; i += 32) {
                         row[i] = p.rope_cos[(size_t)pos * (HD / 2) + i];
@@ -236,7 +240,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
                 float* qdst = reinterpret_cast<float*>(region);
                 for (int e = lane * 4; e < p.group * HD; e += 128)
                     *reinterpret_cast<uint4*>(qdst + e) = ld_cg_v4(qsrc + e);
-                const int pos = p.positions[a.batch];
+                const int pos = g_pos[a.batch];
                 const size_t off = kv_off(p, l, a.batch, a.group, pos);
                 uint16_t* kv = reinterpret_cast<uint16_t*>(region + (size_t)p.group * HD * 4);
                 constexpr int kPieces = HD / 8;  // 16-byte pieces per row
@@ -418,7 +422,7 @@ template <int HD>
 __device__ bool compute_attn(const Params& p, const Ring& ring, const mk_instr& a,
                              const uint8_t* region, float* scores, int lane) {
     const int b = a.batch, g = a.group;
-    const int pos = p.positions[b];
+    const int pos = g_pos[b];
     const int kps = p.keys_per_stage;
     const float* q = reinterpret_cast<const float*>(region);
     const uint16_t* knew = reinterpret_cast<const uint16_t*>(region + (size_t)p.group * HD * 4);
@@ -506,7 +510,7 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
     const size_t lbase = p.off_layer0 + (size_t)in.layer * p.layer_stride;
     switch (in.op) {
         case MK_OP_ATTN: {
-            const int pos = p.positions[in.batch];
+            const int pos = g_pos[in.batch];
             const int ka = (int)in.first + (int)t * p.keys_per_stage;
             const int kend = min(ka + p.keys_per_stage, (int)(in.first + in.count));
             const int np = max(0, min(kend, pos) - ka);  // cached keys (< pos)
@@ -530,43 +534,50 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
     }
 }
 
-// One thread streams the SM's fills into the ring. A second cursor runs
-// `l2_prefetch_fills` fills ahead of it and pulls those bytes into L2, so HBM
-// keeps streaming while the ring is full and the compute warps wait for
-// activations; the ring copies then hit L2.
+// One thread streams the SM's fills into the ring. While the ring is full of
+// landed fills the compute warps are waiting on activations; a second cursor
+// then pulls the next fills (up to `l2_prefetch_fills` ahead) into L2, so HBM
+// keeps streaming and the ring copies that follow hit L2.
 __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
     int pf_i = i0;
     uint32_t pf_t = 0, pf_seq = 0;
+    const uint64_t pf_pol = p.l2_prefetch_evict_last ? l2_evict_last_policy() : l2_evict_normal_policy();
     for (int i = i0; i < i1; ++i) {
         const mk_instr in = p.instrs[i];
         for (uint32_t t = 0; t < in.nfill; ++t) {
             const uint32_t seq = in.seq + t;
             const uint32_t s = seq % ring.S, use = seq / ring.S;
-            // keep the L2 prefetch cursor ahead
-            while (pf_seq < seq + (uint32_t)p.l2_prefetch_fills && pf_i < i1) {
-                const mk_instr pin = p.instrs[pf_i];
-                if (pf_t >= pin.nfill) {
-                    ++pf_i;
-                    pf_t = 0;
-                    continue;
-                }
-                if (pf_seq >= seq + (uint32_t)ring.S) {  // fills closer than the ring are copied soon
-                    const FillSrc f = fill_source(p, pin, pf_t);
-                    if (f.bytes) {
-                        prefetch_l2(f.a, f.bytes);
-                        if (f.b) prefetch_l2(f.b, f.bytes);
-                    }
-                }
-                ++pf_t;
-                ++pf_seq;
-            }
             if (use > 0) {
-                // wait for the compute warps to release the previous fill of this stage
+                // Wait for the compute warps to release the previous fill of this
+                // stage. If that fill has already landed, the compute warps are the
+                // ones waiting (on activations) and HBM would idle: meanwhile pull
+                // the next fills into L2, up to l2_prefetch_fills ahead.
                 uint64_t t0 = 0;
                 bool ok = true;
+                if (pf_seq < seq) {  // the cursor never trails the ring
+                    while (pf_i < i1 && pf_seq < seq) {
+                        const uint32_t nf = p.instrs[pf_i].nfill;
+                        const uint32_t step = min(nf - pf_t, seq - pf_seq);
+                        pf_t += step;
+                        pf_seq += step;
+                        if (pf_t >= nf) { ++pf_i; pf_t = 0; }
+                    }
+                }
                 for (uint32_t it = 0; !mbar_try_wait(ring.empty + s, (use - 1) & 1u); ++it) {
+                    if (p.l2_prefetch_fills > 0 && (it & 3u) == 3u && pf_i < i1 &&
+                        pf_seq < seq + (uint32_t)p.l2_prefetch_fills &&
+                        mbar_try_wait(ring.full + s, (use - 1) & 1u)) {
+                        const mk_instr pin = p.instrs[pf_i];
+                        const FillSrc f = fill_source(p, pin, pf_t);
+                        if (f.bytes) {
+                            prefetch_l2(f.a, f.bytes, pf_pol);
+                            if (f.b) prefetch_l2(f.b, f.bytes, pf_pol);
+                        }
+                        ++pf_seq;
+                        if (++pf_t >= pin.nfill) { ++pf_i; pf_t = 0; }
+                    }
                     if ((it & 15u) == 15u) {
                         if (t0 == 0) t0 = global_timer_ns();
                         if (aborted(p)) { ok = false; break; }
@@ -656,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         if (!skip) {
             for (int b = 0; b < p.B; ++b) {
                 const int tok = p.tokens[b], pos = p.positions[b];
+                g_pos[b] = pos;
                 uint32_t code = 0;
                 if (tok < 0 || tok >= p.V) code = MK_ERR_BAD_TOKEN;
                 else if (pos < 0 || pos >= p.max_seq || pos + 1 > p.max_ctx) code = MK_ERR_BAD_POSITION;

@@ -103,8 +103,22 @@ __device__ __forceinline__ uint32_t atom_shared_acq_rel_add(uint32_t* p, uint32_
 }
 
 // Pull a byte range into L2 ahead of its use (no completion tracking).
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes, uint64_t policy) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src),
+                 "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
 
 __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
@@ -273,6 +287,61 @@ __device__ __forceinline__ void rmsnorm_vec(X& x, const uint16_t* w, float eps, 
     }
 }
 
+// RMSNorm of a vector read from global memory (fp32, or bf16 when SRC_BF16),
+// with every load -- the vector and the norm weights -- issued before the
+// reduction. The arithmetic (per-lane sum of squares in element order, the
+// butterfly, (x * r) * w) is the same as load_vec + rmsnorm_vec.
+template <int KC, bool SRC_BF16, class X>
+__device__ __forceinline__ void load_rmsnorm(const void* src, const uint16_t* w, float eps, X& x,
+                                             int lane) {
+    uint4 ra[KC], rb[KC], wv[KC];
+    const uint4* sp = reinterpret_cast<const uint4*>(src);
+    const uint4* wp = reinterpret_cast<const uint4*>(w);
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        if (SRC_BF16) {
+            ra[kc] = ld_cg_v4(sp + kc * 32 + lane);
+        } else {
+            ra[kc] = ld_cg_v4(sp + (kc * 32 + lane) * 2);
+            rb[kc] = ld_cg_v4(sp + (kc * 32 + lane) * 2 + 1);
+        }
+        wv[kc] = ld_cg_v4(wp + kc * 32 + lane);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        float e[8];
+        if (SRC_BF16) {
+            unpack8(ra[kc], e);
+        } else {
+            e[0] = __uint_as_float(ra[kc].x); e[1] = __uint_as_float(ra[kc].y);
+            e[2] = __uint_as_float(ra[kc].z); e[3] = __uint_as_float(ra[kc].w);
+            e[4] = __uint_as_float(rb[kc].x); e[5] = __uint_as_float(rb[kc].y);
+            e[6] = __uint_as_float(rb[kc].z); e[7] = __uint_as_float(rb[kc].w);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
+    }
+    ss = warp_sum(ss);
+    const float r = 1.0f / sqrtf(ss / (float)(KC * 256) + eps);
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+        float e[8], wf[8];
+        if (SRC_BF16) {
+            unpack8(ra[kc], e);
+        } else {
+            e[0] = __uint_as_float(ra[kc].x); e[1] = __uint_as_float(ra[kc].y);
+            e[2] = __uint_as_float(ra[kc].z); e[3] = __uint_as_float(ra[kc].w);
+            e[4] = __uint_as_float(rb[kc].x); e[5] = __uint_as_float(rb[kc].y);
+            e[6] = __uint_as_float(rb[kc].z); e[7] = __uint_as_float(rb[kc].w);
+        }
+        unpack8(wv[kc], wf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(__fmul_rn(e[i], r), wf[i]);
+        x.put(kc, lane, e);
+    }
+}
+
 // ------------------------------------------------------------------ the 4-row tile
 
 __device__ __forceinline__ void fma8(float& acc, uint4 w, const float* x) {
@@ -416,17 +485,17 @@ __device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t
 template <int OP, int KC, class X>
 __device__ __forceinline__ void prep_input(const Params& p, int l, int b, X& x, int lane) {
     if constexpr (OP == MK_OP_QKV) {
-        if (l == 0) load_vec_bf16<KC>(embed_row(p, b), x, lane);
-        else load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
-        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2), p.eps, lane);
+        const uint16_t* w = norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2);
+        if (l == 0) load_rmsnorm<KC, true>(embed_row(p, b), w, p.eps, x, lane);
+        else load_rmsnorm<KC, false>(p.x + (size_t)b * p.H, w, p.eps, x, lane);
     } else if constexpr (OP == MK_OP_GATEUP) {
-        load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
-        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, lane);
+        load_rmsnorm<KC, false>(p.x + (size_t)b * p.H,
+                                norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, x, lane);
     } else if constexpr (OP == MK_OP_OPROJ) {
         load_vec<KC>(p.attn + (size_t)b * p.Q, x, lane);
     } else {  // LM head
-        load_vec<KC>(p.x + (size_t)b * p.H, x, lane);
-        rmsnorm_vec<KC>(x, norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, lane);
+        load_rmsnorm<KC, false>(p.x + (size_t)b * p.H,
+                                norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, x, lane);
     }
 }
 
@@ -497,7 +566,8 @@ __device__ __forceinline__ void attn_init(const Params& p, const float* qg, Attn
 // come from Kc/Vc (row 0 = key ka); the key at `pos`, written earlier in this
 // step, from Kpos/Vpos. All four are bf16 rows in shared memory when SMEM, else
 // in global memory. `s` is this warp's score scratch in shared memory,
-// [kMaxGroup][ks] floats.
+// [kMaxGroup][ks] floats. Independent passes are unrolled and the heads'
+// reductions interleaved, so the chunk's latency is a few dependent steps.
 template <int HD, bool SMEM>
 __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, const uint16_t* Kc,
                                            const uint16_t* Vc, const uint16_t* Kpos,
@@ -507,7 +577,8 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
     const int n = kend - ka;
     const int dc = lane % S::LPK, kk = lane / S::LPK;
     const float scale = 1.0f / sqrtf((float)HD);
-    // scores
+    // scores: S::KPI keys per pass, LPK lanes per key
+#pragma unroll 4
     for (int base = 0; base < n; base += S::KPI) {
         const int j = base + kk;
         float part[kMaxGroup];
@@ -525,10 +596,9 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
                 for (int e = 0; e < 8; ++e) part[h] = fmaf(st.q[h][e], kv[e], part[h]);
         }
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
+        for (int m = S::LPK / 2; m > 0; m >>= 1)
 #pragma unroll
-            for (int m = S::LPK / 2; m > 0; m >>= 1)
-                part[h] += __shfl_xor_sync(0xffffffffu, part[h], m);
+            for (int h = 0; h < kMaxGroup; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], m);
         if (j < n && dc < p.group) {
             float mine = 0.f;
 #pragma unroll
@@ -538,29 +608,47 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
         }
     }
     __syncwarp();
-    // online softmax update per head
+    // online softmax update, all heads together
+    float cm[kMaxGroup], cs[kMaxGroup], m_new[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) cm[h] = -INFINITY;
+    for (int j = lane; j < n; j += 32)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+            if (h < p.group) cm[h] = fmaxf(cm[h], s[h * ks + j]);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) cm[h] = fmaxf(cm[h], __shfl_xor_sync(0xffffffffu, cm[h], m));
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        m_new[h] = fmaxf(st.m[h], cm[h]);
+        cs[h] = 0.f;
+    }
+    for (int j = lane; j < n; j += 32)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+            if (h < p.group) {
+                const float e = expf(s[h * ks + j] - m_new[h]);
+                s[h * ks + j] = e;
+                cs[h] += e;
+            }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) cs[h] += __shfl_xor_sync(0xffffffffu, cs[h], m);
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) {
         if (h >= p.group) continue;
-        float cm = -INFINITY;
-        for (int j = lane; j < n; j += 32) cm = fmaxf(cm, s[h * ks + j]);
-        cm = warp_max(cm);
-        const float m_new = fmaxf(st.m[h], cm);
-        const float alpha = expf(st.m[h] - m_new);   // 0 on the first chunk (m = -inf)
-        float cs = 0.f;
-        for (int j = lane; j < n; j += 32) {
-            const float e = expf(s[h * ks + j] - m_new);
-            s[h * ks + j] = e;
-            cs += e;
-        }
-        cs = warp_sum(cs);
-        st.l[h] = fmaf(st.l[h], alpha, cs);
+        const float alpha = expf(st.m[h] - m_new[h]);   // 0 on the first chunk (m = -inf)
+        st.l[h] = fmaf(st.l[h], alpha, cs[h]);
 #pragma unroll
         for (int e = 0; e < S::DPL; ++e) st.o[h][e] *= alpha;
-        st.m[h] = m_new;
+        st.m[h] = m_new[h];
     }
     __syncwarp();
-    // values
+    // values: keys in order, unrolled so the loads of several keys are in flight
+#pragma unroll 4
     for (int j = 0; j < n; ++j) {
         const int key = ka + j;
         float v[S::DPL];

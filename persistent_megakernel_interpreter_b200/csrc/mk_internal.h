@@ -134,7 +134,8 @@ struct Params {
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
     uint32_t attn_item_bytes;  // one attention item's q and new key/value inside a slot
     int n_counters;
-    int l2_prefetch_fills;     // how far (in fills) the L2 prefetch runs ahead of the ring
+    int l2_prefetch_fills;     // how far (in fills) the L2 prefetch may run ahead (0 = off)
+    int l2_prefetch_evict_last;
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)
     uint64_t* trace;
