@@ -217,7 +217,8 @@ mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_tot
  * uint64 [n_sm][jobs][8] globaltimer nanoseconds -- 0 activation warp starts
  * waiting for a free input slot, 1 slot free (input counter wait starts),
  * 2 input counter reached, 3 input prepared, 4 compute warp 0 starts, 5 the
- * job's last compute warp finished, 6 op | layer << 8 | chunk << 24; 7 unused.
+ * job's last compute warp finished, 6 op | layer << 8 | chunk << 24, 7 compute
+ * warp 0 has its first ring fill of the job (0 if it had none).
  * *jobs receives the per-SM job capacity; at most `bytes` are copied.
  * Synchronous. */
 mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs);

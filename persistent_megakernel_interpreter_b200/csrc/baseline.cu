@@ -108,18 +108,20 @@ __global__ void __launch_bounds__(kBaseThreads) k_attn_partial(const __grid_cons
     if (b >= p.B) return;
     float* sbuf = sbuf_all + (size_t)warp * kMaxGroup * p.keys_per_stage;
     const int pos = p.positions[b];
-    const int k0 = j * p.part_keys, k1 = min(k0 + p.part_keys, p.max_ctx);
+    const uint32_t first = (uint32_t)(j * p.part_keys);
+    const uint32_t count = (uint32_t)min(p.part_keys, p.max_ctx - (int)first);
     AttnState<HD> st;
     attn_init<HD, false>(p, p.q + (size_t)b * p.Q + (size_t)g * p.group * HD, st, lane);
     const uint16_t* Kpos = p.kc + kv_off(p, l, b, g, pos);
     const uint16_t* Vpos = p.vc + kv_off(p, l, b, g, pos);
-    for (int ka = k0; ka < k1; ka += p.keys_per_stage) {
-        const int kend = min(min(ka + p.keys_per_stage, k1), pos + 1);
-        if (ka >= kend) break;
-        attn_chunk<HD, false>(p, st, p.kc + kv_off(p, l, b, g, ka), p.vc + kv_off(p, l, b, g, ka),
-                              Kpos, Vpos, ka, kend, pos, sbuf, p.keys_per_stage, lane);
-    }
-    attn_store_partial<HD>(p, st, b, g, j, lane);
+    const size_t base = kv_off(p, l, b, g, (int)first);
+    auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
+        K = p.kc + base + (size_t)f * p.keys_per_stage * HD;
+        V = p.vc + base + (size_t)f * p.keys_per_stage * HD;
+        return true;
+    };
+    auto done = [](int) {};
+    attn_item_serial<HD, false>(p, st, first, count, pos, Kpos, Vpos, sbuf, lane, rows, done, b, g);
 }
 
 template <int HD>

@@ -150,6 +150,18 @@ __device__ __forceinline__ void release_fill(const Ring& r, uint32_t seq, int la
     if (lane == 0) mbar_arrive(r.empty + seq % r.S);
 }
 
+// Barrier of the 8 compute warps (an mbarrier of count 8; bounded, abort-aware,
+// so a warp that left on an error cannot leave the others waiting forever).
+// `uses` counts this warp's passes; all compute warps pass it in the same jobs.
+__device__ __forceinline__ bool compute_barrier(const Params& p, uint64_t* cbar, uint32_t& uses,
+                                                int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    const bool ok = wait_bar(p, cbar, uses & 1u, nullptr, uses, 5, lane);
+    ++uses;
+    return ok;
+}
+
 // ------------------------------------------------------------------ activation warp
 
 // The down-projection's chunk-c target (chunks may have different job counts).
@@ -292,7 +304,8 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 // arithmetic is the merge's (max, then fmaf sums in partition order), only the
 // loads are issued together: each lane holds one partition's (m, l).
 template <int HD>
-__device__ void merge_partials(const Params& p, float* sv, int KO, int warp, int lane) {
+__device__ bool merge_partials(const Params& p, float* sv, int KO, int warp, int lane,
+                               uint64_t* cbar, uint32_t& cuses) {
     using S = AttnShape<HD>;
     constexpr int kHW = 4;     // heads per warp (n_heads <= 32)
     constexpr int kFast = 8;   // partitions whose outputs are loaded in one batch
@@ -366,15 +379,16 @@ __device__ void merge_partials(const Params& p, float* sv, int KO, int warp, int
                 xs_store(v, KO, h * HD + lane * S::DPL + d, __fdiv_rn(O[hi][d], L[hi]));
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    return compute_barrier(p, cbar, cuses, lane);
 }
 
 template <int OP, int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
-                              const float* sv, int warp, int lane, uint64_t pol) {
+                              const float* sv, int warp, int lane, uint64_t pol, uint32_t job) {
     for (uint32_t t = warp; t < in.count; t += kConsumerWarps) {
         const uint32_t seq = in.seq + t;
         if (!wait_fill(p, ring, seq, lane)) return false;
+        if (t == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
         const uint8_t* tile = ring.stage(seq);
         for (int b = 0; b < p.B; ++b) {
             float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
@@ -397,10 +411,12 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
 // its running sums, chunks in order 0..3; after chunk 3 the residual.
 template <int KF>
 __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
-                             const float* sv, float* tot, int warp, int lane, uint64_t pol) {
+                             const float* sv, float* tot, int warp, int lane, uint64_t pol,
+                             uint32_t job) {
     for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
+        if (r == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
         for (int b = 0; b < p.B; ++b) {
             float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
             XSmem<KF> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KF * 32};
@@ -418,38 +434,112 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
     return true;
 }
 
+// An attention job of `items` items. A lone item whose fills all fit in the
+// ring: its kSubRanges sub-ranges run on the 8 compute warps at once, the
+// sub-range partials meet in the slot and warp 0 folds them in order. Otherwise
+// warp w runs item w's sub-ranges one after another.
 template <int HD>
-__device__ bool compute_attn(const Params& p, const Ring& ring, const mk_instr& a,
-                             const uint8_t* region, float* scores, int lane) {
-    const int b = a.batch, g = a.group;
-    const int pos = g_pos[b];
+__device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr* ins, int items,
+                                 uint8_t* slot, float* scores, int warp, int lane, uint64_t* cbar,
+                                 uint32_t& cuses) {
+    using S = AttnShape<HD>;
     const int kps = p.keys_per_stage;
+    if (items == 1 && ins[0].nfill <= ring.S) {
+        const mk_instr& a = ins[0];
+        const int b = a.batch, g = a.group, pos = g_pos[b];
+        const float* q = reinterpret_cast<const float*>(slot);
+        const uint16_t* knew = reinterpret_cast<const uint16_t*>(slot + (size_t)p.group * HD * 4);
+        const uint16_t* vnew = knew + HD;
+        AttnState<HD> st;
+        attn_init<HD, true>(p, q, st, lane);
+        int lo, hi;
+        sub_range(a.first, a.count, warp, &lo, &hi);
+        auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
+            if (!wait_fill(p, ring, a.seq + f, lane)) return false;
+            K = reinterpret_cast<const uint16_t*>(ring.stage(a.seq + f));
+            V = K + (size_t)kps * HD;
+            return true;
+        };
+        const bool ok = attn_sub<HD, true>(p, st, a.first, lo, hi, pos, knew, vnew, scores, lane, rows,
+                                           [](int) {});
+        constexpr int kSubFloats = 2 * kMaxGroup + kMaxGroup * HD;
+        float* subs = reinterpret_cast<float*>(slot + p.attn_item_bytes);
+        float* mine = subs + (size_t)warp * kSubFloats;
+        if (lane == 0)
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) {
+                mine[h] = st.m[h];
+                mine[kMaxGroup + h] = st.l[h];
+            }
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d) mine[2 * kMaxGroup + h * HD + lane * S::DPL + d] = st.o[h][d];
+        if (!compute_barrier(p, cbar, cuses, lane) || !ok) return false;
+        if (warp == 0) {
+            float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
+            for (int u = 0; u < kSubRanges; ++u) {
+                const float* su = subs + (size_t)u * kSubFloats;
+                float sm[kMaxGroup], sl[kMaxGroup], so[kMaxGroup][S::DPL];
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h) {
+                    sm[h] = su[h];
+                    sl[h] = su[kMaxGroup + h];
+#pragma unroll
+                    for (int d = 0; d < S::DPL; ++d) so[h][d] = su[2 * kMaxGroup + h * HD + lane * S::DPL + d];
+                }
+                if (u == 0) {
+#pragma unroll
+                    for (int h = 0; h < kMaxGroup; ++h) {
+                        rm[h] = sm[h];
+                        rl[h] = sl[h];
+#pragma unroll
+                        for (int d = 0; d < S::DPL; ++d) ro[h][d] = so[h][d];
+                    }
+                } else {
+                    fold_partial<HD>(rm, rl, ro, sm, sl, so);
+                }
+            }
+            attn_store_partial<HD>(p, rm, rl, ro, b, g, (int)(a.first / (uint32_t)p.part_keys), lane);
+            __syncwarp();
+            if (lane == 0)
+                for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+        }
+        return true;
+    }
+    if (warp >= items) return true;
+    const mk_instr& a = ins[warp];
+    const uint8_t* region = slot + (size_t)warp * p.attn_item_bytes;
+    const int b = a.batch, g = a.group, pos = g_pos[b];
     const float* q = reinterpret_cast<const float*>(region);
     const uint16_t* knew = reinterpret_cast<const uint16_t*>(region + (size_t)p.group * HD * 4);
     const uint16_t* vnew = knew + HD;
     AttnState<HD> st;
     attn_init<HD, true>(p, q, st, lane);
-    for (uint32_t ci = 0; ci < a.nfill; ++ci) {
-        const uint32_t seq = a.seq + ci;
-        if (!wait_fill(p, ring, seq, lane)) return false;
-        const int ka = (int)a.first + (int)ci * kps;
-        const int kend = min(min(ka + kps, (int)(a.first + a.count)), pos + 1);
-        if (ka < kend) {
-            const uint16_t* Ks = reinterpret_cast<const uint16_t*>(ring.stage(seq));
-            const uint16_t* Vs = Ks + (size_t)kps * HD;
-            attn_chunk<HD, true>(p, st, Ks, Vs, knew, vnew, ka, kend, pos, scores, kps, lane);
-        }
-        release_fill(ring, seq, lane);
+    uint32_t released = 0;  // fills [0, released) handed back to the loader
+    auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
+        for (; released < (uint32_t)f; ++released) release_fill(ring, a.seq + released, lane);
+        if (!wait_fill(p, ring, a.seq + f, lane)) return false;
+        K = reinterpret_cast<const uint16_t*>(ring.stage(a.seq + f));
+        V = K + (size_t)kps * HD;
+        return true;
+    };
+    if (!attn_item_serial<HD, true>(p, st, a.first, a.count, pos, knew, vnew, scores, lane, rows,
+                                    [](int) {}, b, g))
+        return false;
+    for (; released < a.nfill; ++released) {
+        // fills never read (keys past pos) still have to land before they are handed back
+        if (!wait_fill(p, ring, a.seq + released, lane)) return false;
+        release_fill(ring, a.seq + released, lane);
     }
-    attn_store_partial<HD>(p, st, b, g, (int)(a.first / (uint32_t)p.part_keys), lane);
     return true;
 }
 
 template <int KH, int KO, int KF, int HD>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
-                             float* tot, int i0, int i1, int warp, int lane) {
+                             float* tot, uint64_t* cbar, int i0, int i1, int warp, int lane) {
     const uint64_t pol = l2_evict_first_policy();
-    uint32_t j = 0;
+    uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
         const int items = (in.op == MK_OP_ATTN) ? (int)in.job_items : 1;
@@ -461,18 +551,17 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             const float* sv = reinterpret_cast<const float*>(sl.slot(j));
             bool ok;
             switch (in.op) {
-                case MK_OP_QKV: ok = compute_tiles<MK_OP_QKV, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
+                case MK_OP_QKV: ok = compute_tiles<MK_OP_QKV, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
                 case MK_OP_OPROJ:
-                    merge_partials<HD>(p, const_cast<float*>(sv), KO, warp, lane);
-                    ok = compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol);
+                    ok = merge_partials<HD>(p, const_cast<float*>(sv), KO, warp, lane, cbar, cuses) &&
+                         compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol, j);
                     break;
-                case MK_OP_GATEUP: ok = compute_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
-                case MK_OP_LMHEAD: ok = compute_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, sv, warp, lane, pol); break;
-                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, pol); break;
+                case MK_OP_GATEUP: ok = compute_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
+                case MK_OP_LMHEAD: ok = compute_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
+                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, pol, j); break;
                 default:
-                    ok = warp >= items ||
-                         compute_attn<HD>(p, ring, p.instrs[i + warp],
-                                          sl.slot(j) + (size_t)warp * p.attn_item_bytes, scores, lane);
+                    ok = compute_attn_job<HD>(p, ring, p.instrs + i, items, sl.slot(j), scores, warp,
+                                              lane, cbar, cuses);
                     break;
             }
             if (!ok) return;
@@ -661,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(sl.empty + s, kConsumerWarps);
             sl.done[s] = 0;
         }
+        mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
         uint32_t skip = ld_volatile_u32(&p.ctl->status) != 0u;
@@ -692,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             float* scores = reinterpret_cast<float*>(smem + m.scores) +
                             (size_t)warp * kMaxGroupHeads * p.keys_per_stage;
             compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
-                                         i0, i1, warp, lane);
+                                         reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane);
         }
     }
     __syncthreads();

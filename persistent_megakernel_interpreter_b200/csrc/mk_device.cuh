@@ -676,22 +676,128 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
     __syncwarp();
 }
 
-// Write the partition's (m, l, o) for the group's heads.
+// ------------------------------------------------------------------ attention items
+//
+// An item is one (sequence, KV group, key range [first, first+count)) of the
+// split-K attention. Its keys are cut into kSubRanges contiguous sub-ranges of
+// ceil(count / kSubRanges) keys; each sub-range gets its own online-softmax
+// partial (chunks cut at ring-stage boundaries, keys_per_stage apart from
+// `first`), and the item's partial is the ordered combination of the
+// sub-range partials, sub-range 0 first. Whether the sub-ranges run in
+// parallel on several warps or one after another on one warp, every value is
+// computed the same way.
+constexpr int kSubRanges = kSubRangeCount;
+
+__device__ __forceinline__ void sub_range(uint32_t first, uint32_t count, int u, int* lo, int* hi) {
+    const int sub = (int)((count + kSubRanges - 1) / kSubRanges);
+    *lo = (int)first + min(u * sub, (int)count);
+    *hi = (int)first + min((u + 1) * sub, (int)count);
+}
+
+// Fold partial `b` into the running partial `a` (a = a (+) b): rescale both to
+// the larger max. Empty partials (m = -inf) leave the other unchanged.
 template <int HD>
-__device__ __forceinline__ void attn_store_partial(const Params& p, const AttnState<HD>& st, int b,
-                                                   int g, int part, int lane) {
+__device__ __forceinline__ void fold_partial(float (&am)[kMaxGroup], float (&al)[kMaxGroup],
+                                             float (&ao)[kMaxGroup][AttnShape<HD>::DPL],
+                                             const float (&bm)[kMaxGroup], const float (&bl)[kMaxGroup],
+                                             const float (&bo)[kMaxGroup][AttnShape<HD>::DPL]) {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (bm[h] == -INFINITY) continue;
+        if (am[h] == -INFINITY) {
+            am[h] = bm[h];
+            al[h] = bl[h];
+#pragma unroll
+            for (int d = 0; d < AttnShape<HD>::DPL; ++d) ao[h][d] = bo[h][d];
+            continue;
+        }
+        const float M = fmaxf(am[h], bm[h]);
+        const float wa = expf(am[h] - M), wb = expf(bm[h] - M);
+        al[h] = fmaf(al[h], wa, bl[h] * wb);
+#pragma unroll
+        for (int d = 0; d < AttnShape<HD>::DPL; ++d) ao[h][d] = fmaf(ao[h][d], wa, bo[h][d] * wb);
+        am[h] = M;
+    }
+}
+
+// One sub-range [lo, hi) of an item, keys < pos + 1 only. `rows(f, K, V)` gives
+// the bf16 K/V rows of the item's fill f (row 0 = key first + f*kps) and may wait
+// for it; `done(f)` is called once the warp no longer needs fill f.
+template <int HD, bool SMEM, class Rows, class Done>
+__device__ __forceinline__ bool attn_sub(const Params& p, AttnState<HD>& st, uint32_t first, int lo,
+                                         int hi, int pos, const uint16_t* Kpos, const uint16_t* Vpos,
+                                         float* s, int lane, Rows&& rows, Done&& done) {
+    using S = AttnShape<HD>;
+    const int kps = p.keys_per_stage;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        st.m[h] = -INFINITY;
+        st.l[h] = 0.f;
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d) st.o[h][d] = 0.f;
+    }
+    hi = min(hi, pos + 1);
+    if (lo >= hi) return true;
+    const int f0 = (lo - (int)first) / kps, f1 = (hi - 1 - (int)first) / kps;
+    for (int f = f0; f <= f1; ++f) {
+        const int fa = (int)first + f * kps;
+        const uint16_t *K, *V;
+        if (!rows(f, K, V)) return false;
+        const int ka = max(lo, fa), kb = min(hi, fa + kps);
+        attn_chunk<HD, SMEM>(p, st, K + (size_t)(ka - fa) * HD, V + (size_t)(ka - fa) * HD, Kpos, Vpos,
+                             ka, kb, pos, s, kps, lane);
+        done(f);
+    }
+    return true;
+}
+
+// Write an item's (m, l, o) for the group's heads.
+template <int HD>
+__device__ __forceinline__ void attn_store_partial(const Params& p, const float (&m)[kMaxGroup],
+                                                   const float (&l)[kMaxGroup],
+                                                   const float (&o)[kMaxGroup][AttnShape<HD>::DPL],
+                                                   int b, int g, int part, int lane) {
     using S = AttnShape<HD>;
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) {
         if (h >= p.group) continue;
         const size_t hp = ((size_t)b * p.nq + (size_t)(g * p.group + h)) * p.n_parts + part;
         if (lane == 0) {
-            p.part_ml[hp * 2] = st.m[h];
-            p.part_ml[hp * 2 + 1] = st.l[h];
+            p.part_ml[hp * 2] = m[h];
+            p.part_ml[hp * 2 + 1] = l[h];
         }
 #pragma unroll
-        for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = st.o[h][d];
+        for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = o[h][d];
     }
+}
+
+// One whole item on one warp: the sub-ranges in order, each folded into the
+// running partial as soon as it is done. `rows`/`done` as for attn_sub.
+template <int HD, bool SMEM, class Rows, class Done>
+__device__ __forceinline__ bool attn_item_serial(const Params& p, AttnState<HD>& st, uint32_t first,
+                                                 uint32_t count, int pos, const uint16_t* Kpos,
+                                                 const uint16_t* Vpos, float* s, int lane, Rows&& rows,
+                                                 Done&& done, int b, int g) {
+    using S = AttnShape<HD>;
+    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
+    for (int u = 0; u < kSubRanges; ++u) {
+        int lo, hi;
+        sub_range(first, count, u, &lo, &hi);
+        if (!attn_sub<HD, SMEM>(p, st, first, lo, hi, pos, Kpos, Vpos, s, lane, rows, done)) return false;
+        if (u == 0) {
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) {
+                rm[h] = st.m[h];
+                rl[h] = st.l[h];
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d) ro[h][d] = st.o[h][d];
+            }
+        } else {
+            fold_partial<HD>(rm, rl, ro, st.m, st.l, st.o);
+        }
+    }
+    attn_store_partial<HD>(p, rm, rl, ro, b, g, (int)(first / (uint32_t)p.part_keys), lane);
+    return true;
 }
 
 // Merge the n_parts partials of one head of sequence b in partition order:

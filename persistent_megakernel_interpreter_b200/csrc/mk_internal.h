@@ -25,6 +25,7 @@ constexpr int kMaxDownRows = 16;                     // row blocks per down inst
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
+constexpr int kSubRangeCount = 8;                    // sub-ranges of an attention item
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
@@ -62,6 +63,7 @@ struct SmemLayout {
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
     uint32_t scores;                          // per compute warp: attention scores
     uint32_t tot;                             // down-projection running sums
+    uint32_t cbar;                            // barrier of the compute warps
     uint32_t total;
 };
 
@@ -81,6 +83,7 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs_done = o;   o = align16(o + 4u * NS);
     m.scores = o;    o += 4u * kConsumerWarps * kMaxGroupHeads * (uint32_t)keys_per_stage;
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
+    m.cbar = o;      o += 8u;
     m.total = align16(o);
     return m;
 }
@@ -151,6 +154,7 @@ enum TraceWord {
     kTrStart = 4,      // compute warp 0 starts the job
     kTrDone = 5,       // last compute warp finished (job counter signalled)
     kTrMeta = 6,       // op | layer << 8 | chunk << 24
+    kTrFill = 7,       // compute warp 0 has its first ring fill of the job
     kTraceWords = 8
 };
 

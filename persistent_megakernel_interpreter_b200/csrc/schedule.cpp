@@ -40,8 +40,11 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
     // per sequence: the input vector, then (QKV jobs) the RoPE row cos[d/2], sin[d/2]
     // and the position
-    sp.slot_bytes = align16(std::max((uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u,
-                                     (uint32_t)kMaxAttnItems * sp.item_bytes));
+    // an attention job: its items' q and new key/value, or one item plus the
+    // kSubRanges sub-range partials (m, l, o) when its warps split it
+    const uint32_t sub_bytes = 4u * kSubRangeCount * (2u * kMaxGroupHeads + kMaxGroupHeads * (uint32_t)L.d);
+    sp.slot_bytes = align16(std::max({(uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u,
+                                      (uint32_t)kMaxAttnItems * sp.item_bytes, sp.item_bytes + sub_bytes}));
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
         while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, sp.keys_per_stage).total + 1024 <=

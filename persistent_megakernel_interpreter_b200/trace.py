@@ -13,7 +13,7 @@ from __future__ import annotations
 import numpy as np
 
 OPS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
-SLOT_WAIT, CTR_WAIT, CTR_DONE, READY, START, DONE, META = range(7)
+SLOT_WAIT, CTR_WAIT, CTR_DONE, READY, START, DONE, META, FILL = range(8)
 
 
 def records(trace: np.ndarray):
@@ -27,7 +27,8 @@ def records(trace: np.ndarray):
             op = meta & 0xFF
             if op == 0 or r[DONE] == 0:
                 continue
-            rows.append([s, j] + [int(x) for x in r[:6]] + [op, (meta >> 8) & 0xFFFF, meta >> 24])
+            rows.append([s, j] + [int(x) for x in r[:6]] + [op, (meta >> 8) & 0xFFFF, meta >> 24,
+                                                           int(r[FILL])])
     return np.array(rows, dtype=np.int64)
 
 
@@ -49,7 +50,10 @@ def summarize(trace: np.ndarray) -> dict:
         prep = (r[:, 2 + READY] - r[:, 2 + CTR_DONE]) / 1e3
         comp = (r[:, 2 + DONE] - r[:, 2 + START]) / 1e3
         slot = (r[:, 2 + CTR_WAIT] - r[:, 2 + SLOT_WAIT]) / 1e3
+        has_fill = r[:, 11] > 0
+        fillw = ((r[has_fill, 11] - r[has_fill, 2 + START]) / 1e3) if has_fill.any() else np.zeros(1)
         out["ops"][name] = {
+            "first_fill_wait_us": {"mean": float(fillw.mean()), "max": float(fillw.max())},
             "jobs": int(m.sum()),
             "counter_wait_us": {"mean": float(ctr.mean()), "max": float(ctr.max())},
             "prep_us": {"mean": float(prep.mean()), "max": float(prep.max())},
@@ -69,11 +73,13 @@ def summarize(trace: np.ndarray) -> dict:
 
 def format_summary(s: dict) -> str:
     lines = [f"step {s['step_us']:.1f} us, {s['jobs']} jobs"]
-    lines.append(f"{'op':8s} {'jobs':>6s} {'ctr wait':>17s} {'prep':>17s} {'compute':>17s} {'slot wait':>17s}")
+    lines.append(f"{'op':8s} {'jobs':>6s} {'ctr wait':>17s} {'prep':>17s} {'compute':>17s} "
+                 f"{'slot wait':>17s} {'1st fill wait':>17s}")
     for name, o in s["ops"].items():
         f = lambda d: f"{d['mean']:7.2f}/{d['max']:8.2f}"
         lines.append(f"{name:8s} {o['jobs']:6d} {f(o['counter_wait_us']):>17s} {f(o['prep_us']):>17s} "
-                     f"{f(o['compute_us']):>17s} {f(o['slot_wait_us']):>17s}")
+                     f"{f(o['compute_us']):>17s} {f(o['slot_wait_us']):>17s} "
+                     f"{f(o['first_fill_wait_us']):>17s}")
     lines.append("per layer: time (us from step start) at which the op's last job finished")
     for row in s["layers"]:
         parts = [f"L{row['layer']:2d}"]
