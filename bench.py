@@ -245,6 +245,8 @@ def run_mk(args):
         sched_opts["l2_prefetch_fills"] = args.l2_prefetch
     if args.l2_evict_last:
         sched_opts["l2_prefetch_evict_last"] = 1
+    if args.max_inflight:
+        sched_opts["max_inflight"] = args.max_inflight
     info = mk.build_schedule(BATCH, past + 1, **sched_opts)
     kd, vd = k.to(dev), v.to(dev)
     tokens = make_tokens(cfg, BATCH, seed=2).to(dev)
@@ -409,6 +411,7 @@ def main(argv=None):
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="L2 prefetch distance in fills (0 = library default, -1 = off)")
     ap.add_argument("--l2-evict-last", action="store_true")
+    ap.add_argument("--max-inflight", type=int, default=0, help="ring fills in flight at most (0 = default)")
     ap.add_argument("--trace", default=None, metavar="FILE",
                     help="after the timed run, trace one step's per-job timestamps and save "
                          "them (.npy) with a text summary beside them")

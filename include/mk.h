@@ -108,6 +108,8 @@ typedef struct mk_schedule_opts {
                                 pulls up to this many fills (counted from the next ring
                                 fill) into L2; 0 = ring stages + 24, negative = off */
     int32_t l2_prefetch_evict_last; /* nonzero: those L2 prefetches carry an evict-last hint */
+    int32_t max_inflight;    /* ring fills the loader keeps in flight at most (landed fills
+                                still fill the whole ring); 0 = no limit */
 } mk_schedule_opts;
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)
@@ -214,11 +216,12 @@ mk_status mk_get_schedule_info(mk_handle* h, mk_schedule_info* info);
 mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_total);
 
 /* Per-job timestamps of the last traced step (schedule built with opts.trace):
- * uint64 [n_sm][jobs][8] globaltimer nanoseconds -- 0 activation warp starts
+ * uint64 [n_sm][jobs][16] globaltimer nanoseconds -- 0 activation warp starts
  * waiting for a free input slot, 1 slot free (input counter wait starts),
  * 2 input counter reached, 3 input prepared, 4 compute warp 0 starts, 5 the
  * job's last compute warp finished, 6 op | layer << 8 | chunk << 24, 7 compute
- * warp 0 has its first ring fill of the job (0 if it had none).
+ * warp 0 has its first ring fill of the job (0 if it had none), 8..15 finer
+ * op-specific points of compute warp 0 (0 where unused).
  * *jobs receives the per-SM job capacity; at most `bytes` are copied.
  * Synchronous. */
 mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs);

@@ -277,6 +277,7 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
                               ? (opts->l2_prefetch_fills < 0 ? 0 : opts->l2_prefetch_fills)
                               : I.n_stages + 24;
     p.l2_prefetch_evict_last = (opts && opts->l2_prefetch_evict_last) ? 1 : 0;
+    p.max_inflight = (opts && opts->max_inflight > 0 && opts->max_inflight < I.n_stages) ? opts->max_inflight : 0;
     p.trace = h->d_trace;
     p.trace_jobs = h->trace_jobs;
     p.timeout_ns = mk::kDefaultTimeoutNs;

@@ -121,7 +121,9 @@ __global__ void __launch_bounds__(kBaseThreads) k_attn_partial(const __grid_cons
         return true;
     };
     auto done = [](int) {};
-    attn_item_serial<HD, false>(p, st, first, count, pos, Kpos, Vpos, sbuf, lane, rows, done, b, g);
+    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][AttnShape<HD>::DPL];
+    attn_item_serial<HD, false>(p, st, first, count, pos, Kpos, Vpos, sbuf, lane, rows, done, rm, rl, ro);
+    attn_store_partial<HD>(p, rm, rl, ro, b, g, j, lane);
 }
 
 template <int HD>
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(kBaseThreads) k_attn_merge(const __grid_consta
     if (gw >= p.B * p.nq) return;
     const int b = gw / p.nq, head = gw % p.nq;
     float* out = p.attn + (size_t)b * p.Q;
-    attn_merge_head<HD>(p, b, head, lane, [&](int e, float x) { out[e] = x; });
+    attn_merge_heads<HD, 1>(p, b, head, 1, p.nq, lane, [&](int e, float x) { out[e] = x; });
 }
 
 // ------------------------------------------------------------------ host-side launch

@@ -99,6 +99,7 @@ __device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uin
         if ((int32_t)(v - target) < 0) {
             const uint64_t t0 = global_timer_ns();
             for (uint32_t it = 1;; ++it) {
+                __nanosleep(32);
                 v = ld_acquire_u32(c);
                 if ((int32_t)(v - target) >= 0) break;
                 if ((it & 31u) == 0u) {
@@ -118,12 +119,20 @@ __device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uin
 }
 
 // All lanes wait for phase `parity` of an mbarrier; warp-uniform exit. With
-// `armed`, first wait until the ring stage holds fill `seq`.
+// `armed`, first wait until the ring stage holds fill `seq`. Waiting threads
+// sleep in the barrier (suspend hint) or back off, so they do not compete for
+// issue slots with the warps that compute.
 __device__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const volatile uint32_t* armed,
                          uint32_t seq, uint32_t site, int lane) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
-        const bool done = (armed == nullptr || *armed == seq) && mbar_try_wait(bar, parity);
+        bool done;
+        if (armed != nullptr && *armed != seq) {
+            __nanosleep(64);
+            done = false;
+        } else {
+            done = mbar_wait_sleep(bar, parity, 20000u);
+        }
         if (__all_sync(0xffffffffu, done)) return true;
         if ((it & 15u) == 15u) {
             int bad = 0;
@@ -190,6 +199,16 @@ __device__ __forceinline__ bool wait_input(const Params& p, uint32_t ctr, uint32
     return ok;
 }
 
+// The job input of QKV, gate/up and the LM head: RMSNorm of x (or of the
+// embedding row) into a slot. One copy of the code for the three ops.
+template <int KC>
+__device__ __noinline__ void prep_norm(const void* src, bool src_bf16, const uint16_t* w, float eps,
+                                       float* v, int lane) {
+    XSmem<KC> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KC * 32};
+    if (src_bf16) load_rmsnorm<KC, true>(src, w, eps, x, lane);
+    else load_rmsnorm<KC, false>(src, w, eps, x, lane);
+}
+
 template <int KH, int KO, int KF, int HD>
 __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane,
                          uint32_t epoch, uint32_t job) {
@@ -206,12 +225,15 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             } else if (lane == 0) {
                 trace(p, job, kTrCtrDone, global_timer_ns());
             }
+            const size_t nrm = in.op == MK_OP_QKV ? (size_t)(2 * l) : in.op == MK_OP_GATEUP
+                                                                 ? (size_t)(2 * l + 1)
+                                                                 : (size_t)(2 * p.L);
+            const uint16_t* w = norm_ptr(p, p.off_norms + nrm * p.H * 2);
             for (int b = 0; b < p.B; ++b) {
-                XSmem<KH> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
-                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KH * 32};
-                if (in.op == MK_OP_QKV) prep_input<MK_OP_QKV, KH>(p, l, b, x, lane);
-                else if (in.op == MK_OP_GATEUP) prep_input<MK_OP_GATEUP, KH>(p, l, b, x, lane);
-                else prep_input<MK_OP_LMHEAD, KH>(p, l, b, x, lane);
+                const bool emb = in.op == MK_OP_QKV && l == 0;
+                const void* src = emb ? static_cast<const void*>(embed_row(p, b))
+                                      : static_cast<const void*>(p.x + (size_t)b * p.H);
+                prep_norm<KH>(src, emb, w, p.eps, sv + (size_t)b * p.xs_vec_floats, lane);
             }
             if (in.op == MK_OP_QKV) {
                 // the RoPE row of each sequence's position, for the epilogues
@@ -228,9 +250,16 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             }
             return true;
         }
-        case MK_OP_OPROJ:
-            // the compute warps merge the attention partials themselves (in parallel)
-            return wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job);
+        case MK_OP_OPROJ: {
+            // the attention output, finished (normalised or merged) by the attention items
+            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
+            for (int b = 0; b < p.B; ++b) {
+                XSmem<KO> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
+                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KO * 32};
+                load_vec<KO>(p.attn + (size_t)b * p.Q, x, lane);
+            }
+            return true;
+        }
         case MK_OP_DOWN: {
             if (!wait_input(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq,
                             lane, job))
@@ -298,111 +327,52 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 
 // ------------------------------------------------------------------ compute warps
 
-// The O-projection's input: the merge of the split-K attention partials, heads
-// split over the compute warps (warp w: heads w, w+8, ...), written into the
-// job's slot; then a barrier among the compute warps. Per element the
-// arithmetic is the merge's (max, then fmaf sums in partition order), only the
-// loads are issued together: each lane holds one partition's (m, l).
-template <int HD>
-__device__ bool merge_partials(const Params& p, float* sv, int KO, int warp, int lane,
-                               uint64_t* cbar, uint32_t& cuses) {
-    using S = AttnShape<HD>;
-    constexpr int kHW = 4;     // heads per warp (n_heads <= 32)
-    constexpr int kFast = 8;   // partitions whose outputs are loaded in one batch
-    const int P = p.n_parts;
-    for (int b = 0; b < p.B; ++b) {
-        float* v = sv + (size_t)b * p.xs_vec_floats;
-        float mreg[kHW], lreg[kHW], M[kHW], L[kHW], O[kHW][S::DPL];
-        float ov[kHW][kFast][S::DPL];
-#pragma unroll
-        for (int hi = 0; hi < kHW; ++hi) {
-            const int h = warp + hi * kConsumerWarps;
-            const size_t h0 = ((size_t)b * p.nq + h) * P;
-            mreg[hi] = -INFINITY;
-            lreg[hi] = 0.f;
-            if (h < p.nq && lane < P) {
-                mreg[hi] = ld_cg_f32(p.part_ml + (h0 + lane) * 2);
-                lreg[hi] = ld_cg_f32(p.part_ml + (h0 + lane) * 2 + 1);
-            }
-#pragma unroll
-            for (int j = 0; j < kFast; ++j)
-#pragma unroll
-                for (int d = 0; d < S::DPL; ++d)
-                    ov[hi][j][d] = (h < p.nq && j < P)
-                                       ? ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d)
-                                       : 0.f;
-        }
-#pragma unroll
-        for (int hi = 0; hi < kHW; ++hi) {
-            M[hi] = warp_max(mreg[hi]);
-            L[hi] = 0.f;
-#pragma unroll
-            for (int d = 0; d < S::DPL; ++d) O[hi][d] = 0.f;
-        }
-        for (int j0 = 0; j0 < P; j0 += kFast) {
-            if (j0 > 0) {  // more than kFast partitions: the next batch of outputs
-#pragma unroll
-                for (int hi = 0; hi < kHW; ++hi) {
-                    const int h = warp + hi * kConsumerWarps;
-                    const size_t h0 = ((size_t)b * p.nq + h) * P;
-#pragma unroll
-                    for (int j = 0; j < kFast; ++j)
-#pragma unroll
-                        for (int d = 0; d < S::DPL; ++d)
-                            ov[hi][j][d] = (h < p.nq && j0 + j < P)
-                                               ? ld_cg_f32(p.part_o + (h0 + j0 + j) * HD + lane * S::DPL + d)
-                                               : 0.f;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kFast; ++j) {
-                if (j0 + j >= P) break;
-#pragma unroll
-                for (int hi = 0; hi < kHW; ++hi) {
-                    const int h = warp + hi * kConsumerWarps;
-                    const float mj = __shfl_sync(0xffffffffu, mreg[hi], j0 + j);
-                    const float lj = __shfl_sync(0xffffffffu, lreg[hi], j0 + j);
-                    if (h >= p.nq) continue;
-                    const float w = expf(mj - M[hi]);   // empty partitions: m = -inf -> 0
-                    L[hi] = fmaf(w, lj, L[hi]);
-#pragma unroll
-                    for (int d = 0; d < S::DPL; ++d) O[hi][d] = fmaf(w, ov[hi][j][d], O[hi][d]);
-                }
-            }
-        }
-#pragma unroll
-        for (int hi = 0; hi < kHW; ++hi) {
-            const int h = warp + hi * kConsumerWarps;
-            if (h >= p.nq) continue;
-#pragma unroll
-            for (int d = 0; d < S::DPL; ++d)
-                xs_store(v, KO, h * HD + lane * S::DPL + d, __fdiv_rn(O[hi][d], L[hi]));
-        }
-    }
-    return compute_barrier(p, cbar, cuses, lane);
+// One 4-row tile against an input vector in shared memory: a single copy of the
+// code per input width, shared by every op (the kernel's instruction footprint
+// is what each SM re-fetches for every layer).
+template <int KC>
+__device__ __noinline__ float4 tile_dot(const uint8_t* tile, const float* v, int lane) {
+    XSmem<KC> x{reinterpret_cast<float4*>(const_cast<float*>(v)),
+                reinterpret_cast<float4*>(const_cast<float*>(v)) + KC * 32};
+    float acc[4];
+    dot4<KC, true>(tile, x, acc, lane, 0);
+    return make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
-template <int OP, int KC, int HD>
+template <int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
-                              const float* sv, int warp, int lane, uint64_t pol, uint32_t job) {
+                              const float* sv, int warp, int lane, uint32_t job) {
+    int k = 0;  // trace: warp 0's first tiles (fill wait start, fill ready, dot done)
+    auto stamp = [&](int w) {
+        if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w, global_timer_ns());
+    };
     for (uint32_t t = warp; t < in.count; t += kConsumerWarps) {
         const uint32_t seq = in.seq + t;
+        if (k < 2) stamp(3 * k);
         if (!wait_fill(p, ring, seq, lane)) return false;
         if (t == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
+        if (k < 2) stamp(3 * k + 1);
         const uint8_t* tile = ring.stage(seq);
         for (int b = 0; b < p.B; ++b) {
-            float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
-            XSmem<KC> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KC * 32};
-            float acc[4];
-            dot4<KC, true>(tile, x, acc, lane, pol);
-            RopeRow rr{nullptr, nullptr, 0};
-            if constexpr (OP == MK_OP_QKV) {
-                const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
-                rr = RopeRow{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
+            const float4 a4 = tile_dot<KC>(tile, sv + (size_t)b * p.xs_vec_floats, lane);
+            if (k < 2 && b == 0) stamp(3 * k + 2);
+            const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
+            const uint32_t tl = in.first + t;
+            switch (in.op) {
+                case MK_OP_QKV: {
+                    const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
+                    const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
+                    qkv_epilogue<HD>(p, in.layer, b, tl, acc, lane, rr);
+                    break;
+                }
+                case MK_OP_GATEUP: gateup_epilogue(p, b, tl, acc, lane); break;
+                case MK_OP_OPROJ: residual_epilogue(p, in.layer == 0, b, tl, acc, lane); break;
+                default: logits_epilogue(p, b, tl, acc, lane); break;
             }
-            tile_epilogue<OP, HD>(p, in.layer, b, in.first + t, acc, lane, rr);
         }
         release_fill(ring, seq, lane);
+        if (k == 1) stamp(6);
+        ++k;
     }
     return true;
 }
@@ -411,17 +381,14 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
 // its running sums, chunks in order 0..3; after chunk 3 the residual.
 template <int KF>
 __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
-                             const float* sv, float* tot, int warp, int lane, uint64_t pol,
-                             uint32_t job) {
+                             const float* sv, float* tot, int warp, int lane, uint32_t job) {
     for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
         if (r == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
         for (int b = 0; b < p.B; ++b) {
-            float* v = const_cast<float*>(sv) + (size_t)b * p.xs_vec_floats;
-            XSmem<KF> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KF * 32};
-            float acc[4];
-            dot4<KF, true>(ring.stage(seq), x, acc, lane, pol);
+            const float4 a4 = tile_dot<KF>(ring.stage(seq), sv + (size_t)b * p.xs_vec_floats, lane);
+            const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
             if (lane < 4) {
                 float* t = tot + ((size_t)r * p.B + b) * 4 + lane;
                 const float y = pick4(acc, lane);
@@ -434,19 +401,64 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
     return true;
 }
 
+// The end of one attention item (sequence b, KV group g, one key partition) for
+// the group's heads h in [h_lo, h_hi), whose item partial (m, l, o) this warp
+// holds. With a single partition the partial is the output, o / l. Otherwise it
+// is stored, the heads' arrival is counted on the (b, g) arrival counter, and
+// the warp that completes the count merges all partitions of the group in
+// partition order. Either way each head of the pair is signalled once on the
+// attention counter, after its output is written.
+template <int HD>
+__device__ __forceinline__ void attn_finish(const Params& p, const mk_instr& a, uint32_t epoch, int h_lo,
+                                            int h_hi, const float (&m)[kMaxGroup],
+                                            const float (&l)[kMaxGroup],
+                                            const float (&o)[kMaxGroup][AttnShape<HD>::DPL], int lane) {
+    if (a.signal_ctr == MK_NO_COUNTER) return;  // failure injection: the item never completes
+    const int b = a.batch, g = a.group, n = h_hi - h_lo;
+    const int part = (int)(a.first / (uint32_t)p.part_keys);
+    uint32_t* sig = p.counters + (size_t)a.signal_ctr * kCounterStride;
+    if (p.n_parts == 1) {
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+            if (h >= h_lo && h < h_hi) attn_store_final_head<HD>(p, l[h], o[h], b, g * p.group + h, lane);
+        __syncwarp();
+        if (lane == 0) red_release_add(sig, (uint32_t)n);
+        return;
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+        if (h >= h_lo && h < h_hi)
+            attn_store_partial_head<HD>(p, m[h], l[h], o[h], b, g * p.group + h, part, lane);
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        const uint32_t target = (epoch + 1u) * (uint32_t)(p.n_parts * p.group);
+        const uint32_t old = atom_acq_rel_add(p.counters + (size_t)a.aux0 * kCounterStride, (uint32_t)n);
+        last = old + (uint32_t)n == target;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
+    if (!last) return;
+    float* out = p.attn + (size_t)b * p.Q;
+    attn_merge_heads<HD, kMaxGroup>(p, b, g * p.group, 1, (g + 1) * p.group, lane,
+                                    [&](int e, float x) { out[e] = x; });
+    __syncwarp();
+    if (lane == 0) red_release_add(sig, (uint32_t)p.group);
+}
+
 // An attention job of `items` items. A lone item whose fills all fit in the
 // ring: its kSubRanges sub-ranges run on the 8 compute warps at once, the
-// sub-range partials meet in the slot and warp 0 folds them in order. Otherwise
-// warp w runs item w's sub-ranges one after another.
+// sub-range partials meet in the slot, and warp h folds head h's in order.
+// Otherwise warp w runs item w's sub-ranges one after another.
 template <int HD>
 __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr* ins, int items,
                                  uint8_t* slot, float* scores, int warp, int lane, uint64_t* cbar,
-                                 uint32_t& cuses) {
+                                 uint32_t& cuses, uint32_t job, uint32_t epoch) {
     using S = AttnShape<HD>;
     const int kps = p.keys_per_stage;
     if (items == 1 && ins[0].nfill <= ring.S) {
         const mk_instr& a = ins[0];
-        const int b = a.batch, g = a.group, pos = g_pos[b];
+        const int pos = g_pos[a.batch];
         const float* q = reinterpret_cast<const float*>(slot);
         const uint16_t* knew = reinterpret_cast<const uint16_t*>(slot + (size_t)p.group * HD * 4);
         const uint16_t* vnew = knew + HD;
@@ -476,41 +488,47 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
 #pragma unroll
             for (int d = 0; d < S::DPL; ++d) mine[2 * kMaxGroup + h * HD + lane * S::DPL + d] = st.o[h][d];
         if (!compute_barrier(p, cbar, cuses, lane) || !ok) return false;
-        if (warp == 0) {
+        if (warp == kConsumerWarps - 1 && lane == 0)  // every warp is done with the fills
+            for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+        if (warp < p.group) {
+            // head `warp`: the kSubRanges partials folded in order
+            const int h = warp;
             float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
-            for (int u = 0; u < kSubRanges; ++u) {
-                const float* su = subs + (size_t)u * kSubFloats;
-                float sm[kMaxGroup], sl[kMaxGroup], so[kMaxGroup][S::DPL];
 #pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h) {
-                    sm[h] = su[h];
-                    sl[h] = su[kMaxGroup + h];
+            for (int x = 0; x < kMaxGroup; ++x) {
+                rm[x] = -INFINITY;
+                rl[x] = 0.f;
 #pragma unroll
-                    for (int d = 0; d < S::DPL; ++d) so[h][d] = su[2 * kMaxGroup + h * HD + lane * S::DPL + d];
-                }
-                if (u == 0) {
-#pragma unroll
-                    for (int h = 0; h < kMaxGroup; ++h) {
-                        rm[h] = sm[h];
-                        rl[h] = sl[h];
-#pragma unroll
-                        for (int d = 0; d < S::DPL; ++d) ro[h][d] = so[h][d];
-                    }
-                } else {
-                    fold_partial<HD>(rm, rl, ro, sm, sl, so);
-                }
+                for (int d = 0; d < S::DPL; ++d) ro[x][d] = 0.f;
             }
-            attn_store_partial<HD>(p, rm, rl, ro, b, g, (int)(a.first / (uint32_t)p.part_keys), lane);
-            __syncwarp();
-            if (lane == 0)
-                for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+            float M = subs[h], Lh = subs[kMaxGroup + h], O[S::DPL];
+#pragma unroll
+            for (int d = 0; d < S::DPL; ++d) O[d] = subs[2 * kMaxGroup + h * HD + lane * S::DPL + d];
+            for (int u = 1; u < kSubRanges; ++u) {
+                const float* su = subs + (size_t)u * kSubFloats;
+                const float bm = su[h], bl = su[kMaxGroup + h];
+                float bo[S::DPL];
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d) bo[d] = su[2 * kMaxGroup + h * HD + lane * S::DPL + d];
+                fold_one<HD>(M, Lh, O, bm, bl, bo);
+            }
+            // scatter into the per-head arrays attn_finish takes (only head h is used)
+#pragma unroll
+            for (int x = 0; x < kMaxGroup; ++x)
+                if (x == h) {
+                    rm[x] = M;
+                    rl[x] = Lh;
+#pragma unroll
+                    for (int d = 0; d < S::DPL; ++d) ro[x][d] = O[d];
+                }
+            attn_finish<HD>(p, a, epoch, h, h + 1, rm, rl, ro, lane);
         }
         return true;
     }
     if (warp >= items) return true;
     const mk_instr& a = ins[warp];
     const uint8_t* region = slot + (size_t)warp * p.attn_item_bytes;
-    const int b = a.batch, g = a.group, pos = g_pos[b];
+    const int pos = g_pos[a.batch];
     const float* q = reinterpret_cast<const float*>(region);
     const uint16_t* knew = reinterpret_cast<const uint16_t*>(region + (size_t)p.group * HD * 4);
     const uint16_t* vnew = knew + HD;
@@ -524,21 +542,23 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
         V = K + (size_t)kps * HD;
         return true;
     };
+    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
     if (!attn_item_serial<HD, true>(p, st, a.first, a.count, pos, knew, vnew, scores, lane, rows,
-                                    [](int) {}, b, g))
+                                    [](int) {}, rm, rl, ro))
         return false;
     for (; released < a.nfill; ++released) {
         // fills never read (keys past pos) still have to land before they are handed back
         if (!wait_fill(p, ring, a.seq + released, lane)) return false;
         release_fill(ring, a.seq + released, lane);
     }
+    attn_finish<HD>(p, a, epoch, 0, p.group, rm, rl, ro, lane);
     return true;
 }
 
 template <int KH, int KO, int KF, int HD>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
-                             float* tot, uint64_t* cbar, int i0, int i1, int warp, int lane) {
-    const uint64_t pol = l2_evict_first_policy();
+                             float* tot, uint64_t* cbar, int i0, int i1, int warp, int lane,
+                             uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
@@ -551,17 +571,14 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             const float* sv = reinterpret_cast<const float*>(sl.slot(j));
             bool ok;
             switch (in.op) {
-                case MK_OP_QKV: ok = compute_tiles<MK_OP_QKV, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
-                case MK_OP_OPROJ:
-                    ok = merge_partials<HD>(p, const_cast<float*>(sv), KO, warp, lane, cbar, cuses) &&
-                         compute_tiles<MK_OP_OPROJ, KO, HD>(p, ring, in, sv, warp, lane, pol, j);
-                    break;
-                case MK_OP_GATEUP: ok = compute_tiles<MK_OP_GATEUP, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
-                case MK_OP_LMHEAD: ok = compute_tiles<MK_OP_LMHEAD, KH, HD>(p, ring, in, sv, warp, lane, pol, j); break;
-                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, pol, j); break;
+                case MK_OP_QKV: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j); break;
+                case MK_OP_OPROJ: ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j); break;
+                case MK_OP_GATEUP:
+                case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j); break;
+                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j); break;
                 default:
                     ok = compute_attn_job<HD>(p, ring, p.instrs + i, items, sl.slot(j), scores, warp,
-                                              lane, cbar, cuses);
+                                              lane, cbar, cuses, j, epoch);
                     break;
             }
             if (!ok) return;
@@ -574,7 +591,8 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
                     trace(p, j, kTrDone, global_timer_ns());
-                    const bool last_chunk = in.op != MK_OP_DOWN || c == 3;
+                    // attention items signal their heads themselves (attn_finish)
+                    const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN;
                     if (last_chunk && in.signal_ctr != MK_NO_COUNTER)
                         red_release_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
                 }
@@ -654,10 +672,12 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
                         if (pf_t >= nf) { ++pf_i; pf_t = 0; }
                     }
                 }
-                for (uint32_t it = 0; !mbar_try_wait(ring.empty + s, (use - 1) & 1u); ++it) {
-                    if (p.l2_prefetch_fills > 0 && (it & 3u) == 3u && pf_i < i1 &&
-                        pf_seq < seq + (uint32_t)p.l2_prefetch_fills &&
-                        mbar_try_wait(ring.full + s, (use - 1) & 1u)) {
+                for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, 500u); ++it) {
+                    for (int k = 0; k < 2; ++k) {  // up to two prefetches per wake-up
+                        if (!(p.l2_prefetch_fills > 0 && pf_i < i1 &&
+                              pf_seq < seq + (uint32_t)p.l2_prefetch_fills &&
+                              mbar_try_wait(ring.full + s, (use - 1) & 1u)))
+                            break;
                         const mk_instr pin = p.instrs[pf_i];
                         const FillSrc f = fill_source(p, pin, pf_t);
                         if (f.bytes) {
@@ -678,6 +698,23 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
                     }
                 }
                 if (!ok) goto drain;
+            }
+            if (p.max_inflight > 0 && seq >= (uint32_t)p.max_inflight) {
+                // At most max_inflight fills in flight: enough to keep HBM busy, few
+                // enough that the step's latency-critical loads do not queue behind
+                // megabytes of weight traffic. Landed fills still pile up in the ring.
+                const uint32_t o = seq - (uint32_t)p.max_inflight;
+                uint64_t t1 = 0;
+                for (uint32_t it = 0; !mbar_wait_sleep(ring.full + o % ring.S, (o / ring.S) & 1u, 500u); ++it) {
+                    if ((it & 15u) == 15u) {
+                        if (t1 == 0) t1 = global_timer_ns();
+                        if (aborted(p)) goto drain;
+                        if (global_timer_ns() - t1 > p.timeout_ns) {
+                            record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffbu, 0, o, 6);
+                            goto drain;
+                        }
+                    }
+                }
             }
             {
                 uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
@@ -706,7 +743,7 @@ drain:
         const uint32_t last_seq = s + ((issued - 1 - s) / ring.S) * ring.S;
         const uint32_t par = (last_seq / ring.S) & 1u;
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(ring.full + s, par)) {
+        while (!mbar_wait_sleep(ring.full + s, par, 20000u)) {
             if (global_timer_ns() - t0 > p.timeout_ns) {
                 record_error(p, MK_ERR_TIMEOUT, last_seq, 0xfffffffcu, 0, par, 4);
                 break;
@@ -782,7 +819,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             float* scores = reinterpret_cast<float*>(smem + m.scores) +
                             (size_t)warp * kMaxGroupHeads * p.keys_per_stage;
             compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
-                                         reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane);
+                                         reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
+                                         s_epoch);
         }
     }
     __syncthreads();

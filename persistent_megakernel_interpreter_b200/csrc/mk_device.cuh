@@ -59,6 +59,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same, but the thread sleeps (up to `ns` nanoseconds) until the phase
+// completes instead of returning at once: waiting warps then leave their
+// scheduler's issue slots to the warps that work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -208,6 +223,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // arrays, so a warp-wide 16-byte load is conflict-free.
 template <int KC>
 struct XRegs {
+    static constexpr int kUnroll = KC;  // register arrays need compile-time indices
     float v[KC][8];
     __device__ __forceinline__ void put(int kc, int lane, const float* e) {
 #pragma unroll
@@ -221,6 +237,7 @@ struct XRegs {
 
 template <int KC>
 struct XSmem {
+    static constexpr int kUnroll = 2;   // short loop body: the megakernel's code stays small
     float4* a;  // [KC*32] elements 0..3 of each 8-element piece
     float4* b;  // [KC*32] elements 4..7
     __device__ __forceinline__ void put(int kc, int lane, const float* e) {
@@ -364,7 +381,7 @@ __device__ __forceinline__ void dot4(const uint8_t* tile, const X& x, float (&ac
     const uint4* t = reinterpret_cast<const uint4*>(tile);
 #pragma unroll
     for (int r = 0; r < 4; ++r) acc[r] = 0.f;
-#pragma unroll
+#pragma unroll (X::kUnroll)
     for (int kc = 0; kc < KC; ++kc) {
         uint4 w[4];
 #pragma unroll
@@ -578,7 +595,7 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
     const int dc = lane % S::LPK, kk = lane / S::LPK;
     const float scale = 1.0f / sqrtf((float)HD);
     // scores: S::KPI keys per pass, LPK lanes per key
-#pragma unroll 4
+#pragma unroll 2
     for (int base = 0; base < n; base += S::KPI) {
         const int j = base + kk;
         float part[kMaxGroup];
@@ -648,7 +665,7 @@ __device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, c
     }
     __syncwarp();
     // values: keys in order, unrolled so the loads of several keys are in flight
-#pragma unroll 4
+#pragma unroll 2
     for (int j = 0; j < n; ++j) {
         const int key = ka + j;
         float v[S::DPL];
@@ -694,30 +711,37 @@ __device__ __forceinline__ void sub_range(uint32_t first, uint32_t count, int u,
     *hi = (int)first + min((u + 1) * sub, (int)count);
 }
 
-// Fold partial `b` into the running partial `a` (a = a (+) b): rescale both to
-// the larger max. Empty partials (m = -inf) leave the other unchanged.
+// Fold one head's partial (bm, bl, bo) into the running (M, L, O): rescale both
+// to the larger max; an empty partial (m = -inf) leaves the other unchanged.
+template <int HD>
+__device__ __forceinline__ void fold_one(float& M, float& L, float (&O)[AttnShape<HD>::DPL], float bm,
+                                         float bl, const float (&bo)[AttnShape<HD>::DPL]) {
+    if (bm == -INFINITY) return;
+    if (M == -INFINITY) {
+        M = bm;
+        L = bl;
+#pragma unroll
+        for (int d = 0; d < AttnShape<HD>::DPL; ++d) O[d] = bo[d];
+        return;
+    }
+    const float Mn = fmaxf(M, bm);
+    const float wa = expf(M - Mn), wb = expf(bm - Mn);
+    L = fmaf(L, wa, bl * wb);
+#pragma unroll
+    for (int d = 0; d < AttnShape<HD>::DPL; ++d) O[d] = fmaf(O[d], wa, bo[d] * wb);
+    M = Mn;
+}
+
+// Fold partial `b` into the running partial `a` (a = a (+) b) for every head:
+// rescale both to the larger max. Empty partials (m = -inf) leave the other
+// unchanged.
 template <int HD>
 __device__ __forceinline__ void fold_partial(float (&am)[kMaxGroup], float (&al)[kMaxGroup],
                                              float (&ao)[kMaxGroup][AttnShape<HD>::DPL],
                                              const float (&bm)[kMaxGroup], const float (&bl)[kMaxGroup],
                                              const float (&bo)[kMaxGroup][AttnShape<HD>::DPL]) {
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (bm[h] == -INFINITY) continue;
-        if (am[h] == -INFINITY) {
-            am[h] = bm[h];
-            al[h] = bl[h];
-#pragma unroll
-            for (int d = 0; d < AttnShape<HD>::DPL; ++d) ao[h][d] = bo[h][d];
-            continue;
-        }
-        const float M = fmaxf(am[h], bm[h]);
-        const float wa = expf(am[h] - M), wb = expf(bm[h] - M);
-        al[h] = fmaf(al[h], wa, bl[h] * wb);
-#pragma unroll
-        for (int d = 0; d < AttnShape<HD>::DPL; ++d) ao[h][d] = fmaf(ao[h][d], wa, bo[h][d] * wb);
-        am[h] = M;
-    }
+    for (int h = 0; h < kMaxGroup; ++h) fold_one<HD>(am[h], al[h], ao[h], bm[h], bl[h], bo[h]);
 }
 
 // One sub-range [lo, hi) of an item, keys < pos + 1 only. `rows(f, K, V)` gives
@@ -751,35 +775,55 @@ __device__ __forceinline__ bool attn_sub(const Params& p, AttnState<HD>& st, uin
     return true;
 }
 
+// Write one head's partial (m, l, o) of partition `part`.
+template <int HD>
+__device__ __forceinline__ void attn_store_partial_head(const Params& p, float m, float l,
+                                                        const float (&o)[AttnShape<HD>::DPL], int b,
+                                                        int head, int part, int lane) {
+    using S = AttnShape<HD>;
+    const size_t hp = ((size_t)b * p.nq + (size_t)head) * p.n_parts + part;
+    if (lane == 0) {
+        p.part_ml[hp * 2] = m;
+        p.part_ml[hp * 2 + 1] = l;
+    }
+#pragma unroll
+    for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = o[d];
+}
+
 // Write an item's (m, l, o) for the group's heads.
 template <int HD>
 __device__ __forceinline__ void attn_store_partial(const Params& p, const float (&m)[kMaxGroup],
                                                    const float (&l)[kMaxGroup],
                                                    const float (&o)[kMaxGroup][AttnShape<HD>::DPL],
                                                    int b, int g, int part, int lane) {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+        if (h < p.group) attn_store_partial_head<HD>(p, m[h], l[h], o[h], b, g * p.group + h, part, lane);
+}
+
+// The attention output of one head from a partial that covers all its keys:
+// o / l, the same value the merge of a single partition gives (weight e^0 = 1).
+template <int HD>
+__device__ __forceinline__ void attn_store_final_head(const Params& p, float l,
+                                                      const float (&o)[AttnShape<HD>::DPL], int b,
+                                                      int head, int lane) {
     using S = AttnShape<HD>;
+    float* out = p.attn + (size_t)b * p.Q + (size_t)head * HD + lane * S::DPL;
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= p.group) continue;
-        const size_t hp = ((size_t)b * p.nq + (size_t)(g * p.group + h)) * p.n_parts + part;
-        if (lane == 0) {
-            p.part_ml[hp * 2] = m[h];
-            p.part_ml[hp * 2 + 1] = l[h];
-        }
-#pragma unroll
-        for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = o[h][d];
-    }
+    for (int d = 0; d < S::DPL; ++d) out[d] = __fdiv_rn(o[d], l);
 }
 
 // One whole item on one warp: the sub-ranges in order, each folded into the
-// running partial as soon as it is done. `rows`/`done` as for attn_sub.
+// running partial as soon as it is done; the item's partial is left in
+// (rm, rl, ro). `rows`/`done` as for attn_sub.
 template <int HD, bool SMEM, class Rows, class Done>
 __device__ __forceinline__ bool attn_item_serial(const Params& p, AttnState<HD>& st, uint32_t first,
                                                  uint32_t count, int pos, const uint16_t* Kpos,
                                                  const uint16_t* Vpos, float* s, int lane, Rows&& rows,
-                                                 Done&& done, int b, int g) {
+                                                 Done&& done, float (&rm)[kMaxGroup],
+                                                 float (&rl)[kMaxGroup],
+                                                 float (&ro)[kMaxGroup][AttnShape<HD>::DPL]) {
     using S = AttnShape<HD>;
-    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
     for (int u = 0; u < kSubRanges; ++u) {
         int lo, hi;
         sub_range(first, count, u, &lo, &hi);
@@ -796,34 +840,79 @@ __device__ __forceinline__ bool attn_item_serial(const Params& p, AttnState<HD>&
             fold_partial<HD>(rm, rl, ro, st.m, st.l, st.o);
         }
     }
-    attn_store_partial<HD>(p, rm, rl, ro, b, g, (int)(first / (uint32_t)p.part_keys), lane);
     return true;
 }
 
-// Merge the n_parts partials of one head of sequence b in partition order:
-// attn = (sum_j e^(m_j - M) o_j) / (sum_j e^(m_j - M) l_j), M = max_j m_j. The
-// lane's DPL dims go to out[lane*DPL + d] through `put`.
-template <int HD, class Put>
-__device__ __forceinline__ void attn_merge_head(const Params& p, int b, int head, int lane,
-                                                Put&& put) {
+// Merge the n_parts partials of NH heads h = h0 + i*hstep (i < NH; heads >=
+// h_end are skipped) of sequence b, in partition order:
+// attn = (sum_j e^(m_j - M) o_j) / (sum_j e^(m_j - M) l_j), M = max_j m_j.
+// Lane j holds partition j's (m, l) and computes its weight (n_parts <= 32);
+// the outputs of kMergeBatch partitions per head are loaded in one batch. The
+// lane's DPL dims of head h go to out[h*HD + lane*DPL + d] through `put`.
+constexpr int kMergeBatch = 8;
+
+template <int HD, int NH, class Put>
+__device__ __forceinline__ void attn_merge_heads(const Params& p, int b, int h0, int hstep, int h_end,
+                                                 int lane, Put&& put) {
     using S = AttnShape<HD>;
-    const size_t h0 = ((size_t)b * p.nq + head) * p.n_parts;
-    float M = -INFINITY;
-    for (int j = 0; j < p.n_parts; ++j) M = fmaxf(M, ld_cg_f32(p.part_ml + (h0 + j) * 2));
-    float L = 0.f, O[S::DPL];
+    const int P = p.n_parts;
+    float w[NH], l[NH], L[NH], O[NH][S::DPL], ov[NH][kMergeBatch][S::DPL];
+    const float* po[NH];
 #pragma unroll
-    for (int d = 0; d < S::DPL; ++d) O[d] = 0.f;
-    for (int j = 0; j < p.n_parts; ++j) {
-        const float mj = ld_cg_f32(p.part_ml + (h0 + j) * 2);
-        const float lj = ld_cg_f32(p.part_ml + (h0 + j) * 2 + 1);
-        const float w = expf(mj - M);   // empty partitions: m = -inf -> 0
-        L = fmaf(w, lj, L);
+    for (int i = 0; i < NH; ++i) {
+        const int h = h0 + i * hstep;
+        const size_t base = ((size_t)b * p.nq + h) * P;
+        po[i] = p.part_o + base * HD + lane * S::DPL;
+        w[i] = -INFINITY;
+        l[i] = 0.f;
+        if (h < h_end && lane < P) {
+            w[i] = ld_cg_f32(p.part_ml + (base + lane) * 2);
+            l[i] = ld_cg_f32(p.part_ml + (base + lane) * 2 + 1);
+        }
+    }
+    auto load_o = [&](int j0) {
 #pragma unroll
-        for (int d = 0; d < S::DPL; ++d)
-            O[d] = fmaf(w, ld_cg_f32(p.part_o + (h0 + j) * HD + lane * S::DPL + d), O[d]);
+        for (int i = 0; i < NH; ++i) {
+            const bool ok = h0 + i * hstep < h_end;
+#pragma unroll
+            for (int j = 0; j < kMergeBatch; ++j)
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d)
+                    ov[i][j][d] = (ok && j0 + j < P) ? ld_cg_f32(po[i] + (j0 + j) * HD + d) : 0.f;
+        }
+    };
+    load_o(0);
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const float M = warp_max(w[i]);
+        w[i] = (lane < P && h0 + i * hstep < h_end) ? expf(w[i] - M) : 0.f;  // empty: e^-inf = 0
+        L[i] = 0.f;
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d) O[i][d] = 0.f;
+    }
+    // partitions past P contribute w = 0 times o = 0 (exact no-ops)
+#pragma unroll 1
+    for (int j0 = 0; j0 < P; j0 += kMergeBatch) {
+        if (j0 > 0) load_o(j0);
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+#pragma unroll
+            for (int i = 0; i < NH; ++i) {
+                const float wj = __shfl_sync(0xffffffffu, w[i], j0 + j);
+                const float lj = __shfl_sync(0xffffffffu, l[i], j0 + j);
+                L[i] = fmaf(wj, lj, L[i]);
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d) O[i][d] = fmaf(wj, ov[i][j][d], O[i][d]);
+            }
+        }
     }
 #pragma unroll
-    for (int d = 0; d < S::DPL; ++d) put(head * HD + lane * S::DPL + d, __fdiv_rn(O[d], L));
+    for (int i = 0; i < NH; ++i) {
+        const int h = h0 + i * hstep;
+        if (h >= h_end) continue;
+#pragma unroll
+        for (int d = 0; d < S::DPL; ++d) put(h * HD + lane * S::DPL + d, __fdiv_rn(O[i][d], L[i]));
+    }
 }
 
 }  // namespace mk

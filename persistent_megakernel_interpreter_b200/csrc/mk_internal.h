@@ -139,6 +139,7 @@ struct Params {
     int n_counters;
     int l2_prefetch_fills;     // how far (in fills) the L2 prefetch may run ahead (0 = off)
     int l2_prefetch_evict_last;
+    int max_inflight;          // ring fills the loader keeps in flight at most (0 = ring size)
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)
     uint64_t* trace;
@@ -155,7 +156,8 @@ enum TraceWord {
     kTrDone = 5,       // last compute warp finished (job counter signalled)
     kTrMeta = 6,       // op | layer << 8 | chunk << 24
     kTrFill = 7,       // compute warp 0 has its first ring fill of the job
-    kTraceWords = 8
+    kTrSub0 = 8,       // 8..15: op-specific stamps of compute warp 0 (see the kernel)
+    kTraceWords = 16
 };
 
 // Device status codes live in Ctl::status (values of mk_status).

@@ -17,7 +17,11 @@
 //    then the LM head. Each SM's list keeps that order, so every wait refers to
 //    work that comes earlier everywhere: with all CTAs resident the step cannot
 //    deadlock.
-//  * Counter targets are the number of jobs that signal each counter.
+//  * Counter targets are the number of jobs that signal each counter, except the
+//    attention counter of a layer: it counts query heads whose output is final
+//    (batch * n_heads). Each (sequence, KV group) pair also has an arrival
+//    counter that its items' heads increment after storing a split-K partial;
+//    the item that completes it merges the pair. No instruction waits on it.
 #include <algorithm>
 #include <numeric>
 #include <queue>
@@ -72,17 +76,20 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const int kps = sp.keys_per_stage;
     if (kps < 1 || sp.stages < 2) return MK_ERR_UNSUPPORTED;
 
-    // attention partitions: about kTargetParts per (sequence, group), each item on
-    // its own SM; a partition is a multiple of 8 keys up to one ring stage, then a
-    // multiple of whole stages (the O-projection merges at most kMaxParts).
-    constexpr int kTargetParts = 8;
+    // attention partitions: one per (sequence, KV group) up to kKeysPerItem keys,
+    // more for longer contexts, but no more items than SMs (and at most
+    // kMaxParts per pair, the merge's limit). A partition is a multiple of 8 keys
+    // up to one ring stage, then a multiple of whole stages.
+    constexpr int kKeysPerItem = 256;
     int part_keys;
     if (o.part_keys > 0) {
         if (o.part_keys > kps && o.part_keys % kps) return MK_ERR_INVALID_ARG;
         part_keys = o.part_keys;
     } else {
-        const int want = std::max((max_ctx + kTargetParts - 1) / kTargetParts,
-                                  (max_ctx + kMaxParts - 1) / kMaxParts);
+        const int pairs = batch * L.nkv;
+        const int cap = std::max(1, std::min(kMaxParts, n_sm / pairs));
+        const int parts = std::max(1, std::min(cap, (max_ctx + kKeysPerItem - 1) / kKeysPerItem));
+        const int want = std::max((max_ctx + parts - 1) / parts, (max_ctx + kMaxParts - 1) / kMaxParts);
         part_keys = want <= kps ? (want + 7) / 8 * 8 : (want + kps - 1) / kps * kps;
     }
     const int n_parts = (max_ctx + part_keys - 1) / part_keys;
@@ -92,10 +99,11 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
 
     // counters
     int nc = 0;
-    std::vector<int> c_qkv(L.L), c_part(L.L), c_o(L.L), c_h(L.L), c_down(L.L);
+    std::vector<int> c_qkv(L.L), c_part(L.L), c_arr(L.L), c_o(L.L), c_h(L.L), c_down(L.L);
     for (int l = 0; l < L.L; ++l) {
         c_qkv[l] = nc; nc += L.nkv;
         c_part[l] = nc++;
+        c_arr[l] = nc; nc += batch * L.nkv;  // per (sequence, group): heads' partials stored
         c_o[l] = nc++;
         c_h[l] = nc; nc += 4;
         c_down[l] = nc++;
@@ -189,6 +197,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     in.nfill = (in.count + kps - 1) / kps;
                     in.wait_ctr = (uint32_t)(c_qkv[l] + g);
                     in.signal_ctr = (uint32_t)c_part[l];
+                    in.aux0 = (uint32_t)(c_arr[l] + b * L.nkv + g);
                     lists[best].push_back(in);
                     load[best] += (uint64_t)in.count * kv_key_bytes + kJobOverhead;
                     items_on[best]++;
@@ -200,9 +209,11 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
             for (int k = 0; k < n; k += kMaxAttnItems) {
                 const int run = std::min(kMaxAttnItems, n - k);
                 for (int r = 0; r < run; ++r) first[k + r].job_items = r == 0 ? (uint32_t)run : 0u;
-                signals[c_part[l]]++;
             }
         }
+        // each (sequence, group) pair signals each of its query heads once, when
+        // the head's output is final
+        signals[c_part[l]] += (uint32_t)(batch * L.nq);
         emit_ranges(share(L.H / 4, L.tile_o), 1 << 30, 1 << 30, [&](int a, int n) {
             mk_instr in = mk_in(MK_OP_OPROJ, l);
             in.first = (uint32_t)a;

@@ -112,13 +112,13 @@ class Megakernel:
         return code.value, buf.value.decode()
 
     def trace(self):
-        """Per-job timestamps of the last step: int64 array [n_sm][jobs][8] (see mk.h)."""
+        """Per-job timestamps of the last step: uint64 array [n_sm][jobs][16] (see mk.h)."""
         import numpy as np
         L = _lib.lib()
         jobs = ctypes.c_int32(0)
         _lib.check(L.mk_read_trace(self._h, None, 0, ctypes.byref(jobs)), "mk_read_trace")
         n_sm = self.schedule_info().n_sm
-        out = np.zeros((n_sm, jobs.value, 8), dtype=np.uint64)
+        out = np.zeros((n_sm, jobs.value, 16), dtype=np.uint64)
         if jobs.value:
             _lib.check(L.mk_read_trace(self._h, out.ctypes.data, out.nbytes, ctypes.byref(jobs)),
                        "mk_read_trace")

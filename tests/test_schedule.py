@@ -4,7 +4,9 @@ synchronisation protocol -- a loader streaming fills through a ring of S
 stages, an activation warp preparing each job's input in one of NS slots once
 its counters are met, and 8 compute warps splitting each job's fills -- that
 must run to completion (the schedule cannot deadlock) and leave every counter
-at its target."""
+at its target. Attention items signal per query head: a (sequence, KV group)
+pair's heads are signalled once its last partition has arrived (with one
+partition, at once)."""
 import collections
 
 import pytest
@@ -55,9 +57,36 @@ def job_fills(lst, job, w):
     return [ins.seq + t for t in range(w, ins.count, W)]
 
 
-def simulate(instrs, offs, n_counters, S, NS=2):
+def job_done_signals(L, job, group, n_parts, arr, ctr):
+    """Counter increments when all compute warps finished `job` (arr: arrival
+    counts per (sequence, group) pair)."""
+    i, c, items = job
+    ins = L[i]
+    if ins.op == _lib.OP_ATTN:
+        for k in range(items):
+            a = L[i + k]
+            if a.signal_ctr == NO:
+                continue
+            arr[a.aux0] += group
+            if arr[a.aux0] == n_parts * group:
+                ctr[a.signal_ctr] += group
+    elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
+        ctr[ins.signal_ctr] += 1
+
+
+def static_signals(instrs, offs, group, n_parts):
+    ctr, arr = collections.Counter(), collections.Counter()
+    for s_ in range(len(offs) - 1):
+        L = instrs[offs[s_]:offs[s_ + 1]]
+        for job in jobs_of(L):
+            job_done_signals(L, job, group, n_parts, arr, ctr)
+    return ctr
+
+
+def simulate(instrs, offs, n_counters, S, NS=2, group=1, n_parts=1):
     n_sm = len(offs) - 1
     ctr = [0] * n_counters
+    arr = collections.Counter()
     lists = [instrs[offs[s]:offs[s + 1]] for s in range(n_sm)]
     jobs = [jobs_of(L) for L in lists]
     total_fills = [sum(i.nfill for i in L) for L in lists]
@@ -97,10 +126,7 @@ def simulate(instrs, offs, n_counters, S, NS=2):
                         continue
                     done[s][j] += 1
                     if done[s][j] == W:
-                        i, c, _ = J[j]
-                        ins = L[i]
-                        if ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
-                            ctr[ins.signal_ctr] += 1
+                        job_done_signals(L, J[j], group, n_parts, arr, ctr)
                     wjob[s][w] += 1
                     wpos[s][w] = 0
                     changed = True
@@ -141,14 +167,22 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
     assert all(cov[(_lib.OP_LMHEAD, cfg.n_layers - 1, t)] for t in range(cfg.vocab // 4))
     assert len(cov) == (cfg.n_layers * (cfg.n_kv_heads * tpg + cfg.hidden // 2 + cfg.ffn // 2
                                         + batch * cfg.n_kv_heads * max_ctx) + cfg.vocab // 4)
-    # every waited counter's target is the number of jobs that signal it
-    signals = collections.Counter()
-    for s_ in range(n_sm):
-        L = instrs[offs[s_]:offs[s_ + 1]]
-        for (i, c, items) in jobs_of(L):
-            ins = L[i]
-            if ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
-                signals[ins.signal_ctr] += 1
+    # arrival counters: one per (layer, sequence, group), shared by exactly that
+    # pair's items, never waited on
+    arr_of = collections.defaultdict(set)
+    for ins in instrs:
+        if ins.op == _lib.OP_ATTN:
+            arr_of[ins.aux0].add((ins.layer, ins.batch, ins.group))
+            assert ins.aux0 < info.n_counters
+    assert all(len(v) == 1 for v in arr_of.values())
+    assert len(arr_of) == cfg.n_layers * batch * cfg.n_kv_heads
+    waited = {ins.wait_ctr for ins in instrs}
+    assert not waited & set(arr_of)
+    # every waited counter's target is the number of signals it receives
+    signals = static_signals(instrs, offs, cfg.group, info.n_parts)
+    for l in range(cfg.n_layers):
+        c = {ins.signal_ctr for ins in instrs if ins.op == _lib.OP_ATTN and ins.layer == l}
+        assert len(c) == 1 and signals[c.pop()] == batch * cfg.n_heads
     for s_ in range(n_sm):
         L = instrs[offs[s_]:offs[s_ + 1]]
         for job in jobs_of(L):
@@ -164,15 +198,9 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
 def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm):
     instrs, offs, info = check_plan(cfg, batch, ctx, n_sm)
     for ns in (1, 2, 3):
-        ok, ctr = simulate(instrs, offs, info.n_counters, info.n_stages, ns)
+        ok, ctr = simulate(instrs, offs, info.n_counters, info.n_stages, ns, cfg.group, info.n_parts)
         assert ok, "simulated step did not complete"
-    n_sm_ = len(offs) - 1
-    signals = collections.Counter()
-    for s_ in range(n_sm_):
-        L = instrs[offs[s_]:offs[s_ + 1]]
-        for (i, c, items) in jobs_of(L):
-            if L[i].signal_ctr != NO and (L[i].op != _lib.OP_DOWN or c == 3):
-                signals[L[i].signal_ctr] += 1
+    signals = static_signals(instrs, offs, cfg.group, info.n_parts)
     for c in range(info.n_counters):
         assert ctr[c] == signals.get(c, 0), c
 
@@ -187,13 +215,28 @@ def test_balance_1b():
 
 def test_seeded_placement_is_also_valid():
     instrs, offs, info = check_plan(TINY, 2, 100, 20, seed=1234)
-    ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
+    ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages, 2, TINY.group, info.n_parts)
     assert ok
 
 
 def test_dropped_item_cannot_complete():
     """The failure-injection hook removes one producer: the protocol must stall
     (on the GPU the bounded waits then end the step with MK_ERR_TIMEOUT)."""
-    instrs, offs, info = plan_schedule(TINY, 1, 64, 16, max_seq=64, test_drop_item=5)
-    ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages)
-    assert not ok
+    for drop in range(1, 12):
+        instrs, offs, info = plan_schedule(TINY, 1, 64, 16, max_seq=64, test_drop_item=drop)
+        if instrs[drop - 1].op == _lib.OP_LMHEAD:
+            continue  # nothing in the step waits for the logits
+        ok, _ = simulate(instrs, offs, info.n_counters, info.n_stages, 2, TINY.group, info.n_parts)
+        assert not ok, drop
+
+
+@pytest.mark.parametrize("cfg,batch,ctx,parts", [
+    (LLAMA_1B, 1, 129, 1), (LLAMA_1B, 1, 1025, 5), (LLAMA_1B, 1, 8193, 17), (LLAMA_3B, 8, 2049, 2),
+    (TINY, 1, 129, 1),
+])
+def test_partition_count(cfg, batch, ctx, parts):
+    """One partition per (sequence, group) up to 256 keys, more for longer
+    contexts, never more items than SMs."""
+    _, _, info = plan_schedule(cfg, batch, ctx, 148, max_batch=8, max_seq=ctx)
+    assert info.n_parts == parts
+    assert info.n_parts * batch * cfg.n_kv_heads <= 148
