@@ -395,7 +395,7 @@ def run_mk(args):
         dist.destroy_process_group()
 
 
-def main(argv=None):
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -418,6 +418,11 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -89,8 +89,10 @@ mk_status mk_create(const mk_config* cfg, const mk_weights* w, int device, mk_ha
 /* Options for mk_build_schedule; pass NULL for defaults. Zero fields mean "auto". */
 typedef struct mk_schedule_opts {
     int32_t n_sm;            /* SMs to use (<= device SMs); 0 = all */
-    int32_t part_keys;       /* keys per attention partition (multiple of the ring's
-                                keys-per-stage); 0 = sized so partitions cover the SMs */
+    int32_t part_keys;       /* keys per attention partition (a multiple of 8 up to the
+                                ring's keys-per-stage, else a multiple of it); 0 = one
+                                partition per (sequence, KV group) up to 256 keys, more
+                                for longer contexts while the items fit on the SMs */
     int32_t tiles_qkv;       /* 4-row tiles per instruction, per op; 0 = defaults */
     int32_t tiles_o;
     int32_t tiles_gateup;
@@ -163,8 +165,9 @@ const char* mk_status_str(mk_status s);
  * attention items form one job, one item per warp). The kinds: */
 enum {
     MK_OP_QKV = 1,     /* RMSNorm + QKV matvec + RoPE; writes q and the KV slot */
-    MK_OP_ATTN = 2,    /* one split-K GQA attention partial (sequence, KV group, key range) */
-    MK_OP_OPROJ = 3,   /* merge of the attention partials + O-projection + residual */
+    MK_OP_ATTN = 2,    /* GQA attention over one key partition of a (sequence, KV group)
+                          pair; the pair's last partition to finish merges the pair */
+    MK_OP_OPROJ = 3,   /* O-projection + residual */
     MK_OP_GATEUP = 4,  /* RMSNorm + gate/up matvec + SiLU-gated product */
     MK_OP_DOWN = 5,    /* down-projection over the 4 MLP chunks + residual */
     MK_OP_LMHEAD = 6   /* final RMSNorm + LM head */
@@ -182,12 +185,14 @@ typedef struct mk_instr {
     uint32_t wait_ctr;   /* counter waited on (MK_NO_COUNTER: none); DOWN waits on the
                             4 consecutive chunk counters wait_ctr .. wait_ctr+3 */
     uint32_t wait_n;     /* increments that counter receives per step (DOWN: chunk 0) */
-    uint32_t signal_ctr; /* counter incremented by one when the instruction (for ATTN:
-                            its job) is done */
+    uint32_t signal_ctr; /* counter incremented by one when the instruction is done;
+                            ATTN: the layer's attention counter, incremented once per
+                            query head when that head's output is final */
     uint32_t job_items;  /* ATTN: items in the job this entry opens (1..8), 0 for the
                             job's later items; others: 1 */
     uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
-                            high 16 bits of aux0) and 3 (aux1); else 0 */
+                            high 16 bits of aux0) and 3 (aux1). ATTN: aux0 = the pair's
+                            arrival counter (heads whose partial is stored). Else 0 */
 } mk_instr;
 
 typedef struct mk_schedule_info {

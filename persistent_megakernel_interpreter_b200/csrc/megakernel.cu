@@ -17,9 +17,13 @@
 //  * Warp 9 (the activation warp) runs ahead of the compute warps: for each job
 //    it waits for the job's input counter (acquire load, bounded spin), loads
 //    the small activation input from L2 and prepares it in one of a few
-//    shared-memory slots -- RMSNorm for QKV, gate/up and the LM head, the merge
-//    of the split-K attention partials for the O-projection, an MLP chunk for
-//    the down-projection, q and the new key/value for attention.
+//    shared-memory slots -- RMSNorm for QKV, gate/up and the LM head, the
+//    finished attention output for the O-projection, an MLP chunk for the
+//    down-projection, q and the new key/value for attention.
+//  * Attention items finish their own heads: with one key partition per
+//    (sequence, KV group) the item writes o / l; with several, each stores its
+//    partial and the one that completes the pair's arrival count merges the
+//    pair in partition order, so no other SM waits on a merge.
 //  * Warps 0..7 (compute) split each job's tiles (tile t goes to warp t mod 8),
 //    write the outputs, and the last warp to finish increments the job's
 //    output counter (release).
