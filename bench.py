@@ -243,8 +243,8 @@ def run_mk(args):
     sched_opts = {}
     if args.l2_prefetch:
         sched_opts["l2_prefetch_fills"] = args.l2_prefetch
-    if args.l2_evict_last:
-        sched_opts["l2_prefetch_evict_last"] = 1
+    if args.l2_evict_normal:
+        sched_opts["l2_prefetch_policy"] = 1
     if args.max_inflight:
         sched_opts["max_inflight"] = args.max_inflight
     info = mk.build_schedule(BATCH, past + 1, **sched_opts)
@@ -410,7 +410,8 @@ def parse_args(argv=None):
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="L2 prefetch distance in fills (0 = library default, -1 = off)")
-    ap.add_argument("--l2-evict-last", action="store_true")
+    ap.add_argument("--l2-evict-normal", action="store_true",
+                    help="L2 prefetches with an evict-normal hint (default: evict-last)")
     ap.add_argument("--max-inflight", type=int, default=0, help="ring fills in flight at most (0 = default)")
     ap.add_argument("--trace", default=None, metavar="FILE",
                     help="after the timed run, trace one step's per-job timestamps and save "

@@ -106,10 +106,13 @@ typedef struct mk_schedule_opts {
                                 (its waiters then end the step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
-    int32_t l2_prefetch_fills; /* while the compute warps wait on activations, the loader
-                                pulls up to this many fills (counted from the next ring
-                                fill) into L2; 0 = ring stages + 24, negative = off */
-    int32_t l2_prefetch_evict_last; /* nonzero: those L2 prefetches carry an evict-last hint */
+    int32_t l2_prefetch_fills; /* a prefetch warp pulls the SM's upcoming fills into L2, at
+                                most this many fills ahead of the loader's next one, so HBM
+                                keeps streaming while the compute warps wait on
+                                activations; 0 or negative = off (the default: measured
+                                slower on the 1B decode step, see the design notes) */
+    int32_t l2_prefetch_policy; /* L2 eviction hint of those prefetches: 0 = evict-last,
+                                   1 = evict-normal */
     int32_t max_inflight;    /* ring fills the loader keeps in flight at most (landed fills
                                 still fill the whole ring); 0 = no limit */
 } mk_schedule_opts;
@@ -188,11 +191,14 @@ typedef struct mk_instr {
     uint32_t signal_ctr; /* counter incremented by one when the instruction is done;
                             ATTN: the layer's attention counter, incremented once per
                             query head when that head's output is final */
-    uint32_t job_items;  /* ATTN: items in the job this entry opens (1..8), 0 for the
-                            job's later items; others: 1 */
+    uint32_t job_items;  /* 1: every instruction (an attention item included) is one
+                            job of the SM's compute warps (DOWN: four, one per chunk) */
     uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
                             high 16 bits of aux0) and 3 (aux1). ATTN: aux0 = the pair's
-                            arrival counter (heads whose partial is stored). Else 0 */
+                            arrival counter (heads whose partial is stored). QKV and
+                            GATEUP: aux1 = how many consecutive counters from signal_ctr
+                            the instruction increments by one each (the KV groups / MLP
+                            chunks its tiles touch; 0 reads as 1). Else 0 */
 } mk_instr;
 
 typedef struct mk_schedule_info {

@@ -18,6 +18,7 @@ cudaError_t megakernel_launch(const Params& p, cudaStream_t stream);
 size_t megakernel_smem_bytes(const Params& p);
 // baseline.cu
 cudaError_t baseline_launch(const Params& p, cudaStream_t stream, int n_sm);
+cudaError_t baseline_prepare(const Params& p);
 
 // Device gather used by the packer: one warp per segment, 16-byte words.
 __global__ void k_gather(const Segment* segs, size_t n, uint8_t* dst) {
@@ -254,18 +255,14 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         p.xs_slots = sp.xs_slots;
         p.xs_slot_bytes = sp.slot_bytes;
         p.xs_vec_floats = sp.vec_floats;
-        p.attn_item_bytes = sp.item_bytes;
     }
     p.n_counters = I.n_counters;
     if (opts && opts->trace) {
         int most = 0;
         for (int s = 0; s < n_sm; ++s) {
             int jobs = 0;
-            for (int i = P.sm_off[s]; i < P.sm_off[s + 1];) {
-                const mk_instr& in = P.instrs[i];
-                jobs += in.op == MK_OP_DOWN ? 4 : 1;
-                i += in.op == MK_OP_ATTN ? (int)in.job_items : 1;
-            }
+            for (int i = P.sm_off[s]; i < P.sm_off[s + 1]; ++i)
+                jobs += P.instrs[i].op == MK_OP_DOWN ? 4 : 1;
             most = jobs > most ? jobs : most;
         }
         h->trace_jobs = most;
@@ -273,10 +270,8 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         MK_CUDA(h, cudaMalloc(&h->d_trace, tb));
         MK_CUDA(h, cudaMemset(h->d_trace, 0, tb));
     }
-    p.l2_prefetch_fills = (opts && opts->l2_prefetch_fills != 0)
-                              ? (opts->l2_prefetch_fills < 0 ? 0 : opts->l2_prefetch_fills)
-                              : I.n_stages + 24;
-    p.l2_prefetch_evict_last = (opts && opts->l2_prefetch_evict_last) ? 1 : 0;
+    p.l2_prefetch_fills = (opts && opts->l2_prefetch_fills > 0) ? opts->l2_prefetch_fills : 0;
+    p.l2_prefetch_policy = (opts && opts->l2_prefetch_policy == 1) ? 1 : 0;
     p.max_inflight = (opts && opts->max_inflight > 0 && opts->max_inflight < I.n_stages) ? opts->max_inflight : 0;
     p.trace = h->d_trace;
     p.trace_jobs = h->trace_jobs;
@@ -284,6 +279,7 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     if (opts && opts->wait_timeout_ms > 0) p.timeout_ns = (uint64_t)opts->wait_timeout_ms * 1000000ull;
 
     MK_CUDA(h, mk::megakernel_prepare(p));
+    MK_CUDA(h, mk::baseline_prepare(p));
     int per_sm = 0;
     MK_CUDA(h, mk::megakernel_occupancy(p, &per_sm));
     if (per_sm < 1) {

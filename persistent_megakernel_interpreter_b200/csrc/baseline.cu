@@ -98,32 +98,67 @@ __global__ void __launch_bounds__(kBaseThreads) k_down(const __grid_constant__ P
     }
 }
 
+// Rows of one item in the baseline's shared memory: kpad is the partition
+// length rounded up to 16 keys (a multiple of every key-class count). All rows,
+// the key at pos included, are read from the cache, in the same order of
+// arithmetic as the megakernel's rows (whose last row, the key at pos, comes
+// from the step's own k/v).
+__host__ __device__ inline int attn_kpad(int part_keys) { return (part_keys + 15) / 16 * 16; }
+
 template <int HD>
-__global__ void __launch_bounds__(kBaseThreads) k_attn_partial(const __grid_constant__ Params p, int l) {
+__host__ __device__ inline size_t attn_item_smem(int G, int kpad) {
+    return (size_t)align16((uint32_t)(G * HD * 4)) + 2 * (size_t)kpad * HD * 2 + (size_t)kAttnScratchFloats * 4;
+}
+
+// One attention item per CTA: the item's rows (keys first .. first + n - 1, the
+// key at pos included, which the QKV kernel has written) are copied into shared
+// memory as one fill, then the same four phases as the megakernel run on them.
+template <int HD>
+__global__ void __launch_bounds__(kBaseThreads) k_attn_item(const __grid_constant__ Params p, int l) {
     if (step_failed(p)) return;
-    extern __shared__ float sbuf_all[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gw = blockIdx.x * kBaseWarps + warp;
-    const int j = gw % p.n_parts, g = (gw / p.n_parts) % p.nkv, b = gw / (p.n_parts * p.nkv);
-    if (b >= p.B) return;
-    float* sbuf = sbuf_all + (size_t)warp * kMaxGroup * p.keys_per_stage;
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x % p.n_parts, g = (blockIdx.x / p.n_parts) % p.nkv;
+    const int b = blockIdx.x / (p.n_parts * p.nkv);
+    const int G = p.group, kpad = attn_kpad(p.part_keys);
+    float* qs = reinterpret_cast<float*>(sm);
+    uint16_t* rows = reinterpret_cast<uint16_t*>(sm + align16((uint32_t)(G * HD * 4)));
+    float* sc = reinterpret_cast<float*>(rows + 2 * (size_t)kpad * HD);
     const int pos = p.positions[b];
-    const uint32_t first = (uint32_t)(j * p.part_keys);
-    const uint32_t count = (uint32_t)min(p.part_keys, p.max_ctx - (int)first);
-    AttnState<HD> st;
-    attn_init<HD, false>(p, p.q + (size_t)b * p.Q + (size_t)g * p.group * HD, st, lane);
-    const uint16_t* Kpos = p.kc + kv_off(p, l, b, g, pos);
-    const uint16_t* Vpos = p.vc + kv_off(p, l, b, g, pos);
-    const size_t base = kv_off(p, l, b, g, (int)first);
-    auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
-        K = p.kc + base + (size_t)f * p.keys_per_stage * HD;
-        V = p.vc + base + (size_t)f * p.keys_per_stage * HD;
+    const int first = j * p.part_keys;
+    const int count = min(p.part_keys, p.max_ctx - first);
+    const int n = min(count, pos + 1 - first);
+    const float* qsrc = p.q + (size_t)b * p.Q + (size_t)g * G * HD;
+    for (int e = threadIdx.x * 4; e < G * HD; e += kBaseThreads * 4)
+        *reinterpret_cast<uint4*>(qs + e) = ld_cg_v4(qsrc + e);
+    const size_t base = kv_off(p, l, b, g, first);
+    for (int i = threadIdx.x; i < n * (HD / 8); i += kBaseThreads) {
+        reinterpret_cast<uint4*>(rows)[i] = ld_cg_v4(p.kc + base + (size_t)i * 8);
+        reinterpret_cast<uint4*>(rows + (size_t)kpad * HD)[i] = ld_cg_v4(p.vc + base + (size_t)i * 8);
+    }
+    __syncthreads();
+    // one fill of kpad rows; no row is special (knew / vnew only stand in for
+    // rows past the item)
+    const AttnRows<HD> R{reinterpret_cast<const uint8_t*>(rows), 0u, 1, 0, kpad, n, -1, rows,
+                         rows + (size_t)kpad * HD};
+    auto bar = []() {
+        __syncthreads();
         return true;
     };
-    auto done = [](int) {};
-    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][AttnShape<HD>::DPL];
-    attn_item_serial<HD, false>(p, st, first, count, pos, Kpos, Vpos, sbuf, lane, rows, done, rm, rl, ro);
-    attn_store_partial<HD>(p, rm, rl, ro, b, g, j, lane);
+    if (p.n_parts == 1) {
+        float* out = p.attn + (size_t)b * p.Q + (size_t)g * G * HD;
+        attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, [](int) {},
+                            [&](int h, int d, float o, float, float l) { out[h * HD + d] = __fdiv_rn(o, l); });
+    } else {
+        attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, [](int) {}, [&](int h, int d, float o, float m, float l) {
+            const size_t hp = ((size_t)b * p.nq + (size_t)(g * G + h)) * p.n_parts + j;
+            p.part_o[hp * HD + d] = o;
+            if (d == 0) {
+                p.part_ml[hp * 2] = m;
+                p.part_ml[hp * 2 + 1] = l;
+            }
+        });
+    }
 }
 
 template <int HD>
@@ -146,16 +181,18 @@ static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
         const uint32_t w = units < warps_cap ? units : warps_cap;
         return (w + kBaseWarps - 1) / kBaseWarps;
     };
-    const size_t attn_smem = (size_t)kBaseWarps * kMaxGroup * p.keys_per_stage * sizeof(float);
+    const size_t attn_smem = attn_item_smem<HD>(p.group, attn_kpad(p.part_keys));
     k_validate<<<1, 32, 0, st>>>(p);
     const uint32_t tpg = (uint32_t)(p.group + 2) * (HD / 4);
     for (int l = 0; l < p.L; ++l) {
         const uint32_t nq = (uint32_t)p.nkv * tpg;
         k_tiles<MK_OP_QKV, KH, HD><<<blocks_for(nq), kBaseThreads, 0, st>>>(p, l, nq, p.tile_h);
         const uint32_t na = (uint32_t)(p.B * p.nkv * p.n_parts);
-        k_attn_partial<HD><<<(na + kBaseWarps - 1) / kBaseWarps, kBaseThreads, attn_smem, st>>>(p, l);
-        const uint32_t nm = (uint32_t)(p.B * p.nq);
-        k_attn_merge<HD><<<(nm + kBaseWarps - 1) / kBaseWarps, kBaseThreads, 0, st>>>(p);
+        k_attn_item<HD><<<na, kBaseThreads, attn_smem, st>>>(p, l);
+        if (p.n_parts > 1) {
+            const uint32_t nm = (uint32_t)(p.B * p.nq);
+            k_attn_merge<HD><<<(nm + kBaseWarps - 1) / kBaseWarps, kBaseThreads, 0, st>>>(p);
+        }
         const uint32_t no = (uint32_t)p.H / 4;
         k_tiles<MK_OP_OPROJ, KO, HD><<<blocks_for(no), kBaseThreads, 0, st>>>(p, l, no, p.tile_o);
         const uint32_t ng = (uint32_t)p.F / 2;
@@ -165,6 +202,19 @@ static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
     const uint32_t nl = (uint32_t)p.V / 4;
     k_tiles<MK_OP_LMHEAD, KH, HD><<<blocks_for(nl), kBaseThreads, 0, st>>>(p, 0, nl, p.tile_h);
     return cudaGetLastError();
+}
+
+// Shared memory of the attention kernel for the current schedule (set once per
+// schedule, outside any stream capture).
+cudaError_t baseline_prepare(const Params& p) {
+    const int kpad = attn_kpad(p.part_keys);
+    if (p.d == 64)
+        return cudaFuncSetAttribute(k_attn_item<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)attn_item_smem<64>(p.group, kpad));
+    if (p.d == 128)
+        return cudaFuncSetAttribute(k_attn_item<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)attn_item_smem<128>(p.group, kpad));
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t baseline_launch(const Params& p, cudaStream_t stream, int n_sm) {

@@ -14,6 +14,9 @@
 //    (cp.async.bulk, completion counted on an mbarrier, L2 evict-first). It
 //    never waits on a dependency counter, so the next instructions' weights
 //    arrive while the step still waits for their activations.
+//  * Warp 10 (the prefetch warp) pulls the fills that follow the ring's into L2
+//    (bulk prefetch, evict-last), a bounded distance ahead of the loader, so
+//    HBM keeps streaming while the ring is full and the SM waits on activations.
 //  * Warp 9 (the activation warp) runs ahead of the compute warps: for each job
 //    it waits for the job's input counter (acquire load, bounded spin), loads
 //    the small activation input from L2 and prepares it in one of a few
@@ -166,13 +169,31 @@ __device__ __forceinline__ void release_fill(const Ring& r, uint32_t seq, int la
 // Barrier of the 8 compute warps (an mbarrier of count 8; bounded, abort-aware,
 // so a warp that left on an error cannot leave the others waiting forever).
 // `uses` counts this warp's passes; all compute warps pass it in the same jobs.
+// The wait is a short spin on the non-blocking probe: the warps arrive within a
+// few hundred cycles of each other, and a sleeping waiter would add its wake-up
+// latency to every pass.
 __device__ __forceinline__ bool compute_barrier(const Params& p, uint64_t* cbar, uint32_t& uses,
                                                 int lane) {
     __syncwarp();
     if (lane == 0) mbar_arrive(cbar);
-    const bool ok = wait_bar(p, cbar, uses & 1u, nullptr, uses, 5, lane);
+    const uint32_t parity = uses & 1u;
     ++uses;
-    return ok;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0; !__all_sync(0xffffffffu, mbar_test_wait(cbar, parity)); ++it) {
+        if ((it & 1023u) == 1023u) {
+            int bad = 0;
+            if (lane == 0) {
+                if (t0 == 0) t0 = global_timer_ns();
+                if (aborted(p)) bad = 1;
+                else if (global_timer_ns() - t0 > p.timeout_ns) {
+                    record_error(p, MK_ERR_TIMEOUT, uses, 0xfffffff5u, 0, parity, 5);
+                    bad = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+        }
+    }
+    return true;
 }
 
 // ------------------------------------------------------------------ activation warp
@@ -275,26 +296,21 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             }
             return true;
         }
-        default: {  // attention items: q of the group's heads and the new key/value
-            const int items = (int)in.job_items;
-            for (int it = 0; it < items; ++it) {
-                const mk_instr& a = ins[it];
-                if (!wait_input(p, a.wait_ctr, target_of(epoch, a.wait_n), a.seq, lane, job)) return false;
-                uint8_t* region = slot + (size_t)it * p.attn_item_bytes;
-                const float* qsrc = p.q + (size_t)a.batch * p.Q + (size_t)a.group * p.group * HD;
-                float* qdst = reinterpret_cast<float*>(region);
-                for (int e = lane * 4; e < p.group * HD; e += 128)
-                    *reinterpret_cast<uint4*>(qdst + e) = ld_cg_v4(qsrc + e);
-                const int pos = g_pos[a.batch];
-                const size_t off = kv_off(p, l, a.batch, a.group, pos);
-                uint16_t* kv = reinterpret_cast<uint16_t*>(region + (size_t)p.group * HD * 4);
-                constexpr int kPieces = HD / 8;  // 16-byte pieces per row
-                if (lane < kPieces) {
-                    *reinterpret_cast<uint4*>(kv + lane * 8) = ld_cg_v4(p.kc + off + lane * 8);
-                } else if (lane < 2 * kPieces) {
-                    const int q = lane - kPieces;
-                    *reinterpret_cast<uint4*>(kv + HD + q * 8) = ld_cg_v4(p.vc + off + q * 8);
-                }
+        default: {  // attention item: q of the group's heads and the new key/value
+            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
+            const float* qsrc = p.q + (size_t)in.batch * p.Q + (size_t)in.group * p.group * HD;
+            float* qdst = reinterpret_cast<float*>(slot);
+            for (int e = lane * 4; e < p.group * HD; e += 128)
+                *reinterpret_cast<uint4*>(qdst + e) = ld_cg_v4(qsrc + e);
+            const int pos = g_pos[in.batch];
+            const size_t off = kv_off(p, l, in.batch, in.group, pos);
+            uint16_t* kv = reinterpret_cast<uint16_t*>(slot + (size_t)p.group * HD * 4);
+            constexpr int kPieces = HD / 8;  // 16-byte pieces per row
+            if (lane < kPieces) {
+                *reinterpret_cast<uint4*>(kv + lane * 8) = ld_cg_v4(p.kc + off + lane * 8);
+            } else if (lane < 2 * kPieces) {
+                const int q = lane - kPieces;
+                *reinterpret_cast<uint4*>(kv + HD + q * 8) = ld_cg_v4(p.vc + off + q * 8);
             }
             return true;
         }
@@ -308,7 +324,6 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
     for (int i = i0; i < i1;) {
         const mk_instr* ins = p.instrs + i;
         const uint32_t op = ins[0].op;
-        const int items = (op == MK_OP_ATTN) ? (int)ins[0].job_items : 1;
         const int njobs = (op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS, use = j / sl.NS;
@@ -325,7 +340,7 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
                 mbar_arrive(sl.full + s);  // release: the slot's contents
             }
         }
-        i += items;
+        ++i;
     }
 }
 
@@ -405,157 +420,79 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
     return true;
 }
 
-// The end of one attention item (sequence b, KV group g, one key partition) for
-// the group's heads h in [h_lo, h_hi), whose item partial (m, l, o) this warp
-// holds. With a single partition the partial is the output, o / l. Otherwise it
-// is stored, the heads' arrival is counted on the (b, g) arrival counter, and
-// the warp that completes the count merges all partitions of the group in
-// partition order. Either way each head of the pair is signalled once on the
-// attention counter, after its output is written.
+// One attention item as one job of all compute warps (see attn_item_block). Every
+// fill of the item must have landed first: each warp reads all of them. With a
+// single partition per (sequence, group) the item writes o / l for its heads;
+// otherwise it stores its partial, counts its heads on the pair's arrival
+// counter, and the item that completes the count merges the pair's partitions
+// in partition order. Either way the group's heads are signalled on the
+// attention counter once their output is written.
 template <int HD>
-__device__ __forceinline__ void attn_finish(const Params& p, const mk_instr& a, uint32_t epoch, int h_lo,
-                                            int h_hi, const float (&m)[kMaxGroup],
-                                            const float (&l)[kMaxGroup],
-                                            const float (&o)[kMaxGroup][AttnShape<HD>::DPL], int lane) {
-    if (a.signal_ctr == MK_NO_COUNTER) return;  // failure injection: the item never completes
-    const int b = a.batch, g = a.group, n = h_hi - h_lo;
-    const int part = (int)(a.first / (uint32_t)p.part_keys);
+__device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr& a, const uint8_t* slot,
+                                 float* sc, int warp, int lane, uint64_t* cbar, uint32_t& cuses,
+                                 uint32_t job, uint32_t epoch) {
+    const int G = p.group, b = a.batch, g = a.group;
+    const int pos = g_pos[b];
+    for (uint32_t f = 0; f < a.nfill; ++f)
+        if (!wait_fill(p, ring, a.seq + f, lane)) return false;
+    if (warp == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
+    const float* qs = reinterpret_cast<const float*>(slot);
+    const uint16_t* knew = reinterpret_cast<const uint16_t*>(slot + (size_t)G * HD * 4);
+    const int jn = pos - (int)a.first;
+    const AttnRows<HD> R{ring.base, ring.stage_bytes, (int)ring.S, (int)(a.seq % ring.S), p.keys_per_stage,
+                         min((int)a.count, jn + 1), (jn >= 0 && jn < (int)a.count) ? jn : -1, knew, knew + HD};
+    auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
+    // trace: warp 0 at the end of each phase and after each barrier
+    auto mark = [&](int k) {
+        if (warp == 0 && lane == 0) trace(p, job, kTrSub0 + k, global_timer_ns());
+    };
+    const int t = warp * 32 + lane;
     uint32_t* sig = p.counters + (size_t)a.signal_ctr * kCounterStride;
     if (p.n_parts == 1) {
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-            if (h >= h_lo && h < h_hi) attn_store_final_head<HD>(p, l[h], o[h], b, g * p.group + h, lane);
-        __syncwarp();
-        if (lane == 0) red_release_add(sig, (uint32_t)n);
-        return;
-    }
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h)
-        if (h >= h_lo && h < h_hi)
-            attn_store_partial_head<HD>(p, m[h], l[h], o[h], b, g * p.group + h, part, lane);
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-        const uint32_t target = (epoch + 1u) * (uint32_t)(p.n_parts * p.group);
-        const uint32_t old = atom_acq_rel_add(p.counters + (size_t)a.aux0 * kCounterStride, (uint32_t)n);
-        last = old + (uint32_t)n == target;
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    __syncwarp();
-    if (!last) return;
-    float* out = p.attn + (size_t)b * p.Q;
-    attn_merge_heads<HD, kMaxGroup>(p, b, g * p.group, 1, (g + 1) * p.group, lane,
-                                    [&](int e, float x) { out[e] = x; });
-    __syncwarp();
-    if (lane == 0) red_release_add(sig, (uint32_t)p.group);
-}
-
-// An attention job of `items` items. A lone item whose fills all fit in the
-// ring: its kSubRanges sub-ranges run on the 8 compute warps at once, the
-// sub-range partials meet in the slot, and warp h folds head h's in order.
-// Otherwise warp w runs item w's sub-ranges one after another.
-template <int HD>
-__device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr* ins, int items,
-                                 uint8_t* slot, float* scores, int warp, int lane, uint64_t* cbar,
-                                 uint32_t& cuses, uint32_t job, uint32_t epoch) {
-    using S = AttnShape<HD>;
-    const int kps = p.keys_per_stage;
-    if (items == 1 && ins[0].nfill <= ring.S) {
-        const mk_instr& a = ins[0];
-        const int pos = g_pos[a.batch];
-        const float* q = reinterpret_cast<const float*>(slot);
-        const uint16_t* knew = reinterpret_cast<const uint16_t*>(slot + (size_t)p.group * HD * 4);
-        const uint16_t* vnew = knew + HD;
-        AttnState<HD> st;
-        attn_init<HD, true>(p, q, st, lane);
-        int lo, hi;
-        sub_range(a.first, a.count, warp, &lo, &hi);
-        auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
-            if (!wait_fill(p, ring, a.seq + f, lane)) return false;
-            K = reinterpret_cast<const uint16_t*>(ring.stage(a.seq + f));
-            V = K + (size_t)kps * HD;
-            return true;
-        };
-        const bool ok = attn_sub<HD, true>(p, st, a.first, lo, hi, pos, knew, vnew, scores, lane, rows,
-                                           [](int) {});
-        constexpr int kSubFloats = 2 * kMaxGroup + kMaxGroup * HD;
-        float* subs = reinterpret_cast<float*>(slot + p.attn_item_bytes);
-        float* mine = subs + (size_t)warp * kSubFloats;
-        if (lane == 0)
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                mine[h] = st.m[h];
-                mine[kMaxGroup + h] = st.l[h];
-            }
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-            for (int d = 0; d < S::DPL; ++d) mine[2 * kMaxGroup + h * HD + lane * S::DPL + d] = st.o[h][d];
-        if (!compute_barrier(p, cbar, cuses, lane) || !ok) return false;
-        if (warp == kConsumerWarps - 1 && lane == 0)  // every warp is done with the fills
-            for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
-        if (warp < p.group) {
-            // head `warp`: the kSubRanges partials folded in order
-            const int h = warp;
-            float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
-#pragma unroll
-            for (int x = 0; x < kMaxGroup; ++x) {
-                rm[x] = -INFINITY;
-                rl[x] = 0.f;
-#pragma unroll
-                for (int d = 0; d < S::DPL; ++d) ro[x][d] = 0.f;
-            }
-            float M = subs[h], Lh = subs[kMaxGroup + h], O[S::DPL];
-#pragma unroll
-            for (int d = 0; d < S::DPL; ++d) O[d] = subs[2 * kMaxGroup + h * HD + lane * S::DPL + d];
-            for (int u = 1; u < kSubRanges; ++u) {
-                const float* su = subs + (size_t)u * kSubFloats;
-                const float bm = su[h], bl = su[kMaxGroup + h];
-                float bo[S::DPL];
-#pragma unroll
-                for (int d = 0; d < S::DPL; ++d) bo[d] = su[2 * kMaxGroup + h * HD + lane * S::DPL + d];
-                fold_one<HD>(M, Lh, O, bm, bl, bo);
-            }
-            // scatter into the per-head arrays attn_finish takes (only head h is used)
-#pragma unroll
-            for (int x = 0; x < kMaxGroup; ++x)
-                if (x == h) {
-                    rm[x] = M;
-                    rl[x] = Lh;
-#pragma unroll
-                    for (int d = 0; d < S::DPL; ++d) ro[x][d] = O[d];
+        float* out = p.attn + (size_t)b * p.Q + (size_t)g * G * HD;
+        if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark,
+                                 [&](int h, int d, float o, float, float l) { out[h * HD + d] = __fdiv_rn(o, l); }))
+            return false;
+    } else {
+        const int part = (int)(a.first / (uint32_t)p.part_keys);
+        if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark, [&](int h, int d, float o, float m, float l) {
+                const size_t hp = ((size_t)b * p.nq + (size_t)(g * G + h)) * p.n_parts + part;
+                p.part_o[hp * HD + d] = o;
+                if (d == 0) {
+                    p.part_ml[hp * 2] = m;
+                    p.part_ml[hp * 2 + 1] = l;
                 }
-            attn_finish<HD>(p, a, epoch, h, h + 1, rm, rl, ro, lane);
+            }))
+            return false;
+    }
+    // every warp has passed the barrier after its last read of the fills
+    if (warp == kConsumerWarps - 1 && lane == 0)
+        for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+    if (!bar()) return false;  // every output of the item is stored
+    if (p.n_parts == 1) {
+        if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_release_add(sig, (uint32_t)G);
+        mark(6);
+        return true;
+    }
+    uint32_t* flag = reinterpret_cast<uint32_t*>(sc + kAttnFlagFloat);
+    if (t == 0) {
+        uint32_t last = 0;
+        if (a.signal_ctr != MK_NO_COUNTER) {  // a dropped item (failure injection) never arrives
+            const uint32_t target = (epoch + 1u) * (uint32_t)(p.n_parts * G);
+            const uint32_t old = atom_acq_rel_add(p.counters + (size_t)a.aux0 * kCounterStride, (uint32_t)G);
+            last = old + (uint32_t)G == target;
         }
-        return true;
+        *flag = last;
     }
-    if (warp >= items) return true;
-    const mk_instr& a = ins[warp];
-    const uint8_t* region = slot + (size_t)warp * p.attn_item_bytes;
-    const int pos = g_pos[a.batch];
-    const float* q = reinterpret_cast<const float*>(region);
-    const uint16_t* knew = reinterpret_cast<const uint16_t*>(region + (size_t)p.group * HD * 4);
-    const uint16_t* vnew = knew + HD;
-    AttnState<HD> st;
-    attn_init<HD, true>(p, q, st, lane);
-    uint32_t released = 0;  // fills [0, released) handed back to the loader
-    auto rows = [&](int f, const uint16_t*& K, const uint16_t*& V) {
-        for (; released < (uint32_t)f; ++released) release_fill(ring, a.seq + released, lane);
-        if (!wait_fill(p, ring, a.seq + f, lane)) return false;
-        K = reinterpret_cast<const uint16_t*>(ring.stage(a.seq + f));
-        V = K + (size_t)kps * HD;
-        return true;
-    };
-    float rm[kMaxGroup], rl[kMaxGroup], ro[kMaxGroup][S::DPL];
-    if (!attn_item_serial<HD, true>(p, st, a.first, a.count, pos, knew, vnew, scores, lane, rows,
-                                    [](int) {}, rm, rl, ro))
-        return false;
-    for (; released < a.nfill; ++released) {
-        // fills never read (keys past pos) still have to land before they are handed back
-        if (!wait_fill(p, ring, a.seq + released, lane)) return false;
-        release_fill(ring, a.seq + released, lane);
+    if (!bar()) return false;
+    if (*reinterpret_cast<volatile uint32_t*>(flag) == 0u) return true;
+    if (warp < G) {
+        float* out = p.attn + (size_t)b * p.Q;
+        const int head = g * G + warp;
+        attn_merge_heads<HD, 1>(p, b, head, 1, head + 1, lane, [&](int e, float x) { out[e] = x; });
     }
-    attn_finish<HD>(p, a, epoch, 0, p.group, rm, rl, ro, lane);
+    if (!bar()) return false;
+    if (t == 0) red_release_add(sig, (uint32_t)G);
     return true;
 }
 
@@ -566,7 +503,6 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
     uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
-        const int items = (in.op == MK_OP_ATTN) ? (int)in.job_items : 1;
         const int njobs = (in.op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS;
@@ -581,8 +517,8 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j); break;
                 case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j); break;
                 default:
-                    ok = compute_attn_job<HD>(p, ring, p.instrs + i, items, sl.slot(j), scores, warp,
-                                              lane, cbar, cuses, j, epoch);
+                    ok = compute_attn_job<HD>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
+                                              epoch);
                     break;
             }
             if (!ok) return;
@@ -595,15 +531,21 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
                     trace(p, j, kTrDone, global_timer_ns());
-                    // attention items signal their heads themselves (attn_finish)
+                    // attention items signal their heads themselves (compute_attn_job)
                     const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN;
-                    if (last_chunk && in.signal_ctr != MK_NO_COUNTER)
-                        red_release_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
+                    if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
+                        // QKV / gate-up: one increment on each KV group / MLP chunk counter
+                        // the job's tiles touched
+                        const uint32_t span =
+                            (in.op == MK_OP_QKV || in.op == MK_OP_GATEUP) && in.aux1 > 1 ? in.aux1 : 1u;
+                        for (uint32_t k = 0; k < span; ++k)
+                            red_release_add(p.counters + (size_t)(in.signal_ctr + k) * kCounterStride, 1u);
+                    }
                 }
                 mbar_arrive(sl.empty + s);
             }
         }
-        i += items;
+        ++i;
     }
 }
 
@@ -645,52 +587,22 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
     }
 }
 
-// One thread streams the SM's fills into the ring. While the ring is full of
-// landed fills the compute warps are waiting on activations; a second cursor
-// then pulls the next fills (up to `l2_prefetch_fills` ahead) into L2, so HBM
-// keeps streaming and the ring copies that follow hit L2.
-__device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
+// One thread streams the SM's fills into the ring, in list order; it never
+// waits on a dependency counter, only for the compute warps to release a stage.
+// `issued_out` publishes how many fills it has issued (for the prefetch warp).
+__device__ void loader(const Params& p, const Ring& ring, int i0, int i1, volatile uint32_t* issued_out) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
-    int pf_i = i0;
-    uint32_t pf_t = 0, pf_seq = 0;
-    const uint64_t pf_pol = p.l2_prefetch_evict_last ? l2_evict_last_policy() : l2_evict_normal_policy();
     for (int i = i0; i < i1; ++i) {
         const mk_instr in = p.instrs[i];
         for (uint32_t t = 0; t < in.nfill; ++t) {
             const uint32_t seq = in.seq + t;
             const uint32_t s = seq % ring.S, use = seq / ring.S;
             if (use > 0) {
-                // Wait for the compute warps to release the previous fill of this
-                // stage. If that fill has already landed, the compute warps are the
-                // ones waiting (on activations) and HBM would idle: meanwhile pull
-                // the next fills into L2, up to l2_prefetch_fills ahead.
+                // wait for the compute warps to release the previous fill of this stage
                 uint64_t t0 = 0;
                 bool ok = true;
-                if (pf_seq < seq) {  // the cursor never trails the ring
-                    while (pf_i < i1 && pf_seq < seq) {
-                        const uint32_t nf = p.instrs[pf_i].nfill;
-                        const uint32_t step = min(nf - pf_t, seq - pf_seq);
-                        pf_t += step;
-                        pf_seq += step;
-                        if (pf_t >= nf) { ++pf_i; pf_t = 0; }
-                    }
-                }
                 for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, 500u); ++it) {
-                    for (int k = 0; k < 2; ++k) {  // up to two prefetches per wake-up
-                        if (!(p.l2_prefetch_fills > 0 && pf_i < i1 &&
-                              pf_seq < seq + (uint32_t)p.l2_prefetch_fills &&
-                              mbar_try_wait(ring.full + s, (use - 1) & 1u)))
-                            break;
-                        const mk_instr pin = p.instrs[pf_i];
-                        const FillSrc f = fill_source(p, pin, pf_t);
-                        if (f.bytes) {
-                            prefetch_l2(f.a, f.bytes, pf_pol);
-                            if (f.b) prefetch_l2(f.b, f.bytes, pf_pol);
-                        }
-                        ++pf_seq;
-                        if (++pf_t >= pin.nfill) { ++pf_i; pf_t = 0; }
-                    }
                     if ((it & 15u) == 15u) {
                         if (t0 == 0) t0 = global_timer_ns();
                         if (aborted(p)) { ok = false; break; }
@@ -737,9 +649,11 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
                 }
             }
             issued = seq + 1;
+            *issued_out = issued;
         }
     }
 drain:
+    *issued_out = 0xffffffffu;  // the prefetch warp stops at once
     // Every copy issued must land before the CTA may exit: wait for the last
     // fill of each stage used (earlier fills of a stage completed before it
     // could be refilled).
@@ -756,15 +670,54 @@ drain:
     }
 }
 
+// One thread keeps HBM busy while the compute warps wait on activations: it
+// pulls the SM's next fills into L2 (bulk prefetch, evict-last by default),
+// at most `l2_prefetch_fills` fills ahead of the loader's next one. When the
+// ring is full of landed fills the loader stops, but the prefetches go on, so
+// the weights the SM needs after the wait are in L2 and the ring refills from
+// there. Fills the loader issues at launch (the first ring's worth) and fills it
+// has already issued are skipped. Every wait is bounded.
+__device__ void prefetcher(const Params& p, int i0, int i1, uint32_t S, const volatile uint32_t* issued) {
+    const uint32_t D = (uint32_t)p.l2_prefetch_fills;
+    if (D == 0) return;
+    const uint64_t pol = p.l2_prefetch_policy == 1 ? l2_evict_normal_policy() : l2_evict_last_policy();
+    uint32_t pf = 0;  // fill number
+    uint64_t t0 = 0;
+    for (int i = i0; i < i1; ++i) {
+        const mk_instr in = p.instrs[i];
+        for (uint32_t t = 0; t < in.nfill; ++t, ++pf) {
+            if (pf < S) continue;
+            uint32_t iss = *issued;
+            for (uint32_t it = 0; pf >= iss + D; ++it) {
+                __nanosleep(128);
+                iss = *issued;
+                if ((it & 63u) == 63u) {
+                    if (aborted(p)) return;
+                    if (t0 == 0) t0 = global_timer_ns();
+                    else if (global_timer_ns() - t0 > p.timeout_ns) return;
+                }
+            }
+            t0 = 0;
+            if (iss == 0xffffffffu) return;  // the loader has stopped
+            if (pf < iss) continue;           // already on its way to the ring
+            const FillSrc f = fill_source(p, in, t);
+            if (f.bytes) {
+                prefetch_l2(f.a, f.bytes, pol);
+                if (f.b) prefetch_l2(f.b, f.bytes, pol);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ the kernel
 
 template <int KH, int KO, int KF, int HD>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
+    __shared__ volatile uint32_t s_issued;  // fills the loader has issued (all: ~0)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes,
-                                     p.keys_per_stage);
+    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes);
     Ring ring;
     ring.base = smem + m.ring;
     ring.full = reinterpret_cast<uint64_t*>(smem + m.full);
@@ -792,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             sl.done[s] = 0;
         }
         mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
+        s_issued = 0u;
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
         uint32_t skip = ld_volatile_u32(&p.ctl->status) != 0u;
@@ -816,12 +770,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (!s_skip) {
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
         if (warp == kLoaderWarp) {
-            if (lane == 0) loader(p, ring, i0, i1);
+            if (lane == 0) loader(p, ring, i0, i1, &s_issued);
+        } else if (warp == kPrefetchWarp) {
+            if (lane == 0) prefetcher(p, i0, i1, ring.S, &s_issued);
         } else if (warp == kPrepWarp) {
             activation_warp<KH, KO, KF, HD>(p, sl, i0, i1, lane, s_epoch);
         } else {
-            float* scores = reinterpret_cast<float*>(smem + m.scores) +
-                            (size_t)warp * kMaxGroupHeads * p.keys_per_stage;
+            float* scores = reinterpret_cast<float*>(smem + m.scores);
             compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
                                          reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
                                          s_epoch);
@@ -849,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ------------------------------------------------------------------ host-side launch
 
 size_t megakernel_smem_bytes(const Params& p) {
-    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, p.keys_per_stage).total;
+    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes).total;
 }
 
 using KernelFn = void (*)(Params);

@@ -59,6 +59,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of phase `parity` (acquire at CTA scope when it has completed).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Same, but the thread sleeps (up to `ns` nanoseconds) until the phase
 // completes instead of returning at once: waiting warps then leave their
 // scheduler's issue slots to the warps that work.
@@ -526,319 +539,265 @@ __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uin
 }
 
 // ------------------------------------------------------------------ decode attention
+//
+// One attention item is one (sequence b, KV group g, key range [first,
+// first + count)) of the split-K decode attention, restricted to keys <= pos
+// (the key at pos is the one this step writes). The whole item runs on the
+// compute warps of one CTA (256 threads) in three phases with a CTA barrier
+// after each. The item is small (at most a few hundred keys), so its time is
+// latency: each phase works on batches of independent keys without divergent
+// branches (out-of-range keys read a valid row and are masked), so that the
+// keys' dependent chains overlap, and rows are addressed incrementally.
+//
+//  1. scores: 8 lanes per key (8 dims each; the group's query heads held in
+//     registers), four keys per warp pass, four passes per batch. The partial
+//     dot products meet in a reduce-scatter butterfly that leaves head
+//     2*b2 + b1 on the lanes with lane bits (b2, b1), as
+//     s_h(j) = (q_h . k_j) * (1/sqrt(HD)). Each warp reduces its keys' maximum
+//     per head. (head_dim 128: 16 lanes per key, bit 3 folded first.)
+//  2. weights, one thread per key: M_h = max of the warps' maxima,
+//     e_h(j) = exp(s_h(j) - M_h), stored as a float4 per key (heads >= G: 0);
+//     each warp reduces its keys' sum per head.
+//  3. values: thread (kq, dp) adds e_h(j) * v_j[2 dp], v_j[2 dp + 1] for all
+//     heads over the keys j = kq (mod KQ) in increasing j, four per batch.
+// Then each output (h, d) is the KQ class sums added in class order, and l_h
+// the warps' sums added in warp order. With one partition per (sequence, group)
+// the output is o_h / l_h; otherwise (M_h, l_h, o_h) is the partition's
+// partial, merged in partition order. The megakernel and the multi-kernel
+// baseline run this same code on the same rows, so their results are identical.
 
-// Lane layout for the scores: LPK lanes share one key (8 dims each); KPI keys per
-// warp-wide step. For the value sum each lane owns DPL consecutive dims.
+// DPL: dims per lane in the partial merge; LPK lanes per key in the scores;
+// KQ key classes in the values.
 template <int HD>
 struct AttnShape {
-    static constexpr int LPK = HD / 8;
-    static constexpr int KPI = 32 / LPK;
     static constexpr int DPL = HD / 32;
+    static constexpr int LPK = HD / 8;
+    static constexpr int KPW = 32 / LPK;                         // keys per warp pass
+    static constexpr int KQ = 32 * kConsumerWarps / (HD / 2);
 };
 
-constexpr int kMaxGroup = 4;  // query heads per KV head handled by one instruction
+constexpr int kMaxGroup = kMaxGroupHeads;  // query heads per KV head handled by one item
 
+// Offsets inside an item's scratch (kAttnScratchFloats floats of shared memory).
+constexpr uint32_t kAttnE = 0;                                       // [kMaxItemKeys][4]
+constexpr uint32_t kAttnWMax = kAttnE + 4 * kMaxItemKeys;            // [warps][4]
+constexpr uint32_t kAttnWSum = kAttnWMax + 4 * kConsumerWarps;       // [warps][4]
+constexpr uint32_t kAttnPart = kAttnWSum + 4 * kConsumerWarps;       // [KQ][4][HD]
+constexpr uint32_t kAttnFlagFloat = kAttnPart + 2 * 32 * kConsumerWarps * 4;
+static_assert(kAttnFlagFloat + 4 <= kAttnScratchFloats, "attention scratch");
+
+// The rows of an item in shared memory (knew and vnew always point at a valid
+// row: they also stand in for rows past the item, whose results are masked). Row j (0 <= j < n) is key first + j. The
+// rows sit in fills of kps rows: fill f is stage (s0 + f) mod S of a ring of S
+// stages of `stage_bytes` at `base`, K rows first, V rows kps rows further on.
+// Row jnew = n - 1, when the item holds the key at pos, is the exception: its
+// key and value come from knew / vnew. n counts the item's keys at or before pos
+// (<= 0: none).
 template <int HD>
-struct AttnState {
-    float q[kMaxGroup][8];                        // this lane's 8 query dims, per head
-    float m[kMaxGroup], l[kMaxGroup];             // running max and sum
-    float o[kMaxGroup][AttnShape<HD>::DPL];       // running unnormalised output
+struct AttnRows {
+    const uint8_t* base;
+    uint32_t stage_bytes;
+    int S, s0, kps;
+    int n;
+    int jnew;  // n - 1 or -1
+    const uint16_t* knew;
+    const uint16_t* vnew;
 };
 
-// q for the group's heads: 8 dims per lane from qh (fp32 [group][HD]), read from
-// shared memory (SMEM) or global memory.
-template <int HD, bool SMEM>
-__device__ __forceinline__ void attn_init(const Params& p, const float* qg, AttnState<HD>& st,
-                                          int lane) {
-    using S = AttnShape<HD>;
-    const int dc = lane % S::LPK;
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h < p.group) {
-            const float* qh = qg + (size_t)h * HD + dc * 8;
-            uint4 a, c;
-            if (SMEM) {
-                a = lds_v4(qh);
-                c = lds_v4(qh + 4);
-            } else {
-                a = ld_cg_v4(qh);
-                c = ld_cg_v4(qh + 4);
-            }
-            st.q[h][0] = __uint_as_float(a.x); st.q[h][1] = __uint_as_float(a.y);
-            st.q[h][2] = __uint_as_float(a.z); st.q[h][3] = __uint_as_float(a.w);
-            st.q[h][4] = __uint_as_float(c.x); st.q[h][5] = __uint_as_float(c.y);
-            st.q[h][6] = __uint_as_float(c.z); st.q[h][7] = __uint_as_float(c.w);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) st.q[h][e] = 0.f;
-        }
-        st.m[h] = -INFINITY;
-        st.l[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < S::DPL; ++e) st.o[h][e] = 0.f;
-    }
+// Branch-free address of row j < R.n of the fills (key rows; V rows are kps
+// rows further on): fill f = j / kps by a multiply-high with m = 2^32 / kps
+// rounded up (exact for the few thousand rows an item can have), stage
+// (s0 + f) mod S by one conditional subtraction (f < S).
+template <int HD>
+__device__ __forceinline__ const uint16_t* attn_row(const AttnRows<HD>& R, uint32_t m, int j) {
+    const int f = (int)__umulhi((uint32_t)j, m);
+    const int r = j - f * R.kps;
+    int s = R.s0 + f;
+    s = s >= R.S ? s - R.S : s;
+    return reinterpret_cast<const uint16_t*>(R.base + (size_t)s * R.stage_bytes) + (size_t)r * HD;
 }
 
-// One chunk of keys [ka, kend) (kend <= pos + 1, ka < kend). Rows of keys < pos
-// come from Kc/Vc (row 0 = key ka); the key at `pos`, written earlier in this
-// step, from Kpos/Vpos. All four are bf16 rows in shared memory when SMEM, else
-// in global memory. `s` is this warp's score scratch in shared memory,
-// [kMaxGroup][ks] floats. Independent passes are unrolled and the heads'
-// reductions interleaved, so the chunk's latency is a few dependent steps.
-template <int HD, bool SMEM>
-__device__ __forceinline__ void attn_chunk(const Params& p, AttnState<HD>& st, const uint16_t* Kc,
-                                           const uint16_t* Vc, const uint16_t* Kpos,
-                                           const uint16_t* Vpos, int ka, int kend, int pos,
-                                           float* s, int ks, int lane) {
+// The item on all compute warps (warp < kConsumerWarps). qs: the group's G query
+// heads, fp32 [G][HD], in shared memory; sc: kAttnScratchFloats of shared
+// memory; bar(): barrier of the compute warps (false: give up); mark(k): trace
+// hook. R.jnew must be -1 or n - 1. On success emit(h, d, o, M_h, l_h) runs once
+// for every output dim d < HD of every head h < G, on the thread that holds it.
+template <int HD, class Bar, class Mark, class Emit>
+__device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const float* qs, int G, float* sc,
+                                                int warp, int lane, Bar&& bar, Mark&& mark, Emit&& emit) {
     using S = AttnShape<HD>;
-    const int n = kend - ka;
-    const int dc = lane % S::LPK, kk = lane / S::LPK;
+    constexpr int NT = 32 * kConsumerWarps;
+    constexpr int KQ = S::KQ;
+    constexpr int PB = 4;  // warp passes / value keys per batch
+    float4* et = reinterpret_cast<float4*>(sc + kAttnE);
+    float4* wmax = reinterpret_cast<float4*>(sc + kAttnWMax);
+    float4* wsum = reinterpret_cast<float4*>(sc + kAttnWSum);
+    float* part = sc + kAttnPart;
+    const int n = R.n, t = warp * 32 + lane;
+    const int nc = R.jnew >= 0 ? n - 1 : n;  // rows read from the fills
     const float scale = 1.0f / sqrtf((float)HD);
-    // scores: S::KPI keys per pass, LPK lanes per key
-#pragma unroll 2
-    for (int base = 0; base < n; base += S::KPI) {
-        const int j = base + kk;
-        float part[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) part[h] = 0.f;
-        if (j < n) {
-            const int key = ka + j;
-            const uint16_t* kr = (key < pos ? Kc + (size_t)j * HD : Kpos) + dc * 8;
-            const uint4 raw = SMEM ? lds_v4(kr) : ld_cg_v4(kr);
-            float kv[8];
-            unpack8(raw, kv);
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) part[h] = fmaf(st.q[h][e], kv[e], part[h]);
-        }
-#pragma unroll
-        for (int m = S::LPK / 2; m > 0; m >>= 1)
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], m);
-        if (j < n && dc < p.group) {
-            float mine = 0.f;
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-                if (dc == h) mine = part[h];
-            s[dc * ks + j] = mine * scale;
-        }
-    }
-    __syncwarp();
-    // online softmax update, all heads together
-    float cm[kMaxGroup], cs[kMaxGroup], m_new[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) cm[h] = -INFINITY;
-    for (int j = lane; j < n; j += 32)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-            if (h < p.group) cm[h] = fmaxf(cm[h], s[h * ks + j]);
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) cm[h] = fmaxf(cm[h], __shfl_xor_sync(0xffffffffu, cm[h], m));
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        m_new[h] = fmaxf(st.m[h], cm[h]);
-        cs[h] = 0.f;
-    }
-    for (int j = lane; j < n; j += 32)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-            if (h < p.group) {
-                const float e = expf(s[h * ks + j] - m_new[h]);
-                s[h * ks + j] = e;
-                cs[h] += e;
-            }
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) cs[h] += __shfl_xor_sync(0xffffffffu, cs[h], m);
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= p.group) continue;
-        const float alpha = expf(st.m[h] - m_new[h]);   // 0 on the first chunk (m = -inf)
-        st.l[h] = fmaf(st.l[h], alpha, cs[h]);
-#pragma unroll
-        for (int e = 0; e < S::DPL; ++e) st.o[h][e] *= alpha;
-        st.m[h] = m_new[h];
-    }
-    __syncwarp();
-    // values: keys in order, unrolled so the loads of several keys are in flight
-#pragma unroll 2
-    for (int j = 0; j < n; ++j) {
-        const int key = ka + j;
-        float v[S::DPL];
-        const uint16_t* vr = (key < pos ? Vc + (size_t)j * HD : Vpos) + lane * S::DPL;
-        if constexpr (S::DPL == 2) {
-            const uint32_t w = SMEM ? *reinterpret_cast<const uint32_t*>(vr) : ld_cg_u32(vr);
-            v[0] = bf_lo(w);
-            v[1] = bf_hi(w);
-        } else {
-            static_assert(S::DPL == 4, "head_dim 64 or 128");
-            const uint2 w = SMEM ? *reinterpret_cast<const uint2*>(vr) : ld_cg_v2(vr);
-            v[0] = bf_lo(w.x);
-            v[1] = bf_hi(w.x);
-            v[2] = bf_lo(w.y);
-            v[3] = bf_hi(w.y);
-        }
+    // 1. scores
+    {
+        const int dc = lane % S::LPK, kk = lane / S::LPK;
+        float q[kMaxGroup][8];
 #pragma unroll
         for (int h = 0; h < kMaxGroup; ++h) {
-            if (h >= p.group) continue;
-            const float e = s[h * ks + j];
+            if (h < G) {
+                const float4 a = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8);
+                const float4 c = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8 + 4);
+                q[h][0] = a.x; q[h][1] = a.y; q[h][2] = a.z; q[h][3] = a.w;
+                q[h][4] = c.x; q[h][5] = c.y; q[h][6] = c.z; q[h][7] = c.w;
+            } else {
 #pragma unroll
-            for (int d = 0; d < S::DPL; ++d) st.o[h][d] = fmaf(e, v[d], st.o[h][d]);
+                for (int e = 0; e < 8; ++e) q[h][e] = 0.f;
+            }
         }
+        const int hh = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);  // head this lane ends up with
+        const bool writer = (lane & (S::LPK == 8 ? 1 : 9)) == 0;
+        constexpr int KPR = S::KPW * kConsumerWarps;  // keys per pass over all warps
+        const int j_first = warp * S::KPW + kk;
+        const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
+        float mx = -INFINITY;
+        for (int j0 = j_first; j0 - kk < n; j0 += PB * KPR) {
+            float acc[PB][kMaxGroup];
+            float kv[PB][8];
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const int j = j0 + i * KPR;
+                // rows past the fills read the new key (a valid stand-in; masked below)
+                const uint16_t* kr = j < nc ? attn_row<HD>(R, m, j) : R.knew;
+                unpack8(lds_v4(kr + dc * 8), kv[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < PB; ++i)
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h) {
+                    acc[i][h] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[i][h] = fmaf(q[h][e], kv[i][e], acc[i][h]);
+                }
+            if (S::LPK == 16) {
+#pragma unroll
+                for (int i = 0; i < PB; ++i)
+#pragma unroll
+                    for (int h = 0; h < kMaxGroup; ++h) acc[i][h] += __shfl_xor_sync(0xffffffffu, acc[i][h], 8);
+            }
+            const bool b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const float k0 = b2 ? acc[i][2] : acc[i][0], k1 = b2 ? acc[i][3] : acc[i][1];
+                const float s0 = b2 ? acc[i][0] : acc[i][2], s1 = b2 ? acc[i][1] : acc[i][3];
+                const float m0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 4);
+                const float m1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 4);
+                const float kp = b1 ? m1 : m0, sp = b1 ? m0 : m1;
+                const float v = kp + __shfl_xor_sync(0xffffffffu, sp, 2);
+                acc[i][0] = v + __shfl_xor_sync(0xffffffffu, v, 1);
+            }
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const int j = j0 + i * KPR;
+                const float s = __fmul_rn(acc[i][0], scale);
+                if (j < n && hh < G) {
+                    mx = fmaxf(mx, s);
+                    if (writer) sc[kAttnE + 4 * j + hh] = s;
+                }
+            }
+        }
+        // the warp's maximum per head: lanes holding the same head differ in bits 0, 3, 4
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (lane < 8 && (lane & 1) == 0) sc[kAttnWMax + 4 * warp + hh] = hh < G ? mx : -INFINITY;
     }
-    __syncwarp();
-}
-
-// ------------------------------------------------------------------ attention items
-//
-// An item is one (sequence, KV group, key range [first, first+count)) of the
-// split-K attention. Its keys are cut into kSubRanges contiguous sub-ranges of
-// ceil(count / kSubRanges) keys; each sub-range gets its own online-softmax
-// partial (chunks cut at ring-stage boundaries, keys_per_stage apart from
-// `first`), and the item's partial is the ordered combination of the
-// sub-range partials, sub-range 0 first. Whether the sub-ranges run in
-// parallel on several warps or one after another on one warp, every value is
-// computed the same way.
-constexpr int kSubRanges = kSubRangeCount;
-
-__device__ __forceinline__ void sub_range(uint32_t first, uint32_t count, int u, int* lo, int* hi) {
-    const int sub = (int)((count + kSubRanges - 1) / kSubRanges);
-    *lo = (int)first + min(u * sub, (int)count);
-    *hi = (int)first + min((u + 1) * sub, (int)count);
-}
-
-// Fold one head's partial (bm, bl, bo) into the running (M, L, O): rescale both
-// to the larger max; an empty partial (m = -inf) leaves the other unchanged.
-template <int HD>
-__device__ __forceinline__ void fold_one(float& M, float& L, float (&O)[AttnShape<HD>::DPL], float bm,
-                                         float bl, const float (&bo)[AttnShape<HD>::DPL]) {
-    if (bm == -INFINITY) return;
-    if (M == -INFINITY) {
-        M = bm;
-        L = bl;
+    mark(0);
+    if (!bar()) return false;
+    mark(1);
+    // 2. weights
+    float M[kMaxGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int d = 0; d < AttnShape<HD>::DPL; ++d) O[d] = bo[d];
-        return;
+    for (int w = 0; w < kConsumerWarps; ++w) {
+        const float4 v = wmax[w];
+        M[0] = fmaxf(M[0], v.x);
+        M[1] = fmaxf(M[1], v.y);
+        M[2] = fmaxf(M[2], v.z);
+        M[3] = fmaxf(M[3], v.w);
     }
-    const float Mn = fmaxf(M, bm);
-    const float wa = expf(M - Mn), wb = expf(bm - Mn);
-    L = fmaf(L, wa, bl * wb);
-#pragma unroll
-    for (int d = 0; d < AttnShape<HD>::DPL; ++d) O[d] = fmaf(O[d], wa, bo[d] * wb);
-    M = Mn;
-}
-
-// Fold partial `b` into the running partial `a` (a = a (+) b) for every head:
-// rescale both to the larger max. Empty partials (m = -inf) leave the other
-// unchanged.
-template <int HD>
-__device__ __forceinline__ void fold_partial(float (&am)[kMaxGroup], float (&al)[kMaxGroup],
-                                             float (&ao)[kMaxGroup][AttnShape<HD>::DPL],
-                                             const float (&bm)[kMaxGroup], const float (&bl)[kMaxGroup],
-                                             const float (&bo)[kMaxGroup][AttnShape<HD>::DPL]) {
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) fold_one<HD>(am[h], al[h], ao[h], bm[h], bl[h], bo[h]);
-}
-
-// One sub-range [lo, hi) of an item, keys < pos + 1 only. `rows(f, K, V)` gives
-// the bf16 K/V rows of the item's fill f (row 0 = key first + f*kps) and may wait
-// for it; `done(f)` is called once the warp no longer needs fill f.
-template <int HD, bool SMEM, class Rows, class Done>
-__device__ __forceinline__ bool attn_sub(const Params& p, AttnState<HD>& st, uint32_t first, int lo,
-                                         int hi, int pos, const uint16_t* Kpos, const uint16_t* Vpos,
-                                         float* s, int lane, Rows&& rows, Done&& done) {
-    using S = AttnShape<HD>;
-    const int kps = p.keys_per_stage;
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        st.m[h] = -INFINITY;
-        st.l[h] = 0.f;
-#pragma unroll
-        for (int d = 0; d < S::DPL; ++d) st.o[h][d] = 0.f;
-    }
-    hi = min(hi, pos + 1);
-    if (lo >= hi) return true;
-    const int f0 = (lo - (int)first) / kps, f1 = (hi - 1 - (int)first) / kps;
-    for (int f = f0; f <= f1; ++f) {
-        const int fa = (int)first + f * kps;
-        const uint16_t *K, *V;
-        if (!rows(f, K, V)) return false;
-        const int ka = max(lo, fa), kb = min(hi, fa + kps);
-        attn_chunk<HD, SMEM>(p, st, K + (size_t)(ka - fa) * HD, V + (size_t)(ka - fa) * HD, Kpos, Vpos,
-                             ka, kb, pos, s, kps, lane);
-        done(f);
-    }
-    return true;
-}
-
-// Write one head's partial (m, l, o) of partition `part`.
-template <int HD>
-__device__ __forceinline__ void attn_store_partial_head(const Params& p, float m, float l,
-                                                        const float (&o)[AttnShape<HD>::DPL], int b,
-                                                        int head, int part, int lane) {
-    using S = AttnShape<HD>;
-    const size_t hp = ((size_t)b * p.nq + (size_t)head) * p.n_parts + part;
-    if (lane == 0) {
-        p.part_ml[hp * 2] = m;
-        p.part_ml[hp * 2 + 1] = l;
-    }
-#pragma unroll
-    for (int d = 0; d < S::DPL; ++d) p.part_o[hp * HD + lane * S::DPL + d] = o[d];
-}
-
-// Write an item's (m, l, o) for the group's heads.
-template <int HD>
-__device__ __forceinline__ void attn_store_partial(const Params& p, const float (&m)[kMaxGroup],
-                                                   const float (&l)[kMaxGroup],
-                                                   const float (&o)[kMaxGroup][AttnShape<HD>::DPL],
-                                                   int b, int g, int part, int lane) {
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h)
-        if (h < p.group) attn_store_partial_head<HD>(p, m[h], l[h], o[h], b, g * p.group + h, part, lane);
-}
-
-// The attention output of one head from a partial that covers all its keys:
-// o / l, the same value the merge of a single partition gives (weight e^0 = 1).
-template <int HD>
-__device__ __forceinline__ void attn_store_final_head(const Params& p, float l,
-                                                      const float (&o)[AttnShape<HD>::DPL], int b,
-                                                      int head, int lane) {
-    using S = AttnShape<HD>;
-    float* out = p.attn + (size_t)b * p.Q + (size_t)head * HD + lane * S::DPL;
-#pragma unroll
-    for (int d = 0; d < S::DPL; ++d) out[d] = __fdiv_rn(o[d], l);
-}
-
-// One whole item on one warp: the sub-ranges in order, each folded into the
-// running partial as soon as it is done; the item's partial is left in
-// (rm, rl, ro). `rows`/`done` as for attn_sub.
-template <int HD, bool SMEM, class Rows, class Done>
-__device__ __forceinline__ bool attn_item_serial(const Params& p, AttnState<HD>& st, uint32_t first,
-                                                 uint32_t count, int pos, const uint16_t* Kpos,
-                                                 const uint16_t* Vpos, float* s, int lane, Rows&& rows,
-                                                 Done&& done, float (&rm)[kMaxGroup],
-                                                 float (&rl)[kMaxGroup],
-                                                 float (&ro)[kMaxGroup][AttnShape<HD>::DPL]) {
-    using S = AttnShape<HD>;
-    for (int u = 0; u < kSubRanges; ++u) {
-        int lo, hi;
-        sub_range(first, count, u, &lo, &hi);
-        if (!attn_sub<HD, SMEM>(p, st, first, lo, hi, pos, Kpos, Vpos, s, lane, rows, done)) return false;
-        if (u == 0) {
+    {
+        float ls[kMaxGroup] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = t; j < n; j += NT) {
+            const float4 v = et[j];
+            const float s[kMaxGroup] = {v.x, v.y, v.z, v.w};
+            float e[kMaxGroup];
 #pragma unroll
             for (int h = 0; h < kMaxGroup; ++h) {
-                rm[h] = st.m[h];
-                rl[h] = st.l[h];
-#pragma unroll
-                for (int d = 0; d < S::DPL; ++d) ro[h][d] = st.o[h][d];
+                e[h] = h < G ? expf(s[h] - M[h]) : 0.f;
+                ls[h] += e[h];
             }
-        } else {
-            fold_partial<HD>(rm, rl, ro, st.m, st.l, st.o);
+            et[j] = make_float4(e[0], e[1], e[2], e[3]);
         }
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) ls[h] = warp_sum(ls[h]);
+        if (lane == 0) wsum[warp] = make_float4(ls[0], ls[1], ls[2], ls[3]);
+    }
+    mark(2);
+    if (!bar()) return false;
+    mark(3);
+    // 3. values: thread (kq, dp), keys kq, kq + KQ, ... (the key at pos last)
+    {
+        const int dp = t % (HD / 2), kq = t / (HD / 2);
+        float a[kMaxGroup][2];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) a[h][0] = a[h][1] = 0.f;
+        const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
+        const size_t vofs = (size_t)R.kps * HD;
+        for (int j0 = kq; j0 < nc; j0 += PB * KQ) {
+            uint32_t w[PB];
+            float4 e[PB];
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const int j = j0 + i * KQ;
+                const bool ok = j < nc;
+                const uint16_t* vr = ok ? attn_row<HD>(R, m, j) + vofs : R.vnew;  // stand-in, masked
+                w[i] = *reinterpret_cast<const uint32_t*>(vr + dp * 2);
+                e[i] = et[ok ? j : 0];
+            }
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                if (j0 + i * KQ >= nc) e[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                const float v0 = bf_lo(w[i]), v1 = bf_hi(w[i]);
+                a[0][0] = fmaf(e[i].x, v0, a[0][0]); a[0][1] = fmaf(e[i].x, v1, a[0][1]);
+                a[1][0] = fmaf(e[i].y, v0, a[1][0]); a[1][1] = fmaf(e[i].y, v1, a[1][1]);
+                a[2][0] = fmaf(e[i].z, v0, a[2][0]); a[2][1] = fmaf(e[i].z, v1, a[2][1]);
+                a[3][0] = fmaf(e[i].w, v0, a[3][0]); a[3][1] = fmaf(e[i].w, v1, a[3][1]);
+            }
+        }
+        if (R.jnew >= 0 && R.jnew % KQ == kq) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(R.vnew + dp * 2);
+            const float v0 = bf_lo(w), v1 = bf_hi(w);
+            const float4 e = et[R.jnew];
+            a[0][0] = fmaf(e.x, v0, a[0][0]); a[0][1] = fmaf(e.x, v1, a[0][1]);
+            a[1][0] = fmaf(e.y, v0, a[1][0]); a[1][1] = fmaf(e.y, v1, a[1][1]);
+            a[2][0] = fmaf(e.z, v0, a[2][0]); a[2][1] = fmaf(e.z, v1, a[2][1]);
+            a[3][0] = fmaf(e.w, v0, a[3][0]); a[3][1] = fmaf(e.w, v1, a[3][1]);
+        }
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+            *reinterpret_cast<float2*>(part + ((size_t)(kq * kMaxGroup + h) * HD + dp * 2)) =
+                make_float2(a[h][0], a[h][1]);
+    }
+    mark(4);
+    if (!bar()) return false;
+    mark(5);
+    // the class sums in class order, the warps' sums in warp order
+    for (int u = t; u < G * HD; u += NT) {
+        const int h = u / HD, d = u % HD;
+        float o = part[(size_t)h * HD + d];
+#pragma unroll
+        for (int kq = 1; kq < KQ; ++kq) o += part[((size_t)(kq * kMaxGroup + h)) * HD + d];
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) l += sc[kAttnWSum + 4 * w + h];
+        emit(h, d, o, M[h], l);
     }
     return true;
 }

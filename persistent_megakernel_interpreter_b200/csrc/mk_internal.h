@@ -18,14 +18,19 @@ namespace mk {
 constexpr int kConsumerWarps = 8;                    // compute warps
 constexpr int kLoaderWarp = kConsumerWarps;          // streams weights and cached KV
 constexpr int kPrepWarp = kConsumerWarps + 1;        // waits on counters, prepares inputs
-constexpr int kThreads = 32 * (kConsumerWarps + 2);
+constexpr int kPrefetchWarp = kConsumerWarps + 2;    // pulls upcoming fills into L2
+constexpr int kThreads = 32 * (kConsumerWarps + 3);
 constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
-constexpr int kMaxAttnItems = kConsumerWarps;        // attention items per job, one per warp
 constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
-constexpr int kSubRangeCount = 8;                    // sub-ranges of an attention item
+constexpr int kMaxItemKeys = 512;                    // keys of one attention item at most
+// Shared-memory scratch of one attention item, in floats: per-key weights
+// [kMaxItemKeys][4], per-warp maxima and sums [kConsumerWarps][4] each, the value
+// phase's class sums (two per compute thread and head), a flag word.
+constexpr uint32_t kAttnScratchFloats =
+    4 * kMaxItemKeys + 8 * kConsumerWarps + 2 * 32 * kConsumerWarps * kMaxGroupHeads + 4;
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
@@ -61,7 +66,7 @@ struct Layout {
 struct SmemLayout {
     uint32_t ring, full, empty, armed;        // weight / cached-KV ring of S stages
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
-    uint32_t scores;                          // per compute warp: attention scores
+    uint32_t scores;                          // attention item scratch (kAttnScratchFloats)
     uint32_t tot;                             // down-projection running sums
     uint32_t cbar;                            // barrier of the compute warps
     uint32_t total;
@@ -69,8 +74,7 @@ struct SmemLayout {
 
 MK_HD inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
-MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes,
-                                    int keys_per_stage) {
+MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes) {
     SmemLayout m;
     uint32_t o = 0;
     m.ring = o;      o += (uint32_t)S * stage_bytes;
@@ -81,7 +85,7 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs_full = o;   o += 8u * NS;
     m.xs_empty = o;  o += 8u * NS;
     m.xs_done = o;   o = align16(o + 4u * NS);
-    m.scores = o;    o += 4u * kConsumerWarps * kMaxGroupHeads * (uint32_t)keys_per_stage;
+    m.scores = o;    o += 4u * kAttnScratchFloats;
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
     m.cbar = o;      o += 8u;
     m.total = align16(o);
@@ -135,10 +139,9 @@ struct Params {
     int xs_slots;              // activation slots (1..3)
     uint32_t xs_slot_bytes;
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
-    uint32_t attn_item_bytes;  // one attention item's q and new key/value inside a slot
     int n_counters;
     int l2_prefetch_fills;     // how far (in fills) the L2 prefetch may run ahead (0 = off)
-    int l2_prefetch_evict_last;
+    int l2_prefetch_policy;    // 0: evict-last, 1: evict-normal
     int max_inflight;          // ring fills the loader keeps in flight at most (0 = ring size)
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)

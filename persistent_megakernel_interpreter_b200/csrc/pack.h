@@ -30,7 +30,7 @@ uint32_t default_stage_bytes(const Layout& L);
 struct SlotPlan {
     int keys_per_stage;
     uint32_t vec_floats;   // one sequence's input vector inside a slot
-    uint32_t item_bytes;   // one attention item (q and the new key/value) inside a slot
+    uint32_t item_bytes;   // an attention item's q and new key/value inside a slot
     uint32_t slot_bytes;
     int xs_slots;
     int stages;

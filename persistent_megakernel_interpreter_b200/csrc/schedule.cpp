@@ -43,16 +43,11 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
     sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
     // per sequence: the input vector, then (QKV jobs) the RoPE row cos[d/2], sin[d/2]
-    // and the position
-    // an attention job: its items' q and new key/value, or one item plus the
-    // kSubRanges sub-range partials (m, l, o) when its warps split it
-    const uint32_t sub_bytes = 4u * kSubRangeCount * (2u * kMaxGroupHeads + kMaxGroupHeads * (uint32_t)L.d);
-    sp.slot_bytes = align16(std::max({(uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u,
-                                      (uint32_t)kMaxAttnItems * sp.item_bytes, sp.item_bytes + sub_bytes}));
+    // and the position; an attention job: its item's q and new key/value
+    sp.slot_bytes = align16(std::max((uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u, sp.item_bytes));
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
-        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, sp.keys_per_stage).total + 1024 <=
-               kSmemBudget)
+        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
             ++S;
         if (S >= (ns > 1 ? 6 : 2) || ns == 1) {
             sp.xs_slots = ns;
@@ -60,8 +55,7 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
             break;
         }
     }
-    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes,
-                                sp.keys_per_stage).total;
+    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes).total;
     return sp;
 }
 
@@ -75,22 +69,32 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const SlotPlan sp = slot_plan(L, batch, stage_bytes);
     const int kps = sp.keys_per_stage;
     if (kps < 1 || sp.stages < 2) return MK_ERR_UNSUPPORTED;
+    // the attention value phase splits an item's keys into classes j mod KQ
+    // (KQ = compute threads / (head_dim / 2)); a ring stage must hold whole rounds
+    const int attn_classes = std::max(1, 32 * kConsumerWarps / (L.d / 2));
+    if (kps % attn_classes) return MK_ERR_UNSUPPORTED;
 
     // attention partitions: one per (sequence, KV group) up to kKeysPerItem keys,
     // more for longer contexts, but no more items than SMs (and at most
-    // kMaxParts per pair, the merge's limit). A partition is a multiple of 8 keys
-    // up to one ring stage, then a multiple of whole stages.
+    // kMaxParts per pair, the merge's limit). An item's fills must all sit in the
+    // ring at once and its scores in the item scratch, so a partition holds at
+    // most min(kMaxItemKeys, stages * keys_per_stage) keys. A partition is a
+    // multiple of 8 keys up to one ring stage, then a multiple of whole stages.
     constexpr int kKeysPerItem = 256;
+    const int max_item = std::min(kMaxItemKeys, sp.stages * kps);
     int part_keys;
     if (o.part_keys > 0) {
         if (o.part_keys > kps && o.part_keys % kps) return MK_ERR_INVALID_ARG;
+        if (o.part_keys > max_item) return MK_ERR_INVALID_ARG;
         part_keys = o.part_keys;
     } else {
         const int pairs = batch * L.nkv;
         const int cap = std::max(1, std::min(kMaxParts, n_sm / pairs));
-        const int parts = std::max(1, std::min(cap, (max_ctx + kKeysPerItem - 1) / kKeysPerItem));
+        int parts = std::max(1, std::min(cap, (max_ctx + kKeysPerItem - 1) / kKeysPerItem));
+        parts = std::max(parts, (max_ctx + max_item - 1) / max_item);
         const int want = std::max((max_ctx + parts - 1) / parts, (max_ctx + kMaxParts - 1) / kMaxParts);
         part_keys = want <= kps ? (want + 7) / 8 * 8 : (want + kps - 1) / kps * kps;
+        if (part_keys > max_item) part_keys = max_item / kps * kps;
     }
     const int n_parts = (max_ctx + part_keys - 1) / part_keys;
     if (n_parts > kMaxParts) return MK_ERR_INVALID_ARG;
@@ -169,7 +173,9 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const int gu_tiles = L.F / 2, gu_chunk = L.F / 8;
     for (int l = 0; l < L.L; ++l) {
         // QKV: tiles grouped by KV group
-        emit_ranges(share(L.nkv * L.tiles_per_group, L.tile_h), L.tiles_per_group, 1 << 30,
+        // One job per SM even where its range crosses a KV-group boundary (one
+        // RMSNorm of x); the job then signals each group it touched.
+        emit_ranges(share(L.nkv * L.tiles_per_group, L.tile_h), 1 << 30, 1 << 30,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_QKV, l);
                         in.group = (uint16_t)(a / L.tiles_per_group);
@@ -177,11 +183,11 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         in.count = in.nfill = (uint32_t)n;
                         if (l > 0) in.wait_ctr = (uint32_t)c_down[l - 1];
                         in.signal_ctr = (uint32_t)(c_qkv[l] + in.group);
-                        signals[in.signal_ctr]++;
+                        in.aux1 = (uint32_t)((a + n - 1) / L.tiles_per_group - in.group + 1);
+                        for (uint32_t k = 0; k < in.aux1; ++k) signals[in.signal_ctr + k]++;
                         return in;
                     });
-        // attention items, each to the least-loaded SM
-        std::vector<int> items_on(n_sm, 0);
+        // attention items, each its own job on the least-loaded SM
         for (int b = 0; b < batch; ++b)
             for (int g = 0; g < L.nkv; ++g)
                 for (int j = 0; j < n_parts; ++j) {
@@ -200,17 +206,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     in.aux0 = (uint32_t)(c_arr[l] + b * L.nkv + g);
                     lists[best].push_back(in);
                     load[best] += (uint64_t)in.count * kv_key_bytes + kJobOverhead;
-                    items_on[best]++;
                 }
-        // group each SM's items of this layer into jobs of up to kMaxAttnItems
-        for (int s = 0; s < n_sm; ++s) {
-            const int n = items_on[s];
-            mk_instr* first = lists[s].data() + lists[s].size() - n;
-            for (int k = 0; k < n; k += kMaxAttnItems) {
-                const int run = std::min(kMaxAttnItems, n - k);
-                for (int r = 0; r < run; ++r) first[k + r].job_items = r == 0 ? (uint32_t)run : 0u;
-            }
-        }
         // each (sequence, group) pair signals each of its query heads once, when
         // the head's output is final
         signals[c_part[l]] += (uint32_t)(batch * L.nq);
@@ -223,14 +219,16 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
             signals[in.signal_ctr]++;
             return in;
         });
-        emit_ranges(share(gu_tiles, L.tile_h), gu_chunk, 1 << 30, [&](int a, int n) {
+        // likewise one gate/up job per SM, signalling each MLP chunk it touched
+        emit_ranges(share(gu_tiles, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
             mk_instr in = mk_in(MK_OP_GATEUP, l);
             in.group = (uint16_t)(a / gu_chunk);
             in.first = (uint32_t)a;
             in.count = in.nfill = (uint32_t)n;
             in.wait_ctr = (uint32_t)c_o[l];
             in.signal_ctr = (uint32_t)(c_h[l] + in.group);
-            signals[in.signal_ctr]++;
+            in.aux1 = (uint32_t)((a + n - 1) / gu_chunk - in.group + 1);
+            for (uint32_t k = 0; k < in.aux1; ++k) signals[in.signal_ctr + k]++;
             return in;
         });
         emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, batch > 1 ? 1 : down_cap,

@@ -71,7 +71,9 @@ def job_done_signals(L, job, group, n_parts, arr, ctr):
             if arr[a.aux0] == n_parts * group:
                 ctr[a.signal_ctr] += group
     elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
-        ctr[ins.signal_ctr] += 1
+        span = max(1, ins.aux1) if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP) else 1
+        for k in range(span):
+            ctr[ins.signal_ctr + k] += 1
 
 
 def static_signals(instrs, offs, group, n_parts):
@@ -156,6 +158,17 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
             for t in range(ins.first, ins.first + ins.count):
                 cov[(ins.op, ins.layer, t)] += 1
     assert all(v == 1 for v in cov.values())
+    # one QKV and one gate/up job per SM and layer (one RMSNorm each); a job whose
+    # tiles cross a KV-group / MLP-chunk boundary signals every counter it touched
+    for s in range(n_sm):
+        per = collections.Counter((ins.op, ins.layer) for ins in instrs[offs[s]:offs[s + 1]]
+                                  if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP))
+        assert all(v == 1 for v in per.values()), per
+    for ins in instrs:
+        if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP):
+            unit = tpg if ins.op == _lib.OP_QKV else cfg.ffn // 8
+            assert ins.group == ins.first // unit
+            assert ins.aux1 == (ins.first + ins.count - 1) // unit - ins.group + 1
     for l in range(cfg.n_layers):
         assert all(cov[(_lib.OP_QKV, l, t)] for t in range(cfg.n_kv_heads * tpg))
         assert all(cov[(_lib.OP_OPROJ, l, t)] for t in range(cfg.hidden // 4))
@@ -231,12 +244,16 @@ def test_dropped_item_cannot_complete():
 
 
 @pytest.mark.parametrize("cfg,batch,ctx,parts", [
-    (LLAMA_1B, 1, 129, 1), (LLAMA_1B, 1, 1025, 5), (LLAMA_1B, 1, 8193, 17), (LLAMA_3B, 8, 2049, 2),
+    (LLAMA_1B, 1, 129, 1), (LLAMA_1B, 1, 1025, 5), (LLAMA_1B, 1, 8193, 17), (LLAMA_3B, 8, 2049, 11),
     (TINY, 1, 129, 1),
 ])
 def test_partition_count(cfg, batch, ctx, parts):
     """One partition per (sequence, group) up to 256 keys, more for longer
-    contexts, never more items than SMs."""
+    contexts; no more items than SMs unless a partition is already as long as an
+    item may be (all its fills in the ring at once, at most 512 keys)."""
     _, _, info = plan_schedule(cfg, batch, ctx, 148, max_batch=8, max_seq=ctx)
     assert info.n_parts == parts
-    assert info.n_parts * batch * cfg.n_kv_heads <= 148
+    max_item = min(512, info.n_stages * info.keys_per_stage)
+    assert info.part_keys <= max_item
+    assert (info.n_parts * batch * cfg.n_kv_heads <= 148
+            or info.part_keys == max_item // info.keys_per_stage * info.keys_per_stage)
