@@ -102,8 +102,9 @@ typedef struct mk_schedule_opts {
                                 seeded shuffle (for robustness tests) */
     int32_t wait_timeout_ms; /* budget of every device wait; 0 = 2000 ms */
     int32_t test_drop_item;  /* failure-detection test hook: 1-based index, in the list
-                                order, of one instruction whose completion is never signalled
-                                (its waiters then end the step with MK_ERR_TIMEOUT); 0 = none */
+                                order, of one instruction that computes but never publishes
+                                its outputs or its completion (its consumers then end the
+                                step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
     int32_t l2_prefetch_fills; /* a prefetch warp pulls the SM's upcoming fills into L2, at

@@ -203,6 +203,11 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     const size_t o_h = take((size_t)batch * L.F * 4);
     const size_t o_ml = take((size_t)batch * L.nq * I.n_parts * 2 * sizeof(float));
     const size_t o_po = take((size_t)batch * L.nq * I.n_parts * L.d * sizeof(float));
+    // tagged activations of the megakernel, contiguous (cleared as one range)
+    const size_t tw_x = (size_t)batch * L.H, tw_q = (size_t)batch * L.Q,
+                 tw_kv = (size_t)batch * L.nkv * 2 * L.d, tw_a = (size_t)batch * L.Q, tw_h = (size_t)batch * L.F;
+    const size_t tagged_words = tw_x + tw_q + tw_kv + tw_a + tw_h;
+    const size_t o_tag = take(tagged_words * sizeof(uint64_t));
     const size_t o_ctr = take((size_t)I.n_counters * mk::kCounterStride * sizeof(uint32_t));
     const size_t o_ctl = take(sizeof(mk::Ctl));
     MK_CUDA(h, cudaMalloc(&h->scratch, off));
@@ -240,6 +245,12 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     p.hbuf = reinterpret_cast<float*>(sb + o_h);
     p.part_ml = reinterpret_cast<float*>(sb + o_ml);
     p.part_o = reinterpret_cast<float*>(sb + o_po);
+    p.x_t = reinterpret_cast<uint64_t*>(sb + o_tag);
+    p.q_t = p.x_t + tw_x;
+    p.kv_t = p.q_t + tw_q;
+    p.attn_t = p.kv_t + tw_kv;
+    p.h_t = p.attn_t + tw_a;
+    p.tagged_words = tagged_words;
     p.counters = h->counters;
     p.ctl = h->ctl;
     p.instrs = h->d_instrs;

@@ -14,6 +14,7 @@ namespace mk {
 
 constexpr int kBaseWarps = 8;
 constexpr int kBaseThreads = 32 * kBaseWarps;
+static_assert(kBaseThreads == kNT, "the block-level input routines assume the megakernel's compute warps");
 
 __device__ __forceinline__ bool step_failed(const Params& p) {
     return ld_volatile_u32(&p.ctl->status) != 0u;
@@ -49,26 +50,53 @@ __device__ __forceinline__ const uint8_t* op_tiles(const Params& p, int op, int 
     }
 }
 
+// One matvec op of one layer. The CTA first builds each sequence's input vector
+// in shared memory (RMSNorm where the op has one) with the same block routine as
+// the megakernel; then each warp takes tiles.
 template <int OP, int KC, int HD>
 __global__ void __launch_bounds__(kBaseThreads) k_tiles(const __grid_constant__ Params p, int l,
                                                         uint32_t ntiles, uint32_t tile_bytes) {
     if (step_failed(p)) return;
-    const int lane = threadIdx.x & 31;
-    const uint32_t gw = blockIdx.x * kBaseWarps + (threadIdx.x >> 5);
+    extern __shared__ __align__(16) float xs_all[];  // [B][KC*256], then kConsumerWarps floats
+    constexpr int N = KC * 256;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    float* red = xs_all + (size_t)p.B * N;
+    auto bar = []() {
+        __syncthreads();
+        return true;
+    };
+    for (int b = 0; b < p.B; ++b) {
+        const float* sf = nullptr;
+        const uint16_t* sh = nullptr;
+        const uint16_t* w = nullptr;
+        if (OP == MK_OP_QKV) {
+            w = norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2);
+            if (l == 0) sh = embed_row(p, b);
+            else sf = p.x + (size_t)b * p.H;
+        } else if (OP == MK_OP_GATEUP) {
+            w = norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2);
+            sf = p.x + (size_t)b * p.H;
+        } else if (OP == MK_OP_OPROJ) {
+            sf = p.attn + (size_t)b * p.Q;
+        } else {
+            w = norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2);
+            sf = p.x + (size_t)b * p.H;
+        }
+        block_input_plain(sf, sh, w, p.eps, N, xs_all + (size_t)b * N, red, t, warp, lane, bar);
+    }
+    const uint32_t gw = blockIdx.x * kBaseWarps + warp;
     const uint32_t nw = gridDim.x * kBaseWarps;
-    if (gw >= ntiles) return;
     const uint64_t pol = l2_evict_first_policy();
     const uint8_t* base = op_tiles(p, OP, l);
-    XRegs<KC> x;
-    if (p.B == 1) prep_input<OP, KC>(p, l, 0, x, lane);
-    for (uint32_t t = gw; t < ntiles; t += nw) {
+    for (uint32_t tl = gw; tl < ntiles; tl += nw) {
         for (int b = 0; b < p.B; ++b) {
-            if (p.B > 1) prep_input<OP, KC>(p, l, b, x, lane);
+            float4* v = reinterpret_cast<float4*>(xs_all + (size_t)b * N);
+            const XSmem<KC> x{v, v + KC * 32};
             float acc[4];
-            dot4<KC, false>(base + (size_t)t * tile_bytes, x, acc, lane, pol);
+            dot4<KC, false>(base + (size_t)tl * tile_bytes, x, acc, lane, pol);
             RopeRow rr{nullptr, nullptr, 0};
             if constexpr (OP == MK_OP_QKV) rr = rope_row_global(p, b);
-            tile_epilogue<OP, HD>(p, l, b, t, acc, lane, rr);
+            tile_epilogue<OP, HD>(p, l, b, tl, acc, lane, rr);
         }
     }
 }
@@ -182,11 +210,13 @@ static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
         return (w + kBaseWarps - 1) / kBaseWarps;
     };
     const size_t attn_smem = attn_item_smem<HD>(p.group, attn_kpad(p.part_keys));
+    const size_t in_h = (size_t)p.B * KH * 256 * 4 + 4 * kConsumerWarps;
+    const size_t in_o = (size_t)p.B * KO * 256 * 4 + 4 * kConsumerWarps;
     k_validate<<<1, 32, 0, st>>>(p);
     const uint32_t tpg = (uint32_t)(p.group + 2) * (HD / 4);
     for (int l = 0; l < p.L; ++l) {
         const uint32_t nq = (uint32_t)p.nkv * tpg;
-        k_tiles<MK_OP_QKV, KH, HD><<<blocks_for(nq), kBaseThreads, 0, st>>>(p, l, nq, p.tile_h);
+        k_tiles<MK_OP_QKV, KH, HD><<<blocks_for(nq), kBaseThreads, in_h, st>>>(p, l, nq, p.tile_h);
         const uint32_t na = (uint32_t)(p.B * p.nkv * p.n_parts);
         k_attn_item<HD><<<na, kBaseThreads, attn_smem, st>>>(p, l);
         if (p.n_parts > 1) {
@@ -194,19 +224,39 @@ static cudaError_t launch_all(const Params& p, cudaStream_t st, int n_sm) {
             k_attn_merge<HD><<<(nm + kBaseWarps - 1) / kBaseWarps, kBaseThreads, 0, st>>>(p);
         }
         const uint32_t no = (uint32_t)p.H / 4;
-        k_tiles<MK_OP_OPROJ, KO, HD><<<blocks_for(no), kBaseThreads, 0, st>>>(p, l, no, p.tile_o);
+        k_tiles<MK_OP_OPROJ, KO, HD><<<blocks_for(no), kBaseThreads, in_o, st>>>(p, l, no, p.tile_o);
         const uint32_t ng = (uint32_t)p.F / 2;
-        k_tiles<MK_OP_GATEUP, KH, HD><<<blocks_for(ng), kBaseThreads, 0, st>>>(p, l, ng, p.tile_h);
+        k_tiles<MK_OP_GATEUP, KH, HD><<<blocks_for(ng), kBaseThreads, in_h, st>>>(p, l, ng, p.tile_h);
         k_down<KF><<<blocks_for((uint32_t)p.H / 4), kBaseThreads, 0, st>>>(p, l);
     }
     const uint32_t nl = (uint32_t)p.V / 4;
-    k_tiles<MK_OP_LMHEAD, KH, HD><<<blocks_for(nl), kBaseThreads, 0, st>>>(p, 0, nl, p.tile_h);
+    k_tiles<MK_OP_LMHEAD, KH, HD><<<blocks_for(nl), kBaseThreads, in_h, st>>>(p, 0, nl, p.tile_h);
     return cudaGetLastError();
 }
 
 // Shared memory of the attention kernel for the current schedule (set once per
 // schedule, outside any stream capture).
+template <int KH, int KO, int HD>
+static cudaError_t prepare_tiles(const Params& p) {
+    const int in_h = (int)((size_t)p.B * KH * 256 * 4 + 4 * kConsumerWarps);
+    const int in_o = (int)((size_t)p.B * KO * 256 * 4 + 4 * kConsumerWarps);
+    cudaError_t e = cudaFuncSetAttribute(k_tiles<MK_OP_QKV, KH, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, in_h);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_tiles<MK_OP_GATEUP, KH, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, in_h);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_tiles<MK_OP_LMHEAD, KH, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, in_h);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_tiles<MK_OP_OPROJ, KO, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, in_o);
+    return e;
+}
+
 cudaError_t baseline_prepare(const Params& p) {
+    const int KH = p.H / 256, KO = p.Q / 256;
+    cudaError_t e = cudaErrorInvalidValue;
+    if (KH == 2 && KO == 2 && p.d == 64) e = prepare_tiles<2, 2, 64>(p);
+    else if (KH == 8 && KO == 8 && p.d == 64) e = prepare_tiles<8, 8, 64>(p);
+    else if (KH == 12 && KO == 12 && p.d == 128) e = prepare_tiles<12, 12, 128>(p);
+    if (e != cudaSuccess) return e;
     const int kpad = attn_kpad(p.part_keys);
     if (p.d == 64)
         return cudaFuncSetAttribute(k_attn_item<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,

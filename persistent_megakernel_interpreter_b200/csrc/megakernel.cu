@@ -102,12 +102,12 @@ __device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uin
     int ok = 1;
     if (lane == 0) {
         const uint32_t* c = p.counters + (size_t)ctr * kCounterStride;
-        uint32_t v = ld_acquire_u32(c);
+        uint32_t v = ld_relaxed_u32(c);
         if ((int32_t)(v - target) < 0) {
             const uint64_t t0 = global_timer_ns();
             for (uint32_t it = 1;; ++it) {
                 __nanosleep(32);
-                v = ld_acquire_u32(c);
+                v = ld_relaxed_u32(c);
                 if ((int32_t)(v - target) >= 0) break;
                 if ((it & 31u) == 0u) {
                     if (aborted(p)) { ok = 0; break; }
@@ -224,97 +224,198 @@ __device__ __forceinline__ bool wait_input(const Params& p, uint32_t ctr, uint32
     return ok;
 }
 
-// The job input of QKV, gate/up and the LM head: RMSNorm of x (or of the
-// embedding row) into a slot. One copy of the code for the three ops.
-template <int KC>
-__device__ __noinline__ void prep_norm(const void* src, bool src_bf16, const uint16_t* w, float eps,
-                                       float* v, int lane) {
-    XSmem<KC> x{reinterpret_cast<float4*>(v), reinterpret_cast<float4*>(v) + KC * 32};
-    if (src_bf16) load_rmsnorm<KC, true>(src, w, eps, x, lane);
-    else load_rmsnorm<KC, false>(src, w, eps, x, lane);
-}
-
-template <int KH, int KO, int KF, int HD>
-__device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane,
-                         uint32_t epoch, uint32_t job) {
-    const mk_instr& in = ins[0];
-    const int l = in.layer;
-    float* sv = reinterpret_cast<float*>(slot);
-    switch (in.op) {
-        case MK_OP_QKV:
-        case MK_OP_GATEUP:
-        case MK_OP_LMHEAD: {
-            if (in.wait_ctr != MK_NO_COUNTER) {
-                if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job))
-                    return false;
-            } else if (lane == 0) {
-                trace(p, job, kTrCtrDone, global_timer_ns());
-            }
-            const size_t nrm = in.op == MK_OP_QKV ? (size_t)(2 * l) : in.op == MK_OP_GATEUP
-                                                                 ? (size_t)(2 * l + 1)
-                                                                 : (size_t)(2 * p.L);
-            const uint16_t* w = norm_ptr(p, p.off_norms + nrm * p.H * 2);
-            for (int b = 0; b < p.B; ++b) {
-                const bool emb = in.op == MK_OP_QKV && l == 0;
-                const void* src = emb ? static_cast<const void*>(embed_row(p, b))
-                                      : static_cast<const void*>(p.x + (size_t)b * p.H);
-                prep_norm<KH>(src, emb, w, p.eps, sv + (size_t)b * p.xs_vec_floats, lane);
-            }
-            if (in.op == MK_OP_QKV) {
-                // the RoPE row of each sequence's position, for the epilogues
-                float* aux = sv + (size_t)p.B * p.xs_vec_floats;
-                for (int b = 0; b < p.B; ++b) {
-                    const int pos = g_pos[b];
-                    float* row = aux + (size_t)b * (HD + 4);
-                    for (int i = lane; i < HD / 2; i += 32) {
-                        row[i] = p.rope_cos[(size_t)pos * (HD / 2) + i];
-                        row[HD / 2 + i] = p.rope_sin[(size_t)pos * (HD / 2) + i];
-                    }
-                    if (lane == 0) reinterpret_cast<int*>(row)[HD] = pos;
-                }
-            }
-            return true;
-        }
-        case MK_OP_OPROJ: {
-            // the attention output, finished (normalised or merged) by the attention items
-            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
-            for (int b = 0; b < p.B; ++b) {
-                XSmem<KO> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
-                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KO * 32};
-                load_vec<KO>(p.attn + (size_t)b * p.Q, x, lane);
-            }
-            return true;
-        }
-        case MK_OP_DOWN: {
-            if (!wait_input(p, in.wait_ctr + c, target_of(epoch, down_chunk_target(in, c)), in.seq,
-                            lane, job))
-                return false;
-            for (int b = 0; b < p.B; ++b) {
-                XSmem<KF> x{reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats),
-                            reinterpret_cast<float4*>(sv + (size_t)b * p.xs_vec_floats) + KF * 32};
-                load_vec<KF>(p.hbuf + (size_t)b * p.F + (size_t)c * (p.F / 4), x, lane);
-            }
-            return true;
-        }
-        default: {  // attention item: q of the group's heads and the new key/value
-            if (!wait_input(p, in.wait_ctr, target_of(epoch, in.wait_n), in.seq, lane, job)) return false;
-            const float* qsrc = p.q + (size_t)in.batch * p.Q + (size_t)in.group * p.group * HD;
-            float* qdst = reinterpret_cast<float*>(slot);
-            for (int e = lane * 4; e < p.group * HD; e += 128)
-                *reinterpret_cast<uint4*>(qdst + e) = ld_cg_v4(qsrc + e);
-            const int pos = g_pos[in.batch];
-            const size_t off = kv_off(p, l, in.batch, in.group, pos);
-            uint16_t* kv = reinterpret_cast<uint16_t*>(slot + (size_t)p.group * HD * 4);
-            constexpr int kPieces = HD / 8;  // 16-byte pieces per row
-            if (lane < kPieces) {
-                *reinterpret_cast<uint4*>(kv + lane * 8) = ld_cg_v4(p.kc + off + lane * 8);
-            } else if (lane < 2 * kPieces) {
-                const int q = lane - kPieces;
-                *reinterpret_cast<uint4*>(kv + HD + q * 8) = ld_cg_v4(p.vc + off + q * 8);
-            }
-            return true;
+// Pause between polls of tagged words that have not arrived yet, bounded by
+// the wait budget and the abort flag (lane 0 decides for the warp).
+__device__ __forceinline__ bool tag_backoff(const Params& p, uint32_t it, uint64_t& t0, uint32_t where,
+                                            int lane) {
+    __nanosleep(64);
+    if ((it & 15u) != 15u) return true;
+    int bad = 0;
+    if (lane == 0) {
+        if (t0 == 0) t0 = global_timer_ns();
+        if (aborted(p)) bad = 1;
+        else if (global_timer_ns() - t0 > p.timeout_ns) {
+            record_error(p, MK_ERR_TIMEOUT, where, 0xfffffff6u, 0, 0, 7);
+            bad = 1;
         }
     }
+    return __shfl_sync(0xffffffffu, bad, 0) == 0;
+}
+
+// A job's input vector from the tagged activations, by all compute warps (the
+// thread's pairs, all loads in flight at once, retried until every tag is the
+// expected one); RMSNorm with the bf16 norm weights w when w is given. Ends
+// with a compute barrier.
+__device__ bool block_input_tagged(const Params& p, const uint64_t* src, uint32_t tag, const uint16_t* w, int n,
+                                   float* xs, float* red, int t, int warp, int lane, uint64_t* cbar,
+                                   uint32_t& cuses) {
+    const int np = n / 2;
+    uint32_t wv[kMaxPairs];
+    float v0[kMaxPairs], v1[kMaxPairs];
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int j = i * kNT + t;
+        wv[i] = (w != nullptr && j < np) ? ld_cg_u32(w + 2 * j) : 0u;
+    }
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint64_t a[kMaxPairs], b[kMaxPairs];
+#pragma unroll
+        for (int i = 0; i < kMaxPairs; ++i) {
+            const int j = i * kNT + t;
+            a[i] = b[i] = 0ull;
+            if (j < np) ld_tagged2(src + 2 * j, a[i], b[i]);
+        }
+        bool ok = true;
+#pragma unroll
+        for (int i = 0; i < kMaxPairs; ++i) {
+            const int j = i * kNT + t;
+            v0[i] = tag_val(a[i]);
+            v1[i] = tag_val(b[i]);
+            if (j < np) ok = ok & tag_ok(a[i], tag) & tag_ok(b[i], tag);
+        }
+        if (__all_sync(0xffffffffu, ok)) break;
+        if (!tag_backoff(p, it, t0, 1, lane)) return false;
+    }
+    auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
+    return block_store_input(v0, v1, wv, w != nullptr, p.eps, n, xs, red, t, warp, lane, bar);
+}
+
+// `rows` (<= kMaxResidRows) consecutive tagged words into dst, by the threads
+// t < rows (whole warps; the others return at once). No barrier.
+__device__ bool rows_tagged(const Params& p, const uint64_t* src, uint32_t tag, int rows, float* dst, int t,
+                            int lane) {
+    if (t >= ((rows + 31) & ~31)) return true;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const uint64_t w = t < rows ? ld_tagged(src + t) : 0ull;
+        if (__all_sync(0xffffffffu, t >= rows || tag_ok(w, tag))) {
+            if (t < rows) dst[t] = tag_val(w);
+            return true;
+        }
+        if (!tag_backoff(p, it, t0, 3, lane)) return false;
+    }
+}
+
+// Where a job's residual rows sit in its slot (per sequence, kMaxResidRows).
+__device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) {
+    return sv + (size_t)p.B * p.xs_vec_floats + (size_t)p.B * (p.d + 4) + (size_t)b * kMaxResidRows;
+}
+
+// The input of a matvec job, built by the compute warps once the activation
+// warp has seen the job's counter: RMSNorm of x (tagged) or of the embedding row
+// (QKV of layer 0) for QKV, gate/up and the LM head; the attention output and
+// the residual rows (x before the O-projection, or the embedding row) for the
+// O-projection; MLP chunk c and, with the last chunk, the residual rows (x after
+// attention) for the down-projection.
+__device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
+                          uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
+    const int t = warp * 32 + lane, l = in.layer;
+    auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
+    for (int b = 0; b < p.B; ++b) {
+        float* xs = sv + (size_t)b * p.xs_vec_floats;
+        switch (in.op) {
+            case MK_OP_QKV:
+            case MK_OP_GATEUP:
+            case MK_OP_LMHEAD: {
+                const size_t nrm = in.op == MK_OP_QKV ? (size_t)(2 * l) : in.op == MK_OP_GATEUP
+                                                                     ? (size_t)(2 * l + 1)
+                                                                     : (size_t)(2 * p.L);
+                const uint16_t* w = norm_ptr(p, p.off_norms + nrm * p.H * 2);
+                if (in.op == MK_OP_QKV && l == 0) {
+                    if (!block_input_plain(nullptr, embed_row(p, b), w, p.eps, p.H, xs, red, t, warp, lane, bar))
+                        return false;
+                } else {
+                    // x after the previous layer's MLP (QKV, LM head) or after this layer's attention
+                    const uint32_t tag = in.op == MK_OP_GATEUP
+                                             ? act_tag(epoch, l, kTagXAttn)
+                                             : act_tag(epoch, in.op == MK_OP_QKV ? l - 1 : l, kTagXMlp);
+                    if (!block_input_tagged(p, p.x_t + (size_t)b * p.H, tag, w, p.H, xs, red, t, warp, lane, cbar,
+                                            cuses))
+                        return false;
+                }
+                break;
+            }
+            case MK_OP_OPROJ: {
+                const int rows = (int)in.count * 4;
+                float* xr = slot_resid(p, sv, b);
+                if (l == 0) {
+                    if (t < rows) xr[t] = bf2f(embed_row(p, b)[(size_t)in.first * 4 + t]);
+                } else if (!rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4,
+                                        act_tag(epoch, l - 1, kTagXMlp), rows, xr, t, lane)) {
+                    return false;
+                }
+                if (!block_input_tagged(p, p.attn_t + (size_t)b * p.Q, act_tag(epoch, l, kTagAttn), nullptr, p.Q,
+                                        xs, red, t, warp, lane, cbar, cuses))
+                    return false;
+                break;
+            }
+            default: {  // down, chunk c
+                if (c == 3 && !rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4,
+                                           act_tag(epoch, l, kTagXAttn), (int)in.count * 4, slot_resid(p, sv, b),
+                                           t, lane))
+                    return false;
+                if (!block_input_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
+                                        nullptr, p.F / 4, xs, red, t, warp, lane, cbar, cuses))
+                    return false;
+                break;
+            }
+        }
+    }
+    return true;
+}
+
+// An attention item's inputs, by the compute warps: q of the group's heads
+// (fp32) and the step's new key and value (bf16) into the slot. Ends with a
+// compute barrier.
+template <int HD>
+__device__ bool attn_input(const Params& p, const mk_instr& in, uint8_t* slot, int warp, int lane, uint64_t* cbar,
+                           uint32_t& cuses, uint32_t epoch) {
+    const int t = warp * 32 + lane;
+    const uint32_t tag = act_tag(epoch, in.layer, kTagQKV);
+    const int nq = p.group * HD;
+    const uint64_t* qsrc = p.q_t + (size_t)in.batch * p.Q + (size_t)in.group * nq;
+    const uint64_t* kvsrc = p.kv_t + (size_t)(in.batch * p.nkv + in.group) * 2 * HD;
+    float* qdst = reinterpret_cast<float*>(slot);
+    uint16_t* kv = reinterpret_cast<uint16_t*>(slot + (size_t)nq * 4);
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        bool ok = true;
+        for (int e = t; e < nq + 2 * HD; e += kNT) {
+            const uint64_t w = ld_tagged(e < nq ? qsrc + e : kvsrc + (e - nq));
+            ok = ok & tag_ok(w, tag);
+            if (e < nq) qdst[e] = tag_val(w);
+            else kv[e - nq] = f2bf(tag_val(w));  // exact: the values are bf16
+        }
+        if (__all_sync(0xffffffffu, ok)) break;
+        if (!tag_backoff(p, it, t0, 5, lane)) return false;
+    }
+    return compute_barrier(p, cbar, cuses, lane);
+}
+
+// The activation warp's part of a job: for QKV jobs, stage the RoPE row of each
+// sequence's position (constant during the step) in the slot. It waits on no
+// dependency: the compute warps poll the tagged inputs themselves, which saves
+// the round trip of a counter read on every hop.
+template <int HD>
+__device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane, uint32_t epoch,
+                         uint32_t job) {
+    const mk_instr& in = ins[0];
+    float* sv = reinterpret_cast<float*>(slot);
+    if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
+    if (in.op == MK_OP_QKV) {
+        float* aux = sv + (size_t)p.B * p.xs_vec_floats;
+        for (int b = 0; b < p.B; ++b) {
+            const int pos = g_pos[b];
+            float* row = aux + (size_t)b * (HD + 4);
+            for (int i = lane; i < HD / 2; i += 32) {
+                row[i] = p.rope_cos[(size_t)pos * (HD / 2) + i];
+                row[HD / 2 + i] = p.rope_sin[(size_t)pos * (HD / 2) + i];
+            }
+            if (lane == 0) reinterpret_cast<int*>(row)[HD] = pos;
+        }
+    }
+    return true;
 }
 
 template <int KH, int KO, int KF, int HD>
@@ -333,7 +434,7 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
             }
             if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
             if (lane == 0) trace(p, j, kTrCtrWait, global_timer_ns());
-            if (!prep_job<KH, KO, KF, HD>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
+            if (!prep_job<HD>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
             if (lane == 0) {
                 trace(p, j, kTrReady, global_timer_ns());
@@ -360,7 +461,9 @@ __device__ __noinline__ float4 tile_dot(const uint8_t* tile, const float* v, int
 
 template <int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
-                              const float* sv, int warp, int lane, uint32_t job) {
+                              const float* sv, int warp, int lane, uint32_t job, uint32_t epoch) {
+    // a dropped instruction (the failure-detection hook) computes but publishes nothing
+    const bool pub = in.signal_ctr != MK_NO_COUNTER;
     int k = 0;  // trace: warp 0's first tiles (fill wait start, fill ready, dot done)
     auto stamp = [&](int w) {
         if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w, global_timer_ns());
@@ -381,11 +484,20 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
                 case MK_OP_QKV: {
                     const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
                     const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
-                    qkv_epilogue<HD>(p, in.layer, b, tl, acc, lane, rr);
+                    if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, lane, rr, act_tag(epoch, in.layer, kTagQKV));
                     break;
                 }
-                case MK_OP_GATEUP: gateup_epilogue(p, b, tl, acc, lane); break;
-                case MK_OP_OPROJ: residual_epilogue(p, in.layer == 0, b, tl, acc, lane); break;
+                case MK_OP_GATEUP:
+                    if (pub) gateup_epilogue<true>(p, b, tl, acc, lane, act_tag(epoch, in.layer, kTagH));
+                    break;
+                case MK_OP_OPROJ:
+                    // x = x_in + W_o attn for the tile's rows; x_in waits in the slot
+                    if (pub && lane < 4) {
+                        const float xin = slot_resid(p, const_cast<float*>(sv), b)[(tl - in.first) * 4 + lane];
+                        st_tagged(p.x_t + (size_t)b * p.H + tl * 4 + lane, __fadd_rn(xin, pick4(acc, lane)),
+                                  act_tag(epoch, in.layer, kTagXAttn));
+                    }
+                    break;
                 default: logits_epilogue(p, b, tl, acc, lane); break;
             }
         }
@@ -400,7 +512,7 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
 // its running sums, chunks in order 0..3; after chunk 3 the residual.
 template <int KF>
 __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
-                             const float* sv, float* tot, int warp, int lane, uint32_t job) {
+                             const float* sv, float* tot, int warp, int lane, uint32_t job, uint32_t epoch) {
     for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
@@ -412,7 +524,11 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
                 float* t = tot + ((size_t)r * p.B + b) * 4 + lane;
                 const float y = pick4(acc, lane);
                 *t = (c == 0) ? y : *t + y;
-                if (c == 3) residual_one(p, false, b, (in.first + r) * 4 + lane, *t);
+                if (c == 3 && in.signal_ctr != MK_NO_COUNTER) {  // x = x_in + W_d h; x_in waits in the slot
+                    const float xin = slot_resid(p, const_cast<float*>(sv), b)[r * 4 + lane];
+                    st_tagged(p.x_t + (size_t)b * p.H + (in.first + r) * 4 + lane, __fadd_rn(xin, *t),
+                              act_tag(epoch, in.layer, kTagXMlp));
+                }
             }
         }
         release_fill(ring, seq, lane);
@@ -449,9 +565,12 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     const int t = warp * 32 + lane;
     uint32_t* sig = p.counters + (size_t)a.signal_ctr * kCounterStride;
     if (p.n_parts == 1) {
-        float* out = p.attn + (size_t)b * p.Q + (size_t)g * G * HD;
-        if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark,
-                                 [&](int h, int d, float o, float, float l) { out[h * HD + d] = __fdiv_rn(o, l); }))
+        uint64_t* out = p.attn_t + (size_t)b * p.Q + (size_t)g * G * HD;
+        const uint32_t tag = act_tag(epoch, a.layer, kTagAttn);
+        const bool pub = a.signal_ctr != MK_NO_COUNTER;  // a dropped item publishes nothing
+        if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark, [&](int h, int d, float o, float, float l) {
+                if (pub) st_tagged(out + h * HD + d, __fdiv_rn(o, l), tag);
+            }))
             return false;
     } else {
         const int part = (int)(a.first / (uint32_t)p.part_keys);
@@ -470,7 +589,7 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
         for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
     if (!bar()) return false;  // every output of the item is stored
     if (p.n_parts == 1) {
-        if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_release_add(sig, (uint32_t)G);
+        if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_relaxed_add(sig, (uint32_t)G);
         mark(6);
         return true;
     }
@@ -487,18 +606,19 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     if (!bar()) return false;
     if (*reinterpret_cast<volatile uint32_t*>(flag) == 0u) return true;
     if (warp < G) {
-        float* out = p.attn + (size_t)b * p.Q;
+        uint64_t* out = p.attn_t + (size_t)b * p.Q;
+        const uint32_t tag = act_tag(epoch, a.layer, kTagAttn);
         const int head = g * G + warp;
-        attn_merge_heads<HD, 1>(p, b, head, 1, head + 1, lane, [&](int e, float x) { out[e] = x; });
+        attn_merge_heads<HD, 1>(p, b, head, 1, head + 1, lane, [&](int e, float x) { st_tagged(out + e, x, tag); });
     }
     if (!bar()) return false;
-    if (t == 0) red_release_add(sig, (uint32_t)G);
+    if (t == 0) red_relaxed_add(sig, (uint32_t)G);
     return true;
 }
 
 template <int KH, int KO, int KF, int HD>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
-                             float* tot, uint64_t* cbar, int i0, int i1, int warp, int lane,
+                             float* tot, float* red, uint64_t* cbar, int i0, int i1, int warp, int lane,
                              uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
@@ -508,14 +628,17 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, sl.full + s, (j / sl.NS) & 1u, nullptr, j, 4, lane)) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrStart, global_timer_ns());
-            const float* sv = reinterpret_cast<const float*>(sl.slot(j));
-            bool ok;
+            float* sv = reinterpret_cast<float*>(sl.slot(j));
+            bool ok = in.op == MK_OP_ATTN ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
+                                          : job_input(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
+            if (!ok) return;
+            if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7, global_timer_ns());
             switch (in.op) {
-                case MK_OP_QKV: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j); break;
-                case MK_OP_OPROJ: ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j); break;
+                case MK_OP_QKV: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
+                case MK_OP_OPROJ: ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
                 case MK_OP_GATEUP:
-                case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j); break;
-                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j); break;
+                case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
+                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch); break;
                 default:
                     ok = compute_attn_job<HD>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
                                               epoch);
@@ -539,7 +662,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                         const uint32_t span =
                             (in.op == MK_OP_QKV || in.op == MK_OP_GATEUP) && in.aux1 > 1 ? in.aux1 : 1u;
                         for (uint32_t k = 0; k < span; ++k)
-                            red_release_add(p.counters + (size_t)(in.signal_ctr + k) * kCounterStride, 1u);
+                            red_relaxed_add(p.counters + (size_t)(in.signal_ctr + k) * kCounterStride, 1u);
                     }
                 }
                 mbar_arrive(sl.empty + s);
@@ -778,26 +901,37 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else {
             float* scores = reinterpret_cast<float*>(smem + m.scores);
             compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
+                                         reinterpret_cast<float*>(smem + m.red),
                                          reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
                                          s_epoch);
         }
     }
     __syncthreads();
 
+    // The last CTA to finish closes the step: it advances the epoch, or, after a
+    // failed step, clears the counters and every tagged word (so no stale tag can
+    // match the restarted epochs) and restarts the epoch at 0.
+    __shared__ uint32_t s_close;  // 0: not last, 1: last, 2: last after a failure
     if (threadIdx.x == 0) {
         __threadfence();
         const uint32_t old = atom_acq_rel_add(&p.ctl->done, 1u);
-        if (old == gridDim.x - 1) {  // last CTA of the step
-            if (ld_volatile_u32(&p.ctl->status) != 0u) {
-                for (int c = 0; c < p.n_counters; ++c) p.counters[(size_t)c * kCounterStride] = 0u;
-                p.ctl->epoch = 0u;
-                p.ctl->abort = 0u;
-            } else {
-                p.ctl->epoch = s_epoch + 1u;
-            }
-            p.ctl->done = 0u;
-            __threadfence();
+        s_close = old == gridDim.x - 1 ? (ld_volatile_u32(&p.ctl->status) != 0u ? 2u : 1u) : 0u;
+    }
+    __syncthreads();
+    if (s_close == 2u) {
+        for (size_t i = threadIdx.x; i < p.tagged_words; i += blockDim.x) p.x_t[i] = 0ull;
+        for (int c = threadIdx.x; c < p.n_counters; c += blockDim.x) p.counters[(size_t)c * kCounterStride] = 0u;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0 && s_close != 0u) {
+        if (s_close == 2u) {
+            p.ctl->epoch = 0u;
+            p.ctl->abort = 0u;
+        } else {
+            p.ctl->epoch = s_epoch + 1u;
         }
+        p.ctl->done = 0u;
+        __threadfence();
     }
 }
 

@@ -104,6 +104,51 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// ------------------------------------------------------------------ tagged activations
+//
+// Inside one megakernel launch, activations that cross SMs (residual stream x,
+// q and the new key/value, attention output, MLP activations) travel as 64-bit
+// words: the fp32 value in the low half and a tag in the high half naming the
+// step, layer and producer. A single 64-bit access is indivisible, so a reader
+// that sees the expected tag sees the value that goes with it; no fence orders
+// the data before the dependency counter, and the counter becomes a hint of
+// when to look. (A GPU-scope release fence waits for every memory operation
+// the SM has in flight, bulk weight copies included: microseconds when the ring
+// is full, on every signal.)
+enum TagKind : uint32_t { kTagQKV = 1, kTagAttn = 2, kTagXAttn = 3, kTagH = 4, kTagXMlp = 5 };
+
+__host__ __device__ __forceinline__ uint32_t act_tag(uint32_t epoch, int layer, uint32_t kind) {
+    return (((epoch + 1u) & 0x3fffffu) << 10) | ((uint32_t)layer << 3) | kind;
+}
+
+__device__ __forceinline__ void st_tagged(uint64_t* p, float v, uint32_t tag) {
+    const uint64_t w = ((uint64_t)tag << 32) | __float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+__device__ __forceinline__ void ld_tagged2(const uint64_t* p, uint64_t& a, uint64_t& b) {
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_tagged(const uint64_t* p) {
+    uint64_t a;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(a) : "l"(p) : "memory");
+    return a;
+}
+
+__device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+__device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_relaxed_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -291,36 +336,33 @@ __device__ __forceinline__ void load_vec_bf16(const uint16_t* src, X& x, int lan
     }
 }
 
-// RMSNorm in place: x <- (x * r) * w with r = 1 / sqrt(mean(x^2) + eps), mean
-// over the KC*256 elements.
+// RMSNorm of the lane's KC x 8 input elements e (fp32) with norm weights w
+// (bf16, the same layout): per-lane sum of squares in element order, the
+// butterfly, then (x * r) * w into x. Every RMSNorm of the step goes through
+// here, whatever the input's source.
 template <int KC, class X>
-__device__ __forceinline__ void rmsnorm_vec(X& x, const uint16_t* w, float eps, int lane) {
+__device__ __forceinline__ void rmsnorm_core(const float (&e)[KC][8], const uint4 (&wv)[KC], float eps, X& x,
+                                             int lane) {
     float ss = 0.f;
 #pragma unroll
-    for (int kc = 0; kc < KC; ++kc) {
-        float e[8];
-        x.get(kc, lane, e);
+    for (int kc = 0; kc < KC; ++kc)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
-    }
+        for (int i = 0; i < 8; ++i) ss = fmaf(e[kc][i], e[kc][i], ss);
     ss = warp_sum(ss);
     const float r = 1.0f / sqrtf(ss / (float)(KC * 256) + eps);
-    const uint4* wp = reinterpret_cast<const uint4*>(w);
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-        float e[8], wv[8];
-        x.get(kc, lane, e);
-        unpack8(ld_cg_v4(wp + kc * 32 + lane), wv);
+        float wf[8], o[8];
+        unpack8(wv[kc], wf);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(__fmul_rn(e[i], r), wv[i]);
-        x.put(kc, lane, e);
+        for (int i = 0; i < 8; ++i) o[i] = __fmul_rn(__fmul_rn(e[kc][i], r), wf[i]);
+        x.put(kc, lane, o);
     }
 }
 
 // RMSNorm of a vector read from global memory (fp32, or bf16 when SRC_BF16),
 // with every load -- the vector and the norm weights -- issued before the
-// reduction. The arithmetic (per-lane sum of squares in element order, the
-// butterfly, (x * r) * w) is the same as load_vec + rmsnorm_vec.
+// reduction.
 template <int KC, bool SRC_BF16, class X>
 __device__ __forceinline__ void load_rmsnorm(const void* src, const uint16_t* w, float eps, X& x,
                                              int lane) {
@@ -337,39 +379,107 @@ __device__ __forceinline__ void load_rmsnorm(const void* src, const uint16_t* w,
         }
         wv[kc] = ld_cg_v4(wp + kc * 32 + lane);
     }
-    float ss = 0.f;
+    float e[KC][8];
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-        float e[8];
         if (SRC_BF16) {
-            unpack8(ra[kc], e);
+            unpack8(ra[kc], e[kc]);
         } else {
-            e[0] = __uint_as_float(ra[kc].x); e[1] = __uint_as_float(ra[kc].y);
-            e[2] = __uint_as_float(ra[kc].z); e[3] = __uint_as_float(ra[kc].w);
-            e[4] = __uint_as_float(rb[kc].x); e[5] = __uint_as_float(rb[kc].y);
-            e[6] = __uint_as_float(rb[kc].z); e[7] = __uint_as_float(rb[kc].w);
+            e[kc][0] = __uint_as_float(ra[kc].x); e[kc][1] = __uint_as_float(ra[kc].y);
+            e[kc][2] = __uint_as_float(ra[kc].z); e[kc][3] = __uint_as_float(ra[kc].w);
+            e[kc][4] = __uint_as_float(rb[kc].x); e[kc][5] = __uint_as_float(rb[kc].y);
+            e[kc][6] = __uint_as_float(rb[kc].z); e[kc][7] = __uint_as_float(rb[kc].w);
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
     }
-    ss = warp_sum(ss);
-    const float r = 1.0f / sqrtf(ss / (float)(KC * 256) + eps);
+    rmsnorm_core<KC>(e, wv, eps, x, lane);
+}
+
+// ------------------------------------------------------------------ block-level job inputs
+//
+// A matvec job's input vector (n elements, n a multiple of 2 * kNT... or less)
+// is loaded, and normalised where the op needs it, by all kConsumerWarps
+// compute warps of the CTA together, into the XSmem order in shared memory.
+// Thread t owns the element pairs j = i * kNT + t (i ascending). RMSNorm: each
+// thread's sum of squares over its pairs in order, the warp butterfly, the warp
+// sums added in warp order; then (x * r) * w for the thread's own elements. The
+// megakernel and the baseline both go through here, so they agree bit for bit.
+constexpr int kNT = 32 * kConsumerWarps;
+constexpr int kMaxPairs = 8;  // vectors of up to 2 * 8 * kNT = 4096 elements
+
+// Float index, inside an XSmem vector of n elements, of element e (its half, its
+// group of 8, its place): elements e and e + 1 (e even) are adjacent.
+__device__ __forceinline__ int xs_index(int n, int e) {
+    return ((e & 4) ? n / 2 : 0) + (e >> 3) * 4 + (e & 3);
+}
+
+// The thread's pairs (v0[i], v1[i]) = elements 2j, 2j + 1 into the XSmem vector
+// at xs; with w (bf16 norm weights of the pairs, pre-loaded in wv), RMSNorm
+// first. `red`: kConsumerWarps floats of shared scratch. Ends with a barrier.
+template <class Bar>
+__device__ __forceinline__ bool block_store_input(const float (&v0)[kMaxPairs], const float (&v1)[kMaxPairs],
+                                                  const uint32_t (&wv)[kMaxPairs], bool norm, float eps,
+                                                  int n, float* xs, float* red, int t, int warp, int lane,
+                                                  Bar&& bar) {
+    const int np = n / 2;
+    float r = 1.f;
+    if (norm) {
+        float ss = 0.f;
 #pragma unroll
-    for (int kc = 0; kc < KC; ++kc) {
-        float e[8], wf[8];
-        if (SRC_BF16) {
-            unpack8(ra[kc], e);
-        } else {
-            e[0] = __uint_as_float(ra[kc].x); e[1] = __uint_as_float(ra[kc].y);
-            e[2] = __uint_as_float(ra[kc].z); e[3] = __uint_as_float(ra[kc].w);
-            e[4] = __uint_as_float(rb[kc].x); e[5] = __uint_as_float(rb[kc].y);
-            e[6] = __uint_as_float(rb[kc].z); e[7] = __uint_as_float(rb[kc].w);
+        for (int i = 0; i < kMaxPairs; ++i)
+            if (i * kNT + t < np) {
+                ss = fmaf(v0[i], v0[i], ss);
+                ss = fmaf(v1[i], v1[i], ss);
+            }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        if (!bar()) return false;
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) tot += red[w];
+        r = 1.0f / sqrtf(tot / (float)n + eps);
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int j = i * kNT + t;
+        if (j < np) {
+            float a = v0[i], b = v1[i];
+            if (norm) {
+                a = __fmul_rn(__fmul_rn(a, r), bf_lo(wv[i]));
+                b = __fmul_rn(__fmul_rn(b, r), bf_hi(wv[i]));
+            }
+            *reinterpret_cast<float2*>(xs + xs_index(n, 2 * j)) = make_float2(a, b);
         }
-        unpack8(wv[kc], wf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(__fmul_rn(e[i], r), wf[i]);
-        x.put(kc, lane, e);
     }
+    return bar();
+}
+
+// The same from a plain source: fp32 (src_f) or bf16 (src_h) in global memory.
+template <class Bar>
+__device__ __forceinline__ bool block_input_plain(const float* src_f, const uint16_t* src_h, const uint16_t* w,
+                                                  float eps, int n, float* xs, float* red, int t, int warp,
+                                                  int lane, Bar&& bar) {
+    const int np = n / 2;
+    float v0[kMaxPairs], v1[kMaxPairs];
+    uint32_t wv[kMaxPairs];
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int j = i * kNT + t;
+        v0[i] = v1[i] = 0.f;
+        wv[i] = 0u;
+        if (j < np) {
+            if (w) wv[i] = ld_cg_u32(w + 2 * j);
+            if (src_f) {
+                const uint2 u = ld_cg_v2(src_f + 2 * j);
+                v0[i] = __uint_as_float(u.x);
+                v1[i] = __uint_as_float(u.y);
+            } else {
+                const uint32_t u = ld_cg_u32(src_h + 2 * j);
+                v0[i] = bf_lo(u);
+                v1[i] = bf_hi(u);
+            }
+        }
+    }
+    return block_store_input(v0, v1, wv, w != nullptr, eps, n, xs, red, t, warp, lane, bar);
 }
 
 // ------------------------------------------------------------------ the 4-row tile
@@ -442,10 +552,13 @@ __device__ __forceinline__ RopeRow rope_row_global(const Params& p, int b) {
 
 // QKV tile epilogue: RoPE on query/key pairs; q stays fp32, the key and value are
 // rounded to bf16 into the cache slot. `tile` is the tile index inside the
-// layer's QKV block.
-template <int HD>
+// layer's QKV block. TAGGED (the megakernel): q, and the new key and value as
+// the bf16 values written to the cache, also go out as tagged words (q_t, kv_t)
+// for the attention items of this step; otherwise q goes to the plain buffer.
+template <int HD, bool TAGGED>
 __device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint32_t tile,
-                                             const float (&acc)[4], int lane, const RopeRow& rr) {
+                                             const float (&acc)[4], int lane, const RopeRow& rr,
+                                             uint32_t tag) {
     if (lane >= 4) return;
     constexpr int TPH = HD / 4;  // tiles per head
     const int g = tile / (uint32_t)((p.group + 2) * TPH);
@@ -470,12 +583,17 @@ __device__ __forceinline__ void qkv_epilogue(const Params& p, int l, int b, uint
         }
         if (hs < p.group) {
             const int head = g * p.group + hs;
-            p.q[(size_t)b * p.Q + (size_t)head * HD + dim] = out;
+            if (TAGGED) st_tagged(p.q_t + (size_t)b * p.Q + (size_t)head * HD + dim, out, tag);
+            else p.q[(size_t)b * p.Q + (size_t)head * HD + dim] = out;
         } else {
-            p.kc[kv_off(p, l, b, g, pos) + dim] = f2bf(out);   // the cache is bf16
+            const uint16_t kb = f2bf(out);   // the cache is bf16
+            p.kc[kv_off(p, l, b, g, pos) + dim] = kb;
+            if (TAGGED) st_tagged(p.kv_t + ((size_t)(b * p.nkv + g) * 2) * HD + dim, bf2f(kb), tag);
         }
     } else {
-        p.vc[kv_off(p, l, b, g, pos) + 4 * j + lane] = f2bf(pick4(acc, lane));
+        const uint16_t vb = f2bf(pick4(acc, lane));
+        p.vc[kv_off(p, l, b, g, pos) + 4 * j + lane] = vb;
+        if (TAGGED) st_tagged(p.kv_t + ((size_t)(b * p.nkv + g) * 2 + 1) * HD + 4 * j + lane, bf2f(vb), tag);
     }
 }
 
@@ -495,12 +613,15 @@ __device__ __forceinline__ void residual_epilogue(const Params& p, bool from_emb
 }
 
 // gate/up tile rows {g 2j, u 2j, g 2j+1, u 2j+1}: h = (g / (1 + e^-g)) * u.
+template <bool TAGGED>
 __device__ __forceinline__ void gateup_epilogue(const Params& p, int b, uint32_t tile,
-                                                const float (&acc)[4], int lane) {
+                                                const float (&acc)[4], int lane, uint32_t tag) {
     if (lane >= 2) return;
     const float g = lane ? acc[2] : acc[0], u = lane ? acc[3] : acc[1];
     const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
-    p.hbuf[(size_t)b * p.F + 2 * tile + lane] = __fmul_rn(silu, u);
+    const float h = __fmul_rn(silu, u);
+    if (TAGGED) st_tagged(p.h_t + (size_t)b * p.F + 2 * tile + lane, h, tag);
+    else p.hbuf[(size_t)b * p.F + 2 * tile + lane] = h;
 }
 
 __device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t tile,
@@ -511,29 +632,11 @@ __device__ __forceinline__ void logits_epilogue(const Params& p, int b, uint32_t
 
 // ------------------------------------------------------------------ matvec op inputs/outputs
 
-// Input vector of a matvec op for sequence b.
-template <int OP, int KC, class X>
-__device__ __forceinline__ void prep_input(const Params& p, int l, int b, X& x, int lane) {
-    if constexpr (OP == MK_OP_QKV) {
-        const uint16_t* w = norm_ptr(p, p.off_norms + (size_t)(2 * l) * p.H * 2);
-        if (l == 0) load_rmsnorm<KC, true>(embed_row(p, b), w, p.eps, x, lane);
-        else load_rmsnorm<KC, false>(p.x + (size_t)b * p.H, w, p.eps, x, lane);
-    } else if constexpr (OP == MK_OP_GATEUP) {
-        load_rmsnorm<KC, false>(p.x + (size_t)b * p.H,
-                                norm_ptr(p, p.off_norms + (size_t)(2 * l + 1) * p.H * 2), p.eps, x, lane);
-    } else if constexpr (OP == MK_OP_OPROJ) {
-        load_vec<KC>(p.attn + (size_t)b * p.Q, x, lane);
-    } else {  // LM head
-        load_rmsnorm<KC, false>(p.x + (size_t)b * p.H,
-                                norm_ptr(p, p.off_norms + (size_t)(2 * p.L) * p.H * 2), p.eps, x, lane);
-    }
-}
-
 template <int OP, int HD>
 __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uint32_t tile,
                                               const float (&acc)[4], int lane, const RopeRow& rr) {
-    if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD>(p, l, b, tile, acc, lane, rr);
-    else if constexpr (OP == MK_OP_GATEUP) gateup_epilogue(p, b, tile, acc, lane);
+    if constexpr (OP == MK_OP_QKV) qkv_epilogue<HD, false>(p, l, b, tile, acc, lane, rr, 0u);
+    else if constexpr (OP == MK_OP_GATEUP) gateup_epilogue<false>(p, b, tile, acc, lane, 0u);
     else if constexpr (OP == MK_OP_OPROJ) residual_epilogue(p, l == 0, b, tile, acc, lane);
     else logits_epilogue(p, b, tile, acc, lane);
 }

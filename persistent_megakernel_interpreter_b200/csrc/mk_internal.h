@@ -22,6 +22,7 @@ constexpr int kPrefetchWarp = kConsumerWarps + 2;    // pulls upcoming fills int
 constexpr int kThreads = 32 * (kConsumerWarps + 3);
 constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
 constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
+constexpr int kMaxResidRows = 64;                    // residual rows per O-proj / down job
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
@@ -68,6 +69,7 @@ struct SmemLayout {
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
     uint32_t scores;                          // attention item scratch (kAttnScratchFloats)
     uint32_t tot;                             // down-projection running sums
+    uint32_t red;                             // per-warp partial sums of a job input
     uint32_t cbar;                            // barrier of the compute warps
     uint32_t total;
 };
@@ -87,6 +89,7 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs_done = o;   o = align16(o + 4u * NS);
     m.scores = o;    o += 4u * kAttnScratchFloats;
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
+    m.red = o;       o += 4u * 32u;
     m.cbar = o;      o += 8u;
     m.total = align16(o);
     return m;
@@ -127,6 +130,13 @@ struct Params {
     float* hbuf;       // [B][F]
     float* part_ml;    // [B][nq][P][2]  (m, l)
     float* part_o;     // [B][nq][P][d]
+    // the megakernel's tagged activations (value | tag << 32, see act_tag)
+    uint64_t* x_t;     // [B][H]   residual stream
+    uint64_t* q_t;     // [B][Q]   queries
+    uint64_t* kv_t;    // [B][nkv][2][d] the step's new key and value (bf16 values)
+    uint64_t* attn_t;  // [B][Q]   attention output
+    uint64_t* h_t;     // [B][F]   gated MLP activations
+    size_t tagged_words;  // total words of the five (contiguous from x_t)
     uint32_t* counters;
     Ctl* ctl;
     // schedule

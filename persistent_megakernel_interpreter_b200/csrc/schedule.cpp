@@ -42,9 +42,12 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     sp.keys_per_stage = (int)(stage_bytes / (4u * (uint32_t)L.d));
     sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
     sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
-    // per sequence: the input vector, then (QKV jobs) the RoPE row cos[d/2], sin[d/2]
-    // and the position; an attention job: its item's q and new key/value
-    sp.slot_bytes = align16(std::max((uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u) * 4u, sp.item_bytes));
+    // per sequence: the input vector; then per sequence (QKV jobs) the RoPE row
+    // cos[d/2], sin[d/2] and the position; then per sequence (O-proj and down
+    // jobs) the residual rows the job updates. An attention job: its item's q and
+    // new key/value.
+    sp.slot_bytes = align16(std::max(
+        (uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u, sp.item_bytes));
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
         while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
@@ -210,7 +213,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         // each (sequence, group) pair signals each of its query heads once, when
         // the head's output is final
         signals[c_part[l]] += (uint32_t)(batch * L.nq);
-        emit_ranges(share(L.H / 4, L.tile_o), 1 << 30, 1 << 30, [&](int a, int n) {
+        emit_ranges(share(L.H / 4, L.tile_o), 1 << 30, kMaxResidRows / 4, [&](int a, int n) {
             mk_instr in = mk_in(MK_OP_OPROJ, l);
             in.first = (uint32_t)a;
             in.count = in.nfill = (uint32_t)n;
