@@ -181,8 +181,11 @@ enum {
 typedef struct mk_instr {
     uint16_t op, layer;
     uint16_t batch;      /* sequence (MK_OP_ATTN), else 0 */
-    uint16_t group;      /* KV group (QKV, ATTN) or MLP chunk (GATEUP), else 0 */
-    uint32_t first;      /* first 4-row tile / row block (DOWN) / first key (ATTN) */
+    uint16_t group;      /* KV group (QKV, ATTN) or MLP chunk (GATEUP); DOWN: 1 = one
+                            job over all four MLP chunks (batch 1; fills in row block,
+                            chunk order), 0 = four jobs, one per chunk (fills chunk-major) */
+    uint32_t first;      /* first 4-row tile / row block (DOWN) / first key (ATTN);
+                            GATEUP: first tile of the SM's slice of each MLP chunk */
     uint32_t count;      /* tiles / row blocks / keys */
     uint32_t seq;        /* index of its first ring stage fill in this SM's stream */
     uint32_t nfill;      /* ring stage fills it consumes */
@@ -193,10 +196,13 @@ typedef struct mk_instr {
                             ATTN: the layer's attention counter, incremented once per
                             query head when that head's output is final */
     uint32_t job_items;  /* 1: every instruction (an attention item included) is one
-                            job of the SM's compute warps (DOWN: four, one per chunk) */
+                            job of the SM's compute warps (DOWN with group 0: four, one
+                            per chunk) */
     uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
                             high 16 bits of aux0) and 3 (aux1). ATTN: aux0 = the pair's
-                            arrival counter (heads whose partial is stored). QKV and
+                            arrival counter (heads whose partial is stored). GATEUP:
+                            aux0 = tiles per chunk; the instruction's tile i is tile
+                            (i / aux0) * (ffn / 8) + first + i % aux0 (chunk-major). QKV and
                             GATEUP: aux1 = how many consecutive counters from signal_ctr
                             the instruction increments by one each (the KV groups / MLP
                             chunks its tiles touch; 0 reads as 1). Else 0 */

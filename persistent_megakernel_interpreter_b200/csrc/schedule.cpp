@@ -48,9 +48,11 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     // new key/value.
     sp.slot_bytes = align16(std::max(
         (uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u, sp.item_bytes));
+    // batch 1: a down instruction is one job whose input is the whole MLP vector
+    sp.big_floats = batch == 1 ? (uint32_t)L.F : 0u;
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
-        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
+        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, sp.big_floats).total + 1024 <= kSmemBudget)
             ++S;
         if (S >= (ns > 1 ? 6 : 2) || ns == 1) {
             sp.xs_slots = ns;
@@ -58,7 +60,7 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
             break;
         }
     }
-    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes).total;
+    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes, sp.big_floats).total;
     return sp;
 }
 
@@ -222,21 +224,32 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
             signals[in.signal_ctr]++;
             return in;
         });
-        // likewise one gate/up job per SM, signalling each MLP chunk it touched
-        emit_ranges(share(gu_tiles, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
-            mk_instr in = mk_in(MK_OP_GATEUP, l);
-            in.group = (uint16_t)(a / gu_chunk);
-            in.first = (uint32_t)a;
-            in.count = in.nfill = (uint32_t)n;
-            in.wait_ctr = (uint32_t)c_o[l];
-            in.signal_ctr = (uint32_t)(c_h[l] + in.group);
-            in.aux1 = (uint32_t)((a + n - 1) / gu_chunk - in.group + 1);
-            for (uint32_t k = 0; k < in.aux1; ++k) signals[in.signal_ctr + k]++;
-            return in;
-        });
+        // gate/up, chunk-major: every SM takes the same slice [a, a + n) of each of
+        // the four MLP chunks and works through the chunks in order, so chunks 0..2
+        // of h are complete well before the layer's last gate/up tile; one job per SM,
+        // which counts once on each chunk counter
+        {
+            const std::vector<int> cnt = share(gu_chunk, 4ull * L.tile_h);
+            int start = 0;
+            for (int s = 0; s < n_sm; ++s) {
+                const int n = cnt[s];
+                if (n == 0) continue;
+                mk_instr in = mk_in(MK_OP_GATEUP, l);
+                in.first = (uint32_t)start;
+                in.count = in.nfill = 4u * (uint32_t)n;
+                in.aux0 = (uint32_t)n;
+                in.wait_ctr = (uint32_t)c_o[l];
+                in.signal_ctr = (uint32_t)c_h[l];
+                in.aux1 = 4;
+                for (uint32_t k = 0; k < 4; ++k) signals[in.signal_ctr + k]++;
+                lists[s].push_back(in);
+                start += n;
+            }
+        }
         emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, batch > 1 ? 1 : down_cap,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_DOWN, l);
+                        in.group = batch == 1 ? 1 : 0;  // 1: one job over all four chunks
                         in.first = (uint32_t)a;
                         in.count = (uint32_t)n;
                         in.nfill = 4u * (uint32_t)n;

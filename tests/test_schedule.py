@@ -26,7 +26,7 @@ def jobs_of(lst):
         ins = lst[i]
         items = ins.job_items if ins.op == _lib.OP_ATTN else 1
         assert items >= 1
-        for c in range(4 if ins.op == _lib.OP_DOWN else 1):
+        for c in range(4 if (ins.op == _lib.OP_DOWN and ins.group != 1) else 1):
             jobs.append((i, c, items))
         i += items
     return jobs
@@ -38,8 +38,10 @@ def job_waits(lst, job):
     if ins.op == _lib.OP_ATTN:
         return [(lst[i + k].wait_ctr, lst[i + k].wait_n) for k in range(items)]
     if ins.op == _lib.OP_DOWN:
-        t = [ins.wait_n, ins.aux0 & 0xFFFF, ins.aux0 >> 16, ins.aux1][c]
-        return [(ins.wait_ctr + c, t)]
+        t = [ins.wait_n, ins.aux0 & 0xFFFF, ins.aux0 >> 16, ins.aux1]
+        if ins.group == 1:  # one job over the whole MLP: every chunk
+            return [(ins.wait_ctr + k, t[k]) for k in range(4)]
+        return [(ins.wait_ctr + c, t[c])]
     return [] if ins.wait_ctr == NO else [(ins.wait_ctr, ins.wait_n)]
 
 
@@ -53,6 +55,8 @@ def job_fills(lst, job, w):
         a = lst[i + w]
         return list(range(a.seq, a.seq + a.nfill))
     if ins.op == _lib.OP_DOWN:
+        if ins.group == 1:  # fills in (row block, chunk) order, tile k to warp k mod W
+            return [ins.seq + k for k in range(w, 4 * ins.count, W)]
         return [ins.seq + c * ins.count + r for r in range(w, ins.count, W)]
     return [ins.seq + t for t in range(w, ins.count, W)]
 
@@ -70,7 +74,7 @@ def job_done_signals(L, job, group, n_parts, arr, ctr):
             arr[a.aux0] += group
             if arr[a.aux0] == n_parts * group:
                 ctr[a.signal_ctr] += group
-    elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
+    elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or ins.group == 1 or c == 3):
         span = max(1, ins.aux1) if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP) else 1
         for k in range(span):
             ctr[ins.signal_ctr + k] += 1
@@ -154,6 +158,11 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
             for k in range(ins.first, ins.first + ins.count):
                 cov[(ins.op, ins.layer, ins.batch, ins.group, k)] += 1
             assert ins.nfill == -(-ins.count // info.keys_per_stage)
+        elif ins.op == _lib.OP_GATEUP:  # chunk-major: the same slice of each chunk
+            assert ins.count == 4 * ins.aux0
+            for i in range(ins.count):
+                t = (i // ins.aux0) * (cfg.ffn // 8) + ins.first + i % ins.aux0
+                cov[(ins.op, ins.layer, t)] += 1
         else:
             for t in range(ins.first, ins.first + ins.count):
                 cov[(ins.op, ins.layer, t)] += 1
@@ -165,10 +174,11 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
                                   if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP))
         assert all(v == 1 for v in per.values()), per
     for ins in instrs:
-        if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP):
-            unit = tpg if ins.op == _lib.OP_QKV else cfg.ffn // 8
-            assert ins.group == ins.first // unit
-            assert ins.aux1 == (ins.first + ins.count - 1) // unit - ins.group + 1
+        if ins.op == _lib.OP_QKV:
+            assert ins.group == ins.first // tpg
+            assert ins.aux1 == (ins.first + ins.count - 1) // tpg - ins.group + 1
+        if ins.op == _lib.OP_GATEUP:  # every chunk counter, once
+            assert ins.aux1 == 4 and ins.first + ins.aux0 <= cfg.ffn // 8
     for l in range(cfg.n_layers):
         assert all(cov[(_lib.OP_QKV, l, t)] for t in range(cfg.n_kv_heads * tpg))
         assert all(cov[(_lib.OP_OPROJ, l, t)] for t in range(cfg.hidden // 4))
