@@ -181,9 +181,7 @@ enum {
 typedef struct mk_instr {
     uint16_t op, layer;
     uint16_t batch;      /* sequence (MK_OP_ATTN), else 0 */
-    uint16_t group;      /* KV group (QKV, ATTN) or MLP chunk (GATEUP); DOWN: 1 = one
-                            job over all four MLP chunks (batch 1; fills in row block,
-                            chunk order), 0 = four jobs, one per chunk (fills chunk-major) */
+    uint16_t group;      /* KV group (QKV, ATTN), else 0 */
     uint32_t first;      /* first 4-row tile / row block (DOWN) / first key (ATTN);
                             GATEUP: first tile of the SM's slice of each MLP chunk */
     uint32_t count;      /* tiles / row blocks / keys */
@@ -196,8 +194,7 @@ typedef struct mk_instr {
                             ATTN: the layer's attention counter, incremented once per
                             query head when that head's output is final */
     uint32_t job_items;  /* 1: every instruction (an attention item included) is one
-                            job of the SM's compute warps (DOWN with group 0: four, one
-                            per chunk) */
+                            job of the SM's compute warps (DOWN: four, one per chunk) */
     uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
                             high 16 bits of aux0) and 3 (aux1). ATTN: aux0 = the pair's
                             arrival counter (heads whose partial is stored). GATEUP:

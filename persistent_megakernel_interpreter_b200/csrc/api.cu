@@ -266,8 +266,6 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         p.xs_slots = sp.xs_slots;
         p.xs_slot_bytes = sp.slot_bytes;
         p.xs_vec_floats = sp.vec_floats;
-        p.big_floats = sp.big_floats;
-        p.down_whole = sp.big_floats != 0u;
     }
     p.n_counters = I.n_counters;
     if (opts && opts->trace) {
@@ -275,7 +273,7 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         for (int s = 0; s < n_sm; ++s) {
             int jobs = 0;
             for (int i = P.sm_off[s]; i < P.sm_off[s + 1]; ++i)
-                jobs += (P.instrs[i].op == MK_OP_DOWN && P.instrs[i].group != 1) ? 4 : 1;
+                jobs += P.instrs[i].op == MK_OP_DOWN ? 4 : 1;
             most = jobs > most ? jobs : most;
         }
         h->trace_jobs = most;

@@ -308,12 +308,11 @@ __device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) 
     return sv + (size_t)p.B * p.xs_vec_floats + (size_t)p.B * (p.d + 4) + (size_t)b * kMaxResidRows;
 }
 
-// The input of a matvec job, built by the compute warps once the activation
-// warp has seen the job's counter: RMSNorm of x (tagged) or of the embedding row
-// (QKV of layer 0) for QKV, gate/up and the LM head; the attention output and
-// the residual rows (x before the O-projection, or the embedding row) for the
-// O-projection; MLP chunk c and, with the last chunk, the residual rows (x after
-// attention) for the down-projection.
+// The input of a matvec job, built by the compute warps (they poll the tagged
+// words themselves): RMSNorm of x (tagged) or of the embedding row (QKV of
+// layer 0) for QKV, gate/up and the LM head; the attention output and the
+// residual rows (x before the O-projection, or the embedding row) for the
+// O-projection. (The down-projection's inputs are staged by the activation warp.)
 __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
                           uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
     const int t = warp * 32 + lane, l = in.layer;
@@ -356,16 +355,6 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
                     return false;
                 break;
             }
-            default: {  // down, chunk c
-                if (c == 3 && !rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4,
-                                           act_tag(epoch, l, kTagXAttn), (int)in.count * 4, slot_resid(p, sv, b),
-                                           t, lane))
-                    return false;
-                if (!block_input_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
-                                        nullptr, p.F / 4, xs, red, t, warp, lane, cbar, cuses))
-                    return false;
-                break;
-            }
         }
     }
     return true;
@@ -399,13 +388,26 @@ __device__ bool attn_input(const Params& p, const mk_instr& in, uint8_t* slot, i
     return compute_barrier(p, cbar, cuses, lane);
 }
 
-// Chunk c of h (tagged, F/4 elements) into its XSmem vector in `big`, by one
-// warp, sixteen pairs per lane in flight; retried until every tag is current.
-__device__ bool warp_load_h_chunk(const Params& p, int c, uint32_t tag, float* big, int lane) {
-    const int n4 = p.F / 4, np = n4 / 2;
-    const uint64_t* src = p.h_t + (size_t)c * n4;
-    float* dst = big + (size_t)c * n4;
+// Waits (lane 0 polls, the warp follows) until the tagged word at `w` carries
+// `tag`: a cheap sign that a vector's producers have written it, before the
+// warp reads the whole vector (whose every tag is still checked).
+__device__ __forceinline__ bool poll_tagged(const Params& p, const uint64_t* w, uint32_t tag, uint32_t where,
+                                            int lane) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const int ok = lane == 0 ? (int)tag_ok(ld_tagged(w), tag) : 1;
+        if (__shfl_sync(0xffffffffu, ok, 0)) return true;
+        if (!tag_backoff(p, it, t0, where, lane)) return false;
+    }
+}
+
+// A tagged vector of n elements into the XSmem vector at dst, by one warp,
+// sixteen pairs per lane in flight; retried until every tag is current.
+__device__ bool warp_load_tagged(const Params& p, const uint64_t* src, uint32_t tag, int n, float* dst,
+                                 uint32_t where, int lane) {
+    const int np = n / 2;
     constexpr int D = 16;
+    if (!poll_tagged(p, src + n - 1, tag, where, lane)) return false;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         bool ok = true;
@@ -422,12 +424,12 @@ __device__ bool warp_load_h_chunk(const Params& p, int c, uint32_t tag, float* b
                 const int j = j0 + i * 32 + lane;
                 if (j < np) {
                     ok = ok & tag_ok(a[i], tag) & tag_ok(b[i], tag);
-                    *reinterpret_cast<float2*>(dst + xs_index(n4, 2 * j)) = make_float2(tag_val(a[i]), tag_val(b[i]));
+                    *reinterpret_cast<float2*>(dst + xs_index(n, 2 * j)) = make_float2(tag_val(a[i]), tag_val(b[i]));
                 }
             }
         }
         if (__all_sync(0xffffffffu, ok)) return true;
-        if (!tag_backoff(p, it, t0, 8, lane)) return false;
+        if (!tag_backoff(p, it, t0, where, lane)) return false;
     }
 }
 
@@ -436,25 +438,38 @@ __device__ bool warp_load_h_chunk(const Params& p, int c, uint32_t tag, float* b
 // dependency: the compute warps poll the tagged inputs themselves, which saves
 // the round trip of a counter read on every hop.
 template <int HD>
-__device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, float* big,
-                         const volatile uint32_t* jobs_done, uint32_t attn_before, int lane, uint32_t epoch,
+__device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane, uint32_t epoch,
                          uint32_t job) {
     const mk_instr& in = ins[0];
     float* sv = reinterpret_cast<float*>(slot);
     if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
-    if (in.op == MK_OP_DOWN && in.group == 1) {
-        // the whole-MLP down job: chunks 0..2 of h as they complete (gate/up runs
-        // chunk-major); the compute warps load chunk 3 when the job starts. `big`
-        // doubles as the attention scratch: first wait until the compute warps are
-        // past the last attention job before this one (no later job before this
-        // one uses it).
-        if (attn_before > 0) {
-            uint64_t t0 = 0;
-            for (uint32_t it = 0; *jobs_done < attn_before; ++it)
-                if (!tag_backoff(p, it, t0, 9, lane)) return false;
+    if (in.op == MK_OP_DOWN) {
+        // down chunk c: h chunk c (gate/up runs chunk-major, so chunks complete one
+        // after another while gate/up still streams) and, with the last chunk, the
+        // residual rows (x after attention), staged ahead of the compute warps
+        for (int b = 0; b < p.B; ++b) {
+            if (!warp_load_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, in.layer, kTagH),
+                                  p.F / 4, sv + (size_t)b * p.xs_vec_floats, 8, lane))
+                return false;
+            if (c == 3) {
+                const int rows = (int)in.count * 4;
+                const uint64_t* xs = p.x_t + (size_t)b * p.H + (size_t)in.first * 4;
+                const uint32_t tag = act_tag(epoch, in.layer, kTagXAttn);
+                float* xr = slot_resid(p, sv, b);
+                for (int r0 = 0; r0 < rows; r0 += 32) {
+                    const int r = r0 + lane;
+                    uint64_t t0 = 0;
+                    for (uint32_t it = 0;; ++it) {
+                        const uint64_t w = r < rows ? ld_tagged(xs + r) : 0ull;
+                        if (__all_sync(0xffffffffu, r >= rows || tag_ok(w, tag))) {
+                            if (r < rows) xr[r] = tag_val(w);
+                            break;
+                        }
+                        if (!tag_backoff(p, it, t0, 4, lane)) return false;
+                    }
+                }
+            }
         }
-        for (int k = 0; k < 3; ++k)
-            if (!warp_load_h_chunk(p, k, act_tag(epoch, in.layer, kTagH), big, lane)) return false;
     }
     if (in.op == MK_OP_QKV) {
         float* aux = sv + (size_t)p.B * p.xs_vec_floats;
@@ -472,14 +487,12 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
 }
 
 template <int KH, int KO, int KF, int HD>
-__device__ void activation_warp(const Params& p, const Slots& sl, float* big, const volatile uint32_t* jobs_done,
-                                int i0, int i1, int lane, uint32_t epoch) {
+__device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1, int lane, uint32_t epoch) {
     uint32_t j = 0;
-    uint32_t attn_before = 0;  // jobs up to and including the last attention job so far
     for (int i = i0; i < i1;) {
         const mk_instr* ins = p.instrs + i;
         const uint32_t op = ins[0].op;
-        const int njobs = (op == MK_OP_DOWN && ins[0].group != 1) ? 4 : 1;
+        const int njobs = (op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS, use = j / sl.NS;
             if (lane == 0) {
@@ -488,8 +501,7 @@ __device__ void activation_warp(const Params& p, const Slots& sl, float* big, co
             }
             if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
             if (lane == 0) trace(p, j, kTrCtrWait, global_timer_ns());
-            if (!prep_job<HD>(p, ins, c, sl.slot(j), big, jobs_done, attn_before, lane, epoch, j)) return;
-            if (op == MK_OP_ATTN) attn_before = j + 1;
+            if (!prep_job<HD>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
             if (lane == 0) {
                 trace(p, j, kTrReady, global_timer_ns());
@@ -591,76 +603,6 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
     return true;
 }
 
-// Batch 1: a down instruction is one job over the whole MLP. Its input is the
-// whole vector h (tagged) as four XSmem vectors of F/4 in the `big` region
-// (chunk c at big + c*F/4) -- chunks 0..2 staged by the activation warp, chunk
-// 3 loaded here by all compute warps -- and the residual rows (x after
-// attention). Ends with a compute barrier.
-__device__ bool down_whole_input(const Params& p, const mk_instr& in, float* sv, float* big, int warp, int lane,
-                                 uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
-    const int t = warp * 32 + lane, l = in.layer;
-    if (!rows_tagged(p, p.x_t + (size_t)in.first * 4, act_tag(epoch, l, kTagXAttn), (int)in.count * 4,
-                     slot_resid(p, sv, 0), t, lane))
-        return false;
-    // chunk 3 of h (chunks 0..2 were loaded by the activation warp)
-    const int n4 = p.F / 4, np = n4 / 2;
-    const uint64_t* src = p.h_t + (size_t)3 * n4;
-    float* dst = big + (size_t)3 * n4;
-    const uint32_t tag = act_tag(epoch, l, kTagH);
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        uint64_t a[kMaxPairs], b[kMaxPairs];
-#pragma unroll
-        for (int i = 0; i < kMaxPairs; ++i) {
-            const int j = i * kNT + t;
-            a[i] = b[i] = 0ull;
-            if (j < np) ld_tagged2(src + 2 * j, a[i], b[i]);
-        }
-        bool ok = true;
-#pragma unroll
-        for (int i = 0; i < kMaxPairs; ++i) {
-            const int j = i * kNT + t;
-            if (j < np) {
-                ok = ok & tag_ok(a[i], tag) & tag_ok(b[i], tag);
-                *reinterpret_cast<float2*>(dst + xs_index(n4, 2 * j)) = make_float2(tag_val(a[i]), tag_val(b[i]));
-            }
-        }
-        if (__all_sync(0xffffffffu, ok)) break;
-        if (!tag_backoff(p, it, t0, 6, lane)) return false;
-    }
-    return compute_barrier(p, cbar, cuses, lane);
-}
-
-// The whole-MLP down job: tile k = (row block k / 4, chunk k % 4) goes to warp
-// k mod 8; each tile's four sums wait in `tot`; then each output row adds its
-// chunks in order 0..3 (as the four-job form and the baseline do) and the
-// residual.
-template <int KF>
-__device__ bool compute_down_whole(const Params& p, const Ring& ring, const mk_instr& in, float* sv,
-                                   const float* big, float* tot, int warp, int lane, uint64_t* cbar,
-                                   uint32_t& cuses, uint32_t job, uint32_t epoch) {
-    const int n4 = p.F / 4;
-    const uint32_t ntile = 4 * in.count;
-    for (uint32_t k = warp; k < ntile; k += kConsumerWarps) {
-        const uint32_t c = k % 4, seq = in.seq + k;
-        if (!wait_fill(p, ring, seq, lane)) return false;
-        if (k == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
-        const float4 a4 = tile_dot<KF>(ring.stage(seq), big + (size_t)c * n4, lane);
-        const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
-        if (lane < 4) tot[k * 4 + lane] = pick4(acc, lane);
-        release_fill(ring, seq, lane);
-    }
-    if (!compute_barrier(p, cbar, cuses, lane)) return false;
-    const int t = warp * 32 + lane;
-    if (t < (int)in.count * 4 && in.signal_ctr != MK_NO_COUNTER) {
-        const float* pr = tot + (size_t)(t / 4) * 16 + (t % 4);  // [row block][chunk][row]
-        const float y = ((pr[0] + pr[4]) + pr[8]) + pr[12];
-        st_tagged(p.x_t + (size_t)in.first * 4 + t, __fadd_rn(slot_resid(p, sv, 0)[t], y),
-                  act_tag(epoch, in.layer, kTagXMlp));
-    }
-    return true;
-}
-
 // One attention item as one job of all compute warps (see attn_item_block). Every
 // fill of the item must have landed first: each warp reads all of them. With a
 // single partition per (sequence, group) the item writes o / l for its heads;
@@ -743,21 +685,22 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
 
 template <int KH, int KO, int KF, int HD>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
-                             float* tot, float* red, uint64_t* cbar, volatile uint32_t* jobs_done, int i0, int i1,
-                             int warp, int lane, uint32_t epoch) {
+                             float* tot, float* red, uint64_t* cbar, int i0, int i1, int warp, int lane,
+                             uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
-        const bool whole = in.op == MK_OP_DOWN && in.group == 1;
-        const int njobs = (in.op == MK_OP_DOWN && !whole) ? 4 : 1;
+        const int njobs = (in.op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, sl.full + s, (j / sl.NS) & 1u, nullptr, j, 4, lane)) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrStart, global_timer_ns());
             float* sv = reinterpret_cast<float*>(sl.slot(j));
-            bool ok = in.op == MK_OP_ATTN ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
-                      : whole ? down_whole_input(p, in, sv, scores, warp, lane, cbar, cuses, epoch)
-                              : job_input(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
+            // inputs: the attention item's q/k/v and every matvec input but the
+            // down-projection's (staged by the activation warp) are loaded here
+            bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
+                      : in.op == MK_OP_DOWN ? true
+                                            : job_input(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7, global_timer_ns());
             switch (in.op) {
@@ -765,10 +708,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 case MK_OP_OPROJ: ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
                 case MK_OP_GATEUP:
                 case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
-                case MK_OP_DOWN:
-                    ok = whole ? compute_down_whole<KF>(p, ring, in, sv, scores, tot, warp, lane, cbar, cuses, j, epoch)
-                               : compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
-                    break;
+                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch); break;
                 default:
                     ok = compute_attn_job<HD>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
                                               epoch);
@@ -783,10 +723,9 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 const uint32_t old = atom_shared_acq_rel_add(sl.done + s, 1u);
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
-                    *jobs_done = j + 1;  // every warp is done with jobs 0..j (see prep_job)
                     trace(p, j, kTrDone, global_timer_ns());
                     // attention items signal their heads themselves (compute_attn_job)
-                    const bool last_chunk = (in.op != MK_OP_DOWN || whole || c == 3) && in.op != MK_OP_ATTN;
+                    const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN;
                     if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
                         // QKV / gate-up: one increment on each KV group / MLP chunk counter
                         // the job's tiles touched
@@ -832,9 +771,7 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
         case MK_OP_GATEUP:
             return {p.packed + lbase + p.rel_gu + (size_t)gu_tile(p, in, t) * p.tile_h, nullptr, p.tile_h};
         case MK_OP_DOWN: {
-            // one job over the whole MLP: fills in (row block, chunk) order, which is also
-            // the packed order; four chunk jobs: chunk-major
-            const uint32_t c = in.group == 1 ? t % 4 : t / in.count, r = in.group == 1 ? t / 4 : t % in.count;
+            const uint32_t c = t / in.count, r = t % in.count;  // chunk-major
             return {p.packed + lbase + p.rel_down + ((size_t)(in.first + r) * 4 + c) * p.tile_f, nullptr,
                     p.tile_f};
         }
@@ -972,9 +909,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
     __shared__ volatile uint32_t s_issued;  // fills the loader has issued (all: ~0)
-    __shared__ volatile uint32_t s_jobs_done;  // jobs the compute warps have finished
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, p.big_floats);
+    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes);
     Ring ring;
     ring.base = smem + m.ring;
     ring.full = reinterpret_cast<uint64_t*>(smem + m.full);
@@ -1003,7 +939,6 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         }
         mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
         s_issued = 0u;
-        s_jobs_done = 0u;
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
         uint32_t skip = ld_volatile_u32(&p.ctl->status) != 0u;
@@ -1032,14 +967,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else if (warp == kPrefetchWarp) {
             if (lane == 0) prefetcher(p, i0, i1, ring.S, &s_issued);
         } else if (warp == kPrepWarp) {
-            activation_warp<KH, KO, KF, HD>(p, sl, reinterpret_cast<float*>(smem + m.scores), &s_jobs_done, i0,
-                                            i1, lane, s_epoch);
+            activation_warp<KH, KO, KF, HD>(p, sl, i0, i1, lane, s_epoch);
         } else {
             float* scores = reinterpret_cast<float*>(smem + m.scores);
             compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
                                          reinterpret_cast<float*>(smem + m.red),
-                                         reinterpret_cast<uint64_t*>(smem + m.cbar), &s_jobs_done, i0, i1, warp,
-                                         lane, s_epoch);
+                                         reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
+                                         s_epoch);
         }
     }
     __syncthreads();
@@ -1074,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ------------------------------------------------------------------ host-side launch
 
 size_t megakernel_smem_bytes(const Params& p) {
-    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, p.big_floats).total;
+    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes).total;
 }
 
 using KernelFn = void (*)(Params);

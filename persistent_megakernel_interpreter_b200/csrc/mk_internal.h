@@ -67,7 +67,7 @@ struct Layout {
 struct SmemLayout {
     uint32_t ring, full, empty, armed;        // weight / cached-KV ring of S stages
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
-    uint32_t scores;                          // attention item scratch / whole-MLP down input
+    uint32_t scores;                          // attention item scratch (kAttnScratchFloats)
     uint32_t tot;                             // down-projection running sums
     uint32_t red;                             // per-warp partial sums of a job input
     uint32_t cbar;                            // barrier of the compute warps
@@ -76,9 +76,7 @@ struct SmemLayout {
 
 MK_HD inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
-// big_floats: the floats of the region shared by an attention item's scratch and
-// a whole-MLP down-projection input (batch 1), whichever is larger.
-MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes, uint32_t big_floats) {
+MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes) {
     SmemLayout m;
     uint32_t o = 0;
     m.ring = o;      o += (uint32_t)S * stage_bytes;
@@ -89,7 +87,7 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs_full = o;   o += 8u * NS;
     m.xs_empty = o;  o += 8u * NS;
     m.xs_done = o;   o = align16(o + 4u * NS);
-    m.scores = o;    o += 4u * (big_floats > kAttnScratchFloats ? big_floats : kAttnScratchFloats);
+    m.scores = o;    o += 4u * kAttnScratchFloats;
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
     m.red = o;       o += 4u * 32u;
     m.cbar = o;      o += 8u;
@@ -148,8 +146,6 @@ struct Params {
     int part_keys, n_parts, keys_per_stage;
     uint32_t stage_bytes;
     int n_stages;
-    int down_whole;            // 1: each down instruction is one job over the whole MLP (batch 1)
-    uint32_t big_floats;       // floats of the attention scratch / down input region
     int xs_slots;              // activation slots (1..3)
     uint32_t xs_slot_bytes;
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot

@@ -32,7 +32,6 @@ struct SlotPlan {
     uint32_t vec_floats;   // one sequence's input vector inside a slot
     uint32_t item_bytes;   // an attention item's q and new key/value inside a slot
     uint32_t slot_bytes;
-    uint32_t big_floats;   // attention scratch / whole-MLP down input region (floats)
     int xs_slots;
     int stages;
     uint32_t smem_bytes;

@@ -48,11 +48,9 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     // new key/value.
     sp.slot_bytes = align16(std::max(
         (uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u, sp.item_bytes));
-    // batch 1: a down instruction is one job whose input is the whole MLP vector
-    sp.big_floats = batch == 1 ? (uint32_t)L.F : 0u;
     for (int ns = 3; ns >= 1; --ns) {
         int S = 0;
-        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, sp.big_floats).total + 1024 <= kSmemBudget)
+        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
             ++S;
         if (S >= (ns > 1 ? 6 : 2) || ns == 1) {
             sp.xs_slots = ns;
@@ -60,7 +58,7 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
             break;
         }
     }
-    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes, sp.big_floats).total;
+    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes).total;
     return sp;
 }
 
@@ -249,7 +247,6 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, batch > 1 ? 1 : down_cap,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_DOWN, l);
-                        in.group = batch == 1 ? 1 : 0;  // 1: one job over all four chunks
                         in.first = (uint32_t)a;
                         in.count = (uint32_t)n;
                         in.nfill = 4u * (uint32_t)n;

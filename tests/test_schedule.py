@@ -26,7 +26,7 @@ def jobs_of(lst):
         ins = lst[i]
         items = ins.job_items if ins.op == _lib.OP_ATTN else 1
         assert items >= 1
-        for c in range(4 if (ins.op == _lib.OP_DOWN and ins.group != 1) else 1):
+        for c in range(4 if ins.op == _lib.OP_DOWN else 1):
             jobs.append((i, c, items))
         i += items
     return jobs
@@ -39,8 +39,6 @@ def job_waits(lst, job):
         return [(lst[i + k].wait_ctr, lst[i + k].wait_n) for k in range(items)]
     if ins.op == _lib.OP_DOWN:
         t = [ins.wait_n, ins.aux0 & 0xFFFF, ins.aux0 >> 16, ins.aux1]
-        if ins.group == 1:  # one job over the whole MLP: every chunk
-            return [(ins.wait_ctr + k, t[k]) for k in range(4)]
         return [(ins.wait_ctr + c, t[c])]
     return [] if ins.wait_ctr == NO else [(ins.wait_ctr, ins.wait_n)]
 
@@ -55,8 +53,6 @@ def job_fills(lst, job, w):
         a = lst[i + w]
         return list(range(a.seq, a.seq + a.nfill))
     if ins.op == _lib.OP_DOWN:
-        if ins.group == 1:  # fills in (row block, chunk) order, tile k to warp k mod W
-            return [ins.seq + k for k in range(w, 4 * ins.count, W)]
         return [ins.seq + c * ins.count + r for r in range(w, ins.count, W)]
     return [ins.seq + t for t in range(w, ins.count, W)]
 
@@ -74,7 +70,7 @@ def job_done_signals(L, job, group, n_parts, arr, ctr):
             arr[a.aux0] += group
             if arr[a.aux0] == n_parts * group:
                 ctr[a.signal_ctr] += group
-    elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or ins.group == 1 or c == 3):
+    elif ins.signal_ctr != NO and (ins.op != _lib.OP_DOWN or c == 3):
         span = max(1, ins.aux1) if ins.op in (_lib.OP_QKV, _lib.OP_GATEUP) else 1
         for k in range(span):
             ctr[ins.signal_ctr + k] += 1
