@@ -261,6 +261,41 @@ size_t mk_packed_bytes(const mk_config* cfg);
 mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights* w, void* dst,
                                size_t dst_bytes);
 
+/* The multi-kernel decode step (as mk_baseline_decode_step) for callers that
+ * cannot allocate device memory -- an engine whose device memory is all handed
+ * out by its own arena, or code running where cudaMalloc is not allowed. It
+ * needs no handle and allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library call); the web pages describe no such entry point, it has
+ * no counterpart there. The caller owns every input and output:
+ *   cfg               the model (as for mk_create)
+ *   packed            device, mk_packed_bytes(cfg) bytes in the mk_pack_weights_host
+ *                     layout (e.g. packed on the host and copied by the caller)
+ *   tokens, positions device int32 [batch]
+ *   k_cache, v_cache  device bf16 [n_layers][max_batch][n_kv_heads][max_seq][head_dim]
+ *                     (as for mk_decode_step: reads slots 0..positions[b], writes
+ *                     slot positions[b])
+ *   logits            device fp32 [batch][vocab]
+ *   batch, max_ctx    1 <= batch <= cfg->max_batch; positions[b] + 1 <= max_ctx <=
+ *                     cfg->max_seq
+ *   status_out        device int32 or NULL: receives the step's device status
+ *                     (MK_OK, MK_ERR_BAD_TOKEN, MK_ERR_BAD_POSITION)
+ *   stream            the CUDA stream the step is enqueued on
+ * Scratch (activations, attention partials, the RoPE table of max_ctx
+ * positions, the error word) lives in one 4 MiB device array of the library,
+ * per device, held until the process exits. The first call on a device (with
+ * that device current) looks up the array's device address; a call whose
+ * configuration (rope_theta, head_dim, max_ctx) differs from the previous call's
+ * uploads a new RoPE table from the stack. Make that first call before any
+ * stream capture. Every call shares the array and leaves its contents for the
+ * next; the error word is cleared by each call. Calls that overlap on the GPU
+ * (on different streams, or from different host threads) race on it.
+ * Returns MK_ERR_INVALID_ARG for bad arguments and for a step whose scratch
+ * exceeds the 4 MiB array (about max_ctx <= 8192 at batch 1 for a 1B-shaped
+ * model; more than 32 attention partitions of 320 keys are refused too). */
+mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const void* packed, const int32_t* tokens,
+                                          const int32_t* positions, void* k_cache, void* v_cache, float* logits,
+                                          int batch, int max_ctx, int32_t* status_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
