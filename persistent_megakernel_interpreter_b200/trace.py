@@ -2,11 +2,13 @@
 
 Each job record (see ``mk_read_trace`` in mk.h) holds, in globaltimer
 nanoseconds: the activation warp starting to wait for a free input slot, the
-slot being free, the input counter being reached, the input being ready, compute
-warp 0 starting, and the job's last compute warp finishing. From these the
-summary separates, per op, time spent waiting for other SMs (counter waits),
-preparing inputs, and computing, and gives per layer the moment each op
-finished on its last SM -- the step's critical path.
+slot being free, the activation warp starting its part of the job, its part
+being ready, compute warp 0 starting (its input polled from the producers'
+tagged words inside the compute time), the first weight stage being ready, and
+the job's last compute warp finishing. From these the summary separates, per
+op, slot waits, the activation warp's staging, and compute (with the input
+wait), and gives per layer the moment each op finished on its last SM -- the
+step's critical path.
 """
 from __future__ import annotations
 
