@@ -151,17 +151,23 @@ def aggregate(elapsed_ms: float, units: float, dist, device=None):
     return float(t.item()), float(u.item())
 
 
-def workload_config(n_gpus: int, layers: int = 16, past: int = PAST):
-    name = "Llama-3.2-1B" if layers == 16 else f"Llama-3.2-1B-shaped ({layers} of 16 layers)"
-    return {"workload": f"{name} decoder, one decode step, batch 1, {past} cached positions "
-                        f"({past + 1} keys), random bf16 weights N(0,0.02), KV N(0,1)",
-            "layers": layers, "hidden": 2048, "heads": "32q/8kv x 64", "ffn": 8192, "vocab": 128256,
-            "global_batch": BATCH * n_gpus, "seq_len": past + 1,
+def workload_config(n_gpus: int, layers: int = 16, past: int = PAST, model: str = "1b", batch: int = BATCH):
+    if model == "3b":
+        name = "Llama-3.2-3B-style" if layers == 28 else f"Llama-3.2-3B-style ({layers} of 28 layers)"
+        dims = {"layers": layers, "hidden": 3072, "heads": "24q/8kv x 128", "ffn": 8192, "vocab": 128256}
+        size = "the 6.4 GB of weights"
+    else:
+        name = "Llama-3.2-1B" if layers == 16 else f"Llama-3.2-1B-shaped ({layers} of 16 layers)"
+        dims = {"layers": layers, "hidden": 2048, "heads": "32q/8kv x 64", "ffn": 8192, "vocab": 128256}
+        size = "the 2.47 GB of weights"
+    return {"workload": f"{name} decoder, one decode step, batch {batch}, {past} cached positions "
+                        f"({past + 1} keys) per sequence, random bf16 weights N(0,0.02), KV N(0,1)",
+            **dims, "global_batch": batch * n_gpus, "seq_len": past + 1,
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
-            "l2": "no flush: the 2.47 GB of weights streamed per step exceed the 126 MB L2"}
+            "l2": f"no flush: {size} streamed per step exceed the 126 MB L2"}
 
 
-def time_oracle(cfg, w, k, v, budget_s: float, past: int):
+def time_oracle(cfg, w, k, v, budget_s: float, past: int, batch: int = BATCH):
     """The CPU oracle on this host's cores: full decode steps of the same workload until
     ``budget_s`` has passed (at least one). Returns (tokens/s, steps, threads, s/step)."""
     import numpy as np
@@ -169,17 +175,17 @@ def time_oracle(cfg, w, k, v, budget_s: float, past: int):
     from persistent_megakernel_interpreter_b200.inputs import make_tokens
     om = oracle.Model(cfg, w)
     kc, vc = oracle.bits(k).copy(), oracle.bits(v).copy()
-    toks = make_tokens(cfg, 1, seed=2).numpy()
+    toks = make_tokens(cfg, batch, seed=2).numpy()
     threads = oracle.max_threads()
     n = 0
     t0 = time.perf_counter()
     while True:
-        om.decode_step(toks, np.array([past]), kc, vc, threads=threads)
+        om.decode_step(toks, np.array([past] * batch), kc, vc, threads=threads)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return BATCH * n / el, n, threads, el / n
+    return batch * n / el, n, threads, el / n
 
 
 def run_reference(args):
@@ -230,12 +236,15 @@ def run_mk(args):
     rank, world, local, dist = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    from persistent_megakernel_interpreter_b200.config import LLAMA_1B
+    from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B
     from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
     from persistent_megakernel_interpreter_b200.model import Megakernel
     import dataclasses
-    cfg = dataclasses.replace(LLAMA_1B, n_layers=args.layers) if args.layers != 16 else LLAMA_1B
+    base_cfg = LLAMA_3B if args.model == "3b" else LLAMA_1B
+    layers = args.layers or base_cfg.n_layers
+    cfg = dataclasses.replace(base_cfg, n_layers=layers) if layers != base_cfg.n_layers else base_cfg
     past = args.past
+    BATCH = args.batch
     w = make_weights(cfg, seed=0)
     k, v = make_kv_cache(cfg, BATCH, past + 1, past, seed=1)
     mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=past + 1)
@@ -354,7 +363,7 @@ def run_mk(args):
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
-        val, n, threads, sps = time_oracle(cfg, w, k, v, args.cpu_budget, past)
+        val, n, threads, sps = time_oracle(cfg, w, k, v, args.cpu_budget, past, BATCH)
         cpu = {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} full decode step(s) of this workload, {sps:.2f} s each"}
 
@@ -364,13 +373,16 @@ def run_mk(args):
         achieved = bytes_step / (per_launch_ms * 1e-3) / 1e9
         traffic = profiled_traffic()
         ms_per_step = t_max / args.steps
+        metric = METRIC if (args.model == "1b" and BATCH == 1) else (
+            f"µs/decode step & tokens/s, {'Llama-3B' if args.model == '3b' else 'Llama-1B'}-style bf16 "
+            f"bs{BATCH}; HBM GB/s vs peak")
         line = {
-            "metric": METRIC, "value": units / (t_max * 1e-3), "unit": "tokens/s",
+            "metric": metric, "value": units / (t_max * 1e-3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "us_per_step": 1e3 * ms_per_step,
             "us_per_launch_median": 1e3 * statistics.median(launch_ms),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(world, cfg.n_layers, past),
+            "data": "synthetic", "config": workload_config(world, cfg.n_layers, past, args.model, BATCH),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
                          "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
@@ -395,6 +407,80 @@ def run_mk(args):
         dist.destroy_process_group()
 
 
+def run_greedy(args):
+    """Greedy decoding at batch 1: a 32-token random prompt fed as decode steps into
+    an empty cache, then ``--greedy`` generated tokens, each the argmax of the
+    previous step's logits (taken on the device, outside the timed region). Every
+    step is timed alone with CUDA events around its launch; prints one JSON line
+    with the per-step latency distribution."""
+    import numpy as np
+    import torch
+    from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B
+    from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
+    from persistent_megakernel_interpreter_b200.model import Megakernel
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = LLAMA_3B if args.model == "3b" else LLAMA_1B
+    n_prompt, n_gen = 32, args.greedy
+    steps = n_prompt + n_gen
+    w = make_weights(cfg, seed=0)
+    k, v = make_kv_cache(cfg, 1, steps, 0, seed=1)
+    mk = Megakernel(cfg, w.to(dev), max_batch=1, max_seq=steps)
+    mk.build_schedule(1, steps)
+    kd, vd = k.to(dev), v.to(dev)
+    prompt = make_tokens(cfg, n_prompt, seed=50).to(dev)
+    tok = torch.zeros(1, dtype=torch.int32, device=dev)
+    pos = torch.zeros(1, dtype=torch.int32, device=dev)
+    logits = torch.empty(1, cfg.vocab, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        tok.copy_(prompt[:1])
+        for _ in range(args.warmup):
+            mk.decode_step(tok, pos, kd, vd, logits, stream)
+        kd.zero_()
+        vd.zero_()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with ClockSampler(0) as clocks:
+            for p in range(steps):
+                pos.fill_(p)
+                if p < n_prompt:
+                    tok.copy_(prompt[p:p + 1])
+                else:
+                    tok.copy_(torch.argmax(logits[0]).to(torch.int32).view(1))
+                ev[p][0].record(stream)
+                mk.decode_step(tok, pos, kd, vd, logits, stream)
+                ev[p][1].record(stream)
+            stream.synchronize()
+    code, msg = mk.status()
+    if code != 0:
+        raise RuntimeError(f"greedy decode failed: {msg}")
+    us = np.array([1e3 * a.elapsed_time(b) for a, b in ev])
+    gen = us[n_prompt:]
+    peak, peak_kind = hbm_peak()
+    line = {
+        "metric": "µs per decode step, greedy decode at batch 1 (each step timed alone)",
+        "value": 1e6 / float(gen.mean()), "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{'Llama-3.2-3B-style' if args.model == '3b' else 'Llama-3.2-1B'} decoder, "
+                               f"greedy decode of {n_gen} tokens after a {n_prompt}-token random prompt "
+                               f"fed as decode steps into an empty cache, batch 1"},
+        "per_step_us": {"generated_mean": float(gen.mean()), "generated_median": float(np.median(gen)),
+                        "generated_p10": float(np.percentile(gen, 10)),
+                        "generated_p90": float(np.percentile(gen, 90)),
+                        "first_prompt_step": float(us[0]), "last_step": float(us[-1]),
+                        "prompt_mean": float(us[:n_prompt].mean())},
+        "roofline_last_step": {"bound": "hbm", "achieved": cfg.step_bytes(1, steps - 1) / (us[-1] * 1e-6) / 1e9,
+                               "peak": peak, "unit": "GB/s",
+                               "frac": cfg.step_bytes(1, steps - 1) / (us[-1] * 1e-6) / 1e9 / peak,
+                               "peak_source": peak_kind},
+        "gpu_launches": steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    mk.close()
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -404,7 +490,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-baseline", action="store_true")
-    ap.add_argument("--layers", type=int, default=16,
+    ap.add_argument("--model", choices=["1b", "3b"], default="1b",
+                    help="1b: the Llama-3.2-1B shape (default); 3b: the 3B-style shape")
+    ap.add_argument("--batch", type=int, default=BATCH, help="sequences per step")
+    ap.add_argument("--layers", type=int, default=0,
                     help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
                          "small profiling captures of the same kernels)")
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
@@ -413,6 +502,9 @@ def parse_args(argv=None):
     ap.add_argument("--l2-evict-normal", action="store_true",
                     help="L2 prefetches with an evict-normal hint (default: evict-last)")
     ap.add_argument("--max-inflight", type=int, default=0, help="ring fills in flight at most (0 = default)")
+    ap.add_argument("--greedy", type=int, default=0, metavar="N",
+                    help="instead of the step benchmark: greedy-decode N tokens after a 32-token "
+                         "prompt at batch 1 and report the per-step latency")
     ap.add_argument("--trace", default=None, metavar="FILE",
                     help="after the timed run, trace one step's per-job timestamps and save "
                          "them (.npy) with a text summary beside them")
@@ -426,6 +518,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.greedy:
+        run_greedy(args)
     else:
         run_mk(args)
 

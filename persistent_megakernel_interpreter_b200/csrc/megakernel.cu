@@ -526,6 +526,21 @@ __device__ __noinline__ float4 tile_dot(const uint8_t* tile, const float* v, int
     return make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
+// The tile against every sequence's input (B > 1): lane l returns the total of
+// sequence l / 4, row l % 4 (see dot4_batch).
+template <int KC>
+__device__ __noinline__ float tile_dot_batch(const uint8_t* tile, const float* sv, uint32_t vec_floats, int B,
+                                             int lane) {
+    return dot4_batch<KC>(tile, sv, vec_floats, B, lane);
+}
+
+// The four rows of sequence lane / 4 gathered from the batched totals, for the
+// 4-row epilogues (lane l then acts as lane l % 4 of sequence l / 4).
+__device__ __forceinline__ void gather4(float tot, int lane, float (&acc)[4]) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r] = __shfl_sync(0xffffffffu, tot, (lane & ~3) + r);
+}
+
 template <int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
                               const float* sv, int warp, int lane, uint32_t job, uint32_t epoch) {
@@ -542,30 +557,45 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
         if (t == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
         if (k < 2) stamp(3 * k + 1);
         const uint8_t* tile = ring.stage(seq);
-        for (int b = 0; b < p.B; ++b) {
-            const float4 a4 = tile_dot<KC>(tile, sv + (size_t)b * p.xs_vec_floats, lane);
-            if (k < 2 && b == 0) stamp(3 * k + 2);
-            const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
+        // batch 1: one pass, every lane holds the 4 totals; batch > 1: one pass over
+        // all sequences, lane l holds sequence l / 4 and acts as lane l % 4 for it
+        const bool batched = p.B > 1;
+        float tb = 0.f;
+        if (batched) tb = tile_dot_batch<KC>(tile, sv, p.xs_vec_floats, p.B, lane);
+        const int nb = batched ? 1 : p.B;
+        for (int bi = 0; bi < nb; ++bi) {
+            int b = bi, el = lane;
+            float acc[4];
+            if (batched) {
+                gather4(tb, lane, acc);
+                b = lane >> 2;
+                el = b < p.B ? (lane & 3) : 32;
+                if (b >= p.B) b = 0;
+            } else {
+                const float4 a4 = tile_dot<KC>(tile, sv + (size_t)b * p.xs_vec_floats, lane);
+                acc[0] = a4.x; acc[1] = a4.y; acc[2] = a4.z; acc[3] = a4.w;
+            }
+            if (k < 2 && bi == 0) stamp(3 * k + 2);
             const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
             switch (in.op) {
                 case MK_OP_QKV: {
                     const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
                     const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
-                    if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, lane, rr, act_tag(epoch, in.layer, kTagQKV));
+                    if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, el, rr, act_tag(epoch, in.layer, kTagQKV));
                     break;
                 }
                 case MK_OP_GATEUP:
-                    if (pub) gateup_epilogue<true>(p, b, tl, acc, lane, act_tag(epoch, in.layer, kTagH));
+                    if (pub) gateup_epilogue<true>(p, b, tl, acc, el, act_tag(epoch, in.layer, kTagH));
                     break;
                 case MK_OP_OPROJ:
                     // x = x_in + W_o attn for the tile's rows; x_in waits in the slot
-                    if (pub && lane < 4) {
-                        const float xin = slot_resid(p, const_cast<float*>(sv), b)[(tl - in.first) * 4 + lane];
-                        st_tagged(p.x_t + (size_t)b * p.H + tl * 4 + lane, __fadd_rn(xin, pick4(acc, lane)),
+                    if (pub && el < 4) {
+                        const float xin = slot_resid(p, const_cast<float*>(sv), b)[(tl - in.first) * 4 + el];
+                        st_tagged(p.x_t + (size_t)b * p.H + tl * 4 + el, __fadd_rn(xin, pick4(acc, el)),
                                   act_tag(epoch, in.layer, kTagXAttn));
                     }
                     break;
-                default: logits_epilogue(p, b, tl, acc, lane); break;
+                default: logits_epilogue(p, b, tl, acc, el); break;
             }
         }
         release_fill(ring, seq, lane);
@@ -584,16 +614,29 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
         if (r == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
-        for (int b = 0; b < p.B; ++b) {
-            const float4 a4 = tile_dot<KF>(ring.stage(seq), sv + (size_t)b * p.xs_vec_floats, lane);
-            const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
-            if (lane < 4) {
-                float* t = tot + ((size_t)r * p.B + b) * 4 + lane;
-                const float y = pick4(acc, lane);
+        // batch > 1: one pass over all sequences, lane l holds sequence l / 4, row l % 4
+        const bool batched = p.B > 1;
+        float tb = 0.f;
+        if (batched) tb = tile_dot_batch<KF>(ring.stage(seq), sv, p.xs_vec_floats, p.B, lane);
+        const int nb = batched ? 1 : p.B;
+        for (int bi = 0; bi < nb; ++bi) {
+            int b = bi, row = lane;
+            float y = 0.f;
+            if (batched) {
+                b = lane >> 2;
+                row = b < p.B ? (lane & 3) : 32;
+                y = tb;
+            } else {
+                const float4 a4 = tile_dot<KF>(ring.stage(seq), sv + (size_t)b * p.xs_vec_floats, lane);
+                const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
+                if (lane < 4) y = pick4(acc, lane);
+            }
+            if (row < 4) {
+                float* t = tot + ((size_t)r * p.B + b) * 4 + row;
                 *t = (c == 0) ? y : *t + y;
                 if (c == 3 && in.signal_ctr != MK_NO_COUNTER) {  // x = x_in + W_d h; x_in waits in the slot
-                    const float xin = slot_resid(p, const_cast<float*>(sv), b)[r * 4 + lane];
-                    st_tagged(p.x_t + (size_t)b * p.H + (in.first + r) * 4 + lane, __fadd_rn(xin, *t),
+                    const float xin = slot_resid(p, const_cast<float*>(sv), b)[r * 4 + row];
+                    st_tagged(p.x_t + (size_t)b * p.H + (in.first + r) * 4 + row, __fadd_rn(xin, *t),
                               act_tag(epoch, in.layer, kTagXMlp));
                 }
             }

@@ -521,6 +521,53 @@ __device__ __forceinline__ void dot4(const uint8_t* tile, const X& x, float (&ac
     for (int r = 0; r < 4; ++r) acc[r] = warp_sum(acc[r]);
 }
 
+// The 4-row tile in shared memory against the input vectors of B <= kMaxBatch
+// sequences (XSmem layout, sequence b at xs + b * vec_floats): each 16-byte
+// weight piece is read and unpacked once and applied to every sequence. Each
+// (sequence, row) total comes from the same lane chains as dot4's and the same
+// xor tree (16, 8, 4, 2, 1) as warp_sum, so it equals dot4's total for that
+// sequence bit for bit; the tree is run as a reduce-scatter, after which lane l
+// holds the total of sequence l / 4, row l % 4 (sequences >= B: zero).
+template <int KC>
+__device__ __forceinline__ float dot4_batch(const uint8_t* tile, const float* xs, uint32_t vec_floats, int B,
+                                            int lane) {
+    const uint4* t = reinterpret_cast<const uint4*>(tile) + lane;
+    float v[kMaxBatch * 4];
+#pragma unroll
+    for (int i = 0; i < kMaxBatch * 4; ++i) v[i] = 0.f;
+#pragma unroll 1
+    for (int kc = 0; kc < KC; ++kc) {
+        float w[4][8];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) unpack8(lds_v4(t + r * KC * 32 + kc * 32), w[r]);
+#pragma unroll
+        for (int b = 0; b < kMaxBatch; ++b) {
+            if (b < B) {
+                const float4* x = reinterpret_cast<const float4*>(xs + (size_t)b * vec_floats);
+                const float4 lo = x[kc * 32 + lane], hi = x[KC * 32 + kc * 32 + lane];
+                const float e[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[b * 4 + r] = fmaf(w[r][i], e[i], v[b * 4 + r]);
+            }
+        }
+    }
+    // reduce-scatter: at mask m the lane keeps the half of its values whose index
+    // bit matches its lane bit, adding the partner lane's partial of each
+#pragma unroll
+    for (int m = 16, n = 16; m > 0; m >>= 1, n >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float keep = up ? v[n + i] : v[i];
+            const float send = up ? v[i] : v[n + i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return v[0];
+}
+
 // ------------------------------------------------------------------ per-op helpers
 
 __device__ __forceinline__ const uint16_t* norm_ptr(const Params& p, size_t off) {

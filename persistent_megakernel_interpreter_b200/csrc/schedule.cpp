@@ -244,7 +244,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                 start += n;
             }
         }
-        emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, batch > 1 ? 1 : down_cap,
+        emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, down_cap,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_DOWN, l);
                         in.first = (uint32_t)a;
