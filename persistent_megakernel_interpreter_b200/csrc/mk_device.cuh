@@ -772,13 +772,13 @@ __device__ __forceinline__ const uint16_t* attn_row(const AttnRows<HD>& R, uint3
 // memory; bar(): barrier of the compute warps (false: give up); mark(k): trace
 // hook. R.jnew must be -1 or n - 1. On success emit(h, d, o, M_h, l_h) runs once
 // for every output dim d < HD of every head h < G, on the thread that holds it.
-template <int HD, class Bar, class Mark, class Emit>
+template <int HD, int PBS = 4, int PBV = 4, class Bar, class Mark, class Emit>
 __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const float* qs, int G, float* sc,
                                                 int warp, int lane, Bar&& bar, Mark&& mark, Emit&& emit) {
     using S = AttnShape<HD>;
     constexpr int NT = 32 * kConsumerWarps;
     constexpr int KQ = S::KQ;
-    constexpr int PB = 4;  // warp passes / value keys per batch
+    // PBS: warp passes per batch of the scores; PBV: keys per batch of the values
     float4* et = reinterpret_cast<float4*>(sc + kAttnE);
     float4* wmax = reinterpret_cast<float4*>(sc + kAttnWMax);
     float4* wsum = reinterpret_cast<float4*>(sc + kAttnWSum);
@@ -808,18 +808,18 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         const int j_first = warp * S::KPW + kk;
         const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
         float mx = -INFINITY;
-        for (int j0 = j_first; j0 - kk < n; j0 += PB * KPR) {
-            float acc[PB][kMaxGroup];
-            float kv[PB][8];
+        for (int j0 = j_first; j0 - kk < n; j0 += PBS * KPR) {
+            float acc[PBS][kMaxGroup];
+            float kv[PBS][8];
 #pragma unroll
-            for (int i = 0; i < PB; ++i) {
+            for (int i = 0; i < PBS; ++i) {
                 const int j = j0 + i * KPR;
                 // rows past the fills read the new key (a valid stand-in; masked below)
                 const uint16_t* kr = j < nc ? attn_row<HD>(R, m, j) : R.knew;
                 unpack8(lds_v4(kr + dc * 8), kv[i]);
             }
 #pragma unroll
-            for (int i = 0; i < PB; ++i)
+            for (int i = 0; i < PBS; ++i)
 #pragma unroll
                 for (int h = 0; h < kMaxGroup; ++h) {
                     acc[i][h] = 0.f;
@@ -828,13 +828,13 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
                 }
             if (S::LPK == 16) {
 #pragma unroll
-                for (int i = 0; i < PB; ++i)
+                for (int i = 0; i < PBS; ++i)
 #pragma unroll
                     for (int h = 0; h < kMaxGroup; ++h) acc[i][h] += __shfl_xor_sync(0xffffffffu, acc[i][h], 8);
             }
             const bool b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
-            for (int i = 0; i < PB; ++i) {
+            for (int i = 0; i < PBS; ++i) {
                 const float k0 = b2 ? acc[i][2] : acc[i][0], k1 = b2 ? acc[i][3] : acc[i][1];
                 const float s0 = b2 ? acc[i][0] : acc[i][2], s1 = b2 ? acc[i][1] : acc[i][3];
                 const float m0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 4);
@@ -844,7 +844,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
                 acc[i][0] = v + __shfl_xor_sync(0xffffffffu, v, 1);
             }
 #pragma unroll
-            for (int i = 0; i < PB; ++i) {
+            for (int i = 0; i < PBS; ++i) {
                 const int j = j0 + i * KPR;
                 const float s = __fmul_rn(acc[i][0], scale);
                 if (j < n && hh < G) {
@@ -900,11 +900,11 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         for (int h = 0; h < kMaxGroup; ++h) a[h][0] = a[h][1] = 0.f;
         const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
         const size_t vofs = (size_t)R.kps * HD;
-        for (int j0 = kq; j0 < nc; j0 += PB * KQ) {
-            uint32_t w[PB];
-            float4 e[PB];
+        for (int j0 = kq; j0 < nc; j0 += PBV * KQ) {
+            uint32_t w[PBV];
+            float4 e[PBV];
 #pragma unroll
-            for (int i = 0; i < PB; ++i) {
+            for (int i = 0; i < PBV; ++i) {
                 const int j = j0 + i * KQ;
                 const bool ok = j < nc;
                 const uint16_t* vr = ok ? attn_row<HD>(R, m, j) + vofs : R.vnew;  // stand-in, masked
@@ -912,7 +912,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
                 e[i] = et[ok ? j : 0];
             }
 #pragma unroll
-            for (int i = 0; i < PB; ++i) {
+            for (int i = 0; i < PBV; ++i) {
                 if (j0 + i * KQ >= nc) e[i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 const float v0 = bf_lo(w[i]), v1 = bf_hi(w[i]);
                 a[0][0] = fmaf(e[i].x, v0, a[0][0]); a[0][1] = fmaf(e[i].x, v1, a[0][1]);

@@ -190,14 +190,20 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         for (uint32_t k = 0; k < in.aux1; ++k) signals[in.signal_ctr + k]++;
                         return in;
                     });
-        // attention items, each its own job on the least-loaded SM
+        // attention items, each its own job on the SM with the fewest items of
+        // this layer so far, then the least-loaded one: an SM that runs two items
+        // runs them one after the other, on the layer's critical path
+        std::vector<int> n_att(n_sm, 0);
         for (int b = 0; b < batch; ++b)
             for (int g = 0; g < L.nkv; ++g)
                 for (int j = 0; j < n_parts; ++j) {
                     int best = 0;
                     for (int s = 1; s < n_sm; ++s)
-                        if (load[s] < load[best] || (load[s] == load[best] && rank[s] < rank[best]))
+                        if (n_att[s] < n_att[best] ||
+                            (n_att[s] == n_att[best] &&
+                             (load[s] < load[best] || (load[s] == load[best] && rank[s] < rank[best]))))
                             best = s;
+                    n_att[best]++;
                     mk_instr in = mk_in(MK_OP_ATTN, l);
                     in.batch = (uint16_t)b;
                     in.group = (uint16_t)g;
