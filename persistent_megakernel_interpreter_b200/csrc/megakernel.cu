@@ -360,6 +360,25 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
     return true;
 }
 
+// A down-projection chunk's inputs at batch > 1, by all compute warps: h chunk c
+// of every sequence and, with the last chunk, the residual rows (x after
+// attention). At batch 1 the activation warp stages them ahead instead (one
+// warp moves one sequence's chunk in time; eight sequences' it does not).
+__device__ __forceinline__ bool down_input_batch(const Params& p, const mk_instr& in, int c, float* sv, float* red,
+                                              int warp, int lane, uint64_t* cbar, uint32_t& cuses,
+                                              uint32_t epoch) {
+    const int t = warp * 32 + lane, l = in.layer;
+    for (int b = 0; b < p.B; ++b) {
+        if (c == 3 && !rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4, act_tag(epoch, l, kTagXAttn),
+                                   (int)in.count * 4, slot_resid(p, sv, b), t, lane))
+            return false;
+        if (!block_input_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
+                                nullptr, p.F / 4, sv + (size_t)b * p.xs_vec_floats, red, t, warp, lane, cbar, cuses))
+            return false;
+    }
+    return true;
+}
+
 // An attention item's inputs, by the compute warps: q of the group's heads
 // (fp32) and the step's new key and value (bf16) into the slot. Ends with a
 // compute barrier.
@@ -437,13 +456,13 @@ __device__ bool warp_load_tagged(const Params& p, const uint64_t* src, uint32_t 
 // sequence's position (constant during the step) in the slot. It waits on no
 // dependency: the compute warps poll the tagged inputs themselves, which saves
 // the round trip of a counter read on every hop.
-template <int HD>
+template <int HD, bool BATCHED>
 __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* slot, int lane, uint32_t epoch,
                          uint32_t job) {
     const mk_instr& in = ins[0];
     float* sv = reinterpret_cast<float*>(slot);
     if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
-    if (in.op == MK_OP_DOWN) {
+    if (!BATCHED && in.op == MK_OP_DOWN) {
         // down chunk c: h chunk c (gate/up runs chunk-major, so chunks complete one
         // after another while gate/up still streams) and, with the last chunk, the
         // residual rows (x after attention), staged ahead of the compute warps
@@ -486,7 +505,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
     return true;
 }
 
-template <int KH, int KO, int KF, int HD>
+template <int KH, int KO, int KF, int HD, bool BATCHED>
 __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1, int lane, uint32_t epoch) {
     uint32_t j = 0;
     for (int i = i0; i < i1;) {
@@ -501,7 +520,7 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
             }
             if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
             if (lane == 0) trace(p, j, kTrCtrWait, global_timer_ns());
-            if (!prep_job<HD>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
+            if (!prep_job<HD, BATCHED>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
             if (lane == 0) {
                 trace(p, j, kTrReady, global_timer_ns());
@@ -726,7 +745,7 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     return true;
 }
 
-template <int KH, int KO, int KF, int HD>
+template <int KH, int KO, int KF, int HD, bool BATCHED>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
                              float* tot, float* red, uint64_t* cbar, int i0, int i1, int warp, int lane,
                              uint32_t epoch) {
@@ -740,9 +759,11 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             if (warp == 0 && lane == 0) trace(p, j, kTrStart, global_timer_ns());
             float* sv = reinterpret_cast<float*>(sl.slot(j));
             // inputs: the attention item's q/k/v and every matvec input but the
-            // down-projection's (staged by the activation warp) are loaded here
+            // down-projection's at batch 1 (staged by the activation warp) are
+            // loaded here
             bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
-                      : in.op == MK_OP_DOWN ? true
+                      : in.op == MK_OP_DOWN ? (!BATCHED || down_input_batch(p, in, c, sv, red, warp, lane, cbar,
+                                                                            cuses, epoch))
                                             : job_input(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7, global_timer_ns());
@@ -947,7 +968,7 @@ __device__ void prefetcher(const Params& p, int i0, int i1, uint32_t S, const vo
 
 // ------------------------------------------------------------------ the kernel
 
-template <int KH, int KO, int KF, int HD>
+template <int KH, int KO, int KF, int HD, bool BATCHED>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
@@ -1010,10 +1031,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else if (warp == kPrefetchWarp) {
             if (lane == 0) prefetcher(p, i0, i1, ring.S, &s_issued);
         } else if (warp == kPrepWarp) {
-            activation_warp<KH, KO, KF, HD>(p, sl, i0, i1, lane, s_epoch);
+            activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch);
         } else {
             float* scores = reinterpret_cast<float*>(smem + m.scores);
-            compute_warp<KH, KO, KF, HD>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
+            compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
                                          reinterpret_cast<float*>(smem + m.red),
                                          reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
                                          s_epoch);
@@ -1056,34 +1077,42 @@ size_t megakernel_smem_bytes(const Params& p) {
 
 using KernelFn = void (*)(Params);
 
-static KernelFn pick(int KH, int KO, int KF, int HD) {
-    if (KH == 2 && KO == 2 && KF == 2 && HD == 64) return megakernel<2, 2, 2, 64>;
-    if (KH == 8 && KO == 8 && KF == 8 && HD == 64) return megakernel<8, 8, 8, 64>;
-    if (KH == 12 && KO == 12 && KF == 8 && HD == 128) return megakernel<12, 12, 8, 128>;
+// One kernel per shape and per batch class: only the batch > 1 kernel carries the
+// compute warps' down-chunk loads (at batch 1 they would change the batch-1
+// kernel's register allocation and cost it a few microseconds per step).
+template <bool BATCHED>
+static KernelFn pick_b(int KH, int KO, int KF, int HD) {
+    if (KH == 2 && KO == 2 && KF == 2 && HD == 64) return megakernel<2, 2, 2, 64, BATCHED>;
+    if (KH == 8 && KO == 8 && KF == 8 && HD == 64) return megakernel<8, 8, 8, 64, BATCHED>;
+    if (KH == 12 && KO == 12 && KF == 8 && HD == 128) return megakernel<12, 12, 8, 128, BATCHED>;
     return nullptr;
+}
+
+static KernelFn pick(int KH, int KO, int KF, int HD, int B) {
+    return B > 1 ? pick_b<true>(KH, KO, KF, HD) : pick_b<false>(KH, KO, KF, HD);
 }
 
 bool megakernel_supported(int H, int Q, int F, int d) {
     if (H % 256 || Q % 256 || F % 1024) return false;
-    return pick(H / 256, Q / 256, F / 1024, d) != nullptr;
+    return pick(H / 256, Q / 256, F / 1024, d, 1) != nullptr;
 }
 
 cudaError_t megakernel_prepare(const Params& p) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d);
+    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
     if (!fn) return cudaErrorInvalidValue;
     return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)megakernel_smem_bytes(p));
 }
 
 cudaError_t megakernel_occupancy(const Params& p, int* blocks_per_sm) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d);
+    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
     if (!fn) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, fn, kThreads,
                                                          megakernel_smem_bytes(p));
 }
 
 cudaError_t megakernel_launch(const Params& p, cudaStream_t stream) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d);
+    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
     if (!fn) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.n_sm);
