@@ -263,3 +263,41 @@ def test_partition_count(cfg, batch, ctx, parts):
     assert info.part_keys <= max_item
     assert (info.n_parts * batch * cfg.n_kv_heads <= 148
             or info.part_keys == max_item // info.keys_per_stage * info.keys_per_stage)
+
+
+@pytest.mark.parametrize("cfg,batch,ctx", [
+    (LLAMA_1B, 1, 129), (LLAMA_1B, 1, 4097), (LLAMA_1B, 1, 8193), (LLAMA_3B, 8, 2049), (TINY, 3, 200),
+])
+def test_attention_items_spread_over_sms(cfg, batch, ctx):
+    """An SM runs its attention items one after the other, so within a layer no
+    SM gets a second item before every SM has one (the layer's attention ends
+    with its slowest SM)."""
+    instrs, offs, info = plan_schedule(cfg, batch, ctx, 148, max_batch=8, max_seq=ctx)
+    per_layer = collections.defaultdict(lambda: collections.Counter())
+    for s in range(148):
+        for ins in instrs[offs[s]:offs[s + 1]]:
+            if ins.op == _lib.OP_ATTN:
+                per_layer[ins.layer][s] += 1
+    items = batch * cfg.n_kv_heads * info.n_parts
+    for layer, cnt in per_layer.items():
+        assert sum(cnt.values()) == items
+        assert max(cnt.values()) == -(-items // 148), (layer, max(cnt.values()))
+        if items >= 148:
+            assert len(cnt) == 148
+
+
+@pytest.mark.parametrize("cfg,batch", [(LLAMA_1B, 1), (LLAMA_3B, 8), (TINY, 2)])
+def test_down_instructions_cover_row_block_ranges(cfg, batch):
+    """Down-projection instructions take contiguous ranges of up to 16 row blocks
+    at every batch size (each chunk's input is loaded once per instruction), and
+    together cover every row block of every layer exactly once."""
+    instrs, offs, _ = plan_schedule(cfg, batch, 129, 148, max_batch=8, max_seq=129)
+    for layer in range(cfg.n_layers):
+        seen = []
+        for ins in instrs:
+            if ins.op == _lib.OP_DOWN and ins.layer == layer:
+                assert 1 <= ins.count <= 16 and ins.nfill == 4 * ins.count
+                seen.extend(range(ins.first, ins.first + ins.count))
+        assert sorted(seen) == list(range(cfg.hidden // 4))
+    n_down = sum(1 for ins in instrs if ins.op == _lib.OP_DOWN)
+    assert n_down <= cfg.n_layers * 148 + cfg.n_layers * (cfg.hidden // 4) // 16
