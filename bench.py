@@ -256,6 +256,8 @@ def run_mk(args):
         sched_opts["l2_prefetch_policy"] = 1
     if args.max_inflight:
         sched_opts["max_inflight"] = args.max_inflight
+    if args.part_keys:
+        sched_opts["part_keys"] = args.part_keys
     info = mk.build_schedule(BATCH, past + 1, **sched_opts)
     kd, vd = k.to(dev), v.to(dev)
     tokens = make_tokens(cfg, BATCH, seed=2).to(dev)
@@ -426,7 +428,7 @@ def run_greedy(args):
     w = make_weights(cfg, seed=0)
     k, v = make_kv_cache(cfg, 1, steps, 0, seed=1)
     mk = Megakernel(cfg, w.to(dev), max_batch=1, max_seq=steps)
-    mk.build_schedule(1, steps)
+    mk.build_schedule(1, steps, **({"part_keys": args.part_keys} if args.part_keys else {}))
     kd, vd = k.to(dev), v.to(dev)
     prompt = make_tokens(cfg, n_prompt, seed=50).to(dev)
     tok = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -502,6 +504,8 @@ def parse_args(argv=None):
     ap.add_argument("--l2-evict-normal", action="store_true",
                     help="L2 prefetches with an evict-normal hint (default: evict-last)")
     ap.add_argument("--max-inflight", type=int, default=0, help="ring fills in flight at most (0 = default)")
+    ap.add_argument("--part-keys", type=int, default=0,
+                    help="keys per attention partition (0 = the schedule builder's choice)")
     ap.add_argument("--greedy", type=int, default=0, metavar="N",
                     help="instead of the step benchmark: greedy-decode N tokens after a 32-token "
                          "prompt at batch 1 and report the per-step latency")

@@ -77,13 +77,15 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const int attn_classes = std::max(1, 32 * kConsumerWarps / (L.d / 2));
     if (kps % attn_classes) return MK_ERR_UNSUPPORTED;
 
-    // attention partitions: one per (sequence, KV group) up to kKeysPerItem keys,
-    // more for longer contexts, but no more items than SMs (and at most
-    // kMaxParts per pair, the merge's limit). An item's fills must all sit in the
+    // attention partitions: one per (sequence, KV group) up to kSingleItemKeys
+    // keys; for longer contexts as many as there are SMs for (an item's time is
+    // mostly per key, and the merge of several partitions costs about as much as
+    // ~340 keys of one item, measured), but no more items than SMs and at most
+    // kMaxParts per pair, the merge's limit. An item's fills must all sit in the
     // ring at once and its scores in the item scratch, so a partition holds at
     // most min(kMaxItemKeys, stages * keys_per_stage) keys. A partition is a
     // multiple of 8 keys up to one ring stage, then a multiple of whole stages.
-    constexpr int kKeysPerItem = 256;
+    constexpr int kSingleItemKeys = 320;
     const int max_item = std::min(kMaxItemKeys, sp.stages * kps);
     int part_keys;
     if (o.part_keys > 0) {
@@ -93,7 +95,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     } else {
         const int pairs = batch * L.nkv;
         const int cap = std::max(1, std::min(kMaxParts, n_sm / pairs));
-        int parts = std::max(1, std::min(cap, (max_ctx + kKeysPerItem - 1) / kKeysPerItem));
+        int parts = max_ctx > kSingleItemKeys ? cap : 1;
         parts = std::max(parts, (max_ctx + max_item - 1) / max_item);
         const int want = std::max((max_ctx + parts - 1) / parts, (max_ctx + kMaxParts - 1) / kMaxParts);
         part_keys = want <= kps ? (want + 7) / 8 * 8 : (want + kps - 1) / kps * kps;

@@ -250,13 +250,14 @@ def test_dropped_item_cannot_complete():
 
 
 @pytest.mark.parametrize("cfg,batch,ctx,parts", [
-    (LLAMA_1B, 1, 129, 1), (LLAMA_1B, 1, 1025, 5), (LLAMA_1B, 1, 8193, 17), (LLAMA_3B, 8, 2049, 11),
-    (TINY, 1, 129, 1),
+    (LLAMA_1B, 1, 129, 1), (LLAMA_1B, 1, 288, 1), (LLAMA_1B, 1, 512, 16), (LLAMA_1B, 1, 1025, 17),
+    (LLAMA_1B, 1, 2048, 16), (LLAMA_1B, 1, 8193, 17), (LLAMA_3B, 8, 2049, 11), (TINY, 1, 129, 1),
 ])
 def test_partition_count(cfg, batch, ctx, parts):
-    """One partition per (sequence, group) up to 256 keys, more for longer
-    contexts; no more items than SMs unless a partition is already as long as an
-    item may be (all its fills in the ring at once, at most 512 keys)."""
+    """One partition per (sequence, group) up to 320 keys; for longer contexts as
+    many as fit one item per SM; more items than SMs only when a partition is
+    already as long as an item may be (all its fills in the ring at once, at most
+    512 keys)."""
     _, _, info = plan_schedule(cfg, batch, ctx, 148, max_batch=8, max_seq=ctx)
     assert info.n_parts == parts
     max_item = min(512, info.n_stages * info.keys_per_stage)
