@@ -129,6 +129,14 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         std::shuffle(rank.begin(), rank.end(), rng);
     }
     constexpr uint64_t kJobOverhead = 4096;  // byte-equivalent cost of one job's sync and prep
+    // Byte-equivalent cost of running an attention item, besides its KV bytes, when
+    // a layer has few items: while the item's SM computes it (and its ring holds KV
+    // fills), the other SMs' rings fill with the layer's gate/up weights, so the
+    // item's SM should take fewer of them. Measured on the 1B step at 128 positions
+    // (8 items): 0 / 32 / 64 / 128 / 256 KB -> 692 / 682 / 683 / 680 / 688 us. With
+    // an item on (nearly) every SM the charge only overloads the SMs without one
+    // (1B at 8192 positions: 900 -> 987 us), so it applies to few items only.
+    const uint64_t attn_item_cost = (uint64_t)batch * L.nkv * n_parts * 8 <= (uint64_t)n_sm ? 128 * 1024 : 0;
     using Key = std::pair<uint64_t, uint32_t>;  // (load, rank)
     std::vector<int> sm_of_rank(n_sm);
     for (int s = 0; s < n_sm; ++s) sm_of_rank[rank[s]] = s;
@@ -216,7 +224,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     in.signal_ctr = (uint32_t)c_part[l];
                     in.aux0 = (uint32_t)(c_arr[l] + b * L.nkv + g);
                     lists[best].push_back(in);
-                    load[best] += (uint64_t)in.count * kv_key_bytes + kJobOverhead;
+                    load[best] += (uint64_t)in.count * kv_key_bytes + kJobOverhead + attn_item_cost;
                 }
         // each (sequence, group) pair signals each of its query heads once, when
         // the head's output is final

@@ -225,10 +225,13 @@ def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm):
 
 
 def test_balance_1b():
+    """Streamed bytes per SM within 3% of the mean: placement balances bytes plus a
+    fixed charge per attention item (the SMs that run attention take fewer gate/up
+    tiles of that layer), so the bytes alone are not exactly even."""
     _, _, info = plan_schedule(LLAMA_1B, 1, 129, 148, max_seq=129)
     mean = info.bytes_per_step / 148
-    assert info.max_sm_bytes <= mean * 1.02
-    assert info.min_sm_bytes >= mean * 0.98
+    assert info.max_sm_bytes <= mean * 1.03
+    assert info.min_sm_bytes >= mean * 0.97
     assert info.stage_bytes == 16384 and info.n_stages >= 10
 
 
