@@ -91,13 +91,16 @@ typedef struct mk_schedule_opts {
     int32_t n_sm;            /* SMs to use (<= device SMs); 0 = all */
     int32_t part_keys;       /* keys per attention partition (a multiple of 8 up to the
                                 ring's keys-per-stage, else a multiple of it); 0 = one
-                                partition per (sequence, KV group) up to 256 keys, more
-                                for longer contexts while the items fit on the SMs */
-    int32_t tiles_qkv;       /* 4-row tiles per instruction, per op; 0 = defaults */
-    int32_t tiles_o;
-    int32_t tiles_gateup;
-    int32_t rowblocks_down;
-    int32_t tiles_lm;
+                                partition per (sequence, KV group) up to 320 keys, beyond
+                                that as many as leave one item per SM (each of at most
+                                512 keys and what the ring holds) */
+    int32_t tiles_qkv;       /* reserved, ignored (QKV, O-proj, gate/up and the LM head
+                                are placed one job per SM per op) */
+    int32_t tiles_o;         /* reserved, ignored */
+    int32_t tiles_gateup;    /* reserved, ignored */
+    int32_t rowblocks_down;  /* 4-row blocks per down-projection instruction at most
+                                (1..16); 0 = 16 */
+    int32_t tiles_lm;        /* reserved, ignored */
     uint32_t seed;           /* 0 = plain greedy placement; else ties are broken by a
                                 seeded shuffle (for robustness tests) */
     int32_t wait_timeout_ms; /* budget of every device wait; 0 = 2000 ms */
@@ -110,8 +113,9 @@ typedef struct mk_schedule_opts {
     int32_t l2_prefetch_fills; /* a prefetch warp pulls the SM's upcoming fills into L2, at
                                 most this many fills ahead of the loader's next one, so HBM
                                 keeps streaming while the compute warps wait on
-                                activations; 0 or negative = off (the default: measured
-                                slower on the 1B decode step, see the design notes) */
+                                activations; 0 or negative = off (the default: on the 1B
+                                decode step the extra requests delay the cross-SM
+                                activation loads on the critical path, measured slower) */
     int32_t l2_prefetch_policy; /* L2 eviction hint of those prefetches: 0 = evict-last,
                                    1 = evict-normal */
     int32_t max_inflight;    /* ring fills the loader keeps in flight at most (landed fills

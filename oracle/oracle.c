@@ -30,10 +30,11 @@
  * Precision: fp32 arithmetic over the bf16 weights and the bf16 KV cache.
  * Activations stay fp32 between steps; the one rounding to bf16 (round to
  * nearest, ties to even) is where the data format forces it: the key and value
- * written to the bf16 cache [KV]. Every sum runs in plain index order. The
- * points where the write-ups are silent (activation precision, RoPE pairing and
- * frequency form, position of the new token) follow the readings listed with
- * the design notes of this repository.
+ * written to the bf16 cache [KV]. Every sum runs in plain index order. Where
+ * the write-ups are silent this follows the plainest reading: fp32 activations,
+ * rotate-half RoPE pairs (i, i + d/2) with inverse frequencies theta^(-2i/d)
+ * and no frequency scaling, and the new token at position p attending to keys
+ * 0..p, its own included.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math, so
  * no reassociation and no fused multiply-add).
