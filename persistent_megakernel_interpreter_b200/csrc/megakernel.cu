@@ -7,31 +7,36 @@
 // activation waits, and static warp-specialised pipelines instead of paging):
 //
 //  * The host writes one instruction list per SM; the CTA runs it in order, one
-//    job at a time for all compute warps.
+//    job at a time for all compute warps (a down-projection instruction is four
+//    jobs, one per MLP chunk).
 //  * Warp 8 (the loader) streams, in list order, every byte the instructions
 //    read from HBM that is final at launch -- weight tiles and the cached KV
 //    slots -- into a ring of shared-memory stages with bulk async copies
 //    (cp.async.bulk, completion counted on an mbarrier, L2 evict-first). It
-//    never waits on a dependency counter, so the next instructions' weights
-//    arrive while the step still waits for their activations.
-//  * Warp 10 (the prefetch warp) pulls the fills that follow the ring's into L2
-//    (bulk prefetch, evict-last), a bounded distance ahead of the loader, so
-//    HBM keeps streaming while the ring is full and the SM waits on activations.
-//  * Warp 9 (the activation warp) runs ahead of the compute warps: for each job
-//    it waits for the job's input counter (acquire load, bounded spin), loads
-//    the small activation input from L2 and prepares it in one of a few
-//    shared-memory slots -- RMSNorm for QKV, gate/up and the LM head, the
-//    finished attention output for the O-projection, an MLP chunk for the
-//    down-projection, q and the new key/value for attention.
+//    never waits on a dependency, so the next instructions' weights arrive
+//    while the step still waits for their activations.
+//  * Activations cross SMs as 64-bit tagged words (value | step, layer, kind)
+//    written with relaxed stores: a consumer polls the words themselves until
+//    every tag is current, so no release fence (which would wait for the SM's
+//    bulk copies in flight) sits on the data path. Counters remain as relaxed
+//    completion counts.
+//  * Warps 0..7 (compute) build each job's input themselves from the tagged
+//    words (RMSNorm for QKV, gate/up and the LM head; the attention output and
+//    the residual rows for the O-projection; q and the new key/value for an
+//    attention item), split the job's tiles (tile t goes to warp t mod 8) and
+//    write the outputs with fused epilogues.
+//  * Warp 9 (the activation warp) runs ahead of the compute warps through the
+//    same jobs: it stages the RoPE rows of QKV jobs and, at batch 1, the h chunk
+//    (and with the last chunk the residual rows) of each down-projection job,
+//    which gate/up completes chunk by chunk while it still streams.
+//  * Warp 10 (the prefetch warp) is optional and off by default: bulk L2
+//    prefetches of the fills a bounded distance past the loader.
 //  * Attention items finish their own heads: with one key partition per
 //    (sequence, KV group) the item writes o / l; with several, each stores its
 //    partial and the one that completes the pair's arrival count merges the
 //    pair in partition order, so no other SM waits on a merge.
-//  * Warps 0..7 (compute) split each job's tiles (tile t goes to warp t mod 8),
-//    write the outputs, and the last warp to finish increments the job's
-//    output counter (release).
-//  * Counters only grow: a step waits for (epoch + 1) * n increments, and the
-//    last CTA to finish advances the epoch, so no reset kernel is needed.
+//  * Counters only grow and tags carry the step's epoch: the last CTA to finish
+//    advances the epoch, so no reset kernel is needed.
 //  * Every wait is bounded by a time budget; on expiry the step records
 //    MK_ERR_TIMEOUT, raises an abort flag that every other wait polls, drains
 //    its own copies in flight and returns. No trap, no unbounded spin.
@@ -99,37 +104,7 @@ __device__ __forceinline__ bool aborted(const Params& p) {
     return ld_volatile_u32(&p.ctl->abort) != 0u;
 }
 
-__device__ __forceinline__ uint32_t target_of(uint32_t epoch, uint32_t n) { return (epoch + 1u) * n; }
 
-// Lane 0 spins until counter `ctr` reaches `target` (wrap-safe); the result is
-// broadcast to the warp. False on abort or timeout.
-__device__ bool wait_counter(const Params& p, uint32_t ctr, uint32_t target, uint32_t where,
-                             int lane) {
-    int ok = 1;
-    if (lane == 0) {
-        const uint32_t* c = p.counters + (size_t)ctr * kCounterStride;
-        uint32_t v = ld_relaxed_u32(c);
-        if ((int32_t)(v - target) < 0) {
-            const uint64_t t0 = global_timer_ns();
-            for (uint32_t it = 1;; ++it) {
-                __nanosleep(32);
-                v = ld_relaxed_u32(c);
-                if ((int32_t)(v - target) >= 0) break;
-                if ((it & 31u) == 0u) {
-                    if (aborted(p)) { ok = 0; break; }
-                    if (global_timer_ns() - t0 > p.timeout_ns) {
-                        record_error(p, MK_ERR_TIMEOUT, where, ctr, v, target, 1);
-                        ok = 0;
-                        break;
-                    }
-                }
-            }
-        }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok != 0;
-}
 
 // All lanes wait for phase `parity` of an mbarrier; warp-uniform exit. With
 // `armed`, first wait until the ring stage holds fill `seq`. Waiting threads
@@ -222,13 +197,6 @@ __device__ __forceinline__ void trace(const Params& p, uint32_t job, int word, u
         p.trace[((size_t)blockIdx.x * p.trace_jobs + job) * kTraceWords + word] = v;
 }
 
-// Wait for the job's input counter, then stamp the trace.
-__device__ __forceinline__ bool wait_input(const Params& p, uint32_t ctr, uint32_t target,
-                                           uint32_t where, int lane, uint32_t job) {
-    const bool ok = wait_counter(p, ctr, target, where, lane);
-    if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
-    return ok;
-}
 
 // Pause between polls of tagged words that have not arrived yet, bounded by
 // the wait budget and the abort flag (lane 0 decides for the warp).
@@ -779,9 +747,9 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                     break;
             }
             if (!ok) return;
-            // job done for this warp; the last of the 8 publishes the job's counter
-            // (acquire-release at CTA scope on the shared count, then a GPU-scope
-            // release: the other warps' stores are ordered before the signal)
+            // job done for this warp; the last of the 8 counts the job's completion
+            // (acquire-release at CTA scope on the shared count, then a relaxed
+            // increment: consumers read the tagged outputs, not the counter)
             __syncwarp();
             if (lane == 0) {
                 const uint32_t old = atom_shared_acq_rel_add(sl.done + s, 1u);
