@@ -827,7 +827,7 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1, volati
                 // wait for the compute warps to release the previous fill of this stage
                 uint64_t t0 = 0;
                 bool ok = true;
-                for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, 500u); ++it) {
+                for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, 20000u); ++it) {
                     if ((it & 15u) == 15u) {
                         if (t0 == 0) t0 = global_timer_ns();
                         if (aborted(p)) { ok = false; break; }
