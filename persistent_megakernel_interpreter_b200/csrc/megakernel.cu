@@ -50,6 +50,8 @@ namespace mk {
 // the step) so the warps do not reload it from global memory.
 __shared__ int g_pos[kMaxBatch];
 
+constexpr int kPairGroups = kConsumerWarps / 2;  // batch > 1: tiles in work at once (two warps each)
+
 struct Ring {
     uint8_t* base;
     uint64_t* full;
@@ -592,6 +594,98 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
     return true;
 }
 
+// Batch > 1: two compute warps share each tile by sequences -- warp w takes tiles
+// t = w (mod 4), sequences [b0, b0 + nb) with b0 = (w / 4) * ceil(B / 2) -- so a
+// stage is held for half the batched arithmetic and all eight warps have a tile
+// while only four stages fit beside the sequences' inputs. Each (sequence, row)
+// total is dot4's for that sequence, bit for bit (dot4_batch4); both warps release
+// the stage (its empty barrier counts two arrivals).
+template <int KC>
+__device__ __noinline__ float tile_dot_batch4(const uint8_t* tile, const float* xs, uint32_t vec_floats, int nb,
+                                              int lane) {
+    return dot4_batch4<KC>(tile, xs, vec_floats, nb, lane);
+}
+
+struct PairSeqs {
+    int b0, nb;  // this warp's sequences
+    __device__ PairSeqs(int B, int warp) {
+        const int per = (B + 1) / 2;
+        b0 = (warp / kPairGroups) * per;
+        nb = min(per, B - b0);
+    }
+};
+
+template <int KC, int HD>
+__device__ bool compute_tiles_pair(const Params& p, const Ring& ring, const mk_instr& in, const float* sv, int warp,
+                                   int lane, uint32_t job, uint32_t epoch) {
+    const bool pub = in.signal_ctr != MK_NO_COUNTER;
+    const PairSeqs ps(p.B, warp);
+    const int sl = lane >> 3;                         // the sequence (of this warp's) the lane holds
+    const bool act = sl < ps.nb && (lane & 1) == 0;   // lanes l and l ^ 1 hold the same total
+    const int b = ps.b0 + (sl < ps.nb ? sl : 0);
+    const int el = act ? ((lane >> 1) & 3) : 32;      // acts as lane `el` of a 4-row epilogue
+    for (uint32_t t = warp % kPairGroups; t < in.count; t += kPairGroups) {
+        const uint32_t seq = in.seq + t;
+        if (!wait_fill(p, ring, seq, lane)) return false;
+        if (t == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill, global_timer_ns());
+        const float tb = tile_dot_batch4<KC>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
+                                             p.xs_vec_floats, ps.nb, lane);
+        float acc[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[r] = __shfl_sync(0xffffffffu, tb, (lane & ~7) + 2 * r);
+        const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
+        switch (in.op) {
+            case MK_OP_QKV: {
+                const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
+                const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
+                if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, el, rr, act_tag(epoch, in.layer, kTagQKV));
+                break;
+            }
+            case MK_OP_GATEUP:
+                if (pub) gateup_epilogue<true>(p, b, tl, acc, el, act_tag(epoch, in.layer, kTagH));
+                break;
+            case MK_OP_OPROJ:
+                if (pub && el < 4) {
+                    const float xin = slot_resid(p, const_cast<float*>(sv), b)[(tl - in.first) * 4 + el];
+                    st_tagged(p.x_t + (size_t)b * p.H + tl * 4 + el, __fadd_rn(xin, pick4(acc, el)),
+                              act_tag(epoch, in.layer, kTagXAttn));
+                }
+                break;
+            default: logits_epilogue(p, b, tl, acc, el); break;
+        }
+        release_fill(ring, seq, lane);
+    }
+    return true;
+}
+
+template <int KF>
+__device__ bool compute_down_pair(const Params& p, const Ring& ring, const mk_instr& in, int c, const float* sv,
+                                  float* tot, int warp, int lane, uint32_t job, uint32_t epoch) {
+    const PairSeqs ps(p.B, warp);
+    const int sl = lane >> 3;
+    const bool act = sl < ps.nb && (lane & 1) == 0;
+    const int b = ps.b0 + (sl < ps.nb ? sl : 0);
+    const int row = (lane >> 1) & 3;
+    for (uint32_t r = warp % kPairGroups; r < in.count; r += kPairGroups) {
+        const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
+        if (!wait_fill(p, ring, seq, lane)) return false;
+        if (r == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill, global_timer_ns());
+        const float y = tile_dot_batch4<KF>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
+                                            p.xs_vec_floats, ps.nb, lane);
+        if (act) {
+            float* t = tot + ((size_t)r * p.B + b) * 4 + row;
+            *t = (c == 0) ? y : *t + y;
+            if (c == 3 && in.signal_ctr != MK_NO_COUNTER) {  // x = x_in + W_d h; x_in waits in the slot
+                const float xin = slot_resid(p, const_cast<float*>(sv), b)[r * 4 + row];
+                st_tagged(p.x_t + (size_t)b * p.H + (in.first + r) * 4 + row, __fadd_rn(xin, *t),
+                          act_tag(epoch, in.layer, kTagXMlp));
+            }
+        }
+        release_fill(ring, seq, lane);
+    }
+    return true;
+}
+
 // Down-projection, chunk c: row block r (warp r mod 8) adds W_d[:, chunk c] . h_c to
 // its running sums, chunks in order 0..3; after chunk 3 the residual.
 template <int KF>
@@ -640,7 +734,7 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
 // counter, and the item that completes the count merges the pair's partitions
 // in partition order. Either way the group's heads are signalled on the
 // attention counter once their output is written.
-template <int HD>
+template <int HD, bool BATCHED>
 __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr& a, const uint8_t* slot,
                                  float* sc, int warp, int lane, uint64_t* cbar, uint32_t& cuses,
                                  uint32_t job, uint32_t epoch) {
@@ -683,7 +777,9 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     }
     // every warp has passed the barrier after its last read of the fills
     if (warp == kConsumerWarps - 1 && lane == 0)
-        for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+        for (uint32_t f = 0; f < a.nfill; ++f)
+            for (int k = 0; k < (BATCHED ? 2 : 1); ++k)  // batch > 1: each stage counts two arrivals
+                mbar_arrive(ring.empty + (a.seq + f) % ring.S);
     if (!bar()) return false;  // every output of the item is stored
     if (p.n_parts == 1) {
         if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_relaxed_add(sig, (uint32_t)G);
@@ -736,14 +832,26 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7, global_timer_ns());
             switch (in.op) {
-                case MK_OP_QKV: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
-                case MK_OP_OPROJ: ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
+                case MK_OP_QKV:
+                    if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    break;
+                case MK_OP_OPROJ:
+                    if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    else ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    break;
                 case MK_OP_GATEUP:
-                case MK_OP_LMHEAD: ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch); break;
-                case MK_OP_DOWN: ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch); break;
+                case MK_OP_LMHEAD:
+                    if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    break;
+                case MK_OP_DOWN:
+                    if constexpr (BATCHED) ok = compute_down_pair<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
+                    else ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
+                    break;
                 default:
-                    ok = compute_attn_job<HD>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
-                                              epoch);
+                    ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
+                                                       epoch);
                     break;
             }
             if (!ok) return;
@@ -961,7 +1069,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
             mbar_init(ring.full + s, 1);
-            mbar_init(ring.empty + s, 1);
+            mbar_init(ring.empty + s, BATCHED ? 2 : 1);  // batch > 1: two warps share each tile
             ring.armed[s] = 0xffffffffu;
         }
         for (int s = 0; s < p.xs_slots; ++s) {

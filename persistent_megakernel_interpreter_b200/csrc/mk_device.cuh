@@ -568,6 +568,49 @@ __device__ __forceinline__ float dot4_batch(const uint8_t* tile, const float* xs
     return v[0];
 }
 
+// The same for at most 4 of the sequences (B4 <= 4, sequence b at xs + b *
+// vec_floats), so that two warps can share a tile by sequences: 16 partial sums
+// per lane, reduce-scattered with warp_sum's masks 16, 8, 4, 2 and summed across
+// the last pair with mask 1, so each total again equals dot4's for its sequence
+// bit for bit. Lanes l and l ^ 1 hold the total of sequence l / 8, row (l / 2) % 4.
+template <int KC>
+__device__ __forceinline__ float dot4_batch4(const uint8_t* tile, const float* xs, uint32_t vec_floats, int B4,
+                                             int lane) {
+    const uint4* t = reinterpret_cast<const uint4*>(tile) + lane;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+#pragma unroll 1
+    for (int kc = 0; kc < KC; ++kc) {
+        float w[4][8];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) unpack8(lds_v4(t + r * KC * 32 + kc * 32), w[r]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (b < B4) {
+                const float4* x = reinterpret_cast<const float4*>(xs + (size_t)b * vec_floats);
+                const float4 lo = x[kc * 32 + lane], hi = x[KC * 32 + kc * 32 + lane];
+                const float e[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[b * 4 + r] = fmaf(w[r][i], e[i], v[b * 4 + r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 16, n = 8; m > 1; m >>= 1, n >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float keep = up ? v[n + i] : v[i];
+            const float send = up ? v[i] : v[n + i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 // ------------------------------------------------------------------ per-op helpers
 
 __device__ __forceinline__ const uint16_t* norm_ptr(const Params& p, size_t off) {
