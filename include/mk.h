@@ -4,12 +4,15 @@
  * One decode step of a Llama-style decoder (batch 1 or a few sequences) runs as
  * ONE persistent sm_100a kernel: one CTA per SM, each working through a
  * host-built list of instructions, with dependencies between instructions
- * expressed as counters in global memory rather than kernel boundaries. This is
- * the design of the "Look Ma, No Bubbles" Llama-3.2-1B megakernel (summaries:
- * sections "Fusing Operations with an On-GPU Interpreter" and "Custom
- * Synchronization Mechanism") and of the Cohere decode megakernel (section
- * "Megakernel 是什么": a resident block per SM reading a host-written task list of
- * tile-sized work items, with atomic-increment / spin-wait counters).
+ * resolved inside the kernel rather than by kernel boundaries. This is the design
+ * of the "Look Ma, No Bubbles" Llama-3.2-1B megakernel (summaries: sections
+ * "Fusing Operations with an On-GPU Interpreter" and "Custom Synchronization
+ * Mechanism") and of the Cohere decode megakernel (section "Megakernel 是什么": a
+ * resident block per SM reading a host-written task list of tile-sized work
+ * items). Those designs wait on atomic-increment counters; here the activations
+ * that cross SMs carry their own validity (64-bit words tagged with the step,
+ * layer and producer), the consumer polls the words themselves, and counters
+ * remain as completion counts (see mk_read_counters).
  *
  * Conventions for every entry point:
  *   - Pointers documented as "device" must be CUDA device memory of the handle's
@@ -236,11 +239,13 @@ mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_tot
 
 /* Per-job timestamps of the last traced step (schedule built with opts.trace):
  * uint64 [n_sm][jobs][16] globaltimer nanoseconds -- 0 activation warp starts
- * waiting for a free input slot, 1 slot free (input counter wait starts),
- * 2 input counter reached, 3 input prepared, 4 compute warp 0 starts, 5 the
- * job's last compute warp finished, 6 op | layer << 8 | chunk << 24, 7 compute
- * warp 0 has its first ring fill of the job (0 if it had none), 8..15 finer
- * op-specific points of compute warp 0 (0 where unused).
+ * waiting for a free input slot, 1 slot free, 2 the activation warp starts its
+ * part of the job, 3 its part is ready (the slot is handed to the compute
+ * warps), 4 compute warp 0 starts (it then builds the job's input from the
+ * producers' tagged words), 5 the job's last compute warp finished, 6 op |
+ * layer << 8 | chunk << 24, 7 compute warp 0 has its first ring fill of the job
+ * (0 if it had none), 8..15 finer op-specific points of compute warp 0 (15: the
+ * job's input built; 0 where unused).
  * *jobs receives the per-SM job capacity; at most `bytes` are copied.
  * Synchronous. */
 mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs);
