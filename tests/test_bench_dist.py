@@ -95,3 +95,23 @@ def test_reference_arm_other_ranks_exit_without_work():
     for rc, out, err in outs:
         assert rc == 0, err[-2000:]
     assert "rank1-done" in outs[1][1] and "rank0-done" in outs[0][1]
+
+
+def test_reference_arm_prints_the_contract_line():
+    """One process, no GPU: `bench.py --impl reference` times the CPU oracle on the
+    benchmark's workload and prints one JSON line with the fields the benchmark
+    contract names (the reference arm's value is the oracle's tokens/s)."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert "workload" in line["config"]
