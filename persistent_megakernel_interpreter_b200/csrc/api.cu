@@ -56,6 +56,7 @@ struct mk_handle {
     uint64_t* d_trace = nullptr;    // per-job timestamps (traced schedules only)
     int trace_jobs = 0;
     int32_t* d_io = nullptr;        // tokens [max_batch], positions [max_batch]
+    int32_t* h_io = nullptr;        // pinned host staging of the same, for mk_decode_step_host
     float* d_logits = nullptr;
     std::string msg;
 };
@@ -78,6 +79,7 @@ void free_schedule(mk_handle* h) {
     cudaFree(h->d_instrs);
     cudaFree(h->d_sm_off);
     cudaFree(h->d_io);
+    cudaFreeHost(h->h_io);
     cudaFree(h->d_logits);
     cudaFree(h->d_trace);
     h->d_trace = nullptr;
@@ -86,6 +88,7 @@ void free_schedule(mk_handle* h) {
     h->d_instrs = nullptr;
     h->d_sm_off = nullptr;
     h->d_io = nullptr;
+    h->h_io = nullptr;
     h->d_logits = nullptr;
     h->has_schedule = false;
 }
@@ -224,6 +227,8 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     MK_CUDA(h, cudaMemcpy(h->d_sm_off, P.sm_off.data(), P.sm_off.size() * sizeof(int32_t),
                           cudaMemcpyHostToDevice));
     MK_CUDA(h, cudaMalloc(&h->d_io, 2 * (size_t)c.max_batch * sizeof(int32_t)));
+    MK_CUDA(h, cudaMallocHost(&h->h_io, 2 * (size_t)c.max_batch * sizeof(int32_t)));
+    memset(h->h_io, 0, 2 * (size_t)c.max_batch * sizeof(int32_t));
     MK_CUDA(h, cudaMalloc(&h->d_logits, (size_t)batch * L.V * sizeof(float)));
 
     mk::Params& p = h->params;
@@ -349,10 +354,12 @@ extern "C" mk_status mk_decode_step_host(mk_handle* h, const int32_t* tokens_hos
     if (!h->has_schedule) return MK_ERR_NO_SCHEDULE;
     if (!tokens_host || !positions_host || !logits_host) return MK_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int B = h->params.B;
-    MK_CUDA(h, cudaMemcpyAsync(h->d_io, tokens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, s));
-    MK_CUDA(h, cudaMemcpyAsync(h->d_io + h->cfg.max_batch, positions_host, B * sizeof(int32_t),
-                               cudaMemcpyHostToDevice, s));
+    const int B = h->params.B, MB = h->cfg.max_batch;
+    // tokens and positions travel in one copy, through the handle's pinned staging
+    // (the previous call's copy has completed: every call ends with a stream sync)
+    memcpy(h->h_io, tokens_host, B * sizeof(int32_t));
+    memcpy(h->h_io + MB, positions_host, B * sizeof(int32_t));
+    MK_CUDA(h, cudaMemcpyAsync(h->d_io, h->h_io, 2 * (size_t)MB * sizeof(int32_t), cudaMemcpyHostToDevice, s));
     mk_status st = mk_decode_step(h, h->d_io, h->d_io + h->cfg.max_batch, k_cache, v_cache,
                                   h->d_logits, stream);
     if (st != MK_OK) return st;
