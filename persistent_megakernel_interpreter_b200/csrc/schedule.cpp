@@ -133,10 +133,10 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     // a layer has few items: while the item's SM computes it (and its ring holds KV
     // fills), the other SMs' rings fill with the layer's gate/up weights, so the
     // item's SM should take fewer of them. Measured on the 1B step at 128 positions
-    // (8 items): 0 / 32 / 64 / 128 / 160 / 192 / 256 KB -> 692 / 682 / 683 / 680 / 682
-    // / 682 / 688 us. With
-    // an item on (nearly) every SM the charge only overloads the SMs without one
-    // (1B at 8192 positions: 900 -> 987 us), so it applies to few items only.
+    // (8 items): 0 / 32 / 64 / 128 / 160 / 192 / 256 KB -> 692 / 682 / 683 / 680 /
+    // 682 / 682 / 688 us. With an item on (nearly) every SM the charge only
+    // overloads the SMs without one (1B at 8192 positions: 900 -> 987 us), so it
+    // applies to few items only.
     const uint64_t attn_item_cost = (uint64_t)batch * L.nkv * n_parts * 8 <= (uint64_t)n_sm ? 128 * 1024 : 0;
     using Key = std::pair<uint64_t, uint32_t>;  // (load, rank)
     std::vector<int> sm_of_rank(n_sm);
