@@ -383,6 +383,9 @@ def run_mk(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "us_per_step": 1e3 * ms_per_step,
             "us_per_launch_median": 1e3 * statistics.median(launch_ms),
+            "us_per_launch_p10_p90": [1e3 * q for q in (statistics.quantiles(launch_ms, n=10)[0],
+                                                         statistics.quantiles(launch_ms, n=10)[8])]
+            if len(launch_ms) >= 2 else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(world, cfg.n_layers, past, args.model, BATCH),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
