@@ -305,3 +305,33 @@ def test_down_instructions_cover_row_block_ranges(cfg, batch):
         assert sorted(seen) == list(range(cfg.hidden // 4))
     n_down = sum(1 for ins in instrs if ins.op == _lib.OP_DOWN)
     assert n_down <= cfg.n_layers * 148 + cfg.n_layers * (cfg.hidden // 4) // 16
+
+
+def test_attention_sms_take_fewer_gateup_tiles_when_items_are_few():
+    """With few attention items per layer (1B, 128 positions: 8 items on 148 SMs)
+    each item is charged extra load, so the SMs that run a layer's attention take
+    fewer of that layer's gate/up tiles than the other SMs; with an item on nearly
+    every SM (8192 positions) no such charge applies."""
+    for ctx, charged in ((129, True), (8193, False)):
+        instrs, offs, _ = plan_schedule(LLAMA_1B, 1, ctx, 148, max_batch=1, max_seq=ctx)
+        fewer = 0
+        layers = 0
+        for layer in range(1, LLAMA_1B.n_layers):
+            att, gu = set(), collections.Counter()
+            for s in range(148):
+                for ins in instrs[offs[s]:offs[s + 1]]:
+                    if ins.layer != layer:
+                        continue
+                    if ins.op == _lib.OP_ATTN:
+                        att.add(s)
+                    elif ins.op == _lib.OP_GATEUP:
+                        gu[s] += ins.count
+            others = [gu[s] for s in range(148) if s not in att]
+            if not att or not others:
+                continue
+            layers += 1
+            fewer += max(gu[s] for s in att) < min(others)
+        if charged:
+            assert fewer == layers, (fewer, layers)
+        else:
+            assert fewer < layers
