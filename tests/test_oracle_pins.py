@@ -15,7 +15,7 @@ import oracle
 
 def bf(x) -> np.ndarray:
     """fp values -> bf16 bits through torch (library rounding)."""
-    t = torch.as_tensor(np.asarray(x, dtype=np.float64)).to(torch.bfloat16)
+    t = torch.as_tensor(np.array(x, dtype=np.float64)).to(torch.bfloat16)
     return t.view(torch.int16).numpy().view(np.uint16).copy()
 
 
