@@ -415,14 +415,15 @@ def run_mk(args):
 def run_greedy(args):
     """Greedy decoding at batch 1: a 32-token random prompt fed as decode steps into
     an empty cache, then ``--greedy`` generated tokens, each the argmax of the
-    previous step's logits (taken on the device, outside the timed region). Every
+    previous step's logits (chosen on the device by mk_greedy_select, outside the
+    timed region). Every
     step is timed alone with CUDA events around its launch; prints one JSON line
     with the per-step latency distribution."""
     import numpy as np
     import torch
     from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B
     from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
-    from persistent_megakernel_interpreter_b200.model import Megakernel
+    from persistent_megakernel_interpreter_b200.model import Megakernel, greedy_select
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     cfg = LLAMA_3B if args.model == "3b" else LLAMA_1B
@@ -452,7 +453,7 @@ def run_greedy(args):
                 if p < n_prompt:
                     tok.copy_(prompt[p:p + 1])
                 else:
-                    tok.copy_(torch.argmax(logits[0]).to(torch.int32).view(1))
+                    greedy_select(logits, tok)
                 ev[p][0].record(stream)
                 mk.decode_step(tok, pos, kd, vd, logits, stream)
                 ev[p][1].record(stream)

@@ -168,6 +168,23 @@ void mk_destroy(mk_handle* h);
 
 const char* mk_status_str(mk_status s);
 
+/* Greedy selection between decode steps: next_tokens[b] = the index v in [0, vocab)
+ * of the largest logits[b][v], the lowest such index where several are equal (the
+ * greedy decoding rule of the decoder's generation loop). NaN entries are never
+ * selected; a row of NaNs gives 0.
+ *   logits       device fp32 [batch][vocab], rows contiguous (mk_decode_step's output)
+ *   batch, vocab >= 1
+ *   next_tokens  device int32 [batch]; may be the tokens buffer of the next
+ *                mk_decode_step, so a decode loop needs no host round trip
+ *   positions    device int32 [batch] or NULL: when given, each positions[b] is
+ *                incremented by one in the same launch
+ *   stream       the CUDA stream the selection is enqueued on
+ * Enqueues one kernel launch (one CTA per sequence); no synchronisation, no
+ * allocation, capturable in a CUDA graph. Returns MK_ERR_INVALID_ARG for a NULL
+ * logits or next_tokens pointer or a size below 1, MK_ERR_CUDA if the launch fails. */
+mk_status mk_greedy_select(const float* logits, int batch, int vocab, int32_t* next_tokens,
+                           int32_t* positions, void* stream);
+
 /* ------------------------------------------------------------------ inspection */
 
 /* One instruction of the per-SM lists (48 bytes). An SM's CTA runs its list in

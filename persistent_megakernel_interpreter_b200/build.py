@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmk.so")
-SOURCES = ["api.cu", "megakernel.cu", "baseline.cu", "noalloc.cu", "pack.cpp", "schedule.cpp"]
+SOURCES = ["api.cu", "megakernel.cu", "baseline.cu", "noalloc.cu", "select.cu", "pack.cpp", "schedule.cpp"]
 HEADERS = ["mk_internal.h", "mk_device.cuh", "pack.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

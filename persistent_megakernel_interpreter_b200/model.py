@@ -3,7 +3,8 @@
 ``Megakernel(cfg, weights, max_batch, max_seq)`` packs device weights into a
 library handle; ``build_schedule``; ``decode_step`` (one persistent kernel
 launch), ``baseline_decode_step`` (the multi-kernel baseline) and
-``decode_step_host`` (host buffers in and out) run one step. PyTorch supplies
+``decode_step_host`` (host buffers in and out) run one step; ``greedy_select``
+picks the next tokens from a step's logits on the device. PyTorch supplies
 device memory and streams only.
 """
 from __future__ import annotations
@@ -131,6 +132,18 @@ class Megakernel:
         arr = (ctypes.c_uint32 * n.value)()
         _lib.check(L.mk_read_counters(self._h, arr, n.value, ctypes.byref(n)), "mk_read_counters")
         return list(arr)
+
+
+def greedy_select(logits: torch.Tensor, next_tokens: torch.Tensor, positions=None, stream=None) -> None:
+    """next_tokens[b] = argmax of logits[b] (lowest index among equal maxima), on the
+    device and asynchronous on ``stream``; ``positions`` (optional) is advanced by one."""
+    assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous() and logits.dim() == 2
+    assert next_tokens.is_cuda and next_tokens.dtype == torch.int32 and next_tokens.numel() >= logits.shape[0]
+    if positions is not None:
+        assert positions.is_cuda and positions.dtype == torch.int32 and positions.numel() >= logits.shape[0]
+    _lib.check(_lib.lib().mk_greedy_select(_ptr(logits), logits.shape[0], logits.shape[1], _ptr(next_tokens),
+                                           _ptr(positions) if positions is not None else None,
+                                           _stream(stream)), "mk_greedy_select")
 
 
 def plan_schedule(cfg: ModelConfig, batch: int, max_ctx: int, n_sm: int, max_batch: int = 8,

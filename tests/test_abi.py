@@ -39,6 +39,12 @@ def test_status_strings_and_struct_sizes():
     assert lib.mk_decode_step(None, None, None, None, None, None, None) == 1
     assert lib.mk_build_schedule(None, 1, 1, None) == 1
     lib.mk_destroy(None)
+    # greedy selection: null buffers and empty sizes are refused before any launch
+    fake = ctypes.c_void_p(256)
+    assert lib.mk_greedy_select(None, 1, 8, fake, None, None) == 1
+    assert lib.mk_greedy_select(fake, 1, 8, None, None, None) == 1
+    assert lib.mk_greedy_select(fake, 0, 8, fake, None, None) == 1
+    assert lib.mk_greedy_select(fake, 1, 0, fake, None, None) == 1
 
 
 def test_create_rejects_unsupported_shapes():
