@@ -23,6 +23,11 @@
  *     returned before anything is enqueued. Errors found by the GPU during a step
  *     are recorded on the device and reported by mk_get_status().
  *   - A handle is not thread-safe; distinct handles are independent.
+ *   - Calls that enqueue GPU work for a handle (the decode steps) run on the calling
+ *     thread's current device and are refused with MK_ERR_INVALID_ARG when that is
+ *     not the handle's device. The synchronous calls (create, schedule, status,
+ *     readers, destroy) switch to the handle's device themselves and give the
+ *     caller's current device back before they return.
  */
 #ifndef MK_H
 #define MK_H
@@ -138,7 +143,10 @@ mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_sched
  *   logits            : device fp32 [batch][vocab]
  * Enqueues exactly one cooperative kernel launch; no host synchronisation, no
  * allocation. A step with a bad token or position writes no KV slot and leaves the
- * logits unspecified; the error is reported by mk_get_status. */
+ * logits unspecified; the error is reported by mk_get_status. Returns
+ * MK_ERR_INVALID_ARG (nothing enqueued) for a NULL pointer, a KV cache that is not
+ * 16-byte aligned, or a calling thread whose current device is not the handle's;
+ * MK_ERR_NO_SCHEDULE before mk_build_schedule. */
 mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions,
                          void* k_cache, void* v_cache, float* logits, void* stream);
 
@@ -179,7 +187,8 @@ const char* mk_status_str(mk_status s);
  *   positions    device int32 [batch] or NULL: when given, each positions[b] is
  *                incremented by one in the same launch
  *   stream       the CUDA stream the selection is enqueued on
- * Enqueues one kernel launch (one CTA per sequence); no synchronisation, no
+ * Enqueues one kernel launch (one CTA per sequence) on the calling thread's current
+ * device, which must own the buffers and the stream; no synchronisation, no
  * allocation, capturable in a CUDA graph. Returns MK_ERR_INVALID_ARG for a NULL
  * logits or next_tokens pointer or a size below 1, MK_ERR_CUDA if the launch fails. */
 mk_status mk_greedy_select(const float* logits, int batch, int vocab, int32_t* next_tokens,

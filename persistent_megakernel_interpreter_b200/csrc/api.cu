@@ -74,6 +74,24 @@ mk_status cuda_fail(mk_handle* h, cudaError_t e, const char* what) {
         if (e_ != cudaSuccess) return cuda_fail(h, e_, #call); \
     } while (0)
 
+// Makes the handle's device current for the calls of one entry point and gives
+// the caller's current device back when the entry point returns.
+struct DeviceScope {
+    int prev = -1;
+    cudaError_t enter(int device) {
+        const cudaError_t e = cudaGetDevice(&prev);
+        if (e != cudaSuccess) {
+            prev = -1;
+            return e;
+        }
+        return prev == device ? cudaSuccess : cudaSetDevice(device);
+    }
+    ~DeviceScope() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
 void free_schedule(mk_handle* h) {
     cudaFree(h->scratch);
     cudaFree(h->d_instrs);
@@ -128,7 +146,8 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
         mk_destroy(h);
         return s;
     };
-    cudaError_t e = cudaSetDevice(device);
+    DeviceScope scope;
+    cudaError_t e = scope.enter(device);
     if (e != cudaSuccess) return bail(MK_ERR_CUDA);
     if (cudaDeviceGetAttribute(&h->dev_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
         return bail(MK_ERR_CUDA);
@@ -185,7 +204,8 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
         return MK_ERR_INVALID_ARG;
     const int n_sm = (opts && opts->n_sm > 0) ? opts->n_sm : h->dev_sms;
     if (n_sm > h->dev_sms) return MK_ERR_INVALID_ARG;
-    MK_CUDA(h, cudaSetDevice(h->device));
+    DeviceScope scope;
+    MK_CUDA(h, scope.enter(h->device));
     mk::Plan P;
     mk_status st = mk::plan_schedule(L, batch, max_ctx, n_sm, opts, 0, &P);
     if (st != MK_OK) return st;
@@ -308,6 +328,18 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     return MK_OK;
 }
 
+// A step is enqueued on the calling thread's current device; one whose handle
+// lives on another device is refused (its buffers are not that device's memory).
+static mk_status current_device_is(mk_handle* h) {
+    int cur = -1;
+    MK_CUDA(h, cudaGetDevice(&cur));
+    if (cur != h->device) {
+        h->msg = "the calling thread's current device is not the handle's device";
+        return MK_ERR_INVALID_ARG;
+    }
+    return MK_OK;
+}
+
 static mk_status step_args(mk_handle* h, const int32_t* tokens, const int32_t* positions,
                            void* k_cache, void* v_cache, float* logits) {
     if (!h) return MK_ERR_INVALID_ARG;
@@ -315,7 +347,7 @@ static mk_status step_args(mk_handle* h, const int32_t* tokens, const int32_t* p
     if (!tokens || !positions || !k_cache || !v_cache || !logits) return MK_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
         return MK_ERR_INVALID_ARG;
-    return MK_OK;
+    return current_device_is(h);
 }
 
 extern "C" mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions,
@@ -353,6 +385,7 @@ extern "C" mk_status mk_decode_step_host(mk_handle* h, const int32_t* tokens_hos
     if (!h) return MK_ERR_INVALID_ARG;
     if (!h->has_schedule) return MK_ERR_NO_SCHEDULE;
     if (!tokens_host || !positions_host || !logits_host) return MK_ERR_INVALID_ARG;
+    if (const mk_status st = current_device_is(h); st != MK_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int B = h->params.B, MB = h->cfg.max_batch;
     // tokens and positions travel in one copy, through the handle's pinned staging
@@ -372,7 +405,8 @@ extern "C" mk_status mk_decode_step_host(mk_handle* h, const int32_t* tokens_hos
 extern "C" mk_status mk_get_status(mk_handle* h, mk_status* device_status, char* msg,
                                    size_t msg_len) {
     if (!h) return MK_ERR_INVALID_ARG;
-    MK_CUDA(h, cudaSetDevice(h->device));
+    DeviceScope scope;
+    MK_CUDA(h, scope.enter(h->device));
     MK_CUDA(h, cudaDeviceSynchronize());
     mk_status dev = MK_OK;
     std::string text = h->msg;
@@ -412,7 +446,8 @@ extern "C" mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, si
     const size_t nc = (size_t)h->info.n_counters;
     if (n_total) *n_total = nc + 2;
     if (!host || n == 0) return MK_OK;
-    MK_CUDA(h, cudaSetDevice(h->device));
+    DeviceScope scope;
+    MK_CUDA(h, scope.enter(h->device));
     MK_CUDA(h, cudaDeviceSynchronize());
     std::vector<uint32_t> raw(nc * mk::kCounterStride);
     MK_CUDA(h, cudaMemcpy(raw.data(), h->counters, raw.size() * sizeof(uint32_t), cudaMemcpyDeviceToHost));
@@ -429,7 +464,8 @@ extern "C" mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, i
     if (jobs) *jobs = h->trace_jobs;
     if (!h->d_trace || !host || bytes == 0) return MK_OK;
     const size_t tb = (size_t)h->params.n_sm * h->trace_jobs * mk::kTraceWords * sizeof(uint64_t);
-    MK_CUDA(h, cudaSetDevice(h->device));
+    DeviceScope scope;
+    MK_CUDA(h, scope.enter(h->device));
     MK_CUDA(h, cudaDeviceSynchronize());
     MK_CUDA(h, cudaMemcpy(host, h->d_trace, bytes < tb ? bytes : tb, cudaMemcpyDeviceToHost));
     return MK_OK;
@@ -437,10 +473,12 @@ extern "C" mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, i
 
 extern "C" void mk_destroy(mk_handle* h) {
     if (!h) return;
-    cudaSetDevice(h->device);
-    cudaDeviceSynchronize();
-    free_schedule(h);
-    cudaFree(h->packed);
-    cudaFree(h->rope);
+    {
+        DeviceScope scope;
+        if (scope.enter(h->device) == cudaSuccess) cudaDeviceSynchronize();
+        free_schedule(h);
+        cudaFree(h->packed);
+        cudaFree(h->rope);
+    }
     delete h;
 }
