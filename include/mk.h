@@ -63,6 +63,11 @@ typedef struct mk_config {
     int32_t max_batch;   /* batch dimension of the KV cache and largest schedulable batch */
     int32_t max_seq;     /* slot dimension of the KV cache */
 } mk_config;
+/* Accepted ranges (else MK_ERR_UNSUPPORTED from mk_create, 0 from mk_packed_bytes):
+ * 1..64 layers; hidden a multiple of 256 up to 65536; head_dim 64 or 128; at most 32
+ * query heads and 4 per KV head; n_heads*head_dim a multiple of 256; ffn a multiple
+ * of 1024 up to 262144; vocab a multiple of 4 up to 2^24; max_batch 1..8; max_seq
+ * 1..2^20. mk_create further needs a shape the kernels are instantiated for. */
 
 /* Weight pointers for mk_create. Matrices are bf16 row-major [out][in]:
  *   wq [n_heads*head_dim][hidden], wk/wv [n_kv_heads*head_dim][hidden],

@@ -10,6 +10,16 @@
 
 namespace mk {
 
+namespace {
+// the largest hidden size, ffn, vocabulary and max_seq a configuration may give (the
+// kernels further limit hidden and ffn to their instantiated shapes); they keep every
+// host-side product of dimensions far from int overflow
+constexpr int kMaxHidden = 1 << 16;
+constexpr int kMaxFfn = 1 << 18;
+constexpr int kMaxVocab = 1 << 24;
+constexpr int kMaxSeq = 1 << 20;
+}  // namespace
+
 bool make_layout(const mk_config& c, Layout* out, const char** why) {
     auto fail = [&](const char* m) {
         if (why) *why = m;
@@ -30,6 +40,8 @@ bool make_layout(const mk_config& c, Layout* out, const char** why) {
     if (c.vocab % 4) return fail("vocab must be a multiple of 4");
     if (c.max_batch < 1 || c.max_batch > 8) return fail("max_batch must be in [1, 8]");
     if (c.max_seq < 1) return fail("max_seq must be positive");
+    if (c.hidden > kMaxHidden || c.ffn > kMaxFfn || c.vocab > kMaxVocab || c.max_seq > kMaxSeq)
+        return fail("a dimension is above the supported maximum");
     if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 0.0)) return fail("bad eps or rope_theta");
     Layout L{};
     L.L = c.n_layers; L.H = c.hidden; L.nq = c.n_heads; L.nkv = c.n_kv_heads; L.d = c.head_dim;

@@ -59,3 +59,9 @@ def test_create_rejects_unsupported_shapes():
     h = ctypes.c_void_p()
     assert lib.mk_create(ctypes.byref(c), ctypes.byref(w), 0, ctypes.byref(h)) == 3
     assert not h.value
+    # dimensions far above any model are refused before any size is computed from them
+    for field, value in (("hidden", 1 << 29), ("ffn", 1 << 30), ("vocab", 1 << 30)):
+        c = _lib.make_config(dataclasses.replace(TINY, **{field: value}), 1, 16)
+        assert lib.mk_packed_bytes(ctypes.byref(c)) == 0, field
+    assert lib.mk_packed_bytes(ctypes.byref(_lib.make_config(TINY, 1, (1 << 20) + 1))) == 0
+    assert lib.mk_packed_bytes(ctypes.byref(_lib.make_config(TINY, 1, 1 << 20))) > 0
