@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <new>
+#include <stdexcept>
 #include <string>
 #include <vector>
 
@@ -92,6 +94,21 @@ struct DeviceScope {
     }
 };
 
+// Runs an entry point's body so that no C++ exception leaves the C ABI: a failed
+// host allocation reads as MK_ERR_OUT_OF_MEMORY, anything else as MK_ERR_INVALID_ARG.
+template <class F>
+mk_status no_throw(F&& body) {
+    try {
+        return body();
+    } catch (const std::bad_alloc&) {
+        return MK_ERR_OUT_OF_MEMORY;
+    } catch (const std::length_error&) {
+        return MK_ERR_OUT_OF_MEMORY;
+    } catch (...) {
+        return MK_ERR_INVALID_ARG;
+    }
+}
+
 void free_schedule(mk_handle* h) {
     cudaFree(h->scratch);
     cudaFree(h->d_instrs);
@@ -128,8 +145,7 @@ extern "C" const char* mk_status_str(mk_status s) {
     return "unknown status";
 }
 
-extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int device,
-                               mk_handle** out) {
+static mk_status create_impl(const mk_config* cfg, const mk_weights* w, int device, mk_handle** out) {
     if (!out) return MK_ERR_INVALID_ARG;
     *out = nullptr;
     if (!cfg || !w) return MK_ERR_INVALID_ARG;
@@ -138,14 +154,16 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
     if (!mk::make_layout(*cfg, &L, &why)) return MK_ERR_UNSUPPORTED;
     if (!mk::megakernel_supported(L.H, L.Q, L.F, L.d)) return MK_ERR_UNSUPPORTED;
     if (!mk::weights_complete(L, *w)) return MK_ERR_INVALID_ARG;
-    mk_handle* h = new mk_handle();
+    // the handle is destroyed on every way out but success, a thrown one included
+    struct Owner {
+        mk_handle* h;
+        ~Owner() { mk_destroy(h); }
+    } owner{new mk_handle()};
+    mk_handle* h = owner.h;
     h->device = device;
     h->cfg = *cfg;
     h->lay = L;
-    auto bail = [&](mk_status s) {
-        mk_destroy(h);
-        return s;
-    };
+    auto bail = [](mk_status s) { return s; };
     DeviceScope scope;
     cudaError_t e = scope.enter(device);
     if (e != cudaSuccess) return bail(MK_ERR_CUDA);
@@ -191,12 +209,17 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
             cudaSuccess)
             return bail(MK_ERR_CUDA);
     }
+    owner.h = nullptr;
     *out = h;
     return MK_OK;
 }
 
-extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
-                                       const mk_schedule_opts* opts) {
+extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int device,
+                               mk_handle** out) {
+    return no_throw([&] { return create_impl(cfg, w, device, out); });
+}
+
+static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts) {
     if (!h) return MK_ERR_INVALID_ARG;
     const mk_config& c = h->cfg;
     const mk::Layout& L = h->lay;
@@ -328,6 +351,11 @@ extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
     return MK_OK;
 }
 
+extern "C" mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx,
+                                       const mk_schedule_opts* opts) {
+    return no_throw([&] { return build_schedule_impl(h, batch, max_ctx, opts); });
+}
+
 // A step is enqueued on the calling thread's current device; one whose handle
 // lives on another device is refused (its buffers are not that device's memory).
 static mk_status current_device_is(mk_handle* h) {
@@ -440,7 +468,7 @@ extern "C" mk_status mk_get_schedule_info(mk_handle* h, mk_schedule_info* info) 
     return MK_OK;
 }
 
-extern "C" mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_total) {
+static mk_status read_counters_impl(mk_handle* h, uint32_t* host, size_t n, size_t* n_total) {
     if (!h) return MK_ERR_INVALID_ARG;
     if (!h->has_schedule) return MK_ERR_NO_SCHEDULE;
     const size_t nc = (size_t)h->info.n_counters;
@@ -456,6 +484,10 @@ extern "C" mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, si
     for (size_t i = 0; i < nc + 2 && i < n; ++i)
         host[i] = i < nc ? raw[i * mk::kCounterStride] : (i == nc ? c.epoch : c.done);
     return MK_OK;
+}
+
+extern "C" mk_status mk_read_counters(mk_handle* h, uint32_t* host, size_t n, size_t* n_total) {
+    return no_throw([&] { return read_counters_impl(h, host, n, n_total); });
 }
 
 extern "C" mk_status mk_read_trace(mk_handle* h, uint64_t* host, size_t bytes, int32_t* jobs) {

@@ -179,8 +179,13 @@ extern "C" mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights
     if (!cfg || !w || !dst) return MK_ERR_INVALID_ARG;
     if (!mk::make_layout(*cfg, &L, nullptr)) return MK_ERR_UNSUPPORTED;
     if (dst_bytes < L.total || !mk::weights_complete(L, *w)) return MK_ERR_INVALID_ARG;
+    std::vector<mk::Segment> segs;
+    try {
+        segs = mk::pack_segments(L, *w);
+    } catch (...) {  // the segment list could not be allocated; nothing is written
+        return MK_ERR_OUT_OF_MEMORY;
+    }
     memset(dst, 0, L.total);
-    for (const mk::Segment& s : mk::pack_segments(L, *w))
-        memcpy(static_cast<uint8_t*>(dst) + s.dst, s.src, s.bytes);
+    for (const mk::Segment& s : segs) memcpy(static_cast<uint8_t*>(dst) + s.dst, s.src, s.bytes);
     return MK_OK;
 }

@@ -23,6 +23,7 @@
 //    counter that its items' heads increment after storing a split-K partial;
 //    the item that completes it merges the pair. No instruction waits on it.
 #include <algorithm>
+#include <new>
 #include <numeric>
 #include <queue>
 #include <random>
@@ -62,11 +63,15 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     return sp;
 }
 
+// the most SMs a plan may spread over (a B200 has 148)
+constexpr int kMaxPlanSms = 1024;
+
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out) {
     mk_schedule_opts o{};
     if (opts) o = *opts;
-    if (batch < 1 || batch > kMaxBatch || max_ctx < 1 || n_sm < 1) return MK_ERR_INVALID_ARG;
+    if (batch < 1 || batch > kMaxBatch || max_ctx < 1 || n_sm < 1 || n_sm > kMaxPlanSms)
+        return MK_ERR_INVALID_ARG;
     if (stage_bytes == 0) stage_bytes = default_stage_bytes(L);
     if (stage_bytes % 128 || stage_bytes < default_stage_bytes(L)) return MK_ERR_INVALID_ARG;
     const SlotPlan sp = slot_plan(L, batch, stage_bytes);
@@ -338,11 +343,9 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     return MK_OK;
 }
 
-}  // namespace mk
-
-extern "C" mk_status mk_plan_schedule_host(const mk_config* cfg, int batch, int max_ctx, int n_sm,
-                                           const mk_schedule_opts* opts, mk_instr* instr_out,
-                                           size_t cap, int32_t* sm_offsets, mk_schedule_info* info) {
+// mk_plan_schedule_host's body (the C entry point below keeps exceptions inside)
+mk_status plan_schedule_host(const mk_config* cfg, int batch, int max_ctx, int n_sm, const mk_schedule_opts* opts,
+                             mk_instr* instr_out, size_t cap, int32_t* sm_offsets, mk_schedule_info* info) {
     if (!cfg) return MK_ERR_INVALID_ARG;
     mk::Layout L;
     if (!mk::make_layout(*cfg, &L, nullptr)) return MK_ERR_UNSUPPORTED;
@@ -357,4 +360,17 @@ extern "C" mk_status mk_plan_schedule_host(const mk_config* cfg, int batch, int 
         std::copy(P.instrs.begin(), P.instrs.end(), instr_out);
     }
     return MK_OK;
+}
+}  // namespace mk
+
+extern "C" mk_status mk_plan_schedule_host(const mk_config* cfg, int batch, int max_ctx, int n_sm,
+                                           const mk_schedule_opts* opts, mk_instr* instr_out,
+                                           size_t cap, int32_t* sm_offsets, mk_schedule_info* info) {
+    try {
+        return mk::plan_schedule_host(cfg, batch, max_ctx, n_sm, opts, instr_out, cap, sm_offsets, info);
+    } catch (const std::bad_alloc&) {
+        return MK_ERR_OUT_OF_MEMORY;
+    } catch (...) {
+        return MK_ERR_INVALID_ARG;
+    }
 }

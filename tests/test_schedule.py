@@ -335,3 +335,24 @@ def test_attention_sms_take_fewer_gateup_tiles_when_items_are_few():
             assert fewer == layers, (fewer, layers)
         else:
             assert fewer < layers
+
+
+def test_planner_refuses_degenerate_arguments():
+    """Zero or negative sizes, a batch above the cache's, a context above max_seq,
+    an SM count far above any GPU's and a too-small output array are refused with
+    MK_ERR_INVALID_ARG; nothing throws through the C boundary."""
+    import ctypes
+    L = _lib.lib()
+    c = _lib.make_config(TINY, 2, 64)
+    info = _lib.MkScheduleInfo()
+
+    def rc(batch, ctx, n_sm):
+        return L.mk_plan_schedule_host(ctypes.byref(c), batch, ctx, n_sm, None, None, 0, None,
+                                       ctypes.byref(info))
+    assert rc(1, 64, 148) == 0
+    for args in ((0, 64, 148), (-1, 64, 148), (3, 64, 148), (1, 0, 148), (1, 65, 148),
+                 (1, 64, 0), (1, 64, -5), (1, 64, 1 << 30)):
+        assert rc(*args) == 1, args
+    instrs = (_lib.MkInstr * 1)()
+    assert L.mk_plan_schedule_host(ctypes.byref(c), 1, 64, 148, None, instrs, 1, None,
+                                   ctypes.byref(info)) == 1
