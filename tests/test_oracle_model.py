@@ -169,3 +169,75 @@ def test_bad_inputs_rejected_without_writes(setup):
     with pytest.raises(ValueError):
         om.decode_step(np.array([1]), np.array([160]), kc[:, :1].copy(), vc[:, :1].copy())
     assert np.array_equal(kc, k0)
+
+
+# The 3B-style head layout (head_dim 128, 3 query heads per KV head) on a small model:
+# the same pins as above for the shape the batch-8 workload uses.
+def _small_3b_style():
+    import dataclasses
+    from persistent_megakernel_interpreter_b200.config import LLAMA_3B
+    return dataclasses.replace(LLAMA_3B, name="3b-heads-small", n_layers=2, hidden=768, n_heads=6,
+                               n_kv_heads=2, ffn=2048, vocab=4096)
+
+
+@pytest.fixture(scope="module")
+def setup_3b_heads():
+    cfg = _small_3b_style()
+    w = make_weights(cfg, seed=7, norm_jitter=0.1)
+    k, v = make_kv_cache(cfg, batch=3, max_seq=96, past=[95, 0, 33], seed=8)
+    toks = make_tokens(cfg, 3, seed=9).numpy()
+    return cfg, w, k, v, toks
+
+
+def test_oracle_vs_fp64_brute_3b_head_layout(setup_3b_heads):
+    cfg, w, k, v, toks = setup_3b_heads
+    assert cfg.head_dim == 128 and cfg.group == 3
+    om = oracle.Model(cfg, w)
+    kc, vc = _np_cache(k), _np_cache(v)
+    pos = np.array([95, 0, 33], np.int32)
+    logits = om.decode_step(toks, pos, kc, vc)
+    br = Brute(cfg, w)
+    for b in range(3):
+        K, V = _brute_caches(cfg, k, v, b)
+        ref = br.decode_step(int(toks[b]), int(pos[b]), K, V, rounding=True)
+        assert np.max(np.abs(logits[b] - ref)) <= 1e-5 * np.max(np.abs(ref)), b
+        assert int(np.argmax(logits[b])) == int(np.argmax(ref))
+
+
+def test_oracle_vs_transformers_llama_3b_head_layout(setup_3b_heads):
+    """The library reduction again, for head_dim 128 and 3 query heads per KV head
+    (HF's repeat_kv maps query head h to KV head h // 3, as the oracle does)."""
+    from transformers import LlamaConfig, LlamaForCausalLM
+    from transformers.cache_utils import DynamicCache
+    cfg, w, k, v, toks = setup_3b_heads
+    hc = LlamaConfig(vocab_size=cfg.vocab, hidden_size=cfg.hidden, intermediate_size=cfg.ffn,
+                     num_hidden_layers=cfg.n_layers, num_attention_heads=cfg.n_heads,
+                     num_key_value_heads=cfg.n_kv_heads, head_dim=cfg.head_dim,
+                     rms_norm_eps=cfg.rms_eps, rope_theta=cfg.rope_theta,
+                     tie_word_embeddings=True, max_position_embeddings=4096,
+                     attention_bias=False, mlp_bias=False)
+    hc._attn_implementation = "eager"
+    model = LlamaForCausalLM(hc).to(torch.float64).eval()
+    sd = {"model.embed_tokens.weight": w.embed, "model.norm.weight": w.final_norm,
+          "lm_head.weight": w.embed}
+    for l in range(cfg.n_layers):
+        p = f"model.layers.{l}."
+        sd.update({p + "self_attn.q_proj.weight": w.wq[l], p + "self_attn.k_proj.weight": w.wk[l],
+                   p + "self_attn.v_proj.weight": w.wv[l], p + "self_attn.o_proj.weight": w.wo[l],
+                   p + "mlp.gate_proj.weight": w.wgate[l], p + "mlp.up_proj.weight": w.wup[l],
+                   p + "mlp.down_proj.weight": w.wdown[l], p + "input_layernorm.weight": w.attn_norm[l],
+                   p + "post_attention_layernorm.weight": w.mlp_norm[l]})
+    model.load_state_dict({n: t.to(torch.float64) for n, t in sd.items()}, strict=False)
+    om = oracle.Model(cfg, w)
+    b, pos = 2, 33
+    kc, vc = _np_cache(k)[:, b:b + 1].copy(), _np_cache(v)[:, b:b + 1].copy()
+    ours = om.decode_step(toks[b:b + 1], np.array([pos], np.int32), kc, vc)
+    cache = DynamicCache()
+    for l in range(cfg.n_layers):
+        cache.update(k[l, b, :, :pos].to(torch.float64)[None], v[l, b, :, :pos].to(torch.float64)[None], l)
+    with torch.no_grad():
+        out = model(input_ids=torch.tensor([[int(toks[b])]]), position_ids=torch.tensor([[pos]]),
+                    past_key_values=cache, use_cache=True)
+    ref = out.logits[0, -1].numpy()
+    assert np.max(np.abs(ours[0] - ref)) <= 1e-2 * np.max(np.abs(ref))
+    assert int(np.argmax(ours[0])) == int(np.argmax(ref))
