@@ -163,25 +163,24 @@ static mk_status create_impl(const mk_config* cfg, const mk_weights* w, int devi
     h->device = device;
     h->cfg = *cfg;
     h->lay = L;
-    auto bail = [](mk_status s) { return s; };
     DeviceScope scope;
     cudaError_t e = scope.enter(device);
-    if (e != cudaSuccess) return bail(MK_ERR_CUDA);
+    if (e != cudaSuccess) return MK_ERR_CUDA;
     if (cudaDeviceGetAttribute(&h->dev_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
-        return bail(MK_ERR_CUDA);
+        return MK_ERR_CUDA;
     int coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
-    if (!coop) return bail(MK_ERR_UNSUPPORTED);
+    if (!coop) return MK_ERR_UNSUPPORTED;
 
-    if (cudaMalloc(&h->packed, L.total) != cudaSuccess) return bail(MK_ERR_OUT_OF_MEMORY);
+    if (cudaMalloc(&h->packed, L.total) != cudaSuccess) return MK_ERR_OUT_OF_MEMORY;
     // pack: gather segments on the device (bit copy)
     {
         std::vector<mk::Segment> segs = mk::pack_segments(L, *w);
         for (const mk::Segment& s : segs)
-            if ((reinterpret_cast<uintptr_t>(s.src) | s.dst | s.bytes) & 15) return bail(MK_ERR_INVALID_ARG);
+            if ((reinterpret_cast<uintptr_t>(s.src) | s.dst | s.bytes) & 15) return MK_ERR_INVALID_ARG;
         mk::Segment* d_segs = nullptr;
         if (cudaMalloc(&d_segs, segs.size() * sizeof(mk::Segment)) != cudaSuccess)
-            return bail(MK_ERR_OUT_OF_MEMORY);
+            return MK_ERR_OUT_OF_MEMORY;
         e = cudaMemcpy(d_segs, segs.data(), segs.size() * sizeof(mk::Segment), cudaMemcpyHostToDevice);
         if (e == cudaSuccess) e = cudaMemset(h->packed, 0, L.total);
         if (e == cudaSuccess) {
@@ -190,7 +189,7 @@ static mk_status create_impl(const mk_config* cfg, const mk_weights* w, int devi
         }
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         cudaFree(d_segs);
-        if (e != cudaSuccess) return bail(MK_ERR_CUDA);
+        if (e != cudaSuccess) return MK_ERR_CUDA;
     }
     // RoPE table: angle pos * theta^(-2i/d) in double, cos/sin stored as float
     {
@@ -204,10 +203,10 @@ static mk_status create_impl(const mk_config* cfg, const mk_weights* w, int devi
                 tab[(size_t)cfg->max_seq * half + (size_t)pos * half + i] = (float)sin(ang);
             }
         if (cudaMalloc(&h->rope, tab.size() * sizeof(float)) != cudaSuccess)
-            return bail(MK_ERR_OUT_OF_MEMORY);
+            return MK_ERR_OUT_OF_MEMORY;
         if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float), cudaMemcpyHostToDevice) !=
             cudaSuccess)
-            return bail(MK_ERR_CUDA);
+            return MK_ERR_CUDA;
     }
     owner.h = nullptr;
     *out = h;
