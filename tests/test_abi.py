@@ -65,3 +65,30 @@ def test_create_rejects_unsupported_shapes():
         assert lib.mk_packed_bytes(ctypes.byref(c)) == 0, field
     assert lib.mk_packed_bytes(ctypes.byref(_lib.make_config(TINY, 1, (1 << 20) + 1))) == 0
     assert lib.mk_packed_bytes(ctypes.byref(_lib.make_config(TINY, 1, 1 << 20))) > 0
+
+
+def test_header_is_plain_c_and_a_c_program_links_against_the_library(tmp_path):
+    """include/mk.h compiles as C99 with warnings as errors, and a C program that
+    takes the address of every declared entry point links against libmk.so."""
+    import shutil
+    import subprocess
+    from persistent_megakernel_interpreter_b200 import build
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        import pytest
+        pytest.skip("gcc not available")
+    names = declared_functions()
+    src = tmp_path / "use_mk.c"
+    src.write_text("#include \"mk.h\"\n#include <stdio.h>\n"
+                   "typedef void (*any_fn)(void);\n"
+                   "int main(void) {\n"
+                   "    any_fn fns[] = {" + ", ".join(f"(any_fn)&{n}" for n in names) + "};\n"
+                   "    printf(\"%d %s\\n\", (int)(sizeof fns / sizeof fns[0]), mk_status_str(MK_OK));\n"
+                   "    return 0;\n}\n")
+    exe = tmp_path / "use_mk"
+    libdir = os.path.dirname(build.LIB)
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           f"-I{os.path.join(ROOT, 'include')}", str(src), "-o", str(exe),
+                           f"-L{libdir}", "-l:libmk.so", f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out == [str(len(names)), "ok"]
