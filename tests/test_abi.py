@@ -92,3 +92,43 @@ def test_header_is_plain_c_and_a_c_program_links_against_the_library(tmp_path):
                            f"-L{libdir}", "-l:libmk.so", f"-Wl,-rpath,{libdir}"])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out == [str(len(names)), "ok"]
+
+
+def test_ctypes_declarations_match_the_c_header(tmp_path):
+    """Every ctypes structure of the binding has the size and field offsets the C
+    compiler gives the header's struct, and the status and opcode numbers agree."""
+    import shutil
+    import subprocess
+    from persistent_megakernel_interpreter_b200 import _lib
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        import pytest
+        pytest.skip("gcc not available")
+    structs = {"mk_config": _lib.MkConfig, "mk_weights": _lib.MkWeights,
+               "mk_schedule_opts": _lib.MkScheduleOpts, "mk_instr": _lib.MkInstr,
+               "mk_schedule_info": _lib.MkScheduleInfo}
+    lines = []
+    want = []
+    for cname, py in structs.items():
+        lines.append(f'printf("%zu\\n", sizeof({cname}));')
+        want.append(ctypes.sizeof(py))
+        for fname, _ in py._fields_:
+            lines.append(f'printf("%zu\\n", offsetof({cname}, {fname}));')
+            want.append(getattr(py, fname).offset)
+    for code, name in sorted(_lib.STATUS.items()):
+        lines.append(f'printf("%d\\n", (int){name});')
+        want.append(code)
+    for name in ("QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD"):
+        lines.append(f'printf("%d\\n", (int)MK_OP_{name});')
+        want.append(getattr(_lib, f"OP_{name}"))
+    lines.append('printf("%u\\n", (unsigned)MK_NO_COUNTER);')
+    want.append(_lib.NO_COUNTER)
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"mk.h\"\nint main(void) {\n    "
+                   + "\n    ".join(lines) + "\n    return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", f"-I{os.path.join(ROOT, 'include')}",
+                           str(src), "-o", str(exe)])
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert got == want
