@@ -1,9 +1,12 @@
 """Weight packer: host packing equals the layout documented in include/mk.h,
 re-derived here independently by unpacking (bit-exact round trip)."""
+import dataclasses
+
 import numpy as np
+import pytest
 import torch
 
-from persistent_megakernel_interpreter_b200.config import TINY, ModelConfig
+from persistent_megakernel_interpreter_b200.config import LLAMA_3B, TINY, ModelConfig
 from persistent_megakernel_interpreter_b200.inputs import make_weights
 from persistent_megakernel_interpreter_b200.model import pack_weights_host
 
@@ -66,8 +69,14 @@ def unpack(cfg: ModelConfig, buf: np.ndarray):
     return E, layers, norms
 
 
-def test_pack_roundtrip_bit_exact():
-    cfg = TINY
+# the 2-layer model, and the 3B-style head layout (head_dim 128, 3 query heads per KV
+# head) on a small model
+SHAPES = [TINY, dataclasses.replace(LLAMA_3B, name="3b-heads-small", n_layers=2, hidden=768, n_heads=6,
+                                    n_kv_heads=2, ffn=2048, vocab=4096)]
+
+
+@pytest.mark.parametrize("cfg", SHAPES, ids=lambda c: c.name)
+def test_pack_roundtrip_bit_exact(cfg):
     w = make_weights(cfg, seed=7, norm_jitter=0.1)
     buf = pack_weights_host(cfg, w).numpy()
     E, layers, norms = unpack(cfg, buf)
@@ -80,9 +89,9 @@ def test_pack_roundtrip_bit_exact():
     assert np.array_equal(norms[2 * cfg.n_layers], _u16(w.final_norm))
 
 
-def test_pack_is_a_permutation_of_the_input_bytes():
+@pytest.mark.parametrize("cfg", SHAPES, ids=lambda c: c.name)
+def test_pack_is_a_permutation_of_the_input_bytes(cfg):
     """Every input element appears exactly once; the rest of the buffer is zero padding."""
-    cfg = TINY
     w = make_weights(cfg, seed=8, norm_jitter=0.1)
     buf = pack_weights_host(cfg, w).numpy().view(np.uint16)
     parts = [_u16(w.embed).ravel(), _u16(w.final_norm)]
