@@ -356,3 +356,30 @@ def test_planner_refuses_degenerate_arguments():
     instrs = (_lib.MkInstr * 1)()
     assert L.mk_plan_schedule_host(ctypes.byref(c), 1, 64, 148, None, instrs, 1, None,
                                    ctypes.byref(info)) == 1
+
+
+@pytest.mark.parametrize("cfg,batch,ctx,n_sm", [
+    (TINY, 5, 77, 148), (TINY, 7, 321, 100), (TINY, 8, 1, 148), (TINY, 4, 2048, 132),
+    (LLAMA_1B, 2, 1025, 148), (LLAMA_1B, 3, 4097, 148), (LLAMA_1B, 8, 129, 132),
+    (LLAMA_3B, 1, 129, 148), (LLAMA_3B, 5, 700, 148), (LLAMA_3B, 6, 1500, 148),
+])
+def test_plan_valid_across_batches_contexts_and_sm_counts(cfg, batch, ctx, n_sm):
+    """Odd batches, a single key, contexts just past a partition boundary, and SM
+    counts other than the B200's: the plan covers every tile once, every waited
+    count equals the signals it receives, and a simulated step completes."""
+    instrs, offs, info = check_plan(cfg, batch, ctx, n_sm)
+    ok, ctr = simulate(instrs, offs, info.n_counters, info.n_stages, 1, cfg.group, info.n_parts)
+    assert ok, "simulated step did not complete"
+
+
+@pytest.mark.parametrize("cfg,batch,limit", [
+    (LLAMA_1B, 1, 16384), (LLAMA_1B, 4, 12288), (LLAMA_1B, 8, 16384),
+    (LLAMA_3B, 1, 10752), (LLAMA_3B, 2, 9216), (LLAMA_3B, 8, 6144),
+])
+def test_context_ceiling_is_the_documented_one(cfg, batch, limit):
+    """The largest max_ctx the planner accepts (32 partitions of at most one ring's
+    keys, and 512) is the one the header states; one key more is refused."""
+    _, _, info = plan_schedule(cfg, batch, limit, 148, max_batch=8, max_seq=limit + 1)
+    assert info.n_parts <= 32 and info.n_parts * info.part_keys >= limit
+    with pytest.raises(_lib.MkError):
+        plan_schedule(cfg, batch, limit + 1, 148, max_batch=8, max_seq=limit + 1)
