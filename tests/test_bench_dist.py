@@ -8,8 +8,6 @@ import socket
 import subprocess
 import sys
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 _WORKER = r"""

@@ -1,7 +1,5 @@
 """Whole-decoder pins for the CPU oracle on the 2-layer config: an fp64 brute
 force, the transformers Llama model, special cases and invariants."""
-import copy
-
 import numpy as np
 import pytest
 import torch
