@@ -189,7 +189,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     };
     std::vector<uint32_t> signals(nc, 0);
     const uint32_t kv_key_bytes = 2u * (uint32_t)L.d * 2u;
-    const int gu_tiles = L.F / 2, gu_chunk = L.F / 8;
+    const int gu_chunk = L.F / 8;
     for (int l = 0; l < L.L; ++l) {
         // QKV: tiles grouped by KV group
         // One job per SM even where its range crosses a KV-group boundary (one
