@@ -250,12 +250,6 @@ def run_mk(args):
     mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=past + 1)
     torch.cuda.empty_cache()
     sched_opts = {}
-    if args.l2_prefetch:
-        sched_opts["l2_prefetch_fills"] = args.l2_prefetch
-    if args.l2_evict_normal:
-        sched_opts["l2_prefetch_policy"] = 1
-    if args.max_inflight:
-        sched_opts["max_inflight"] = args.max_inflight
     if args.part_keys:
         sched_opts["part_keys"] = args.part_keys
     info = mk.build_schedule(BATCH, past + 1, **sched_opts)
@@ -503,11 +497,6 @@ def parse_args(argv=None):
                     help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
                          "small profiling captures of the same kernels)")
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
-    ap.add_argument("--l2-prefetch", type=int, default=0,
-                    help="L2 prefetch distance in fills (0 = library default, -1 = off)")
-    ap.add_argument("--l2-evict-normal", action="store_true",
-                    help="L2 prefetches with an evict-normal hint (default: evict-last)")
-    ap.add_argument("--max-inflight", type=int, default=0, help="ring fills in flight at most (0 = default)")
     ap.add_argument("--part-keys", type=int, default=0,
                     help="keys per attention partition (0 = the schedule builder's choice)")
     ap.add_argument("--greedy", type=int, default=0, metavar="N",

@@ -107,13 +107,8 @@ typedef struct mk_schedule_opts {
                                 partition per (sequence, KV group) up to 320 keys, beyond
                                 that as many as leave one item per SM (each of at most
                                 512 keys and what the ring holds) */
-    int32_t tiles_qkv;       /* reserved, ignored (QKV, O-proj, gate/up and the LM head
-                                are placed one job per SM per op) */
-    int32_t tiles_o;         /* reserved, ignored */
-    int32_t tiles_gateup;    /* reserved, ignored */
     int32_t rowblocks_down;  /* 4-row blocks per down-projection instruction at most
                                 (1..16); 0 = 16 */
-    int32_t tiles_lm;        /* reserved, ignored */
     uint32_t seed;           /* 0 = plain greedy placement; else ties are broken by a
                                 seeded shuffle (for robustness tests) */
     int32_t wait_timeout_ms; /* budget of every device wait; 0 = 2000 ms */
@@ -123,16 +118,6 @@ typedef struct mk_schedule_opts {
                                 step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
-    int32_t l2_prefetch_fills; /* a prefetch warp pulls the SM's upcoming fills into L2, at
-                                most this many fills ahead of the loader's next one, so HBM
-                                keeps streaming while the compute warps wait on
-                                activations; 0 or negative = off (the default: on the 1B
-                                decode step the extra requests delay the cross-SM
-                                activation loads on the critical path, measured slower) */
-    int32_t l2_prefetch_policy; /* L2 eviction hint of those prefetches: 0 = evict-last,
-                                   1 = evict-normal */
-    int32_t max_inflight;    /* ring fills the loader keeps in flight at most (landed fills
-                                still fill the whole ring); 0 = no limit */
 } mk_schedule_opts;
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)

@@ -28,11 +28,9 @@ class MkWeights(ctypes.Structure):
 
 
 class MkScheduleOpts(ctypes.Structure):
-    _fields_ = [("n_sm", I32), ("part_keys", I32), ("tiles_qkv", I32), ("tiles_o", I32),
-                ("tiles_gateup", I32), ("rowblocks_down", I32), ("tiles_lm", I32),
+    _fields_ = [("n_sm", I32), ("part_keys", I32), ("rowblocks_down", I32),
                 ("seed", ctypes.c_uint32), ("wait_timeout_ms", I32), ("test_drop_item", I32),
-                ("trace", I32), ("l2_prefetch_fills", I32), ("l2_prefetch_policy", I32),
-                ("max_inflight", I32)]
+                ("trace", I32)]
 
 
 class MkInstr(ctypes.Structure):

@@ -328,9 +328,6 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
         MK_CUDA(h, cudaMalloc(&h->d_trace, tb));
         MK_CUDA(h, cudaMemset(h->d_trace, 0, tb));
     }
-    p.l2_prefetch_fills = (opts && opts->l2_prefetch_fills > 0) ? opts->l2_prefetch_fills : 0;
-    p.l2_prefetch_policy = (opts && opts->l2_prefetch_policy == 1) ? 1 : 0;
-    p.max_inflight = (opts && opts->max_inflight > 0 && opts->max_inflight < I.n_stages) ? opts->max_inflight : 0;
     p.trace = h->d_trace;
     p.trace_jobs = h->trace_jobs;
     p.timeout_ns = mk::kDefaultTimeoutNs;

@@ -29,8 +29,6 @@
 //    same jobs: it stages the RoPE rows of QKV jobs and, at batch 1, the h chunk
 //    (and with the last chunk the residual rows) of each down-projection job,
 //    which gate/up completes chunk by chunk while it still streams.
-//  * Warp 10 (the prefetch warp) is optional and off by default: bulk L2
-//    prefetches of the fills a bounded distance past the loader.
 //  * Attention items finish their own heads: with one key partition per
 //    (sequence, KV group) the item writes o / l; with several, each stores its
 //    partial and the one that completes the pair's arrival count merges the
@@ -40,11 +38,25 @@
 //  * Every wait is bounded by a time budget; on expiry the step records
 //    MK_ERR_TIMEOUT, raises an abort flag that every other wait polls, drains
 //    its own copies in flight and returns. No trap, no unbounded spin.
+//
+// This file is compiled twice: as is, and with MK_TRACE=1 (megakernel_trace.cu)
+// into a second namespace whose kernels also record per-job timestamps. The
+// timestamps stay out of the production kernels altogether: the code a kernel
+// carries is what every SM re-fetches as it moves between ops.
 #include <cuda_runtime.h>
 
 #include "mk_device.cuh"
 
+#ifndef MK_TRACE
+#define MK_TRACE 0
+#endif
+
 namespace mk {
+#if MK_TRACE
+namespace traced {
+#else
+namespace plain {
+#endif
 
 // Each sequence's position, read once per step by thread 0 (constant during
 // the step) so the warps do not reload it from global memory.
@@ -88,7 +100,7 @@ __device__ __forceinline__ uint32_t gu_tile(const Params& p, const mk_instr& in,
 
 // ------------------------------------------------------------------ errors and waits
 
-__device__ void record_error(const Params& p, uint32_t code, uint32_t a, uint32_t b, uint32_t c,
+__device__ __noinline__ void record_error(const Params& p, uint32_t code, uint32_t a, uint32_t b, uint32_t c,
                              uint32_t d, uint32_t e) {
     if (atomicCAS(&p.ctl->status, 0u, code) == 0u) {
         p.ctl->info[0] = blockIdx.x;
@@ -111,9 +123,10 @@ __device__ __forceinline__ bool aborted(const Params& p) {
 // All lanes wait for phase `parity` of an mbarrier; warp-uniform exit. With
 // `armed`, first wait until the ring stage holds fill `seq`. Waiting threads
 // sleep in the barrier (suspend hint) or back off, so they do not compete for
-// issue slots with the warps that compute.
-__device__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const volatile uint32_t* armed,
-                         uint32_t seq, uint32_t site, int lane) {
+// issue slots with the warps that compute. Out of line: the inline wait_bar
+// below tries once first.
+__device__ __noinline__ bool wait_bar_slow(const Params& p, uint64_t* bar, uint32_t parity,
+                                           const volatile uint32_t* armed, uint32_t seq, uint32_t site, int lane) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         bool done;
@@ -139,6 +152,13 @@ __device__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const 
     }
 }
 
+__device__ __forceinline__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const volatile uint32_t* armed,
+                                         uint32_t seq, uint32_t site, int lane) {
+    const bool ready = (armed == nullptr || *armed == seq) && mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, ready)) return true;
+    return wait_bar_slow(p, bar, parity, armed, seq, site, lane);
+}
+
 __device__ __forceinline__ bool wait_fill(const Params& p, const Ring& r, uint32_t seq, int lane) {
     const uint32_t s = seq % r.S;
     return wait_bar(p, r.full + s, (seq / r.S) & 1u, r.armed + s, seq, 2, lane);
@@ -155,12 +175,8 @@ __device__ __forceinline__ void release_fill(const Ring& r, uint32_t seq, int la
 // The wait is a short spin on the non-blocking probe: the warps arrive within a
 // few hundred cycles of each other, and a sleeping waiter would add its wake-up
 // latency to every pass.
-__device__ __forceinline__ bool compute_barrier(const Params& p, uint64_t* cbar, uint32_t& uses,
-                                                int lane) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(cbar);
-    const uint32_t parity = uses & 1u;
-    ++uses;
+__device__ __noinline__ bool compute_barrier_wait(const Params& p, uint64_t* cbar, uint32_t uses, uint32_t parity,
+                                                  int lane) {
     uint64_t t0 = 0;
     for (uint32_t it = 0; !__all_sync(0xffffffffu, mbar_test_wait(cbar, parity)); ++it) {
         if ((it & 1023u) == 1023u) {
@@ -179,6 +195,15 @@ __device__ __forceinline__ bool compute_barrier(const Params& p, uint64_t* cbar,
     return true;
 }
 
+__device__ __forceinline__ bool compute_barrier(const Params& p, uint64_t* cbar, uint32_t& uses, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(cbar);
+    const uint32_t parity = uses & 1u;
+    ++uses;
+    if (__all_sync(0xffffffffu, mbar_test_wait(cbar, parity))) return true;
+    return compute_barrier_wait(p, cbar, uses, parity, lane);
+}
+
 // ------------------------------------------------------------------ activation warp
 
 // The down-projection's chunk-c target (chunks may have different job counts).
@@ -193,11 +218,19 @@ __device__ __forceinline__ void xs_store(float* v, int KC, int e, float x) {
     arr[g8 * 4 + (i & 3)] = x;
 }
 
-// Optional per-job timestamps (see TraceWord).
+// Per-job timestamps (see TraceWord), in the traced build only.
+#if MK_TRACE
 __device__ __forceinline__ void trace(const Params& p, uint32_t job, int word, uint64_t v) {
     if (p.trace != nullptr && job < (uint32_t)p.trace_jobs)
         p.trace[((size_t)blockIdx.x * p.trace_jobs + job) * kTraceWords + word] = v;
 }
+__device__ __forceinline__ void trace(const Params& p, uint32_t job, int word) {
+    trace(p, job, word, global_timer_ns());
+}
+#else
+__device__ __forceinline__ void trace(const Params&, uint32_t, int, uint64_t) {}
+__device__ __forceinline__ void trace(const Params&, uint32_t, int) {}
+#endif
 
 
 // Pause between polls of tagged words that have not arrived yet, bounded by
@@ -221,8 +254,8 @@ __device__ __forceinline__ bool tag_backoff(const Params& p, uint32_t it, uint64
 // A job's input vector from the tagged activations, by all compute warps (the
 // thread's pairs, all loads in flight at once, retried until every tag is the
 // expected one); RMSNorm with the bf16 norm weights w when w is given. Ends
-// with a compute barrier.
-__device__ bool block_input_tagged(const Params& p, const uint64_t* src, uint32_t tag, const uint16_t* w, int n,
+// with a compute barrier. Out of line: one copy for every job that needs it.
+__device__ __noinline__ bool block_input_tagged(const Params& p, const uint64_t* src, uint32_t tag, const uint16_t* w, int n,
                                    float* xs, float* red, int t, int warp, int lane, uint64_t* cbar,
                                    uint32_t& cuses) {
     const int np = n / 2;
@@ -283,11 +316,13 @@ __device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) 
 // layer 0) for QKV, gate/up and the LM head; the attention output and the
 // residual rows (x before the O-projection, or the embedding row) for the
 // O-projection. (The down-projection's inputs are staged by the activation warp.)
+template <bool BATCHED>
 __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
                           uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
     const int t = warp * 32 + lane, l = in.layer;
     auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
-    for (int b = 0; b < p.B; ++b) {
+    const int B = BATCHED ? p.B : 1;
+    for (int b = 0; b < B; ++b) {
         float* xs = sv + (size_t)b * p.xs_vec_floats;
         switch (in.op) {
             case MK_OP_QKV:
@@ -431,12 +466,12 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
                          uint32_t job) {
     const mk_instr& in = ins[0];
     float* sv = reinterpret_cast<float*>(slot);
-    if (lane == 0) trace(p, job, kTrCtrDone, global_timer_ns());
+    if (lane == 0) trace(p, job, kTrCtrDone);
     if (!BATCHED && in.op == MK_OP_DOWN) {
         // down chunk c: h chunk c (gate/up runs chunk-major, so chunks complete one
         // after another while gate/up still streams) and, with the last chunk, the
         // residual rows (x after attention), staged ahead of the compute warps
-        for (int b = 0; b < p.B; ++b) {
+        for (int b = 0; b < (BATCHED ? p.B : 1); ++b) {
             if (!warp_load_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, in.layer, kTagH),
                                   p.F / 4, sv + (size_t)b * p.xs_vec_floats, 8, lane))
                 return false;
@@ -462,7 +497,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
     }
     if (in.op == MK_OP_QKV) {
         float* aux = sv + (size_t)p.B * p.xs_vec_floats;
-        for (int b = 0; b < p.B; ++b) {
+        for (int b = 0; b < (BATCHED ? p.B : 1); ++b) {
             const int pos = g_pos[b];
             float* row = aux + (size_t)b * (HD + 4);
             for (int i = lane; i < HD / 2; i += 32) {
@@ -485,15 +520,15 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS, use = j / sl.NS;
             if (lane == 0) {
-                trace(p, j, kTrSlotWait, global_timer_ns());
+                trace(p, j, kTrSlotWait);
                 trace(p, j, kTrMeta, op | ((uint32_t)ins[0].layer << 8) | ((uint32_t)c << 24));
             }
             if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
-            if (lane == 0) trace(p, j, kTrCtrWait, global_timer_ns());
+            if (lane == 0) trace(p, j, kTrCtrWait);
             if (!prep_job<HD, BATCHED>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
             if (lane == 0) {
-                trace(p, j, kTrReady, global_timer_ns());
+                trace(p, j, kTrReady);
                 mbar_arrive(sl.full + s);  // release: the slot's contents
             }
         }
@@ -515,21 +550,7 @@ __device__ __noinline__ float4 tile_dot(const uint8_t* tile, const float* v, int
     return make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
-// The tile against every sequence's input (B > 1): lane l returns the total of
-// sequence l / 4, row l % 4 (see dot4_batch).
-template <int KC>
-__device__ __noinline__ float tile_dot_batch(const uint8_t* tile, const float* sv, uint32_t vec_floats, int B,
-                                             int lane) {
-    return dot4_batch<KC>(tile, sv, vec_floats, B, lane);
-}
-
-// The four rows of sequence lane / 4 gathered from the batched totals, for the
-// 4-row epilogues (lane l then acts as lane l % 4 of sequence l / 4).
-__device__ __forceinline__ void gather4(float tot, int lane, float (&acc)[4]) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) acc[r] = __shfl_sync(0xffffffffu, tot, (lane & ~3) + r);
-}
-
+// Batch 1 (batch > 1 runs compute_tiles_pair).
 template <int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
                               const float* sv, int warp, int lane, uint32_t job, uint32_t epoch) {
@@ -537,34 +558,24 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
     const bool pub = in.signal_ctr != MK_NO_COUNTER;
     int k = 0;  // trace: warp 0's first tiles (fill wait start, fill ready, dot done)
     auto stamp = [&](int w) {
-        if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w, global_timer_ns());
+        if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w);
     };
     for (uint32_t t = warp; t < in.count; t += kConsumerWarps) {
         const uint32_t seq = in.seq + t;
         if (k < 2) stamp(3 * k);
         if (!wait_fill(p, ring, seq, lane)) return false;
-        if (t == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
+        if (t == 0 && lane == 0) trace(p, job, kTrFill);
         if (k < 2) stamp(3 * k + 1);
         const uint8_t* tile = ring.stage(seq);
-        // batch 1: one pass, every lane holds the 4 totals; batch > 1: one pass over
-        // all sequences, lane l holds sequence l / 4 and acts as lane l % 4 for it
-        const bool batched = p.B > 1;
-        float tb = 0.f;
-        if (batched) tb = tile_dot_batch<KC>(tile, sv, p.xs_vec_floats, p.B, lane);
-        const int nb = batched ? 1 : p.B;
-        for (int bi = 0; bi < nb; ++bi) {
-            int b = bi, el = lane;
+        {
+            constexpr int b = 0;  // batch 1: every lane holds the 4 totals
+            const int el = lane;
             float acc[4];
-            if (batched) {
-                gather4(tb, lane, acc);
-                b = lane >> 2;
-                el = b < p.B ? (lane & 3) : 32;
-                if (b >= p.B) b = 0;
-            } else {
-                const float4 a4 = tile_dot<KC>(tile, sv + (size_t)b * p.xs_vec_floats, lane);
+            {
+                const float4 a4 = tile_dot<KC>(tile, sv, lane);
                 acc[0] = a4.x; acc[1] = a4.y; acc[2] = a4.z; acc[3] = a4.w;
             }
-            if (k < 2 && bi == 0) stamp(3 * k + 2);
+            if (k < 2) stamp(3 * k + 2);
             const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
             switch (in.op) {
                 case MK_OP_QKV: {
@@ -627,7 +638,7 @@ __device__ bool compute_tiles_pair(const Params& p, const Ring& ring, const mk_i
     for (uint32_t t = warp % kPairGroups; t < in.count; t += kPairGroups) {
         const uint32_t seq = in.seq + t;
         if (!wait_fill(p, ring, seq, lane)) return false;
-        if (t == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill, global_timer_ns());
+        if (t == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill);
         const float tb = tile_dot_batch4<KC>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
                                              p.xs_vec_floats, ps.nb, lane);
         float acc[4];
@@ -669,7 +680,7 @@ __device__ bool compute_down_pair(const Params& p, const Ring& ring, const mk_in
     for (uint32_t r = warp % kPairGroups; r < in.count; r += kPairGroups) {
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
-        if (r == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill, global_timer_ns());
+        if (r == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill);
         const float y = tile_dot_batch4<KF>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
                                             p.xs_vec_floats, ps.nb, lane);
         if (act) {
@@ -686,29 +697,22 @@ __device__ bool compute_down_pair(const Params& p, const Ring& ring, const mk_in
     return true;
 }
 
-// Down-projection, chunk c: row block r (warp r mod 8) adds W_d[:, chunk c] . h_c to
-// its running sums, chunks in order 0..3; after chunk 3 the residual.
+// Down-projection at batch 1 (batch > 1 runs compute_down_pair), chunk c: row
+// block r (warp r mod 8) adds W_d[:, chunk c] . h_c to its running sums, chunks in
+// order 0..3; after chunk 3 the residual.
 template <int KF>
 __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
                              const float* sv, float* tot, int warp, int lane, uint32_t job, uint32_t epoch) {
     for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
         const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
         if (!wait_fill(p, ring, seq, lane)) return false;
-        if (r == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
-        // batch > 1: one pass over all sequences, lane l holds sequence l / 4, row l % 4
-        const bool batched = p.B > 1;
-        float tb = 0.f;
-        if (batched) tb = tile_dot_batch<KF>(ring.stage(seq), sv, p.xs_vec_floats, p.B, lane);
-        const int nb = batched ? 1 : p.B;
-        for (int bi = 0; bi < nb; ++bi) {
-            int b = bi, row = lane;
+        if (r == 0 && lane == 0) trace(p, job, kTrFill);
+        {
+            constexpr int b = 0;  // batch 1
+            const int row = lane;
             float y = 0.f;
-            if (batched) {
-                b = lane >> 2;
-                row = b < p.B ? (lane & 3) : 32;
-                y = tb;
-            } else {
-                const float4 a4 = tile_dot<KF>(ring.stage(seq), sv + (size_t)b * p.xs_vec_floats, lane);
+            {
+                const float4 a4 = tile_dot<KF>(ring.stage(seq), sv, lane);
                 const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
                 if (lane < 4) y = pick4(acc, lane);
             }
@@ -742,7 +746,7 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     const int pos = g_pos[b];
     for (uint32_t f = 0; f < a.nfill; ++f)
         if (!wait_fill(p, ring, a.seq + f, lane)) return false;
-    if (warp == 0 && lane == 0) trace(p, job, kTrFill, global_timer_ns());
+    if (warp == 0 && lane == 0) trace(p, job, kTrFill);
     const float* qs = reinterpret_cast<const float*>(slot);
     const uint16_t* knew = reinterpret_cast<const uint16_t*>(slot + (size_t)G * HD * 4);
     const int jn = pos - (int)a.first;
@@ -751,21 +755,23 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
     // trace: warp 0 at the end of each phase and after each barrier
     auto mark = [&](int k) {
-        if (warp == 0 && lane == 0) trace(p, job, kTrSub0 + k, global_timer_ns());
+        if (warp == 0 && lane == 0) trace(p, job, kTrSub0 + k);
     };
     const int t = warp * 32 + lane;
     uint32_t* sig = p.counters + (size_t)a.signal_ctr * kCounterStride;
-    if (p.n_parts == 1) {
+    {
+        // one instance of the item's code for both outputs (the kernel's code size
+        // is what every SM re-fetches): o / l with one partition, else the partial
         uint64_t* out = p.attn_t + (size_t)b * p.Q + (size_t)g * G * HD;
         const uint32_t tag = act_tag(epoch, a.layer, kTagAttn);
         const bool pub = a.signal_ctr != MK_NO_COUNTER;  // a dropped item publishes nothing
-        if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark, [&](int h, int d, float o, float, float l) {
-                if (pub) st_tagged(out + h * HD + d, __fdiv_rn(o, l), tag);
-            }))
-            return false;
-    } else {
+        const bool single = p.n_parts == 1;
         const int part = (int)(a.first / (uint32_t)p.part_keys);
         if (!attn_item_block<HD>(R, qs, G, sc, warp, lane, bar, mark, [&](int h, int d, float o, float m, float l) {
+                if (single) {
+                    if (pub) st_tagged(out + h * HD + d, __fdiv_rn(o, l), tag);
+                    return;
+                }
                 const size_t hp = ((size_t)b * p.nq + (size_t)(g * G + h)) * p.n_parts + part;
                 p.part_o[hp * HD + d] = o;
                 if (d == 0) {
@@ -820,7 +826,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
         for (int c = 0; c < njobs; ++c, ++j) {
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, sl.full + s, (j / sl.NS) & 1u, nullptr, j, 4, lane)) return;
-            if (warp == 0 && lane == 0) trace(p, j, kTrStart, global_timer_ns());
+            if (warp == 0 && lane == 0) trace(p, j, kTrStart);
             float* sv = reinterpret_cast<float*>(sl.slot(j));
             // inputs: the attention item's q/k/v and every matvec input but the
             // down-projection's at batch 1 (staged by the activation warp) are
@@ -828,31 +834,25 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
                       : in.op == MK_OP_DOWN ? (!BATCHED || down_input_batch(p, in, c, sv, red, warp, lane, cbar,
                                                                             cuses, epoch))
-                                            : job_input(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
+                                            : job_input<BATCHED>(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
             if (!ok) return;
-            if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7, global_timer_ns());
-            switch (in.op) {
-                case MK_OP_QKV:
-                    if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    break;
-                case MK_OP_OPROJ:
+            if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7);
+            // one call site per routine: the kernel's code is what every SM re-fetches
+            // from L2 as it moves between ops, so nothing is inlined twice
+            if (in.op == MK_OP_ATTN) {
+                ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
+                                                   epoch);
+            } else if (in.op == MK_OP_DOWN) {
+                if constexpr (BATCHED) ok = compute_down_pair<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
+                else ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
+            } else if (KO != KH && in.op == MK_OP_OPROJ) {
+                if constexpr (KO != KH) {
                     if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
                     else ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    break;
-                case MK_OP_GATEUP:
-                case MK_OP_LMHEAD:
-                    if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    break;
-                case MK_OP_DOWN:
-                    if constexpr (BATCHED) ok = compute_down_pair<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
-                    else ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
-                    break;
-                default:
-                    ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
-                                                       epoch);
-                    break;
+                }
+            } else {  // QKV, gate/up, the LM head (and the O-projection when its width is the hidden size)
+                if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
             }
             if (!ok) return;
             // job done for this warp; the last of the 8 counts the job's completion
@@ -863,7 +863,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
                 const uint32_t old = atom_shared_acq_rel_add(sl.done + s, 1u);
                 if (old == kConsumerWarps - 1) {
                     sl.done[s] = 0;
-                    trace(p, j, kTrDone, global_timer_ns());
+                    trace(p, j, kTrDone);
                     // attention items signal their heads themselves (compute_attn_job)
                     const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN;
                     if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
@@ -922,8 +922,7 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
 
 // One thread streams the SM's fills into the ring, in list order; it never
 // waits on a dependency counter, only for the compute warps to release a stage.
-// `issued_out` publishes how many fills it has issued (for the prefetch warp).
-__device__ void loader(const Params& p, const Ring& ring, int i0, int i1, volatile uint32_t* issued_out) {
+__device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
     for (int i = i0; i < i1; ++i) {
@@ -948,23 +947,6 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1, volati
                 }
                 if (!ok) goto drain;
             }
-            if (p.max_inflight > 0 && seq >= (uint32_t)p.max_inflight) {
-                // At most max_inflight fills in flight: enough to keep HBM busy, few
-                // enough that the step's latency-critical loads do not queue behind
-                // megabytes of weight traffic. Landed fills still pile up in the ring.
-                const uint32_t o = seq - (uint32_t)p.max_inflight;
-                uint64_t t1 = 0;
-                for (uint32_t it = 0; !mbar_wait_sleep(ring.full + o % ring.S, (o / ring.S) & 1u, 500u); ++it) {
-                    if ((it & 15u) == 15u) {
-                        if (t1 == 0) t1 = global_timer_ns();
-                        if (aborted(p)) goto drain;
-                        if (global_timer_ns() - t1 > p.timeout_ns) {
-                            record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffbu, 0, o, 6);
-                            goto drain;
-                        }
-                    }
-                }
-            }
             {
                 uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
                 uint64_t* bar = ring.full + s;
@@ -982,11 +964,9 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1, volati
                 }
             }
             issued = seq + 1;
-            *issued_out = issued;
         }
     }
 drain:
-    *issued_out = 0xffffffffu;  // the prefetch warp stops at once
     // Every copy issued must land before the CTA may exit: wait for the last
     // fill of each stage used (earlier fills of a stage completed before it
     // could be refilled).
@@ -1003,52 +983,12 @@ drain:
     }
 }
 
-// One thread keeps HBM busy while the compute warps wait on activations: it
-// pulls the SM's next fills into L2 (bulk prefetch, evict-last by default),
-// at most `l2_prefetch_fills` fills ahead of the loader's next one. When the
-// ring is full of landed fills the loader stops, but the prefetches go on, so
-// the weights the SM needs after the wait are in L2 and the ring refills from
-// there. Fills the loader issues at launch (the first ring's worth) and fills it
-// has already issued are skipped. Every wait is bounded.
-__device__ void prefetcher(const Params& p, int i0, int i1, uint32_t S, const volatile uint32_t* issued) {
-    const uint32_t D = (uint32_t)p.l2_prefetch_fills;
-    if (D == 0) return;
-    const uint64_t pol = p.l2_prefetch_policy == 1 ? l2_evict_normal_policy() : l2_evict_last_policy();
-    uint32_t pf = 0;  // fill number
-    uint64_t t0 = 0;
-    for (int i = i0; i < i1; ++i) {
-        const mk_instr in = p.instrs[i];
-        for (uint32_t t = 0; t < in.nfill; ++t, ++pf) {
-            if (pf < S) continue;
-            uint32_t iss = *issued;
-            for (uint32_t it = 0; pf >= iss + D; ++it) {
-                __nanosleep(128);
-                iss = *issued;
-                if ((it & 63u) == 63u) {
-                    if (aborted(p)) return;
-                    if (t0 == 0) t0 = global_timer_ns();
-                    else if (global_timer_ns() - t0 > p.timeout_ns) return;
-                }
-            }
-            t0 = 0;
-            if (iss == 0xffffffffu) return;  // the loader has stopped
-            if (pf < iss) continue;           // already on its way to the ring
-            const FillSrc f = fill_source(p, in, t);
-            if (f.bytes) {
-                prefetch_l2(f.a, f.bytes, pol);
-                if (f.b) prefetch_l2(f.b, f.bytes, pol);
-            }
-        }
-    }
-}
-
 // ------------------------------------------------------------------ the kernel
 
 template <int KH, int KO, int KF, int HD, bool BATCHED>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
-    __shared__ volatile uint32_t s_issued;  // fills the loader has issued (all: ~0)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes);
     Ring ring;
@@ -1078,7 +1018,6 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             sl.done[s] = 0;
         }
         mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
-        s_issued = 0u;
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
         uint32_t skip = ld_volatile_u32(&p.ctl->status) != 0u;
@@ -1103,9 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (!s_skip) {
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
         if (warp == kLoaderWarp) {
-            if (lane == 0) loader(p, ring, i0, i1, &s_issued);
-        } else if (warp == kPrefetchWarp) {
-            if (lane == 0) prefetcher(p, i0, i1, ring.S, &s_issued);
+            if (lane == 0) loader(p, ring, i0, i1);
         } else if (warp == kPrepWarp) {
             activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch);
         } else {
@@ -1147,7 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 
 // ------------------------------------------------------------------ host-side launch
 
-size_t megakernel_smem_bytes(const Params& p) {
+size_t smem_bytes(const Params& p) {
     return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes).total;
 }
 
@@ -1168,32 +1105,32 @@ static KernelFn pick(int KH, int KO, int KF, int HD, int B) {
     return B > 1 ? pick_b<true>(KH, KO, KF, HD) : pick_b<false>(KH, KO, KF, HD);
 }
 
-bool megakernel_supported(int H, int Q, int F, int d) {
+static KernelFn pick(const Params& p) { return pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B); }
+
+bool supported(int H, int Q, int F, int d) {
     if (H % 256 || Q % 256 || F % 1024) return false;
     return pick(H / 256, Q / 256, F / 1024, d, 1) != nullptr;
 }
 
-cudaError_t megakernel_prepare(const Params& p) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
+cudaError_t prepare(const Params& p) {
+    KernelFn fn = pick(p);
     if (!fn) return cudaErrorInvalidValue;
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)megakernel_smem_bytes(p));
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(p));
 }
 
-cudaError_t megakernel_occupancy(const Params& p, int* blocks_per_sm) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
+cudaError_t occupancy(const Params& p, int* blocks_per_sm) {
+    KernelFn fn = pick(p);
     if (!fn) return cudaErrorInvalidValue;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, fn, kThreads,
-                                                         megakernel_smem_bytes(p));
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, fn, kThreads, smem_bytes(p));
 }
 
-cudaError_t megakernel_launch(const Params& p, cudaStream_t stream) {
-    KernelFn fn = pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B);
+cudaError_t launch(const Params& p, cudaStream_t stream) {
+    KernelFn fn = pick(p);
     if (!fn) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.n_sm);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = megakernel_smem_bytes(p);
+    cfg.dynamicSmemBytes = smem_bytes(p);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -1202,5 +1139,27 @@ cudaError_t megakernel_launch(const Params& p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, fn, p);
 }
+
+}  // namespace plain / traced
+
+#if !MK_TRACE
+// The library's entry points: the traced kernels when the schedule records
+// timestamps (p.trace set), else the plain ones.
+namespace traced {
+cudaError_t prepare(const Params& p);
+cudaError_t occupancy(const Params& p, int* blocks_per_sm);
+cudaError_t launch(const Params& p, cudaStream_t stream);
+}  // namespace traced
+
+size_t megakernel_smem_bytes(const Params& p) { return plain::smem_bytes(p); }
+bool megakernel_supported(int H, int Q, int F, int d) { return plain::supported(H, Q, F, d); }
+cudaError_t megakernel_prepare(const Params& p) { return p.trace ? traced::prepare(p) : plain::prepare(p); }
+cudaError_t megakernel_occupancy(const Params& p, int* blocks_per_sm) {
+    return p.trace ? traced::occupancy(p, blocks_per_sm) : plain::occupancy(p, blocks_per_sm);
+}
+cudaError_t megakernel_launch(const Params& p, cudaStream_t stream) {
+    return p.trace ? traced::launch(p, stream) : plain::launch(p, stream);
+}
+#endif
 
 }  // namespace mk

@@ -175,25 +175,6 @@ __device__ __forceinline__ uint32_t atom_shared_acq_rel_add(uint32_t* p, uint32_
     return old;
 }
 
-// Pull a byte range into L2 ahead of its use (no completion tracking).
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src),
-                 "r"(bytes), "l"(policy)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint64_t l2_evict_last_policy() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
 __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
     uint32_t old;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
@@ -851,6 +832,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         const int j_first = warp * S::KPW + kk;
         const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
         float mx = -INFINITY;
+#pragma unroll 1
         for (int j0 = j_first; j0 - kk < n; j0 += PBS * KPR) {
             float acc[PBS][kMaxGroup];
             float kv[PBS][8];
@@ -917,6 +899,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
     }
     {
         float ls[kMaxGroup] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
         for (int j = t; j < n; j += NT) {
             const float4 v = et[j];
             const float s[kMaxGroup] = {v.x, v.y, v.z, v.w};
@@ -943,6 +926,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         for (int h = 0; h < kMaxGroup; ++h) a[h][0] = a[h][1] = 0.f;
         const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
         const size_t vofs = (size_t)R.kps * HD;
+#pragma unroll 1
         for (int j0 = kq; j0 < nc; j0 += PBV * KQ) {
             uint32_t w[PBV];
             float4 e[PBV];
@@ -982,6 +966,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
     if (!bar()) return false;
     mark(5);
     // the class sums in class order, the warps' sums in warp order
+#pragma unroll 1
     for (int u = t; u < G * HD; u += NT) {
         const int h = u / HD, d = u % HD;
         float o = part[(size_t)h * HD + d];

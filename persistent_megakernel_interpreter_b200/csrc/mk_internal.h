@@ -17,9 +17,8 @@ namespace mk {
 
 constexpr int kConsumerWarps = 8;                    // compute warps
 constexpr int kLoaderWarp = kConsumerWarps;          // streams weights and cached KV
-constexpr int kPrepWarp = kConsumerWarps + 1;        // waits on counters, prepares inputs
-constexpr int kPrefetchWarp = kConsumerWarps + 2;    // pulls upcoming fills into L2
-constexpr int kThreads = 32 * (kConsumerWarps + 3);
+constexpr int kPrepWarp = kConsumerWarps + 1;        // stages RoPE rows and down-projection inputs
+constexpr int kThreads = 32 * (kConsumerWarps + 2);
 constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
 constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
 constexpr int kMaxResidRows = 64;                    // residual rows per O-proj / down job
@@ -150,9 +149,6 @@ struct Params {
     uint32_t xs_slot_bytes;
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
     int n_counters;
-    int l2_prefetch_fills;     // how far (in fills) the L2 prefetch may run ahead (0 = off)
-    int l2_prefetch_policy;    // 0: evict-last, 1: evict-normal
-    int max_inflight;          // ring fills the loader keeps in flight at most (0 = ring size)
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)
     uint64_t* trace;

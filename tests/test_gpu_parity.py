@@ -137,8 +137,8 @@ def test_schedule_placement_does_not_change_results(tiny):
     pos = [128, 57]
     info = tiny.mk.schedule_info()
     ref = tiny.gpu_step(toks, pos)
-    for opts in (dict(n_sm=37), dict(seed=99), dict(n_sm=5, tiles_lm=3, tiles_qkv=1),
-                 dict(rowblocks_down=3, tiles_gateup=8, tiles_o=1)):
+    for opts in (dict(n_sm=37), dict(seed=99), dict(n_sm=5), dict(n_sm=5, seed=7, rowblocks_down=1),
+                 dict(rowblocks_down=3)):
         tiny.mk.build_schedule(2, 160, part_keys=info.part_keys, **opts)
         assert np.array_equal(tiny.gpu_step(toks, pos), ref), opts
     tiny.mk.build_schedule(2, 160)
