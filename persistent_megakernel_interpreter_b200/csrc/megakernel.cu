@@ -26,9 +26,9 @@
 //    attention item), split the job's tiles (tile t goes to warp t mod 8) and
 //    write the outputs with fused epilogues.
 //  * Warp 9 (the activation warp) runs ahead of the compute warps through the
-//    same jobs: it stages the RoPE rows of QKV jobs and, at batch 1, the h chunk
-//    (and with the last chunk the residual rows) of each down-projection job,
-//    which gate/up completes chunk by chunk while it still streams.
+//    same jobs: it stages the RoPE rows of QKV jobs and, at batch 1, the h
+//    chunks of the first down-projection jobs, which gate/up completes chunk by
+//    chunk while it still streams (the compute warps load the last ones).
 //  * Attention items finish their own heads: with one key partition per
 //    (sequence, KV group) the item writes o / l; with several, each stores its
 //    partial and the one that completes the pair's arrival count merges the
@@ -63,6 +63,10 @@ namespace plain {
 __shared__ int g_pos[kMaxBatch];
 
 constexpr int kPairGroups = kConsumerWarps / 2;  // batch > 1: tiles in work at once (two warps each)
+// Batch 1: the activation warp stages the h chunks of down-projection chunks
+// c < kDownStaged ahead (they complete while gate/up still streams); the later
+// chunks, which complete only as gate/up ends, are loaded by all compute warps.
+constexpr int kDownStaged = 2;
 
 struct Ring {
     uint8_t* base;
@@ -315,7 +319,7 @@ __device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) 
 // words themselves): RMSNorm of x (tagged) or of the embedding row (QKV of
 // layer 0) for QKV, gate/up and the LM head; the attention output and the
 // residual rows (x before the O-projection, or the embedding row) for the
-// O-projection. (The down-projection's inputs are staged by the activation warp.)
+// O-projection. (The down-projection's inputs: down_input_batch / prep_job.)
 template <bool BATCHED>
 __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
                           uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
@@ -365,10 +369,11 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
     return true;
 }
 
-// A down-projection chunk's inputs at batch > 1, by all compute warps: h chunk c
-// of every sequence and, with the last chunk, the residual rows (x after
-// attention). At batch 1 the activation warp stages them ahead instead (one
-// warp moves one sequence's chunk in time; eight sequences' it does not).
+// A down-projection chunk's inputs, by all compute warps: h chunk c of every
+// sequence and, with the last chunk, the residual rows (x after attention). At
+// batch 1 the activation warp stages chunks c < kDownStaged ahead instead (one
+// warp moves one sequence's early chunk in time; eight sequences' it does not,
+// nor the chunks that complete only as gate/up ends).
 __device__ __forceinline__ bool down_input_batch(const Params& p, const mk_instr& in, int c, float* sv, float* red,
                                               int warp, int lane, uint64_t* cbar, uint32_t& cuses,
                                               uint32_t epoch) {
@@ -467,7 +472,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
     const mk_instr& in = ins[0];
     float* sv = reinterpret_cast<float*>(slot);
     if (lane == 0) trace(p, job, kTrCtrDone);
-    if (!BATCHED && in.op == MK_OP_DOWN) {
+    if (!BATCHED && in.op == MK_OP_DOWN && c < kDownStaged) {
         // down chunk c: h chunk c (gate/up runs chunk-major, so chunks complete one
         // after another while gate/up still streams) and, with the last chunk, the
         // residual rows (x after attention), staged ahead of the compute warps
@@ -475,7 +480,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
             if (!warp_load_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, in.layer, kTagH),
                                   p.F / 4, sv + (size_t)b * p.xs_vec_floats, 8, lane))
                 return false;
-            if (c == 3) {
+            if (kDownStaged > 3 && c == 3) {
                 const int rows = (int)in.count * 4;
                 const uint64_t* xs = p.x_t + (size_t)b * p.H + (size_t)in.first * 4;
                 const uint32_t tag = act_tag(epoch, in.layer, kTagXAttn);
@@ -829,11 +834,12 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             if (warp == 0 && lane == 0) trace(p, j, kTrStart);
             float* sv = reinterpret_cast<float*>(sl.slot(j));
             // inputs: the attention item's q/k/v and every matvec input but the
-            // down-projection's at batch 1 (staged by the activation warp) are
-            // loaded here
+            // early down-projection chunks at batch 1 (staged by the activation
+            // warp) are loaded here
             bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
-                      : in.op == MK_OP_DOWN ? (!BATCHED || down_input_batch(p, in, c, sv, red, warp, lane, cbar,
-                                                                            cuses, epoch))
+                      : in.op == MK_OP_DOWN ? ((!BATCHED && c < kDownStaged) ||
+                                                     down_input_batch(p, in, c, sv, red, warp, lane, cbar, cuses,
+                                                                      epoch))
                                             : job_input<BATCHED>(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7);

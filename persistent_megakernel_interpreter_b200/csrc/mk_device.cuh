@@ -717,47 +717,49 @@ __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uin
 // One attention item is one (sequence b, KV group g, key range [first,
 // first + count)) of the split-K decode attention, restricted to keys <= pos
 // (the key at pos is the one this step writes). The whole item runs on the
-// compute warps of one CTA (256 threads) in three phases with a CTA barrier
-// after each. The item is small (at most a few hundred keys), so its time is
-// latency: each phase works on batches of independent keys without divergent
-// branches (out-of-range keys read a valid row and are masked), so that the
-// keys' dependent chains overlap, and rows are addressed incrementally.
+// compute warps of one CTA (256 threads), in one pass per warp and one merge:
 //
-//  1. scores: 8 lanes per key (8 dims each; the group's query heads held in
-//     registers), four keys per warp pass, four passes per batch. The partial
-//     dot products meet in a reduce-scatter butterfly that leaves head
-//     2*b2 + b1 on the lanes with lane bits (b2, b1), as
-//     s_h(j) = (q_h . k_j) * (1/sqrt(HD)). Each warp reduces its keys' maximum
-//     per head. (head_dim 128: 16 lanes per key, bit 3 folded first.)
-//  2. weights, one thread per key: M_h = max of the warps' maxima,
-//     e_h(j) = exp(s_h(j) - M_h), stored as a float4 per key (heads >= G: 0);
-//     each warp reduces its keys' sum per head.
-//  3. values: thread (kq, dp) adds e_h(j) * v_j[2 dp], v_j[2 dp + 1] for all
-//     heads over the keys j = kq (mod KQ) in increasing j, four per batch.
-// Then each output (h, d) is the KQ class sums added in class order, and l_h
-// the warps' sums added in warp order. With one partition per (sequence, group)
-// the output is o_h / l_h; otherwise (M_h, l_h, o_h) is the partition's
-// partial, merged in partition order. The megakernel and the multi-kernel
-// baseline run this same code on the same rows, so their results are identical.
+//  * The keys are cut into passes of KPW keys (4 at head_dim 64, 2 at 128);
+//    warp w takes passes w, w + 8, w + 16, ... and runs an online softmax over
+//    them, NB passes at a time, for all of the group's query heads at once.
+//  * Scores: LPK lanes per key (8 dims each), the group's query heads held in
+//    registers. The partial dot products meet in a reduce-scatter butterfly
+//    that leaves head 2*b2 + b1 on the lanes with lane bits (b2, b1), as
+//    s_h(j) = (q_h . k_j) * (1/sqrt(HD)) (head_dim 128: bit 3 folded first).
+//  * After each block of NB passes the warp's running maximum m_h becomes
+//    max(m_h, block maximum), the running sums are scaled by e^(m_old - m_new),
+//    the block's weights e_h(j) = exp(s_h(j) - m_h) are published to the warp's
+//    scratch, and every lane adds e_h(j) * v_j over its DPL dims for every head.
+//  * One CTA barrier; then thread (h, d) merges the warps in warp order:
+//    M_h = max_w m_w,h, f_w = e^(m_w,h - M_h), l_h = sum_w f_w l_w,h,
+//    o_h[d] = sum_w f_w o_w,h[d].
+// With one partition per (sequence, group) the output is o_h / l_h; otherwise
+// (M_h, l_h, o_h) is the partition's partial, merged in partition order. Every
+// order of summation depends only on the key indices and the shape, not on
+// where a row sits, so the megakernel (rows in its ring) and the multi-kernel
+// baseline (rows copied to shared memory) give identical results.
 
-// DPL: dims per lane in the partial merge; LPK lanes per key in the scores;
-// KQ key classes in the values.
+// DPL: dims per lane in the values and the partial merge; LPK lanes per key in
+// the scores; KPW keys per warp pass.
 template <int HD>
 struct AttnShape {
     static constexpr int DPL = HD / 32;
     static constexpr int LPK = HD / 8;
-    static constexpr int KPW = 32 / LPK;                         // keys per warp pass
-    static constexpr int KQ = 32 * kConsumerWarps / (HD / 2);
+    static constexpr int KPW = 32 / LPK;
+    static constexpr int NB = 5;                 // passes per online-softmax block (129 keys: one block per warp)
+    static constexpr int BK = NB * KPW;          // keys per block
 };
 
 constexpr int kMaxGroup = kMaxGroupHeads;  // query heads per KV head handled by one item
 
-// Offsets inside an item's scratch (kAttnScratchFloats floats of shared memory).
-constexpr uint32_t kAttnE = 0;                                       // [kMaxItemKeys][4]
-constexpr uint32_t kAttnWMax = kAttnE + 4 * kMaxItemKeys;            // [warps][4]
-constexpr uint32_t kAttnWSum = kAttnWMax + 4 * kConsumerWarps;       // [warps][4]
-constexpr uint32_t kAttnPart = kAttnWSum + 4 * kConsumerWarps;       // [KQ][4][HD]
-constexpr uint32_t kAttnFlagFloat = kAttnPart + 2 * 32 * kConsumerWarps * 4;
+// Offsets inside an item's scratch (kAttnScratchFloats floats of shared memory):
+// per warp a region of kAttnWarpFloats, holding a block's weights [BK][4] while
+// the warp runs, then the warp's value sums [4][HD]; the warps' maxima and sums
+// [warps][4] each; a flag word.
+constexpr uint32_t kAttnWarpFloats = 4 * 128;
+constexpr uint32_t kAttnWM = kConsumerWarps * kAttnWarpFloats;       // [warps][4]
+constexpr uint32_t kAttnWL = kAttnWM + 4 * kConsumerWarps;          // [warps][4]
+constexpr uint32_t kAttnFlagFloat = kAttnWL + 4 * kConsumerWarps;
 static_assert(kAttnFlagFloat + 4 <= kAttnScratchFloats, "attention scratch");
 
 // The rows of an item in shared memory (knew and vnew always point at a valid
@@ -791,60 +793,68 @@ __device__ __forceinline__ const uint16_t* attn_row(const AttnRows<HD>& R, uint3
     return reinterpret_cast<const uint16_t*>(R.base + (size_t)s * R.stage_bytes) + (size_t)r * HD;
 }
 
+// e^(a - b) for a running maximum a that may still be -inf (no key yet): 0.
+__device__ __forceinline__ float exp_rel(float a, float b) { return a == -INFINITY ? 0.f : expf(a - b); }
+
 // The item on all compute warps (warp < kConsumerWarps). qs: the group's G query
 // heads, fp32 [G][HD], in shared memory; sc: kAttnScratchFloats of shared
 // memory; bar(): barrier of the compute warps (false: give up); mark(k): trace
 // hook. R.jnew must be -1 or n - 1. On success emit(h, d, o, M_h, l_h) runs once
 // for every output dim d < HD of every head h < G, on the thread that holds it.
-template <int HD, int PBS = 4, int PBV = 4, class Bar, class Mark, class Emit>
+template <int HD, class Bar, class Mark, class Emit>
 __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const float* qs, int G, float* sc,
                                                 int warp, int lane, Bar&& bar, Mark&& mark, Emit&& emit) {
     using S = AttnShape<HD>;
     constexpr int NT = 32 * kConsumerWarps;
-    constexpr int KQ = S::KQ;
-    // PBS: warp passes per batch of the scores; PBV: keys per batch of the values
-    float4* et = reinterpret_cast<float4*>(sc + kAttnE);
-    float4* wmax = reinterpret_cast<float4*>(sc + kAttnWMax);
-    float4* wsum = reinterpret_cast<float4*>(sc + kAttnWSum);
-    float* part = sc + kAttnPart;
+    constexpr int DPL = S::DPL, KPW = S::KPW, NB = S::NB;
+    static_assert(4 * S::BK <= (int)kAttnWarpFloats && kMaxGroup * HD <= (int)kAttnWarpFloats, "attention scratch");
     const int n = R.n, t = warp * 32 + lane;
     const int nc = R.jnew >= 0 ? n - 1 : n;  // rows read from the fills
     const float scale = 1.0f / sqrtf((float)HD);
-    // 1. scores
-    {
-        const int dc = lane % S::LPK, kk = lane / S::LPK;
-        float q[kMaxGroup][8];
+    float* ew = sc + (size_t)warp * kAttnWarpFloats;  // this warp's region
+    const int dc = lane % S::LPK, kk = lane / S::LPK;
+    const int hh = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);  // head this lane's scores belong to
+    const bool writer = (lane & (S::LPK == 8 ? 1 : 9)) == 0;    // one lane per (key, head)
+    const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
+    const size_t vofs = (size_t)R.kps * HD;
+    float q[kMaxGroup][8];
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h < G) {
-                const float4 a = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8);
-                const float4 c = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8 + 4);
-                q[h][0] = a.x; q[h][1] = a.y; q[h][2] = a.z; q[h][3] = a.w;
-                q[h][4] = c.x; q[h][5] = c.y; q[h][6] = c.z; q[h][7] = c.w;
-            } else {
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h < G) {
+            const float4 a = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8);
+            const float4 c = *reinterpret_cast<const float4*>(qs + h * HD + dc * 8 + 4);
+            q[h][0] = a.x; q[h][1] = a.y; q[h][2] = a.z; q[h][3] = a.w;
+            q[h][4] = c.x; q[h][5] = c.y; q[h][6] = c.z; q[h][7] = c.w;
+        } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) q[h][e] = 0.f;
-            }
+            for (int e = 0; e < 8; ++e) q[h][e] = 0.f;
         }
-        const int hh = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);  // head this lane ends up with
-        const bool writer = (lane & (S::LPK == 8 ? 1 : 9)) == 0;
-        constexpr int KPR = S::KPW * kConsumerWarps;  // keys per pass over all warps
-        const int j_first = warp * S::KPW + kk;
-        const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int j0 = j_first; j0 - kk < n; j0 += PBS * KPR) {
-            float acc[PBS][kMaxGroup];
-            float kv[PBS][8];
+    }
+    // running state: the maximum of head hh (lane's scores), the lane's share of
+    // l_hh, and the value sums o[h][dd] of dims lane * DPL + dd for every head
+    float mrun = -INFINITY, lpart = 0.f;
+    float o[kMaxGroup][DPL];
 #pragma unroll
-            for (int i = 0; i < PBS; ++i) {
-                const int j = j0 + i * KPR;
+    for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+        for (int dd = 0; dd < DPL; ++dd) o[h][dd] = 0.f;
+    const int npass = (n + KPW - 1) / KPW;
+#pragma unroll 1
+    for (int p0 = warp; p0 < npass; p0 += NB * kConsumerWarps) {
+        // scores of NB passes: pass i covers keys (p0 + 8 i) * KPW + kk
+        float s[NB];
+        {
+            float acc[NB][kMaxGroup];
+            float kv[NB][8];
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                const int j = (p0 + i * kConsumerWarps) * KPW + kk;
                 // rows past the fills read the new key (a valid stand-in; masked below)
                 const uint16_t* kr = j < nc ? attn_row<HD>(R, m, j) : R.knew;
                 unpack8(lds_v4(kr + dc * 8), kv[i]);
             }
 #pragma unroll
-            for (int i = 0; i < PBS; ++i)
+            for (int i = 0; i < NB; ++i)
 #pragma unroll
                 for (int h = 0; h < kMaxGroup; ++h) {
                     acc[i][h] = 0.f;
@@ -853,129 +863,110 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
                 }
             if (S::LPK == 16) {
 #pragma unroll
-                for (int i = 0; i < PBS; ++i)
+                for (int i = 0; i < NB; ++i)
 #pragma unroll
                     for (int h = 0; h < kMaxGroup; ++h) acc[i][h] += __shfl_xor_sync(0xffffffffu, acc[i][h], 8);
             }
             const bool b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
-            for (int i = 0; i < PBS; ++i) {
+            for (int i = 0; i < NB; ++i) {
                 const float k0 = b2 ? acc[i][2] : acc[i][0], k1 = b2 ? acc[i][3] : acc[i][1];
                 const float s0 = b2 ? acc[i][0] : acc[i][2], s1 = b2 ? acc[i][1] : acc[i][3];
                 const float m0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 4);
                 const float m1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 4);
                 const float kp = b1 ? m1 : m0, sp = b1 ? m0 : m1;
                 const float v = kp + __shfl_xor_sync(0xffffffffu, sp, 2);
-                acc[i][0] = v + __shfl_xor_sync(0xffffffffu, v, 1);
-            }
-#pragma unroll
-            for (int i = 0; i < PBS; ++i) {
-                const int j = j0 + i * KPR;
-                const float s = __fmul_rn(acc[i][0], scale);
-                if (j < n && hh < G) {
-                    mx = fmaxf(mx, s);
-                    if (writer) sc[kAttnE + 4 * j + hh] = s;
-                }
+                const float tot = v + __shfl_xor_sync(0xffffffffu, v, 1);
+                const int j = (p0 + i * kConsumerWarps) * KPW + kk;
+                s[i] = (j < n && hh < G) ? __fmul_rn(tot, scale) : -INFINITY;
             }
         }
-        // the warp's maximum per head: lanes holding the same head differ in bits 0, 3, 4
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if (lane < 8 && (lane & 1) == 0) sc[kAttnWMax + 4 * warp + hh] = hh < G ? mx : -INFINITY;
+        // the block's maximum per head: lanes holding the same head differ in bits 0, 3, 4
+        float bm = s[0];
+#pragma unroll
+        for (int i = 1; i < NB; ++i) bm = fmaxf(bm, s[i]);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+        const float mnew = fmaxf(mrun, bm);
+        const float f = exp_rel(mrun, mnew);  // rescale of what the warp summed so far
+        mrun = mnew;
+        __syncwarp();  // the previous block's weights have been read
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+            const float e = s[i] == -INFINITY ? 0.f : expf(s[i] - mnew);
+            if (writer) {
+                lpart = (i == 0 ? lpart * f : lpart) + e;
+                ew[(i * KPW + kk) * 4 + hh] = e;
+            }
+        }
+        // heads' rescale factors from the lanes holding them (lane 2h holds head h)
+        float fh[kMaxGroup];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) fh[h] = __shfl_sync(0xffffffffu, f, 2 * h);
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+            for (int dd = 0; dd < DPL; ++dd) o[h][dd] *= fh[h];
+        __syncwarp();
+        // values: every key of the block, in pass order, for the lane's DPL dims
+#pragma unroll
+        for (int i = 0; i < NB; ++i)
+#pragma unroll
+            for (int k2 = 0; k2 < KPW; ++k2) {
+                const int j = (p0 + i * kConsumerWarps) * KPW + k2;
+                const uint16_t* vr = j < nc ? attn_row<HD>(R, m, j) + vofs : R.vnew;  // stand-in, masked
+                float v[DPL];
+                if constexpr (DPL == 2) {
+                    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vr + lane * 2);
+                    v[0] = bf_lo(w2);
+                    v[1] = bf_hi(w2);
+                } else {
+                    const uint2 w4 = *reinterpret_cast<const uint2*>(vr + lane * 4);
+                    v[0] = bf_lo(w4.x);
+                    v[1] = bf_hi(w4.x);
+                    v[2] = bf_lo(w4.y);
+                    v[3] = bf_hi(w4.y);
+                }
+                const float4 e4 = *reinterpret_cast<const float4*>(ew + (i * KPW + k2) * 4);
+                const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+                    for (int dd = 0; dd < DPL; ++dd) o[h][dd] = fmaf(ev[h], v[dd], o[h][dd]);
+            }
     }
+    // the warp's l per head: its writer lanes' shares, added over lane bits 3, 4
+    lpart += __shfl_xor_sync(0xffffffffu, lpart, 8);
+    lpart += __shfl_xor_sync(0xffffffffu, lpart, 16);
+    __syncwarp();  // the last block's weights have been read
+    if (lane < 8 && (lane & 1) == 0) {
+        sc[kAttnWM + 4 * warp + hh] = hh < G ? mrun : -INFINITY;
+        sc[kAttnWL + 4 * warp + hh] = hh < G ? lpart : 0.f;
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+        if (h < G)
+#pragma unroll
+            for (int dd = 0; dd < DPL; ++dd) ew[h * HD + lane * DPL + dd] = o[h][dd];
     mark(0);
     if (!bar()) return false;
     mark(1);
-    // 2. weights
-    float M[kMaxGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-        const float4 v = wmax[w];
-        M[0] = fmaxf(M[0], v.x);
-        M[1] = fmaxf(M[1], v.y);
-        M[2] = fmaxf(M[2], v.z);
-        M[3] = fmaxf(M[3], v.w);
-    }
-    {
-        float ls[kMaxGroup] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int j = t; j < n; j += NT) {
-            const float4 v = et[j];
-            const float s[kMaxGroup] = {v.x, v.y, v.z, v.w};
-            float e[kMaxGroup];
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                e[h] = h < G ? expf(s[h] - M[h]) : 0.f;
-                ls[h] += e[h];
-            }
-            et[j] = make_float4(e[0], e[1], e[2], e[3]);
-        }
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) ls[h] = warp_sum(ls[h]);
-        if (lane == 0) wsum[warp] = make_float4(ls[0], ls[1], ls[2], ls[3]);
-    }
-    mark(2);
-    if (!bar()) return false;
-    mark(3);
-    // 3. values: thread (kq, dp), keys kq, kq + KQ, ... (the key at pos last)
-    {
-        const int dp = t % (HD / 2), kq = t / (HD / 2);
-        float a[kMaxGroup][2];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) a[h][0] = a[h][1] = 0.f;
-        const uint32_t m = 0xffffffffu / (uint32_t)R.kps + 1u;
-        const size_t vofs = (size_t)R.kps * HD;
-#pragma unroll 1
-        for (int j0 = kq; j0 < nc; j0 += PBV * KQ) {
-            uint32_t w[PBV];
-            float4 e[PBV];
-#pragma unroll
-            for (int i = 0; i < PBV; ++i) {
-                const int j = j0 + i * KQ;
-                const bool ok = j < nc;
-                const uint16_t* vr = ok ? attn_row<HD>(R, m, j) + vofs : R.vnew;  // stand-in, masked
-                w[i] = *reinterpret_cast<const uint32_t*>(vr + dp * 2);
-                e[i] = et[ok ? j : 0];
-            }
-#pragma unroll
-            for (int i = 0; i < PBV; ++i) {
-                if (j0 + i * KQ >= nc) e[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                const float v0 = bf_lo(w[i]), v1 = bf_hi(w[i]);
-                a[0][0] = fmaf(e[i].x, v0, a[0][0]); a[0][1] = fmaf(e[i].x, v1, a[0][1]);
-                a[1][0] = fmaf(e[i].y, v0, a[1][0]); a[1][1] = fmaf(e[i].y, v1, a[1][1]);
-                a[2][0] = fmaf(e[i].z, v0, a[2][0]); a[2][1] = fmaf(e[i].z, v1, a[2][1]);
-                a[3][0] = fmaf(e[i].w, v0, a[3][0]); a[3][1] = fmaf(e[i].w, v1, a[3][1]);
-            }
-        }
-        if (R.jnew >= 0 && R.jnew % KQ == kq) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(R.vnew + dp * 2);
-            const float v0 = bf_lo(w), v1 = bf_hi(w);
-            const float4 e = et[R.jnew];
-            a[0][0] = fmaf(e.x, v0, a[0][0]); a[0][1] = fmaf(e.x, v1, a[0][1]);
-            a[1][0] = fmaf(e.y, v0, a[1][0]); a[1][1] = fmaf(e.y, v1, a[1][1]);
-            a[2][0] = fmaf(e.z, v0, a[2][0]); a[2][1] = fmaf(e.z, v1, a[2][1]);
-            a[3][0] = fmaf(e.w, v0, a[3][0]); a[3][1] = fmaf(e.w, v1, a[3][1]);
-        }
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-            *reinterpret_cast<float2*>(part + ((size_t)(kq * kMaxGroup + h) * HD + dp * 2)) =
-                make_float2(a[h][0], a[h][1]);
-    }
-    mark(4);
-    if (!bar()) return false;
-    mark(5);
-    // the class sums in class order, the warps' sums in warp order
+    // merge the warps in warp order
 #pragma unroll 1
     for (int u = t; u < G * HD; u += NT) {
         const int h = u / HD, d = u % HD;
-        float o = part[(size_t)h * HD + d];
+        float M = -INFINITY;
 #pragma unroll
-        for (int kq = 1; kq < KQ; ++kq) o += part[((size_t)(kq * kMaxGroup + h)) * HD + d];
-        float l = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[kAttnWM + 4 * w + h]);
+        float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) l += sc[kAttnWSum + 4 * w + h];
-        emit(h, d, o, M[h], l);
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float fw = exp_rel(sc[kAttnWM + 4 * w + h], M);
+            L = fmaf(fw, sc[kAttnWL + 4 * w + h], L);
+            O = fmaf(fw, sc[(size_t)w * kAttnWarpFloats + h * HD + d], O);
+        }
+        emit(h, d, O, M, L);
     }
     return true;
 }

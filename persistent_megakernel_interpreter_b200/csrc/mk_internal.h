@@ -26,11 +26,10 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
 constexpr int kMaxItemKeys = 512;                    // keys of one attention item at most
-// Shared-memory scratch of one attention item, in floats: per-key weights
-// [kMaxItemKeys][4], per-warp maxima and sums [kConsumerWarps][4] each, the value
-// phase's class sums (two per compute thread and head), a flag word.
-constexpr uint32_t kAttnScratchFloats =
-    4 * kMaxItemKeys + 8 * kConsumerWarps + 2 * 32 * kConsumerWarps * kMaxGroupHeads + 4;
+// Shared-memory scratch of one attention item, in floats: per compute warp a
+// region of 4 * 128 (a block's weights while the warp runs, then its value sums
+// for up to 4 heads of up to 128 dims), the warps' maxima and sums, a flag word.
+constexpr uint32_t kAttnScratchFloats = 4 * 128 * kConsumerWarps + 8 * kConsumerWarps + 4;
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
