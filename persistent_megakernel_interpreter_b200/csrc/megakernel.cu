@@ -64,9 +64,10 @@ __shared__ int g_pos[kMaxBatch];
 
 constexpr int kPairGroups = kConsumerWarps / 2;  // batch > 1: tiles in work at once (two warps each)
 // Batch 1: the activation warp stages the h chunks of down-projection chunks
-// c < kDownStaged ahead (they complete while gate/up still streams); the later
-// chunks, which complete only as gate/up ends, are loaded by all compute warps.
-constexpr int kDownStaged = 2;
+// c < kDownStaged ahead (they complete while gate/up still streams); the last
+// chunk, which completes only as gate/up ends, is loaded by all compute warps
+// (1B step, same box: staging 1 / 2 / 3 chunks ahead 627 / 611 / 594 us).
+constexpr int kDownStaged = 3;
 
 struct Ring {
     uint8_t* base;

@@ -188,6 +188,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         }
     };
     std::vector<uint32_t> signals(nc, 0);
+    std::vector<int> att_sm;  // the SM of each attention item, chosen in layer 0
     const uint32_t kv_key_bytes = 2u * (uint32_t)L.d * 2u;
     const int gu_chunk = L.F / 8;
     for (int l = 0; l < L.L; ++l) {
@@ -208,17 +209,26 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     });
         // attention items, each its own job on the SM with the fewest items of
         // this layer so far, then the least-loaded one: an SM that runs two items
-        // runs them one after the other, on the layer's critical path
+        // runs them one after the other, on the layer's critical path. Later
+        // layers put each item on the SM the first layer chose for it: the
+        // attention code then stays in those SMs' instruction caches, where a
+        // new SM each layer would fetch it from L2 on the critical path.
         std::vector<int> n_att(n_sm, 0);
+        int item = 0;
         for (int b = 0; b < batch; ++b)
             for (int g = 0; g < L.nkv; ++g)
-                for (int j = 0; j < n_parts; ++j) {
+                for (int j = 0; j < n_parts; ++j, ++item) {
                     int best = 0;
-                    for (int s = 1; s < n_sm; ++s)
-                        if (n_att[s] < n_att[best] ||
-                            (n_att[s] == n_att[best] &&
-                             (load[s] < load[best] || (load[s] == load[best] && rank[s] < rank[best]))))
-                            best = s;
+                    if (l > 0) {
+                        best = att_sm[item];
+                    } else {
+                        for (int s = 1; s < n_sm; ++s)
+                            if (n_att[s] < n_att[best] ||
+                                (n_att[s] == n_att[best] &&
+                                 (load[s] < load[best] || (load[s] == load[best] && rank[s] < rank[best]))))
+                                best = s;
+                        att_sm.push_back(best);
+                    }
                     n_att[best]++;
                     mk_instr in = mk_in(MK_OP_ATTN, l);
                     in.batch = (uint16_t)b;
