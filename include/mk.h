@@ -126,8 +126,8 @@ typedef struct mk_schedule_opts {
  * The attention of a (sequence, KV group) is split into at most 32 key partitions,
  * each holding at most what the SM's weight ring holds at once (and 512 keys), so
  * max_ctx has a ceiling that depends on the shape and batch: 16384 keys for the
- * Llama-3.2-1B shape (12288 at batch 4); for head_dim 128 with 24 query and 8 KV
- * heads, 10752 at batch 1, 9216 at batch 2-4 and 6144 at batch 8. A larger max_ctx
+ * Llama-3.2-1B shape; for head_dim 128 with 24 query and 8 KV heads, 12288 at
+ * batch 1-2 and 6144 at batch 3-8. A larger max_ctx
  * (or a part_keys that needs more than 32 partitions) returns MK_ERR_INVALID_ARG. */
 mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts);
 

@@ -308,6 +308,20 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     p.keys_per_stage = I.keys_per_stage;
     p.stage_bytes = (uint32_t)I.stage_bytes;
     p.n_stages = I.n_stages;
+    // Tensor Memory: one slot per weight tile of up to a stage's bytes, in one lane
+    // quarter (32 lanes of stage_bytes / 32 bytes each); as many as 512 columns hold
+    // per quarter, four quarters
+    p.tslot_cols = (uint32_t)I.stage_bytes / 128u;
+    {
+        int per_q = p.tslot_cols ? (int)(mk::kTmemCols / p.tslot_cols) : 0;
+        if (per_q > mk::kMaxTmemSlots / 4) per_q = mk::kMaxTmemSlots / 4;
+        p.n_tslots = 4 * per_q;
+    }
+    if (p.n_tslots < 4 || I.stage_bytes % 128 != 0) {
+        h->msg = "a weight tile does not fit the SM's Tensor Memory";
+        free_schedule(h);
+        return MK_ERR_UNSUPPORTED;
+    }
     {
         const mk::SlotPlan sp = mk::slot_plan(L, batch, (uint32_t)I.stage_bytes);
         p.xs_slots = sp.xs_slots;

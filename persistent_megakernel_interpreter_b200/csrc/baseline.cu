@@ -135,7 +135,7 @@ __host__ __device__ inline int attn_kpad(int part_keys) { return (part_keys + 15
 
 template <int HD>
 __host__ __device__ inline size_t attn_item_smem(int G, int kpad) {
-    return (size_t)align16((uint32_t)(G * HD * 4)) + 2 * (size_t)kpad * HD * 2 + (size_t)kAttnScratchFloats * 4;
+    return (size_t)align16((uint32_t)(G * HD * 4)) + 2 * (size_t)kpad * HD * 2 + (size_t)attn_scratch_floats(HD) * 4;
 }
 
 // One attention item per CTA: the item's rows (keys first .. first + n - 1, the

@@ -73,15 +73,88 @@ struct Ring {
     uint8_t* base;
     uint64_t* full;
     uint64_t* empty;
-    // Fill number the loader last armed on each stage. Compute warps take a
-    // job's tiles in any order and may look for a fill up to several laps
-    // ahead; an mbarrier parity alone only tells phases one lap apart, so a
-    // warp first waits until its stage holds its fill, then waits on the parity.
+    // Fill number the loader last armed on each stage. The mover warps and (for
+    // an attention item's cached KV) the compute warps may look for a fill several
+    // laps ahead; an mbarrier parity alone only tells phases one lap
+    // apart, so a warp first waits until its stage holds its fill, then waits on
+    // the parity.
     volatile uint32_t* armed;
     uint32_t stage_bytes;
     uint32_t S;
     __device__ __forceinline__ uint8_t* stage(uint32_t seq) const {
         return base + (size_t)(seq % S) * stage_bytes;
+    }
+};
+
+// ------------------------------------------------------------------ Tensor Memory
+//
+// The SM's 256 KB of Tensor Memory hold weight tiles that have landed in the
+// ring, so the ring's stages are free again for the next fills as soon as a
+// tile is moved: the SM then keeps stages + Tensor Memory slots worth of weights
+// on chip while its compute warps wait on the step's dependency chain. A warp
+// may only address the 32 lanes of its quarter (its warp index mod 4); slot k
+// lies in quarter k mod 4, columns (k / 4) * cols .. +cols, and holds the tile of
+// fill seq with seq mod n = k. The mover warp of that quarter stores it, the
+// compute warp seq mod 8 (two at batch > 1, seq mod 4 and seq mod 4 + 4) reads it.
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Lane i of the warp stores r[0..15] into lane (quarter base + i), columns
+// ta .. ta + 15.
+__device__ __forceinline__ void tmem_st16(uint32_t ta, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16};" ::"r"(ta),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// The reverse of tmem_st16. The registers are valid only after tmem_wait_ld,
+// which names them as operands so the compiler reads none of them earlier.
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(ta));
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+struct Tmem {
+    uint32_t base;              // address of the allocation (lane 0, its first column)
+    uint64_t* full;             // [n] the mover arrives when a slot holds its fill
+    uint64_t* empty;            // [n] the compute warp(s) arrive when done with it
+    volatile uint32_t* armed;   // [n] the fill a slot holds (or last held)
+    uint32_t n;                 // slots (a multiple of 4)
+    uint32_t cols;              // columns of one slot
+    // the slot of fill seq, addressed by `warp` (which must be in the slot's quarter)
+    __device__ __forceinline__ uint32_t addr(uint32_t seq, int warp) const {
+        const uint32_t k = seq % n;
+        return base + ((32u * (uint32_t)(warp & 3)) << 16) + (k / 4u) * cols;
     }
 };
 
@@ -172,6 +245,22 @@ __device__ __forceinline__ bool wait_fill(const Params& p, const Ring& r, uint32
 __device__ __forceinline__ void release_fill(const Ring& r, uint32_t seq, int lane) {
     __syncwarp();
     if (lane == 0) mbar_arrive(r.empty + seq % r.S);
+}
+
+// A compute warp waits until the Tensor Memory slot of fill seq holds it (the
+// slot's fill number first: a warp may look several laps ahead of the mover).
+__device__ __forceinline__ bool wait_tile(const Params& p, const Tmem& tm, uint32_t seq, int lane) {
+    const uint32_t k = seq % tm.n;
+    if (!wait_bar(p, tm.full + k, (seq / tm.n) & 1u, tm.armed + k, seq, 6, lane)) return false;
+    tmem_fence_after();
+    return true;
+}
+
+// After the warp's reads of the slot have completed (tmem_wait_ld).
+__device__ __forceinline__ void release_tile(const Tmem& tm, uint32_t seq, int lane) {
+    tmem_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tm.empty + seq % tm.n);
 }
 
 // Barrier of the 8 compute warps (an mbarrier of count 8; bounded, abort-aware,
@@ -544,21 +633,48 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 
 // ------------------------------------------------------------------ compute warps
 
-// One 4-row tile against an input vector in shared memory: a single copy of the
-// code per input width, shared by every op (the kernel's instruction footprint
-// is what each SM re-fetches for every layer).
+// One 4-row tile, read from the warp's Tensor Memory slot at `ta`, against an
+// input vector in shared memory: the same lane mapping and order of arithmetic as
+// dot4 (lane ln holds the 16-byte pieces (row r, kc*32 + ln); the mover stored
+// row r's piece kc at columns kc*16 + 4r .. +3), so the totals equal dot4's bit
+// for bit. A single copy of the code per input width, shared by every op (the
+// kernel's instruction footprint is what each SM re-fetches for every layer).
 template <int KC>
-__device__ __noinline__ float4 tile_dot(const uint8_t* tile, const float* v, int lane) {
-    XSmem<KC> x{reinterpret_cast<float4*>(const_cast<float*>(v)),
-                reinterpret_cast<float4*>(const_cast<float*>(v)) + KC * 32};
-    float acc[4];
-    dot4<KC, true>(tile, x, acc, lane, 0);
+__device__ __noinline__ float4 tile_dot(uint32_t ta, const float* v, int lane) {
+    static_assert(KC % 2 == 0, "pieces are read in pairs");
+    const XSmem<KC> x{reinterpret_cast<float4*>(const_cast<float*>(v)),
+                      reinterpret_cast<float4*>(const_cast<float*>(v)) + KC * 32};
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    auto use = [&](const uint32_t (&r)[16], int kc) {
+        float e[8];
+        x.get(kc, lane, e);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+            fma8(acc[rr], make_uint4(r[4 * rr], r[4 * rr + 1], r[4 * rr + 2], r[4 * rr + 3]), e);
+    };
+    // the next piece's load is in flight while the current one is used
+    uint32_t a[16], b[16];
+    tmem_ld16(ta, a);
+    tmem_wait_ld(a);
+#pragma unroll 1
+    for (int kc = 0; kc < KC; kc += 2) {
+        tmem_ld16(ta + (uint32_t)(kc + 1) * 16u, b);
+        use(a, kc);
+        tmem_wait_ld(b);
+        if (kc + 2 < KC) tmem_ld16(ta + (uint32_t)(kc + 2) * 16u, a);
+        use(b, kc + 1);
+        if (kc + 2 < KC) tmem_wait_ld(a);
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) acc[rr] = warp_sum(acc[rr]);
     return make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
-// Batch 1 (batch > 1 runs compute_tiles_pair).
+// Batch 1 (batch > 1 runs compute_tiles_pair). Tile t of the job is the SM's fill
+// seq = in.seq + t; compute warp seq mod 8 takes it (its Tensor Memory quarter,
+// seq mod 4, is the one the mover stored it in).
 template <int KC, int HD>
-__device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr& in,
+__device__ bool compute_tiles(const Params& p, const Tmem& tm, const mk_instr& in,
                               const float* sv, int warp, int lane, uint32_t job, uint32_t epoch) {
     // a dropped instruction (the failure-detection hook) computes but publishes nothing
     const bool pub = in.signal_ctr != MK_NO_COUNTER;
@@ -566,21 +682,21 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
     auto stamp = [&](int w) {
         if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w);
     };
-    for (uint32_t t = warp; t < in.count; t += kConsumerWarps) {
+    for (uint32_t t = (uint32_t)(warp - (int)in.seq) & 7u; t < in.count; t += kConsumerWarps) {
         const uint32_t seq = in.seq + t;
         if (k < 2) stamp(3 * k);
-        if (!wait_fill(p, ring, seq, lane)) return false;
+        if (!wait_tile(p, tm, seq, lane)) return false;
         if (t == 0 && lane == 0) trace(p, job, kTrFill);
         if (k < 2) stamp(3 * k + 1);
-        const uint8_t* tile = ring.stage(seq);
         {
             constexpr int b = 0;  // batch 1: every lane holds the 4 totals
             const int el = lane;
             float acc[4];
             {
-                const float4 a4 = tile_dot<KC>(tile, sv, lane);
+                const float4 a4 = tile_dot<KC>(tm.addr(seq, warp), sv, lane);
                 acc[0] = a4.x; acc[1] = a4.y; acc[2] = a4.z; acc[3] = a4.w;
             }
+            release_tile(tm, seq, lane);
             if (k < 2) stamp(3 * k + 2);
             const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
             switch (in.op) {
@@ -604,23 +720,47 @@ __device__ bool compute_tiles(const Params& p, const Ring& ring, const mk_instr&
                 default: logits_epilogue(p, b, tl, acc, el); break;
             }
         }
-        release_fill(ring, seq, lane);
         if (k == 1) stamp(6);
         ++k;
     }
     return true;
 }
 
-// Batch > 1: two compute warps share each tile by sequences -- warp w takes tiles
-// t = w (mod 4), sequences [b0, b0 + nb) with b0 = (w / 4) * ceil(B / 2) -- so a
-// stage is held for half the batched arithmetic and all eight warps have a tile
-// while only four stages fit beside the sequences' inputs. Each (sequence, row)
-// total is dot4's for that sequence, bit for bit (dot4_batch4); both warps release
-// the stage (its empty barrier counts two arrivals).
+// Batch > 1: two compute warps share each tile by sequences -- the warps w with
+// w mod 4 = seq mod 4 (the tile's Tensor Memory quarter), sequences [b0, b0 + nb)
+// with b0 = (w / 4) * ceil(B / 2) -- so a tile is held for half the batched
+// arithmetic. Each (sequence, row) total is dot4's for that sequence, bit for bit
+// (the arithmetic of dot4_batch4 on the pieces read from Tensor Memory); both
+// warps release the slot (its empty barrier counts two arrivals).
 template <int KC>
-__device__ __noinline__ float tile_dot_batch4(const uint8_t* tile, const float* xs, uint32_t vec_floats, int nb,
+__device__ __noinline__ float tile_dot_batch4(uint32_t ta, const float* xs, uint32_t vec_floats, int B4,
                                               int lane) {
-    return dot4_batch4<KC>(tile, xs, vec_floats, nb, lane);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+#pragma unroll 1
+    for (int kc = 0; kc < KC; ++kc) {
+        uint32_t r[16];
+        tmem_ld16(ta + (uint32_t)kc * 16u, r);
+        tmem_wait_ld(r);
+        float w[4][8];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+            unpack8(make_uint4(r[4 * rr], r[4 * rr + 1], r[4 * rr + 2], r[4 * rr + 3]), w[rr]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (b < B4) {
+                const float4* x = reinterpret_cast<const float4*>(xs + (size_t)b * vec_floats);
+                const float4 lo = x[kc * 32 + lane], hi = x[KC * 32 + kc * 32 + lane];
+                const float e[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[b * 4 + rr] = fmaf(w[rr][i], e[i], v[b * 4 + rr]);
+            }
+        }
+    }
+    return reduce_batch4(v, lane);
 }
 
 struct PairSeqs {
@@ -633,7 +773,7 @@ struct PairSeqs {
 };
 
 template <int KC, int HD>
-__device__ bool compute_tiles_pair(const Params& p, const Ring& ring, const mk_instr& in, const float* sv, int warp,
+__device__ bool compute_tiles_pair(const Params& p, const Tmem& tm, const mk_instr& in, const float* sv, int warp,
                                    int lane, uint32_t job, uint32_t epoch) {
     const bool pub = in.signal_ctr != MK_NO_COUNTER;
     const PairSeqs ps(p.B, warp);
@@ -641,12 +781,13 @@ __device__ bool compute_tiles_pair(const Params& p, const Ring& ring, const mk_i
     const bool act = sl < ps.nb && (lane & 1) == 0;   // lanes l and l ^ 1 hold the same total
     const int b = ps.b0 + (sl < ps.nb ? sl : 0);
     const int el = act ? ((lane >> 1) & 3) : 32;      // acts as lane `el` of a 4-row epilogue
-    for (uint32_t t = warp % kPairGroups; t < in.count; t += kPairGroups) {
+    for (uint32_t t = (uint32_t)(warp - (int)in.seq) & 3u; t < in.count; t += kPairGroups) {
         const uint32_t seq = in.seq + t;
-        if (!wait_fill(p, ring, seq, lane)) return false;
-        if (t == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill);
-        const float tb = tile_dot_batch4<KC>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
+        if (!wait_tile(p, tm, seq, lane)) return false;
+        if (t == 0 && lane == 0 && warp < kPairGroups) trace(p, job, kTrFill);
+        const float tb = tile_dot_batch4<KC>(tm.addr(seq, warp), sv + (size_t)ps.b0 * p.xs_vec_floats,
                                              p.xs_vec_floats, ps.nb, lane);
+        release_tile(tm, seq, lane);
         float acc[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[r] = __shfl_sync(0xffffffffu, tb, (lane & ~7) + 2 * r);
@@ -670,25 +811,29 @@ __device__ bool compute_tiles_pair(const Params& p, const Ring& ring, const mk_i
                 break;
             default: logits_epilogue(p, b, tl, acc, el); break;
         }
-        release_fill(ring, seq, lane);
     }
     return true;
 }
 
+// Every chunk job at batch > 1 starts with the compute warps' input barrier
+// (down_input_batch), so a running sum that another warp added to in the previous
+// chunk is complete before this chunk adds to it.
 template <int KF>
-__device__ bool compute_down_pair(const Params& p, const Ring& ring, const mk_instr& in, int c, const float* sv,
+__device__ bool compute_down_pair(const Params& p, const Tmem& tm, const mk_instr& in, int c, const float* sv,
                                   float* tot, int warp, int lane, uint32_t job, uint32_t epoch) {
     const PairSeqs ps(p.B, warp);
     const int sl = lane >> 3;
     const bool act = sl < ps.nb && (lane & 1) == 0;
     const int b = ps.b0 + (sl < ps.nb ? sl : 0);
     const int row = (lane >> 1) & 3;
-    for (uint32_t r = warp % kPairGroups; r < in.count; r += kPairGroups) {
-        const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
-        if (!wait_fill(p, ring, seq, lane)) return false;
-        if (r == 0 && lane == 0 && warp == 0) trace(p, job, kTrFill);
-        const float y = tile_dot_batch4<KF>(ring.stage(seq), sv + (size_t)ps.b0 * p.xs_vec_floats,
+    const uint32_t base = in.seq + (uint32_t)c * in.count;
+    for (uint32_t r = (uint32_t)(warp - (int)base) & 3u; r < in.count; r += kPairGroups) {
+        const uint32_t seq = base + r;
+        if (!wait_tile(p, tm, seq, lane)) return false;
+        if (r == 0 && lane == 0 && warp < kPairGroups) trace(p, job, kTrFill);
+        const float y = tile_dot_batch4<KF>(tm.addr(seq, warp), sv + (size_t)ps.b0 * p.xs_vec_floats,
                                             p.xs_vec_floats, ps.nb, lane);
+        release_tile(tm, seq, lane);
         if (act) {
             float* t = tot + ((size_t)r * p.B + b) * 4 + row;
             *t = (c == 0) ? y : *t + y;
@@ -698,41 +843,42 @@ __device__ bool compute_down_pair(const Params& p, const Ring& ring, const mk_in
                           act_tag(epoch, in.layer, kTagXMlp));
             }
         }
-        release_fill(ring, seq, lane);
     }
     return true;
 }
 
 // Down-projection at batch 1 (batch > 1 runs compute_down_pair), chunk c: row
-// block r (warp r mod 8) adds W_d[:, chunk c] . h_c to its running sums, chunks in
-// order 0..3; after chunk 3 the residual.
+// block r's tile of chunk c is fill seq = in.seq + c * count + r, taken by compute
+// warp seq mod 8 -- a different warp in each chunk -- so chunks 0..2 store their
+// totals y_c apart, and chunk 3, whose inputs the compute warps load behind a
+// barrier of all of them (kDownStaged <= 3), adds ((y_0 + y_1) + y_2) + y_3 and the
+// residual.
+static_assert(kDownStaged <= 3, "chunk 3 must start with the compute warps' input barrier");
 template <int KF>
-__device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& in, int c,
+__device__ bool compute_down(const Params& p, const Tmem& tm, const mk_instr& in, int c,
                              const float* sv, float* tot, int warp, int lane, uint32_t job, uint32_t epoch) {
-    for (uint32_t r = warp; r < in.count; r += kConsumerWarps) {
-        const uint32_t seq = in.seq + (uint32_t)c * in.count + r;
-        if (!wait_fill(p, ring, seq, lane)) return false;
+    const uint32_t base = in.seq + (uint32_t)c * in.count;
+    for (uint32_t r = (uint32_t)(warp - (int)base) & 7u; r < in.count; r += kConsumerWarps) {
+        const uint32_t seq = base + r;
+        if (!wait_tile(p, tm, seq, lane)) return false;
         if (r == 0 && lane == 0) trace(p, job, kTrFill);
+        float y;
         {
-            constexpr int b = 0;  // batch 1
-            const int row = lane;
-            float y = 0.f;
-            {
-                const float4 a4 = tile_dot<KF>(ring.stage(seq), sv, lane);
-                const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
-                if (lane < 4) y = pick4(acc, lane);
-            }
-            if (row < 4) {
-                float* t = tot + ((size_t)r * p.B + b) * 4 + row;
-                *t = (c == 0) ? y : *t + y;
-                if (c == 3 && in.signal_ctr != MK_NO_COUNTER) {  // x = x_in + W_d h; x_in waits in the slot
-                    const float xin = slot_resid(p, const_cast<float*>(sv), b)[r * 4 + row];
-                    st_tagged(p.x_t + (size_t)b * p.H + (in.first + r) * 4 + row, __fadd_rn(xin, *t),
-                              act_tag(epoch, in.layer, kTagXMlp));
-                }
+            const float4 a4 = tile_dot<KF>(tm.addr(seq, warp), sv, lane);
+            const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
+            y = pick4(acc, lane & 3);
+        }
+        release_tile(tm, seq, lane);
+        if (lane < 4) {
+            float* yc = tot + r * 4 + lane;  // y_c at yc[c * kMaxDownRows * 4]
+            if (c < 3) {
+                yc[c * kMaxDownRows * 4] = y;
+            } else if (in.signal_ctr != MK_NO_COUNTER) {  // x = x_in + W_d h; x_in waits in the slot
+                const float sum = ((yc[0] + yc[kMaxDownRows * 4]) + yc[2 * kMaxDownRows * 4]) + y;
+                const float xin = slot_resid(p, const_cast<float*>(sv), 0)[r * 4 + lane];
+                st_tagged(p.x_t + (in.first + r) * 4 + lane, __fadd_rn(xin, sum), act_tag(epoch, in.layer, kTagXMlp));
             }
         }
-        release_fill(ring, seq, lane);
     }
     return true;
 }
@@ -745,10 +891,11 @@ __device__ bool compute_down(const Params& p, const Ring& ring, const mk_instr& 
 // in partition order. Either way the group's heads are signalled on the
 // attention counter once their output is written.
 template <int HD, bool BATCHED>
-__device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr& a, const uint8_t* slot,
-                                 float* sc, int warp, int lane, uint64_t* cbar, uint32_t& cuses,
-                                 uint32_t job, uint32_t epoch) {
+__device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_instr& a, uint8_t* slot, int warp,
+                                 int lane, uint64_t* cbar, uint32_t& cuses, uint32_t job, uint32_t epoch) {
     const int G = p.group, b = a.batch, g = a.group;
+    // the item's scratch follows its q and new key/value in the job's slot
+    float* sc = reinterpret_cast<float*>(slot + attn_item_bytes(G, HD));
     const int pos = g_pos[b];
     for (uint32_t f = 0; f < a.nfill; ++f)
         if (!wait_fill(p, ring, a.seq + f, lane)) return false;
@@ -789,16 +936,14 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     }
     // every warp has passed the barrier after its last read of the fills
     if (warp == kConsumerWarps - 1 && lane == 0)
-        for (uint32_t f = 0; f < a.nfill; ++f)
-            for (int k = 0; k < (BATCHED ? 2 : 1); ++k)  // batch > 1: each stage counts two arrivals
-                mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+        for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
     if (!bar()) return false;  // every output of the item is stored
     if (p.n_parts == 1) {
         if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_relaxed_add(sig, (uint32_t)G);
         mark(6);
         return true;
     }
-    uint32_t* flag = reinterpret_cast<uint32_t*>(sc + kAttnFlagFloat);
+    uint32_t* flag = reinterpret_cast<uint32_t*>(sc + AttnScratch<HD>::kFlag);
     if (t == 0) {
         uint32_t last = 0;
         if (a.signal_ctr != MK_NO_COUNTER) {  // a dropped item (failure injection) never arrives
@@ -822,7 +967,7 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
 }
 
 template <int KH, int KO, int KF, int HD, bool BATCHED>
-__device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl, float* scores,
+__device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, const Slots& sl,
                              float* tot, float* red, uint64_t* cbar, int i0, int i1, int warp, int lane,
                              uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
@@ -847,19 +992,19 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
             // one call site per routine: the kernel's code is what every SM re-fetches
             // from L2 as it moves between ops, so nothing is inlined twice
             if (in.op == MK_OP_ATTN) {
-                ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), scores, warp, lane, cbar, cuses, j,
+                ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), warp, lane, cbar, cuses, j,
                                                    epoch);
             } else if (in.op == MK_OP_DOWN) {
-                if constexpr (BATCHED) ok = compute_down_pair<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
-                else ok = compute_down<KF>(p, ring, in, c, sv, tot, warp, lane, j, epoch);
+                if constexpr (BATCHED) ok = compute_down_pair<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
+                else ok = compute_down<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
             } else if (KO != KH && in.op == MK_OP_OPROJ) {
                 if constexpr (KO != KH) {
-                    if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                    else ok = compute_tiles<KO, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                    if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, tm, in, sv, warp, lane, j, epoch);
+                    else ok = compute_tiles<KO, HD>(p, tm, in, sv, warp, lane, j, epoch);
                 }
             } else {  // QKV, gate/up, the LM head (and the O-projection when its width is the hidden size)
-                if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
-                else ok = compute_tiles<KH, HD>(p, ring, in, sv, warp, lane, j, epoch);
+                if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, tm, in, sv, warp, lane, j, epoch);
+                else ok = compute_tiles<KH, HD>(p, tm, in, sv, warp, lane, j, epoch);
             }
             if (!ok) return;
             // job done for this warp; the last of the 8 counts the job's completion
@@ -889,7 +1034,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Slots& sl,
     }
 }
 
-// ------------------------------------------------------------------ the loader warp
+// ------------------------------------------------------------------ the loader and the mover warps
 
 // Global source of ring fill t of instruction `in`: one range (weights), or two
 // ranges of `bytes` each for attention (the cached keys and values < pos).
@@ -927,8 +1072,24 @@ __device__ __forceinline__ FillSrc fill_source(const Params& p, const mk_instr& 
     }
 }
 
-// One thread streams the SM's fills into the ring, in list order; it never
-// waits on a dependency counter, only for the compute warps to release a stage.
+// Position of fill `seq` in the SM's list: the instruction holding it (an SM's
+// fills are numbered consecutively, instruction by instruction).
+struct FillCur {
+    int i;
+    uint32_t seq;
+};
+
+__device__ __forceinline__ void fill_seek(const Params& p, FillCur& c, int i1) {
+    while (c.i < i1 && c.seq >= p.instrs[c.i].seq + p.instrs[c.i].nfill) ++c.i;
+}
+
+// One thread (the loader warp's lane 0) streams the SM's fills into the ring, in
+// list order: weight tiles and the cached KV of attention items, all final at
+// launch. It never waits on a dependency counter, only for a stage to be free
+// again: moved to Tensor Memory by a mover warp (weights), or read by its
+// attention item (KV). So the next instructions' weights arrive while the step
+// still waits for their activations. It issues nothing else, so a freed stage is
+// refilled at once.
 __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
@@ -990,6 +1151,63 @@ drain:
     }
 }
 
+// Mover warp q (its lanes converged throughout; its warp index mod 4 is q, the
+// Tensor Memory lane quarter it may address) takes the SM's fills seq = q (mod 4)
+// in list order. A landed weight tile goes into Tensor Memory slot seq mod n once
+// the compute warp has released that slot's previous tile; its ring stage is then
+// free for the loader. A cached-KV fill stays in the ring for its attention item
+// (which frees the stage); its slot is passed over (marked and released at once).
+// The waits block, bounded: the slot's previous tile is an earlier fill and every
+// earlier fill has been issued, so the compute warps can reach it; the fill itself
+// is issued in order by the loader.
+template <bool BATCHED>
+__device__ void mover(const Params& p, const Ring& ring, const Tmem& tm, int i0, int i1, int q, int lane) {
+    const uint32_t S = ring.S;
+    FillCur mov{i0, (uint32_t)q};
+    fill_seek(p, mov, i1);
+    while (mov.i < i1) {
+        const mk_instr& in = p.instrs[mov.i];
+        const uint32_t seq = mov.seq, s = seq % S, k = seq % tm.n;
+        const bool kv = in.op == MK_OP_ATTN;
+        if (seq >= tm.n && !wait_bar(p, tm.empty + k, (seq / tm.n - 1u) & 1u, nullptr, seq, 8, lane)) return;
+        if (!kv) {
+            if (!wait_bar(p, ring.full + s, (seq / S) & 1u, ring.armed + s, seq, 9, lane)) return;
+            tmem_fence_after();
+            const uint32_t bytes = in.op == MK_OP_OPROJ ? p.tile_o : in.op == MK_OP_DOWN ? p.tile_f : p.tile_h;
+            const int KC = (int)(bytes / 2048u);  // even for every supported width
+            const uint4* src = reinterpret_cast<const uint4*>(ring.stage(seq)) + lane;
+            const uint32_t ta = tm.addr(seq, q);
+#pragma unroll 1
+            for (int kc = 0; kc < KC; kc += 2) {
+                uint32_t r0[16], r1[16];
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const uint4 v0 = lds_v4(src + (rr * KC + kc) * 32);
+                    const uint4 v1 = lds_v4(src + (rr * KC + kc + 1) * 32);
+                    r0[4 * rr] = v0.x; r0[4 * rr + 1] = v0.y; r0[4 * rr + 2] = v0.z; r0[4 * rr + 3] = v0.w;
+                    r1[4 * rr] = v1.x; r1[4 * rr + 1] = v1.y; r1[4 * rr + 2] = v1.z; r1[4 * rr + 3] = v1.w;
+                }
+                tmem_st16(ta + (uint32_t)kc * 16u, r0);
+                tmem_st16(ta + (uint32_t)(kc + 1) * 16u, r1);
+            }
+            tmem_wait_st();
+            tmem_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) {
+            tm.armed[k] = seq;  // published by the release of the arrive below
+            mbar_arrive(tm.full + k);
+            if (kv) {
+                for (int j = 0; j < (BATCHED ? 2 : 1); ++j) mbar_arrive(tm.empty + k);
+            } else {
+                mbar_arrive(ring.empty + s);  // the stage is free for the next fill
+            }
+        }
+        mov.seq += kMoveWarps;
+        fill_seek(p, mov, i1);
+    }
+}
+
 // ------------------------------------------------------------------ the kernel
 
 template <int KH, int KO, int KF, int HD, bool BATCHED>
@@ -1012,12 +1230,31 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     sl.done = reinterpret_cast<uint32_t*>(smem + m.xs_done);
     sl.bytes = p.xs_slot_bytes;
     sl.NS = (uint32_t)p.xs_slots;
+    Tmem tm;
+    tm.full = reinterpret_cast<uint64_t*>(smem + m.tfull);
+    tm.empty = reinterpret_cast<uint64_t*>(smem + m.tempty);
+    tm.armed = reinterpret_cast<volatile uint32_t*>(smem + m.tarmed);
+    tm.n = (uint32_t)p.n_tslots;
+    tm.cols = p.tslot_cols;
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(smem + m.tbase);
 
+    // All of the SM's Tensor Memory for this CTA (one CTA per SM; the previous
+    // step's CTA released it before exiting). Warp 0, converged.
+    if (warp == 0) {
+        tmem_alloc(tbase, kTmemCols);
+        tmem_relinquish();
+        tmem_fence_before();
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
             mbar_init(ring.full + s, 1);
-            mbar_init(ring.empty + s, BATCHED ? 2 : 1);  // batch > 1: two warps share each tile
+            mbar_init(ring.empty + s, 1);  // released by a mover (weights) or the attention item (KV)
             ring.armed[s] = 0xffffffffu;
+        }
+        for (int k = 0; k < p.n_tslots; ++k) {
+            mbar_init(tm.full + k, 1);
+            mbar_init(tm.empty + k, BATCHED ? 2 : 1);  // batch > 1: two warps share each tile
+            tm.armed[k] = 0xffffffffu;
         }
         for (int s = 0; s < p.xs_slots; ++s) {
             mbar_init(sl.full + s, 1);
@@ -1045,22 +1282,31 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         s_skip = skip;
     }
     __syncthreads();
+    tmem_fence_after();
+    tm.base = *reinterpret_cast<volatile uint32_t*>(tbase);
 
     if (!s_skip) {
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
-        if (warp == kLoaderWarp) {
+        if (warp >= kConsumerWarps && warp < kConsumerWarps + kMoveWarps) {
+            mover<BATCHED>(p, ring, tm, i0, i1, warp & 3, lane);
+        } else if (warp == kLoaderWarp) {
             if (lane == 0) loader(p, ring, i0, i1);
         } else if (warp == kPrepWarp) {
             activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch);
         } else {
-            float* scores = reinterpret_cast<float*>(smem + m.scores);
-            compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, sl, scores, reinterpret_cast<float*>(smem + m.tot),
+            compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, tm, sl, reinterpret_cast<float*>(smem + m.tot),
                                          reinterpret_cast<float*>(smem + m.red),
                                          reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
                                          s_epoch);
         }
     }
+    // every warp's Tensor Memory reads and writes have completed (waited for)
+    tmem_fence_before();
     __syncthreads();
+    if (warp == 0) {
+        tmem_fence_after();
+        tmem_dealloc(tm.base, kTmemCols);
+    }
 
     // The last CTA to finish closes the step: it advances the epoch, or, after a
     // failed step, clears the counters and every tagged word (so no stale tag can

@@ -549,36 +549,13 @@ __device__ __forceinline__ float dot4_batch(const uint8_t* tile, const float* xs
     return v[0];
 }
 
-// The same for at most 4 of the sequences (B4 <= 4, sequence b at xs + b *
-// vec_floats), so that two warps can share a tile by sequences: 16 partial sums
-// per lane, reduce-scattered with warp_sum's masks 16, 8, 4, 2 and summed across
-// the last pair with mask 1, so each total again equals dot4's for its sequence
-// bit for bit. Lanes l and l ^ 1 hold the total of sequence l / 8, row (l / 2) % 4.
-template <int KC>
-__device__ __forceinline__ float dot4_batch4(const uint8_t* tile, const float* xs, uint32_t vec_floats, int B4,
-                                             int lane) {
-    const uint4* t = reinterpret_cast<const uint4*>(tile) + lane;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-#pragma unroll 1
-    for (int kc = 0; kc < KC; ++kc) {
-        float w[4][8];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) unpack8(lds_v4(t + r * KC * 32 + kc * 32), w[r]);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            if (b < B4) {
-                const float4* x = reinterpret_cast<const float4*>(xs + (size_t)b * vec_floats);
-                const float4 lo = x[kc * 32 + lane], hi = x[KC * 32 + kc * 32 + lane];
-                const float e[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) v[b * 4 + r] = fmaf(w[r][i], e[i], v[b * 4 + r]);
-            }
-        }
-    }
+// The batched tile's reduction for at most 4 sequences: each lane holds 16
+// partial sums v[b * 4 + r] (sequence b, row r) of its own input pieces, in dot4's
+// lane order. They are reduce-scattered with warp_sum's masks 16, 8, 4, 2 and
+// summed across the last pair with mask 1, so each total equals dot4's for its
+// sequence bit for bit; lanes l and l ^ 1 hold the total of sequence l / 8, row
+// (l / 2) % 4.
+__device__ __forceinline__ float reduce_batch4(float (&v)[16], int lane) {
 #pragma unroll
     for (int m = 16, n = 8; m > 1; m >>= 1, n >>= 1) {
         const bool up = (lane & m) != 0;
@@ -752,15 +729,18 @@ struct AttnShape {
 
 constexpr int kMaxGroup = kMaxGroupHeads;  // query heads per KV head handled by one item
 
-// Offsets inside an item's scratch (kAttnScratchFloats floats of shared memory):
-// per warp a region of kAttnWarpFloats, holding a block's weights [BK][4] while
-// the warp runs, then the warp's value sums [4][HD]; the warps' maxima and sums
-// [warps][4] each; a flag word.
-constexpr uint32_t kAttnWarpFloats = 4 * 128;
-constexpr uint32_t kAttnWM = kConsumerWarps * kAttnWarpFloats;       // [warps][4]
-constexpr uint32_t kAttnWL = kAttnWM + 4 * kConsumerWarps;          // [warps][4]
-constexpr uint32_t kAttnFlagFloat = kAttnWL + 4 * kConsumerWarps;
-static_assert(kAttnFlagFloat + 4 <= kAttnScratchFloats, "attention scratch");
+// Offsets inside an item's scratch (attn_scratch_floats(HD) floats of shared
+// memory): per warp a region of 4 * HD floats, holding a block's weights [BK][4]
+// while the warp runs, then the warp's value sums [4][HD]; the warps' maxima and
+// sums [warps][4] each; a flag word.
+template <int HD>
+struct AttnScratch {
+    static constexpr uint32_t kWarp = 4 * HD;
+    static constexpr uint32_t kWM = kConsumerWarps * kWarp;       // [warps][4]
+    static constexpr uint32_t kWL = kWM + 4 * kConsumerWarps;    // [warps][4]
+    static constexpr uint32_t kFlag = kWL + 4 * kConsumerWarps;
+    static_assert(kFlag + 4 == attn_scratch_floats(HD), "attention scratch");
+};
 
 // The rows of an item in shared memory (knew and vnew always point at a valid
 // row: they also stand in for rows past the item, whose results are masked). Row j (0 <= j < n) is key first + j. The
@@ -797,7 +777,7 @@ __device__ __forceinline__ const uint16_t* attn_row(const AttnRows<HD>& R, uint3
 __device__ __forceinline__ float exp_rel(float a, float b) { return a == -INFINITY ? 0.f : expf(a - b); }
 
 // The item on all compute warps (warp < kConsumerWarps). qs: the group's G query
-// heads, fp32 [G][HD], in shared memory; sc: kAttnScratchFloats of shared
+// heads, fp32 [G][HD], in shared memory; sc: attn_scratch_floats(HD) of shared
 // memory; bar(): barrier of the compute warps (false: give up); mark(k): trace
 // hook. R.jnew must be -1 or n - 1. On success emit(h, d, o, M_h, l_h) runs once
 // for every output dim d < HD of every head h < G, on the thread that holds it.
@@ -807,11 +787,12 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
     using S = AttnShape<HD>;
     constexpr int NT = 32 * kConsumerWarps;
     constexpr int DPL = S::DPL, KPW = S::KPW, NB = S::NB;
-    static_assert(4 * S::BK <= (int)kAttnWarpFloats && kMaxGroup * HD <= (int)kAttnWarpFloats, "attention scratch");
+    using SC = AttnScratch<HD>;
+    static_assert(4 * S::BK <= (int)SC::kWarp && kMaxGroup * HD <= (int)SC::kWarp, "attention scratch");
     const int n = R.n, t = warp * 32 + lane;
     const int nc = R.jnew >= 0 ? n - 1 : n;  // rows read from the fills
     const float scale = 1.0f / sqrtf((float)HD);
-    float* ew = sc + (size_t)warp * kAttnWarpFloats;  // this warp's region
+    float* ew = sc + (size_t)warp * SC::kWarp;  // this warp's region
     const int dc = lane % S::LPK, kk = lane / S::LPK;
     const int hh = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);  // head this lane's scores belong to
     const bool writer = (lane & (S::LPK == 8 ? 1 : 9)) == 0;    // one lane per (key, head)
@@ -941,8 +922,8 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
     lpart += __shfl_xor_sync(0xffffffffu, lpart, 16);
     __syncwarp();  // the last block's weights have been read
     if (lane < 8 && (lane & 1) == 0) {
-        sc[kAttnWM + 4 * warp + hh] = hh < G ? mrun : -INFINITY;
-        sc[kAttnWL + 4 * warp + hh] = hh < G ? lpart : 0.f;
+        sc[SC::kWM + 4 * warp + hh] = hh < G ? mrun : -INFINITY;
+        sc[SC::kWL + 4 * warp + hh] = hh < G ? lpart : 0.f;
     }
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h)
@@ -958,13 +939,13 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         const int h = u / HD, d = u % HD;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[kAttnWM + 4 * w + h]);
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[SC::kWM + 4 * w + h]);
         float L = 0.f, O = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
-            const float fw = exp_rel(sc[kAttnWM + 4 * w + h], M);
-            L = fmaf(fw, sc[kAttnWL + 4 * w + h], L);
-            O = fmaf(fw, sc[(size_t)w * kAttnWarpFloats + h * HD + d], O);
+            const float fw = exp_rel(sc[SC::kWM + 4 * w + h], M);
+            L = fmaf(fw, sc[SC::kWL + 4 * w + h], L);
+            O = fmaf(fw, sc[(size_t)w * SC::kWarp + h * HD + d], O);
         }
         emit(h, d, O, M, L);
     }

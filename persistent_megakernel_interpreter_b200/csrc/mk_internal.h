@@ -16,9 +16,17 @@
 namespace mk {
 
 constexpr int kConsumerWarps = 8;                    // compute warps
-constexpr int kLoaderWarp = kConsumerWarps;          // streams weights and cached KV
-constexpr int kPrepWarp = kConsumerWarps + 1;        // stages RoPE rows and down-projection inputs
-constexpr int kThreads = 32 * (kConsumerWarps + 2);
+// Mover warps kConsumerWarps .. +3: mover q (its warp index mod 4 is q, the Tensor
+// Memory lane quarter it may access) moves each landed weight tile of the ring
+// fills seq = q (mod 4) into Tensor Memory.
+constexpr int kMoveWarps = 4;
+constexpr int kPrepWarp = kConsumerWarps + kMoveWarps;   // stages RoPE rows and down-projection inputs
+constexpr int kLoaderWarp = kPrepWarp + 1;               // lane 0 issues every ring fill
+constexpr int kThreads = 32 * (kLoaderWarp + 1);
+// 14 warps: two of the SM's four schedulers (16384 registers each) host four of
+// them, so a thread gets at most 16384 / (4 * 32) = 128 registers.
+constexpr uint32_t kTmemCols = 512;                  // all of an SM's Tensor Memory (256 KB)
+constexpr int kMaxTmemSlots = 64;                    // weight tiles Tensor Memory holds at most
 constexpr int kRowsPerTile = 4;                      // every matvec tile holds 4 rows
 constexpr int kMaxDownRows = 16;                     // row blocks per down instruction
 constexpr int kMaxResidRows = 64;                    // residual rows per O-proj / down job
@@ -26,10 +34,18 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroupHeads = 4;                    // query heads per KV head
 constexpr int kMaxParts = 32;                        // split-K partitions per (sequence, group)
 constexpr int kMaxItemKeys = 512;                    // keys of one attention item at most
-// Shared-memory scratch of one attention item, in floats: per compute warp a
-// region of 4 * 128 (a block's weights while the warp runs, then its value sums
-// for up to 4 heads of up to 128 dims), the warps' maxima and sums, a flag word.
-constexpr uint32_t kAttnScratchFloats = 4 * 128 * kConsumerWarps + 8 * kConsumerWarps + 4;
+// Shared-memory scratch of one attention item (inside its job slot, after the
+// item's q and new key/value), in floats: per compute warp a region of 4 * hd
+// (a block's weights while the warp runs, then its value sums for up to 4 heads
+// of hd dims), the warps' maxima and sums, a flag word.
+MK_HD constexpr uint32_t attn_scratch_floats(int hd) {
+    return 4u * (uint32_t)hd * kConsumerWarps + 8u * kConsumerWarps + 4u;
+}
+// An attention item's q (fp32 [group][hd]) and new key and value (bf16 [2][hd]) at
+// the start of its job slot, 16-byte aligned; the scratch follows.
+MK_HD constexpr uint32_t attn_item_bytes(int group, int hd) {
+    return ((uint32_t)(group * hd * 4 + 2 * hd * 2) + 15u) & ~15u;
+}
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
@@ -65,10 +81,11 @@ struct Layout {
 struct SmemLayout {
     uint32_t ring, full, empty, armed;        // weight / cached-KV ring of S stages
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
-    uint32_t scores;                          // attention item scratch (kAttnScratchFloats)
     uint32_t tot;                             // down-projection running sums
     uint32_t red;                             // per-warp partial sums of a job input
     uint32_t cbar;                            // barrier of the compute warps
+    uint32_t tfull, tempty, tarmed;           // Tensor Memory slots: landed / released / fill held
+    uint32_t tbase;                           // Tensor Memory address of the allocation
     uint32_t total;
 };
 
@@ -85,10 +102,14 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs_full = o;   o += 8u * NS;
     m.xs_empty = o;  o += 8u * NS;
     m.xs_done = o;   o = align16(o + 4u * NS);
-    m.scores = o;    o += 4u * kAttnScratchFloats;
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
     m.red = o;       o += 4u * 32u;
     m.cbar = o;      o += 8u;
+    o = (o + 7u) & ~7u;
+    m.tfull = o;     o += 8u * kMaxTmemSlots;
+    m.tempty = o;    o += 8u * kMaxTmemSlots;
+    m.tarmed = o;    o += 4u * kMaxTmemSlots;
+    m.tbase = o;     o += 4u;
     m.total = align16(o);
     return m;
 }
@@ -143,7 +164,9 @@ struct Params {
     int n_sm;
     int part_keys, n_parts, keys_per_stage;
     uint32_t stage_bytes;
-    int n_stages;
+    int n_stages;              // ring stages (a multiple of 4)
+    int n_tslots;              // Tensor Memory slots (a multiple of 4; slot k in lane quarter k % 4)
+    uint32_t tslot_cols;       // columns of one slot: a stage's bytes / (32 lanes * 4 bytes)
     int xs_slots;              // activation slots (1..3)
     uint32_t xs_slot_bytes;
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot

@@ -42,22 +42,33 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
     SlotPlan sp{};
     sp.keys_per_stage = (int)(stage_bytes / (4u * (uint32_t)L.d));
     sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
-    sp.item_bytes = align16((uint32_t)(L.group * L.d * 4 + 2 * L.d * 2));
+    sp.item_bytes = attn_item_bytes(L.group, L.d) + 4u * attn_scratch_floats(L.d);
     // per sequence: the input vector; then per sequence (QKV jobs) the RoPE row
     // cos[d/2], sin[d/2] and the position; then per sequence (O-proj and down
     // jobs) the residual rows the job updates. An attention job: its item's q and
-    // new key/value.
+    // new key/value, then the item's scratch.
     sp.slot_bytes = align16(std::max(
         (uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u, sp.item_bytes));
-    for (int ns = 3; ns >= 1; --ns) {
-        int S = 0;
-        while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
-            ++S;
-        if (S >= (ns > 1 ? 6 : 2) || ns == 1) {
-            sp.xs_slots = ns;
-            sp.stages = S;
-            break;
+    // the most job slots that leave at least 8 stages (an attention item's keys all
+    // sit in the ring at once), else at least 4; the stage count is a multiple of
+    // 4, so each stage's fills belong to one mover warp
+    sp.xs_slots = 0;
+    for (int min_s = 8; min_s >= kMoveWarps && sp.xs_slots == 0; min_s -= 4) {
+        for (int ns = 3; ns >= 1; --ns) {
+            int S = 0;
+            while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
+                ++S;
+            S -= S % kMoveWarps;
+            if (S >= min_s) {
+                sp.xs_slots = ns;
+                sp.stages = S;
+                break;
+            }
         }
+    }
+    if (sp.xs_slots == 0) {  // nothing fits: reported by the caller (fewer than 4 stages)
+        sp.xs_slots = 1;
+        sp.stages = 0;
     }
     sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes).total;
     return sp;
@@ -76,7 +87,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     if (stage_bytes % 128 || stage_bytes < default_stage_bytes(L)) return MK_ERR_INVALID_ARG;
     const SlotPlan sp = slot_plan(L, batch, stage_bytes);
     const int kps = sp.keys_per_stage;
-    if (kps < 1 || sp.stages < 2) return MK_ERR_UNSUPPORTED;
+    if (kps < 1 || sp.stages < kMoveWarps) return MK_ERR_UNSUPPORTED;
     // the attention value phase splits an item's keys into classes j mod KQ
     // (KQ = compute threads / (head_dim / 2)); a ring stage must hold whole rounds
     const int attn_classes = std::max(1, 32 * kConsumerWarps / (L.d / 2));
