@@ -160,7 +160,11 @@ struct Tmem {
 
 struct Slots {
     uint8_t* base;
-    uint64_t* full;    // the activation warp arrives when a job's input is ready
+    uint64_t* full;    // the job's preparer (activation or stage warp) arrives when its input is ready
+    // The job each slot was last prepared for. Several warps prepare jobs, so the
+    // preparer of job j first waits until its slot was prepared for job j - NS, and
+    // only then on the empty parity (which tells phases one lap apart only).
+    volatile uint32_t* job;
     uint64_t* empty;   // each compute warp arrives when it is done with the job
     uint32_t* done;    // compute warps finished with the job (the last one signals)
     uint32_t bytes;
@@ -605,25 +609,39 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
     return true;
 }
 
+// The preparer of `job`: -1 is the activation warp, h >= 0 stage warp h (at batch
+// 1, the down-projection chunk-h jobs, h < kStageWarps and h < kDownStaged).
+template <bool BATCHED>
+__device__ __forceinline__ int preparer(uint32_t op, int c) {
+    return (!BATCHED && op == MK_OP_DOWN && c < kStageWarps && c < kDownStaged) ? c : -1;
+}
+
+// The activation warp (role -1) or stage warp h (role h) walks the SM's jobs and
+// prepares its own: it waits for the job's slot (prepared for job j - NS, then
+// released by the compute warps), stages what the job needs ahead (prep_job),
+// records the job in the slot and arrives on the slot's full barrier.
 template <int KH, int KO, int KF, int HD, bool BATCHED>
-__device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1, int lane, uint32_t epoch) {
+__device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1, int lane, uint32_t epoch,
+                                int role) {
     uint32_t j = 0;
     for (int i = i0; i < i1;) {
         const mk_instr* ins = p.instrs + i;
         const uint32_t op = ins[0].op;
         const int njobs = (op == MK_OP_DOWN) ? 4 : 1;
         for (int c = 0; c < njobs; ++c, ++j) {
+            if (preparer<BATCHED>(op, c) != role) continue;
             const uint32_t s = j % sl.NS, use = j / sl.NS;
             if (lane == 0) {
                 trace(p, j, kTrSlotWait);
                 trace(p, j, kTrMeta, op | ((uint32_t)ins[0].layer << 8) | ((uint32_t)c << 24));
             }
-            if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, nullptr, j, 3, lane)) return;
+            if (use > 0 && !wait_bar(p, sl.empty + s, (use - 1) & 1u, sl.job + s, j - sl.NS, 3, lane)) return;
             if (lane == 0) trace(p, j, kTrCtrWait);
             if (!prep_job<HD, BATCHED>(p, ins, c, sl.slot(j), lane, epoch, j)) return;
             __syncwarp();
             if (lane == 0) {
                 trace(p, j, kTrReady);
+                sl.job[s] = j;             // published by the release of the arrive below
                 mbar_arrive(sl.full + s);  // release: the slot's contents
             }
         }
@@ -1228,6 +1246,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     sl.full = reinterpret_cast<uint64_t*>(smem + m.xs_full);
     sl.empty = reinterpret_cast<uint64_t*>(smem + m.xs_empty);
     sl.done = reinterpret_cast<uint32_t*>(smem + m.xs_done);
+    sl.job = reinterpret_cast<volatile uint32_t*>(smem + m.xs_job);
     sl.bytes = p.xs_slot_bytes;
     sl.NS = (uint32_t)p.xs_slots;
     Tmem tm;
@@ -1260,6 +1279,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(sl.full + s, 1);
             mbar_init(sl.empty + s, kConsumerWarps);
             sl.done[s] = 0;
+            sl.job[s] = 0xffffffffu;
         }
         mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
         fence_mbar_init();
@@ -1291,8 +1311,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mover<BATCHED>(p, ring, tm, i0, i1, warp & 3, lane);
         } else if (warp == kLoaderWarp) {
             if (lane == 0) loader(p, ring, i0, i1);
-        } else if (warp == kPrepWarp) {
-            activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch);
+        } else if (warp == kPrepWarp || warp >= kStageWarp0) {
+            // one call site: the stage warps have jobs at batch 1 only
+            if (warp == kPrepWarp || !BATCHED)
+                activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch,
+                                                         warp == kPrepWarp ? -1 : warp - kStageWarp0);
         } else {
             compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, tm, sl, reinterpret_cast<float*>(smem + m.tot),
                                          reinterpret_cast<float*>(smem + m.red),

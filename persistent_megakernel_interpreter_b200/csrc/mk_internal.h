@@ -22,8 +22,12 @@ constexpr int kConsumerWarps = 8;                    // compute warps
 constexpr int kMoveWarps = 4;
 constexpr int kPrepWarp = kConsumerWarps + kMoveWarps;   // stages RoPE rows and down-projection inputs
 constexpr int kLoaderWarp = kPrepWarp + 1;               // lane 0 issues every ring fill
-constexpr int kThreads = 32 * (kLoaderWarp + 1);
-// 14 warps: two of the SM's four schedulers (16384 registers each) host four of
+// Stage warps: at batch 1, stage warp h stages the h chunk of every down-projection
+// chunk-h job (h < kStageWarps), in parallel with the activation warp's other jobs.
+constexpr int kStageWarps = 2;
+constexpr int kStageWarp0 = kLoaderWarp + 1;
+constexpr int kThreads = 32 * (kStageWarp0 + kStageWarps);
+// 16 warps: each of the SM's four schedulers (16384 registers each) hosts four of
 // them, so a thread gets at most 16384 / (4 * 32) = 128 registers.
 constexpr uint32_t kTmemCols = 512;                  // all of an SM's Tensor Memory (256 KB)
 constexpr int kMaxTmemSlots = 64;                    // weight tiles Tensor Memory holds at most
@@ -81,6 +85,7 @@ struct Layout {
 struct SmemLayout {
     uint32_t ring, full, empty, armed;        // weight / cached-KV ring of S stages
     uint32_t xs, xs_full, xs_empty, xs_done;  // NS activation slots
+    uint32_t xs_job;                          // the job each slot was last prepared for
     uint32_t tot;                             // down-projection running sums
     uint32_t red;                             // per-warp partial sums of a job input
     uint32_t cbar;                            // barrier of the compute warps
@@ -101,7 +106,8 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.xs = o;        o += (uint32_t)NS * slot_bytes;
     m.xs_full = o;   o += 8u * NS;
     m.xs_empty = o;  o += 8u * NS;
-    m.xs_done = o;   o = align16(o + 4u * NS);
+    m.xs_done = o;   o += 4u * NS;
+    m.xs_job = o;    o = align16(o + 4u * NS);
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
     m.red = o;       o += 4u * 32u;
     m.cbar = o;      o += 8u;
