@@ -67,8 +67,73 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+class NvmlClocks:
+    """Read-only NVML queries in this process: the SM clock and the clock-event
+    (throttle) reasons, sampled at the start and the end of the timed region and
+    every few milliseconds in between, so a short timed region still has a record.
+    Changes nothing on the GPU."""
+    # NVML clock-event reason bits (nvmlClocksEventReason*)
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.dev, self.period = device_index, period_s
+        self.samples, self.max_mhz, self.handle = [], None, None
+        self._stop = threading.Event()
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(self.dev)
+            bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.sample()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        except Exception:  # no NVML on this machine: the nvidia-smi record stands alone
+            self.handle = None
+        return self
+
+    def sample(self):
+        if self.handle is None:
+            return
+        try:
+            mhz = float(self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
+            bits = int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            self.samples.append((mhz, bits))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.wait(self.period):
+            self.sample()
+
+    def __exit__(self, *exc):
+        if self.handle is None:
+            return
+        self._stop.set()
+        self.thread.join(timeout=2)
+        self.sample()
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+
+    def summary(self):
+        reasons = sorted({n for _, b in self.samples for n, m in self.REASONS.items() if b & m})
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and throttle reasons during the timed region: nvidia-smi samples
+    every 100 ms and in-process NVML samples (NvmlClocks), merged."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -77,8 +142,10 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.nvml = NvmlClocks(gpu_index)
 
     def __enter__(self):
+        self.nvml.__enter__()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
@@ -95,6 +162,7 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        self.nvml.__exit__(*exc)
         if self.proc:
             self.proc.terminate()
             try:
@@ -118,8 +186,14 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max_mhz,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        nv = self.nvml.summary()
+        reasons |= set(nv["reasons"])
+        nv_mhz = [m for m, _ in self.nvml.samples]
+        allm = mhz + nv_mhz
+        return {"sm_mhz": statistics.median(allm) if allm else None,
+                "sm_max_mhz": max_mhz if max_mhz is not None else nv["sm_max_mhz"],
+                "reasons": sorted(reasons), "samples": len(allm),
+                "samples_nvidia_smi": len(mhz), "samples_nvml": len(nv_mhz)}
 
 
 def dist_setup(n_gpus: int):
@@ -457,6 +531,42 @@ def run_greedy(args):
         raise RuntimeError(f"greedy decode failed: {msg}")
     us = np.array([1e3 * a.elapsed_time(b) for a, b in ev])
     gen = us[n_prompt:]
+
+    # The generated tokens again, each variant timed as a whole from the same state
+    # (the prompt decoded into an empty cache): (a) mk_decode_step + mk_greedy_select
+    # launches, selection inside the timed region; (b) mk_decode_steps_greedy, the
+    # choice fused into each step's LM head, one call for all tokens.
+    def after_prompt():
+        kd.zero_()
+        vd.zero_()
+        for p in range(n_prompt):
+            pos.fill_(p)
+            tok.copy_(prompt[p:p + 1])
+            mk.decode_step(tok, pos, kd, vd, logits, stream)
+        greedy_select(logits, tok, pos)  # the first generated token, position n_prompt
+
+    timed = {}
+    seqs = {}
+    with torch.cuda.stream(stream):
+        for variant in ("select_launch", "fused"):
+            after_prompt()
+            out = torch.empty(n_gen, 1, dtype=torch.int32, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if variant == "fused":
+                mk.decode_steps_greedy(tok, pos, kd, vd, logits, n_gen, generated=out, stream=stream)
+            else:
+                for i in range(n_gen):
+                    mk.decode_step(tok, pos, kd, vd, logits, stream)
+                    greedy_select(logits, tok, pos, stream=stream)
+                    out[i].copy_(tok)
+            e1.record(stream)
+            stream.synchronize()
+            timed[variant] = 1e3 * e0.elapsed_time(e1) / n_gen
+            seqs[variant] = out.cpu().numpy().ravel()
+    code, msg = mk.status()
+    if code != 0:
+        raise RuntimeError(f"greedy decode failed: {msg}")
     peak, peak_kind = hbm_peak()
     line = {
         "metric": "µs per decode step, greedy decode at batch 1 (each step timed alone)",
@@ -475,6 +585,10 @@ def run_greedy(args):
                                "frac": cfg.step_bytes(1, steps - 1) / (us[-1] * 1e-6) / 1e9 / peak,
                                "peak_source": peak_kind},
         "gpu_launches": steps,
+        "per_token_us_selection_inside": {
+            "decode_step_then_greedy_select_launch": timed["select_launch"],
+            "fused_into_lm_head_one_call": timed["fused"],
+            "same_tokens": bool(np.array_equal(seqs["select_launch"], seqs["fused"]))},
         "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)

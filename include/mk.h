@@ -96,7 +96,12 @@ typedef struct mk_handle mk_handle;
 /* Create a handle on `device`: validates the shape, packs the weights into one
  * library-owned device buffer (layout: see mk_pack_weights_host), builds the RoPE
  * table (angles in double, cos/sin stored as float) and allocates the scratch
- * (activations, attention partials, counters). Synchronous. On error *out is NULL. */
+ * (activations, attention partials, counters). Synchronous. On error *out is NULL.
+ * Defining passage: the Cohere decode megakernel page ("Cohere 开源 Megakernel 推理
+ * 系统"), section "Megakernel 是什么": one resident thread block per SM for the
+ * whole decode step, working from host-prepared tile-sized tasks; the handle
+ * holds what those tasks read, laid out once before any step (weights as
+ * contiguous tiles, the RoPE table, the counters and scratch in global memory). */
 mk_status mk_create(const mk_config* cfg, const mk_weights* w, int device, mk_handle** out);
 
 /* Options for mk_build_schedule; pass NULL for defaults. Zero fields mean "auto". */
@@ -123,6 +128,13 @@ typedef struct mk_schedule_opts {
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)
  * whose steps use at most `max_ctx` keys (position + 1 <= max_ctx <= max_seq), and
  * upload them. Replaces any earlier schedule. Synchronous.
+ * Defining passages: the "Look Ma, No Bubbles" summary, section "Fusing Operations
+ * with an On-GPU Interpreter" (each SM executes a sequence of instructions such as
+ * fused RMSNorm + QKV + RoPE, attention, ...), and the Stanford write-up
+ * ("斯坦福团队新作：Llama-1B实现毫秒级推理获Andrej Karpathy盛赞"), section
+ * "Megakernel：从零设计的融合思路" (an execution plan per SM, dependencies between
+ * instructions arranged statically before the run); the Cohere page, section
+ * "Megakernel 是什么" (the host writes the task list into global memory).
  * The attention of a (sequence, KV group) is split into at most 32 key partitions,
  * each holding at most what the SM's weight ring holds at once (and 512 keys), so
  * max_ctx has a ceiling that depends on the shape and batch: 16384 keys for the
@@ -132,6 +144,11 @@ typedef struct mk_schedule_opts {
 mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts);
 
 /* One decode step of the persistent megakernel, asynchronous on `stream`.
+ * Defining passage: the "Look Ma, No Bubbles" summary, section "Megakernel: The
+ * Core Solution" (the whole Llama-1B forward pass as one kernel, so loads and
+ * compute continue across what would be kernel boundaries), with section "Custom
+ * Synchronization Mechanism" (dependencies inside the kernel; the MLP's
+ * intermediate state in four chunks so the down-projection starts early).
  *   tokens, positions : device int32 [batch]
  *   k_cache, v_cache  : device bf16 [n_layers][max_batch][n_kv_heads][max_seq][head_dim],
  *                       caller-owned; sequence b reads slots 0..positions[b] and writes
@@ -145,6 +162,24 @@ mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_sched
  * MK_ERR_NO_SCHEDULE before mk_build_schedule. */
 mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const int32_t* positions,
                          void* k_cache, void* v_cache, float* logits, void* stream);
+
+/* n_steps greedy decode steps back to back, asynchronous on `stream`, with no host
+ * work between them: each is mk_decode_step with the greedy choice fused into its
+ * LM head. Each LM-head instruction reduces its rows to the best (largest logit,
+ * lowest index among equal ones, NaN never chosen; an all-NaN row gives 0) per
+ * sequence; the SM that completes the step's LM head picks each sequence's next
+ * token from those and writes it over tokens[b], writes positions[b] + 1 over
+ * positions[b], and, when `generated` (device int32 [n_steps][batch]) is given,
+ * stores it at generated[step][b]. The next launch then decodes it. The tokens
+ * equal mk_greedy_select's on the same logits, bit for bit; `logits` holds the
+ * last step's. Arguments as for mk_decode_step (tokens and positions are read and
+ * written); n_steps >= 1 launches are enqueued. The caller keeps the positions
+ * below max_ctx: a step past it is skipped and reported (MK_ERR_BAD_POSITION), as
+ * are the steps after it. Defining passage: the "Look Ma, No Bubbles" summary,
+ * section "Megakernel: The Core Solution" (no kernel boundaries inside a forward
+ * pass): here the token choice, too, stays inside the step's kernel. */
+mk_status mk_decode_steps_greedy(mk_handle* h, int32_t* tokens, int32_t* positions, void* k_cache,
+                                 void* v_cache, float* logits, int32_t* generated, int n_steps, void* stream);
 
 /* The same step as a sequence of ordinary kernels (one per op and layer), the
  * multi-kernel "bubble" baseline; identical arguments, identical arithmetic, so
@@ -226,7 +261,8 @@ typedef struct mk_instr {
                             job of the SM's compute warps (DOWN: four, one per chunk) */
     uint32_t aux0, aux1; /* DOWN: per-step increments of chunk counters 1, 2 (low and
                             high 16 bits of aux0) and 3 (aux1). ATTN: aux0 = the pair's
-                            arrival counter (heads whose partial is stored). GATEUP:
+                            arrival counter (heads whose partial is stored). LMHEAD:
+                            aux0 = its ordinal among the step's LM-head instructions. GATEUP:
                             aux0 = tiles per chunk; the instruction's tile i is tile
                             (i / aux0) * (ffn / 8) + first + i % aux0 (chunk-major). QKV and
                             GATEUP: aux1 = how many consecutive counters from signal_ctr
@@ -311,18 +347,23 @@ mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights* w, void* 
  *   status_out        device int32 or NULL: receives the step's device status
  *                     (MK_OK, MK_ERR_BAD_TOKEN, MK_ERR_BAD_POSITION)
  *   stream            the CUDA stream the step is enqueued on
- * Scratch (activations, attention partials, the RoPE table of max_ctx
- * positions, the error word) lives in one 4 MiB device array of the library,
- * per device, held until the process exits. The first call on a device (with
- * that device current) looks up the array's device address; a call whose
- * configuration (rope_theta, head_dim, max_ctx) differs from the previous call's
- * uploads a new RoPE table from the stack. Make that first call before any
- * stream capture. Every call shares the array and leaves its contents for the
- * next; the error word is cleared by each call. Calls that overlap on the GPU
- * (on different streams, or from different host threads) race on it.
- * Returns MK_ERR_INVALID_ARG for bad arguments and for a step whose scratch
- * exceeds the 4 MiB array (about max_ctx <= 8192 at batch 1 for a 1B-shaped
- * model; more than 32 attention partitions of 320 keys are refused too). */
+ * Scratch (activations, attention partials, the RoPE table, the error word) lives
+ * in one 4 MiB device array of the library, per device, held until the process
+ * exits. Its layout does not depend on max_ctx: the RoPE table holds a fixed
+ * number of positions per head_dim (8192 at 64, 4096 at 128) in a 2 MiB region,
+ * the activations follow at a fixed offset. The first call on a device (with that
+ * device current) looks up the array's device address, and a call whose
+ * rope_theta or head_dim differs from the table in the array uploads a new table
+ * from the stack: make those calls before any stream capture (during a capture
+ * such a call returns MK_ERR_INVALID_ARG), and do not replay a graph captured
+ * before a change of rope_theta or head_dim. Every call shares the array and
+ * leaves its contents for the next; the error word is cleared by each call. Calls
+ * that overlap on the GPU (on different streams, or from different host threads)
+ * race on it.
+ * Returns MK_ERR_INVALID_ARG for bad arguments, for max_ctx beyond the RoPE
+ * table's positions, and for a step whose activations and attention partials
+ * exceed the array's other 2 MiB (more than 32 attention partitions of 320 keys
+ * are refused too). */
 mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const void* packed, const int32_t* tokens,
                                           const int32_t* positions, void* k_cache, void* v_cache, float* logits,
                                           int batch, int max_ctx, int32_t* status_out, void* stream);

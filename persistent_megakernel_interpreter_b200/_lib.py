@@ -102,7 +102,8 @@ def lib() -> ctypes.CDLL:
     L.mk_baseline_decode_step_noalloc.argtypes = [ctypes.POINTER(MkConfig), P, P, P, P, P, P, ctypes.c_int,
                                                   ctypes.c_int, P, P]
     L.mk_greedy_select.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P]
-    for f in ("mk_create", "mk_build_schedule", "mk_decode_step", "mk_baseline_decode_step",
+    L.mk_decode_steps_greedy.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P]
+    for f in ("mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_steps_greedy", "mk_baseline_decode_step",
               "mk_decode_step_host", "mk_get_status", "mk_plan_schedule_host",
               "mk_get_schedule_info", "mk_read_counters", "mk_pack_weights_host", "mk_read_trace",
               "mk_baseline_decode_step_noalloc", "mk_greedy_select"):

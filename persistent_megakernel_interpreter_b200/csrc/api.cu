@@ -255,6 +255,9 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     const size_t o_tag = take(tagged_words * sizeof(uint64_t));
     const size_t o_ctr = take((size_t)I.n_counters * mk::kCounterStride * sizeof(uint32_t));
     const size_t o_ctl = take(sizeof(mk::Ctl));
+    int n_lm = 0;  // LM-head instructions: one greedy-selection entry each per sequence
+    for (const mk_instr& in : P.instrs) n_lm += in.op == MK_OP_LMHEAD;
+    const size_t o_sel = take((size_t)batch * n_lm * 2 * sizeof(uint32_t));
     MK_CUDA(h, cudaMalloc(&h->scratch, off));
     MK_CUDA(h, cudaMemset(h->scratch, 0, off));
     h->scratch_bytes = off;
@@ -300,6 +303,8 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     p.tagged_words = tagged_words;
     p.counters = h->counters;
     p.ctl = h->ctl;
+    p.sel_best = reinterpret_cast<uint32_t*>(sb + o_sel);
+    p.n_lm_jobs = n_lm;
     p.instrs = h->d_instrs;
     p.sm_off = h->d_sm_off;
     p.n_sm = n_sm;
@@ -399,6 +404,30 @@ extern "C" mk_status mk_decode_step(mk_handle* h, const int32_t* tokens, const i
     p.vc = static_cast<uint16_t*>(v_cache);
     p.logits = logits;
     MK_CUDA(h, mk::megakernel_launch(p, static_cast<cudaStream_t>(stream)));
+    return MK_OK;
+}
+
+extern "C" mk_status mk_decode_steps_greedy(mk_handle* h, int32_t* tokens, int32_t* positions, void* k_cache,
+                                            void* v_cache, float* logits, int32_t* generated, int n_steps,
+                                            void* stream) {
+    mk_status st = step_args(h, tokens, positions, k_cache, v_cache, logits);
+    if (st != MK_OK) return st;
+    if (n_steps < 1) return MK_ERR_INVALID_ARG;
+    mk::Params p = h->params;
+    p.tokens = tokens;
+    p.positions = positions;
+    p.kc = static_cast<uint16_t*>(k_cache);
+    p.vc = static_cast<uint16_t*>(v_cache);
+    p.logits = logits;
+    // the step's selection overwrites the tokens and advances the positions it read
+    // (their last reads come long before the LM head), so the next launch decodes
+    // the chosen tokens with no host work in between
+    p.next_tokens = tokens;
+    p.next_positions = positions;
+    for (int s = 0; s < n_steps; ++s) {
+        p.gen_tokens = generated ? generated + (size_t)s * p.B : nullptr;
+        MK_CUDA(h, mk::megakernel_launch(p, static_cast<cudaStream_t>(stream)));
+    }
     return MK_OK;
 }
 

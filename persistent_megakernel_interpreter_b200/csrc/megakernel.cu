@@ -651,6 +651,31 @@ __device__ void activation_warp(const Params& p, const Slots& sl, int i0, int i1
 
 // ------------------------------------------------------------------ compute warps
 
+// Greedy selection: (value, index) pairs, the larger value first, the lower index
+// among equal values; a NaN value is never chosen (an all-NaN row gives index 0).
+struct Best {
+    float v;
+    uint32_t i;
+};
+__device__ __forceinline__ Best best_none() { return {__int_as_float(0x7fffffff), 0xffffffffu}; }
+__device__ __forceinline__ bool best_before(float v, uint32_t i, const Best& b) {
+    if (v != v) return false;          // NaN: never
+    if (b.v != b.v) return true;       // anything beats nothing
+    return v > b.v || (v == b.v && i < b.i);
+}
+__device__ __forceinline__ void best_take(Best& b, float v, uint32_t i) {
+    if (best_before(v, i, b)) b = {v, i};
+}
+// Over the lanes whose bits under `mask` differ (an xor butterfly).
+__device__ __forceinline__ Best best_reduce(Best b, uint32_t masks_from, uint32_t masks_to) {
+    for (uint32_t m = masks_from; m >= masks_to && m > 0; m >>= 1) {
+        const float v = __shfl_xor_sync(0xffffffffu, b.v, (int)m);
+        const uint32_t i = __shfl_xor_sync(0xffffffffu, b.i, (int)m);
+        best_take(b, v, i);
+    }
+    return b;
+}
+
 // One 4-row tile, read from the warp's Tensor Memory slot at `ta`, against an
 // input vector in shared memory: the same lane mapping and order of arithmetic as
 // dot4 (lane ln holds the 16-byte pieces (row r, kc*32 + ln); the mover stored
@@ -693,9 +718,11 @@ __device__ __noinline__ float4 tile_dot(uint32_t ta, const float* v, int lane) {
 // seq mod 4, is the one the mover stored it in).
 template <int KC, int HD>
 __device__ bool compute_tiles(const Params& p, const Tmem& tm, const mk_instr& in,
-                              const float* sv, int warp, int lane, uint32_t job, uint32_t epoch) {
+                              const float* sv, int warp, int lane, uint32_t job, uint32_t epoch, uint2* selp) {
     // a dropped instruction (the failure-detection hook) computes but publishes nothing
     const bool pub = in.signal_ctr != MK_NO_COUNTER;
+    const bool sel = in.op == MK_OP_LMHEAD && p.next_tokens != nullptr;
+    Best best = best_none();  // the lane's LM-head row (lanes 0..3)
     int k = 0;  // trace: warp 0's first tiles (fill wait start, fill ready, dot done)
     auto stamp = [&](int w) {
         if (warp == 0 && lane == 0 && w < 8) trace(p, job, kTrSub0 + w);
@@ -735,11 +762,18 @@ __device__ bool compute_tiles(const Params& p, const Tmem& tm, const mk_instr& i
                                   act_tag(epoch, in.layer, kTagXAttn));
                     }
                     break;
-                default: logits_epilogue(p, b, tl, acc, el); break;
+                default:
+                    logits_epilogue(p, b, tl, acc, el);
+                    if (sel && el < 4) best_take(best, pick4(acc, el), tl * 4 + el);
+                    break;
             }
         }
         if (k == 1) stamp(6);
         ++k;
+    }
+    if (sel) {  // the warp's best of the job, for the job's last warp (publish_best)
+        best = best_reduce(best, 16, 1);
+        if (lane == 0) selp[warp * kMaxBatch] = make_uint2(__float_as_uint(best.v), best.i);
     }
     return true;
 }
@@ -792,8 +826,10 @@ struct PairSeqs {
 
 template <int KC, int HD>
 __device__ bool compute_tiles_pair(const Params& p, const Tmem& tm, const mk_instr& in, const float* sv, int warp,
-                                   int lane, uint32_t job, uint32_t epoch) {
+                                   int lane, uint32_t job, uint32_t epoch, uint2* selp) {
     const bool pub = in.signal_ctr != MK_NO_COUNTER;
+    const bool sel = in.op == MK_OP_LMHEAD && p.next_tokens != nullptr;
+    Best best = best_none();  // the lane's row of its sequence (active lanes)
     const PairSeqs ps(p.B, warp);
     const int sl = lane >> 3;                         // the sequence (of this warp's) the lane holds
     const bool act = sl < ps.nb && (lane & 1) == 0;   // lanes l and l ^ 1 hold the same total
@@ -827,7 +863,19 @@ __device__ bool compute_tiles_pair(const Params& p, const Tmem& tm, const mk_ins
                               act_tag(epoch, in.layer, kTagXAttn));
                 }
                 break;
-            default: logits_epilogue(p, b, tl, acc, el); break;
+            default:
+                logits_epilogue(p, b, tl, acc, el);
+                if (sel && el < 4) best_take(best, pick4(acc, el), tl * 4 + el);
+                break;
+        }
+    }
+    if (sel) {
+        // lanes 8 s' .. 8 s' + 7 hold the warp's sequence b0 + s' (the active ones)
+        best = best_reduce(best, 4, 1);
+        for (int s2 = 0; s2 < 4; ++s2) {
+            const float v = __shfl_sync(0xffffffffu, best.v, 8 * s2);
+            const uint32_t i = __shfl_sync(0xffffffffu, best.i, 8 * s2);
+            if (lane == 0 && s2 < ps.nb) selp[warp * kMaxBatch + ps.b0 + s2] = make_uint2(__float_as_uint(v), i);
         }
     }
     return true;
@@ -984,10 +1032,57 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     return true;
 }
 
+// The LM-head job's last compute warp (all lanes): the SM's best row of each
+// sequence from its warps' bests (at batch > 1 a sequence's tiles were shared by
+// the warps w with w / 4 = its half), stored at the job's ordinal in.aux0; then
+// one acquire-release increment of the LM-head counter. The job that completes the
+// step's count (epoch + 1) * n_lm_jobs reduces every job's best, one lane per
+// job, and writes each sequence's next token, its next position, and the token
+// into the generated list. Every step writes every entry before it counts, so no
+// stale entry is read.
+__device__ __noinline__ void publish_best(const Params& p, const mk_instr& in, const uint2* selp, int lane,
+                                          uint32_t epoch) {
+    const int per = (p.B + 1) / 2;
+    if (lane < p.B) {
+        const int b = lane;
+        const int w0 = p.B > 1 ? (b < per ? 0 : kPairGroups) : 0;
+        const int w1 = p.B > 1 ? w0 + kPairGroups : kConsumerWarps;
+        Best bb = best_none();
+        for (int w = w0; w < w1; ++w) {
+            const uint2 e = selp[w * kMaxBatch + b];
+            best_take(bb, __uint_as_float(e.x), e.y);
+        }
+        __stcg(reinterpret_cast<uint2*>(p.sel_best) + (size_t)b * p.n_lm_jobs + in.aux0,
+               make_uint2(__float_as_uint(bb.v), bb.i));
+    }
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        const uint32_t old = atom_acq_rel_add(p.counters + (size_t)in.signal_ctr * kCounterStride, 1u);
+        last = old + 1u == (epoch + 1u) * (uint32_t)p.n_lm_jobs;
+    }
+    if (!__shfl_sync(0xffffffffu, last, 0)) return;
+    for (int b = 0; b < p.B; ++b) {
+        Best bb = best_none();
+        for (int k = lane; k < p.n_lm_jobs; k += 32) {
+            const uint2 e = __ldcg(reinterpret_cast<const uint2*>(p.sel_best) + (size_t)b * p.n_lm_jobs + k);
+            best_take(bb, __uint_as_float(e.x), e.y);
+        }
+        bb = best_reduce(bb, 16, 1);
+        if (lane == 0) {
+            const int32_t tok = bb.i == 0xffffffffu ? 0 : (int32_t)bb.i;  // all NaN: 0
+            p.next_tokens[b] = tok;
+            if (p.next_positions) p.next_positions[b] = g_pos[b] + 1;
+            if (p.gen_tokens) p.gen_tokens[b] = tok;
+        }
+    }
+}
+
 template <int KH, int KO, int KF, int HD, bool BATCHED>
 __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, const Slots& sl,
-                             float* tot, float* red, uint64_t* cbar, int i0, int i1, int warp, int lane,
-                             uint32_t epoch) {
+                             float* tot, float* red, uint64_t* cbar, uint2* selp, int i0, int i1, int warp,
+                             int lane, uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
@@ -1017,25 +1112,35 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
                 else ok = compute_down<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
             } else if (KO != KH && in.op == MK_OP_OPROJ) {
                 if constexpr (KO != KH) {
-                    if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, tm, in, sv, warp, lane, j, epoch);
-                    else ok = compute_tiles<KO, HD>(p, tm, in, sv, warp, lane, j, epoch);
+                    if constexpr (BATCHED) ok = compute_tiles_pair<KO, HD>(p, tm, in, sv, warp, lane, j, epoch, selp);
+                    else ok = compute_tiles<KO, HD>(p, tm, in, sv, warp, lane, j, epoch, selp);
                 }
             } else {  // QKV, gate/up, the LM head (and the O-projection when its width is the hidden size)
-                if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, tm, in, sv, warp, lane, j, epoch);
-                else ok = compute_tiles<KH, HD>(p, tm, in, sv, warp, lane, j, epoch);
+                if constexpr (BATCHED) ok = compute_tiles_pair<KH, HD>(p, tm, in, sv, warp, lane, j, epoch, selp);
+                else ok = compute_tiles<KH, HD>(p, tm, in, sv, warp, lane, j, epoch, selp);
             }
             if (!ok) return;
             // job done for this warp; the last of the 8 counts the job's completion
             // (acquire-release at CTA scope on the shared count, then a relaxed
             // increment: consumers read the tagged outputs, not the counter)
             __syncwarp();
+            int last_warp = 0;
             if (lane == 0) {
                 const uint32_t old = atom_shared_acq_rel_add(sl.done + s, 1u);
-                if (old == kConsumerWarps - 1) {
+                last_warp = old == kConsumerWarps - 1;
+            }
+            last_warp = __shfl_sync(0xffffffffu, last_warp, 0);
+            // greedy selection: the LM-head job's last warp publishes the SM's best;
+            // the SM that completes the step's count picks the next tokens
+            if (last_warp && in.op == MK_OP_LMHEAD && p.next_tokens != nullptr && in.signal_ctr != MK_NO_COUNTER)
+                publish_best(p, in, selp, lane, epoch);
+            if (lane == 0) {
+                if (last_warp) {
                     sl.done[s] = 0;
                     trace(p, j, kTrDone);
                     // attention items signal their heads themselves (compute_attn_job)
-                    const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN;
+                    const bool last_chunk = (in.op != MK_OP_DOWN || c == 3) && in.op != MK_OP_ATTN &&
+                                            !(in.op == MK_OP_LMHEAD && p.next_tokens != nullptr);
                     if (last_chunk && in.signal_ctr != MK_NO_COUNTER) {
                         // QKV / gate-up: one increment on each KV group / MLP chunk counter
                         // the job's tiles touched
@@ -1318,9 +1423,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
                                                          warp == kPrepWarp ? -1 : warp - kStageWarp0);
         } else {
             compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, tm, sl, reinterpret_cast<float*>(smem + m.tot),
-                                         reinterpret_cast<float*>(smem + m.red),
-                                         reinterpret_cast<uint64_t*>(smem + m.cbar), i0, i1, warp, lane,
-                                         s_epoch);
+                                                  reinterpret_cast<float*>(smem + m.red),
+                                                  reinterpret_cast<uint64_t*>(smem + m.cbar),
+                                                  reinterpret_cast<uint2*>(smem + m.sel), i0, i1, warp, lane,
+                                                  s_epoch);
         }
     }
     // every warp's Tensor Memory reads and writes have completed (waited for)

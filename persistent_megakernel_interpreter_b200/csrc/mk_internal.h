@@ -89,6 +89,7 @@ struct SmemLayout {
     uint32_t tot;                             // down-projection running sums
     uint32_t red;                             // per-warp partial sums of a job input
     uint32_t cbar;                            // barrier of the compute warps
+    uint32_t sel;                             // [warps][kMaxBatch] LM-head best per warp (greedy)
     uint32_t tfull, tempty, tarmed;           // Tensor Memory slots: landed / released / fill held
     uint32_t tbase;                           // Tensor Memory address of the allocation
     uint32_t total;
@@ -111,6 +112,7 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.tot = o;       o += 4u * kMaxDownRows * kMaxBatch * 4u;
     m.red = o;       o += 4u * 32u;
     m.cbar = o;      o += 8u;
+    m.sel = o;       o += 8u * kConsumerWarps * kMaxBatch;
     o = (o + 7u) & ~7u;
     m.tfull = o;     o += 8u * kMaxTmemSlots;
     m.tempty = o;    o += 8u * kMaxTmemSlots;
@@ -148,6 +150,14 @@ struct Params {
     uint16_t* kc;
     uint16_t* vc;
     float* logits;
+    // greedy selection fused into the LM head (all NULL: off): the next token of
+    // sequence b goes to next_tokens[b], its position + 1 to next_positions[b], and
+    // the token also to gen_tokens[b] when that is set
+    int32_t* next_tokens;
+    int32_t* next_positions;
+    int32_t* gen_tokens;
+    uint32_t* sel_best;  // [B][n_lm_jobs][2] each LM-head job's best (value bits, index)
+    int n_lm_jobs;
     // scratch
     float* x;          // [B][H]   residual stream (fp32)
     float* q;          // [B][Q]

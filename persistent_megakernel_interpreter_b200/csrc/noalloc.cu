@@ -25,20 +25,29 @@ cudaError_t baseline_prepare(const Params& p);
 
 namespace {
 
-// The scratch of every no-allocation step on a device: 4 MiB (the 1B-shaped
-// model at batch 1 needs about 2.3 MiB at 8192 positions, mostly the RoPE table).
+// The scratch of every no-allocation step on a device: 4 MiB. Its layout does not
+// depend on the call's max_ctx: the control block (cleared by every call), then
+// the RoPE table in a fixed 2 MiB region -- cos [kRopeRows(d)][d/2], then sin, for
+// as many positions as the region holds at that head_dim (8192 at 64, 4096 at
+// 128) -- then the step's activations and attention partials.
 constexpr size_t kScratchBytes = 4u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kCtlBytes = 512;  // the control block first, cleared by every call
+constexpr size_t kCtlBytes = 512;
+constexpr size_t kRopeOff = kCtlBytes;
+constexpr size_t kRopeBytes = 2u << 20;
+constexpr size_t kActOff = kRopeOff + kRopeBytes;
+
+// Positions the RoPE region holds at head dim d (cos and sin, d/2 floats each).
+int rope_rows(int d) { return (int)(kRopeBytes / ((size_t)d * sizeof(float))); }
 
 struct DeviceState {
     unsigned char* base = nullptr;  // device address of g_noalloc_scratch
     int n_sm = 0;
-    // the RoPE table left in the array by the last call (rebuilt when these change)
+    // the RoPE table in the array (rebuilt when either changes)
     double theta = 0.0;
-    int head_dim = 0, rows = 0;
+    int head_dim = 0;
 };
 
 std::mutex g_mutex;
@@ -66,9 +75,9 @@ extern "C" mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const
 
     // the scratch plan; calls whose scratch exceeds the array are refused
     const int half = L.d / 2;
-    size_t off = kCtlBytes;
-    const size_t o_rope = off;
-    off = up256(off + (size_t)2 * max_ctx * half * sizeof(float));
+    const int rows = rope_rows(L.d);
+    if (max_ctx > rows) return MK_ERR_INVALID_ARG;
+    size_t off = kActOff;
     const size_t o_x = off;
     off = up256(off + (size_t)batch * L.H * sizeof(float));
     const size_t o_q = off;
@@ -96,16 +105,20 @@ extern "C" mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const
     }
     unsigned char* sb = ds.base;
 
-    // the RoPE table of positions 0..max_ctx-1 (angle pos * theta^(-2i/d) in double,
-    // cos and sin stored as float), uploaded in pieces from the stack when the
-    // configuration differs from the last call's
-    if (ds.theta != cfg->rope_theta || ds.head_dim != L.d || ds.rows != max_ctx) {
+    // the RoPE table of positions 0..rows-1 (angle pos * theta^(-2i/d) in double,
+    // cos and sin stored as float), uploaded in pieces from the stack when theta or
+    // the head dim differs from the table in the array. A capture cannot take the
+    // upload (its source is on the stack): refused while the stream captures.
+    float* cos_dst = reinterpret_cast<float*>(sb + kRopeOff);
+    float* sin_dst = cos_dst + (size_t)rows * half;
+    if (ds.theta != cfg->rope_theta || ds.head_dim != L.d) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MK_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return MK_ERR_INVALID_ARG;
         constexpr int kChunk = 2048;
         float buf[kChunk];
-        float* cos_dst = reinterpret_cast<float*>(sb + o_rope);
-        float* sin_dst = cos_dst + (size_t)max_ctx * half;
         for (int table = 0; table < 2; ++table) {
-            const size_t total = (size_t)max_ctx * half;
+            const size_t total = (size_t)rows * half;
             for (size_t e0 = 0; e0 < total; e0 += kChunk) {
                 const size_t n = total - e0 < (size_t)kChunk ? total - e0 : (size_t)kChunk;
                 for (size_t k = 0; k < n; ++k) {
@@ -122,7 +135,6 @@ extern "C" mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const
         }
         ds.theta = cfg->rope_theta;
         ds.head_dim = L.d;
-        ds.rows = max_ctx;
     }
     // the control block must start at zero (the step's error word)
     if (cudaMemsetAsync(sb, 0, kCtlBytes, st) != cudaSuccess) return MK_ERR_CUDA;
@@ -137,8 +149,8 @@ extern "C" mk_status mk_baseline_decode_step_noalloc(const mk_config* cfg, const
     p.rel_qkv = L.rel_qkv; p.rel_o = L.rel_o; p.rel_gu = L.rel_gu; p.rel_down = L.rel_down;
     p.off_norms = L.off_norms;
     p.tile_h = L.tile_h; p.tile_o = L.tile_o; p.tile_f = L.tile_f;
-    p.rope_cos = reinterpret_cast<const float*>(sb + o_rope);
-    p.rope_sin = p.rope_cos + (size_t)max_ctx * half;
+    p.rope_cos = cos_dst;
+    p.rope_sin = sin_dst;
     p.tokens = tokens;
     p.positions = positions;
     p.kc = static_cast<uint16_t*>(k_cache);

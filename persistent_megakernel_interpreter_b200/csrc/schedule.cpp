@@ -299,8 +299,10 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         return in;
                     });
     }
+    uint32_t lm_ord = 0;  // LM-head instructions, numbered in SM order (greedy selection slots)
     emit_ranges(share(L.V / 4, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
         mk_instr in = mk_in(MK_OP_LMHEAD, L.L - 1);
+        in.aux0 = lm_ord++;
         in.first = (uint32_t)a;
         in.count = in.nfill = (uint32_t)n;
         in.wait_ctr = (uint32_t)c_down[L.L - 1];

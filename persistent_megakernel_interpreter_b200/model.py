@@ -91,6 +91,22 @@ class Megakernel:
         """One step of the persistent megakernel, asynchronous on ``stream``."""
         self._step(_lib.lib().mk_decode_step, tokens, positions, k_cache, v_cache, logits, stream)
 
+    def decode_steps_greedy(self, tokens, positions, k_cache, v_cache, logits, n_steps: int,
+                            generated=None, stream=None) -> None:
+        """``n_steps`` greedy steps back to back (the choice fused into each step's LM
+        head): tokens and positions are overwritten with the next ones after every
+        step; ``generated`` (int32 [n_steps][batch], optional) receives the tokens."""
+        for t, dt in ((tokens, torch.int32), (positions, torch.int32), (logits, torch.float32)):
+            assert t.is_cuda and t.dtype == dt and t.is_contiguous()
+        assert k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16
+        if generated is not None:
+            assert generated.is_cuda and generated.dtype == torch.int32 and generated.is_contiguous()
+            assert generated.numel() >= n_steps * tokens.numel()
+        _lib.check(_lib.lib().mk_decode_steps_greedy(
+            self._h, _ptr(tokens), _ptr(positions), _ptr(k_cache), _ptr(v_cache), _ptr(logits),
+            _ptr(generated) if generated is not None else None, int(n_steps), _stream(stream)),
+            "mk_decode_steps_greedy")
+
     def baseline_decode_step(self, tokens, positions, k_cache, v_cache, logits, stream=None) -> None:
         """The same step as one kernel per op and layer."""
         self._step(_lib.lib().mk_baseline_decode_step, tokens, positions, k_cache, v_cache, logits,

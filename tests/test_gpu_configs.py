@@ -14,7 +14,7 @@ import pytest
 from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B
 from persistent_megakernel_interpreter_b200.inputs import make_tokens, make_weights
 
-from test_gpu_parity import TOL, Case, _bits, assert_kv_ok, assert_logits_close
+from test_gpu_parity import REG, TOL, Case, _bits, assert_kv_ok, assert_logits_close, bf16_ulp, reg_bar
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +36,7 @@ def test_llama1b_long_contexts(w1b):
         gpu = c.gpu_step(toks, pos)
         assert c.mk.status()[0] == 0
         ref, kc, vc = c.oracle_step(toks, pos)
-        assert_logits_close(gpu, ref)
+        assert_logits_close(gpu, ref, pos)
         assert_kv_ok(c, kc, vc, pos)
     c.mk.close()
 
@@ -56,18 +56,25 @@ def test_llama1b_greedy_256_after_32_token_prompt(w1b):
     for p in range(steps):
         gpu = c.gpu_step([tok], [p])
         ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
-        assert np.max(np.abs(gpu[0] - ref[0])) <= TOL * np.max(np.abs(ref[0])), p
+        err = np.max(np.abs(gpu[0] - ref[0])) / np.max(np.abs(ref[0]))
+        # the two caches grow apart by bf16 roundings of slightly different values,
+        # so the regression bar's floor is ten times the single-step one
+        assert err <= TOL and err <= reg_bar(p, 10 * REG), (p, err)
         agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
         tok = int(prompt[p + 1]) if p + 1 < n_prompt else int(np.argmax(gpu[0]))
     assert agree >= 0.99 * steps
     assert c.mk.status()[0] == 0
-    # the cache each side built holds the same keys and values (bf16, within the bound)
+    # the cache each side built holds the same keys and values, each within two bf16
+    # ulps at the scale of its head row (one rounding each side, of inputs that
+    # differ by earlier roundings)
     kg, vg = _bits(c.kd), _bits(c.vd)
     import oracle
     for got, ref in ((kg, kc), (vg, vc)):
         g = oracle.bf16_to_f32(got).astype(np.float64)
         r = oracle.bf16_to_f32(ref).astype(np.float64)
         assert np.max(np.abs(g - r)) <= TOL * np.max(np.abs(r))
+        scale = bf16_ulp(np.max(np.abs(r), axis=-1, keepdims=True))
+        assert np.all(np.abs(g - r) <= 2 * scale), np.max(np.abs(g - r) / scale)
     c.mk.close()
 
 
@@ -81,7 +88,7 @@ def test_3b_shape_batch8_full_depth():
     gpu = c.gpu_step(toks, past)
     assert c.mk.status()[0] == 0
     ref, kc, vc = c.oracle_step(toks, past)
-    assert_logits_close(gpu, ref)
+    assert_logits_close(gpu, ref, past)
     assert_kv_ok(c, kc, vc, past)
     c.reset_kv()
     assert np.array_equal(c.gpu_step(toks, past, baseline=True), gpu)

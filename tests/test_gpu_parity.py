@@ -2,8 +2,19 @@
 the integer/protocol properties that must hold bit for bit.
 
 Tolerance (stated in the decode-step target): max |logit_gpu - logit_oracle|
-<= 1e-2 * max |logit_oracle| per step, and greedy argmax agreement. Integer work
-is exact: untouched KV slots, counters, token ids."""
+<= 1e-2 * max |logit_oracle| per step, and greedy argmax agreement. A second,
+tighter bar catches regressions the pass line would let through (one wrong head,
+a dropped residual row): 1e-4 * max |logit_oracle| for a sequence with many keys
+(fp32 arithmetic in two summation orders; measured about 2e-5 on the 1B step at
+128 positions). A sequence with few keys gets 2^-7 / (position + 1) instead when
+that is larger: the step's own key and value are rounded to bf16 on each side,
+and where the fp32 values sit near a rounding boundary the two roundings differ by
+one ulp (2^-8 relative); that key weighs up to 1 / (position + 1) in the softmax
+(measured: 6e-4 with 2 keys on the 3B-style shape). The new key and value
+themselves are within one bf16 ulp at the scale of their head (the largest
+magnitude of the head's row): RoPE's a*c - b*s and the value's dot product can
+cancel, so a small element's own ulp is no bound. Integer work is exact:
+untouched KV slots, counters, token ids."""
 import dataclasses
 
 import numpy as np
@@ -16,7 +27,8 @@ from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_to
 
 pytestmark = pytest.mark.gpu
 
-TOL = 1e-2
+TOL = 1e-2   # pass line
+REG = 1e-4   # regression bar
 
 
 def _bits(t):
@@ -58,11 +70,26 @@ class Case:
         return self.orc.decode_step(np.asarray(tokens), np.asarray(positions), kc, vc), kc, vc
 
 
-def assert_logits_close(gpu, ref):
+def reg_bar(position, floor=REG):
+    """The regression bar of a sequence decoding at `position` (see the module notes)."""
+    return max(floor, 2.0 ** -7 / (int(position) + 1))
+
+
+def assert_logits_close(gpu, ref, positions=None, floor=REG):
     for b in range(ref.shape[0]):
         err = np.max(np.abs(gpu[b] - ref[b]))
-        assert err <= TOL * np.max(np.abs(ref[b])), (b, err, np.max(np.abs(ref[b])))
+        top = np.max(np.abs(ref[b]))
+        assert err <= TOL * top, (b, err, top)
+        bar = reg_bar(positions[b], floor) if positions is not None else floor
+        assert err <= bar * top, ("regression bar", b, err / top, bar)
         assert int(np.argmax(gpu[b])) == int(np.argmax(ref[b]))
+
+
+def bf16_ulp(x):
+    """The spacing of bf16 values at |x| (8 significant bits); the smallest normal's
+    at 0."""
+    a = np.maximum(np.abs(x), np.float64(2.0 ** -126))
+    return np.exp2(np.floor(np.log2(a)) - 7)
 
 
 def assert_kv_ok(case, kc_ref, vc_ref, positions):
@@ -75,9 +102,10 @@ def assert_kv_ok(case, kc_ref, vc_ref, positions):
         assert np.array_equal(kg[:, b][:, :, mask], k0[:, b][:, :, mask])
         assert np.array_equal(vg[:, b][:, :, mask], v0[:, b][:, :, mask])
         for got, ref in ((kg, kc_ref), (vg, vc_ref)):
-            g = oracle.bf16_to_f32(got[:, b, :, p]).astype(np.float64)
+            g = oracle.bf16_to_f32(got[:, b, :, p]).astype(np.float64)  # [layer][kv head][dim]
             r = oracle.bf16_to_f32(ref[:, b, :, p]).astype(np.float64)
-            assert np.max(np.abs(g - r)) <= TOL * np.max(np.abs(r))
+            scale = bf16_ulp(np.max(np.abs(r), axis=-1, keepdims=True))  # one ulp at the head's scale
+            assert np.all(np.abs(g - r) <= scale), np.max(np.abs(g - r) / scale)
 
 
 @pytest.fixture(scope="module")
@@ -101,7 +129,7 @@ def test_tiny_step_matches_oracle(tiny):
     code, msg = tiny.mk.status()
     assert code == 0, msg
     ref, kc, vc = tiny.oracle_step(toks, pos)
-    assert_logits_close(gpu, ref)
+    assert_logits_close(gpu, ref, pos)
     assert_kv_ok(tiny, kc, vc, pos)
 
 
@@ -153,7 +181,7 @@ def test_split_k_partitions_agree_with_oracle(tiny):
     for pk in (kps, 2 * kps, 160 // kps * kps + kps):
         tiny.mk.build_schedule(2, 160, part_keys=pk)
         tiny.reset_kv()
-        assert_logits_close(tiny.gpu_step(toks, pos), ref)
+        assert_logits_close(tiny.gpu_step(toks, pos), ref, pos)
     tiny.mk.build_schedule(2, 160)
 
 
@@ -182,7 +210,7 @@ def test_bad_token_and_position_are_reported_and_write_nothing(tiny):
     tiny.reset_kv()
     toks, pos = make_tokens(TINY, 2, seed=8).numpy(), [128, 57]
     ref, _, _ = tiny.oracle_step(toks, pos)
-    assert_logits_close(tiny.gpu_step(toks, pos), ref)
+    assert_logits_close(tiny.gpu_step(toks, pos), ref, pos)
     assert tiny.mk.status()[0] == 0
 
 
@@ -199,7 +227,7 @@ def test_wait_timeout_is_reported_without_hanging(tiny):
     tiny.reset_kv()
     toks, pos = make_tokens(TINY, 2, seed=9).numpy(), [128, 57]
     ref, _, _ = tiny.oracle_step(toks, pos)
-    assert_logits_close(tiny.gpu_step(toks, pos), ref)
+    assert_logits_close(tiny.gpu_step(toks, pos), ref, pos)
     assert tiny.mk.status()[0] == 0
 
 
@@ -215,7 +243,8 @@ def test_tiny_greedy_decode_teacher_forced():
     for p in range(56):
         gpu = c.gpu_step([tok], [p])
         ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
-        assert np.max(np.abs(gpu[0] - ref[0])) <= TOL * np.max(np.abs(ref[0]))
+        err = np.max(np.abs(gpu[0] - ref[0])) / np.max(np.abs(ref[0]))
+        assert err <= TOL and err <= reg_bar(p, 10 * REG), (p, err)  # the caches grow apart by roundings
         agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
         tok = int(prompt[p + 1]) if p + 1 < 32 else int(np.argmax(gpu[0]))
     assert agree >= 0.99 * 56
@@ -228,7 +257,7 @@ def test_tiny_with_non_unit_norm_weights():
     c.mk.build_schedule(1, 140)
     toks, pos = make_tokens(TINY, 1, seed=22).numpy(), [130]
     ref, kc, vc = c.oracle_step(toks, pos)
-    assert_logits_close(c.gpu_step(toks, pos), ref)
+    assert_logits_close(c.gpu_step(toks, pos), ref, pos)
     assert_kv_ok(c, kc, vc, pos)
     c.mk.close()
 
@@ -244,7 +273,7 @@ def test_3b_shape_batch8_two_layers():
     ref, kc, vc = c.oracle_step(toks, past)
     gpu = c.gpu_step(toks, past)
     assert c.mk.status()[0] == 0
-    assert_logits_close(gpu, ref)
+    assert_logits_close(gpu, ref, past)
     assert_kv_ok(c, kc, vc, past)
     assert np.array_equal(c.gpu_step(toks, past, baseline=True), gpu)
     c.mk.close()
@@ -270,7 +299,7 @@ def test_llama1b_step_matches_oracle(llama1b):
     gpu = llama1b.gpu_step(toks, pos)
     assert llama1b.mk.status()[0] == 0
     ref, kc, vc = llama1b.oracle_step(toks, pos)
-    assert_logits_close(gpu, ref)
+    assert_logits_close(gpu, ref, pos)
     assert_kv_ok(llama1b, kc, vc, pos)
 
 

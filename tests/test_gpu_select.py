@@ -93,3 +93,67 @@ def test_decode_loop_selects_on_the_device():
                 top2 = np.sort(ref[b])[-2:]
                 assert top2[1] - top2[0] <= 2 * TOL * scale, (p, b)
     c.mk.close()
+
+
+@pytest.mark.parametrize("batch", [1, 3])
+def test_fused_greedy_steps_equal_select_between_steps(batch):
+    """mk_decode_steps_greedy (the choice fused into each step's LM head, N launches
+    with no host work) against mk_decode_step + mk_greedy_select per step on a
+    copy of the same caches: the same tokens at every step, the same positions,
+    the last step's logits bit for bit, and identical caches. Batch 3 runs the
+    batched kernel (its LM-head rows shared by two warps per tile)."""
+    n = 24
+    c = Case(TINY, batch=batch, max_seq=64, past=0, seed=5)
+    c.mk.build_schedule(batch, 64)
+    k2, v2 = c.kd.clone(), c.vd.clone()
+    t0 = torch.as_tensor(make_tokens(TINY, batch, seed=6).numpy(), dtype=torch.int32).cuda()
+    # the fused loop
+    tok_f, pos_f = t0.clone(), torch.zeros(batch, dtype=torch.int32, device="cuda")
+    gen = torch.full((n, batch), -1, dtype=torch.int32, device="cuda")
+    logits_f = torch.empty(batch, TINY.vocab, dtype=torch.float32, device="cuda")
+    c.mk.decode_steps_greedy(tok_f, pos_f, c.kd, c.vd, logits_f, n, generated=gen)
+    torch.cuda.synchronize()
+    assert c.mk.status()[0] == 0
+    # the step-by-step loop with the separate selection kernel
+    tok_s, pos_s = t0.clone(), torch.zeros(batch, dtype=torch.int32, device="cuda")
+    logits_s = torch.empty(batch, TINY.vocab, dtype=torch.float32, device="cuda")
+    seq = []
+    for _ in range(n):
+        c.mk.decode_step(tok_s, pos_s, k2, v2, logits_s)
+        greedy_select(logits_s, tok_s, pos_s)
+        seq.append(tok_s.clone())
+    torch.cuda.synchronize()
+    assert np.array_equal(gen.cpu().numpy(), torch.stack(seq).cpu().numpy())
+    assert np.array_equal(tok_f.cpu().numpy(), tok_s.cpu().numpy())
+    assert np.array_equal(pos_f.cpu().numpy(), np.full(batch, n))
+    assert np.array_equal(logits_f.cpu().numpy(), logits_s.cpu().numpy())
+    assert np.array_equal(_bits(c.kd), _bits(k2)) and np.array_equal(_bits(c.vd), _bits(v2))
+    c.mk.close()
+
+
+def test_fused_greedy_steps_1b():
+    """The same equality on the Llama-3.2-1B shape for 6 steps from 128 cached
+    positions (the LM head spread over every SM)."""
+    from persistent_megakernel_interpreter_b200.config import LLAMA_1B
+    n = 6
+    c = Case(LLAMA_1B, batch=1, max_seq=136, past=128, seed=0)
+    c.mk.build_schedule(1, 136)
+    k2, v2 = c.kd.clone(), c.vd.clone()
+    t0 = torch.as_tensor(make_tokens(LLAMA_1B, 1, seed=2).numpy(), dtype=torch.int32).cuda()
+    tok_f, pos_f = t0.clone(), torch.full((1,), 128, dtype=torch.int32, device="cuda")
+    gen = torch.full((n, 1), -1, dtype=torch.int32, device="cuda")
+    logits_f = torch.empty(1, LLAMA_1B.vocab, dtype=torch.float32, device="cuda")
+    c.mk.decode_steps_greedy(tok_f, pos_f, c.kd, c.vd, logits_f, n, generated=gen)
+    tok_s, pos_s = t0.clone(), torch.full((1,), 128, dtype=torch.int32, device="cuda")
+    logits_s = torch.empty(1, LLAMA_1B.vocab, dtype=torch.float32, device="cuda")
+    seq = []
+    for _ in range(n):
+        c.mk.decode_step(tok_s, pos_s, k2, v2, logits_s)
+        greedy_select(logits_s, tok_s, pos_s)
+        seq.append(tok_s.clone())
+    torch.cuda.synchronize()
+    assert c.mk.status()[0] == 0
+    assert np.array_equal(gen.cpu().numpy(), torch.stack(seq).cpu().numpy())
+    assert int(pos_f.item()) == 128 + n
+    assert np.array_equal(logits_f.cpu().numpy(), logits_s.cpu().numpy())
+    c.mk.close()
