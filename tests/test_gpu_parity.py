@@ -92,6 +92,37 @@ def bf16_ulp(x):
     return np.exp2(np.floor(np.log2(a)) - 7)
 
 
+def assert_slot_close(kg, vg, kc_ref, vc_ref, b, p):
+    """Slot p of sequence b (bf16 bits, [layer][seq][kv head][slot][dim]) within one
+    bf16 ulp of the oracle's at the scale of each head row."""
+    for got, ref in ((kg, kc_ref), (vg, vc_ref)):
+        g = oracle.bf16_to_f32(got[:, b, :, p]).astype(np.float64)  # [layer][kv head][dim]
+        r = oracle.bf16_to_f32(ref[:, b, :, p]).astype(np.float64)
+        scale = bf16_ulp(np.max(np.abs(r), axis=-1, keepdims=True))
+        assert np.all(np.abs(g - r) <= scale), np.max(np.abs(g - r) / scale)
+
+
+def greedy_teacher_forced(c, prompt, steps):
+    """Greedy decoding at batch 1 from an empty cache: the prompt's tokens, then the
+    GPU's argmax. Every step the oracle decodes the GPU's token from the GPU's own
+    cache as it stood before the step (teacher forcing on tokens and cache), so the
+    two differ only by the step's arithmetic: the logits are held to the single-step
+    bars and the written slot to one ulp at its head's scale. Returns the number of
+    steps whose argmaxes agree."""
+    tok, agree = int(prompt[0]), 0
+    for p in range(steps):
+        kc, vc = _bits(c.kd), _bits(c.vd)
+        gpu = c.gpu_step([tok], [p])
+        ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
+        err = np.max(np.abs(gpu[0] - ref[0])) / np.max(np.abs(ref[0]))
+        assert err <= TOL and err <= reg_bar(p), (p, err)
+        assert_slot_close(_bits(c.kd), _bits(c.vd), kc, vc, 0, p)
+        agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
+        tok = int(prompt[p + 1]) if p + 1 < len(prompt) else int(np.argmax(gpu[0]))
+    assert c.mk.status()[0] == 0
+    return agree
+
+
 def assert_kv_ok(case, kc_ref, vc_ref, positions):
     """New slots close to the oracle's; every other slot bit-identical to before."""
     kg, vg = _bits(case.kd), _bits(case.vd)
@@ -101,11 +132,7 @@ def assert_kv_ok(case, kc_ref, vc_ref, positions):
         mask[p] = False
         assert np.array_equal(kg[:, b][:, :, mask], k0[:, b][:, :, mask])
         assert np.array_equal(vg[:, b][:, :, mask], v0[:, b][:, :, mask])
-        for got, ref in ((kg, kc_ref), (vg, vc_ref)):
-            g = oracle.bf16_to_f32(got[:, b, :, p]).astype(np.float64)  # [layer][kv head][dim]
-            r = oracle.bf16_to_f32(ref[:, b, :, p]).astype(np.float64)
-            scale = bf16_ulp(np.max(np.abs(r), axis=-1, keepdims=True))  # one ulp at the head's scale
-            assert np.all(np.abs(g - r) <= scale), np.max(np.abs(g - r) / scale)
+        assert_slot_close(kg, vg, kc_ref, vc_ref, b, p)
 
 
 @pytest.fixture(scope="module")
@@ -232,23 +259,12 @@ def test_wait_timeout_is_reported_without_hanging(tiny):
 
 
 def test_tiny_greedy_decode_teacher_forced():
-    """32-token prompt from an empty cache, then greedy decoding; the oracle is fed
-    the GPU's tokens (teacher forcing) and must agree on every step's argmax."""
+    """32-token prompt from an empty cache, then greedy decoding (greedy_teacher_forced);
+    the argmax agrees on every step."""
     c = Case(TINY, batch=1, max_seq=64, past=0, seed=11)
     c.mk.build_schedule(1, 64)
-    kc, vc = _bits(c.k), _bits(c.v)
     prompt = make_tokens(TINY, 32, seed=12).numpy()
-    tok = int(prompt[0])
-    agree = 0
-    for p in range(56):
-        gpu = c.gpu_step([tok], [p])
-        ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
-        err = np.max(np.abs(gpu[0] - ref[0])) / np.max(np.abs(ref[0]))
-        assert err <= TOL and err <= reg_bar(p, 10 * REG), (p, err)  # the caches grow apart by roundings
-        agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
-        tok = int(prompt[p + 1]) if p + 1 < 32 else int(np.argmax(gpu[0]))
-    assert agree >= 0.99 * 56
-    assert c.mk.status()[0] == 0
+    assert greedy_teacher_forced(c, prompt, 56) >= 0.99 * 56
     c.mk.close()
 
 
