@@ -10,7 +10,10 @@ a dropped residual row): 1e-4 * max |logit_oracle| for a sequence with many keys
 that is larger: the step's own key and value are rounded to bf16 on each side,
 and where the fp32 values sit near a rounding boundary the two roundings differ by
 one ulp (2^-8 relative); that key weighs up to 1 / (position + 1) in the softmax
-(measured: 6e-4 with 2 keys on the 3B-style shape). The new key and value
+(measured: 6e-4 with 2 keys on the 3B-style shape). Greedy decoding from an
+empty cache attends over the model's own keys, where that weight can reach 1: each
+step is held to 2^-8 there and the median step to 1e-4 (measured: 1.5e-4 at 99
+keys on the 1B shape). The new key and value
 themselves are within one bf16 ulp at the scale of their head (the largest
 magnitude of the head's row): RoPE's a*c - b*s and the value's dot product can
 cancel, so a small element's own ulp is no bound. Integer work is exact:
@@ -107,19 +110,27 @@ def greedy_teacher_forced(c, prompt, steps):
     GPU's argmax. Every step the oracle decodes the GPU's token from the GPU's own
     cache as it stood before the step (teacher forcing on tokens and cache), so the
     two differ only by the step's arithmetic: the logits are held to the single-step
-    bars and the written slot to one ulp at its head's scale. Returns the number of
-    steps whose argmaxes agree."""
-    tok, agree = int(prompt[0]), 0
+    bars, with one difference: the cache here is the model's own, whose attention
+    can rest on a few keys, so the step's own key and value (rounded to bf16 on
+    each side, one ulp apart where the fp32 value sits near a rounding boundary)
+    can carry up to all of a head's softmax weight. A step is held to one bf16 ulp
+    (2^-8) relative, and the median step to the regression bar. The written slot is
+    within one ulp at its head's scale. Returns the number of steps whose argmaxes
+    agree."""
+    tok, agree, errs = int(prompt[0]), 0, []
     for p in range(steps):
         kc, vc = _bits(c.kd), _bits(c.vd)
         gpu = c.gpu_step([tok], [p])
         ref, kc, vc = c.oracle_step([tok], [p], kc, vc)
         err = np.max(np.abs(gpu[0] - ref[0])) / np.max(np.abs(ref[0]))
-        assert err <= TOL and err <= reg_bar(p), (p, err)
+        errs.append(err)
+        assert err <= TOL and err <= 2.0 ** -8, (p, err)
         assert_slot_close(_bits(c.kd), _bits(c.vd), kc, vc, 0, p)
         agree += int(np.argmax(gpu[0]) == np.argmax(ref[0]))
         tok = int(prompt[p + 1]) if p + 1 < len(prompt) else int(np.argmax(gpu[0]))
     assert c.mk.status()[0] == 0
+    print(f"greedy: max relative error {max(errs):.3g}, median {np.median(errs):.3g} over {steps} steps")
+    assert np.median(errs) <= REG, np.median(errs)
     return agree
 
 
