@@ -45,9 +45,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(default_workload=True):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel source and this run times its workload, the default one
+    (else None)."""
+    if not default_workload:
+        return None
     try:
         text = open(PROFILE_FILE).read()
     except OSError:
@@ -323,7 +326,7 @@ def run_mk(args):
     k, v = make_kv_cache(cfg, BATCH, past + 1, past, seed=1)
     mk = Megakernel(cfg, w.to(dev), max_batch=BATCH, max_seq=past + 1)
     torch.cuda.empty_cache()
-    sched_opts = {}
+    sched_opts = {"proj": {"auto": 0, "cuda": 1, "tensor": 2}[args.proj]}
     if args.part_keys:
         sched_opts["part_keys"] = args.part_keys
     info = mk.build_schedule(BATCH, past + 1, **sched_opts)
@@ -441,7 +444,8 @@ def run_mk(args):
         peak, peak_kind = hbm_peak()
         per_launch_ms = statistics.mean(launch_ms)
         achieved = bytes_step / (per_launch_ms * 1e-3) / 1e9
-        traffic = profiled_traffic()
+        traffic = profiled_traffic(args.model == "1b" and BATCH == 1 and past == PAST and
+                                   cfg.n_layers == LLAMA_1B.n_layers)
         ms_per_step = t_max / args.steps
         metric = METRIC if (args.model == "1b" and BATCH == 1) else (
             f"µs/decode step & tokens/s, {'Llama-3B' if args.model == '3b' else 'Llama-1B'}-style bf16 "
@@ -471,7 +475,8 @@ def run_mk(args):
             "multikernel_baseline": base,
             "schedule": {"n_sm": info.n_sm, "instructions": info.n_instr,
                          "ring_stages": info.n_stages, "stage_bytes": info.stage_bytes,
-                         "attn_partitions": info.n_parts},
+                         "attn_partitions": info.n_parts,
+                         "projections": "tensor cores (tcgen05)" if info.proj == 2 else "CUDA cores"},
         }
         print(json.dumps(line), flush=True)
     mk.close()
@@ -611,6 +616,8 @@ def parse_args(argv=None):
                     help="decoder layers (16 = the Llama-3.2-1B workload; fewer only for "
                          "small profiling captures of the same kernels)")
     ap.add_argument("--past", type=int, default=PAST, help="cached positions before the step")
+    ap.add_argument("--proj", choices=["auto", "cuda", "tensor"], default="auto",
+                    help="projections at batch > 1: tensor cores (auto) or CUDA cores")
     ap.add_argument("--part-keys", type=int, default=0,
                     help="keys per attention partition (0 = the schedule builder's choice)")
     ap.add_argument("--greedy", type=int, default=0, metavar="N",

@@ -123,7 +123,21 @@ typedef struct mk_schedule_opts {
                                 step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
+    int32_t proj;            /* the projections' arithmetic at batch > 1: MK_PROJ_AUTO,
+                                MK_PROJ_CUDA_CORES or MK_PROJ_TENSOR_CORES (batch 1
+                                always runs on the CUDA cores) */
 } mk_schedule_opts;
+
+/* mk_schedule_opts.proj. Tensor cores: each instruction's weight rows stream as
+ * 64-column TMA boxes (128-byte swizzle) and one thread issues tcgen05.mma
+ * (M = 128 weight rows, N = 16: the batch's fp32 inputs split into bf16 high and
+ * low parts, K = 16 per instruction) into an fp32 accumulator in Tensor Memory,
+ * read back by the compute warps for the same fused epilogues. CUDA cores: each
+ * 4-row tile's batched fp32 dot product, as at batch 1. AUTO picks the tensor
+ * cores. The two differ only in the order and form of the fp32 accumulation. */
+#define MK_PROJ_AUTO 0
+#define MK_PROJ_CUDA_CORES 1
+#define MK_PROJ_TENSOR_CORES 2
 
 /* Build the per-SM instruction lists for `batch` sequences (1 <= batch <= max_batch)
  * whose steps use at most `max_ctx` keys (position + 1 <= max_ctx <= max_seq), and
@@ -139,7 +153,8 @@ typedef struct mk_schedule_opts {
  * each holding at most what the SM's weight ring holds at once (and 512 keys), so
  * max_ctx has a ceiling that depends on the shape and batch: 16384 keys for the
  * Llama-3.2-1B shape; for head_dim 128 with 24 query and 8 KV heads, 12288 at
- * batch 1-2 and 6144 at batch 3-8. A larger max_ctx
+ * batch 1, then on the tensor-core path 7680 at batch 2-5 and 6144 at 6-8 (on the
+ * CUDA-core path 12288 at batch 2, 6144 at 3-8). A larger max_ctx
  * (or a part_keys that needs more than 32 partitions) returns MK_ERR_INVALID_ARG. */
 mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts);
 
@@ -276,6 +291,8 @@ typedef struct mk_schedule_info {
     uint64_t bytes_per_step;    /* weight + KV bytes one step streams */
     uint64_t max_sm_bytes;      /* largest per-SM share of those bytes */
     uint64_t min_sm_bytes;
+    int32_t proj;               /* the projections' path: MK_PROJ_CUDA_CORES or _TENSOR_CORES */
+    int32_t reserved0;
 } mk_schedule_info;
 
 /* Plans a schedule on the host only (no device, no handle): writes up to

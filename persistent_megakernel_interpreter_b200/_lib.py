@@ -30,7 +30,7 @@ class MkWeights(ctypes.Structure):
 class MkScheduleOpts(ctypes.Structure):
     _fields_ = [("n_sm", I32), ("part_keys", I32), ("rowblocks_down", I32),
                 ("seed", ctypes.c_uint32), ("wait_timeout_ms", I32), ("test_drop_item", I32),
-                ("trace", I32)]
+                ("trace", I32), ("proj", I32)]
 
 
 class MkInstr(ctypes.Structure):
@@ -45,10 +45,11 @@ class MkScheduleInfo(ctypes.Structure):
                                    "keys_per_stage", "stage_bytes", "n_stages", "n_counters",
                                    "n_instr")] + [
         ("bytes_per_step", ctypes.c_uint64), ("max_sm_bytes", ctypes.c_uint64),
-        ("min_sm_bytes", ctypes.c_uint64)]
+        ("min_sm_bytes", ctypes.c_uint64), ("proj", I32), ("reserved0", I32)]
 
 
 OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD = 1, 2, 3, 4, 5, 6
+PROJ_AUTO, PROJ_CUDA_CORES, PROJ_TENSOR_CORES = 0, 1, 2
 NO_COUNTER = 0xFFFFFFFF
 
 STATUS = {0: "MK_OK", 1: "MK_ERR_INVALID_ARG", 2: "MK_ERR_CUDA", 3: "MK_ERR_UNSUPPORTED",

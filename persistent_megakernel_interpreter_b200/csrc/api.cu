@@ -1,4 +1,5 @@
 // The C ABI of libmk.so (declarations and contracts in include/mk.h).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdio.h>
@@ -43,6 +44,7 @@ struct mk_handle {
     mk::Layout lay{};
     uint8_t* packed = nullptr;
     float* rope = nullptr;          // cos table then sin table
+    void* d_tmaps = nullptr;        // tensor maps of the packed weights (tensor-core path)
     // scratch (sized by mk_build_schedule)
     void* scratch = nullptr;
     size_t scratch_bytes = 0;
@@ -218,6 +220,81 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
     return no_throw([&] { return create_impl(cfg, w, device, out); });
 }
 
+// Tensor maps of the packed weights for the tensor-core path, one per (matrix,
+// box height 4 << k rows), all boxes 64 bf16 columns wide with the 128-byte
+// swizzle that the MMA's shared-memory descriptors read. Built once per handle.
+//   QKV / O / gate-up: {K, rows, layer}; LM head (the embedding rows): {K, rows};
+//   down: {ffn/4, 4 rows, 4 chunks, hidden/4 row blocks, layer}, a box of
+//   {64, 4, 1, 1 << k, 1} (the row blocks' rows of one chunk).
+static mk_status make_tmaps(mk_handle* h) {
+    if (h->d_tmaps) return MK_OK;
+    typedef CUresult (*Encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        h->msg = "cuTensorMapEncodeTiled is not available";
+        return MK_ERR_UNSUPPORTED;
+    }
+    const Encode encode = reinterpret_cast<Encode>(fn);
+    const mk::Layout& L = h->lay;
+    std::vector<CUtensorMap> maps((size_t)mk::kTmKinds * mk::kBoxHeights);
+    memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+    const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
+    auto enc = [&](int kind, int hk, uint8_t* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                   const cuuint32_t* box) {
+        const CUresult r = encode(&maps[(size_t)kind * mk::kBoxHeights + hk], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                  (cuuint32_t)rank, base, dims, strides, box, unit, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        return r == CUDA_SUCCESS;
+    };
+    uint8_t* pk = h->packed;
+    const cuuint64_t ls = (cuuint64_t)L.layer_stride;
+    bool ok = true;
+    for (int hk = 0; hk < mk::kBoxHeights && ok; ++hk) {
+        const cuuint32_t rows = 4u << hk;
+        const cuuint32_t box3[3] = {mk::kBoxK, rows, 1};
+        {
+            const cuuint64_t dims[3] = {(cuuint64_t)L.H, (cuuint64_t)L.qkv_rows, (cuuint64_t)L.L};
+            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, ls};
+            ok = ok && enc(mk::kTmQKV, hk, pk + L.off_layer0 + L.rel_qkv, 3, dims, st, box3);
+        }
+        {
+            const cuuint64_t dims[3] = {(cuuint64_t)L.Q, (cuuint64_t)L.H, (cuuint64_t)L.L};
+            const cuuint64_t st[2] = {(cuuint64_t)L.Q * 2, ls};
+            ok = ok && enc(mk::kTmO, hk, pk + L.off_layer0 + L.rel_o, 3, dims, st, box3);
+        }
+        {
+            const cuuint64_t dims[3] = {(cuuint64_t)L.H, (cuuint64_t)(2 * L.F), (cuuint64_t)L.L};
+            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, ls};
+            ok = ok && enc(mk::kTmGU, hk, pk + L.off_layer0 + L.rel_gu, 3, dims, st, box3);
+        }
+        {
+            const cuuint64_t dims[2] = {(cuuint64_t)L.H, (cuuint64_t)L.V};
+            const cuuint64_t st[1] = {(cuuint64_t)L.H * 2};
+            const cuuint32_t box2[2] = {mk::kBoxK, rows};
+            ok = ok && enc(mk::kTmLM, hk, pk + L.off_embed, 2, dims, st, box2);
+        }
+        if (hk < 5) {  // down: at most 16 row blocks (64 rows) per instruction
+            const cuuint64_t f4 = (cuuint64_t)(L.F / 4);
+            const cuuint64_t dims[5] = {f4, 4, 4, (cuuint64_t)(L.H / 4), (cuuint64_t)L.L};
+            const cuuint64_t st[4] = {f4 * 2, f4 * 2 * 4, f4 * 2 * 16, ls};
+            const cuuint32_t box5[5] = {mk::kBoxK, 4, 1, 1u << hk, 1};
+            ok = ok && enc(mk::kTmDown, hk, pk + L.off_layer0 + L.rel_down, 5, dims, st, box5);
+        }
+    }
+    if (!ok) {
+        h->msg = "cuTensorMapEncodeTiled refused a weight tensor map";
+        return MK_ERR_UNSUPPORTED;
+    }
+    MK_CUDA(h, cudaMalloc(&h->d_tmaps, maps.size() * sizeof(CUtensorMap)));
+    MK_CUDA(h, cudaMemcpy(h->d_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    return MK_OK;
+}
+
 static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts) {
     if (!h) return MK_ERR_INVALID_ARG;
     const mk_config& c = h->cfg;
@@ -231,7 +308,12 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     mk::Plan P;
     mk_status st = mk::plan_schedule(L, batch, max_ctx, n_sm, opts, 0, &P);
     if (st != MK_OK) return st;
+    const bool mma = P.info.proj == MK_PROJ_TENSOR_CORES;
     MK_CUDA(h, cudaDeviceSynchronize());
+    if (mma) {
+        st = make_tmaps(h);
+        if (st != MK_OK) return st;
+    }
     free_schedule(h);
 
     // scratch: activations, attention partials, counters, control block
@@ -317,21 +399,35 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     // quarter (32 lanes of stage_bytes / 32 bytes each); as many as 512 columns hold
     // per quarter, four quarters
     p.tslot_cols = (uint32_t)I.stage_bytes / 128u;
-    {
+    if (mma) {
+        // Tensor Memory holds the MMA accumulators instead of weight tiles
+        p.mma = MK_PROJ_TENSOR_CORES;
+        p.tmaps = h->d_tmaps;
+        p.n_tslots = 0;
+    } else {
         int per_q = p.tslot_cols ? (int)(mk::kTmemCols / p.tslot_cols) : 0;
         if (per_q > mk::kMaxTmemSlots / 4) per_q = mk::kMaxTmemSlots / 4;
         p.n_tslots = 4 * per_q;
-    }
-    if (p.n_tslots < 4 || I.stage_bytes % 128 != 0) {
-        h->msg = "a weight tile does not fit the SM's Tensor Memory";
-        free_schedule(h);
-        return MK_ERR_UNSUPPORTED;
+        if (p.n_tslots < 4 || I.stage_bytes % 128 != 0) {
+            h->msg = "a weight tile does not fit the SM's Tensor Memory";
+            free_schedule(h);
+            return MK_ERR_UNSUPPORTED;
+        }
     }
     {
-        const mk::SlotPlan sp = mk::slot_plan(L, batch, (uint32_t)I.stage_bytes);
+        const mk::SlotPlan sp = mk::slot_plan(L, batch, (uint32_t)I.stage_bytes, mma);
         p.xs_slots = sp.xs_slots;
         p.xs_slot_bytes = sp.slot_bytes;
         p.xs_vec_floats = sp.vec_floats;
+        p.xs_aux_floats = sp.aux_floats;
+        // an MMA reads 128 rows from each box's start, rows past the segment's own
+        // (never used) included: the shared memory after the ring must cover them
+        const mk::SmemLayout m = mk::smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, mma);
+        if (mma && m.total < m.ring + (uint32_t)p.n_stages * p.stage_bytes + mk::kMmaRows * 128u) {
+            h->msg = "shared memory too small for the tensor-core path";
+            free_schedule(h);
+            return MK_ERR_UNSUPPORTED;
+        }
     }
     p.n_counters = I.n_counters;
     if (opts && opts->trace) {
@@ -550,6 +646,7 @@ extern "C" void mk_destroy(mk_handle* h) {
         free_schedule(h);
         cudaFree(h->packed);
         cudaFree(h->rope);
+        cudaFree(h->d_tmaps);
     }
     delete h;
 }

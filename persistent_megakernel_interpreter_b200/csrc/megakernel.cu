@@ -158,6 +158,54 @@ struct Tmem {
     }
 };
 
+// ------------------------------------------------------------------ tensor-core MMA (batch > 1)
+//
+// On the tensor-core path Tensor Memory holds fp32 accumulators instead of weight
+// tiles: accumulator a is columns a * 16 .. +15 of all 128 lanes, lane m the
+// segment's row m, column n the input row n (sequence n's high bf16 part for
+// n < 8, sequence n - 8's low part above).
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
+// (8-row atoms of 128-byte rows, atoms 1024 bytes apart): start address >> 4
+// (bits 0-13), leading offset 1 (unused by this layout, bits 16-29), stride
+// 1024 >> 4 between atoms (bits 32-45), descriptor version 1 (bits 46-47),
+// layout 2 = 128-byte swizzle (bits 61-63). K advances by 16 elements inside an
+// atom by adding 32 bytes to the start address.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
+// bf16 (bits 7-9 and 10-12 = 1), both K-major, N = 16 (bits 17-22 = N / 8),
+// M = 128 (bits 24-28 = M / 16).
+constexpr uint32_t kMmaIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((kMmaRows >> 4) << 24);
+
+// D[tmem] (+)= A * B^T for one K = 16 step, issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kMmaIdesc), "r"(accumulate)
+        : "memory");
+}
+// One arrival on `bar` once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// The slot barriers complete one phase per matvec job in the slot (attention jobs,
+// which use slots too, pass them by): the issuer and the compute warps each keep
+// the slots' phase bits as they walk the same job sequence.
+struct MmaBars {
+    uint64_t* opnd;    // [NS] each compute warp arrives once the job's operand is written
+    uint64_t* mdone;   // [NS] the issuer's commit: the job's MMAs are done with its slot
+    uint64_t* afull;   // [kMaxAcc] the issuer's commit: a segment's accumulator is final
+    uint64_t* aempty;  // [kMaxAcc] each compute warp arrives once it has read it out
+    uint64_t* fin;     // the issuer's last commit
+};
+
 struct Slots {
     uint8_t* base;
     uint64_t* full;    // the job's preparer (activation or stage warp) arrives when its input is ready
@@ -353,9 +401,10 @@ __device__ __forceinline__ bool tag_backoff(const Params& p, uint32_t it, uint64
 // thread's pairs, all loads in flight at once, retried until every tag is the
 // expected one); RMSNorm with the bf16 norm weights w when w is given. Ends
 // with a compute barrier. Out of line: one copy for every job that needs it.
+template <bool MMAOP = false>
 __device__ __noinline__ bool block_input_tagged(const Params& p, const uint64_t* src, uint32_t tag, const uint16_t* w, int n,
                                    float* xs, float* red, int t, int warp, int lane, uint64_t* cbar,
-                                   uint32_t& cuses) {
+                                   uint32_t& cuses, int orow = 0) {
     const int np = n / 2;
     uint32_t wv[kMaxPairs];
     float v0[kMaxPairs], v1[kMaxPairs];
@@ -385,7 +434,7 @@ __device__ __noinline__ bool block_input_tagged(const Params& p, const uint64_t*
         if (!tag_backoff(p, it, t0, 1, lane)) return false;
     }
     auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
-    return block_store_input(v0, v1, wv, w != nullptr, p.eps, n, xs, red, t, warp, lane, bar);
+    return block_store_input<MMAOP>(v0, v1, wv, w != nullptr, p.eps, n, xs, red, t, warp, lane, bar, orow);
 }
 
 // `rows` (<= kMaxResidRows) consecutive tagged words into dst, by the threads
@@ -406,22 +455,24 @@ __device__ bool rows_tagged(const Params& p, const uint64_t* src, uint32_t tag, 
 
 // Where a job's residual rows sit in its slot (per sequence, kMaxResidRows).
 __device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) {
-    return sv + (size_t)p.B * p.xs_vec_floats + (size_t)p.B * (p.d + 4) + (size_t)b * kMaxResidRows;
+    return sv + (size_t)p.xs_aux_floats + (size_t)p.B * (p.d + 4) + (size_t)b * kMaxResidRows;
 }
 
 // The input of a matvec job, built by the compute warps (they poll the tagged
 // words themselves): RMSNorm of x (tagged) or of the embedding row (QKV of
 // layer 0) for QKV, gate/up and the LM head; the attention output and the
 // residual rows (x before the O-projection, or the embedding row) for the
-// O-projection. (The down-projection's inputs: down_input_batch / prep_job.)
-template <bool BATCHED>
+// O-projection. (The down-projection's inputs: down_input_batch / prep_job.) On the
+// tensor-core path (MMA) every sequence's vector goes into the slot's MMA
+// operand, row b (mma_opnd_store).
+template <bool BATCHED, bool MMA = false>
 __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
                           uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
     const int t = warp * 32 + lane, l = in.layer;
     auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
     const int B = BATCHED ? p.B : 1;
     for (int b = 0; b < B; ++b) {
-        float* xs = sv + (size_t)b * p.xs_vec_floats;
+        float* xs = MMA ? sv : sv + (size_t)b * p.xs_vec_floats;
         switch (in.op) {
             case MK_OP_QKV:
             case MK_OP_GATEUP:
@@ -431,15 +482,16 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
                                                                      : (size_t)(2 * p.L);
                 const uint16_t* w = norm_ptr(p, p.off_norms + nrm * p.H * 2);
                 if (in.op == MK_OP_QKV && l == 0) {
-                    if (!block_input_plain(nullptr, embed_row(p, b), w, p.eps, p.H, xs, red, t, warp, lane, bar))
+                    if (!block_input_plain<MMA>(nullptr, embed_row(p, b), w, p.eps, p.H, xs, red, t, warp, lane, bar,
+                                                b))
                         return false;
                 } else {
                     // x after the previous layer's MLP (QKV, LM head) or after this layer's attention
                     const uint32_t tag = in.op == MK_OP_GATEUP
                                              ? act_tag(epoch, l, kTagXAttn)
                                              : act_tag(epoch, in.op == MK_OP_QKV ? l - 1 : l, kTagXMlp);
-                    if (!block_input_tagged(p, p.x_t + (size_t)b * p.H, tag, w, p.H, xs, red, t, warp, lane, cbar,
-                                            cuses))
+                    if (!block_input_tagged<MMA>(p, p.x_t + (size_t)b * p.H, tag, w, p.H, xs, red, t, warp, lane,
+                                                 cbar, cuses, b))
                         return false;
                 }
                 break;
@@ -453,8 +505,8 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
                                         act_tag(epoch, l - 1, kTagXMlp), rows, xr, t, lane)) {
                     return false;
                 }
-                if (!block_input_tagged(p, p.attn_t + (size_t)b * p.Q, act_tag(epoch, l, kTagAttn), nullptr, p.Q,
-                                        xs, red, t, warp, lane, cbar, cuses))
+                if (!block_input_tagged<MMA>(p, p.attn_t + (size_t)b * p.Q, act_tag(epoch, l, kTagAttn), nullptr,
+                                             p.Q, xs, red, t, warp, lane, cbar, cuses, b))
                     return false;
                 break;
             }
@@ -468,6 +520,7 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
 // batch 1 the activation warp stages chunks c < kDownStaged ahead instead (one
 // warp moves one sequence's early chunk in time; eight sequences' it does not,
 // nor the chunks that complete only as gate/up ends).
+template <bool MMA = false>
 __device__ __forceinline__ bool down_input_batch(const Params& p, const mk_instr& in, int c, float* sv, float* red,
                                               int warp, int lane, uint64_t* cbar, uint32_t& cuses,
                                               uint32_t epoch) {
@@ -476,8 +529,9 @@ __device__ __forceinline__ bool down_input_batch(const Params& p, const mk_instr
         if (c == 3 && !rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4, act_tag(epoch, l, kTagXAttn),
                                    (int)in.count * 4, slot_resid(p, sv, b), t, lane))
             return false;
-        if (!block_input_tagged(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
-                                nullptr, p.F / 4, sv + (size_t)b * p.xs_vec_floats, red, t, warp, lane, cbar, cuses))
+        if (!block_input_tagged<MMA>(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
+                                     nullptr, p.F / 4, MMA ? sv : sv + (size_t)b * p.xs_vec_floats, red, t, warp,
+                                     lane, cbar, cuses, b))
             return false;
     }
     return true;
@@ -595,7 +649,7 @@ __device__ bool prep_job(const Params& p, const mk_instr* ins, int c, uint8_t* s
         }
     }
     if (in.op == MK_OP_QKV) {
-        float* aux = sv + (size_t)p.B * p.xs_vec_floats;
+        float* aux = sv + (size_t)p.xs_aux_floats;
         for (int b = 0; b < (BATCHED ? p.B : 1); ++b) {
             const int pos = g_pos[b];
             float* row = aux + (size_t)b * (HD + 4);
@@ -746,7 +800,7 @@ __device__ bool compute_tiles(const Params& p, const Tmem& tm, const mk_instr& i
             const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
             switch (in.op) {
                 case MK_OP_QKV: {
-                    const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
+                    const float* row = sv + (size_t)p.xs_aux_floats + (size_t)b * (HD + 4);
                     const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
                     if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, el, rr, act_tag(epoch, in.layer, kTagQKV));
                     break;
@@ -848,7 +902,7 @@ __device__ bool compute_tiles_pair(const Params& p, const Tmem& tm, const mk_ins
         const uint32_t tl = in.op == MK_OP_GATEUP ? gu_tile(p, in, t) : in.first + t;
         switch (in.op) {
             case MK_OP_QKV: {
-                const float* row = sv + (size_t)p.B * p.xs_vec_floats + (size_t)b * (HD + 4);
+                const float* row = sv + (size_t)p.xs_aux_floats + (size_t)b * (HD + 4);
                 const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
                 if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, el, rr, act_tag(epoch, in.layer, kTagQKV));
                 break;
@@ -944,6 +998,110 @@ __device__ bool compute_down(const Params& p, const Tmem& tm, const mk_instr& in
                 const float xin = slot_resid(p, const_cast<float*>(sv), 0)[r * 4 + lane];
                 st_tagged(p.x_t + (in.first + r) * 4 + lane, __fadd_rn(xin, sum), act_tag(epoch, in.layer, kTagXMlp));
             }
+        }
+    }
+    return true;
+}
+
+// Tensor-core path: the outputs of one segment row of sequence b, as the fused
+// epilogues of the CUDA-core path take them (a tile's 4 rows in acc, this lane
+// its row `el`). Returns the row's value (the LM head's greedy selection).
+template <int HD>
+__device__ __noinline__ void mma_epilogue(const Params& p, const mk_instr& in, int b, uint32_t tl,
+                                          const float (&acc)[4], int el, const float* sv, uint32_t epoch) {
+    const bool pub = in.signal_ctr != MK_NO_COUNTER;  // a dropped instruction publishes nothing
+    switch (in.op) {
+        case MK_OP_QKV: {
+            const float* row = sv + (size_t)p.xs_aux_floats + (size_t)b * (HD + 4);
+            const RopeRow rr{row, row + HD / 2, reinterpret_cast<const int*>(row)[HD]};
+            if (pub) qkv_epilogue<HD, true>(p, in.layer, b, tl, acc, el, rr, act_tag(epoch, in.layer, kTagQKV));
+            break;
+        }
+        case MK_OP_GATEUP:
+            if (pub) gateup_epilogue<true>(p, b, tl, acc, el, act_tag(epoch, in.layer, kTagH));
+            break;
+        case MK_OP_OPROJ:
+        case MK_OP_DOWN:
+            // x = x_in + W y for the instruction's rows; x_in waits in the slot
+            if (pub) {
+                const float xin = slot_resid(p, const_cast<float*>(sv), b)[(tl - in.first) * 4 + el];
+                st_tagged(p.x_t + (size_t)b * p.H + tl * 4 + el, __fadd_rn(xin, pick4(acc, el)),
+                          act_tag(epoch, in.layer, in.op == MK_OP_OPROJ ? kTagXAttn : kTagXMlp));
+            }
+            break;
+        default:
+            logits_epilogue(p, b, tl, acc, el);
+            break;
+    }
+}
+
+// Tensor-core path, a matvec job of the compute warps once its operand is in the
+// slot: for each of the instruction's segments (the down-projection's only after
+// its last chunk), wait for the accumulator, read this warp's lane quarter (rows
+// 32 q .. 32 q + 31 of the segment, q = warp mod 4) and release it, then run the
+// epilogues of the warp's sequences (the first half of the batch for warps 0-3,
+// the second for 4-7, as on the CUDA-core path): y = high + low column. `sg` is
+// the SM's number of the instruction's first segment (the issuer counts alike).
+template <int HD>
+__device__ bool mma_job(const Params& p, const MmaBars& mb, uint32_t tbase, const mk_instr& in, int c, uint32_t sg,
+                        const float* sv, int warp, int lane, uint32_t job, uint32_t epoch, uint2* selp) {
+    const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
+    if (c + 1 < (int)g.jobs) return true;  // down chunks 0-2 only accumulate
+    const bool sel = in.op == MK_OP_LMHEAD && p.next_tokens != nullptr;
+    const uint32_t q = (uint32_t)warp & 3u;
+    const PairSeqs ps(p.B, warp);
+    const int el = lane & 3;
+    Best best[4] = {best_none(), best_none(), best_none(), best_none()};
+    for (uint32_t rg = 0; rg < g.nrange; ++rg) {
+        for (uint32_t sgi = 0; sgi < g.segs; ++sgi) {
+            const uint32_t sn = sg + rg * g.segs + sgi, a = sn % (uint32_t)kMaxAcc;
+            if (!wait_bar(p, mb.afull + a, (sn / (uint32_t)kMaxAcc) & 1u, nullptr, sn, 13, lane)) return false;
+            if (rg == 0 && sgi == 0 && warp == 0 && lane == 0) trace(p, job, kTrFill);
+            tmem_fence_after();
+            uint32_t d[16];
+            tmem_ld16(tbase + ((32u * q) << 16) + a * kAccCols, d);
+            tmem_wait_ld(d);
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mb.aempty + a);
+            const uint32_t left = g.rows - sgi * kMmaRows;
+            const uint32_t rows = left < kMmaRows ? left : kMmaRows;
+            const uint32_t m = 32u * q + (uint32_t)lane;  // the lane's row of the segment
+            const uint32_t first = in.op == MK_OP_GATEUP ? rg * (uint32_t)(p.F / 8) + in.first : in.first;
+            const uint32_t tl = first + sgi * (kMmaRows / 4) + (m >> 2);
+            // the warp's sequences' totals, high + low (register indices fixed at compile time)
+            float y[4];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                float hi = 0.f, lo = 0.f;
+#pragma unroll
+                for (int b = 0; b < kMaxBatch; ++b)
+                    if (b == ps.b0 + bb) {
+                        hi = __uint_as_float(d[b]);
+                        lo = __uint_as_float(d[kMaxBatch + b]);
+                    }
+                y[bb] = __fadd_rn(hi, lo);
+            }
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                if (bb < ps.nb) {  // warp-uniform
+                    float acc[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[r] = __shfl_sync(0xffffffffu, y[bb], (lane & ~3) | r);
+                    if (m < rows) {
+                        mma_epilogue<HD>(p, in, ps.b0 + bb, tl, acc, el, sv, epoch);
+                        if (sel) best_take(best[bb], y[bb], tl * 4 + el);
+                    }
+                }
+            }
+        }
+    }
+    if (sel) {  // the warp's best row of each of its sequences (publish_best)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+            const Best r = best_reduce(best[bb], 16, 1);
+            if (lane == 0 && bb < ps.nb)
+                selp[warp * kMaxBatch + ps.b0 + bb] = make_uint2(__float_as_uint(r.v), r.i);
         }
     }
     return true;
@@ -1079,11 +1237,13 @@ __device__ __noinline__ void publish_best(const Params& p, const mk_instr& in, c
     }
 }
 
-template <int KH, int KO, int KF, int HD, bool BATCHED>
-__device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, const Slots& sl,
+template <int KH, int KO, int KF, int HD, bool BATCHED, bool MMA>
+__device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, const Slots& sl, const MmaBars& mb,
                              float* tot, float* red, uint64_t* cbar, uint2* selp, int i0, int i1, int warp,
                              int lane, uint32_t epoch) {
     uint32_t j = 0, cuses = 0;
+    uint32_t sg = 0;  // tensor-core path: the SM's segments so far (mma_issuer counts alike)
+    uint32_t ph = 0;  // tensor-core path: bit s, the phase of slot s's operand / MMA-done barriers
     for (int i = i0; i < i1;) {
         const mk_instr in = p.instrs[i];
         const int njobs = (in.op == MK_OP_DOWN) ? 4 : 1;
@@ -1097,9 +1257,10 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
             // warp) are loaded here
             bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
                       : in.op == MK_OP_DOWN ? ((!BATCHED && c < kDownStaged) ||
-                                                     down_input_batch(p, in, c, sv, red, warp, lane, cbar, cuses,
-                                                                      epoch))
-                                            : job_input<BATCHED>(p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
+                                                     down_input_batch<MMA>(p, in, c, sv, red, warp, lane, cbar,
+                                                                           cuses, epoch))
+                                            : job_input<BATCHED, MMA>(p, in, c, sv, red, warp, lane, cbar, cuses,
+                                                                      epoch);
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7);
             // one call site per routine: the kernel's code is what every SM re-fetches
@@ -1107,6 +1268,16 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
             if (in.op == MK_OP_ATTN) {
                 ok = compute_attn_job<HD, BATCHED>(p, ring, in, sl.slot(j), warp, lane, cbar, cuses, j,
                                                    epoch);
+            } else if constexpr (MMA) {
+                // the operand is complete (the input's last barrier): hand it to the
+                // tensor cores (async proxy), then read the accumulators; the slot is
+                // free once the job's MMAs are done
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mb.opnd + s);
+                ok = mma_job<HD>(p, mb, tm.base, in, c, sg, sv, warp, lane, j, epoch, selp) &&
+                     wait_bar(p, mb.mdone + s, (ph >> s) & 1u, nullptr, j, 12, lane);
+                ph ^= 1u << s;
             } else if (in.op == MK_OP_DOWN) {
                 if constexpr (BATCHED) ok = compute_down_pair<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
                 else ok = compute_down<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
@@ -1151,6 +1322,12 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
                     }
                 }
                 mbar_arrive(sl.empty + s);
+            }
+        }
+        if constexpr (MMA) {
+            if (in.op != MK_OP_ATTN) {
+                const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
+                sg += g.nrange * g.segs;
             }
         }
         ++i;
@@ -1206,6 +1383,54 @@ __device__ __forceinline__ void fill_seek(const Params& p, FillCur& c, int i1) {
     while (c.i < i1 && c.seq >= p.instrs[c.i].seq + p.instrs[c.i].nfill) ++c.i;
 }
 
+// The tensor map of weight matrix `kind` whose boxes are 4 << hk rows high.
+__device__ __forceinline__ const void* tmap(const Params& p, int kind, int hk) {
+    return static_cast<const uint8_t*>(p.tmaps) + (size_t)(kind * kBoxHeights + hk) * 128u;
+}
+
+// Tensor-core path: fill t of matvec instruction `in` into the stage at dst. The
+// fill is K-boxes [kf * nb, kf * nb + nb) of one segment (fewer at the end of K),
+// box i of the fill at i * r8 rows into the stage; each box is assembled from
+// TMA boxes of 128, 64, ..., 4 rows (the segment's row count in binary, larger
+// first, so every piece starts on a 1024-byte boundary of the swizzle).
+__device__ void issue_mma_fill(const Params& p, const mk_instr& in, uint32_t t, uint8_t* dst, uint64_t* bar,
+                               uint64_t pol) {
+    const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
+    const uint32_t per = g.per_job();
+    const uint32_t c = t / per;
+    const MmaFill f = mma_fill(g, t % per);
+    const uint32_t b0 = f.kf * g.nb, b1 = min(b0 + g.nb, g.k64);
+    mbar_arrive_expect_tx(bar, (b1 - b0) * f.rows * 128u);
+    int kind;
+    uint32_t row0;  // the segment's first row in the matrix's packed row order
+    switch (in.op) {
+        case MK_OP_QKV: kind = kTmQKV; row0 = 4u * in.first; break;
+        case MK_OP_OPROJ: kind = kTmO; row0 = 4u * in.first; break;
+        case MK_OP_GATEUP: kind = kTmGU; row0 = 4u * (f.rg * (uint32_t)(p.F / 8) + in.first); break;
+        case MK_OP_DOWN: kind = kTmDown; row0 = 4u * in.first; break;
+        default: kind = kTmLM; row0 = 4u * in.first; break;
+    }
+    row0 += f.seg * kMmaRows;
+    for (uint32_t bx = b0; bx < b1; ++bx) {
+        uint8_t* bd = dst + (size_t)(bx - b0) * g.r8 * 128u;
+        const int k = (int)(bx * kBoxK);
+        uint32_t ro = 0;
+        for (int hk = kBoxHeights - 1; hk >= 0; --hk) {
+            const uint32_t h = 4u << hk;
+            if (!(f.rows & h)) continue;
+            const void* m = tmap(p, kind, hk);
+            const uint32_t row = row0 + ro;
+            if (kind == kTmDown)  // {col, row in block, chunk, row block, layer}
+                tma_load_5d(bd + ro * 128u, m, k, 0, (int)c, (int)(row / 4u), (int)in.layer, bar, pol);
+            else if (kind == kTmLM)
+                tma_load_2d(bd + ro * 128u, m, k, (int)row, bar, pol);
+            else
+                tma_load_3d(bd + ro * 128u, m, k, (int)row, (int)in.layer, bar, pol);
+            ro += h;
+        }
+    }
+}
+
 // One thread (the loader warp's lane 0) streams the SM's fills into the ring, in
 // list order: weight tiles and the cached KV of attention items, all final at
 // launch. It never waits on a dependency counter, only for a stage to be free
@@ -1213,6 +1438,7 @@ __device__ __forceinline__ void fill_seek(const Params& p, FillCur& c, int i1) {
 // attention item (KV). So the next instructions' weights arrive while the step
 // still waits for their activations. It issues nothing else, so a freed stage is
 // refilled at once.
+template <bool MMA>
 __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
@@ -1242,6 +1468,11 @@ __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
                 uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
                 uint64_t* bar = ring.full + s;
                 ring.armed[s] = seq;  // published by the release of the arrive below
+                if (MMA && in.op != MK_OP_ATTN) {
+                    issue_mma_fill(p, in, t, dst, bar, pol);
+                    issued = seq + 1;
+                    continue;
+                }
                 const FillSrc f = fill_source(p, in, t);
                 if (f.b != nullptr) {  // attention: keys, then values half a stage later
                     mbar_arrive_expect_tx(bar, 2 * f.bytes);
@@ -1272,6 +1503,80 @@ drain:
             }
         }
     }
+}
+
+// Tensor-core path: warp 8, converged (lane 0 issues), walks the SM's jobs in
+// order. For a matvec job it waits until the compute warps have written the job's
+// operand into its slot, then for each fill: that its segment's accumulator has
+// been read out since its previous use (first fill of the segment), that the
+// fill has landed; it issues the fill's MMAs (4 per 64-column box, K = 16 each;
+// the segment's first overwrites the accumulator) and commits them to the
+// stage's empty barrier, so the loader refills the stage once they have read it.
+// A segment's last fill also commits to its accumulator's full barrier, a job's
+// last to the slot's MMA-done barrier. Before it returns, on every way out, it
+// waits until all the MMAs it issued have completed (the CTA then releases
+// Tensor Memory). Every wait is bounded.
+__device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb, const Slots& sl, uint32_t tbase,
+                           int i0, int i1, int lane) {
+    uint32_t j = 0, sg = 0;
+    uint32_t ph = 0;  // bit s: phase of slot s's operand / MMA-done barriers (matvec jobs only)
+    bool any = false;
+    for (int i = i0; i < i1; ++i) {
+        const mk_instr in = p.instrs[i];
+        if (in.op == MK_OP_ATTN) {
+            ++j;
+            continue;
+        }
+        const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
+        const uint32_t per = g.per_job();
+        for (uint32_t c = 0; c < g.jobs; ++c, ++j) {
+            const uint32_t s = j % sl.NS;
+            if (!wait_bar(p, mb.opnd + s, (ph >> s) & 1u, nullptr, j, 10, lane)) goto out;
+            ph ^= 1u << s;
+            {
+                const uint32_t opnd = smem_addr(sl.slot(j));
+                for (uint32_t r = 0; r < per; ++r) {
+                    const MmaFill f = mma_fill(g, r);
+                    const uint32_t sn = sg + f.rg * g.segs + f.seg;
+                    const uint32_t a = sn % (uint32_t)kMaxAcc, use = sn / (uint32_t)kMaxAcc;
+                    if (c == 0 && f.kf == 0 && use > 0 &&
+                        !wait_bar(p, mb.aempty + a, (use - 1u) & 1u, nullptr, sn, 11, lane))
+                        goto out;
+                    const uint32_t seq = in.seq + c * per + r;
+                    if (!wait_fill(p, ring, seq, lane)) goto out;
+                    tmem_fence_after();
+                    if (lane == 0) {
+                        const uint32_t st = smem_addr(ring.stage(seq));
+                        const uint32_t b0 = f.kf * g.nb, b1 = min(b0 + g.nb, g.k64);
+                        for (uint32_t bx = b0; bx < b1; ++bx)
+#pragma unroll
+                            for (uint32_t kk = 0; kk < 4; ++kk)
+                                mma_bf16(tbase + a * kAccCols, sw128_desc(st + (bx - b0) * g.r8 * 128u + kk * 32u),
+                                         sw128_desc(opnd + bx * 2048u + kk * 32u), (c | bx | kk) != 0u);
+                        mma_commit(ring.empty + seq % ring.S);
+                        if (c + 1 == g.jobs && f.kf + 1 == g.fps) mma_commit(mb.afull + a);
+                    }
+                    __syncwarp();
+                    any = true;
+                }
+            }
+            if (lane == 0) mma_commit(mb.mdone + s);
+            __syncwarp();
+        }
+        sg += g.nrange * g.segs;
+    }
+out:
+    if (any && lane == 0) {
+        mma_commit(mb.fin);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_wait_sleep(mb.fin, 0u, 20000u)) {
+            if (global_timer_ns() - t0 > p.timeout_ns) {
+                record_error(p, MK_ERR_TIMEOUT, j, 0xfffffff9u, 0, 0, 14);
+                break;
+            }
+        }
+    }
+    __syncwarp();
 }
 
 // Mover warp q (its lanes converged throughout; its warp index mod 4 is q, the
@@ -1333,12 +1638,12 @@ __device__ void mover(const Params& p, const Ring& ring, const Tmem& tm, int i0,
 
 // ------------------------------------------------------------------ the kernel
 
-template <int KH, int KO, int KF, int HD, bool BATCHED>
+template <int KH, int KO, int KF, int HD, bool BATCHED, bool MMA>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_epoch, s_skip;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes);
+    const SmemLayout m = smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, MMA);
     Ring ring;
     ring.base = smem + m.ring;
     ring.full = reinterpret_cast<uint64_t*>(smem + m.full);
@@ -1361,6 +1666,12 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     tm.n = (uint32_t)p.n_tslots;
     tm.cols = p.tslot_cols;
     uint32_t* tbase = reinterpret_cast<uint32_t*>(smem + m.tbase);
+    MmaBars mb;
+    mb.opnd = reinterpret_cast<uint64_t*>(smem + m.opnd);
+    mb.mdone = reinterpret_cast<uint64_t*>(smem + m.mdone);
+    mb.afull = reinterpret_cast<uint64_t*>(smem + m.afull);
+    mb.aempty = reinterpret_cast<uint64_t*>(smem + m.aempty);
+    mb.fin = reinterpret_cast<uint64_t*>(smem + m.fin);
 
     // All of the SM's Tensor Memory for this CTA (one CTA per SM; the previous
     // step's CTA released it before exiting). Warp 0, converged.
@@ -1387,9 +1698,25 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             sl.job[s] = 0xffffffffu;
         }
         mbar_init(reinterpret_cast<uint64_t*>(smem + m.cbar), kConsumerWarps);
+        if (MMA) {
+            for (int s = 0; s < p.xs_slots; ++s) {
+                mbar_init(mb.opnd + s, kConsumerWarps);
+                mbar_init(mb.mdone + s, 1);
+            }
+            for (int a = 0; a < kMaxAcc; ++a) {
+                mbar_init(mb.afull + a, 1);
+                mbar_init(mb.aempty + a, kConsumerWarps);
+            }
+            mbar_init(mb.fin, 1);
+        }
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
         uint32_t skip = ld_volatile_u32(&p.ctl->status) != 0u;
+        // the tensor-core path's swizzled operands need 1024-byte-aligned slots and stages
+        if (!skip && MMA && ((smem_addr(smem) | smem_addr(smem + m.xs)) & 1023u) != 0u) {
+            skip = 1;
+            if (blockIdx.x == 0) record_error(p, MK_ERR_UNSUPPORTED, smem_addr(smem), smem_addr(smem + m.xs), 0, 0, 15);
+        }
         if (!skip) {
             for (int b = 0; b < p.B; ++b) {
                 const int tok = p.tokens[b], pos = p.positions[b];
@@ -1413,16 +1740,20 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (!s_skip) {
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
         if (warp >= kConsumerWarps && warp < kConsumerWarps + kMoveWarps) {
-            mover<BATCHED>(p, ring, tm, i0, i1, warp & 3, lane);
+            if constexpr (MMA) {
+                if (warp == kConsumerWarps) mma_issuer(p, ring, mb, sl, tm.base, i0, i1, lane);
+            } else {
+                mover<BATCHED>(p, ring, tm, i0, i1, warp & 3, lane);
+            }
         } else if (warp == kLoaderWarp) {
-            if (lane == 0) loader(p, ring, i0, i1);
+            if (lane == 0) loader<MMA>(p, ring, i0, i1);
         } else if (warp == kPrepWarp || warp >= kStageWarp0) {
             // one call site: the stage warps have jobs at batch 1 only
             if (warp == kPrepWarp || !BATCHED)
                 activation_warp<KH, KO, KF, HD, BATCHED>(p, sl, i0, i1, lane, s_epoch,
                                                          warp == kPrepWarp ? -1 : warp - kStageWarp0);
         } else {
-            compute_warp<KH, KO, KF, HD, BATCHED>(p, ring, tm, sl, reinterpret_cast<float*>(smem + m.tot),
+            compute_warp<KH, KO, KF, HD, BATCHED, MMA>(p, ring, tm, sl, mb, reinterpret_cast<float*>(smem + m.tot),
                                                   reinterpret_cast<float*>(smem + m.red),
                                                   reinterpret_cast<uint64_t*>(smem + m.cbar),
                                                   reinterpret_cast<uint2*>(smem + m.sel), i0, i1, warp, lane,
@@ -1467,7 +1798,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ------------------------------------------------------------------ host-side launch
 
 size_t smem_bytes(const Params& p) {
-    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes).total;
+    return smem_layout(p.n_stages, p.stage_bytes, p.xs_slots, p.xs_slot_bytes, p.mma != 0).total;
 }
 
 using KernelFn = void (*)(Params);
@@ -1475,23 +1806,25 @@ using KernelFn = void (*)(Params);
 // One kernel per shape and per batch class: only the batch > 1 kernel carries the
 // compute warps' down-chunk loads (at batch 1 they would change the batch-1
 // kernel's register allocation and cost it a few microseconds per step).
-template <bool BATCHED>
+template <bool BATCHED, bool MMA>
 static KernelFn pick_b(int KH, int KO, int KF, int HD) {
-    if (KH == 2 && KO == 2 && KF == 2 && HD == 64) return megakernel<2, 2, 2, 64, BATCHED>;
-    if (KH == 8 && KO == 8 && KF == 8 && HD == 64) return megakernel<8, 8, 8, 64, BATCHED>;
-    if (KH == 12 && KO == 12 && KF == 8 && HD == 128) return megakernel<12, 12, 8, 128, BATCHED>;
+    if (KH == 2 && KO == 2 && KF == 2 && HD == 64) return megakernel<2, 2, 2, 64, BATCHED, MMA>;
+    if (KH == 8 && KO == 8 && KF == 8 && HD == 64) return megakernel<8, 8, 8, 64, BATCHED, MMA>;
+    if (KH == 12 && KO == 12 && KF == 8 && HD == 128) return megakernel<12, 12, 8, 128, BATCHED, MMA>;
     return nullptr;
 }
 
-static KernelFn pick(int KH, int KO, int KF, int HD, int B) {
-    return B > 1 ? pick_b<true>(KH, KO, KF, HD) : pick_b<false>(KH, KO, KF, HD);
+// Batch > 1: the CUDA-core kernel or the tensor-core one (p.mma).
+static KernelFn pick(int KH, int KO, int KF, int HD, int B, bool mma) {
+    if (B <= 1) return pick_b<false, false>(KH, KO, KF, HD);
+    return mma ? pick_b<true, true>(KH, KO, KF, HD) : pick_b<true, false>(KH, KO, KF, HD);
 }
 
-static KernelFn pick(const Params& p) { return pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B); }
+static KernelFn pick(const Params& p) { return pick(p.H / 256, p.Q / 256, p.F / 1024, p.d, p.B, p.mma != 0); }
 
 bool supported(int H, int Q, int F, int d) {
     if (H % 256 || Q % 256 || F % 1024) return false;
-    return pick(H / 256, Q / 256, F / 1024, d, 1) != nullptr;
+    return pick(H / 256, Q / 256, F / 1024, d, 1, false) != nullptr;
 }
 
 cudaError_t prepare(const Params& p) {

@@ -104,6 +104,40 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// Tiled TMA loads (global -> this CTA's shared memory) through a tensor map in
+// global memory, completion counted on `bar`. Coordinates innermost first; the
+// innermost is a multiple of 64 elements here (128 bytes). No multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int c0, int c1, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, int c1, int c2, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(void* dst, const void* map, int c0, int c1, int c2, int c3, int c4,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Generic-proxy writes to shared memory by this thread become visible to the
+// async proxy (the tensor cores' operand reads) after this fence.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tagged activations
 //
 // Inside one megakernel launch, activations that cross SMs (residual stream x,
@@ -396,11 +430,29 @@ __device__ __forceinline__ int xs_index(int n, int e) {
 // The thread's pairs (v0[i], v1[i]) = elements 2j, 2j + 1 into the XSmem vector
 // at xs; with w (bf16 norm weights of the pairs, pre-loaded in wv), RMSNorm
 // first. `red`: kConsumerWarps floats of shared scratch. Ends with a barrier.
-template <class Bar>
+// The tensor cores' input operand (the megakernel's tensor-core path): row `row`
+// (a sequence's high bf16 part; its low part is row 8 + row) of a K-major operand
+// of 16 rows, stored as 64-column chunks of two 8-row atoms (2048 bytes a chunk),
+// each 128-byte row with its 16-byte pieces swizzled by the row index (piece i at
+// i ^ row). Elements k, k + 1 (k even) of x: the high parts round x to bf16, the
+// low parts the exact fp32 remainder x - high, so high + low carries x to about
+// 2^-17 relative.
+__device__ __forceinline__ void mma_opnd_store(float* base, int row, int k, float x0, float x1) {
+    uint8_t* p8 = reinterpret_cast<uint8_t*>(base) + (size_t)(k >> 6) * 2048 + row * 128 +
+                  ((((k >> 3) & 7) ^ row) << 4) + (k & 7) * 2;
+    const uint16_t h0 = f2bf(x0), h1 = f2bf(x1);
+    const uint16_t l0 = f2bf(__fsub_rn(x0, bf2f(h0))), l1 = f2bf(__fsub_rn(x1, bf2f(h1)));
+    *reinterpret_cast<uint32_t*>(p8) = (uint32_t)h0 | ((uint32_t)h1 << 16);
+    *reinterpret_cast<uint32_t*>(p8 + 1024) = (uint32_t)l0 | ((uint32_t)l1 << 16);
+}
+
+// With MMAOP the pairs go into the tensor cores' operand at xs, row `orow`
+// (mma_opnd_store) instead of an XSmem vector.
+template <bool MMAOP = false, class Bar>
 __device__ __forceinline__ bool block_store_input(const float (&v0)[kMaxPairs], const float (&v1)[kMaxPairs],
                                                   const uint32_t (&wv)[kMaxPairs], bool norm, float eps,
                                                   int n, float* xs, float* red, int t, int warp, int lane,
-                                                  Bar&& bar) {
+                                                  Bar&& bar, int orow = 0) {
     const int np = n / 2;
     float r = 1.f;
     if (norm) {
@@ -428,17 +480,18 @@ __device__ __forceinline__ bool block_store_input(const float (&v0)[kMaxPairs], 
                 a = __fmul_rn(__fmul_rn(a, r), bf_lo(wv[i]));
                 b = __fmul_rn(__fmul_rn(b, r), bf_hi(wv[i]));
             }
-            *reinterpret_cast<float2*>(xs + xs_index(n, 2 * j)) = make_float2(a, b);
+            if constexpr (MMAOP) mma_opnd_store(xs, orow, 2 * j, a, b);
+            else *reinterpret_cast<float2*>(xs + xs_index(n, 2 * j)) = make_float2(a, b);
         }
     }
     return bar();
 }
 
 // The same from a plain source: fp32 (src_f) or bf16 (src_h) in global memory.
-template <class Bar>
+template <bool MMAOP = false, class Bar>
 __device__ __forceinline__ bool block_input_plain(const float* src_f, const uint16_t* src_h, const uint16_t* w,
                                                   float eps, int n, float* xs, float* red, int t, int warp,
-                                                  int lane, Bar&& bar) {
+                                                  int lane, Bar&& bar, int orow = 0) {
     const int np = n / 2;
     float v0[kMaxPairs], v1[kMaxPairs];
     uint32_t wv[kMaxPairs];
@@ -460,7 +513,7 @@ __device__ __forceinline__ bool block_input_plain(const float* src_f, const uint
             }
         }
     }
-    return block_store_input(v0, v1, wv, w != nullptr, eps, n, xs, red, t, warp, lane, bar);
+    return block_store_input<MMAOP>(v0, v1, wv, w != nullptr, eps, n, xs, red, t, warp, lane, bar, orow);
 }
 
 // ------------------------------------------------------------------ the 4-row tile

@@ -50,6 +50,75 @@ MK_HD constexpr uint32_t attn_scratch_floats(int hd) {
 MK_HD constexpr uint32_t attn_item_bytes(int group, int hd) {
     return ((uint32_t)(group * hd * 4 + 2 * hd * 2) + 15u) & ~15u;
 }
+// Tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES). An instruction's
+// weight rows are cut into segments of at most 128 rows (gate/up: per MLP chunk);
+// each segment streams as 64-column TMA boxes (128 bytes: the swizzle span), a
+// fill holding nb boxes of the segment side by side, and accumulates in its own
+// Tensor Memory accumulator of 16 fp32 columns (8 sequences, high and low bf16
+// parts of the input) over lanes = rows.
+constexpr uint32_t kAccCols = 16;
+constexpr int kMaxAcc = (int)(kTmemCols / kAccCols);  // accumulators in use at once
+constexpr uint32_t kMmaRows = 128;                   // M of every MMA: rows of a segment
+constexpr uint32_t kBoxK = 64;                        // K columns of one TMA box
+constexpr int kBoxHeights = 6;                        // box heights 4, 8, ..., 128 rows
+// Tensor maps, one per (weight matrix, box height): index kind * kBoxHeights + h.
+enum TmapKind { kTmQKV = 0, kTmO = 1, kTmGU = 2, kTmDown = 3, kTmLM = 4, kTmKinds = 5 };
+
+// Fills of a matvec instruction on the tensor-core path. Fill t of the instruction
+// is job c = t / (nrange * segs * fps) (the down-projection's chunk), then range,
+// segment and K-fill in that order (see mma_fill).
+struct MmaGeom {
+    uint32_t k64;     // 64-column boxes along K
+    uint32_t rows;    // weight rows of one range
+    uint32_t nrange;  // 4 for gate/up (one per MLP chunk), else 1
+    uint32_t segs;    // segments of <= 128 rows per range
+    uint32_t r8;      // rows of a full segment rounded up to 8: a box's pitch in a fill
+    uint32_t nb;      // boxes per fill
+    uint32_t fps;     // fills per segment and job
+    uint32_t jobs;    // 4 chunk jobs for the down-projection, else 1
+    MK_HD uint32_t per_job() const { return nrange * segs * fps; }
+    MK_HD uint32_t nfill() const { return jobs * per_job(); }
+};
+
+MK_HD inline MmaGeom mma_geom(uint32_t op, uint32_t count, uint32_t aux0, int H, int Q, int F,
+                              uint32_t stage_bytes) {
+    MmaGeom g{};
+    g.jobs = 1;
+    g.nrange = 1;
+    g.rows = 4u * count;
+    g.k64 = (uint32_t)H / kBoxK;
+    if (op == MK_OP_OPROJ) {
+        g.k64 = (uint32_t)Q / kBoxK;
+    } else if (op == MK_OP_DOWN) {
+        g.k64 = (uint32_t)(F / 4) / kBoxK;
+        g.jobs = 4;
+    } else if (op == MK_OP_GATEUP) {
+        g.rows = 4u * aux0;
+        g.nrange = 4;
+    }
+    g.segs = (g.rows + kMmaRows - 1) / kMmaRows;
+    g.r8 = g.rows < kMmaRows ? (g.rows + 7u) & ~7u : kMmaRows;
+    g.nb = stage_bytes / (g.r8 * 128u);
+    if (g.nb < 1) g.nb = 1;
+    if (g.nb > g.k64) g.nb = g.k64;
+    g.fps = (g.k64 + g.nb - 1) / g.nb;
+    return g;
+}
+
+// Fill r (< per_job) of one job: its range, segment, K-fill and the segment's rows.
+struct MmaFill {
+    uint32_t rg, seg, kf, rows;
+};
+MK_HD inline MmaFill mma_fill(const MmaGeom& g, uint32_t r) {
+    MmaFill f;
+    f.rg = r / (g.segs * g.fps);
+    f.seg = (r / g.fps) % g.segs;
+    f.kf = r % g.fps;
+    const uint32_t left = g.rows - f.seg * kMmaRows;
+    f.rows = left < kMmaRows ? left : kMmaRows;
+    return f;
+}
+
 constexpr int kMaxLayers = 64;
 constexpr int kCounterStride = 32;                   // uint32 per counter: one per 128 B line
 constexpr size_t kSmemBudget = 227 * 1024;           // dynamic shared memory per CTA
@@ -92,18 +161,27 @@ struct SmemLayout {
     uint32_t sel;                             // [warps][kMaxBatch] LM-head best per warp (greedy)
     uint32_t tfull, tempty, tarmed;           // Tensor Memory slots: landed / released / fill held
     uint32_t tbase;                           // Tensor Memory address of the allocation
+    // tensor-core path only (zero bytes otherwise)
+    uint32_t opnd;                            // [NS] a job's MMA operand is in its slot
+    uint32_t mdone;                           // [NS] the job's MMAs have completed
+    uint32_t afull, aempty;                   // [kMaxAcc] accumulator written / read
+    uint32_t fin;                             // every MMA issued has completed
     uint32_t total;
 };
 
 MK_HD inline uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
-MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes) {
+// With `mma` (the tensor-core path) the slots start on a 1024-byte boundary (each
+// holds its MMA operand in 128-byte-swizzled atoms of 8 rows) and the MMA
+// barriers are added.
+MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_t slot_bytes, bool mma = false) {
     SmemLayout m;
     uint32_t o = 0;
     m.ring = o;      o += (uint32_t)S * stage_bytes;
     m.full = o;      o += 8u * S;
     m.empty = o;     o += 8u * S;
     m.armed = o;     o = align16(o + 4u * S);
+    if (mma) o = (o + 1023u) & ~1023u;
     m.xs = o;        o += (uint32_t)NS * slot_bytes;
     m.xs_full = o;   o += 8u * NS;
     m.xs_empty = o;  o += 8u * NS;
@@ -118,6 +196,13 @@ MK_HD inline SmemLayout smem_layout(int S, uint32_t stage_bytes, int NS, uint32_
     m.tempty = o;    o += 8u * kMaxTmemSlots;
     m.tarmed = o;    o += 4u * kMaxTmemSlots;
     m.tbase = o;     o += 4u;
+    o = (o + 7u) & ~7u;
+    const uint32_t nacc = mma ? (uint32_t)kMaxAcc : 0u, nsl = mma ? (uint32_t)NS : 0u;
+    m.opnd = o;      o += 8u * nsl;
+    m.mdone = o;     o += 8u * nsl;
+    m.afull = o;     o += 8u * nacc;
+    m.aempty = o;    o += 8u * nacc;
+    m.fin = o;       o += mma ? 8u : 0u;
     m.total = align16(o);
     return m;
 }
@@ -186,6 +271,10 @@ struct Params {
     int xs_slots;              // activation slots (1..3)
     uint32_t xs_slot_bytes;
     uint32_t xs_vec_floats;    // stride of one sequence's vector inside a slot
+    uint32_t xs_aux_floats;    // offset of the slot's RoPE rows and residual rows
+    // tensor-core projections (batch > 1): MK_PROJ_TENSOR_CORES, else 0
+    int mma;
+    const void* tmaps;         // [kTmKinds * kBoxHeights] CUtensorMap (64-byte aligned, global)
     int n_counters;
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)

@@ -24,19 +24,23 @@ struct Plan {
 };
 
 // Ring stage size the kernel uses for this shape.
-uint32_t default_stage_bytes(const Layout& L);
+uint32_t default_stage_bytes(const Layout& L, bool mma = false);
 
 // Shared-memory budget split: activation slots and ring stages.
 struct SlotPlan {
     int keys_per_stage;
     uint32_t vec_floats;   // one sequence's input vector inside a slot
     uint32_t item_bytes;   // an attention item's q and new key/value inside a slot
+    uint32_t aux_floats;   // where the RoPE rows and residual rows start inside a slot
     uint32_t slot_bytes;
     int xs_slots;
     int stages;
     uint32_t smem_bytes;
 };
-SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes);
+SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma = false);
+// Whether a schedule for `batch` with these options runs the projections on the
+// tensor cores.
+bool use_mma(int batch, const mk_schedule_opts* opts);
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);

@@ -33,32 +33,43 @@
 
 namespace mk {
 
-uint32_t default_stage_bytes(const Layout& L) {
+uint32_t default_stage_bytes(const Layout& L, bool mma) {
     uint32_t s = std::max(L.tile_h, std::max(L.tile_o, L.tile_f));
-    return (uint32_t)align_up(s, 128);
+    // the tensor-core path places its boxes on 1024-byte boundaries (swizzle atoms),
+    // and a fill holds at least one 64-column box of a full 128-row segment
+    if (mma) s = std::max(s, kMmaRows * kBoxK * 2u);
+    return (uint32_t)align_up(s, mma ? 1024 : 128);
 }
 
-SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
+SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma) {
     SlotPlan sp{};
     sp.keys_per_stage = (int)(stage_bytes / (4u * (uint32_t)L.d));
-    sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 4);
+    sp.vec_floats = (uint32_t)align_up((size_t)std::max(std::max(L.H, L.Q), L.F / 4), 64);
     sp.item_bytes = attn_item_bytes(L.group, L.d) + 4u * attn_scratch_floats(L.d);
     // per sequence: the input vector; then per sequence (QKV jobs) the RoPE row
     // cos[d/2], sin[d/2] and the position; then per sequence (O-proj and down
     // jobs) the residual rows the job updates. An attention job: its item's q and
-    // new key/value, then the item's scratch.
-    sp.slot_bytes = align16(std::max(
-        (uint32_t)batch * (sp.vec_floats + (uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u, sp.item_bytes));
+    // new key/value, then the item's scratch. On the tensor-core path the input
+    // vectors are the MMA operand instead: 16 rows (each sequence's high and low
+    // bf16 parts) of vec_floats bf16 each, whatever the batch.
+    const uint32_t aux = (uint32_t)batch * ((uint32_t)L.d + 4u + (uint32_t)kMaxResidRows) * 4u;
+    if (mma) {
+        sp.aux_floats = sp.vec_floats * 8u;
+        sp.slot_bytes = (uint32_t)align_up(std::max(sp.vec_floats * 32u + aux, sp.item_bytes), 1024);
+    } else {
+        sp.aux_floats = (uint32_t)batch * sp.vec_floats;
+        sp.slot_bytes = align16(std::max((uint32_t)batch * sp.vec_floats * 4u + aux, sp.item_bytes));
+    }
     // the most job slots that leave at least 8 stages (an attention item's keys all
-    // sit in the ring at once), else at least 4; the stage count is a multiple of
-    // 4, so each stage's fills belong to one mover warp
+    // sit in the ring at once), else at least 4; on the CUDA-core path the stage
+    // count is a multiple of 4, so each stage's fills belong to one mover warp
     sp.xs_slots = 0;
     for (int min_s = 8; min_s >= kMoveWarps && sp.xs_slots == 0; min_s -= 4) {
         for (int ns = 3; ns >= 1; --ns) {
             int S = 0;
-            while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes).total + 1024 <= kSmemBudget)
+            while (smem_layout(S + 1, stage_bytes, ns, sp.slot_bytes, mma).total + 1024 <= kSmemBudget)
                 ++S;
-            S -= S % kMoveWarps;
+            if (!mma) S -= S % kMoveWarps;
             if (S >= min_s) {
                 sp.xs_slots = ns;
                 sp.stages = S;
@@ -70,8 +81,12 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes) {
         sp.xs_slots = 1;
         sp.stages = 0;
     }
-    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes).total;
+    sp.smem_bytes = smem_layout(sp.stages, stage_bytes, sp.xs_slots, sp.slot_bytes, mma).total;
     return sp;
+}
+
+bool use_mma(int batch, const mk_schedule_opts* opts) {
+    return batch > 1 && !(opts && opts->proj == MK_PROJ_CUDA_CORES);
 }
 
 // the most SMs a plan may spread over (a B200 has 148)
@@ -83,9 +98,11 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     if (opts) o = *opts;
     if (batch < 1 || batch > kMaxBatch || max_ctx < 1 || n_sm < 1 || n_sm > kMaxPlanSms)
         return MK_ERR_INVALID_ARG;
-    if (stage_bytes == 0) stage_bytes = default_stage_bytes(L);
-    if (stage_bytes % 128 || stage_bytes < default_stage_bytes(L)) return MK_ERR_INVALID_ARG;
-    const SlotPlan sp = slot_plan(L, batch, stage_bytes);
+    if (o.proj < MK_PROJ_AUTO || o.proj > MK_PROJ_TENSOR_CORES) return MK_ERR_INVALID_ARG;
+    const bool mma = use_mma(batch, &o);
+    if (stage_bytes == 0) stage_bytes = default_stage_bytes(L, mma);
+    if (stage_bytes % (mma ? 1024 : 128) || stage_bytes < default_stage_bytes(L, mma)) return MK_ERR_INVALID_ARG;
+    const SlotPlan sp = slot_plan(L, batch, stage_bytes, mma);
     const int kps = sp.keys_per_stage;
     if (kps < 1 || sp.stages < kMoveWarps) return MK_ERR_UNSUPPORTED;
     // the attention value phase splits an item's keys into classes j mod KQ
@@ -319,6 +336,8 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         uint32_t seq = 0;
         for (mk_instr in : lists[s]) {
             if (in.wait_ctr != MK_NO_COUNTER) in.wait_n = signals[in.wait_ctr];
+            if (mma && in.op != MK_OP_ATTN)  // the same rows, streamed as 64-column boxes
+                in.nfill = mma_geom(in.op, in.count, in.aux0, L.H, L.Q, L.F, stage_bytes).nfill();
             in.seq = seq;
             seq += in.nfill;
             P.instrs.push_back(in);
@@ -354,11 +373,12 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     uint64_t bytes = 0;
     for (const mk_instr& in : P.instrs) {
         if (in.op == MK_OP_ATTN) bytes += (uint64_t)in.count * kv_key_bytes;
-        else if (in.op == MK_OP_DOWN) bytes += (uint64_t)in.nfill * L.tile_f;
+        else if (in.op == MK_OP_DOWN) bytes += 4ull * in.count * L.tile_f;
         else if (in.op == MK_OP_OPROJ) bytes += (uint64_t)in.count * L.tile_o;
         else bytes += (uint64_t)in.count * L.tile_h;
     }
     I.bytes_per_step = bytes;
+    I.proj = mma ? MK_PROJ_TENSOR_CORES : MK_PROJ_CUDA_CORES;
     I.max_sm_bytes = *std::max_element(load.begin(), load.end());
     I.min_sm_bytes = *std::min_element(load.begin(), load.end());
     (void)total;

@@ -56,7 +56,9 @@ def test_llama1b_greedy_256_after_32_token_prompt(w1b):
 
 def test_3b_shape_batch8_full_depth():
     """All 28 layers of the 3B-style shape at batch 8, every sequence with 2048
-    cached positions; the megakernel and the multi-kernel baseline agree bit for bit."""
+    cached positions, on the tensor-core path (the default) and the CUDA-core path
+    against the oracle; the CUDA-core megakernel and the multi-kernel baseline agree
+    bit for bit."""
     past = [2048] * 8
     c = Case(LLAMA_3B, batch=8, max_seq=2049, past=past, seed=60)
     c.mk.build_schedule(8, 2049)
@@ -66,6 +68,12 @@ def test_3b_shape_batch8_full_depth():
     ref, kc, vc = c.oracle_step(toks, past)
     assert_logits_close(gpu, ref, past)
     assert_kv_ok(c, kc, vc, past)
+    # the CUDA-core path: within the same bars, and bit for bit the baseline's
     c.reset_kv()
-    assert np.array_equal(c.gpu_step(toks, past, baseline=True), gpu)
+    c.mk.build_schedule(8, 2049, proj=1)
+    cc = c.gpu_step(toks, past)
+    assert c.mk.status()[0] == 0
+    assert_logits_close(cc, ref, past)
+    c.reset_kv()
+    assert np.array_equal(c.gpu_step(toks, past, baseline=True), cc)
     c.mk.close()

@@ -172,11 +172,16 @@ def test_tiny_step_matches_oracle(tiny):
 
 
 def test_megakernel_equals_baseline_bit_for_bit(tiny):
+    """The megakernel on the CUDA cores and the multi-kernel baseline share every
+    order of arithmetic (the tensor-core path accumulates in its own order: it is
+    held to the oracle instead, test_gpu_mma.py)."""
     toks = make_tokens(TINY, 2, seed=3).numpy()
     pos = [100, 3]
+    tiny.mk.build_schedule(2, 160, proj=1)
     a = tiny.gpu_step(toks, pos)
     ka, va = _bits(tiny.kd), _bits(tiny.vd)
     b = tiny.gpu_step(toks, pos, baseline=True)
+    tiny.mk.build_schedule(2, 160)
     assert tiny.mk.status()[0] == 0
     assert np.array_equal(a, b)
     assert np.array_equal(ka, _bits(tiny.kd)) and np.array_equal(va, _bits(tiny.vd))
@@ -302,7 +307,14 @@ def test_3b_shape_batch8_two_layers():
     assert c.mk.status()[0] == 0
     assert_logits_close(gpu, ref, past)
     assert_kv_ok(c, kc, vc, past)
-    assert np.array_equal(c.gpu_step(toks, past, baseline=True), gpu)
+    # the CUDA-core path: the oracle's bars too, and the baseline's bits
+    c.reset_kv()
+    c.mk.build_schedule(8, 2049, proj=1)
+    cc = c.gpu_step(toks, past)
+    assert c.mk.status()[0] == 0
+    assert_logits_close(cc, ref, past)
+    c.reset_kv()
+    assert np.array_equal(c.gpu_step(toks, past, baseline=True), cc)
     c.mk.close()
 
 

@@ -185,7 +185,173 @@ def simulate(instrs, offs, n_counters, S, NS=2, group=1, n_parts=1, NT=16, batch
     return ok, ctr
 
 
+# ---- the tensor-core path (batch > 1): fill geometry and protocol
+
+def mma_geom(ins, cfg, stage_bytes):
+    """Fills of a matvec instruction on the tensor-core path (restated from the
+    library's header): rows cut into segments of <= 128 per range (gate/up: one range
+    per MLP chunk), each streamed as 64-column boxes, nb boxes a fill."""
+    jobs, nrange, rows, k64 = 1, 1, 4 * ins.count, cfg.hidden // 64
+    if ins.op == _lib.OP_OPROJ:
+        k64 = cfg.n_heads * cfg.head_dim // 64
+    elif ins.op == _lib.OP_DOWN:
+        k64, jobs = cfg.ffn // 4 // 64, 4
+    elif ins.op == _lib.OP_GATEUP:
+        rows, nrange = 4 * ins.aux0, 4
+    segs = -(-rows // 128)
+    r8 = (rows + 7) // 8 * 8 if rows < 128 else 128
+    nb = max(1, min(k64, stage_bytes // (r8 * 128)))
+    fps = -(-k64 // nb)
+    return dict(jobs=jobs, nrange=nrange, rows=rows, k64=k64, segs=segs, r8=r8, nb=nb, fps=fps)
+
+
+def mma_fills(ins, cfg, stage_bytes):
+    """Per fill t of the instruction: (job c, range, segment, K boxes, segment rows)."""
+    g = mma_geom(ins, cfg, stage_bytes)
+    per = g["nrange"] * g["segs"] * g["fps"]
+    out = []
+    for t in range(g["jobs"] * per):
+        c, r = divmod(t, per)
+        rg, seg, kf = r // (g["segs"] * g["fps"]), (r // g["fps"]) % g["segs"], r % g["fps"]
+        boxes = range(kf * g["nb"], min(kf * g["nb"] + g["nb"], g["k64"]))
+        out.append((c, rg, seg, boxes, min(128, g["rows"] - 128 * seg)))
+    return g, out
+
+
+def simulate_mma(instrs, offs, n_counters, S, NS, group, n_parts, cfg, stage_bytes, n_acc=32):
+    """The tensor-core protocol: the loader as above; an activation warp preparing
+    each job once its slot is free and its counters are met; the compute warps (as
+    one) writing a matvec job's operand, then reading out each of its segments'
+    accumulators once final (the down-projection: after its last chunk), then
+    waiting for the job's MMAs before freeing the slot; an attention item as
+    above; the issuer walking the jobs in order, each once its operand is written:
+    each fill once it has landed and, for a segment's first fill, once the
+    segment n_acc earlier (same accumulator) has been read out; the fill's MMAs
+    free its stage, a segment's last fill makes its accumulator final, a job's
+    last marks the job's MMAs done."""
+    n_sm = len(offs) - 1
+    ctr = [0] * n_counters
+    arr = collections.Counter()
+    ok_all = True
+    lists = [instrs[offs[s]:offs[s + 1]] for s in range(n_sm)]
+    jobs = [jobs_of(L) for L in lists]
+    # per SM: each job's fills (seq, segment number, first of segment, last of segment)
+    # and the segments its epilogue reads
+    plan = []
+    for L, J in zip(lists, jobs):
+        sn0, per_job, reads = 0, [], []
+        for (i, c, items) in J:
+            ins = L[i]
+            if ins.op == _lib.OP_ATTN:
+                per_job.append(None)
+                reads.append([])
+                continue
+            g, fl = mma_fills(ins, cfg, stage_bytes)
+            per = len(fl) // g["jobs"]
+            mine = []
+            for r in range(per):
+                cc, rg, seg, boxes, rows = fl[c * per + r]
+                assert cc == c
+                kf = r % g["fps"]
+                sn = sn0 + rg * g["segs"] + seg
+                mine.append((ins.seq + c * per + r, sn, c == 0 and kf == 0,
+                             c == g["jobs"] - 1 and kf == g["fps"] - 1))
+            per_job.append(mine)
+            reads.append([sn0 + k for k in range(g["nrange"] * g["segs"])] if c == g["jobs"] - 1 else [])
+            if c == g["jobs"] - 1:
+                sn0 += g["nrange"] * g["segs"]
+        plan.append((per_job, reads))
+    total = [sum(ins.nfill for ins in L) for L in lists]
+    kv_of = []
+    for L, J in zip(lists, jobs):
+        kv_of.append([job_fills(L, job)[1] for job in J])
+    n_iss = [0] * n_sm
+    issued = [bytearray(t) for t in total]
+    freed = [bytearray(t) for t in total]
+    prepared = [0] * n_sm
+    opnd = [bytearray(len(J)) for J in jobs]
+    mdone = [bytearray(len(J)) for J in jobs]
+    afull, aread = [set() for _ in range(n_sm)], [set() for _ in range(n_sm)]
+    done = [bytearray(len(J)) for J in jobs]
+    ij, ip = [0] * n_sm, [0] * n_sm     # issuer: job, fill within it
+    cj, cr = [0] * n_sm, [0] * n_sm     # compute warps: job, segments read in it
+    changed = True
+    while changed:
+        changed = False
+        for s in range(n_sm):
+            L, J = lists[s], jobs[s]
+            per_job, reads = plan[s]
+            while True:
+                f = n_iss[s]
+                if f >= total[s] or (f >= S and not freed[s][f - S]):
+                    break
+                issued[s][f] = 1
+                n_iss[s] += 1
+                changed = True
+            while prepared[s] < len(J):
+                j = prepared[s]
+                if j >= NS and not done[s][j - NS]:
+                    break
+                if any(ctr[c] < t for c, t in job_waits(L, J[j])):
+                    break
+                prepared[s] += 1
+                changed = True
+            while ij[s] < len(J):  # the issuer
+                j = ij[s]
+                if per_job[j] is None:
+                    ij[s] += 1
+                    changed = True
+                    continue
+                if not opnd[s][j]:
+                    break
+                if ip[s] < len(per_job[j]):
+                    f, sn, first, last = per_job[j][ip[s]]
+                    if first and sn >= n_acc and (sn - n_acc) not in aread[s]:
+                        break
+                    if not issued[s][f]:
+                        break
+                    freed[s][f] = 1
+                    if last:
+                        afull[s].add(sn)
+                    ip[s] += 1
+                    changed = True
+                    continue
+                mdone[s][j] = 1
+                ij[s] += 1
+                ip[s] = 0
+                changed = True
+            while cj[s] < len(J) and cj[s] < prepared[s]:  # the compute warps
+                j = cj[s]
+                if per_job[j] is None:
+                    if not all(issued[s][f] for f in kv_of[s][j]):
+                        break
+                    for f in kv_of[s][j]:
+                        freed[s][f] = 1
+                else:
+                    opnd[s][j] = 1
+                    if cr[s] < len(reads[j]):
+                        sn = reads[j][cr[s]]
+                        if sn not in afull[s]:
+                            break
+                        aread[s].add(sn)
+                        cr[s] += 1
+                        changed = True
+                        continue
+                    if not mdone[s][j]:
+                        break
+                done[s][j] = 1
+                job_done_signals(L, J[j], group, n_parts, arr, ctr)
+                cj[s] += 1
+                cr[s] = 0
+                changed = True
+        ok_all = all(all(d for d in dj) for dj in done)
+    return ok_all, ctr
+
+
 def sim(instrs, offs, info, ns, cfg):
+    if info.proj == _lib.PROJ_TENSOR_CORES:
+        return simulate_mma(instrs, offs, info.n_counters, info.n_stages, ns, cfg.group, info.n_parts, cfg,
+                            info.stage_bytes)
     return simulate(instrs, offs, info.n_counters, info.n_stages, ns, cfg.group, info.n_parts,
                     NT=tmem_slots(info.stage_bytes), batched=info.batch > 1)
 
@@ -264,12 +430,16 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
     return instrs, offs, info
 
 
-@pytest.mark.parametrize("cfg,batch,ctx,n_sm", [
-    (TINY, 1, 129, 148), (TINY, 2, 200, 37), (TINY, 3, 64, 7), (TINY, 1, 1, 148),
-    (LLAMA_1B, 1, 129, 148), (LLAMA_1B, 1, 8193, 148), (LLAMA_3B, 8, 2049, 148),
+@pytest.mark.parametrize("cfg,batch,ctx,n_sm,proj", [
+    (TINY, 1, 129, 148, 0), (TINY, 2, 200, 37, 0), (TINY, 2, 200, 37, 1), (TINY, 3, 64, 7, 0),
+    (TINY, 3, 64, 7, 1), (TINY, 1, 1, 148, 0), (LLAMA_1B, 1, 129, 148, 0), (LLAMA_1B, 1, 8193, 148, 0),
+    (LLAMA_3B, 8, 2049, 148, 0), (LLAMA_3B, 8, 2049, 148, 1),
 ])
-def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm):
-    instrs, offs, info = check_plan(cfg, batch, ctx, n_sm)
+def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm, proj):
+    """Both projection paths at batch > 1 (proj 0: the default, tensor cores; 1:
+    CUDA cores)."""
+    instrs, offs, info = check_plan(cfg, batch, ctx, n_sm, proj=proj)
+    assert info.proj == (_lib.PROJ_TENSOR_CORES if batch > 1 and proj != 1 else _lib.PROJ_CUDA_CORES)
     for ns in (1, 2, 3):
         ok, ctr = sim(instrs, offs, info, ns, cfg)
         assert ok, "simulated step did not complete"
@@ -350,7 +520,7 @@ def test_down_instructions_cover_row_block_ranges(cfg, batch):
     """Down-projection instructions take contiguous ranges of up to 16 row blocks
     at every batch size (each chunk's input is loaded once per instruction), and
     together cover every row block of every layer exactly once."""
-    instrs, offs, _ = plan_schedule(cfg, batch, 129, 148, max_batch=8, max_seq=129)
+    instrs, offs, _ = plan_schedule(cfg, batch, 129, 148, max_batch=8, max_seq=129, proj=1)
     for layer in range(cfg.n_layers):
         seen = []
         for ins in instrs:
@@ -427,14 +597,60 @@ def test_plan_valid_across_batches_contexts_and_sm_counts(cfg, batch, ctx, n_sm)
     assert ok, "simulated step did not complete"
 
 
-@pytest.mark.parametrize("cfg,batch,limit", [
-    (LLAMA_1B, 1, 16384), (LLAMA_1B, 4, 16384), (LLAMA_1B, 8, 16384),
-    (LLAMA_3B, 1, 12288), (LLAMA_3B, 2, 12288), (LLAMA_3B, 4, 6144), (LLAMA_3B, 8, 6144),
+@pytest.mark.parametrize("cfg,batch,proj,limit", [
+    (LLAMA_1B, 1, 0, 16384), (LLAMA_1B, 4, 0, 16384), (LLAMA_1B, 8, 0, 16384), (LLAMA_1B, 8, 1, 16384),
+    (LLAMA_3B, 1, 0, 12288), (LLAMA_3B, 2, 0, 7680), (LLAMA_3B, 5, 0, 7680), (LLAMA_3B, 6, 0, 6144),
+    (LLAMA_3B, 8, 0, 6144), (LLAMA_3B, 2, 1, 12288), (LLAMA_3B, 3, 1, 6144), (LLAMA_3B, 8, 1, 6144),
 ])
-def test_context_ceiling_is_the_documented_one(cfg, batch, limit):
+def test_context_ceiling_is_the_documented_one(cfg, batch, proj, limit):
     """The largest max_ctx the planner accepts (32 partitions of at most one ring's
     keys, and 512) is the one the header states; one key more is refused."""
-    _, _, info = plan_schedule(cfg, batch, limit, 148, max_batch=8, max_seq=limit + 1)
+    _, _, info = plan_schedule(cfg, batch, limit, 148, max_batch=8, max_seq=limit + 1, proj=proj)
     assert info.n_parts <= 32 and info.n_parts * info.part_keys >= limit
     with pytest.raises(_lib.MkError):
-        plan_schedule(cfg, batch, limit + 1, 148, max_batch=8, max_seq=limit + 1)
+        plan_schedule(cfg, batch, limit + 1, 148, max_batch=8, max_seq=limit + 1, proj=proj)
+
+
+@pytest.mark.parametrize("cfg,batch,n_sm", [(TINY, 2, 37), (TINY, 8, 148), (LLAMA_1B, 8, 148),
+                                            (LLAMA_3B, 8, 148), (LLAMA_3B, 3, 100)])
+def test_tensor_core_fills_cover_every_weight_once(cfg, batch, n_sm):
+    """On the tensor-core path every matvec instruction's fills (64-column boxes of
+    <= 128-row segments, nb boxes a fill) cover each (row, 64-column block) of its
+    weight rows exactly once, each fill fits one ring stage, the box pieces (the
+    segment's rows in binary: 128, 64, ..., 4) start on 8-row (1024-byte)
+    boundaries, and the planner's fill counts are these. The bytes streamed are
+    the CUDA-core path's, row for row."""
+    instrs, offs, info = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129)
+    assert info.proj == _lib.PROJ_TENSOR_CORES
+    _, _, info_cc = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129, proj=1)
+    assert info.bytes_per_step == info_cc.bytes_per_step
+    sb = info.stage_bytes
+    assert sb % 1024 == 0
+    cov = collections.Counter()
+    for ins in instrs:
+        if ins.op == _lib.OP_ATTN:
+            continue
+        g, fills = mma_fills(ins, cfg, sb)
+        assert ins.nfill == len(fills)
+        for c, rg, seg, boxes, rows in fills:
+            assert len(boxes) * g["r8"] * 128 <= sb and 4 <= rows <= 128 and rows % 4 == 0
+            ro = 0
+            for hk in range(5, -1, -1):
+                if rows & (4 << hk):
+                    assert ro % 8 == 0
+                    ro += 4 << hk
+            assert ro == rows
+            if ins.op == _lib.OP_GATEUP:
+                row0 = 4 * (rg * (cfg.ffn // 8) + ins.first)
+            else:
+                row0 = 4 * ins.first
+            row0 += 128 * seg
+            for r in range(row0, row0 + rows):
+                for bx in boxes:
+                    cov[(ins.op, ins.layer, c, r, bx)] += 1
+    assert all(v == 1 for v in cov.values())
+    k_h, k_o, k_f = cfg.hidden // 64, cfg.n_heads * cfg.head_dim // 64, cfg.ffn // 4 // 64
+    qkv_rows = (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    want = cfg.n_layers * (qkv_rows * k_h + cfg.hidden * k_o + 2 * cfg.ffn * k_h + 4 * cfg.hidden * k_f) \
+        + cfg.vocab * k_h
+    assert len(cov) == want
