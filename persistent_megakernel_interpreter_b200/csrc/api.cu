@@ -45,6 +45,7 @@ struct mk_handle {
     uint8_t* packed = nullptr;
     float* rope = nullptr;          // cos table then sin table
     void* d_tmaps = nullptr;        // tensor maps of the packed weights (tensor-core path)
+    uint32_t tmap_stage_bytes = 0;  // the ring stage size they were built for
     // scratch (sized by mk_build_schedule)
     void* scratch = nullptr;
     size_t scratch_bytes = 0;
@@ -220,14 +221,18 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
     return no_throw([&] { return create_impl(cfg, w, device, out); });
 }
 
-// Tensor maps of the packed weights for the tensor-core path, one per (matrix,
-// box height 4 << k rows), all boxes 64 bf16 columns wide with the 128-byte
-// swizzle that the MMA's shared-memory descriptors read. Built once per handle.
-//   QKV / O / gate-up: {K, rows, layer}; LM head (the embedding rows): {K, rows};
-//   down: {ffn/4, 4 rows, 4 chunks, hidden/4 row blocks, layer}, a box of
-//   {64, 4, 1, 1 << k, 1} (the row blocks' rows of one chunk).
-static mk_status make_tmaps(mk_handle* h) {
-    if (h->d_tmaps) return MK_OK;
+// Tensor maps of the packed weights for the tensor-core path: one per (matrix,
+// segment rows R = 8, 16, ..., 128), whose box is one fill of such a segment:
+// {64 columns, R rows, nb(R) 64-column blocks}, landing as nb boxes of R rows x
+// 128 bytes side by side, in the 128-byte swizzle the MMA's shared-memory
+// descriptors read. The K dimension is split into (64, K / 64) so that one copy
+// takes several boxes; a fill past the end of K reads zeros there (never used).
+//   QKV / O / gate-up: {64, rows, K / 64, layer}; LM head (the embedding rows):
+//   {64, rows, K / 64}; down chunk c: {64, 4 rows of a block, hidden / 4 row
+//   blocks, (ffn / 4) / 64, layer}, R <= 64.
+// nb depends on the ring's stage size, so the maps are rebuilt when it changes.
+static mk_status make_tmaps(mk_handle* h, uint32_t stage_bytes) {
+    if (h->d_tmaps && h->tmap_stage_bytes == stage_bytes) return MK_OK;
     typedef CUresult (*Encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -238,60 +243,67 @@ static mk_status make_tmaps(mk_handle* h) {
         h->msg = "cuTensorMapEncodeTiled is not available";
         return MK_ERR_UNSUPPORTED;
     }
+    static_assert(sizeof(CUtensorMap) == mk::kTmBytes, "tensor map size");
     const Encode encode = reinterpret_cast<Encode>(fn);
     const mk::Layout& L = h->lay;
-    std::vector<CUtensorMap> maps((size_t)mk::kTmKinds * mk::kBoxHeights);
+    std::vector<CUtensorMap> maps((size_t)mk::kTmCount);
     memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
     const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
-    auto enc = [&](int kind, int hk, uint8_t* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+    auto enc = [&](int idx, uint8_t* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
                    const cuuint32_t* box) {
-        const CUresult r = encode(&maps[(size_t)kind * mk::kBoxHeights + hk], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                                  (cuuint32_t)rank, base, dims, strides, box, unit, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        const CUresult r = encode(&maps[(size_t)idx], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, base, dims,
+                                  strides, box, unit, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         return r == CUDA_SUCCESS;
     };
     uint8_t* pk = h->packed;
     const cuuint64_t ls = (cuuint64_t)L.layer_stride;
+    const uint32_t kh = (uint32_t)L.H / mk::kBoxK, kq = (uint32_t)L.Q / mk::kBoxK, kf = (uint32_t)(L.F / 4) / mk::kBoxK;
     bool ok = true;
-    for (int hk = 0; hk < mk::kBoxHeights && ok; ++hk) {
-        const cuuint32_t rows = 4u << hk;
-        const cuuint32_t box3[3] = {mk::kBoxK, rows, 1};
+    for (int hk = 0; hk < mk::kTmPerKind && ok; ++hk) {
+        const cuuint32_t R = 8u * (cuuint32_t)(hk + 1);
         {
-            const cuuint64_t dims[3] = {(cuuint64_t)L.H, (cuuint64_t)L.qkv_rows, (cuuint64_t)L.L};
-            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, ls};
-            ok = ok && enc(mk::kTmQKV, hk, pk + L.off_layer0 + L.rel_qkv, 3, dims, st, box3);
+            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)L.qkv_rows, kh, (cuuint64_t)L.L};
+            const cuuint64_t st[3] = {(cuuint64_t)L.H * 2, 128, ls};
+            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes), 1};
+            ok = ok && enc(mk::kTmQKV * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_qkv, 4, dims, st, box);
         }
         {
-            const cuuint64_t dims[3] = {(cuuint64_t)L.Q, (cuuint64_t)L.H, (cuuint64_t)L.L};
-            const cuuint64_t st[2] = {(cuuint64_t)L.Q * 2, ls};
-            ok = ok && enc(mk::kTmO, hk, pk + L.off_layer0 + L.rel_o, 3, dims, st, box3);
+            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)L.H, kq, (cuuint64_t)L.L};
+            const cuuint64_t st[3] = {(cuuint64_t)L.Q * 2, 128, ls};
+            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kq, stage_bytes), 1};
+            ok = ok && enc(mk::kTmO * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_o, 4, dims, st, box);
         }
         {
-            const cuuint64_t dims[3] = {(cuuint64_t)L.H, (cuuint64_t)(2 * L.F), (cuuint64_t)L.L};
-            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, ls};
-            ok = ok && enc(mk::kTmGU, hk, pk + L.off_layer0 + L.rel_gu, 3, dims, st, box3);
+            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)(2 * L.F), kh, (cuuint64_t)L.L};
+            const cuuint64_t st[3] = {(cuuint64_t)L.H * 2, 128, ls};
+            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes), 1};
+            ok = ok && enc(mk::kTmGU * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_gu, 4, dims, st, box);
         }
         {
-            const cuuint64_t dims[2] = {(cuuint64_t)L.H, (cuuint64_t)L.V};
-            const cuuint64_t st[1] = {(cuuint64_t)L.H * 2};
-            const cuuint32_t box2[2] = {mk::kBoxK, rows};
-            ok = ok && enc(mk::kTmLM, hk, pk + L.off_embed, 2, dims, st, box2);
+            const cuuint64_t dims[3] = {mk::kBoxK, (cuuint64_t)L.V, kh};
+            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, 128};
+            const cuuint32_t box[3] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes)};
+            ok = ok && enc(mk::kTmLM * mk::kTmPerKind + hk, pk + L.off_embed, 3, dims, st, box);
         }
-        if (hk < 5) {  // down: at most 16 row blocks (64 rows) per instruction
+        if (R <= 64) {
             const cuuint64_t f4 = (cuuint64_t)(L.F / 4);
-            const cuuint64_t dims[5] = {f4, 4, 4, (cuuint64_t)(L.H / 4), (cuuint64_t)L.L};
-            const cuuint64_t st[4] = {f4 * 2, f4 * 2 * 4, f4 * 2 * 16, ls};
-            const cuuint32_t box5[5] = {mk::kBoxK, 4, 1, 1u << hk, 1};
-            ok = ok && enc(mk::kTmDown, hk, pk + L.off_layer0 + L.rel_down, 5, dims, st, box5);
+            for (int c = 0; c < 4 && ok; ++c) {
+                const cuuint64_t dims[5] = {mk::kBoxK, 4, (cuuint64_t)(L.H / 4), kf, (cuuint64_t)L.L};
+                const cuuint64_t st[4] = {f4 * 2, f4 * 2 * 16, 128, ls};
+                const cuuint32_t box[5] = {mk::kBoxK, 4, R / 4, mk::mma_nb(R, kf, stage_bytes), 1};
+                ok = ok && enc(mk::kTmDown0 + c * 8 + hk, pk + L.off_layer0 + L.rel_down + (size_t)c * f4 * 2 * 4, 5,
+                               dims, st, box);
+            }
         }
     }
     if (!ok) {
         h->msg = "cuTensorMapEncodeTiled refused a weight tensor map";
         return MK_ERR_UNSUPPORTED;
     }
-    MK_CUDA(h, cudaMalloc(&h->d_tmaps, maps.size() * sizeof(CUtensorMap)));
+    if (!h->d_tmaps) MK_CUDA(h, cudaMalloc(&h->d_tmaps, maps.size() * sizeof(CUtensorMap)));
     MK_CUDA(h, cudaMemcpy(h->d_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    h->tmap_stage_bytes = stage_bytes;
     return MK_OK;
 }
 
@@ -311,7 +323,7 @@ static mk_status build_schedule_impl(mk_handle* h, int batch, int max_ctx, const
     const bool mma = P.info.proj == MK_PROJ_TENSOR_CORES;
     MK_CUDA(h, cudaDeviceSynchronize());
     if (mma) {
-        st = make_tmaps(h);
+        st = make_tmaps(h, (uint32_t)P.info.stage_bytes);
         if (st != MK_OK) return st;
     }
     free_schedule(h);

@@ -161,9 +161,10 @@ struct Tmem {
 // ------------------------------------------------------------------ tensor-core MMA (batch > 1)
 //
 // On the tensor-core path Tensor Memory holds fp32 accumulators instead of weight
-// tiles: accumulator a is columns a * 16 .. +15 of all 128 lanes, lane m the
-// segment's row m, column n the input row n (sequence n's high bf16 part for
-// n < 8, sequence n - 8's low part above).
+// tiles: segment accumulator a is columns a * 64 .. +63 of all 128 lanes, four
+// partial sums u of 16 columns; lane m is the segment's row m, column u * 16 + n
+// the input row n (sequence n's high bf16 part for n < 8, sequence n - 8's low
+// part above).
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
 // (8-row atoms of 128-byte rows, atoms 1024 bytes apart): start address >> 4
@@ -256,7 +257,8 @@ __device__ __forceinline__ bool aborted(const Params& p) {
 // issue slots with the warps that compute. Out of line: the inline wait_bar
 // below tries once first.
 __device__ __noinline__ bool wait_bar_slow(const Params& p, uint64_t* bar, uint32_t parity,
-                                           const volatile uint32_t* armed, uint32_t seq, uint32_t site, int lane) {
+                                           const volatile uint32_t* armed, uint32_t seq, uint32_t site, int lane,
+                                           uint32_t sleep_ns) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         bool done;
@@ -264,7 +266,7 @@ __device__ __noinline__ bool wait_bar_slow(const Params& p, uint64_t* bar, uint3
             __nanosleep(64);
             done = false;
         } else {
-            done = mbar_wait_sleep(bar, parity, 20000u);
+            done = mbar_wait_sleep(bar, parity, sleep_ns);
         }
         if (__all_sync(0xffffffffu, done)) return true;
         if ((it & 15u) == 15u) {
@@ -282,11 +284,17 @@ __device__ __noinline__ bool wait_bar_slow(const Params& p, uint64_t* bar, uint3
     }
 }
 
+// The sleep hint bounds how long a waiting thread stays suspended; a phase that
+// completes by a thread's arrival or a copy's bytes wakes it at once.
+constexpr uint32_t kSleepNs = 20000u;
+// Phases completed by tcgen05.commit: waiters poll with a short hint instead.
+constexpr uint32_t kCommitSleepNs = 256u;
+
 __device__ __forceinline__ bool wait_bar(const Params& p, uint64_t* bar, uint32_t parity, const volatile uint32_t* armed,
-                                         uint32_t seq, uint32_t site, int lane) {
+                                         uint32_t seq, uint32_t site, int lane, uint32_t sleep_ns = kSleepNs) {
     const bool ready = (armed == nullptr || *armed == seq) && mbar_try_wait(bar, parity);
     if (__all_sync(0xffffffffu, ready)) return true;
-    return wait_bar_slow(p, bar, parity, armed, seq, site, lane);
+    return wait_bar_slow(p, bar, parity, armed, seq, site, lane, sleep_ns);
 }
 
 __device__ __forceinline__ bool wait_fill(const Params& p, const Ring& r, uint32_t seq, int lane) {
@@ -1055,12 +1063,30 @@ __device__ bool mma_job(const Params& p, const MmaBars& mb, uint32_t tbase, cons
     for (uint32_t rg = 0; rg < g.nrange; ++rg) {
         for (uint32_t sgi = 0; sgi < g.segs; ++sgi) {
             const uint32_t sn = sg + rg * g.segs + sgi, a = sn % (uint32_t)kMaxAcc;
-            if (!wait_bar(p, mb.afull + a, (sn / (uint32_t)kMaxAcc) & 1u, nullptr, sn, 13, lane)) return false;
+            if (!wait_bar(p, mb.afull + a, (sn / (uint32_t)kMaxAcc) & 1u, nullptr, sn, 13, lane, kCommitSleepNs))
+                return false;
             if (rg == 0 && sgi == 0 && warp == 0 && lane == 0) trace(p, job, kTrFill);
             tmem_fence_after();
-            uint32_t d[16];
-            tmem_ld16(tbase + ((32u * q) << 16) + a * kAccCols, d);
-            tmem_wait_ld(d);
+            // the warp's sequences' high and low sums over the partial sums, in order
+            float shi[4] = {0.f, 0.f, 0.f, 0.f}, slo[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+            for (uint32_t u = 0; u < kSubAcc; ++u) {
+                uint32_t d[16];
+                tmem_ld16(tbase + ((32u * q) << 16) + (a * kSubAcc + u) * kAccCols, d);
+                tmem_wait_ld(d);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    float hi = 0.f, lo = 0.f;
+#pragma unroll
+                    for (int b = 0; b < kMaxBatch; ++b)
+                        if (b == ps.b0 + bb) {
+                            hi = __uint_as_float(d[b]);
+                            lo = __uint_as_float(d[kMaxBatch + b]);
+                        }
+                    shi[bb] = __fadd_rn(shi[bb], hi);
+                    slo[bb] = __fadd_rn(slo[bb], lo);
+                }
+            }
             tmem_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(mb.aempty + a);
@@ -1072,16 +1098,7 @@ __device__ bool mma_job(const Params& p, const MmaBars& mb, uint32_t tbase, cons
             // the warp's sequences' totals, high + low (register indices fixed at compile time)
             float y[4];
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                float hi = 0.f, lo = 0.f;
-#pragma unroll
-                for (int b = 0; b < kMaxBatch; ++b)
-                    if (b == ps.b0 + bb) {
-                        hi = __uint_as_float(d[b]);
-                        lo = __uint_as_float(d[kMaxBatch + b]);
-                    }
-                y[bb] = __fadd_rn(hi, lo);
-            }
+            for (int bb = 0; bb < 4; ++bb) y[bb] = __fadd_rn(shi[bb], slo[bb]);
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
                 if (bb < ps.nb) {  // warp-uniform
@@ -1276,7 +1293,7 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(mb.opnd + s);
                 ok = mma_job<HD>(p, mb, tm.base, in, c, sg, sv, warp, lane, j, epoch, selp) &&
-                     wait_bar(p, mb.mdone + s, (ph >> s) & 1u, nullptr, j, 12, lane);
+                     wait_bar(p, mb.mdone + s, (ph >> s) & 1u, nullptr, j, 12, lane, kCommitSleepNs);
                 ph ^= 1u << s;
             } else if (in.op == MK_OP_DOWN) {
                 if constexpr (BATCHED) ok = compute_down_pair<KF>(p, tm, in, c, sv, tot, warp, lane, j, epoch);
@@ -1383,107 +1400,119 @@ __device__ __forceinline__ void fill_seek(const Params& p, FillCur& c, int i1) {
     while (c.i < i1 && c.seq >= p.instrs[c.i].seq + p.instrs[c.i].nfill) ++c.i;
 }
 
-// The tensor map of weight matrix `kind` whose boxes are 4 << hk rows high.
-__device__ __forceinline__ const void* tmap(const Params& p, int kind, int hk) {
-    return static_cast<const uint8_t*>(p.tmaps) + (size_t)(kind * kBoxHeights + hk) * 128u;
+// Tensor-core path: the segments of a matvec instruction in fill order -- job
+// (the down-projection's chunk), range, segment -- each with its rows, its first
+// row in the matrix's packed row order, its boxes per fill, fills and tensor map.
+// The loader and the issuer walk the same sequence.
+struct MmaSeg {
+    uint32_t rows, row0, nb, fps;
+    const void* map;
+};
+__device__ __forceinline__ MmaSeg mma_seg(const Params& p, const mk_instr& in, const MmaGeom& g, uint32_t c,
+                                          uint32_t rg, uint32_t sgi) {
+    MmaSeg m;
+    const bool last = sgi + 1 == g.segs;
+    m.rows = last ? g.rows_l : kMmaRows;
+    m.nb = last ? g.nb_l : g.nb_f;
+    m.fps = last ? g.fps_l : g.fps_f;
+    const uint32_t hk = m.rows / 8u - 1u;
+    int idx;
+    switch (in.op) {
+        case MK_OP_QKV: idx = kTmQKV * kTmPerKind; m.row0 = 4u * in.first; break;
+        case MK_OP_OPROJ: idx = kTmO * kTmPerKind; m.row0 = 4u * in.first; break;
+        case MK_OP_GATEUP: idx = kTmGU * kTmPerKind; m.row0 = 4u * (rg * (uint32_t)(p.F / 8) + in.first); break;
+        case MK_OP_DOWN: idx = kTmDown0 + (int)c * 8; m.row0 = 4u * in.first; break;
+        default: idx = kTmLM * kTmPerKind; m.row0 = 4u * in.first; break;
+    }
+    m.row0 += sgi * kMmaRows;
+    m.map = static_cast<const uint8_t*>(p.tmaps) + (size_t)(idx + (int)hk) * kTmBytes;
+    return m;
 }
 
-// Tensor-core path: fill t of matvec instruction `in` into the stage at dst. The
-// fill is K-boxes [kf * nb, kf * nb + nb) of one segment (fewer at the end of K),
-// box i of the fill at i * r8 rows into the stage; each box is assembled from
-// TMA boxes of 128, 64, ..., 4 rows (the segment's row count in binary, larger
-// first, so every piece starts on a 1024-byte boundary of the swizzle).
-__device__ void issue_mma_fill(const Params& p, const mk_instr& in, uint32_t t, uint8_t* dst, uint64_t* bar,
-                               uint64_t pol) {
-    const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
-    const uint32_t per = g.per_job();
-    const uint32_t c = t / per;
-    const MmaFill f = mma_fill(g, t % per);
-    const uint32_t b0 = f.kf * g.nb, b1 = min(b0 + g.nb, g.k64);
-    mbar_arrive_expect_tx(bar, (b1 - b0) * f.rows * 128u);
-    int kind;
-    uint32_t row0;  // the segment's first row in the matrix's packed row order
-    switch (in.op) {
-        case MK_OP_QKV: kind = kTmQKV; row0 = 4u * in.first; break;
-        case MK_OP_OPROJ: kind = kTmO; row0 = 4u * in.first; break;
-        case MK_OP_GATEUP: kind = kTmGU; row0 = 4u * (f.rg * (uint32_t)(p.F / 8) + in.first); break;
-        case MK_OP_DOWN: kind = kTmDown; row0 = 4u * in.first; break;
-        default: kind = kTmLM; row0 = 4u * in.first; break;
-    }
-    row0 += f.seg * kMmaRows;
-    for (uint32_t bx = b0; bx < b1; ++bx) {
-        uint8_t* bd = dst + (size_t)(bx - b0) * g.r8 * 128u;
-        const int k = (int)(bx * kBoxK);
-        uint32_t ro = 0;
-        for (int hk = kBoxHeights - 1; hk >= 0; --hk) {
-            const uint32_t h = 4u << hk;
-            if (!(f.rows & h)) continue;
-            const void* m = tmap(p, kind, hk);
-            const uint32_t row = row0 + ro;
-            if (kind == kTmDown)  // {col, row in block, chunk, row block, layer}
-                tma_load_5d(bd + ro * 128u, m, k, 0, (int)c, (int)(row / 4u), (int)in.layer, bar, pol);
-            else if (kind == kTmLM)
-                tma_load_2d(bd + ro * 128u, m, k, (int)row, bar, pol);
-            else
-                tma_load_3d(bd + ro * 128u, m, k, (int)row, (int)in.layer, bar, pol);
-            ro += h;
-        }
-    }
+// One fill of a segment: a single TMA copy of nb 64-column boxes from K-box kb0
+// (past the end of K the boxes read zeros, never used), landing as nb boxes of
+// the segment's rows side by side at dst.
+__device__ __forceinline__ void issue_mma_fill(const Params& p, const mk_instr& in, const MmaSeg& m, uint32_t kb0,
+                                               uint8_t* dst, uint64_t* bar, uint64_t pol) {
+    mbar_arrive_expect_tx(bar, m.nb * m.rows * 128u);
+    if (in.op == MK_OP_DOWN)  // {column, row in block, row block, K-box, layer}
+        tma_load_5d(dst, m.map, 0, 0, (int)(m.row0 / 4u), (int)kb0, (int)in.layer, bar, pol);
+    else if (in.op == MK_OP_LMHEAD)
+        tma_load_3d(dst, m.map, 0, (int)m.row0, (int)kb0, bar, pol);
+    else
+        tma_load_4d(dst, m.map, 0, (int)m.row0, (int)kb0, (int)in.layer, bar, pol);
 }
 
 // One thread (the loader warp's lane 0) streams the SM's fills into the ring, in
 // list order: weight tiles and the cached KV of attention items, all final at
 // launch. It never waits on a dependency counter, only for a stage to be free
-// again: moved to Tensor Memory by a mover warp (weights), or read by its
-// attention item (KV). So the next instructions' weights arrive while the step
-// still waits for their activations. It issues nothing else, so a freed stage is
-// refilled at once.
+// again: moved to Tensor Memory by a mover warp (weights), read by the tensor
+// cores (weights, tensor-core path) or read by its attention item (KV). So the
+// next instructions' weights arrive while the step still waits for their
+// activations. It issues nothing else, so a freed stage is refilled at once.
 template <bool MMA>
 __device__ void loader(const Params& p, const Ring& ring, int i0, int i1) {
     const uint64_t pol = l2_evict_first_policy();
     uint32_t issued = 0;  // fills issued so far (they are numbered 0, 1, 2, ...)
-    for (int i = i0; i < i1; ++i) {
+    uint32_t job0 = 0;    // the instruction's first job (trace)
+    // Waits until stage seq mod S is free for fill seq and arms it (bounded).
+    auto acquire = [&](uint32_t seq) {
+        const uint32_t s = seq % ring.S, use = seq / ring.S;
+        if (use > 0) {
+            uint64_t t0 = 0;
+            for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, MMA ? kCommitSleepNs : kSleepNs);
+                 ++it) {
+                if ((it & 15u) == 15u) {
+                    if (t0 == 0) t0 = global_timer_ns();
+                    if (aborted(p)) return false;
+                    if (global_timer_ns() - t0 > p.timeout_ns) {
+                        record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffdu, 0, use, 3);
+                        return false;
+                    }
+                }
+            }
+        }
+        ring.armed[s] = seq;  // published by the release of the fill's arrive
+        return true;
+    };
+    for (int i = i0; i < i1; job0 += p.instrs[i].op == MK_OP_DOWN ? 4u : 1u, ++i) {
         const mk_instr in = p.instrs[i];
-        for (uint32_t t = 0; t < in.nfill; ++t) {
-            const uint32_t seq = in.seq + t;
-            const uint32_t s = seq % ring.S, use = seq / ring.S;
-            if (use > 0) {
-                // wait for the compute warps to release the previous fill of this stage
-                uint64_t t0 = 0;
-                bool ok = true;
-                for (uint32_t it = 0; !mbar_wait_sleep(ring.empty + s, (use - 1) & 1u, 20000u); ++it) {
-                    if ((it & 15u) == 15u) {
-                        if (t0 == 0) t0 = global_timer_ns();
-                        if (aborted(p)) { ok = false; break; }
-                        if (global_timer_ns() - t0 > p.timeout_ns) {
-                            record_error(p, MK_ERR_TIMEOUT, seq, 0xfffffffdu, 0, use, 3);
-                            ok = false;
-                            break;
+        if (MMA && in.op != MK_OP_ATTN) {
+            const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
+            uint32_t seq = in.seq;
+            for (uint32_t c = 0; c < g.jobs; ++c) {
+                if (MK_TRACE) trace(p, job0 + c, kTrSub0 + 0);  // the job's first fill is issued next
+                for (uint32_t rg = 0; rg < g.nrange; ++rg)
+                    for (uint32_t sgi = 0; sgi < g.segs; ++sgi) {
+                        const MmaSeg m = mma_seg(p, in, g, c, rg, sgi);
+                        for (uint32_t kf = 0; kf < m.fps; ++kf, ++seq) {
+                            if (!acquire(seq)) goto drain;
+                            const uint32_t s = seq % ring.S;
+                            issue_mma_fill(p, in, m, kf * m.nb, ring.base + (size_t)s * ring.stage_bytes,
+                                           ring.full + s, pol);
+                            issued = seq + 1;
                         }
                     }
-                }
-                if (!ok) goto drain;
+                if (MK_TRACE) trace(p, job0 + c, kTrSub0 + 1);  // the job's last fill is issued
             }
-            {
-                uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
-                uint64_t* bar = ring.full + s;
-                ring.armed[s] = seq;  // published by the release of the arrive below
-                if (MMA && in.op != MK_OP_ATTN) {
-                    issue_mma_fill(p, in, t, dst, bar, pol);
-                    issued = seq + 1;
-                    continue;
-                }
-                const FillSrc f = fill_source(p, in, t);
-                if (f.b != nullptr) {  // attention: keys, then values half a stage later
-                    mbar_arrive_expect_tx(bar, 2 * f.bytes);
-                    if (f.bytes) {
-                        bulk_g2s(dst, f.a, f.bytes, bar, pol);
-                        bulk_g2s(dst + (size_t)p.keys_per_stage * p.d * 2, f.b, f.bytes, bar, pol);
-                    }
-                } else {
-                    mbar_arrive_expect_tx(bar, f.bytes);
+            continue;
+        }
+        for (uint32_t t = 0; t < in.nfill; ++t) {
+            const uint32_t seq = in.seq + t;
+            if (!acquire(seq)) goto drain;
+            const uint32_t s = seq % ring.S;
+            uint8_t* dst = ring.base + (size_t)s * ring.stage_bytes;
+            uint64_t* bar = ring.full + s;
+            const FillSrc f = fill_source(p, in, t);
+            if (f.b != nullptr) {  // attention: keys, then values half a stage later
+                mbar_arrive_expect_tx(bar, 2 * f.bytes);
+                if (f.bytes) {
                     bulk_g2s(dst, f.a, f.bytes, bar, pol);
+                    bulk_g2s(dst + (size_t)p.keys_per_stage * p.d * 2, f.b, f.bytes, bar, pol);
                 }
+            } else {
+                mbar_arrive_expect_tx(bar, f.bytes);
+                bulk_g2s(dst, f.a, f.bytes, bar, pol);
             }
             issued = seq + 1;
         }
@@ -1528,39 +1557,61 @@ __device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb,
             continue;
         }
         const MmaGeom g = mma_geom(in.op, in.count, in.aux0, p.H, p.Q, p.F, p.stage_bytes);
-        const uint32_t per = g.per_job();
+        uint32_t seq = in.seq;
         for (uint32_t c = 0; c < g.jobs; ++c, ++j) {
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, mb.opnd + s, (ph >> s) & 1u, nullptr, j, 10, lane)) goto out;
             ph ^= 1u << s;
+            if (lane == 0) trace(p, j, kTrSub0 + 2);  // the operand is in the slot
             {
                 const uint32_t opnd = smem_addr(sl.slot(j));
-                for (uint32_t r = 0; r < per; ++r) {
-                    const MmaFill f = mma_fill(g, r);
-                    const uint32_t sn = sg + f.rg * g.segs + f.seg;
-                    const uint32_t a = sn % (uint32_t)kMaxAcc, use = sn / (uint32_t)kMaxAcc;
-                    if (c == 0 && f.kf == 0 && use > 0 &&
-                        !wait_bar(p, mb.aempty + a, (use - 1u) & 1u, nullptr, sn, 11, lane))
-                        goto out;
-                    const uint32_t seq = in.seq + c * per + r;
-                    if (!wait_fill(p, ring, seq, lane)) goto out;
-                    tmem_fence_after();
-                    if (lane == 0) {
-                        const uint32_t st = smem_addr(ring.stage(seq));
-                        const uint32_t b0 = f.kf * g.nb, b1 = min(b0 + g.nb, g.k64);
-                        for (uint32_t bx = b0; bx < b1; ++bx)
-#pragma unroll
-                            for (uint32_t kk = 0; kk < 4; ++kk)
-                                mma_bf16(tbase + a * kAccCols, sw128_desc(st + (bx - b0) * g.r8 * 128u + kk * 32u),
-                                         sw128_desc(opnd + bx * 2048u + kk * 32u), (c | bx | kk) != 0u);
-                        mma_commit(ring.empty + seq % ring.S);
-                        if (c + 1 == g.jobs && f.kf + 1 == g.fps) mma_commit(mb.afull + a);
+                for (uint32_t rg = 0; rg < g.nrange; ++rg)
+                    for (uint32_t sgi = 0; sgi < g.segs; ++sgi) {
+                        const MmaSeg m = mma_seg(p, in, g, c, rg, sgi);
+                        const uint32_t sn = sg + rg * g.segs + sgi;
+                        const uint32_t a = sn % (uint32_t)kMaxAcc, use = sn / (uint32_t)kMaxAcc;
+                        if (c == 0 && use > 0 && !wait_bar(p, mb.aempty + a, (use - 1u) & 1u, nullptr, sn, 11, lane))
+                            goto out;
+                        const uint32_t ta = tbase + a * (kAccCols * kSubAcc);
+                        for (uint32_t kf = 0; kf < m.fps; ++kf, ++seq) {
+                            if (!wait_bar(p, ring.full + seq % ring.S, (seq / ring.S) & 1u, ring.armed + seq % ring.S,
+                                          seq, 2, lane, kCommitSleepNs))
+                                goto out;
+                            tmem_fence_after();
+                            if (lane == 0) {
+                                const uint32_t b0 = kf * m.nb, nbx = min(m.nb, g.k64 - b0);
+                                // descriptors advance by adding to their start-address field
+                                // (addresses stay below 256 KB, so the field never carries):
+                                // a box further is rows * 128 bytes in the stage and 2048 in
+                                // the operand, a K step 32 bytes in both
+                                uint64_t da = sw128_desc(smem_addr(ring.stage(seq)));
+                                uint64_t db = sw128_desc(opnd + b0 * 2048u);
+                                const uint64_t astep = (uint64_t)(m.rows * 128u) >> 4;
+                                // K step (b0 + bx) * 4 + kk goes to partial sum kk (kSubAcc = 4);
+                                // the first box of the segment's first job starts each of them
+                                uint32_t acc = (c | kf) != 0u;
+#pragma unroll 2
+                                for (uint32_t bx = 0; bx < nbx; ++bx) {
+                                    mma_bf16(ta, da, db, acc);
+                                    mma_bf16(ta + kAccCols, da + 2u, db + 2u, acc);
+                                    mma_bf16(ta + 2u * kAccCols, da + 4u, db + 4u, acc);
+                                    mma_bf16(ta + 3u * kAccCols, da + 6u, db + 6u, acc);
+                                    da += astep;
+                                    db += 2048u >> 4;
+                                    acc = 1u;
+                                }
+                                mma_commit(ring.empty + seq % ring.S);
+                                if (c + 1 == g.jobs && kf + 1 == m.fps) mma_commit(mb.afull + a);
+                            }
+                            __syncwarp();
+                            any = true;
+                        }
                     }
-                    __syncwarp();
-                    any = true;
-                }
             }
-            if (lane == 0) mma_commit(mb.mdone + s);
+            if (lane == 0) {
+                mma_commit(mb.mdone + s);
+                trace(p, j, kTrSub0 + 5);  // every MMA of the job issued
+            }
             __syncwarp();
         }
         sg += g.nrange * g.segs;
@@ -1569,7 +1620,7 @@ out:
     if (any && lane == 0) {
         mma_commit(mb.fin);
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_wait_sleep(mb.fin, 0u, 20000u)) {
+        while (!mbar_wait_sleep(mb.fin, 0u, kCommitSleepNs)) {
             if (global_timer_ns() - t0 > p.timeout_ns) {
                 record_error(p, MK_ERR_TIMEOUT, j, 0xfffffff9u, 0, 0, 14);
                 break;

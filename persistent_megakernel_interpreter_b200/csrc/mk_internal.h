@@ -51,32 +51,48 @@ MK_HD constexpr uint32_t attn_item_bytes(int group, int hd) {
     return ((uint32_t)(group * hd * 4 + 2 * hd * 2) + 15u) & ~15u;
 }
 // Tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES). An instruction's
-// weight rows are cut into segments of at most 128 rows (gate/up: per MLP chunk);
-// each segment streams as 64-column TMA boxes (128 bytes: the swizzle span), a
-// fill holding nb boxes of the segment side by side, and accumulates in its own
-// Tensor Memory accumulator of 16 fp32 columns (8 sequences, high and low bf16
-// parts of the input) over lanes = rows.
+// weight rows (a multiple of 8 on this path) are cut into segments of at most 128
+// rows (gate/up: per MLP chunk). A segment of R rows streams in fills of nb(R)
+// 64-column boxes (128 bytes: the swizzle span), each fill one TMA copy of a
+// {64 columns, R rows, nb boxes} block that lands as nb boxes of R rows side by
+// side, and accumulates in its own Tensor Memory accumulator over lanes = rows:
+// kSubAcc partial sums of 16 fp32 columns each (8 sequences, high and low bf16
+// parts of the input), the K = 16 steps taken in turn.
 constexpr uint32_t kAccCols = 16;
-constexpr int kMaxAcc = (int)(kTmemCols / kAccCols);  // accumulators in use at once
-constexpr uint32_t kMmaRows = 128;                   // M of every MMA: rows of a segment
-constexpr uint32_t kBoxK = 64;                        // K columns of one TMA box
-constexpr int kBoxHeights = 6;                        // box heights 4, 8, ..., 128 rows
-// Tensor maps, one per (weight matrix, box height): index kind * kBoxHeights + h.
-enum TmapKind { kTmQKV = 0, kTmO = 1, kTmGU = 2, kTmDown = 3, kTmLM = 4, kTmKinds = 5 };
+constexpr uint32_t kSubAcc = 4;
+constexpr int kMaxAcc = (int)(kTmemCols / (kAccCols * kSubAcc));  // segment accumulators in use at once
+constexpr uint32_t kMmaRows = 128;                   // M of every MMA: rows of a full segment
+constexpr uint32_t kBoxK = 64;                        // K columns of one box
+// Tensor maps, one per (weight matrix, segment rows R = 8 (h + 1)): QKV, O, gate/up
+// and the LM head at kind * 16 + h; the down-projection's chunk c at 64 + c * 8 + h
+// (its segments are at most 64 rows).
+enum TmapKind { kTmQKV = 0, kTmO = 1, kTmGU = 2, kTmLM = 3 };
+constexpr int kTmPerKind = 16;
+constexpr int kTmDown0 = 4 * kTmPerKind;
+constexpr int kTmCount = kTmDown0 + 4 * 8;
+constexpr uint32_t kTmBytes = 128;                    // sizeof(CUtensorMap)
 
-// Fills of a matvec instruction on the tensor-core path. Fill t of the instruction
-// is job c = t / (nrange * segs * fps) (the down-projection's chunk), then range,
-// segment and K-fill in that order (see mma_fill).
+// Boxes per fill of a segment of R rows: as many as a ring stage holds, at most
+// the row's k64 boxes.
+MK_HD inline uint32_t mma_nb(uint32_t R, uint32_t k64, uint32_t stage_bytes) {
+    uint32_t nb = stage_bytes / (R * 128u);
+    if (nb < 1) nb = 1;
+    return nb > k64 ? k64 : nb;
+}
+
+// Fills of a matvec instruction on the tensor-core path, in the order job c (the
+// down-projection's chunk), range, segment, K-fill. Every segment but the last
+// of a range is full (128 rows).
 struct MmaGeom {
-    uint32_t k64;     // 64-column boxes along K
-    uint32_t rows;    // weight rows of one range
-    uint32_t nrange;  // 4 for gate/up (one per MLP chunk), else 1
-    uint32_t segs;    // segments of <= 128 rows per range
-    uint32_t r8;      // rows of a full segment rounded up to 8: a box's pitch in a fill
-    uint32_t nb;      // boxes per fill
-    uint32_t fps;     // fills per segment and job
-    uint32_t jobs;    // 4 chunk jobs for the down-projection, else 1
-    MK_HD uint32_t per_job() const { return nrange * segs * fps; }
+    uint32_t k64;           // 64-column boxes along K
+    uint32_t rows;          // weight rows of one range
+    uint32_t nrange;        // 4 for gate/up (one per MLP chunk), else 1
+    uint32_t segs;          // segments per range
+    uint32_t jobs;          // 4 chunk jobs for the down-projection, else 1
+    uint32_t nb_f, fps_f;   // a full segment: boxes per fill, fills
+    uint32_t rows_l, nb_l, fps_l;  // the last segment
+    MK_HD uint32_t per_range() const { return (segs - 1u) * fps_f + fps_l; }
+    MK_HD uint32_t per_job() const { return nrange * per_range(); }
     MK_HD uint32_t nfill() const { return jobs * per_job(); }
 };
 
@@ -97,26 +113,12 @@ MK_HD inline MmaGeom mma_geom(uint32_t op, uint32_t count, uint32_t aux0, int H,
         g.nrange = 4;
     }
     g.segs = (g.rows + kMmaRows - 1) / kMmaRows;
-    g.r8 = g.rows < kMmaRows ? (g.rows + 7u) & ~7u : kMmaRows;
-    g.nb = stage_bytes / (g.r8 * 128u);
-    if (g.nb < 1) g.nb = 1;
-    if (g.nb > g.k64) g.nb = g.k64;
-    g.fps = (g.k64 + g.nb - 1) / g.nb;
+    g.nb_f = mma_nb(kMmaRows, g.k64, stage_bytes);
+    g.fps_f = (g.k64 + g.nb_f - 1) / g.nb_f;
+    g.rows_l = g.rows - (g.segs - 1u) * kMmaRows;
+    g.nb_l = mma_nb(g.rows_l, g.k64, stage_bytes);
+    g.fps_l = (g.k64 + g.nb_l - 1) / g.nb_l;
     return g;
-}
-
-// Fill r (< per_job) of one job: its range, segment, K-fill and the segment's rows.
-struct MmaFill {
-    uint32_t rg, seg, kf, rows;
-};
-MK_HD inline MmaFill mma_fill(const MmaGeom& g, uint32_t r) {
-    MmaFill f;
-    f.rg = r / (g.segs * g.fps);
-    f.seg = (r / g.fps) % g.segs;
-    f.kf = r % g.fps;
-    const uint32_t left = g.rows - f.seg * kMmaRows;
-    f.rows = left < kMmaRows ? left : kMmaRows;
-    return f;
 }
 
 constexpr int kMaxLayers = 64;
@@ -274,7 +276,7 @@ struct Params {
     uint32_t xs_aux_floats;    // offset of the slot's RoPE rows and residual rows
     // tensor-core projections (batch > 1): MK_PROJ_TENSOR_CORES, else 0
     int mma;
-    const void* tmaps;         // [kTmKinds * kBoxHeights] CUtensorMap (64-byte aligned, global)
+    const void* tmaps;         // [kTmCount] CUtensorMap (64-byte aligned, global)
     int n_counters;
     uint64_t timeout_ns;
     // optional per-job timestamps: [n_sm][trace_jobs][kTraceWords] (nullptr = off)

@@ -40,7 +40,7 @@ struct SlotPlan {
 SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma = false);
 // Whether a schedule for `batch` with these options runs the projections on the
 // tensor cores.
-bool use_mma(int batch, const mk_schedule_opts* opts);
+bool use_mma(const Layout& L, int batch, const mk_schedule_opts* opts);
 
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);

@@ -34,11 +34,11 @@
 namespace mk {
 
 uint32_t default_stage_bytes(const Layout& L, bool mma) {
-    uint32_t s = std::max(L.tile_h, std::max(L.tile_o, L.tile_f));
-    // the tensor-core path places its boxes on 1024-byte boundaries (swizzle atoms),
-    // and a fill holds at least one 64-column box of a full 128-row segment
-    if (mma) s = std::max(s, kMmaRows * kBoxK * 2u);
-    return (uint32_t)align_up(s, mma ? 1024 : 128);
+    // the tensor-core path streams 64-column boxes, not 4-row tiles: a stage holds
+    // one box of a full 128-row segment (16 KB; as many boxes of a shorter one)
+    if (mma) return kMmaRows * kBoxK * 2u;
+    const uint32_t s = std::max(L.tile_h, std::max(L.tile_o, L.tile_f));
+    return (uint32_t)align_up(s, 128);
 }
 
 SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma) {
@@ -85,8 +85,13 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma) {
     return sp;
 }
 
-bool use_mma(int batch, const mk_schedule_opts* opts) {
-    return batch > 1 && !(opts && opts->proj == MK_PROJ_CUDA_CORES);
+bool use_mma(const Layout& L, int batch, const mk_schedule_opts* opts) {
+    // Only on request: measured on the 3B-style shape at batch 8 the tensor-core
+    // projections lose to the CUDA cores (each SM's share of an op is 20-40 rows, and
+    // every tcgen05.mma of 128 x 16 x 16 costs the SM ~50 ns however few rows are
+    // real). The path takes rows in pairs of 4-row tiles (segments of a multiple
+    // of 8 rows), so the LM head's vocabulary must be a multiple of 8.
+    return batch > 1 && L.V % 8 == 0 && opts && opts->proj == MK_PROJ_TENSOR_CORES;
 }
 
 // the most SMs a plan may spread over (a B200 has 148)
@@ -99,7 +104,10 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     if (batch < 1 || batch > kMaxBatch || max_ctx < 1 || n_sm < 1 || n_sm > kMaxPlanSms)
         return MK_ERR_INVALID_ARG;
     if (o.proj < MK_PROJ_AUTO || o.proj > MK_PROJ_TENSOR_CORES) return MK_ERR_INVALID_ARG;
-    const bool mma = use_mma(batch, &o);
+    const bool mma = use_mma(L, batch, &o);
+    // units of work: single 4-row tiles, or pairs of them on the tensor-core path
+    // (every segment a multiple of 8 rows: whole 1024-byte swizzle atoms)
+    const int gran = mma ? 2 : 1;
     if (stage_bytes == 0) stage_bytes = default_stage_bytes(L, mma);
     if (stage_bytes % (mma ? 1024 : 128) || stage_bytes < default_stage_bytes(L, mma)) return MK_ERR_INVALID_ARG;
     const SlotPlan sp = slot_plan(L, batch, stage_bytes, mma);
@@ -136,8 +144,8 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     }
     const int n_parts = (max_ctx + part_keys - 1) / part_keys;
     if (n_parts > kMaxParts) return MK_ERR_INVALID_ARG;
-    const int down_cap = std::max(1, std::min(o.rowblocks_down > 0 ? o.rowblocks_down : kMaxDownRows,
-                                              kMaxDownRows));
+    int down_cap = std::max(1, std::min(o.rowblocks_down > 0 ? o.rowblocks_down : kMaxDownRows, kMaxDownRows));
+    down_cap = (down_cap + gran - 1) / gran * gran;
 
     // counters
     int nc = 0;
@@ -191,6 +199,12 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         }
         return cnt;
     };
+    // the same in units of `gran` tiles (every total here is a multiple of 2); counts in tiles
+    auto share_g = [&](int tiles, uint64_t tile_cost) {
+        std::vector<int> cnt = share(tiles / gran, tile_cost * gran);
+        for (int& c : cnt) c *= gran;
+        return cnt;
+    };
     auto mk_in = [](uint16_t op, int l) {
         mk_instr in{};
         in.op = op;
@@ -223,7 +237,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         // QKV: tiles grouped by KV group
         // One job per SM even where its range crosses a KV-group boundary (one
         // RMSNorm of x); the job then signals each group it touched.
-        emit_ranges(share(L.nkv * L.tiles_per_group, L.tile_h), 1 << 30, 1 << 30,
+        emit_ranges(share_g(L.nkv * L.tiles_per_group, L.tile_h), 1 << 30, 1 << 30,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_QKV, l);
                         in.group = (uint16_t)(a / L.tiles_per_group);
@@ -273,7 +287,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         // each (sequence, group) pair signals each of its query heads once, when
         // the head's output is final
         signals[c_part[l]] += (uint32_t)(batch * L.nq);
-        emit_ranges(share(L.H / 4, L.tile_o), 1 << 30, kMaxResidRows / 4, [&](int a, int n) {
+        emit_ranges(share_g(L.H / 4, L.tile_o), 1 << 30, kMaxResidRows / 4, [&](int a, int n) {
             mk_instr in = mk_in(MK_OP_OPROJ, l);
             in.first = (uint32_t)a;
             in.count = in.nfill = (uint32_t)n;
@@ -287,7 +301,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
         // of h are complete well before the layer's last gate/up tile; one job per SM,
         // which counts once on each chunk counter
         {
-            const std::vector<int> cnt = share(gu_chunk, 4ull * L.tile_h);
+            const std::vector<int> cnt = share_g(gu_chunk, 4ull * L.tile_h);
             int start = 0;
             for (int s = 0; s < n_sm; ++s) {
                 const int n = cnt[s];
@@ -304,7 +318,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                 start += n;
             }
         }
-        emit_ranges(share(L.H / 4, 4ull * L.tile_f), 1 << 30, down_cap,
+        emit_ranges(share_g(L.H / 4, 4ull * L.tile_f), 1 << 30, down_cap,
                     [&](int a, int n) {
                         mk_instr in = mk_in(MK_OP_DOWN, l);
                         in.first = (uint32_t)a;
@@ -317,7 +331,7 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                     });
     }
     uint32_t lm_ord = 0;  // LM-head instructions, numbered in SM order (greedy selection slots)
-    emit_ranges(share(L.V / 4, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
+    emit_ranges(share_g(L.V / 4, L.tile_h), 1 << 30, 1 << 30, [&](int a, int n) {
         mk_instr in = mk_in(MK_OP_LMHEAD, L.L - 1);
         in.aux0 = lm_ord++;
         in.first = (uint32_t)a;

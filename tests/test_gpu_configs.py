@@ -61,7 +61,7 @@ def test_3b_shape_batch8_full_depth():
     bit for bit."""
     past = [2048] * 8
     c = Case(LLAMA_3B, batch=8, max_seq=2049, past=past, seed=60)
-    c.mk.build_schedule(8, 2049)
+    c.mk.build_schedule(8, 2049, proj=2)  # the tensor-core path first
     toks = make_tokens(LLAMA_3B, 8, seed=61).numpy()
     gpu = c.gpu_step(toks, past)
     assert c.mk.status()[0] == 0

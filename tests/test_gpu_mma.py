@@ -1,5 +1,5 @@
-"""The tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES, the default
-there): every projection's weight rows stream as 64-column boxes into the ring
+"""The tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES, on request;
+the CUDA cores are the default, being faster at batch 8): every projection's weight rows stream as 64-column boxes into the ring
 and one thread issues tcgen05.mma (128 weight rows x 16 input rows: each
 sequence's fp32 input split into a bf16 high part and the bf16 rounding of the
 remainder) into fp32 accumulators in Tensor Memory, read back for the fused
@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 def _both_paths(c, batch, max_ctx, toks, pos):
     """Logits of one step on each path, from the same caches."""
-    info = c.mk.build_schedule(batch, max_ctx)
+    info = c.mk.build_schedule(batch, max_ctx, proj=_lib.PROJ_TENSOR_CORES)
     assert info.proj == _lib.PROJ_TENSOR_CORES
     tc = c.gpu_step(toks, pos)
     assert c.mk.status()[0] == 0, c.mk.status()
@@ -54,7 +54,7 @@ def test_tiny_tensor_core_step_matches_oracle(batch, past):
     ref, kc, vc = c.oracle_step(toks, past)
     assert_logits_close(tc, ref, past)
     _paths_agree(tc, cc, past)
-    c.mk.build_schedule(batch, 160)
+    c.mk.build_schedule(batch, 160, proj=_lib.PROJ_TENSOR_CORES)
     c.gpu_step(toks, past)
     assert_kv_ok(c, kc, vc, past)
     c.mk.close()
@@ -64,7 +64,7 @@ def test_tiny_tensor_core_repeated_steps_identical():
     """The same step three times gives the same bits (a fixed order of MMAs and
     accumulators, whatever the timing)."""
     c = Case(TINY, batch=4, max_seq=160, past=[10, 20, 30, 40], seed=91)
-    c.mk.build_schedule(4, 160)
+    c.mk.build_schedule(4, 160, proj=_lib.PROJ_TENSOR_CORES)
     toks = make_tokens(TINY, 4, seed=92).numpy()
     outs = []
     for _ in range(3):
@@ -95,11 +95,11 @@ def test_tensor_core_schedule_options_do_not_change_results():
     stay the same."""
     c = Case(TINY, batch=3, max_seq=160, past=[100, 37, 5], seed=93)
     toks = make_tokens(TINY, 3, seed=94).numpy()
-    info = c.mk.build_schedule(3, 160)
+    info = c.mk.build_schedule(3, 160, proj=_lib.PROJ_TENSOR_CORES)
     ref = c.gpu_step(toks, [100, 37, 5])
     for opts in (dict(n_sm=37), dict(seed=5), dict(n_sm=5, rowblocks_down=1), dict(rowblocks_down=3)):
         c.reset_kv()
-        c.mk.build_schedule(3, 160, part_keys=info.part_keys, **opts)
+        c.mk.build_schedule(3, 160, part_keys=info.part_keys, proj=_lib.PROJ_TENSOR_CORES, **opts)
         assert np.array_equal(c.gpu_step(toks, [100, 37, 5]), ref), opts
     assert c.mk.status()[0] == 0
     c.mk.close()

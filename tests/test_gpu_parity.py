@@ -300,7 +300,7 @@ def test_3b_shape_batch8_two_layers():
     cfg = dataclasses.replace(LLAMA_3B, n_layers=2, name="3b-shape-2l")
     past = [2048, 1, 700, 2047, 0, 64, 1500, 333]
     c = Case(cfg, batch=8, max_seq=2049, past=past, seed=31)
-    c.mk.build_schedule(8, 2049)
+    c.mk.build_schedule(8, 2049, proj=2)  # the tensor-core path first
     toks = make_tokens(cfg, 8, seed=32).numpy()
     ref, kc, vc = c.oracle_step(toks, past)
     gpu = c.gpu_step(toks, past)

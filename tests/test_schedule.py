@@ -16,6 +16,8 @@ pair's heads are signalled once its last partition has arrived (with one
 partition, at once)."""
 import collections
 
+import numpy as np
+
 import pytest
 
 from persistent_megakernel_interpreter_b200 import _lib
@@ -189,8 +191,9 @@ def simulate(instrs, offs, n_counters, S, NS=2, group=1, n_parts=1, NT=16, batch
 
 def mma_geom(ins, cfg, stage_bytes):
     """Fills of a matvec instruction on the tensor-core path (restated from the
-    library's header): rows cut into segments of <= 128 per range (gate/up: one range
-    per MLP chunk), each streamed as 64-column boxes, nb boxes a fill."""
+    library's header): rows (a multiple of 8) cut into segments of <= 128 per range
+    (gate/up: one range per MLP chunk); a segment of R rows streams in fills of
+    nb(R) 64-column boxes, as many as a ring stage holds."""
     jobs, nrange, rows, k64 = 1, 1, 4 * ins.count, cfg.hidden // 64
     if ins.op == _lib.OP_OPROJ:
         k64 = cfg.n_heads * cfg.head_dim // 64
@@ -199,26 +202,28 @@ def mma_geom(ins, cfg, stage_bytes):
     elif ins.op == _lib.OP_GATEUP:
         rows, nrange = 4 * ins.aux0, 4
     segs = -(-rows // 128)
-    r8 = (rows + 7) // 8 * 8 if rows < 128 else 128
-    nb = max(1, min(k64, stage_bytes // (r8 * 128)))
-    fps = -(-k64 // nb)
-    return dict(jobs=jobs, nrange=nrange, rows=rows, k64=k64, segs=segs, r8=r8, nb=nb, fps=fps)
+    seg_rows = [128] * (segs - 1) + [rows - 128 * (segs - 1)]
+    nb = [max(1, min(k64, stage_bytes // (r * 128))) for r in seg_rows]
+    fps = [-(-k64 // n) for n in nb]
+    return dict(jobs=jobs, nrange=nrange, rows=rows, k64=k64, segs=segs, seg_rows=seg_rows, nb=nb, fps=fps)
 
 
 def mma_fills(ins, cfg, stage_bytes):
-    """Per fill t of the instruction: (job c, range, segment, K boxes, segment rows)."""
+    """Per fill of the instruction, in order: (job c, range, segment, fill index kf,
+    K boxes it uses, segment rows, boxes the copy spans)."""
     g = mma_geom(ins, cfg, stage_bytes)
-    per = g["nrange"] * g["segs"] * g["fps"]
     out = []
-    for t in range(g["jobs"] * per):
-        c, r = divmod(t, per)
-        rg, seg, kf = r // (g["segs"] * g["fps"]), (r // g["fps"]) % g["segs"], r % g["fps"]
-        boxes = range(kf * g["nb"], min(kf * g["nb"] + g["nb"], g["k64"]))
-        out.append((c, rg, seg, boxes, min(128, g["rows"] - 128 * seg)))
+    for c in range(g["jobs"]):
+        for rg in range(g["nrange"]):
+            for seg in range(g["segs"]):
+                nb = g["nb"][seg]
+                for kf in range(g["fps"][seg]):
+                    boxes = range(kf * nb, min(kf * nb + nb, g["k64"]))
+                    out.append((c, rg, seg, kf, boxes, g["seg_rows"][seg], nb))
     return g, out
 
 
-def simulate_mma(instrs, offs, n_counters, S, NS, group, n_parts, cfg, stage_bytes, n_acc=32):
+def simulate_mma(instrs, offs, n_counters, S, NS, group, n_parts, cfg, stage_bytes, n_acc=8):
     """The tensor-core protocol: the loader as above; an activation warp preparing
     each job once its slot is free and its counters are met; the compute warps (as
     one) writing a matvec job's operand, then reading out each of its segments'
@@ -250,12 +255,11 @@ def simulate_mma(instrs, offs, n_counters, S, NS, group, n_parts, cfg, stage_byt
             per = len(fl) // g["jobs"]
             mine = []
             for r in range(per):
-                cc, rg, seg, boxes, rows = fl[c * per + r]
+                cc, rg, seg, kf, boxes, rows, nb = fl[c * per + r]
                 assert cc == c
-                kf = r % g["fps"]
                 sn = sn0 + rg * g["segs"] + seg
                 mine.append((ins.seq + c * per + r, sn, c == 0 and kf == 0,
-                             c == g["jobs"] - 1 and kf == g["fps"] - 1))
+                             c == g["jobs"] - 1 and kf == g["fps"][seg] - 1))
             per_job.append(mine)
             reads.append([sn0 + k for k in range(g["nrange"] * g["segs"])] if c == g["jobs"] - 1 else [])
             if c == g["jobs"] - 1:
@@ -431,15 +435,15 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
 
 
 @pytest.mark.parametrize("cfg,batch,ctx,n_sm,proj", [
-    (TINY, 1, 129, 148, 0), (TINY, 2, 200, 37, 0), (TINY, 2, 200, 37, 1), (TINY, 3, 64, 7, 0),
-    (TINY, 3, 64, 7, 1), (TINY, 1, 1, 148, 0), (LLAMA_1B, 1, 129, 148, 0), (LLAMA_1B, 1, 8193, 148, 0),
-    (LLAMA_3B, 8, 2049, 148, 0), (LLAMA_3B, 8, 2049, 148, 1),
+    (TINY, 1, 129, 148, 0), (TINY, 2, 200, 37, 0), (TINY, 2, 200, 37, 2), (TINY, 3, 64, 7, 0),
+    (TINY, 3, 64, 7, 2), (TINY, 1, 1, 148, 2), (LLAMA_1B, 1, 129, 148, 0), (LLAMA_1B, 1, 8193, 148, 0),
+    (LLAMA_3B, 8, 2049, 148, 0), (LLAMA_3B, 8, 2049, 148, 2),
 ])
 def test_plan_valid_and_deadlock_free(cfg, batch, ctx, n_sm, proj):
-    """Both projection paths at batch > 1 (proj 0: the default, tensor cores; 1:
-    CUDA cores)."""
+    """Both projection paths at batch > 1 (proj 0: the default, CUDA cores; 2:
+    tensor cores, which batch 1 ignores)."""
     instrs, offs, info = check_plan(cfg, batch, ctx, n_sm, proj=proj)
-    assert info.proj == (_lib.PROJ_TENSOR_CORES if batch > 1 and proj != 1 else _lib.PROJ_CUDA_CORES)
+    assert info.proj == (_lib.PROJ_TENSOR_CORES if batch > 1 and proj == 2 else _lib.PROJ_CUDA_CORES)
     for ns in (1, 2, 3):
         ok, ctr = sim(instrs, offs, info, ns, cfg)
         assert ok, "simulated step did not complete"
@@ -598,9 +602,9 @@ def test_plan_valid_across_batches_contexts_and_sm_counts(cfg, batch, ctx, n_sm)
 
 
 @pytest.mark.parametrize("cfg,batch,proj,limit", [
-    (LLAMA_1B, 1, 0, 16384), (LLAMA_1B, 4, 0, 16384), (LLAMA_1B, 8, 0, 16384), (LLAMA_1B, 8, 1, 16384),
-    (LLAMA_3B, 1, 0, 12288), (LLAMA_3B, 2, 0, 7680), (LLAMA_3B, 5, 0, 7680), (LLAMA_3B, 6, 0, 6144),
-    (LLAMA_3B, 8, 0, 6144), (LLAMA_3B, 2, 1, 12288), (LLAMA_3B, 3, 1, 6144), (LLAMA_3B, 8, 1, 6144),
+    (LLAMA_1B, 1, 0, 16384), (LLAMA_1B, 4, 0, 16384), (LLAMA_1B, 8, 0, 16384),
+    (LLAMA_3B, 1, 0, 12288), (LLAMA_3B, 2, 0, 12288), (LLAMA_3B, 3, 0, 6144), (LLAMA_3B, 8, 0, 6144),
+    (LLAMA_3B, 2, 2, 7168), (LLAMA_3B, 5, 2, 7168), (LLAMA_3B, 8, 2, 7168), (LLAMA_1B, 8, 2, 16384),
 ])
 def test_context_ceiling_is_the_documented_one(cfg, batch, proj, limit):
     """The largest max_ctx the planner accepts (32 partitions of at most one ring's
@@ -614,43 +618,41 @@ def test_context_ceiling_is_the_documented_one(cfg, batch, proj, limit):
 @pytest.mark.parametrize("cfg,batch,n_sm", [(TINY, 2, 37), (TINY, 8, 148), (LLAMA_1B, 8, 148),
                                             (LLAMA_3B, 8, 148), (LLAMA_3B, 3, 100)])
 def test_tensor_core_fills_cover_every_weight_once(cfg, batch, n_sm):
-    """On the tensor-core path every matvec instruction's fills (64-column boxes of
-    <= 128-row segments, nb boxes a fill) cover each (row, 64-column block) of its
-    weight rows exactly once, each fill fits one ring stage, the box pieces (the
-    segment's rows in binary: 128, 64, ..., 4) start on 8-row (1024-byte)
-    boundaries, and the planner's fill counts are these. The bytes streamed are
-    the CUDA-core path's, row for row."""
-    instrs, offs, info = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129)
+    """On the tensor-core path every matvec instruction's fills (one copy of nb
+    64-column boxes of a <= 128-row segment) cover each (row, 64-column block) of
+    its weight rows exactly once, each fill fits one ring stage, every segment is
+    whole 8-row swizzle atoms (the down-projection's at most 64 rows: its tensor
+    maps), and the planner's fill counts are these. The bytes streamed are the
+    CUDA-core path's, row for row."""
+    instrs, offs, info = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129, proj=2)
     assert info.proj == _lib.PROJ_TENSOR_CORES
     _, _, info_cc = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129, proj=1)
     assert info.bytes_per_step == info_cc.bytes_per_step
     sb = info.stage_bytes
     assert sb % 1024 == 0
-    cov = collections.Counter()
+    k_h, k_o, k_f = cfg.hidden // 64, cfg.n_heads * cfg.head_dim // 64, cfg.ffn // 4 // 64
+    qkv_rows = (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    shape = {_lib.OP_QKV: (qkv_rows, k_h), _lib.OP_OPROJ: (cfg.hidden, k_o), _lib.OP_GATEUP: (2 * cfg.ffn, k_h),
+             _lib.OP_DOWN: (cfg.hidden, k_f), _lib.OP_LMHEAD: (cfg.vocab, k_h)}
+    cov = {}  # (op, layer, chunk) -> hits per (row, 64-column block)
     for ins in instrs:
         if ins.op == _lib.OP_ATTN:
             continue
         g, fills = mma_fills(ins, cfg, sb)
         assert ins.nfill == len(fills)
-        for c, rg, seg, boxes, rows in fills:
-            assert len(boxes) * g["r8"] * 128 <= sb and 4 <= rows <= 128 and rows % 4 == 0
-            ro = 0
-            for hk in range(5, -1, -1):
-                if rows & (4 << hk):
-                    assert ro % 8 == 0
-                    ro += 4 << hk
-            assert ro == rows
+        for c, rg, seg, kf, boxes, rows, nb in fills:
+            # one copy of nb boxes of whole 8-row swizzle atoms, within a stage
+            assert nb * rows * 128 <= sb and 8 <= rows <= 128 and rows % 8 == 0
+            assert ins.op != _lib.OP_DOWN or rows <= 64
             if ins.op == _lib.OP_GATEUP:
                 row0 = 4 * (rg * (cfg.ffn // 8) + ins.first)
             else:
                 row0 = 4 * ins.first
             row0 += 128 * seg
-            for r in range(row0, row0 + rows):
-                for bx in boxes:
-                    cov[(ins.op, ins.layer, c, r, bx)] += 1
-    assert all(v == 1 for v in cov.values())
-    k_h, k_o, k_f = cfg.hidden // 64, cfg.n_heads * cfg.head_dim // 64, cfg.ffn // 4 // 64
-    qkv_rows = (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
-    want = cfg.n_layers * (qkv_rows * k_h + cfg.hidden * k_o + 2 * cfg.ffn * k_h + 4 * cfg.hidden * k_f) \
-        + cfg.vocab * k_h
+            key = (ins.op, ins.layer, c)
+            if key not in cov:
+                cov[key] = np.zeros(shape[ins.op], np.int32)
+            cov[key][row0:row0 + rows, boxes.start:boxes.stop] += 1
+    assert all(np.all(v == 1) for v in cov.values())
+    want = cfg.n_layers * 4 + 1 + cfg.n_layers * 3  # QKV, O, gate/up, down chunk 0; LM head; down chunks 1-3
     assert len(cov) == want
