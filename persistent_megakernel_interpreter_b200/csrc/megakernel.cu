@@ -445,6 +445,90 @@ __device__ __noinline__ bool block_input_tagged(const Params& p, const uint64_t*
     return block_store_input<MMAOP>(v0, v1, wv, w != nullptr, p.eps, n, xs, red, t, warp, lane, bar, orow);
 }
 
+// Batch > 1: the input vectors of two sequences at once (xs0 / operand row orow,
+// xs1 / row orow + 1), all their loads in flight together and one barrier for both
+// norms, so a job's inputs take half the rounds. Each vector's arithmetic is
+// block_input_tagged's exactly (the same pairs per thread, sums in the same order).
+// PP: pairs per thread of one vector (n / 2 / threads, rounded up).
+template <int PP, bool MMAOP>
+__device__ __noinline__ bool block_input_tagged2(const Params& p, const uint64_t* src0, const uint64_t* src1,
+                                                 uint32_t tag, const uint16_t* w, int n, float* xs0, float* xs1,
+                                                 float* red, int t, int warp, int lane, uint64_t* cbar,
+                                                 uint32_t& cuses, int orow) {
+    static_assert(2 * kConsumerWarps <= 32, "two vectors' warp sums fit the reduction words");
+    const int np = n / 2;
+    uint32_t wv[PP];
+#pragma unroll
+    for (int i = 0; i < PP; ++i) {
+        const int j = i * kNT + t;
+        wv[i] = (w != nullptr && j < np) ? ld_cg_u32(w + 2 * j) : 0u;
+    }
+    float v0[2][PP], v1[2][PP];
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint64_t a[2][PP], b[2][PP];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int i = 0; i < PP; ++i) {
+                const int j = i * kNT + t;
+                a[k][i] = b[k][i] = 0ull;
+                if (j < np) ld_tagged2((k ? src1 : src0) + 2 * j, a[k][i], b[k][i]);
+            }
+        bool ok = true;
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int i = 0; i < PP; ++i) {
+                const int j = i * kNT + t;
+                v0[k][i] = tag_val(a[k][i]);
+                v1[k][i] = tag_val(b[k][i]);
+                if (j < np) ok = ok & tag_ok(a[k][i], tag) & tag_ok(b[k][i], tag);
+            }
+        if (__all_sync(0xffffffffu, ok)) break;
+        if (!tag_backoff(p, it, t0, 1, lane)) return false;
+    }
+    float r[2] = {1.f, 1.f};
+    if (w != nullptr) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < PP; ++i)
+                if (i * kNT + t < np) {
+                    ss = fmaf(v0[k][i], v0[k][i], ss);
+                    ss = fmaf(v1[k][i], v1[k][i], ss);
+                }
+            ss = warp_sum(ss);
+            if (lane == 0) red[k * kConsumerWarps + warp] = ss;
+        }
+        if (!compute_barrier(p, cbar, cuses, lane)) return false;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            float tot = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kConsumerWarps; ++ww) tot += red[k * kConsumerWarps + ww];
+            r[k] = 1.0f / sqrtf(tot / (float)n + p.eps);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int i = 0; i < PP; ++i) {
+            const int j = i * kNT + t;
+            if (j < np) {
+                float x0 = v0[k][i], x1 = v1[k][i];
+                if (w != nullptr) {
+                    x0 = __fmul_rn(__fmul_rn(x0, r[k]), bf_lo(wv[i]));
+                    x1 = __fmul_rn(__fmul_rn(x1, r[k]), bf_hi(wv[i]));
+                }
+                if constexpr (MMAOP) mma_opnd_store(xs0, orow + k, 2 * j, x0, x1);
+                else *reinterpret_cast<float2*>((k ? xs1 : xs0) + xs_index(n, 2 * j)) = make_float2(x0, x1);
+            }
+        }
+    return compute_barrier(p, cbar, cuses, lane);
+}
+
 // `rows` (<= kMaxResidRows) consecutive tagged words into dst, by the threads
 // t < rows (whole warps; the others return at once). No barrier.
 __device__ bool rows_tagged(const Params& p, const uint64_t* src, uint32_t tag, int rows, float* dst, int t,
@@ -473,14 +557,18 @@ __device__ __forceinline__ float* slot_resid(const Params& p, float* sv, int b) 
 // O-projection. (The down-projection's inputs: down_input_batch / prep_job.) On the
 // tensor-core path (MMA) every sequence's vector goes into the slot's MMA
 // operand, row b (mma_opnd_store).
-template <bool BATCHED, bool MMA = false>
+template <bool BATCHED, bool MMA = false, int PPH = 1, int PPQ = 1>
 __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv, float* red, int warp, int lane,
                           uint64_t* cbar, uint32_t& cuses, uint32_t epoch) {
     const int t = warp * 32 + lane, l = in.layer;
     auto bar = [&]() { return compute_barrier(p, cbar, cuses, lane); };
     const int B = BATCHED ? p.B : 1;
-    for (int b = 0; b < B; ++b) {
+    // at batch > 1 two sequences at a time (block_input_tagged2) where the input is tagged
+    const bool pairs = BATCHED && !(in.op == MK_OP_QKV && l == 0);
+    for (int b = 0; b < B;) {
+        const bool two = pairs && b + 1 < B;
         float* xs = MMA ? sv : sv + (size_t)b * p.xs_vec_floats;
+        float* xs1 = MMA ? sv : sv + (size_t)(b + 1) * p.xs_vec_floats;
         switch (in.op) {
             case MK_OP_QKV:
             case MK_OP_GATEUP:
@@ -498,49 +586,76 @@ __device__ bool job_input(const Params& p, const mk_instr& in, int c, float* sv,
                     const uint32_t tag = in.op == MK_OP_GATEUP
                                              ? act_tag(epoch, l, kTagXAttn)
                                              : act_tag(epoch, in.op == MK_OP_QKV ? l - 1 : l, kTagXMlp);
-                    if (!block_input_tagged<MMA>(p, p.x_t + (size_t)b * p.H, tag, w, p.H, xs, red, t, warp, lane,
-                                                 cbar, cuses, b))
+                    const uint64_t* src = p.x_t + (size_t)b * p.H;
+                    if (BATCHED && two) {
+                        if (!block_input_tagged2<PPH, MMA>(p, src, src + p.H, tag, w, p.H, xs, xs1, red, t, warp,
+                                                           lane, cbar, cuses, b))
+                            return false;
+                    } else if (!block_input_tagged<MMA>(p, src, tag, w, p.H, xs, red, t, warp, lane, cbar, cuses,
+                                                        b)) {
                         return false;
+                    }
                 }
                 break;
             }
             case MK_OP_OPROJ: {
                 const int rows = (int)in.count * 4;
-                float* xr = slot_resid(p, sv, b);
-                if (l == 0) {
-                    if (t < rows) xr[t] = bf2f(embed_row(p, b)[(size_t)in.first * 4 + t]);
-                } else if (!rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4,
-                                        act_tag(epoch, l - 1, kTagXMlp), rows, xr, t, lane)) {
+                for (int k = 0; k < (two ? 2 : 1); ++k) {
+                    float* xr = slot_resid(p, sv, b + k);
+                    if (l == 0) {
+                        if (t < rows) xr[t] = bf2f(embed_row(p, b + k)[(size_t)in.first * 4 + t]);
+                    } else if (!rows_tagged(p, p.x_t + (size_t)(b + k) * p.H + (size_t)in.first * 4,
+                                            act_tag(epoch, l - 1, kTagXMlp), rows, xr, t, lane)) {
+                        return false;
+                    }
+                }
+                const uint64_t* src = p.attn_t + (size_t)b * p.Q;
+                const uint32_t tag = act_tag(epoch, l, kTagAttn);
+                if (BATCHED && two) {
+                    if (!block_input_tagged2<PPQ, MMA>(p, src, src + p.Q, tag, nullptr, p.Q, xs, xs1, red, t, warp,
+                                                       lane, cbar, cuses, b))
+                        return false;
+                } else if (!block_input_tagged<MMA>(p, src, tag, nullptr, p.Q, xs, red, t, warp, lane, cbar, cuses,
+                                                    b)) {
                     return false;
                 }
-                if (!block_input_tagged<MMA>(p, p.attn_t + (size_t)b * p.Q, act_tag(epoch, l, kTagAttn), nullptr,
-                                             p.Q, xs, red, t, warp, lane, cbar, cuses, b))
-                    return false;
                 break;
             }
         }
+        b += two ? 2 : 1;
     }
     return true;
 }
 
 // A down-projection chunk's inputs, by all compute warps: h chunk c of every
-// sequence and, with the last chunk, the residual rows (x after attention). At
-// batch 1 the activation warp stages chunks c < kDownStaged ahead instead (one
-// warp moves one sequence's early chunk in time; eight sequences' it does not,
-// nor the chunks that complete only as gate/up ends).
-template <bool MMA = false>
+// sequence, two at a time, and, with the last chunk, the residual rows (x after
+// attention). At batch 1 the stage and activation warps stage chunks c <
+// kDownStaged ahead instead (one warp moves one sequence's early chunk in time;
+// eight sequences' it does not, nor the chunks that complete only as gate/up ends).
+template <bool MMA = false, int PPF = 1>
 __device__ __forceinline__ bool down_input_batch(const Params& p, const mk_instr& in, int c, float* sv, float* red,
                                               int warp, int lane, uint64_t* cbar, uint32_t& cuses,
                                               uint32_t epoch) {
     const int t = warp * 32 + lane, l = in.layer;
-    for (int b = 0; b < p.B; ++b) {
-        if (c == 3 && !rows_tagged(p, p.x_t + (size_t)b * p.H + (size_t)in.first * 4, act_tag(epoch, l, kTagXAttn),
-                                   (int)in.count * 4, slot_resid(p, sv, b), t, lane))
+    const uint32_t tag = act_tag(epoch, l, kTagH);
+    for (int b = 0; b < p.B;) {
+        const bool two = b + 1 < p.B;
+        for (int k = 0; k < (two ? 2 : 1); ++k)
+            if (c == 3 && !rows_tagged(p, p.x_t + (size_t)(b + k) * p.H + (size_t)in.first * 4,
+                                       act_tag(epoch, l, kTagXAttn), (int)in.count * 4, slot_resid(p, sv, b + k), t,
+                                       lane))
+                return false;
+        const uint64_t* src = p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4);
+        float* xs = MMA ? sv : sv + (size_t)b * p.xs_vec_floats;
+        if (two) {
+            if (!block_input_tagged2<PPF, MMA>(p, src, src + p.F, tag, nullptr, p.F / 4, xs,
+                                               MMA ? sv : sv + (size_t)(b + 1) * p.xs_vec_floats, red, t, warp, lane,
+                                               cbar, cuses, b))
+                return false;
+        } else if (!block_input_tagged<MMA>(p, src, tag, nullptr, p.F / 4, xs, red, t, warp, lane, cbar, cuses, b)) {
             return false;
-        if (!block_input_tagged<MMA>(p, p.h_t + (size_t)b * p.F + (size_t)c * (p.F / 4), act_tag(epoch, l, kTagH),
-                                     nullptr, p.F / 4, MMA ? sv : sv + (size_t)b * p.xs_vec_floats, red, t, warp,
-                                     lane, cbar, cuses, b))
-            return false;
+        }
+        b += two ? 2 : 1;
     }
     return true;
 }
@@ -1274,10 +1389,10 @@ __device__ void compute_warp(const Params& p, const Ring& ring, const Tmem& tm, 
             // warp) are loaded here
             bool ok = in.op == MK_OP_ATTN   ? attn_input<HD>(p, in, sl.slot(j), warp, lane, cbar, cuses, epoch)
                       : in.op == MK_OP_DOWN ? ((!BATCHED && c < kDownStaged) ||
-                                                     down_input_batch<MMA>(p, in, c, sv, red, warp, lane, cbar,
-                                                                           cuses, epoch))
-                                            : job_input<BATCHED, MMA>(p, in, c, sv, red, warp, lane, cbar, cuses,
-                                                                      epoch);
+                                                     down_input_batch<MMA, (KF + 1) / 2>(p, in, c, sv, red, warp,
+                                                                                         lane, cbar, cuses, epoch))
+                                            : job_input<BATCHED, MMA, (KH + 1) / 2, (KO + 1) / 2>(
+                                                  p, in, c, sv, red, warp, lane, cbar, cuses, epoch);
             if (!ok) return;
             if (warp == 0 && lane == 0) trace(p, j, kTrSub0 + 7);
             // one call site per routine: the kernel's code is what every SM re-fetches
