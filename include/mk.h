@@ -135,7 +135,7 @@ typedef struct mk_schedule_opts {
  * read back by the compute warps for the same fused epilogues. CUDA cores: each
  * 4-row tile's batched fp32 dot product, as at batch 1. AUTO picks the CUDA cores:
  * measured on the 3B-style shape at batch 8 and 2048 positions (one B200) the
- * tensor-core step takes 7.6-7.8 ms against 6.8 ms. The two differ only in the
+ * tensor-core step takes 7.2 ms against 6.65 ms. The two differ only in the
  * order and form of the fp32 accumulation. The tensor-core path needs a
  * vocabulary that is a multiple of 8 (else the CUDA cores run). */
 #define MK_PROJ_AUTO 0
