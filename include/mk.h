@@ -123,21 +123,23 @@ typedef struct mk_schedule_opts {
                                 step with MK_ERR_TIMEOUT); 0 = none */
     int32_t trace;           /* nonzero: every step records per-job timestamps (see
                                 mk_read_trace) */
-    int32_t proj;            /* the projections' arithmetic at batch > 1: MK_PROJ_AUTO,
-                                MK_PROJ_CUDA_CORES or MK_PROJ_TENSOR_CORES (batch 1
-                                always runs on the CUDA cores) */
+    int32_t proj;            /* the projections' arithmetic at batch > 1: MK_PROJ_AUTO
+                                (the tensor cores), MK_PROJ_CUDA_CORES or
+                                MK_PROJ_TENSOR_CORES (batch 1 always runs on the CUDA
+                                cores) */
 } mk_schedule_opts;
 
 /* mk_schedule_opts.proj. Tensor cores: each instruction's weight rows stream as
  * 64-column TMA boxes (128-byte swizzle) and one thread issues tcgen05.mma
  * (M = 128 weight rows, N = 16: the batch's fp32 inputs split into bf16 high and
  * low parts, K = 16 per instruction) into an fp32 accumulator in Tensor Memory,
- * read back by the compute warps for the same fused epilogues. CUDA cores: each
- * 4-row tile's batched fp32 dot product, as at batch 1. AUTO picks the CUDA cores:
- * measured on the 3B-style shape at batch 8 and 2048 positions (one B200) the
- * tensor-core step takes 7.2 ms against 6.65 ms. The two differ only in the
- * order and form of the fp32 accumulation. The tensor-core path needs a
- * vocabulary that is a multiple of 8 (else the CUDA cores run). */
+ * read back by the compute warps for the same fused epilogues; four warps issue
+ * the MMAs, one per K step of each box. CUDA cores: each 4-row tile's batched fp32
+ * dot product, as at batch 1. AUTO picks the tensor cores: measured on the
+ * 3B-style shape at batch 8 and 2048 positions (one B200) the step takes 6.30 ms
+ * against 6.63 ms. The two differ only in the order and form of the fp32
+ * accumulation. The tensor-core path needs a vocabulary that is a multiple of 8
+ * (else the CUDA cores run). */
 #define MK_PROJ_AUTO 0
 #define MK_PROJ_CUDA_CORES 1
 #define MK_PROJ_TENSOR_CORES 2
@@ -156,8 +158,8 @@ typedef struct mk_schedule_opts {
  * each holding at most what the SM's weight ring holds at once (and 512 keys), so
  * max_ctx has a ceiling that depends on the shape and batch: 16384 keys for the
  * Llama-3.2-1B shape; for head_dim 128 with 24 query and 8 KV heads, 12288 at
- * batch 1-2 and 6144 at batch 3-8 (on the tensor-core path 7168 at batch 2-8). A
- * larger max_ctx
+ * batch 1 and 7168 at batch 2-8 (on the CUDA-core path 12288 at batch 2 and 6144 at
+ * 3-8). A larger max_ctx
  * (or a part_keys that needs more than 32 partitions) returns MK_ERR_INVALID_ARG. */
 mk_status mk_build_schedule(mk_handle* h, int batch, int max_ctx, const mk_schedule_opts* opts);
 

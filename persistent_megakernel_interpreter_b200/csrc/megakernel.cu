@@ -1292,7 +1292,8 @@ __device__ bool compute_attn_job(const Params& p, const Ring& ring, const mk_ins
     }
     // every warp has passed the barrier after its last read of the fills
     if (warp == kConsumerWarps - 1 && lane == 0)
-        for (uint32_t f = 0; f < a.nfill; ++f) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
+        for (uint32_t f = 0; f < a.nfill; ++f)  // (the tensor-core path counts one per issuer)
+            for (int r = 0; r < (p.mma ? kIssuers : 1); ++r) mbar_arrive(ring.empty + (a.seq + f) % ring.S);
     if (!bar()) return false;  // every output of the item is stored
     if (p.n_parts == 1) {
         if (t == 0 && a.signal_ctr != MK_NO_COUNTER) red_relaxed_add(sig, (uint32_t)G);
@@ -1649,22 +1650,23 @@ drain:
     }
 }
 
-// Tensor-core path: warp 8, converged (lane 0 issues), walks the SM's jobs in
-// order. For a matvec job it waits until the compute warps have written the job's
-// operand into its slot, then for each fill: that its segment's accumulator has
-// been read out since its previous use (first fill of the segment), that the
-// fill has landed; it issues the fill's MMAs (4 per 64-column box, K = 16 each;
-// the segment's first overwrites the accumulator) and commits them to the
-// stage's empty barrier, so the loader refills the stage once they have read it.
-// A segment's last fill also commits to its accumulator's full barrier, a job's
-// last to the slot's MMA-done barrier. Before it returns, on every way out, it
-// waits until all the MMAs it issued have completed (the CTA then releases
-// Tensor Memory). Every wait is bounded.
+// Tensor-core path: issuer u (warps 8-11, the mover warps' places; converged, lane
+// 0 issues) walks the SM's jobs in order. For a matvec job it waits until the
+// compute warps have written the job's operand into its slot, then for each fill:
+// that its segment's accumulator has been read out since its previous use (first
+// fill of the segment), that the fill has landed; it issues its K step of every
+// box of the fill (K = 16 at byte 32 u of the box's 128-byte rows) into partial
+// sum u of the segment's accumulator (the segment's first overwrites it) and
+// commits them to the stage's empty barrier, which completes once all four
+// issuers' MMAs have read the stage. A segment's last fill also commits to its
+// accumulator's full barrier, a job's last to the slot's MMA-done barrier (each
+// counts the four issuers). Before it returns, on every way out, it waits until
+// the MMAs of all four have completed (the CTA then releases Tensor Memory). Every
+// wait is bounded.
 __device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb, const Slots& sl, uint32_t tbase,
-                           int i0, int i1, int lane) {
+                           int i0, int i1, int u, int lane) {
     uint32_t j = 0, sg = 0;
     uint32_t ph = 0;  // bit s: phase of slot s's operand / MMA-done barriers (matvec jobs only)
-    bool any = false;
     for (int i = i0; i < i1; ++i) {
         const mk_instr in = p.instrs[i];
         if (in.op == MK_OP_ATTN) {
@@ -1677,7 +1679,7 @@ __device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb,
             const uint32_t s = j % sl.NS;
             if (!wait_bar(p, mb.opnd + s, (ph >> s) & 1u, nullptr, j, 10, lane)) goto out;
             ph ^= 1u << s;
-            if (lane == 0) trace(p, j, kTrSub0 + 2);  // the operand is in the slot
+            if (lane == 0 && u == 0) trace(p, j, kTrSub0 + 2);  // the operand is in the slot
             {
                 const uint32_t opnd = smem_addr(sl.slot(j));
                 for (uint32_t rg = 0; rg < g.nrange; ++rg)
@@ -1699,18 +1701,17 @@ __device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb,
                                 // (addresses stay below 256 KB, so the field never carries):
                                 // a box further is rows * 128 bytes in the stage and 2048 in
                                 // the operand, a K step 32 bytes in both
-                                uint64_t da = sw128_desc(smem_addr(ring.stage(seq)));
-                                uint64_t db = sw128_desc(opnd + b0 * 2048u);
+                                // this issuer's K step of every box: 32 bytes into the box
+                                uint64_t da = sw128_desc(smem_addr(ring.stage(seq)) + 32u * (uint32_t)u);
+                                uint64_t db = sw128_desc(opnd + b0 * 2048u + 32u * (uint32_t)u);
                                 const uint64_t astep = (uint64_t)(m.rows * 128u) >> 4;
-                                // K step (b0 + bx) * 4 + kk goes to partial sum kk (kSubAcc = 4);
-                                // the first box of the segment's first job starts each of them
+                                const uint32_t tu = ta + (uint32_t)u * kAccCols;
+                                // K step (b0 + bx) * 4 + u goes to partial sum u; the first box
+                                // of the segment's first job starts it
                                 uint32_t acc = (c | kf) != 0u;
-#pragma unroll 2
+#pragma unroll 4
                                 for (uint32_t bx = 0; bx < nbx; ++bx) {
-                                    mma_bf16(ta, da, db, acc);
-                                    mma_bf16(ta + kAccCols, da + 2u, db + 2u, acc);
-                                    mma_bf16(ta + 2u * kAccCols, da + 4u, db + 4u, acc);
-                                    mma_bf16(ta + 3u * kAccCols, da + 6u, db + 6u, acc);
+                                    mma_bf16(tu, da, db, acc);
                                     da += astep;
                                     db += 2048u >> 4;
                                     acc = 1u;
@@ -1719,20 +1720,19 @@ __device__ void mma_issuer(const Params& p, const Ring& ring, const MmaBars& mb,
                                 if (c + 1 == g.jobs && kf + 1 == m.fps) mma_commit(mb.afull + a);
                             }
                             __syncwarp();
-                            any = true;
                         }
                     }
             }
             if (lane == 0) {
                 mma_commit(mb.mdone + s);
-                trace(p, j, kTrSub0 + 5);  // every MMA of the job issued
+                if (u == 0) trace(p, j, kTrSub0 + 5);  // every MMA of the job issued
             }
             __syncwarp();
         }
         sg += g.nrange * g.segs;
     }
 out:
-    if (any && lane == 0) {
+    if (lane == 0) {  // a commit with nothing issued arrives at once
         mma_commit(mb.fin);
         const uint64_t t0 = global_timer_ns();
         while (!mbar_wait_sleep(mb.fin, 0u, kCommitSleepNs)) {
@@ -1849,7 +1849,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.n_stages; ++s) {
             mbar_init(ring.full + s, 1);
-            mbar_init(ring.empty + s, 1);  // released by a mover (weights) or the attention item (KV)
+            // released by a mover (weights) or the attention item (KV); on the tensor-core
+            // path by each issuer's commit (weights) or kIssuers arrivals of the item (KV)
+            mbar_init(ring.empty + s, MMA ? kIssuers : 1);
             ring.armed[s] = 0xffffffffu;
         }
         for (int k = 0; k < p.n_tslots; ++k) {
@@ -1867,13 +1869,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         if (MMA) {
             for (int s = 0; s < p.xs_slots; ++s) {
                 mbar_init(mb.opnd + s, kConsumerWarps);
-                mbar_init(mb.mdone + s, 1);
+                mbar_init(mb.mdone + s, kIssuers);
             }
             for (int a = 0; a < kMaxAcc; ++a) {
-                mbar_init(mb.afull + a, 1);
+                mbar_init(mb.afull + a, kIssuers);
                 mbar_init(mb.aempty + a, kConsumerWarps);
             }
-            mbar_init(mb.fin, 1);
+            mbar_init(mb.fin, kIssuers);
         }
         fence_mbar_init();
         s_epoch = ld_volatile_u32(&p.ctl->epoch);
@@ -1907,7 +1909,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         const int i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
         if (warp >= kConsumerWarps && warp < kConsumerWarps + kMoveWarps) {
             if constexpr (MMA) {
-                if (warp == kConsumerWarps) mma_issuer(p, ring, mb, sl, tm.base, i0, i1, lane);
+                mma_issuer(p, ring, mb, sl, tm.base, i0, i1, warp - kConsumerWarps, lane);
             } else {
                 mover<BATCHED>(p, ring, tm, i0, i1, warp & 3, lane);
             }

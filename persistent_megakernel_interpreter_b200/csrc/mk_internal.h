@@ -60,6 +60,10 @@ MK_HD constexpr uint32_t attn_item_bytes(int group, int hd) {
 // parts of the input), the K = 16 steps taken in turn.
 constexpr uint32_t kAccCols = 16;
 constexpr uint32_t kSubAcc = 4;
+// Issuing warps of the tensor-core path (the mover warps' places): issuer u issues
+// the MMAs of partial sum u, so the four K steps of a box go out from four threads.
+constexpr int kIssuers = 4;
+static_assert(kIssuers == (int)kSubAcc, "one issuer per partial sum");
 constexpr int kMaxAcc = (int)(kTmemCols / (kAccCols * kSubAcc));  // segment accumulators in use at once
 constexpr uint32_t kMmaRows = 128;                   // M of every MMA: rows of a full segment
 constexpr uint32_t kBoxK = 64;                        // K columns of one box

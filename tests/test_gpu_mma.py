@@ -1,5 +1,5 @@
-"""The tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES, on request;
-the CUDA cores are the default, being faster at batch 8): every projection's weight rows stream as 64-column boxes into the ring
+"""The tensor-core projections at batch > 1 (MK_PROJ_TENSOR_CORES, the default
+there; MK_PROJ_CUDA_CORES selects the batched CUDA-core dot): every projection's weight rows stream as 64-column boxes into the ring
 and one thread issues tcgen05.mma (128 weight rows x 16 input rows: each
 sequence's fp32 input split into a bf16 high part and the bf16 rounding of the
 remainder) into fp32 accumulators in Tensor Memory, read back for the fused
