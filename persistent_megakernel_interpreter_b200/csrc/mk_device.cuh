@@ -763,14 +763,17 @@ __device__ __forceinline__ void tile_epilogue(const Params& p, int l, int b, uin
 //  * Scores: LPK lanes per key (8 dims each), the group's query heads held in
 //    registers. The partial dot products meet in a reduce-scatter butterfly
 //    that leaves head 2*b2 + b1 on the lanes with lane bits (b2, b1), as
-//    s_h(j) = (q_h . k_j) * (1/sqrt(HD)) (head_dim 128: bit 3 folded first).
+//    s_h(j) = (q_h . k_j) * (log2(e) / sqrt(HD)) (head_dim 128: bit 3 folded
+//    first): the softmax runs in base 2, 2^(s - m) being e^((q . k) / sqrt(HD) - m')
+//    for the same maximum.
 //  * After each block of NB passes the warp's running maximum m_h becomes
-//    max(m_h, block maximum), the running sums are scaled by e^(m_old - m_new),
-//    the block's weights e_h(j) = exp(s_h(j) - m_h) are published to the warp's
+//    max(m_h, block maximum), the running sums are scaled by 2^(m_old - m_new),
+//    the block's weights e_h(j) = 2^(s_h(j) - m_h) are published to the warp's
 //    scratch, and every lane adds e_h(j) * v_j over its DPL dims for every head.
 //  * One CTA barrier; then thread (h, d) merges the warps in warp order:
-//    M_h = max_w m_w,h, f_w = e^(m_w,h - M_h), l_h = sum_w f_w l_w,h,
-//    o_h[d] = sum_w f_w o_w,h[d].
+//    M_h = max_w m_w,h, f_w = 2^(m_w,h - M_h), l_h = sum_w f_w l_w,h,
+//    o_h[d] = sum_w f_w o_w,h[d]. Partials of several partitions (M_h in the same
+//    base-2 units) merge the same way.
 // With one partition per (sequence, group) the output is o_h / l_h; otherwise
 // (M_h, l_h, o_h) is the partition's partial, merged in partition order. Every
 // order of summation depends only on the key indices and the shape, not on
@@ -835,7 +838,7 @@ __device__ __forceinline__ const uint16_t* attn_row(const AttnRows<HD>& R, uint3
 }
 
 // e^(a - b) for a running maximum a that may still be -inf (no key yet): 0.
-__device__ __forceinline__ float exp_rel(float a, float b) { return a == -INFINITY ? 0.f : expf(a - b); }
+__device__ __forceinline__ float exp_rel(float a, float b) { return a == -INFINITY ? 0.f : exp2f(a - b); }
 
 // The item on all compute warps (warp < kConsumerWarps). qs: the group's G query
 // heads, fp32 [G][HD], in shared memory; sc: attn_scratch_floats(HD) of shared
@@ -852,7 +855,8 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
     static_assert(4 * S::BK <= (int)SC::kWarp && kMaxGroup * HD <= (int)SC::kWarp, "attention scratch");
     const int n = R.n, t = warp * 32 + lane;
     const int nc = R.jnew >= 0 ? n - 1 : n;  // rows read from the fills
-    const float scale = 1.0f / sqrtf((float)HD);
+    // scores in base 2: s = (q . k) * log2(e) / sqrt(HD), weights 2^(s - m) = e^((q . k) / sqrt(HD) - m')
+    const float scale = 1.44269504088896341f / sqrtf((float)HD);
     float* ew = sc + (size_t)warp * SC::kWarp;  // this warp's region
     const int dc = lane % S::LPK, kk = lane / S::LPK;
     const int hh = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);  // head this lane's scores belong to
@@ -936,7 +940,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
         __syncwarp();  // the previous block's weights have been read
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
-            const float e = s[i] == -INFINITY ? 0.f : expf(s[i] - mnew);
+            const float e = s[i] == -INFINITY ? 0.f : exp2f(s[i] - mnew);
             if (writer) {
                 lpart = (i == 0 ? lpart * f : lpart) + e;
                 ew[(i * KPW + kk) * 4 + hh] = e;
@@ -951,13 +955,17 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
 #pragma unroll
             for (int dd = 0; dd < DPL; ++dd) o[h][dd] *= fh[h];
         __syncwarp();
-        // values: every key of the block, in pass order, for the lane's DPL dims
+        // values: every key of the block, in pass order, for the lane's DPL dims. A
+        // pass's KPW rows sit in one fill (a stage holds a multiple of KPW keys), so
+        // its row address is found once per pass.
 #pragma unroll
-        for (int i = 0; i < NB; ++i)
+        for (int i = 0; i < NB; ++i) {
+            const int j0 = (p0 + i * kConsumerWarps) * KPW;
+            const uint16_t* vb = attn_row<HD>(R, m, j0 < nc ? j0 : 0) + vofs;
 #pragma unroll
             for (int k2 = 0; k2 < KPW; ++k2) {
-                const int j = (p0 + i * kConsumerWarps) * KPW + k2;
-                const uint16_t* vr = j < nc ? attn_row<HD>(R, m, j) + vofs : R.vnew;  // stand-in, masked
+                const int j = j0 + k2;
+                const uint16_t* vr = j < nc ? vb + (size_t)k2 * HD : R.vnew;  // stand-in, masked
                 float v[DPL];
                 if constexpr (DPL == 2) {
                     const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vr + lane * 2);
@@ -977,6 +985,7 @@ __device__ __forceinline__ bool attn_item_block(const AttnRows<HD>& R, const flo
 #pragma unroll
                     for (int dd = 0; dd < DPL; ++dd) o[h][dd] = fmaf(ev[h], v[dd], o[h][dd]);
             }
+        }
     }
     // the warp's l per head: its writer lanes' shares, added over lane bits 3, 4
     lpart += __shfl_xor_sync(0xffffffffu, lpart, 8);
@@ -1055,7 +1064,7 @@ __device__ __forceinline__ void attn_merge_heads(const Params& p, int b, int h0,
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
         const float M = warp_max(w[i]);
-        w[i] = (lane < P && h0 + i * hstep < h_end) ? expf(w[i] - M) : 0.f;  // empty: e^-inf = 0
+        w[i] = (lane < P && h0 + i * hstep < h_end) ? exp2f(w[i] - M) : 0.f;  // empty: 2^-inf = 0
         L[i] = 0.f;
 #pragma unroll
         for (int d = 0; d < S::DPL; ++d) O[i][d] = 0.f;

@@ -112,10 +112,10 @@ mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
     const SlotPlan sp = slot_plan(L, batch, stage_bytes, mma);
     const int kps = sp.keys_per_stage;
     if (kps < 1 || sp.stages < kMoveWarps) return MK_ERR_UNSUPPORTED;
-    // the attention value phase splits an item's keys into classes j mod KQ
-    // (KQ = compute threads / (head_dim / 2)); a ring stage must hold whole rounds
-    const int attn_classes = std::max(1, 32 * kConsumerWarps / (L.d / 2));
-    if (kps % attn_classes) return MK_ERR_UNSUPPORTED;
+    // an attention item reads each pass of 256 / head_dim keys from one fill, so a
+    // ring stage holds whole passes
+    const int attn_pass = std::max(1, 256 / L.d);
+    if (kps % attn_pass) return MK_ERR_UNSUPPORTED;
 
     // attention partitions: one per (sequence, KV group) up to kSingleItemKeys
     // keys; for longer contexts as many as there are SMs for (an item's time is
