@@ -309,6 +309,26 @@ mk_status mk_plan_schedule_host(const mk_config* cfg, int batch, int max_ctx, in
                                 const mk_schedule_opts* opts, mk_instr* instr_out, size_t cap,
                                 int32_t* sm_offsets, mk_schedule_info* info);
 
+/* One tensor map of the tensor-core path (mk_schedule_opts.proj): a view of the
+ * packed weights (mk_pack_weights_host's layout) as bf16 elements. Element
+ * (c_0, ..., c_{rank-1}) sits at byte base_offset + 2 * c_0 + sum_{i >= 1} c_i *
+ * strides[i - 1] of the packed buffer; box is the block one TMA copy reads (one
+ * fill: 64 columns x rows x boxes of 64 columns). index is the map's place in the
+ * kernel's table. */
+typedef struct mk_tmap_spec {
+    int32_t index, rank;
+    uint64_t base_offset;
+    uint64_t dims[5];
+    uint64_t strides[4];
+    uint32_t box[5];
+} mk_tmap_spec;
+
+/* The tensor maps a schedule with ring stages of `stage_bytes` uses (host only, for
+ * inspection and tests): writes up to `cap` specs to out (may be NULL to query)
+ * and their count to *n. MK_ERR_UNSUPPORTED for a shape the kernels do not take. */
+mk_status mk_tensor_map_specs_host(const mk_config* cfg, uint32_t stage_bytes, mk_tmap_spec* out, size_t cap,
+                                   size_t* n);
+
 /* Summary of the handle's current schedule. */
 mk_status mk_get_schedule_info(mk_handle* h, mk_schedule_info* info);
 

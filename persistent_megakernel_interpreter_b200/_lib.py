@@ -48,6 +48,11 @@ class MkScheduleInfo(ctypes.Structure):
         ("min_sm_bytes", ctypes.c_uint64), ("proj", I32), ("reserved0", I32)]
 
 
+class MkTmapSpec(ctypes.Structure):
+    _fields_ = [("index", I32), ("rank", I32), ("base_offset", ctypes.c_uint64),
+                ("dims", ctypes.c_uint64 * 5), ("strides", ctypes.c_uint64 * 4), ("box", ctypes.c_uint32 * 5)]
+
+
 OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LMHEAD = 1, 2, 3, 4, 5, 6
 PROJ_AUTO, PROJ_CUDA_CORES, PROJ_TENSOR_CORES = 0, 1, 2
 NO_COUNTER = 0xFFFFFFFF
@@ -104,10 +109,12 @@ def lib() -> ctypes.CDLL:
                                                   ctypes.c_int, P, P]
     L.mk_greedy_select.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P]
     L.mk_decode_steps_greedy.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P]
+    L.mk_tensor_map_specs_host.argtypes = [ctypes.POINTER(MkConfig), ctypes.c_uint32, ctypes.POINTER(MkTmapSpec),
+                                           ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]
     for f in ("mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_steps_greedy", "mk_baseline_decode_step",
               "mk_decode_step_host", "mk_get_status", "mk_plan_schedule_host",
               "mk_get_schedule_info", "mk_read_counters", "mk_pack_weights_host", "mk_read_trace",
-              "mk_baseline_decode_step_noalloc", "mk_greedy_select"):
+              "mk_baseline_decode_step_noalloc", "mk_greedy_select", "mk_tensor_map_specs_host"):
         getattr(L, f).restype = st
     _lib = L
     return L

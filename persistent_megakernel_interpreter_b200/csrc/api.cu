@@ -221,16 +221,10 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, int de
     return no_throw([&] { return create_impl(cfg, w, device, out); });
 }
 
-// Tensor maps of the packed weights for the tensor-core path: one per (matrix,
-// segment rows R = 8, 16, ..., 128), whose box is one fill of such a segment:
-// {64 columns, R rows, nb(R) 64-column blocks}, landing as nb boxes of R rows x
-// 128 bytes side by side, in the 128-byte swizzle the MMA's shared-memory
-// descriptors read. The K dimension is split into (64, K / 64) so that one copy
-// takes several boxes; a fill past the end of K reads zeros there (never used).
-//   QKV / O / gate-up: {64, rows, K / 64, layer}; LM head (the embedding rows):
-//   {64, rows, K / 64}; down chunk c: {64, 4 rows of a block, hidden / 4 row
-//   blocks, (ffn / 4) / 64, layer}, R <= 64.
-// nb depends on the ring's stage size, so the maps are rebuilt when it changes.
+// Tensor maps of the packed weights for the tensor-core path (mk::tmap_specs: one
+// per matrix and segment height, the box one fill of such a segment), encoded with
+// the 128-byte swizzle the MMA's shared-memory descriptors read. nb depends on the
+// ring's stage size, so the maps are rebuilt when it changes.
 static mk_status make_tmaps(mk_handle* h, uint32_t stage_bytes) {
     if (h->d_tmaps && h->tmap_stage_bytes == stage_bytes) return MK_OK;
     typedef CUresult (*Encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -256,46 +250,16 @@ static mk_status make_tmaps(mk_handle* h, uint32_t stage_bytes) {
                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         return r == CUDA_SUCCESS;
     };
-    uint8_t* pk = h->packed;
-    const cuuint64_t ls = (cuuint64_t)L.layer_stride;
-    const uint32_t kh = (uint32_t)L.H / mk::kBoxK, kq = (uint32_t)L.Q / mk::kBoxK, kf = (uint32_t)(L.F / 4) / mk::kBoxK;
     bool ok = true;
-    for (int hk = 0; hk < mk::kTmPerKind && ok; ++hk) {
-        const cuuint32_t R = 8u * (cuuint32_t)(hk + 1);
-        {
-            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)L.qkv_rows, kh, (cuuint64_t)L.L};
-            const cuuint64_t st[3] = {(cuuint64_t)L.H * 2, 128, ls};
-            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes), 1};
-            ok = ok && enc(mk::kTmQKV * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_qkv, 4, dims, st, box);
+    for (const mk_tmap_spec& t : mk::tmap_specs(L, stage_bytes)) {
+        cuuint64_t dims[5], strides[4];
+        cuuint32_t box[5];
+        for (int i = 0; i < t.rank; ++i) {
+            dims[i] = (cuuint64_t)t.dims[i];
+            box[i] = (cuuint32_t)t.box[i];
+            if (i + 1 < t.rank) strides[i] = (cuuint64_t)t.strides[i];
         }
-        {
-            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)L.H, kq, (cuuint64_t)L.L};
-            const cuuint64_t st[3] = {(cuuint64_t)L.Q * 2, 128, ls};
-            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kq, stage_bytes), 1};
-            ok = ok && enc(mk::kTmO * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_o, 4, dims, st, box);
-        }
-        {
-            const cuuint64_t dims[4] = {mk::kBoxK, (cuuint64_t)(2 * L.F), kh, (cuuint64_t)L.L};
-            const cuuint64_t st[3] = {(cuuint64_t)L.H * 2, 128, ls};
-            const cuuint32_t box[4] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes), 1};
-            ok = ok && enc(mk::kTmGU * mk::kTmPerKind + hk, pk + L.off_layer0 + L.rel_gu, 4, dims, st, box);
-        }
-        {
-            const cuuint64_t dims[3] = {mk::kBoxK, (cuuint64_t)L.V, kh};
-            const cuuint64_t st[2] = {(cuuint64_t)L.H * 2, 128};
-            const cuuint32_t box[3] = {mk::kBoxK, R, mk::mma_nb(R, kh, stage_bytes)};
-            ok = ok && enc(mk::kTmLM * mk::kTmPerKind + hk, pk + L.off_embed, 3, dims, st, box);
-        }
-        if (R <= 64) {
-            const cuuint64_t f4 = (cuuint64_t)(L.F / 4);
-            for (int c = 0; c < 4 && ok; ++c) {
-                const cuuint64_t dims[5] = {mk::kBoxK, 4, (cuuint64_t)(L.H / 4), kf, (cuuint64_t)L.L};
-                const cuuint64_t st[4] = {f4 * 2, f4 * 2 * 16, 128, ls};
-                const cuuint32_t box[5] = {mk::kBoxK, 4, R / 4, mk::mma_nb(R, kf, stage_bytes), 1};
-                ok = ok && enc(mk::kTmDown0 + c * 8 + hk, pk + L.off_layer0 + L.rel_down + (size_t)c * f4 * 2 * 4, 5,
-                               dims, st, box);
-            }
-        }
+        ok = ok && enc(t.index, h->packed + t.base_offset, t.rank, dims, strides, box);
     }
     if (!ok) {
         h->msg = "cuTensorMapEncodeTiled refused a weight tensor map";

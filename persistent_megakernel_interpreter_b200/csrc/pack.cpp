@@ -4,6 +4,7 @@
 // by a gather kernel on the device (mk_create) or by memcpy on the host.
 #include <string.h>
 
+#include <initializer_list>
 #include <vector>
 
 #include "pack.h"
@@ -154,6 +155,52 @@ std::vector<Segment> pack_segments(const Layout& L, const mk_weights& w) {
     return v;
 }
 
+// One map per (matrix, segment rows R = 8 (h + 1)), whose box is one fill of such a
+// segment: {64 columns, R rows, nb(R) 64-column blocks}, K viewed as (64, K / 64):
+//   QKV / O / gate-up: {64, rows, K / 64, layer}; LM head (the embedding rows):
+//   {64, rows, K / 64}; down chunk c: {64, 4 rows of a block, hidden / 4 row blocks,
+//   (ffn / 4) / 64, layer}, R <= 64 (a down instruction has at most 64 rows).
+std::vector<mk_tmap_spec> tmap_specs(const Layout& L, uint32_t stage_bytes) {
+    std::vector<mk_tmap_spec> v;
+    const uint64_t ls = (uint64_t)L.layer_stride;
+    const uint32_t kh = (uint32_t)L.H / kBoxK, kq = (uint32_t)L.Q / kBoxK, kf = (uint32_t)(L.F / 4) / kBoxK;
+    auto add_spec = [&](int idx, size_t base, int rank, std::initializer_list<uint64_t> dims,
+                        std::initializer_list<uint64_t> strides, std::initializer_list<uint32_t> box) {
+        mk_tmap_spec t{};
+        t.index = idx;
+        t.rank = rank;
+        t.base_offset = base;
+        int i = 0;
+        for (uint64_t d : dims) t.dims[i++] = d;
+        i = 0;
+        for (uint64_t st : strides) t.strides[i++] = st;
+        i = 0;
+        for (uint32_t b : box) t.box[i++] = b;
+        v.push_back(t);
+    };
+    for (int hk = 0; hk < kTmPerKind; ++hk) {
+        const uint32_t R = 8u * (uint32_t)(hk + 1);
+        add_spec(kTmQKV * kTmPerKind + hk, L.off_layer0 + L.rel_qkv, 4,
+                 {kBoxK, (uint64_t)L.qkv_rows, kh, (uint64_t)L.L}, {(uint64_t)L.H * 2, 128, ls},
+                 {kBoxK, R, mma_nb(R, kh, stage_bytes), 1});
+        add_spec(kTmO * kTmPerKind + hk, L.off_layer0 + L.rel_o, 4, {kBoxK, (uint64_t)L.H, kq, (uint64_t)L.L},
+                 {(uint64_t)L.Q * 2, 128, ls}, {kBoxK, R, mma_nb(R, kq, stage_bytes), 1});
+        add_spec(kTmGU * kTmPerKind + hk, L.off_layer0 + L.rel_gu, 4,
+                 {kBoxK, (uint64_t)(2 * L.F), kh, (uint64_t)L.L}, {(uint64_t)L.H * 2, 128, ls},
+                 {kBoxK, R, mma_nb(R, kh, stage_bytes), 1});
+        add_spec(kTmLM * kTmPerKind + hk, L.off_embed, 3, {kBoxK, (uint64_t)L.V, kh}, {(uint64_t)L.H * 2, 128},
+                 {kBoxK, R, mma_nb(R, kh, stage_bytes)});
+        if (R <= 64) {
+            const uint64_t f4 = (uint64_t)(L.F / 4);
+            for (int c = 0; c < 4; ++c)
+                add_spec(kTmDown0 + c * 8 + hk, L.off_layer0 + L.rel_down + (size_t)c * f4 * 2 * 4, 5,
+                         {kBoxK, 4, (uint64_t)(L.H / 4), kf, (uint64_t)L.L}, {f4 * 2, f4 * 2 * 16, 128, ls},
+                         {kBoxK, 4, R / 4, mma_nb(R, kf, stage_bytes), 1});
+        }
+    }
+    return v;
+}
+
 bool weights_complete(const Layout& L, const mk_weights& w) {
     if (!w.embed || !w.final_norm || !w.attn_norm || !w.wq || !w.wk || !w.wv || !w.wo ||
         !w.mlp_norm || !w.wgate || !w.wup || !w.wdown)
@@ -171,6 +218,24 @@ extern "C" size_t mk_packed_bytes(const mk_config* cfg) {
     mk::Layout L;
     if (!cfg || !mk::make_layout(*cfg, &L, nullptr)) return 0;
     return L.total;
+}
+
+extern "C" mk_status mk_tensor_map_specs_host(const mk_config* cfg, uint32_t stage_bytes, mk_tmap_spec* out,
+                                               size_t cap, size_t* n) {
+    mk::Layout L;
+    if (!cfg || !n || stage_bytes == 0) return MK_ERR_INVALID_ARG;
+    if (!mk::make_layout(*cfg, &L, nullptr)) return MK_ERR_UNSUPPORTED;
+    try {
+        const std::vector<mk_tmap_spec> v = mk::tmap_specs(L, stage_bytes);
+        *n = v.size();
+        if (out) {
+            if (cap < v.size()) return MK_ERR_INVALID_ARG;
+            for (size_t i = 0; i < v.size(); ++i) out[i] = v[i];
+        }
+    } catch (...) {
+        return MK_ERR_OUT_OF_MEMORY;
+    }
+    return MK_OK;
 }
 
 extern "C" mk_status mk_pack_weights_host(const mk_config* cfg, const mk_weights* w, void* dst,

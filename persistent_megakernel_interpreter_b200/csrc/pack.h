@@ -42,6 +42,9 @@ SlotPlan slot_plan(const Layout& L, int batch, uint32_t stage_bytes, bool mma = 
 // tensor cores.
 bool use_mma(const Layout& L, int batch, const mk_schedule_opts* opts);
 
+// The tensor-core path's tensor maps for ring stages of stage_bytes (mk_tmap_spec).
+std::vector<mk_tmap_spec> tmap_specs(const Layout& L, uint32_t stage_bytes);
+
 mk_status plan_schedule(const Layout& L, int batch, int max_ctx, int n_sm,
                         const mk_schedule_opts* opts, uint32_t stage_bytes, Plan* out);
 
