@@ -33,25 +33,29 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def load(path: str) -> ctypes.CDLL:
+    """Open a build of ``oracle.c`` at ``path`` and declare its entry points."""
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    L.orc_round_bf16.argtypes = [P, P, ctypes.c_int64]
+    L.orc_bf16_to_f32.argtypes = [P, P, ctypes.c_int64]
+    L.orc_rmsnorm.argtypes = [P, P, ctypes.c_int, ctypes.c_float, P]
+    L.orc_rope.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_double]
+    L.orc_matvec.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+    L.orc_attention.argtypes = [P, P, P] + [ctypes.c_int] * 5 + [P]
+    L.orc_silu_mul.argtypes = [P, P, ctypes.c_int, P]
+    L.orc_argmax.argtypes = [P, ctypes.c_int]
+    L.orc_argmax.restype = ctypes.c_int
+    L.orc_decode_step.argtypes = [P, ctypes.c_int, P, P, P, P, ctypes.c_int, P, ctypes.c_int]
+    L.orc_decode_step.restype = ctypes.c_int
+    L.orc_max_threads.restype = ctypes.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        L.orc_round_bf16.argtypes = [P, P, ctypes.c_int64]
-        L.orc_bf16_to_f32.argtypes = [P, P, ctypes.c_int64]
-        L.orc_rmsnorm.argtypes = [P, P, ctypes.c_int, ctypes.c_float, P]
-        L.orc_rope.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_double]
-        L.orc_matvec.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
-        L.orc_attention.argtypes = [P, P, P] + [ctypes.c_int] * 5 + [P]
-        L.orc_silu_mul.argtypes = [P, P, ctypes.c_int, P]
-        L.orc_argmax.argtypes = [P, ctypes.c_int]
-        L.orc_argmax.restype = ctypes.c_int
-        L.orc_decode_step.argtypes = [P, ctypes.c_int, P, P, P, P, ctypes.c_int, P, ctypes.c_int]
-        L.orc_decode_step.restype = ctypes.c_int
-        L.orc_max_threads.restype = ctypes.c_int
-        _lib = L
+        _lib = load(build())
     return _lib
 
 
