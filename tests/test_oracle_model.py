@@ -47,7 +47,7 @@ def test_oracle_vs_fp64_brute_same_rounding_points(setup, tiny_weights):
                 assert np.all(np.abs(g - want[l][:, pos[b]]) <= 2.0 ** -7 * np.abs(want[l][:, pos[b]]))
 
 
-def test_oracle_vs_exact_fp64_decoder(setup, tiny_weights):
+def test_oracle_vs_fp64_brute_exact(setup, tiny_weights):
     cfg, om, k, v, toks = setup
     kc, vc = _np_cache(k), _np_cache(v)
     pos = np.array([128, 40], np.int32)
