@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from persistent_megakernel_interpreter_b200 import _lib
-from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B, TINY
+from persistent_megakernel_interpreter_b200.config import LLAMA_1B, TINY
 from persistent_megakernel_interpreter_b200.inputs import make_tokens
 from test_gpu_parity import Case, assert_kv_ok, assert_logits_close, reg_bar
 
