@@ -302,6 +302,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / steps, "us_per_step": 1e6 * el / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "arithmetic": "fp32 over bf16 weights and KV cache, fp32 activations (the oracle)",
             "data": "synthetic", "config": workload_config(args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -463,7 +464,12 @@ def run_mk(args):
             "us_per_launch_p10_p90": [1e3 * q for q in (statistics.quantiles(launch_ms, n=10)[0],
                                                          statistics.quantiles(launch_ms, n=10)[8])]
             if len(launch_ms) >= 2 else None,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            # the type the products are computed in; weights and KV cache are bf16 either way
+            "dtype": "bf16" if info.proj == 2 else "f32",
+            "arithmetic": ("bf16 tcgen05 MMA (activations as bf16 high + low parts), fp32 accumulation"
+                           if info.proj == 2 else
+                           "fp32 FMA over bf16 weights and KV cache, fp32 activations"),
             "data": "synthetic", "config": workload_config(world, cfg.n_layers, past, args.model, BATCH),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
