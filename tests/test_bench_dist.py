@@ -113,3 +113,4 @@ def test_reference_arm_prints_the_contract_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert "workload" in line["config"]
+    assert line["dtype"] == "f32" and "fp32" in line["arithmetic"]  # the oracle computes in fp32
