@@ -9,14 +9,17 @@ for QKV / O / gate-up, {0, row0, kb0} for the LM head, {0, 0, row0 / 4, kb0, lay
 for down chunk c. A wrong stride, dimension order or box size shows up as an
 address mismatch, with no GPU."""
 import ctypes
+import dataclasses
 
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings, strategies as st
 
 from persistent_megakernel_interpreter_b200 import _lib
 from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B, TINY
 from persistent_megakernel_interpreter_b200.model import plan_schedule
 from test_schedule import mma_fills
+from test_schedule_fuzz import shapes
 
 
 def specs(cfg, stage_bytes):
@@ -71,6 +74,19 @@ def box_addr(s, coords):
 @pytest.mark.parametrize("cfg,batch,n_sm", [(TINY, 2, 37), (TINY, 8, 148), (LLAMA_1B, 8, 148),
                                             (LLAMA_3B, 8, 148), (LLAMA_3B, 3, 100)])
 def test_every_fill_reads_its_rows(cfg, batch, n_sm):
+    check_fills(cfg, batch, n_sm)
+
+
+@settings(max_examples=80, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+@given(cfg=shapes(), batch=st.integers(2, 8), n_sm=st.integers(1, 148))
+def test_every_fill_reads_its_rows_random_shapes(cfg, batch, n_sm):
+    """The same check on drawn shapes (head_dim 64 / 128, 1-4 query heads per KV head,
+    hidden 256-1024, ffn 1024-3072), vocabularies rounded to whole 8-row units."""
+    check_fills(dataclasses.replace(cfg, vocab=cfg.vocab // 8 * 8), batch, n_sm)
+
+
+def check_fills(cfg, batch, n_sm):
     instrs, offs, info = plan_schedule(cfg, batch, 129, n_sm, max_batch=8, max_seq=129, proj=2)
     assert info.proj == _lib.PROJ_TENSOR_CORES
     sb = info.stage_bytes
