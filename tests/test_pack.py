@@ -5,10 +5,12 @@ import dataclasses
 import numpy as np
 import pytest
 import torch
+from hypothesis import HealthCheck, given, settings
 
 from persistent_megakernel_interpreter_b200.config import LLAMA_3B, TINY, ModelConfig
 from persistent_megakernel_interpreter_b200.inputs import make_weights
 from persistent_megakernel_interpreter_b200.model import pack_weights_host
+from test_schedule_fuzz import shapes
 
 
 def _u16(t):
@@ -77,6 +79,19 @@ SHAPES = [TINY, dataclasses.replace(LLAMA_3B, name="3b-heads-small", n_layers=2,
 
 @pytest.mark.parametrize("cfg", SHAPES, ids=lambda c: c.name)
 def test_pack_roundtrip_bit_exact(cfg):
+    check_roundtrip(cfg)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+@given(cfg=shapes())
+def test_pack_roundtrip_bit_exact_random_shapes(cfg):
+    """The same round trip on drawn shapes (head_dim 64 / 128, 1-4 query heads per KV
+    head, 1-3 layers, hidden 256-1024, ffn 1024-3072, vocab any multiple of 4)."""
+    check_roundtrip(cfg)
+
+
+def check_roundtrip(cfg):
     w = make_weights(cfg, seed=7, norm_jitter=0.1)
     buf = pack_weights_host(cfg, w).numpy()
     E, layers, norms = unpack(cfg, buf)
