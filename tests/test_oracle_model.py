@@ -8,7 +8,7 @@ from hypothesis import HealthCheck, assume, given, settings, strategies as st
 import oracle
 from oracle.brute import Brute, bf16_bits_to_f64
 from persistent_megakernel_interpreter_b200.inputs import make_kv_cache, make_tokens, make_weights
-from test_schedule_fuzz import shapes
+from strategies import shapes
 
 
 def _np_cache(t):

@@ -10,7 +10,7 @@ from hypothesis import HealthCheck, given, settings
 from persistent_megakernel_interpreter_b200.config import LLAMA_3B, TINY, ModelConfig
 from persistent_megakernel_interpreter_b200.inputs import make_weights
 from persistent_megakernel_interpreter_b200.model import pack_weights_host
-from test_schedule_fuzz import shapes
+from strategies import shapes
 
 
 def _u16(t):

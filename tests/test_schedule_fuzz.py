@@ -2,35 +2,17 @@
 paths and schedule options drawn inside the ranges mk.h accepts (hypothesis, with a
 fixed seed so that every run draws the same cases). For each draw the host planner
 either refuses an explicit attention partition size exactly when mk.h's rule makes it
-illegal (MK_ERR_INVALID_ARG), or returns a plan that passes the same checks as the hand-picked cases in test_schedule.py: every
-weight tile, row block and cached key covered exactly once, every waited count equal
-to the signals that counter receives, and a simulated step of the megakernel's
-synchronisation protocol that runs to completion with every counter at its target."""
-import dataclasses
-
+illegal (MK_ERR_INVALID_ARG), or returns a plan that passes the same checks as the
+hand-picked cases in test_schedule.py: every weight tile, row block and cached key
+covered exactly once, every waited count equal to the signals that counter receives,
+and a simulated step of the megakernel's synchronisation protocol that runs to
+completion with every counter at its target."""
 from hypothesis import HealthCheck, event, given, settings, strategies as st
 
 from persistent_megakernel_interpreter_b200 import _lib
-from persistent_megakernel_interpreter_b200.config import TINY
 from persistent_megakernel_interpreter_b200.model import plan_schedule
+from strategies import shapes
 from test_schedule import check_plan, sim, static_signals
-
-
-@st.composite
-def shapes(draw):
-    head_dim = draw(st.sampled_from([64, 128]))
-    n_kv = draw(st.sampled_from([1, 2, 4]))
-    group = draw(st.sampled_from([1, 2, 3, 4]))
-    n_heads = group * n_kv
-    if (n_heads * head_dim) % 256:
-        n_heads = group * n_kv * (256 // head_dim)  # widen to the next legal head count
-        n_kv = n_heads // group
-    cfg = dataclasses.replace(
-        TINY, name="fuzz", n_layers=draw(st.integers(1, 3)),
-        hidden=draw(st.sampled_from([256, 512, 768, 1024])), n_heads=n_heads, n_kv_heads=n_kv,
-        head_dim=head_dim, ffn=draw(st.sampled_from([1024, 2048, 3072])),
-        vocab=4 * draw(st.integers(16, 600)))
-    return cfg
 
 
 @settings(max_examples=150, deadline=None, derandomize=True,

@@ -19,7 +19,7 @@ from persistent_megakernel_interpreter_b200 import _lib
 from persistent_megakernel_interpreter_b200.config import LLAMA_1B, LLAMA_3B, TINY
 from persistent_megakernel_interpreter_b200.model import plan_schedule
 from test_schedule import mma_fills
-from test_schedule_fuzz import shapes
+from strategies import shapes
 
 
 def specs(cfg, stage_bytes):
