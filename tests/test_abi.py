@@ -132,3 +132,13 @@ def test_ctypes_declarations_match_the_c_header(tmp_path):
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
                                           check=True).stdout.split()]
     assert got == want
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: with libmk.so absent, loading raises instead of returning a
+    stand-in (the binding's only compute path is the CUDA library)."""
+    from persistent_megakernel_interpreter_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libmk.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.lib()
