@@ -4,6 +4,8 @@ import ctypes
 import os
 import re
 
+import pytest
+
 from conftest import ROOT
 
 HEADER = os.path.join(ROOT, "include", "mk.h")
