@@ -364,6 +364,12 @@ def sim(instrs, offs, info, ns, cfg):
 
 def check_plan(cfg, batch, max_ctx, n_sm, **opts):
     instrs, offs, info = plan_schedule(cfg, batch, max_ctx, n_sm, max_batch=8, max_seq=max_ctx, **opts)
+    check_lists(cfg, batch, max_ctx, instrs, offs, info)
+    return instrs, offs, info
+
+
+def check_lists(cfg, batch, max_ctx, instrs, offs, info):
+    """The static checks of a plan's per-SM lists (raise AssertionError on a fault)."""
     n_sm = len(offs) - 1
     assert info.n_instr == len(instrs) and offs[-1] == len(instrs)
     # per-SM fill numbering is the prefix sum of fills
@@ -433,7 +439,6 @@ def check_plan(cfg, batch, max_ctx, n_sm, **opts):
         for job in jobs_of(L):
             for c, t in job_waits(L, job):
                 assert signals[c] == t, (c, t, signals[c])
-    return instrs, offs, info
 
 
 @pytest.mark.parametrize("cfg,batch,ctx,n_sm,proj", [
@@ -481,6 +486,72 @@ def test_dropped_item_cannot_complete():
             continue  # nothing in the step waits for the logits
         ok, _ = sim(instrs, offs, info, 2, TINY)
         assert not ok, drop
+
+
+def _copy(ins):
+    return _lib.MkInstr.from_buffer_copy(ins)
+
+
+def _renumber(instrs, offs):
+    """Recompute each SM's fill numbering (seq) after a list was edited."""
+    for s_ in range(len(offs) - 1):
+        seq = 0
+        for ins in instrs[offs[s_]:offs[s_ + 1]]:
+            ins.seq = seq
+            seq += ins.nfill
+
+
+def _plant(instrs, offs, kind):
+    """A copy of the plan with one planted mistake of the given kind."""
+    L = [_copy(i) for i in instrs]
+    if kind == "waited count one too high":
+        next(i for i in L if i.op == _lib.OP_OPROJ).wait_n += 1
+    elif kind == "a tile computed twice, another never":
+        next(i for i in L if i.op == _lib.OP_OPROJ and i.count > 1).first += 1
+    elif kind == "fill numbering off by one":
+        next(i for i in L if i.op == _lib.OP_GATEUP).seq += 1
+    elif kind == "attention item signals the wrong layer":
+        a = [i for i in L if i.op == _lib.OP_ATTN]
+        a[0].signal_ctr = next(i.signal_ctr for i in a if i.layer != a[0].layer)
+    elif kind == "consumer ahead of its producer on one SM":
+        # an attention item moved in front of the QKV job of its own layer on the
+        # same SM, whose group counter it waits on
+        for s_ in range(len(offs) - 1):
+            lst = L[offs[s_]:offs[s_ + 1]]
+            q = [k for k, i in enumerate(lst) if i.op == _lib.OP_QKV]
+            a = [k for k, i in enumerate(lst) if i.op == _lib.OP_ATTN and i.job_items == 1
+                 and any(lst[j].layer == i.layer and lst[j].signal_ctr <= i.wait_ctr
+                         < lst[j].signal_ctr + max(1, lst[j].aux1) for j in q if j < k)]
+            if a:
+                k = a[0]
+                j = next(j for j in q if j < k and lst[j].layer == lst[k].layer)
+                lst.insert(j, lst.pop(k))
+                L[offs[s_]:offs[s_ + 1]] = lst
+                _renumber(L, offs)
+                return L
+        raise AssertionError("no attention item shares an SM with its QKV producer")
+    return L
+
+
+@pytest.mark.parametrize("kind", ["waited count one too high", "a tile computed twice, another never",
+                                  "fill numbering off by one", "attention item signals the wrong layer",
+                                  "consumer ahead of its producer on one SM"])
+def test_checks_catch_planted_plan_errors(kind):
+    """The plan checks and the protocol simulator are themselves tested: each planted
+    mistake in a valid plan fails a static check or leaves the simulated step stuck
+    (an ordering mistake passes every static check; only the simulation sees it)."""
+    instrs, offs, info = check_plan(TINY, 2, 129, 37, proj=1)
+    bad = _plant(instrs, offs, kind)
+    try:
+        check_lists(TINY, 2, 129, bad, offs, info)
+    except AssertionError:
+        static = True
+    else:
+        static = False
+    ok, _ = sim(bad, offs, info, 2, TINY)
+    assert static or not ok, kind
+    if kind == "consumer ahead of its producer on one SM":
+        assert not static and not ok
 
 
 @pytest.mark.parametrize("cfg,batch,ctx,parts", [
