@@ -533,14 +533,17 @@ def _plant(instrs, offs, kind):
     return L
 
 
+@pytest.mark.parametrize("proj", [1, 2])
 @pytest.mark.parametrize("kind", ["waited count one too high", "a tile computed twice, another never",
                                   "fill numbering off by one", "attention item signals the wrong layer",
                                   "consumer ahead of its producer on one SM"])
-def test_checks_catch_planted_plan_errors(kind):
-    """The plan checks and the protocol simulator are themselves tested: each planted
-    mistake in a valid plan fails a static check or leaves the simulated step stuck
-    (an ordering mistake passes every static check; only the simulation sees it)."""
-    instrs, offs, info = check_plan(TINY, 2, 129, 37, proj=1)
+def test_checks_catch_planted_plan_errors(kind, proj):
+    """The plan checks and the protocol simulators (CUDA-core and tensor-core paths) are
+    themselves tested: each planted mistake in a valid plan fails a static check or
+    leaves the simulated step stuck (an ordering mistake passes every static check;
+    only the simulation sees it)."""
+    instrs, offs, info = check_plan(TINY, 2, 129, 37, proj=proj)
+    assert info.proj == (_lib.PROJ_CUDA_CORES if proj == 1 else _lib.PROJ_TENSOR_CORES)
     bad = _plant(instrs, offs, kind)
     try:
         check_lists(TINY, 2, 129, bad, offs, info)
