@@ -691,6 +691,16 @@ def test_context_ceiling_is_the_documented_one(cfg, batch, proj, limit):
         plan_schedule(cfg, batch, limit + 1, 148, max_batch=8, max_seq=limit + 1, proj=proj)
 
 
+@pytest.mark.parametrize("cfg,batch,ctx", [(LLAMA_1B, 1, 16384), (LLAMA_3B, 1, 12288), (LLAMA_3B, 8, 7168)])
+def test_plans_at_the_context_ceiling_simulate_to_completion(cfg, batch, ctx):
+    """At the longest context each shape takes (32 partitions per (sequence, KV
+    group)) the plan passes the static checks and its simulated step completes."""
+    instrs, offs, info = check_plan(cfg, batch, ctx, 148)
+    assert info.n_parts == 32
+    ok, _ = sim(instrs, offs, info, 1, cfg)
+    assert ok, "simulated step did not complete"
+
+
 @pytest.mark.parametrize("cfg,batch,n_sm", [(TINY, 2, 37), (TINY, 8, 148), (LLAMA_1B, 8, 148),
                                             (LLAMA_3B, 8, 148), (LLAMA_3B, 3, 100)])
 def test_tensor_core_fills_cover_every_weight_once(cfg, batch, n_sm):
