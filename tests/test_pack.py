@@ -118,3 +118,42 @@ def test_pack_is_a_permutation_of_the_input_bytes(cfg):
     counts = np.bincount(buf, minlength=65536)
     counts[0] -= buf.size - src.size
     assert np.array_equal(counts, np.bincount(src, minlength=65536))
+
+
+def test_host_packer_refuses_bad_arguments_without_writing():
+    """Null pointers, a destination one byte short, an incomplete weight set and an
+    unsupported shape are refused (MK_ERR_INVALID_ARG / MK_ERR_UNSUPPORTED) before
+    any byte of the destination is written."""
+    import ctypes
+    from persistent_megakernel_interpreter_b200 import _lib
+    L = _lib.lib()
+    c = _lib.make_config(TINY, 1, 1)
+    n = L.mk_packed_bytes(ctypes.byref(c))
+    w = make_weights(TINY, seed=3)
+    keep = []
+
+    def tab(ts):
+        ts = [t.contiguous() for t in ts]
+        keep.extend(ts)
+        arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+        keep.append(arr)
+        return ctypes.cast(arr, ctypes.c_void_p)
+
+    mw = _lib.MkWeights()
+    mw.embed, mw.final_norm = w.embed.data_ptr(), w.final_norm.data_ptr()
+    for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "wgate", "wup", "wdown"):
+        setattr(mw, name, tab(getattr(w, name)))
+    dst = np.full(n, 0xA5, np.uint8)
+    p = dst.ctypes.data_as(ctypes.c_void_p)
+    assert L.mk_pack_weights_host(None, ctypes.byref(mw), p, n) == 1
+    assert L.mk_pack_weights_host(ctypes.byref(c), None, p, n) == 1
+    assert L.mk_pack_weights_host(ctypes.byref(c), ctypes.byref(mw), None, n) == 1
+    assert L.mk_pack_weights_host(ctypes.byref(c), ctypes.byref(mw), p, n - 1) == 1
+    partial = _lib.MkWeights.from_buffer_copy(mw)
+    partial.wdown = None
+    assert L.mk_pack_weights_host(ctypes.byref(c), ctypes.byref(partial), p, n) == 1
+    bad = _lib.make_config(dataclasses.replace(TINY, head_dim=96), 1, 1)
+    assert L.mk_pack_weights_host(ctypes.byref(bad), ctypes.byref(mw), p, n) == 3
+    assert np.all(dst == 0xA5)
+    assert L.mk_pack_weights_host(ctypes.byref(c), ctypes.byref(mw), p, n) == 0
+    assert not np.all(dst == 0xA5)
